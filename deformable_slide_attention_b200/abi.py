@@ -1,0 +1,170 @@
+"""ctypes binding over ``libdsa3d.so`` (declared in ``include/dsa3d.h``).
+
+The ``dsa3d_*`` functions here carry the C names and take plain integers for pointers and the
+stream; they only marshal arguments.  :func:`forward` and :func:`backward` are conveniences for
+torch CUDA tensors: they validate shapes, allocate the outputs (and the backward workspace) with
+torch's caching allocator and call the C entry points on the current stream.
+
+There is no fallback: if the library is missing, or no CUDA device is present, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libdsa3d.so"
+_lib = None
+_lock = threading.Lock()
+
+DSA3D_F32 = 0
+DSA3D_BF16 = 1
+
+_STATUS = {0: "DSA3D_OK", 1: "DSA3D_ERR_INVALID_ARGUMENT", 2: "DSA3D_ERR_UNSUPPORTED",
+           3: "DSA3D_ERR_WORKSPACE_TOO_SMALL", 4: "DSA3D_ERR_CUDA", 5: "DSA3D_ERR_DEVICE_CHECK"}
+
+
+class Dsa3dError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, status)} ({dsa3d_status_string(status)})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m "
+                               "deformable_slide_attention_b200.build` (there is no CPU fallback)")
+        lib = ctypes.CDLL(path)
+        I, Z, P = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+        dims = [I] * 8
+        lib.dsa3d_abi_version.restype = I
+        lib.dsa3d_abi_version.argtypes = []
+        lib.dsa3d_status_string.restype = ctypes.c_char_p
+        lib.dsa3d_status_string.argtypes = [I]
+        lib.dsa3d_forward.restype = I
+        lib.dsa3d_forward.argtypes = [P, P, P, P, P, P, *dims, I, P]
+        lib.dsa3d_backward_workspace_bytes.restype = Z
+        lib.dsa3d_backward_workspace_bytes.argtypes = [*dims, I]
+        lib.dsa3d_backward.restype = I
+        lib.dsa3d_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
+        lib.dsa3d_check_device.restype = I
+        lib.dsa3d_check_device.argtypes = [P]
+        _lib = lib
+        return lib
+
+
+# --- the C entry points, one to one -----------------------------------------------------------
+def dsa3d_abi_version() -> int:
+    return _load().dsa3d_abi_version()
+
+
+def dsa3d_status_string(status: int) -> str:
+    try:
+        return _load().dsa3d_status_string(int(status)).decode()
+    except RuntimeError:
+        return _STATUS.get(status, "unknown status")
+
+
+def dsa3d_forward(q, k, v, offsets, out, lse, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream) -> int:
+    return _load().dsa3d_forward(q, k, v, offsets, out, lse, F, Hp, Wp, heads, dh, kt, kh, kw,
+                                 dtype, stream)
+
+
+def dsa3d_backward_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype) -> int:
+    return _load().dsa3d_backward_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype)
+
+
+def dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, workspace,
+                   workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream) -> int:
+    return _load().dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, workspace,
+                                  workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream)
+
+
+def dsa3d_check_device(stream) -> int:
+    return _load().dsa3d_check_device(stream)
+
+
+# --- torch conveniences -----------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return DSA3D_F32
+    if t.dtype == torch.bfloat16:
+        return DSA3D_BF16
+    raise TypeError(f"3D-DSA takes float32 or bfloat16 tensors, got {t.dtype}")
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check(status, what):
+    if status != 0:
+        raise Dsa3dError(status, what)
+
+
+def _shapes(q, offsets, dims):
+    F, Hp, Wp = dims
+    N = F * Hp * Wp
+    if q.dim() != 3 or q.shape[0] != N:
+        raise ValueError(f"q must be [N={N}][heads][dh], got {tuple(q.shape)}")
+    heads, dh = q.shape[1], q.shape[2]
+    if tuple(offsets.shape) != (heads, N, 3):
+        raise ValueError(f"offsets must be [heads][N][3] = {(heads, N, 3)}, got {tuple(offsets.shape)}")
+    return N, heads, dh
+
+
+def forward(q, k, v, offsets, dims, window, out=None, lse=None, stream=None, want_lse=True):
+    """3D-DSA forward on CUDA tensors.  Returns (out [N][heads][dh], lse [heads][N] or None)."""
+    torch = _torch()
+    N, heads, dh = _shapes(q, offsets, dims)
+    for t in (q, k, v, offsets):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((heads, N), dtype=torch.float32, device=q.device)
+    _check(dsa3d_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(), out.data_ptr(),
+                         lse.data_ptr() if lse is not None else None, *dims, heads, dh, *window,
+                         _dtype_code(q), _stream_handle(stream)), "dsa3d_forward")
+    return out, lse
+
+
+def backward(q, k, v, offsets, out, lse, dout, dims, window, workspace=None, stream=None,
+             grads=None):
+    """3D-DSA backward on CUDA tensors.  Returns (dq, dk, dv, doffsets)."""
+    torch = _torch()
+    N, heads, dh = _shapes(q, offsets, dims)
+    code = _dtype_code(q)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty_like(offsets))
+    dq, dk, dv, doff = grads
+    need = dsa3d_backward_workspace_bytes(*dims, heads, dh, *window, code)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(dsa3d_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(), out.data_ptr(),
+                          lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          doff.data_ptr(), ws_ptr, ws_bytes, *dims, heads, dh, *window, code,
+                          _stream_handle(stream)), "dsa3d_backward")
+    return dq, dk, dv, doff

@@ -1,0 +1,205 @@
+"""CPU oracle for 3D Deformable Slide Attention (3D-DSA).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package; the product path never does.  It shares no code with the CUDA path.
+
+The arithmetic lives in ``dsa3d_oracle.c`` (plain C, double precision, one tap at a time).  This
+module compiles it with gcc on first use and marshals numpy/torch CPU arrays through ctypes.
+
+Source of the operator: MegaSlide-DiT (arXiv 2607.22696), the 3D-DSA definition (Eq. 1 and the
+softmax over the k_t x k_h x k_w neighbourhood that follows it).  The readings the paper leaves
+open are listed in the C file's header (R1..R7).
+
+Parity pins: every routine here is pinned by ``tests/test_oracle_pins.py`` against brute-force
+dense attention, torch's ``grid_sample``, finite differences and an independent torch autograd
+restatement.  The one unpinned reading is the score scale (R3, 1/sqrt(dh)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsa3d_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libdsa3d_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+IO_F32 = 0
+IO_BF16 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (OpenMP, strict IEEE arithmetic)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+               "-std=c11", "-Wall", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            # DSA3D_ORACLE_LIB lets the oracle's own mutation test load a deliberately broken copy
+            path = os.environ.get("DSA3D_ORACLE_LIB") or build()
+            lib = ctypes.CDLL(path)
+            i64p = ctypes.POINTER(ctypes.c_int64)
+            vp = ctypes.c_void_p
+            dims = [ctypes.c_int] * 8
+            lib.dsa3d_oracle_forward.restype = ctypes.c_int64
+            lib.dsa3d_oracle_forward.argtypes = [ctypes.c_int, vp, vp, vp, vp, *dims, i64p,
+                                                 ctypes.c_int64, vp, vp, ctypes.c_int]
+            lib.dsa3d_oracle_backward.restype = ctypes.c_int
+            lib.dsa3d_oracle_backward.argtypes = [ctypes.c_int, vp, vp, vp, vp, vp, *dims, i64p,
+                                                  ctypes.c_int64, vp, vp, i64p, ctypes.c_int64,
+                                                  vp, vp, ctypes.c_int]
+            lib.dsa3d_oracle_tap.restype = ctypes.c_int
+            lib.dsa3d_oracle_tap.argtypes = [ctypes.c_int, vp, vp, *dims, ctypes.c_int,
+                                             ctypes.c_int64, ctypes.c_int, i64p, vp, vp, vp]
+            _lib = lib
+    return _lib
+
+
+def _as_io(x):
+    """Return (contiguous numpy array, io code) for an fp32 or bf16 array (numpy or torch)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return x.view(torch.int16).numpy().view(np.uint16), IO_BF16
+            if x.dtype == torch.float32:
+                return x.numpy(), IO_F32
+            raise TypeError(f"oracle inputs must be float32 or bfloat16, got {x.dtype}")
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.float32:
+        return x, IO_F32
+    if x.dtype == np.uint16:
+        return x, IO_BF16
+    raise TypeError(f"oracle inputs must be float32 or bf16 bits (uint16), got {x.dtype}")
+
+
+def _f32(x):
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None and a.size else ctypes.c_void_p(0)
+
+
+def _items(items, total):
+    if items is None:
+        items = np.arange(total, dtype=np.int64)
+    items = np.ascontiguousarray(items, dtype=np.int64)
+    return items, items.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+
+
+def _threads(n):
+    return int(n) if n else (os.cpu_count() or 1)
+
+
+def forward(q, k, v, offsets, dims, window, items=None, threads=None, return_reads=False):
+    """Forward of 3D-DSA.
+
+    q, k, v: [N][heads][dh] (fp32 or bf16); offsets: [heads][N][3] fp32; dims = (F, Hp, Wp);
+    window = (kt, kh, kw).  ``items`` lists h*N + n; None means every (h, n), head-major.
+    Returns (out [n_items][dh] float64, lse [n_items] float64).
+    """
+    qa, io = _as_io(q)
+    ka, io_k = _as_io(k)
+    va, io_v = _as_io(v)
+    if not (io == io_k == io_v):
+        raise TypeError("q, k, v must share one dtype")
+    off = _f32(offsets)
+    N = dims[0] * dims[1] * dims[2]
+    heads, dh = qa.shape[-2], qa.shape[-1]
+    it, itp = _items(items, N * heads)
+    out = np.zeros((len(it), dh), np.float64)
+    lse = np.zeros(len(it), np.float64)
+    reads = _load().dsa3d_oracle_forward(io, _ptr(qa), _ptr(ka), _ptr(va), _ptr(off), *dims, heads,
+                                         dh, *window, itp, len(it), _ptr(out), _ptr(lse),
+                                         _threads(threads))
+    if reads < 0:
+        raise ValueError("oracle forward rejected its arguments")
+    return (out, lse, reads) if return_reads else (out, lse)
+
+
+def backward(q, k, v, offsets, dout, dims, window, q_items=None, k_items=None, threads=None):
+    """Backward of 3D-DSA.
+
+    Returns (dq [n_q][dh], doff [n_q][3], dk [n_k][dh], dv [n_k][dh]) in float64.  ``q_items``
+    and ``k_items`` list h*N + n; None means every item.  dk/dv at a key gather the contributions
+    of every query of that head.
+    """
+    qa, io = _as_io(q)
+    ka, _ = _as_io(k)
+    va, _ = _as_io(v)
+    da, io_d = _as_io(dout)
+    if io_d != io:
+        raise TypeError("dout must share the dtype of q")
+    off = _f32(offsets)
+    N = dims[0] * dims[1] * dims[2]
+    heads, dh = qa.shape[-2], qa.shape[-1]
+    qi, qip = _items(q_items, N * heads)
+    ki, kip = _items(k_items, N * heads)
+    dq = np.zeros((len(qi), dh), np.float64)
+    doff = np.zeros((len(qi), 3), np.float64)
+    dk = np.zeros((len(ki), dh), np.float64)
+    dv = np.zeros((len(ki), dh), np.float64)
+    rc = _load().dsa3d_oracle_backward(io, _ptr(qa), _ptr(ka), _ptr(va), _ptr(off), _ptr(da), *dims,
+                                       heads, dh, *window, qip, len(qi), _ptr(dq), _ptr(doff), kip,
+                                       len(ki), _ptr(dk), _ptr(dv), _threads(threads))
+    if rc != 0:
+        raise ValueError("oracle backward rejected its arguments")
+    return dq, doff, dk, dv
+
+
+def tap(src, offsets, dims, window, h, n, tau):
+    """One tap: (valid, base[3] int64, frac[3] float32, sample[dh], dsample[3][dh])."""
+    sa, io = _as_io(src)
+    off = _f32(offsets)
+    heads, dh = sa.shape[-2], sa.shape[-1]
+    base = np.zeros(3, np.int64)
+    frac = np.zeros(3, np.float32)
+    samp = np.zeros(dh, np.float64)
+    dsamp = np.zeros((3, dh), np.float64)
+    rc = _load().dsa3d_oracle_tap(io, _ptr(sa), _ptr(off), *dims, heads, dh, *window, h, n, tau,
+                                  base.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _ptr(frac),
+                                  _ptr(samp), _ptr(dsamp))
+    if rc < 0:
+        raise ValueError("oracle tap rejected its arguments")
+    return bool(rc), base, frac, samp, dsamp
+
+
+def full_forward(q, k, v, offsets, dims, window, threads=None):
+    """Forward over every (n, h), returned in the [N][heads][dh] / [heads][N] layouts."""
+    N = dims[0] * dims[1] * dims[2]
+    heads, dh = q.shape[-2], q.shape[-1]
+    out, lse = forward(q, k, v, offsets, dims, window, None, threads)
+    out = out.reshape(heads, N, dh).transpose(1, 0, 2).copy()
+    return out, lse.reshape(heads, N)
+
+
+def full_backward(q, k, v, offsets, dout, dims, window, threads=None):
+    """Backward over every item, returned as dq/dk/dv [N][heads][dh] and doff [heads][N][3]."""
+    N = dims[0] * dims[1] * dims[2]
+    heads, dh = q.shape[-2], q.shape[-1]
+    dq, doff, dk, dv = backward(q, k, v, offsets, dout, dims, window, None, None, threads)
+    r = lambda a: a.reshape(heads, N, dh).transpose(1, 0, 2).copy()
+    return r(dq), doff.reshape(heads, N, 3), r(dk), r(dv)
