@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark: 3D-DSA forward + backward throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole path over one batch: the forward (saving lse) and the backward
+(dq, dk, dv, doffsets) of 3D Deformable Slide Attention on the named synthetic workload (default:
+the 1080p long-video workload, 256 frames x 68 x 120 tokens, 32 heads x 128, window 3x9x9, bf16).
+Inputs are resident in HBM when the timed region starts; every input tensor is larger than L2,
+so no extra L2 flush is needed between steps.  Multi-GPU runs (torchrun) are weak scaling: each
+rank processes its own independent clip (seed + rank); 3D-DSA has no exchange step.
+
+``--impl reference`` times the CPU oracle (the only other implementation) on a bounded sample.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "3D-DSA fwd+bwd tokens/s at N≈2.1M (1 B200) and % of HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FP32_LANES_PER_SM = 128
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="1080p-long-bf16")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    return ap.parse_args(argv)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
+
+
+# --- algorithmic units -------------------------------------------------------------------------
+def alg_bytes_per_item(w, kernel):
+    """Algorithmic HBM bytes per (token, head): each tensor read or written once."""
+    s = 4 if w.dtype == "f32" else 2
+    if kernel == "fwd":
+        return 4 * w.dh * s + 12 + 4            # q, k, v read, out written; offsets, lse
+    return 8 * w.dh * s + 12 + 4 + 12           # q, k, v, out, dO read; dq, dk, dv written;
+    #                                             offsets, lse read; doffsets written
+
+
+def alg_flop_per_item(w, kernel):
+    """Factorised fp32 work per (token, head): box dots and box axpys of length dh."""
+    B = (w.window[0] + 1) * (w.window[1] + 1) * (w.window[2] + 1)
+    return (4 if kernel == "fwd" else 10) * w.dh * B
+
+
+# --- clocks ------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9 and (not self.uuid or self.uuid in parts[0]):
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in self.rows:
+            for i, n in enumerate(names[1:], start=5):
+                if r[i].lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+# --- CPU oracle leg ----------------------------------------------------------------------------
+def oracle_sample(w, head_inputs, n_items, seed, threads):
+    """Time the oracle on n_items seeded (token) queries of one head of workload w: its forward
+    and the query side of its backward (dq, doffsets).  Returns seconds."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    items = np.sort(rng.choice(w.N, size=n_items, replace=False)).astype(np.int64)
+    q, k, v, off, do = head_inputs
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, off, w.dims, w.window, items, threads)
+    oracle.backward(q, k, v, off, do, w.dims, w.window, items, [], threads)
+    return time.perf_counter() - t0
+
+
+def head_inputs_for_oracle(w, inp, head=0):
+    """One head's inputs as contiguous CPU tensors ([N][1][dh] and [1][N][3])."""
+    pick = lambda t: t[:, head:head + 1, :].contiguous().cpu()
+    return (pick(inp["q"]), pick(inp["k"]), pick(inp["v"]),
+            inp["offsets"][head:head + 1].contiguous().cpu(), pick(inp["dout"]))
+
+
+def calibrated_items(w, hin, threads, budget_s):
+    t1 = oracle_sample(w, hin, max(threads, 1), 12345, threads)
+    per_round = t1  # one item per thread
+    rounds = max(1, int(budget_s / max(per_round, 1e-6)))
+    return rounds * max(threads, 1)
+
+
+def cpu_baseline(w, inp, budget_s):
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    hin = head_inputs_for_oracle(w, inp)
+    n_items = calibrated_items(w, hin, threads, budget_s)
+    secs = oracle_sample(w, hin, n_items, 777, threads)
+    tokens = n_items / w.heads  # one token = all heads
+    return {"value": tokens / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": (f"{n_items} seeded query tokens of head 0 of the {w.name} workload: oracle "
+                       f"forward + query-side backward (dq, doffsets; dk/dv excluded), "
+                       f"{secs:.1f} s on {threads} threads; tokens = items / {w.heads} heads")}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle, K timed steps of a bounded sample each."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from deformable_slide_attention_b200 import inputs
+    import oracle
+    oracle.build()
+    w = inputs.BY_NAME[args.workload]
+    dev = "cuda" if (w.device_generated and torch.cuda.is_available()) else "cpu"
+    if w.device_generated and dev == "cpu":
+        # the 1080p workload is drawn on the device; without one, draw the same recipe on the CPU
+        w = dataclasses.replace(w, device_generated=False)
+    inp = inputs.make(w, dev, with_dout=True)
+    hin = head_inputs_for_oracle(w, inp)
+    del inp
+    threads = os.cpu_count() or 1
+    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    n_items = calibrated_items(w, hin, threads, per_step)
+    for i in range(args.warmup):
+        oracle_sample(w, hin, n_items, 1000 + i, threads)
+    secs = [oracle_sample(w, hin, n_items, 2000 + i, threads) for i in range(args.steps)]
+    total = sum(secs)
+    tokens_per_step = n_items / w.heads
+    value = tokens_per_step * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "tokens": w.N, "heads": w.heads, "dh": w.dh,
+                   "window": list(w.window)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"per step {n_items} seeded query tokens of head 0: oracle forward "
+                                   f"+ query-side backward (dq, doffsets); tokens = items / {w.heads}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --- GPU leg -----------------------------------------------------------------------------------
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+    from deformable_slide_attention_b200 import abi, build, inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+    build.build()
+
+    base = inputs.BY_NAME[args.workload]
+    w = dataclasses.replace(base, seed=base.seed + 1000 * rank)
+    inp = inputs.make(w, dev, with_dout=True)
+    code = abi.DSA3D_BF16 if w.dtype == "bf16" else abi.DSA3D_F32
+    q, k, v, off, do = (inp[n] for n in ("q", "k", "v", "offsets", "dout"))
+    out = torch.empty_like(q)
+    lse = torch.empty((w.heads, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv, doff = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(off)
+    full_ws = abi.dsa3d_backward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
+    per_head = full_ws // w.heads if full_ws else 0
+    free, _ = torch.cuda.mem_get_info(dev)
+    margin = 6 << 30
+    heads_per_pass = w.heads if not per_head else max(1, min(w.heads, (free - margin) // per_head))
+    ws = torch.empty(max(per_head * heads_per_pass, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        abi.forward(q, k, v, off, w.dims, w.window, out=out, lse=lse)
+        abi.backward(q, k, v, off, out, lse, do, w.dims, w.window, workspace=ws, grads=(dq, dk, dv, doff))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", "") or "")
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.5)
+    abi.dsa3d_timing_reset()
+    abi.dsa3d_timing_enable(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    abi.dsa3d_timing_enable(False)
+    ktimes = abi.dsa3d_timing_read()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = w.N * world / (ms / 1000.0)
+    launches = sum(n for n, _ in ktimes.values())
+
+    peaks, peak_src = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    dominant = max(ktimes.items(), key=lambda kv: kv[1][1]) if ktimes else None
+    roof = None
+    alu = None
+    kernel_table = {kname: {"launches": n, "avg_ms": tot / n, "share": tot / sum(x[1] for x in ktimes.values())}
+                    for kname, (n, tot) in ktimes.items()}
+    if dominant:
+        kname, (n, tot) = dominant
+        avg_ms = tot / n
+        kind = "fwd" if "fwd" in kname else "bwd"
+        items_per_launch = w.heads * w.N if kind == "fwd" else w.N * heads_per_pass
+        alg = alg_bytes_per_item(w, kind) * items_per_launch
+        achieved = alg / (avg_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None, "kernel": kname,
+                "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"
+                               if peak_src == "measured" else "fallback 6.65 TB/s"}
+        mhz = clocks["sm_mhz"] or float(peaks.get("sm_max_mhz", 1965.0))
+        fp32_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+        flops = alg_flop_per_item(w, kind) * items_per_launch
+        alu = {"bound": "alu", "achieved": flops / (avg_ms / 1000.0) / 1e12, "unit": "TFLOP/s",
+               "peak": fp32_peak, "frac": flops / (avg_ms / 1000.0) / 1e12 / fp32_peak,
+               "peak_basis": f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {mhz:.0f} MHz"}
+    step_bytes = w.heads * w.N * (alg_bytes_per_item(w, "fwd") + alg_bytes_per_item(w, "bwd"))
+    step_roof = {"alg_bytes_per_step": step_bytes,
+                 "achieved_gbs": step_bytes / (ms / 1000.0) / 1e9,
+                 "frac_of_hbm": step_bytes / (ms / 1000.0) / 1e9 / hbm}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_leg(args, w, inp, abi, torch, dev, ws, world, (out, lse, dq, dk, dv, doff))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "frames": w.F, "grid": [w.Hp, w.Wp], "tokens": w.N,
+                   "heads": w.heads, "dh": w.dh, "window": list(w.window),
+                   "heads_per_backward_pass": heads_per_pass,
+                   "l2": "inputs larger than L2 (each tensor > 126 MB); no flush",
+                   "parallelism": f"independent clip per GPU x{world}"},
+        "roofline": roof, "alu_roofline": alu, "step_roofline": step_roof,
+        "kernels": kernel_table, "gpu_launches": launches, "clocks": clocks,
+        "e2e": e2e, "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
+    """Same step through the public API with pinned host inputs and results: every step copies
+    the inputs host->device and reads back every output (out, lse, dq, dk, dv, doffsets)."""
+    names_in = ("q", "k", "v", "offsets", "dout")
+    in_bytes = sum(inp[n].numel() * inp[n].element_size() for n in names_in)
+    out_bytes = in_bytes - inp["offsets"].numel() * 4 + (w.heads * w.N * 4) * 4
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except ImportError:
+        avail = 0
+    # pinned host memory: all inputs, and every output if that stays under 60% of free RAM;
+    # otherwise the step's read-back is the offset gradient and lse only
+    read_all = in_bytes + out_bytes < 0.6 * avail
+    if in_bytes > 0.6 * avail:
+        return {"value": None, "unit": UNIT, "skipped": f"host RAM {avail >> 30} GiB too small"}
+    h_in = {}
+    try:
+        for n in names_in:
+            h_in[n] = torch.empty(inp[n].shape, dtype=inp[n].dtype, pin_memory=True)
+            h_in[n].copy_(inp[n])
+        h_out = {"lse": torch.empty((w.heads, w.N), dtype=torch.float32, pin_memory=True),
+                 "doffsets": torch.empty(inp["offsets"].shape, dtype=torch.float32, pin_memory=True)}
+        if read_all:
+            for n in ("out", "dq", "dk", "dv"):
+                h_out[n] = torch.empty(inp["q"].shape, dtype=inp["q"].dtype, pin_memory=True)
+    except RuntimeError as e:
+        return {"value": None, "unit": UNIT, "skipped": f"pinned host buffers unavailable: {e}"[:200]}
+    d_in = {n: inp[n] for n in names_in}
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for n in names_in:
+            d_in[n].copy_(h_in[n], non_blocking=True)
+        out, lse = abi.forward(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], w.dims, w.window,
+                               out=outs[0], lse=outs[1])
+        dq, dk, dv, doff = abi.backward(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], out, lse,
+                                        d_in["dout"], w.dims, w.window, workspace=ws, grads=outs[2:])
+        for n, t in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("doffsets", doff)):
+            if n in h_out:
+                h_out[n].copy_(t, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 3))
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    bi = sum(t.numel() * t.element_size() for t in h_in.values())
+    bo = sum(t.numel() * t.element_size() for t in h_out.values())
+    return {"value": w.N * world / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "read_back": sorted(h_out)}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -19,6 +19,9 @@ from .abi import (  # noqa: F401
     dsa3d_check_device,
     dsa3d_forward,
     dsa3d_status_string,
+    dsa3d_timing_enable,
+    dsa3d_timing_read,
+    dsa3d_timing_reset,
     backward,
     forward,
     library_path,

@@ -59,8 +59,19 @@ def _load():
         lib.dsa3d_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
         lib.dsa3d_check_device.restype = I
         lib.dsa3d_check_device.argtypes = [P]
+        lib.dsa3d_timing_enable.restype = I
+        lib.dsa3d_timing_enable.argtypes = [I]
+        lib.dsa3d_timing_read.restype = I
+        lib.dsa3d_timing_read.argtypes = [ctypes.POINTER(KernelTime), I]
+        lib.dsa3d_timing_reset.restype = None
+        lib.dsa3d_timing_reset.argtypes = []
         _lib = lib
         return lib
+
+
+class KernelTime(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char_p), ("launches", ctypes.c_longlong),
+                ("total_ms", ctypes.c_double)]
 
 
 # --- the C entry points, one to one -----------------------------------------------------------
@@ -92,6 +103,21 @@ def dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, works
 
 def dsa3d_check_device(stream) -> int:
     return _load().dsa3d_check_device(stream)
+
+
+def dsa3d_timing_enable(enable: bool) -> int:
+    return _load().dsa3d_timing_enable(1 if enable else 0)
+
+
+def dsa3d_timing_read() -> dict:
+    """{kernel name: (launches, total ms)} accumulated since the last reset."""
+    buf = (KernelTime * 16)()
+    n = _load().dsa3d_timing_read(buf, 16)
+    return {buf[i].kernel.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n, 16))}
+
+
+def dsa3d_timing_reset() -> None:
+    _load().dsa3d_timing_reset()
 
 
 # --- torch conveniences -----------------------------------------------------------------------

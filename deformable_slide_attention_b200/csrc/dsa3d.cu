@@ -1,0 +1,395 @@
+// dsa3d.cu -- C ABI of the 3D-DSA library: argument validation, launch configuration and the
+// extern "C" entry points declared in include/dsa3d.h.  All device work is in the kernels of
+// dsa3d_fwd.cuh / dsa3d_bwd.cuh; this file allocates no device memory.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "dsa3d.h"
+#include "dsa3d_bwd.cuh"
+#include "dsa3d_fwd.cuh"
+#include "dsa3d_timing.cuh"
+
+namespace dsa3d {
+namespace {
+
+constexpr int kWarps = 4;  // warps per CTA (one (head, query) item per warp at a time)
+
+struct Shape {
+  int F, Hp, Wp, heads, dh, kt, kh, kw;
+  int64_t N;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+Range range_of(const void* p, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return {a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+size_t elem_size(dsa3d_dtype_t t) { return t == DSA3D_F32 ? 4 : 2; }
+
+Geo make_geo(const Shape& s) {
+  Geo g;
+  g.F = s.F; g.Hp = s.Hp; g.Wp = s.Wp; g.heads = s.heads;
+  g.kt = s.kt; g.kh = s.kh; g.kw = s.kw;
+  g.Bt = s.kt + 1; g.Bh = s.kh + 1; g.Bw = s.kw + 1;
+  g.B = g.Bt * g.Bh * g.Bw;
+  g.K = s.kt * s.kh * s.kw;
+  g.HW = s.Hp * s.Wp;
+  g.N = s.N;
+  g.scale = 1.0f / std::sqrt((float)s.dh);
+  return g;
+}
+
+// Shape checks shared by every entry point.
+dsa3d_status_t check_shape(const Shape& s, dsa3d_dtype_t dtype, int warp_bytes_per_box_elem) {
+  (void)warp_bytes_per_box_elem;
+  if (dtype != DSA3D_F32 && dtype != DSA3D_BF16) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (s.F < 1 || s.Hp < 1 || s.Wp < 1 || s.heads < 1 || s.dh < 1) return DSA3D_ERR_INVALID_ARGUMENT;
+  const int dims[3] = {s.F, s.Hp, s.Wp}, win[3] = {s.kt, s.kh, s.kw};
+  for (int a = 0; a < 3; a++) {
+    if (win[a] < 1 || (win[a] & 1) == 0) return DSA3D_ERR_INVALID_ARGUMENT;
+    if ((int64_t)win[a] > 2 * (int64_t)dims[a] - 1 || win[a] > 1022) return DSA3D_ERR_UNSUPPORTED;
+  }
+  if (s.dh != 32 && s.dh != 64 && s.dh != 128) return DSA3D_ERR_UNSUPPORTED;
+  const int64_t N = (int64_t)s.F * s.Hp * s.Wp;
+  if (N >= (int64_t(1) << 31)) return DSA3D_ERR_UNSUPPORTED;
+  if ((double)N * s.heads * s.dh >= 4.0e18) return DSA3D_ERR_UNSUPPORTED;
+  const int64_t B = (int64_t)(s.kt + 1) * (s.kh + 1) * (s.kw + 1);
+  if (B > 32767) return DSA3D_ERR_UNSUPPORTED;  // box indices are stored as int16
+  return DSA3D_OK;
+}
+
+int smem_bytes(const Geo& g, int warps, bool backward) {
+  return table_smem(g.B, g.K) + warps * (backward ? bwd_warp_smem(g.B, g.K) : fwd_warp_smem(g.B, g.K));
+}
+
+// Choose warps per CTA so that the dynamic shared memory fits; 0 if even one warp does not.
+int pick_warps(const Geo& g, bool backward, int max_smem) {
+  for (int w = kWarps; w >= 1; w >>= 1)
+    if (smem_bytes(g, w, backward) <= max_smem) return w;
+  return 0;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem = 0;
+};
+DeviceInfo device_info() {
+  DeviceInfo d;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  return d;
+}
+
+template <typename Kern>
+dsa3d_status_t launch_persistent(Kern kern, int warps, int smem, int64_t items, cudaStream_t st,
+                                 int& grid_out) {
+  const DeviceInfo d = device_info();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return DSA3D_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, warps * 32, smem) != cudaSuccess)
+    return DSA3D_ERR_CUDA;
+  if (per_sm < 1) return DSA3D_ERR_UNSUPPORTED;
+  const int64_t need = (items + warps - 1) / warps;
+  int64_t grid = (int64_t)d.sms * per_sm;
+  if (need < grid) grid = need;
+  if (grid < 1) grid = 1;
+  grid_out = (int)grid;
+  (void)st;
+  return DSA3D_OK;
+}
+
+template <typename T, int DH, int W>
+dsa3d_status_t fwd_launch(const Shape& s, const void* q, const void* k, const void* v,
+                          const float* off, void* out, float* lse, cudaStream_t st) {
+  const Geo g = make_geo(s);
+  const int smem = smem_bytes(g, W, false);
+  auto kern = dsa3d_fwd_kernel<T, DH, W>;
+  int grid = 0;
+  const int64_t items = (int64_t)s.heads * s.N;
+  dsa3d_status_t rc = launch_persistent(kern, W, smem, items, st, grid);
+  if (rc != DSA3D_OK) return rc;
+  TimedLaunch tl(kKernFwd, st);
+  kern<<<grid, W * 32, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                   static_cast<const T*>(v), off, static_cast<T*>(out), lse, g, items);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+template <typename T, int DH>
+dsa3d_status_t fwd_dispatch_w(const Shape& s, int warps, const void* q, const void* k,
+                              const void* v, const float* off, void* out, float* lse,
+                              cudaStream_t st) {
+  switch (warps) {
+    case 4: return fwd_launch<T, DH, 4>(s, q, k, v, off, out, lse, st);
+    case 2: return fwd_launch<T, DH, 2>(s, q, k, v, off, out, lse, st);
+    case 1: return fwd_launch<T, DH, 1>(s, q, k, v, off, out, lse, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename T>
+dsa3d_status_t fwd_dispatch(const Shape& s, int warps, const void* q, const void* k, const void* v,
+                            const float* off, void* out, float* lse, cudaStream_t st) {
+  switch (s.dh) {
+    case 32: return fwd_dispatch_w<T, 32>(s, warps, q, k, v, off, out, lse, st);
+    case 64: return fwd_dispatch_w<T, 64>(s, warps, q, k, v, off, out, lse, st);
+    case 128: return fwd_dispatch_w<T, 128>(s, warps, q, k, v, off, out, lse, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+struct BwdArgs {
+  const void *q, *k, *v, *out, *dout;
+  const float *off, *lse;
+  void *dq, *dk, *dv;
+  float* doff;
+  float *acc_k, *acc_v;
+  int acc_heads, h0, hc;
+};
+
+template <typename T, int DH, int W>
+dsa3d_status_t bwd_launch(const Shape& s, const BwdArgs& a, cudaStream_t st) {
+  const Geo g = make_geo(s);
+  const int smem = smem_bytes(g, W, true);
+  auto kern = dsa3d_bwd_kernel<T, DH, W>;
+  int grid = 0;
+  const int64_t items = (int64_t)a.hc * s.N;
+  dsa3d_status_t rc = launch_persistent(kern, W, smem, items, st, grid);
+  if (rc != DSA3D_OK) return rc;
+  TimedLaunch tl(kKernBwd, st);
+  kern<<<grid, W * 32, smem, st>>>(
+      static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.off,
+      static_cast<const T*>(a.out), a.lse, static_cast<const T*>(a.dout), static_cast<T*>(a.dq),
+      a.doff, a.acc_k, a.acc_v, a.acc_heads, a.h0, g, items);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+template <typename T, int DH>
+dsa3d_status_t bwd_finalize(const Shape& s, const BwdArgs& a, cudaStream_t st) {
+  const DeviceInfo d = device_info();
+  const int64_t chunks = s.N * a.hc * (DH / Elems<T>::kPerLoad);
+  int64_t grid = (chunks + 255) / 256;
+  if (grid > (int64_t)d.sms * 16) grid = (int64_t)d.sms * 16;
+  if (grid < 1) grid = 1;
+  TimedLaunch tl(kKernBwdFinalize, st);
+  dsa3d_bwd_finalize_kernel<T, DH><<<(int)grid, 256, 0, st>>>(
+      a.acc_k, a.acc_v, static_cast<T*>(a.dk), static_cast<T*>(a.dv), s.heads, a.h0, a.hc, s.N);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+template <typename T, int DH>
+dsa3d_status_t bwd_dispatch_w(const Shape& s, int warps, const BwdArgs& a, cudaStream_t st) {
+  switch (warps) {
+    case 4: return bwd_launch<T, DH, 4>(s, a, st);
+    case 2: return bwd_launch<T, DH, 2>(s, a, st);
+    case 1: return bwd_launch<T, DH, 1>(s, a, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename T>
+dsa3d_status_t bwd_dispatch(const Shape& s, int warps, const BwdArgs& a, cudaStream_t st,
+                            bool finalize) {
+  dsa3d_status_t rc;
+  switch (s.dh) {
+    case 32: rc = bwd_dispatch_w<T, 32>(s, warps, a, st); break;
+    case 64: rc = bwd_dispatch_w<T, 64>(s, warps, a, st); break;
+    case 128: rc = bwd_dispatch_w<T, 128>(s, warps, a, st); break;
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+  if (rc != DSA3D_OK || !finalize) return rc;
+  switch (s.dh) {
+    case 32: return bwd_finalize<T, 32>(s, a, st);
+    case 64: return bwd_finalize<T, 64>(s, a, st);
+    case 128: return bwd_finalize<T, 128>(s, a, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+// Zero n16 16-byte words at p (the backward's fp32 accumulators).
+dsa3d_status_t zero16(void* p, size_t n16, cudaStream_t st) {
+  const DeviceInfo d = device_info();
+  int64_t grid = ((int64_t)n16 + 255) / 256;
+  if (grid > (int64_t)d.sms * 8) grid = (int64_t)d.sms * 8;
+  if (grid < 1) grid = 1;
+  TimedLaunch tl(kKernZero, st);
+  dsa3d_zero_kernel<<<(int)grid, 256, 0, st>>>(static_cast<uint4*>(p), (int64_t)n16);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+size_t acc_bytes_per_head(const Shape& s) { return (size_t)2 * s.N * s.dh * sizeof(float); }
+
+}  // namespace
+}  // namespace dsa3d
+
+using namespace dsa3d;
+
+extern "C" {
+
+int dsa3d_abi_version(void) { return DSA3D_ABI_VERSION; }
+
+const char* dsa3d_status_string(dsa3d_status_t status) {
+  switch (status) {
+    case DSA3D_OK: return "ok";
+    case DSA3D_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case DSA3D_ERR_UNSUPPORTED: return "unsupported shape or window";
+    case DSA3D_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case DSA3D_ERR_CUDA: return "CUDA error";
+    case DSA3D_ERR_DEVICE_CHECK: return "device-side check failed";
+    default: return "unknown status";
+  }
+}
+
+dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const float* offsets,
+                             void* out, float* lse, int F, int Hp, int Wp, int heads, int dh,
+                             int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  dsa3d_status_t rc = check_shape(s, dtype, 0);
+  if (rc != DSA3D_OK) return rc;
+  if (!q || !k || !v || !offsets || !out) return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al[] = {q, k, v, offsets, out};
+  for (const void* p : al)
+    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DSA3D_ERR_INVALID_ARGUMENT;
+  const size_t tb = (size_t)s.N * heads * dh * elem_size(dtype);
+  const Range in[] = {range_of(q, tb), range_of(k, tb), range_of(v, tb),
+                      range_of(offsets, (size_t)heads * s.N * 12)};
+  const Range ro = range_of(out, tb);
+  const Range rl = range_of(lse, lse ? (size_t)heads * s.N * 4 : 0);
+  for (const Range& r : in)
+    if (overlap(r, ro) || (lse && overlap(r, rl))) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (lse && overlap(ro, rl)) return DSA3D_ERR_INVALID_ARGUMENT;
+
+  const Geo g = make_geo(s);
+  const DeviceInfo d = device_info();
+  const int warps = pick_warps(g, false, d.max_smem);
+  if (warps == 0) return DSA3D_ERR_UNSUPPORTED;
+  if (dtype == DSA3D_F32)
+    return fwd_dispatch<float>(s, warps, q, k, v, offsets, out, lse, stream);
+  return fwd_dispatch<__nv_bfloat16>(s, warps, q, k, v, offsets, out, lse, stream);
+}
+
+size_t dsa3d_backward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,
+                                      int kw, dsa3d_dtype_t dtype) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  if (check_shape(s, dtype, 0) != DSA3D_OK) return 0;
+  if (dtype == DSA3D_F32) return 0;
+  return acc_bytes_per_head(s) * (size_t)heads;
+}
+
+dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const float* offsets,
+                              const void* out, const float* lse, const void* dout, void* dq,
+                              void* dk, void* dv, float* doffsets, void* workspace,
+                              size_t workspace_bytes, int F, int Hp, int Wp, int heads, int dh,
+                              int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  dsa3d_status_t rc = check_shape(s, dtype, 0);
+  if (rc != DSA3D_OK) return rc;
+  if (!q || !k || !v || !offsets || !out || !lse || !dout || !dq || !dk || !dv || !doffsets)
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al[] = {q, k, v, offsets, out, dout, dq, dk, dv, doffsets};
+  for (const void* p : al)
+    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return DSA3D_ERR_INVALID_ARGUMENT;
+  const size_t tb = (size_t)s.N * heads * dh * elem_size(dtype);
+  const size_t ob = (size_t)heads * s.N * 12;
+  const Range ins[] = {range_of(q, tb), range_of(k, tb), range_of(v, tb), range_of(offsets, ob),
+                       range_of(out, tb), range_of(lse, (size_t)heads * s.N * 4),
+                       range_of(dout, tb)};
+  const Range outs[] = {range_of(dq, tb), range_of(dk, tb), range_of(dv, tb),
+                        range_of(doffsets, ob)};
+  for (int i = 0; i < 4; i++) {
+    for (const Range& r : ins)
+      if (overlap(r, outs[i])) return DSA3D_ERR_INVALID_ARGUMENT;
+    for (int j = i + 1; j < 4; j++)
+      if (overlap(outs[i], outs[j])) return DSA3D_ERR_INVALID_ARGUMENT;
+  }
+
+  const size_t per_head = acc_bytes_per_head(s);
+  if (dtype == DSA3D_BF16) {
+    if (!workspace || workspace_bytes < per_head) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return DSA3D_ERR_INVALID_ARGUMENT;
+    const Range rw = range_of(workspace, workspace_bytes);
+    for (const Range& r : ins)
+      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+    for (const Range& r : outs)
+      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+  }
+
+  const Geo g = make_geo(s);
+  const DeviceInfo d = device_info();
+  const int warps = pick_warps(g, true, d.max_smem);
+  if (warps == 0) return DSA3D_ERR_UNSUPPORTED;
+
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.off = offsets; a.lse = lse;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.doff = doffsets;
+
+  if (dtype == DSA3D_F32) {
+    // accumulate straight into the fp32 outputs
+    if ((rc = zero16(dk, tb / 16, stream)) != DSA3D_OK) return rc;
+    if ((rc = zero16(dv, tb / 16, stream)) != DSA3D_OK) return rc;
+    a.acc_k = static_cast<float*>(dk);
+    a.acc_v = static_cast<float*>(dv);
+    a.acc_heads = heads;
+    a.h0 = 0;
+    a.hc = heads;
+    return bwd_dispatch<float>(s, warps, a, stream, false);
+  }
+
+  int hc_max = (int)(workspace_bytes / per_head);
+  if (hc_max > heads) hc_max = heads;
+  for (int h0 = 0; h0 < heads; h0 += hc_max) {
+    const int hc = (heads - h0 < hc_max) ? heads - h0 : hc_max;
+    const size_t half = (size_t)s.N * hc * dh;  // floats per accumulator
+    a.acc_k = static_cast<float*>(workspace);
+    a.acc_v = a.acc_k + half;
+    a.acc_heads = hc;
+    a.h0 = h0;
+    a.hc = hc;
+    if ((rc = zero16(workspace, 2 * half * sizeof(float) / 16, stream)) != DSA3D_OK) return rc;
+    rc = bwd_dispatch<__nv_bfloat16>(s, warps, a, stream, true);
+    if (rc != DSA3D_OK) return rc;
+  }
+  return DSA3D_OK;
+}
+
+dsa3d_status_t dsa3d_timing_enable(int enable) {
+  Timing::get().enable(enable != 0);
+  return DSA3D_OK;
+}
+
+int dsa3d_timing_read(dsa3d_kernel_time_t* out, int max_entries) {
+  return Timing::get().read(out, max_entries);
+}
+
+void dsa3d_timing_reset(void) { Timing::get().reset(); }
+
+dsa3d_status_t dsa3d_check_device(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return DSA3D_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_dsa3d_check, sizeof(int)) != cudaSuccess) return DSA3D_ERR_CUDA;
+  if (flag) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_dsa3d_check, &zero, sizeof(int)) != cudaSuccess) return DSA3D_ERR_CUDA;
+    return DSA3D_ERR_DEVICE_CHECK;
+  }
+  return DSA3D_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,130 @@
+/*
+ * dsa3d.h -- C ABI of the B200 (sm_100a) 3D Deformable Slide Attention library (libdsa3d.so).
+ *
+ * Operator: 3D-DSA from MegaSlide-DiT, "Memory-Centric Adaptation and Deformable Local Attention
+ * for Efficient Video Diffusion" (arXiv 2607.22696), the 3D-DSA definition: Eq. 1's attention
+ * term and the softmax over the k_t x k_h x k_w neighbourhood that follows it.  For every head h
+ * and query token p = (t, y, x) of a T x H' x W' token grid:
+ *
+ *   out[p,h] = sum_tau alpha_tau * Trilinear(V[.,h], p + tau + delta[h,p])
+ *   alpha    = softmax_tau( q[p,h] . Trilinear(K[.,h], p + tau + delta[h,p]) / sqrt(dh) )
+ *
+ * with tau over the centred window [-r_t..r_t] x [-r_h..r_h] x [-r_w..r_w], r = (k-1)/2, and one
+ * offset 3-vector delta = (dt, dy, dx) per (token, head).  Positions follow grid_sample's
+ * align_corners=True convention (integer coordinate = token centre).  The offset is decoded in
+ * single precision: i = floor(delta), f = delta - i (round to nearest), f == 1 carries into i.
+ * A tap whose sample position leaves the closed box [0, dim-1] on any axis is masked out of the
+ * softmax; trilinear corners outside the volume read as zero.  A query with no valid tap, or with
+ * a non-finite offset or |offset| > 2^24, gets out = 0 and lse = -inf and has zero gradient.
+ * No causal mask.  The DWConv3D term of Eq. 1 is not computed here: the caller adds it.
+ *
+ * Layouts (row-major, token n = (t*H' + y)*W' + x, N = T*H'*W'):
+ *   q, k, v, out, dout, dq, dk, dv : [N][heads][dh]   in the I/O type (fp32 or bf16)
+ *   offsets, doffsets              : [heads][N][3]    fp32, order (dt, dy, dx)
+ *   lse                            : [heads][N]       fp32, natural log of the softmax sum
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, 16-byte aligned.  Outputs are
+ *     fully overwritten (never accumulated) and must not overlap any input or each other.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; 0 = the legacy default
+ *     stream).  The returned status covers argument validation and launch errors only; a later
+ *     device-side failure surfaces through CUDA's own error reporting or dsa3d_check_device.
+ *   - The library allocates no device memory.  The backward takes a caller-owned workspace.
+ *   - Supported: dh in {32, 64, 128}; odd window sizes 1 <= k <= 2*dim - 1 on each axis;
+ *     every extent >= 1; N*heads*dh < 2^62.  Other shapes return DSA3D_ERR_UNSUPPORTED.
+ *   - Thread safety: calls on different streams may run concurrently.
+ */
+#ifndef DSA3D_H
+#define DSA3D_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA3D_ABI_VERSION 1
+
+typedef enum {
+    DSA3D_OK = 0,
+    DSA3D_ERR_INVALID_ARGUMENT = 1,   /* null/misaligned pointer, bad extent, aliasing, bad dtype */
+    DSA3D_ERR_UNSUPPORTED = 2,        /* valid arguments this build does not handle (dh, window) */
+    DSA3D_ERR_WORKSPACE_TOO_SMALL = 3,
+    DSA3D_ERR_CUDA = 4,               /* a CUDA runtime call or kernel launch failed */
+    DSA3D_ERR_DEVICE_CHECK = 5        /* a kernel recorded a failed internal check */
+} dsa3d_status_t;
+
+typedef enum { DSA3D_F32 = 0, DSA3D_BF16 = 1 } dsa3d_dtype_t;
+
+/* DSA3D_ABI_VERSION of the loaded library. */
+int dsa3d_abi_version(void);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *dsa3d_status_string(dsa3d_status_t status);
+
+/*
+ * Forward: out (and lse, if non-NULL) for every (token, head).
+ *   q, k, v  [N][heads][dh] I/O type;  offsets [heads][N][3] fp32;
+ *   out      [N][heads][dh] I/O type (written);  lse [heads][N] fp32 (written; may be NULL).
+ *   F, Hp, Wp: frames and token grid (T, H', W');  kt, kh, kw: window (odd).
+ * The backward needs lse; pass NULL only for inference.
+ */
+dsa3d_status_t dsa3d_forward(const void *q, const void *k, const void *v, const float *offsets,
+                             void *out, float *lse, int F, int Hp, int Wp, int heads, int dh,
+                             int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * Bytes of workspace dsa3d_backward needs to process all heads in one pass.  Any workspace of at
+ * least the size returned for heads = 1 works (heads are then processed in groups that fit);
+ * larger is faster.  Returns 0 when no workspace is needed (fp32 I/O), and 0 for unsupported or
+ * invalid shapes (the backward call itself then reports the error).
+ */
+size_t dsa3d_backward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,
+                                      int kw, dsa3d_dtype_t dtype);
+
+/*
+ * Backward: gradients of sum(out * dout) with respect to q, k, v and the offsets.
+ *   q, k, v, offsets: the forward's inputs;  out, lse: the forward's outputs (lse required);
+ *   dout [N][heads][dh] I/O type;
+ *   dq, dk, dv [N][heads][dh] I/O type (written);  doffsets [heads][N][3] fp32 (written);
+ *   workspace: device scratch of workspace_bytes bytes (contents on entry are ignored).
+ * The offset gradient is the derivative of the trilinear weights within the cell [i, i+1]; the
+ * mask and the integer part of the offset are held fixed.
+ */
+dsa3d_status_t dsa3d_backward(const void *q, const void *k, const void *v, const float *offsets,
+                              const void *out, const float *lse, const void *dout, void *dq,
+                              void *dk, void *dv, float *doffsets, void *workspace,
+                              size_t workspace_bytes, int F, int Hp, int Wp, int heads, int dh,
+                              int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * Synchronises `stream` and reports DSA3D_ERR_DEVICE_CHECK if any kernel of this library on the
+ * current device recorded a failed internal check since the last call (the record is then
+ * cleared), DSA3D_ERR_CUDA if the stream reports an error, else DSA3D_OK.
+ */
+dsa3d_status_t dsa3d_check_device(cudaStream_t stream);
+
+/*
+ * Per-kernel timing (profiling aid; off by default).  While enabled, every kernel this library
+ * launches is bracketed by two CUDA events recorded on the launch's own stream.
+ * dsa3d_timing_read waits for the pending events, adds each launch's duration to the totals of
+ * its kernel, and copies up to max_entries totals (kernel name, launch count, total ms) into
+ * out; it returns the number of kernels with totals.  dsa3d_timing_reset clears the totals.
+ * Host-side state is process-wide and mutex-protected.
+ */
+typedef struct {
+    const char *kernel;  /* static string */
+    long long launches;
+    double total_ms;
+} dsa3d_kernel_time_t;
+
+dsa3d_status_t dsa3d_timing_enable(int enable);
+int dsa3d_timing_read(dsa3d_kernel_time_t *out, int max_entries);
+void dsa3d_timing_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA3D_H */

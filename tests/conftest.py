@@ -18,3 +18,14 @@ def oracle_lib():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def gpu_lib():
+    """The CUDA library, built in-tree if stale; a GPU test without a CUDA device fails loudly."""
+    import torch
+    from deformable_slide_attention_b200 import abi, build
+    build.build()
+    assert torch.cuda.is_available(), "GPU test run without a CUDA device"
+    assert abi.dsa3d_abi_version() == 1
+    return abi

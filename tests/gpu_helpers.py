@@ -1,0 +1,78 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI binding and
+compare with the CPU oracle on the same seeded inputs."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from deformable_slide_attention_b200 import abi
+
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+
+
+def to_cuda(inp):
+    return {k: v.cuda().contiguous() for k, v in inp.items()}
+
+
+def gpu_forward(d, dims, window):
+    out, lse = abi.forward(d["q"], d["k"], d["v"], d["offsets"], dims, window)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def gpu_backward(d, out, lse, dims, window):
+    grads = abi.backward(d["q"], d["k"], d["v"], d["offsets"], out, lse, d["dout"], dims, window)
+    torch.cuda.synchronize()
+    return grads
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def items_of(heads, N, n_sample, seed, include_edges=True):
+    """A seeded sample of h*N + n items, with each head's first and last tokens included."""
+    g = np.random.default_rng(seed)
+    items = set(g.integers(0, heads * N, size=n_sample).tolist())
+    if include_edges:
+        for h in range(heads):
+            items.update([h * N, h * N + N - 1])
+    return np.array(sorted(items), dtype=np.int64)
+
+
+def gather_rows(t, items, N):
+    """t [N][heads][dh] -> rows [len(items)][dh] for items h*N + n."""
+    h, n = items // N, items % N
+    return f64(t)[n, h]
+
+
+def assert_close(name, got, ref, tol):
+    got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.isfinite(got), fin), f"{name}: finiteness differs"
+    err = np.abs(got[fin] - ref[fin]).max(initial=0.0)
+    scale = np.abs(ref[fin]).max(initial=0.0)
+    assert err <= tol, f"{name}: max-abs error {err:.3e} > {tol:.1e} (max |ref| {scale:.3g})"
+    eq_inf = got[~fin] == ref[~fin]
+    assert eq_inf.all(), f"{name}: non-finite entries differ"
+    return err
+
+
+def full_parity(inp, dims, window, dtype, backward=True):
+    """Element-by-element comparison of every output with the oracle."""
+    tol = TOL[dtype]
+    d = to_cuda(inp)
+    out, lse = gpu_forward(d, dims, window)
+    r_out, r_lse = oracle.full_forward(inp["q"], inp["k"], inp["v"], inp["offsets"], dims, window)
+    errs = {"out": assert_close("out", f64(out), r_out, tol),
+            "lse": assert_close("lse", f64(lse), r_lse, max(tol, 1e-5))}
+    if backward:
+        dq, dk, dv, doff = gpu_backward(d, out, lse, dims, window)
+        r = oracle.full_backward(inp["q"], inp["k"], inp["v"], inp["offsets"], inp["dout"], dims,
+                                 window)
+        for name, got, ref in (("dq", dq, r[0]), ("doff", doff, r[1]), ("dk", dk, r[2]),
+                               ("dv", dv, r[3])):
+            errs[name] = assert_close(name, f64(got), ref, tol)
+    return errs

@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every function the
+header declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from deformable_slide_attention_b200 import abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ctypes.CDLL(abi.library_path())
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(dsa3d_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"dsa3d_forward", "dsa3d_backward", "dsa3d_backward_workspace_bytes",
+            "dsa3d_abi_version", "dsa3d_status_string", "dsa3d_check_device"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_abi_version_and_status_strings():
+    assert abi.dsa3d_abi_version() == 1
+    for s in range(6):
+        assert abi.dsa3d_status_string(s)
+    assert abi.dsa3d_status_string(0) == "ok"
+
+
+ARGS = dict(F=4, Hp=8, Wp=8, heads=2, dh=64, kt=3, kh=3, kw=3)
+P = 1 << 20  # a fake 16-byte-aligned address; validation fails before any device access
+
+
+def fwd(**kw):
+    a = {**ARGS, **kw}
+    ptrs = [kw.get(n, P * (i + 1)) for i, n in enumerate(["q", "k", "v", "off", "out", "lse"])]
+    return abi.dsa3d_forward(*ptrs, a["F"], a["Hp"], a["Wp"], a["heads"], a["dh"], a["kt"], a["kh"],
+                             a["kw"], kw.get("dtype", abi.DSA3D_BF16), 0)
+
+
+def test_forward_rejects_bad_arguments():
+    INV, UNS = 1, 2
+    assert fwd(q=0) == INV
+    assert fwd(out=P + 8) == INV  # misaligned
+    assert fwd(kt=2) == INV       # even window
+    assert fwd(kw=0) == INV
+    assert fwd(F=0) == INV
+    assert fwd(heads=0) == INV
+    assert fwd(dtype=7) == INV
+    assert fwd(dh=48) == UNS
+    assert fwd(kh=17) == UNS      # larger than 2*Hp-1
+    # out overlapping q
+    assert fwd(q=P, out=P + 4096) == INV
+
+
+def test_backward_workspace_bytes():
+    ws = abi.dsa3d_backward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_BF16)
+    assert ws == 2 * 256 * 64 * 4 * 2
+    assert abi.dsa3d_backward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_F32) == 0
+    assert abi.dsa3d_backward_workspace_bytes(4, 8, 8, 2, 48, 3, 3, 3, abi.DSA3D_BF16) == 0
+
+
+def test_backward_rejects_bad_arguments():
+    ptr = [P * (i + 1) for i in range(12)]
+    a = ARGS
+    call = lambda ptrs, wsb=0, dtype=abi.DSA3D_BF16, **kw: abi.dsa3d_backward(
+        *ptrs, wsb, kw.get("F", a["F"]), a["Hp"], a["Wp"], a["heads"], a["dh"], a["kt"], a["kh"],
+        a["kw"], dtype, 0)
+    bad = list(ptr)
+    bad[2] = 0
+    assert call(bad) == 1
+    # workspace too small for one head
+    assert call(ptr, wsb=1000) == 3
+    # dk aliasing q
+    alias = list(ptr)
+    alias[8] = ptr[0]
+    assert call(alias, wsb=1 << 30) == 1
