@@ -57,6 +57,8 @@ def _load():
         lib.dsa3d_backward_workspace_bytes.argtypes = [*dims, I]
         lib.dsa3d_backward.restype = I
         lib.dsa3d_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
+        lib.dsa3d_backward_noalloc.restype = I
+        lib.dsa3d_backward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P, *dims, I, P]
         lib.dsa3d_check_device.restype = I
         lib.dsa3d_check_device.argtypes = [P]
         lib.dsa3d_timing_enable.restype = I
@@ -99,6 +101,14 @@ def dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, works
                    workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream) -> int:
     return _load().dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, workspace,
                                   workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream)
+
+
+def dsa3d_backward_noalloc(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, F, Hp, Wp,
+                           heads, dh, kt, kh, kw, dtype, stream) -> int:
+    """The backward for callers that cannot allocate: its scratch is a fixed device array inside
+    the library (see include/dsa3d.h)."""
+    return _load().dsa3d_backward_noalloc(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets,
+                                          F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream)
 
 
 def dsa3d_check_device(stream) -> int:

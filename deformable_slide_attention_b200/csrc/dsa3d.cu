@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "dsa3d.h"
 #include "dsa3d_bwd.cuh"
@@ -234,6 +235,29 @@ dsa3d_status_t zero16(void* p, size_t n16, cudaStream_t st) {
 
 size_t acc_bytes_per_head(const Shape& s) { return (size_t)2 * s.N * s.dh * sizeof(float); }
 
+// Scratch of dsa3d_backward_noalloc: a file-scope device array, so that entry point never
+// allocates.  Host code must not use the symbol as an address; noalloc_scratch() looks up the
+// device address once per device (with that device current) and caches it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DSA3D_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+dsa3d_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSA3D_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DSA3D_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DSA3D_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA3D_OK;
+}
+
 }  // namespace
 }  // namespace dsa3d
 
@@ -367,6 +391,26 @@ dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const
     if (rc != DSA3D_OK) return rc;
   }
   return DSA3D_OK;
+}
+
+dsa3d_status_t dsa3d_backward_noalloc(const void* q, const void* k, const void* v,
+                                      const float* offsets, const void* out, const float* lse,
+                                      const void* dout, void* dq, void* dk, void* dv,
+                                      float* doffsets, int F, int Hp, int Wp, int heads, int dh,
+                                      int kt, int kh, int kw, dsa3d_dtype_t dtype,
+                                      cudaStream_t stream) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  const dsa3d_status_t rc = check_shape(s, dtype, 0);
+  if (rc != DSA3D_OK) return rc;
+  // reject, before any device work, a head that does not fit the fixed scratch
+  if (dtype == DSA3D_BF16 && acc_bytes_per_head(s) > DSA3D_NOALLOC_SCRATCH_BYTES)
+    return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  const dsa3d_status_t sc = noalloc_scratch(&scratch);
+  if (sc != DSA3D_OK) return sc;
+  return dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, scratch,
+                        DSA3D_NOALLOC_SCRATCH_BYTES, F, Hp, Wp, heads, dh, kt, kh, kw, dtype,
+                        stream);
 }
 
 dsa3d_status_t dsa3d_timing_enable(int enable) {

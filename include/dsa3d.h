@@ -99,6 +99,33 @@ dsa3d_status_t dsa3d_backward(const void *q, const void *k, const void *v, const
                               int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * Backward without a caller workspace (the paper has no counterpart: this is a library-usage
+ * entry point).  For callers that cannot allocate device memory or pass a workspace: plugin hosts
+ * that own every device allocation and hand the operator only its tensors, fixed call signatures
+ * with no workspace argument, and steps that must not pay cudaMalloc's device-wide
+ * synchronisation.  Arguments, results and errors are those of dsa3d_backward.
+ *
+ * Its scratch (the fp32 dK/dV accumulators of one head group) is a file-scope device array of
+ * DSA3D_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the library holds
+ * until the process exits.  Heads are processed in groups that fit; a problem whose single head
+ * needs more than the array (2 * N * dh * 4 bytes with bf16 I/O; fp32 I/O needs none) is
+ * rejected with DSA3D_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ * The first call on each device looks up the array's device address (on the current device) and
+ * caches it; make that first call before any stream capture.  The array is shared by every call
+ * and keeps the previous call's contents (the accumulators are cleared before use): calls that
+ * overlap on the GPU -- on different streams, or from different threads -- race on it.
+ * The function calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define DSA3D_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+dsa3d_status_t dsa3d_backward_noalloc(const void *q, const void *k, const void *v,
+                                      const float *offsets, const void *out, const float *lse,
+                                      const void *dout, void *dq, void *dk, void *dv,
+                                      float *doffsets, int F, int Hp, int Wp, int heads, int dh,
+                                      int kt, int kh, int kw, dsa3d_dtype_t dtype,
+                                      cudaStream_t stream);
+
+/*
  * Synchronises `stream` and reports DSA3D_ERR_DEVICE_CHECK if any kernel of this library on the
  * current device recorded a failed internal check since the last call (the record is then
  * cleared), DSA3D_ERR_CUDA if the stream reports an error, else DSA3D_OK.
