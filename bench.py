@@ -239,6 +239,8 @@ def main(argv=None):
     out = torch.empty_like(q)
     lse = torch.empty((w.heads, w.N), dtype=torch.float32, device=dev)
     dq, dk, dv, doff = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(off)
+    fws_bytes = abi.dsa3d_forward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
+    fws = torch.empty(fws_bytes, dtype=torch.uint8, device=dev) if fws_bytes else None
     full_ws = abi.dsa3d_backward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
     per_head = full_ws // w.heads if full_ws else 0
     free, _ = torch.cuda.mem_get_info(dev)
@@ -248,8 +250,8 @@ def main(argv=None):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        abi.forward(q, k, v, off, w.dims, w.window, out=out, lse=lse)
-        abi.backward(q, k, v, off, out, lse, do, w.dims, w.window, workspace=ws, grads=(dq, dk, dv, doff))
+        abi.forward(q, k, v, off, w.dims, w.window, out=out, lse=lse, workspace=fws)
+        abi.backward(q, k, v, off, lse, do, w.dims, w.window, workspace=ws, grads=(dq, dk, dv, doff))
 
     def barrier():
         if world > 1:
@@ -297,7 +299,8 @@ def main(argv=None):
         kname, (n, tot) = dominant
         avg_ms = tot / n
         kind = "fwd" if "fwd" in kname else "bwd"
-        items_per_launch = w.heads * w.N if kind == "fwd" else w.N * heads_per_pass
+        launches_per_step = n / args.steps
+        items_per_launch = w.heads * w.N / launches_per_step
         alg = alg_bytes_per_item(w, kind) * items_per_launch
         achieved = alg / (avg_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
@@ -318,7 +321,7 @@ def main(argv=None):
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_leg(args, w, inp, abi, torch, dev, ws, world, (out, lse, dq, dk, dv, doff))
+        e2e = e2e_leg(args, w, inp, abi, torch, dev, (fws, ws), world, (out, lse, dq, dk, dv, doff))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -380,9 +383,9 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
         for n in names_in:
             d_in[n].copy_(h_in[n], non_blocking=True)
         out, lse = abi.forward(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], w.dims, w.window,
-                               out=outs[0], lse=outs[1])
-        dq, dk, dv, doff = abi.backward(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], out, lse,
-                                        d_in["dout"], w.dims, w.window, workspace=ws, grads=outs[2:])
+                               out=outs[0], lse=outs[1], workspace=ws[0])
+        dq, dk, dv, doff = abi.backward(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], lse,
+                                        d_in["dout"], w.dims, w.window, workspace=ws[1], grads=outs[2:])
         for n, t in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("doffsets", doff)):
             if n in h_out:
                 h_out[n].copy_(t, non_blocking=True)

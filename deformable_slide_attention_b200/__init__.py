@@ -18,6 +18,7 @@ from .abi import (  # noqa: F401
     dsa3d_backward_workspace_bytes,
     dsa3d_check_device,
     dsa3d_forward,
+    dsa3d_forward_workspace_bytes,
     dsa3d_status_string,
     dsa3d_timing_enable,
     dsa3d_timing_read,

@@ -52,13 +52,15 @@ def _load():
         lib.dsa3d_status_string.restype = ctypes.c_char_p
         lib.dsa3d_status_string.argtypes = [I]
         lib.dsa3d_forward.restype = I
-        lib.dsa3d_forward.argtypes = [P, P, P, P, P, P, *dims, I, P]
+        lib.dsa3d_forward.argtypes = [P, P, P, P, P, P, P, Z, *dims, I, P]
+        lib.dsa3d_forward_workspace_bytes.restype = Z
+        lib.dsa3d_forward_workspace_bytes.argtypes = [*dims, I]
         lib.dsa3d_backward_workspace_bytes.restype = Z
         lib.dsa3d_backward_workspace_bytes.argtypes = [*dims, I]
         lib.dsa3d_backward.restype = I
-        lib.dsa3d_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
+        lib.dsa3d_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
         lib.dsa3d_backward_noalloc.restype = I
-        lib.dsa3d_backward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P, *dims, I, P]
+        lib.dsa3d_backward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, *dims, I, P]
         lib.dsa3d_check_device.restype = I
         lib.dsa3d_check_device.argtypes = [P]
         lib.dsa3d_timing_enable.restype = I
@@ -88,26 +90,31 @@ def dsa3d_status_string(status: int) -> str:
         return _STATUS.get(status, "unknown status")
 
 
-def dsa3d_forward(q, k, v, offsets, out, lse, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream) -> int:
-    return _load().dsa3d_forward(q, k, v, offsets, out, lse, F, Hp, Wp, heads, dh, kt, kh, kw,
-                                 dtype, stream)
+def dsa3d_forward(q, k, v, offsets, out, lse, workspace, workspace_bytes, F, Hp, Wp, heads, dh,
+                  kt, kh, kw, dtype, stream) -> int:
+    return _load().dsa3d_forward(q, k, v, offsets, out, lse, workspace, workspace_bytes, F, Hp, Wp,
+                                 heads, dh, kt, kh, kw, dtype, stream)
+
+
+def dsa3d_forward_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype) -> int:
+    return _load().dsa3d_forward_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype)
 
 
 def dsa3d_backward_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype) -> int:
     return _load().dsa3d_backward_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype)
 
 
-def dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, workspace,
-                   workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream) -> int:
-    return _load().dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, workspace,
+def dsa3d_backward(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace, workspace_bytes,
+                   F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream) -> int:
+    return _load().dsa3d_backward(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace,
                                   workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream)
 
 
-def dsa3d_backward_noalloc(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, F, Hp, Wp,
-                           heads, dh, kt, kh, kw, dtype, stream) -> int:
+def dsa3d_backward_noalloc(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, F, Hp, Wp, heads,
+                           dh, kt, kh, kw, dtype, stream) -> int:
     """The backward for callers that cannot allocate: its scratch is a fixed device array inside
     the library (see include/dsa3d.h)."""
-    return _load().dsa3d_backward_noalloc(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets,
+    return _load().dsa3d_backward_noalloc(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets,
                                           F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream)
 
 
@@ -167,25 +174,36 @@ def _shapes(q, offsets, dims):
     return N, heads, dh
 
 
-def forward(q, k, v, offsets, dims, window, out=None, lse=None, stream=None, want_lse=True):
-    """3D-DSA forward on CUDA tensors.  Returns (out [N][heads][dh], lse [heads][N] or None)."""
+def forward(q, k, v, offsets, dims, window, out=None, lse=None, stream=None, want_lse=True,
+            workspace="auto"):
+    """3D-DSA forward on CUDA tensors.  Returns (out [N][heads][dh], lse [heads][N] or None).
+
+    workspace: "auto" allocates what dsa3d_forward_workspace_bytes asks for (the sorted
+    tensor-core path where the shape has one); None runs the general CUDA-core kernel; a uint8
+    CUDA tensor is used as given.
+    """
     torch = _torch()
     N, heads, dh = _shapes(q, offsets, dims)
     for t in (q, k, v, offsets):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError("inputs must be contiguous CUDA tensors")
+    code = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((heads, N), dtype=torch.float32, device=q.device)
+    if isinstance(workspace, str):
+        need = dsa3d_forward_workspace_bytes(*dims, heads, dh, *window, code)
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device) if need else None
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(dsa3d_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(), out.data_ptr(),
-                         lse.data_ptr() if lse is not None else None, *dims, heads, dh, *window,
-                         _dtype_code(q), _stream_handle(stream)), "dsa3d_forward")
+                         lse.data_ptr() if lse is not None else None, ws_ptr, ws_bytes, *dims, heads,
+                         dh, *window, code, _stream_handle(stream)), "dsa3d_forward")
     return out, lse
 
 
-def backward(q, k, v, offsets, out, lse, dout, dims, window, workspace=None, stream=None,
-             grads=None):
+def backward(q, k, v, offsets, lse, dout, dims, window, workspace=None, stream=None, grads=None):
     """3D-DSA backward on CUDA tensors.  Returns (dq, dk, dv, doffsets)."""
     torch = _torch()
     N, heads, dh = _shapes(q, offsets, dims)
@@ -199,7 +217,7 @@ def backward(q, k, v, offsets, out, lse, dout, dims, window, workspace=None, str
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(dsa3d_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(), out.data_ptr(),
+    _check(dsa3d_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(),
                           lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                           doff.data_ptr(), ws_ptr, ws_bytes, *dims, heads, dh, *window, code,
                           _stream_handle(stream)), "dsa3d_backward")

@@ -11,6 +11,8 @@
 #include "dsa3d.h"
 #include "dsa3d_bwd.cuh"
 #include "dsa3d_fwd.cuh"
+#include "dsa3d_fwd_mma.cuh"
+#include "dsa3d_sort.cuh"
 #include "dsa3d_timing.cuh"
 
 namespace dsa3d {
@@ -151,8 +153,113 @@ dsa3d_status_t fwd_dispatch(const Shape& s, int warps, const void* q, const void
   }
 }
 
+// --- sorted tensor-core forward ---------------------------------------------------------------
+bool mma_forward_ok(const Shape& s, dsa3d_dtype_t dtype) {
+  return dtype == DSA3D_BF16 && (s.dh == 64 || s.dh == 128) && s.kw <= 15;
+}
+
+SortGeo make_sort_geo(const Shape& s) {
+  SortGeo sg;
+  sg.Et = s.F + s.kt;
+  sg.Ey = s.Hp + s.kh;
+  sg.Ex = s.Wp + s.kw;
+  sg.E1 = (int64_t)sg.Et * sg.Ey * sg.Ex + 1;
+  return sg;
+}
+
+// Workspace layout for hg heads: cnt/start [hg*E1] | qkey [hg*N] | qrank [hg*N] |
+// sorted_n [hg*N] | sorted_ex [hg*N] | block sums; every part 16-byte aligned.
+struct SortWs {
+  int *cnt, *qkey, *qrank, *sorted_n, *sorted_ex, *bsum;
+  int64_t cnt_elems, nb;
+};
+size_t align16(size_t b) { return (b + 15) & ~size_t(15); }
+size_t sort_ws_bytes(const Shape& s, int hg) {
+  const SortGeo sg = make_sort_geo(s);
+  const int64_t cnt = (int64_t)hg * sg.E1;
+  const int64_t nb = (cnt + kScanTile - 1) / kScanTile;
+  return align16(cnt * 4) + 4 * align16((size_t)hg * s.N * 4) + align16(nb * 4);
+}
+SortWs carve_sort_ws(const Shape& s, int hg, void* base) {
+  const SortGeo sg = make_sort_geo(s);
+  SortWs w;
+  w.cnt_elems = (int64_t)hg * sg.E1;
+  w.nb = (w.cnt_elems + kScanTile - 1) / kScanTile;
+  char* p = static_cast<char*>(base);
+  w.cnt = reinterpret_cast<int*>(p);
+  p += align16(w.cnt_elems * 4);
+  const size_t qb = align16((size_t)hg * s.N * 4);
+  w.qkey = reinterpret_cast<int*>(p);
+  p += qb;
+  w.qrank = reinterpret_cast<int*>(p);
+  p += qb;
+  w.sorted_n = reinterpret_cast<int*>(p);
+  p += qb;
+  w.sorted_ex = reinterpret_cast<int*>(p);
+  p += qb;
+  w.bsum = reinterpret_cast<int*>(p);
+  return w;
+}
+
+int grid_for(int64_t work, int threads, int per_sm_cap) {
+  const DeviceInfo d = device_info();
+  int64_t grid = (work + threads - 1) / threads;
+  const int64_t cap = (int64_t)d.sms * per_sm_cap;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  return (int)grid;
+}
+
+dsa3d_status_t zero16(void* p, size_t n16, cudaStream_t st);
+
+template <int DH>
+dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const void* v,
+                             const float* off, void* out, float* lse, const SortWs& w, int h0,
+                             int hg, cudaStream_t st) {
+  const Geo g = make_geo(s);
+  const SortGeo sg = make_sort_geo(s);
+  dsa3d_status_t rc = zero16(w.cnt, align16(w.cnt_elems * 4) / 16, st);
+  if (rc != DSA3D_OK) return rc;
+  const int64_t items = (int64_t)hg * s.N;
+  {
+    TimedLaunch tl(kKernSortCount, st);
+    dsa3d_sort_count_kernel<__nv_bfloat16, DH><<<grid_for(items, 256, 16), 256, 0, st>>>(
+        off, g, sg, h0, hg, w.cnt, w.qkey, w.qrank, static_cast<__nv_bfloat16*>(out), lse);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    TimedLaunch tl(kKernScan, st);
+    dsa3d_scan_blocks_kernel<<<(unsigned)w.nb, kScanThreads, 0, st>>>(w.cnt, w.cnt_elems, w.bsum);
+    dsa3d_scan_sums_kernel<<<1, kScanThreads, 0, st>>>(w.bsum, (int)w.nb);
+    dsa3d_scan_apply_kernel<<<(unsigned)w.nb, kScanThreads, 0, st>>>(w.cnt, w.cnt_elems, w.bsum);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    TimedLaunch tl(kKernSortFill, st);
+    dsa3d_sort_fill_kernel<<<grid_for(items, 256, 16), 256, 0, st>>>(w.cnt, w.qkey, w.qrank, g, sg, hg,
+                                                                     w.sorted_n, w.sorted_ex);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    auto kern = dsa3d_fwd_mma_kernel<DH>;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, 0) != cudaSuccess)
+      return DSA3D_ERR_CUDA;
+    if (per_sm < 1) return DSA3D_ERR_UNSUPPORTED;
+    const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
+    const int grid = grid_for(rows, 4, 1 << 20);  // one row per warp; the scheduler balances rows
+    TimedLaunch tl(kKernFwdMma, st);
+    kern<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                               static_cast<const __nv_bfloat16*>(v), off,
+                               static_cast<__nv_bfloat16*>(out), lse, w.cnt, w.sorted_n, w.sorted_ex, g,
+                               sg, h0, hg);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  return DSA3D_OK;
+}
+
 struct BwdArgs {
-  const void *q, *k, *v, *out, *dout;
+  const void *q, *k, *v, *dout;
   const float *off, *lse;
   void *dq, *dk, *dv;
   float* doff;
@@ -172,7 +279,7 @@ dsa3d_status_t bwd_launch(const Shape& s, const BwdArgs& a, cudaStream_t st) {
   TimedLaunch tl(kKernBwd, st);
   kern<<<grid, W * 32, smem, st>>>(
       static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.off,
-      static_cast<const T*>(a.out), a.lse, static_cast<const T*>(a.dout), static_cast<T*>(a.dq),
+      a.lse, static_cast<const T*>(a.dout), static_cast<T*>(a.dq),
       a.doff, a.acc_k, a.acc_v, a.acc_heads, a.h0, g, items);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
@@ -280,8 +387,9 @@ const char* dsa3d_status_string(dsa3d_status_t status) {
 }
 
 dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const float* offsets,
-                             void* out, float* lse, int F, int Hp, int Wp, int heads, int dh,
-                             int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream) {
+                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             int F, int Hp, int Wp, int heads, int dh, int kt, int kh, int kw,
+                             dsa3d_dtype_t dtype, cudaStream_t stream) {
   const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
   dsa3d_status_t rc = check_shape(s, dtype, 0);
   if (rc != DSA3D_OK) return rc;
@@ -299,6 +407,27 @@ dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const 
     if (overlap(r, ro) || (lse && overlap(r, rl))) return DSA3D_ERR_INVALID_ARGUMENT;
   if (lse && overlap(ro, rl)) return DSA3D_ERR_INVALID_ARGUMENT;
 
+  if (workspace && workspace_bytes > 0 && mma_forward_ok(s, dtype)) {
+    const size_t one = sort_ws_bytes(s, 1);
+    if (workspace_bytes < one) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace)) return DSA3D_ERR_INVALID_ARGUMENT;
+    const Range rw = range_of(workspace, workspace_bytes);
+    for (const Range& r : in)
+      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+    if (overlap(ro, rw) || (lse && overlap(rl, rw))) return DSA3D_ERR_INVALID_ARGUMENT;
+    int hg = heads;
+    while (hg > 1 && sort_ws_bytes(s, hg) > workspace_bytes) hg = (hg + 1) / 2;
+    for (int h0 = 0; h0 < heads; h0 += hg) {
+      const int n = (heads - h0 < hg) ? heads - h0 : hg;
+      const SortWs wn = carve_sort_ws(s, n, workspace);
+      const dsa3d_status_t r = (dh == 128)
+                                   ? fwd_mma_group<128>(s, q, k, v, offsets, out, lse, wn, h0, n, stream)
+                                   : fwd_mma_group<64>(s, q, k, v, offsets, out, lse, wn, h0, n, stream);
+      if (r != DSA3D_OK) return r;
+    }
+    return DSA3D_OK;
+  }
+
   const Geo g = make_geo(s);
   const DeviceInfo d = device_info();
   const int warps = pick_warps(g, false, d.max_smem);
@@ -306,6 +435,13 @@ dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const 
   if (dtype == DSA3D_F32)
     return fwd_dispatch<float>(s, warps, q, k, v, offsets, out, lse, stream);
   return fwd_dispatch<__nv_bfloat16>(s, warps, q, k, v, offsets, out, lse, stream);
+}
+
+size_t dsa3d_forward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,
+                                     int kw, dsa3d_dtype_t dtype) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  if (check_shape(s, dtype, 0) != DSA3D_OK || !mma_forward_ok(s, dtype)) return 0;
+  return sort_ws_bytes(s, heads);
 }
 
 size_t dsa3d_backward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,
@@ -317,24 +453,23 @@ size_t dsa3d_backward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, 
 }
 
 dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const float* offsets,
-                              const void* out, const float* lse, const void* dout, void* dq,
+                              const float* lse, const void* dout, void* dq,
                               void* dk, void* dv, float* doffsets, void* workspace,
                               size_t workspace_bytes, int F, int Hp, int Wp, int heads, int dh,
                               int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream) {
   const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
   dsa3d_status_t rc = check_shape(s, dtype, 0);
   if (rc != DSA3D_OK) return rc;
-  if (!q || !k || !v || !offsets || !out || !lse || !dout || !dq || !dk || !dv || !doffsets)
+  if (!q || !k || !v || !offsets || !lse || !dout || !dq || !dk || !dv || !doffsets)
     return DSA3D_ERR_INVALID_ARGUMENT;
-  const void* al[] = {q, k, v, offsets, out, dout, dq, dk, dv, doffsets};
+  const void* al[] = {q, k, v, offsets, dout, dq, dk, dv, doffsets};
   for (const void* p : al)
     if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return DSA3D_ERR_INVALID_ARGUMENT;
   const size_t tb = (size_t)s.N * heads * dh * elem_size(dtype);
   const size_t ob = (size_t)heads * s.N * 12;
   const Range ins[] = {range_of(q, tb), range_of(k, tb), range_of(v, tb), range_of(offsets, ob),
-                       range_of(out, tb), range_of(lse, (size_t)heads * s.N * 4),
-                       range_of(dout, tb)};
+                       range_of(lse, (size_t)heads * s.N * 4), range_of(dout, tb)};
   const Range outs[] = {range_of(dq, tb), range_of(dk, tb), range_of(dv, tb),
                         range_of(doffsets, ob)};
   for (int i = 0; i < 4; i++) {
@@ -361,7 +496,7 @@ dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const
   if (warps == 0) return DSA3D_ERR_UNSUPPORTED;
 
   BwdArgs a;
-  a.q = q; a.k = k; a.v = v; a.out = out; a.dout = dout; a.off = offsets; a.lse = lse;
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.off = offsets; a.lse = lse;
   a.dq = dq; a.dk = dk; a.dv = dv; a.doff = doffsets;
 
   if (dtype == DSA3D_F32) {
@@ -394,7 +529,7 @@ dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const
 }
 
 dsa3d_status_t dsa3d_backward_noalloc(const void* q, const void* k, const void* v,
-                                      const float* offsets, const void* out, const float* lse,
+                                      const float* offsets, const float* lse,
                                       const void* dout, void* dq, void* dk, void* dv,
                                       float* doffsets, int F, int Hp, int Wp, int heads, int dh,
                                       int kt, int kh, int kw, dsa3d_dtype_t dtype,
@@ -408,7 +543,7 @@ dsa3d_status_t dsa3d_backward_noalloc(const void* q, const void* k, const void* 
   void* scratch = nullptr;
   const dsa3d_status_t sc = noalloc_scratch(&scratch);
   if (sc != DSA3D_OK) return sc;
-  return dsa3d_backward(q, k, v, offsets, out, lse, dout, dq, dk, dv, doffsets, scratch,
+  return dsa3d_backward(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, scratch,
                         DSA3D_NOALLOC_SCRATCH_BYTES, F, Hp, Wp, heads, dh, kt, kh, kw, dtype,
                         stream);
 }

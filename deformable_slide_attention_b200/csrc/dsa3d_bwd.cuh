@@ -3,7 +3,8 @@
 // The paper trains through the operator (full-parameter adaptation, MegaSlide-DiT arXiv
 // 2607.22696) but gives no backward; this is the exact derivative of the forward with the tap
 // mask and the integer offset parts held fixed.  Per (head, query), with P = exp(s - lse),
-// D = dO . out, dP_tau = dO . v~_tau and dS_tau = P_tau (dP_tau - D):
+// dP_tau = dO . v~_tau, D = sum_tau P_tau dP_tau (= dO . out for the exact out, so the stored,
+// rounded out is not needed) and dS_tau = P_tau (dP_tau - D):
 //   dq        = scale * sum_tau dS_tau k~_tau        = scale * sum_j gamma[j] K[j]
 //   dK[j]    += scale * gamma[j] * q,   gamma[j] = sum_c w_c dS[j - c]
 //   dV[j]    += beta[j] * dO,           beta[j]  = sum_c w_c P[j - c]
@@ -31,8 +32,8 @@ __device__ __forceinline__ void red_add16(float* p, const float* x) {
 template <typename T, int DH, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32)
     dsa3d_bwd_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                     const float* __restrict__ off, const T* __restrict__ out,
-                     const float* __restrict__ lse, const T* __restrict__ dout, T* __restrict__ dq,
+                     const float* __restrict__ off, const float* __restrict__ lse,
+                     const T* __restrict__ dout, T* __restrict__ dq,
                      float* __restrict__ doff, float* __restrict__ acc_k, float* __restrict__ acc_v,
                      const int acc_heads, const int h0, const Geo g, const int64_t n_items) {
   constexpr int E = Elems<T>::kPerLoad;
@@ -83,17 +84,6 @@ __global__ void __launch_bounds__(WARPS * 32)
     float qv[E], gv[E];
     load16(q + row, qv);
     load16(dout + row, gv);
-    float D;
-    {
-      float ov[E];
-      load16(out + row, ov);
-      float d = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; e++) d = fmaf(gv[e], ov[e], d);
-#pragma unroll
-      for (int w = 1; w < L; w <<= 1) d += __shfl_xor_sync(kFull, d, w);
-      D = d;
-    }
 
     const int count = compact_box(g, Q, relB, tok, bidx, sraw, praw, lane);
     __syncwarp();
@@ -129,51 +119,58 @@ __global__ void __launch_bounds__(WARPS * 32)
     }
     __syncwarp();
 
-    // taps: P, dS, and the offset gradient
+    // taps: P, dP and the sums that give D and the offset gradient.  With ds_a, dp_a the
+    // derivatives of the tap's score (log2 units) and dP along f_a:
+    //   doff_a = sum P (dP - D) ds_a ln2 + P dp_a = ln2 (A_a - D B_a) + C_a,
+    //   A_a = sum P dP ds_a,  B_a = sum P ds_a,  C_a = sum P dp_a,  D = sum P dP.
     float w8[8], dw[3][8];
     corner_weights(Q.f, w8);
     corner_dweights(Q.f, dw);
     const float lse2 = lse_n * kLog2e;
-    float go0 = 0.f, go1 = 0.f, go2 = 0.f;
+    float Dp = 0.f, A[3] = {0.f, 0.f, 0.f}, Bs[3] = {0.f, 0.f, 0.f}, C[3] = {0.f, 0.f, 0.f};
     for (int tau = lane; tau < g.K; tau += 32) {
       int u, vv, w;
       unpack3(relT[tau], u, vv, w);
-      float P = 0.f, dS = 0.f;
+      float P = 0.f, PdP = 0.f;
       if (u >= Q.lo[0] && u <= Q.hi[0] && vv >= Q.lo[1] && vv <= Q.hi[1] && w >= Q.lo[2] &&
           w <= Q.hi[2]) {
         const int e = (u * g.Bh + vv) * g.Bw + w;
-        float s = 0.f, dP = 0.f, ds0 = 0.f, ds1 = 0.f, ds2 = 0.f, dp0 = 0.f, dp1 = 0.f, dp2 = 0.f;
+        float s = 0.f, dP = 0.f, ds[3] = {0.f, 0.f, 0.f}, dp[3] = {0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 8; c++) {
           const float a = sraw[e + cs[c]], b = praw[e + cs[c]];
           s = fmaf(w8[c], a, s);
           dP = fmaf(w8[c], b, dP);
-          ds0 = fmaf(dw[0][c], a, ds0);
-          ds1 = fmaf(dw[1][c], a, ds1);
-          ds2 = fmaf(dw[2][c], a, ds2);
-          dp0 = fmaf(dw[0][c], b, dp0);
-          dp1 = fmaf(dw[1][c], b, dp1);
-          dp2 = fmaf(dw[2][c], b, dp2);
+#pragma unroll
+          for (int ax = 0; ax < 3; ax++) {
+            ds[ax] = fmaf(dw[ax][c], a, ds[ax]);
+            dp[ax] = fmaf(dw[ax][c], b, dp[ax]);
+          }
         }
         P = exp2f(s - lse2);
-        dS = P * (dP - D);
-        // sraw is in log2 units: scale * q.K = sraw * ln2
-        const float dsl = dS * kLn2;
-        go0 += fmaf(dsl, ds0, P * dp0);
-        go1 += fmaf(dsl, ds1, P * dp1);
-        go2 += fmaf(dsl, ds2, P * dp2);
+        PdP = P * dP;
+        Dp += PdP;
+#pragma unroll
+        for (int ax = 0; ax < 3; ax++) {
+          A[ax] = fmaf(PdP, ds[ax], A[ax]);
+          Bs[ax] = fmaf(P, ds[ax], Bs[ax]);
+          C[ax] = fmaf(P, dp[ax], C[ax]);
+        }
       }
       ptap[tau] = P;
-      dstap[tau] = dS;
+      dstap[tau] = PdP;
     }
-    go0 = warp_sum(go0);
-    go1 = warp_sum(go1);
-    go2 = warp_sum(go2);
+    const float D = warp_sum(Dp);
+#pragma unroll
+    for (int ax = 0; ax < 3; ax++) {
+      A[ax] = warp_sum(A[ax]);
+      Bs[ax] = warp_sum(Bs[ax]);
+      C[ax] = warp_sum(C[ax]);
+    }
     if (lane == 0) {
       float* od = doff + ((int64_t)h * g.N + n) * 3;
-      od[0] = go0;
-      od[1] = go1;
-      od[2] = go2;
+#pragma unroll
+      for (int ax = 0; ax < 3; ax++) od[ax] = fmaf(kLn2, fmaf(-D, Bs[ax], A[ax]), C[ax]);
     }
     __syncwarp();
 
@@ -181,17 +178,17 @@ __global__ void __launch_bounds__(WARPS * 32)
     for (int c = lane; c < count; c += 32) {
       int jt, jy, jx;
       unpack3(relB[bidx[c]], jt, jy, jx);
-      float ga = 0.f, be = 0.f;
+      float gp = 0.f, be = 0.f;  // splats of P dP and of P; gamma = splat(P (dP - D))
 #pragma unroll
       for (int cc = 0; cc < 8; cc++) {
         const int u = jt - ((cc >> 2) & 1), vv = jy - ((cc >> 1) & 1), w = jx - (cc & 1);
         if (u >= 0 && u < g.kt && vv >= 0 && vv < g.kh && w >= 0 && w < g.kw) {
           const int t = (u * g.kh + vv) * g.kw + w;
-          ga = fmaf(w8[cc], dstap[t], ga);
+          gp = fmaf(w8[cc], dstap[t], gp);
           be = fmaf(w8[cc], ptap[t], be);
         }
       }
-      gam[c] = ga;
+      gam[c] = fmaf(-D, be, gp);
       bet[c] = be;
     }
     __syncwarp();

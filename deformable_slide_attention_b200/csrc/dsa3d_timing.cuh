@@ -11,10 +11,22 @@
 
 namespace dsa3d {
 
-enum KernelId { kKernFwd = 0, kKernBwd, kKernBwdFinalize, kKernZero, kKernCount };
+enum KernelId {
+  kKernFwd = 0,
+  kKernBwd,
+  kKernBwdFinalize,
+  kKernZero,
+  kKernFwdMma,
+  kKernSortCount,
+  kKernScan,
+  kKernSortFill,
+  kKernCount
+};
 inline const char* kernel_name(int id) {
-  static const char* names[kKernCount] = {"dsa3d_fwd_kernel", "dsa3d_bwd_kernel",
-                                          "dsa3d_bwd_finalize_kernel", "dsa3d_zero_kernel"};
+  static const char* names[kKernCount] = {
+      "dsa3d_fwd_kernel",      "dsa3d_bwd_kernel",        "dsa3d_bwd_finalize_kernel",
+      "dsa3d_zero_kernel",     "dsa3d_fwd_mma_kernel",    "dsa3d_sort_count_kernel",
+      "dsa3d_scan_kernels",    "dsa3d_sort_fill_kernel"};
   return names[id];
 }
 
@@ -94,8 +106,8 @@ class Timing {
   std::mutex mu_;
   std::vector<Pending> pending_;
   std::vector<cudaEvent_t> free_;
-  long long launches_[kKernCount] = {0, 0, 0, 0};
-  double total_ms_[kKernCount] = {0, 0, 0, 0};
+  long long launches_[kKernCount] = {};
+  double total_ms_[kKernCount] = {};
 };
 
 // RAII bracket around one launch.

@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define DSA3D_ABI_VERSION 1
+#define DSA3D_ABI_VERSION 2
 
 typedef enum {
     DSA3D_OK = 0,
@@ -67,12 +67,26 @@ const char *dsa3d_status_string(dsa3d_status_t status);
  * Forward: out (and lse, if non-NULL) for every (token, head).
  *   q, k, v  [N][heads][dh] I/O type;  offsets [heads][N][3] fp32;
  *   out      [N][heads][dh] I/O type (written);  lse [heads][N] fp32 (written; may be NULL).
+ *   workspace: device scratch of workspace_bytes bytes (contents on entry ignored), or NULL.
  *   F, Hp, Wp: frames and token grid (T, H', W');  kt, kh, kw: window (odd).
- * The backward needs lse; pass NULL only for inference.
+ * With bf16 I/O, dh in {64, 128}, kw <= 15 and a workspace of at least
+ * dsa3d_forward_workspace_bytes(..., heads = 1, ...) bytes, the forward sorts each head's
+ * queries by window origin and runs the tensor-core kernel (heads in groups that fit the
+ * workspace).  Otherwise (no workspace, fp32, other shapes) it runs the general CUDA-core kernel;
+ * both compute the same function.  A non-NULL workspace smaller than one head's need is
+ * DSA3D_ERR_WORKSPACE_TOO_SMALL.  The backward needs lse; pass NULL only for inference.
  */
 dsa3d_status_t dsa3d_forward(const void *q, const void *k, const void *v, const float *offsets,
-                             void *out, float *lse, int F, int Hp, int Wp, int heads, int dh,
-                             int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
+                             void *out, float *lse, void *workspace, size_t workspace_bytes,
+                             int F, int Hp, int Wp, int heads, int dh, int kt, int kh, int kw,
+                             dsa3d_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * Bytes of forward workspace for all heads in one pass (0 if the shape has no tensor-core path,
+ * or is invalid).  Per head: 4 * ((F+kt)(Hp+kh)(Wp+kw) + 1 + 4N) bytes, plus scan scratch.
+ */
+size_t dsa3d_forward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,
+                                     int kw, dsa3d_dtype_t dtype);
 
 /*
  * Bytes of workspace dsa3d_backward needs to process all heads in one pass.  Any workspace of at
@@ -85,15 +99,17 @@ size_t dsa3d_backward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, 
 
 /*
  * Backward: gradients of sum(out * dout) with respect to q, k, v and the offsets.
- *   q, k, v, offsets: the forward's inputs;  out, lse: the forward's outputs (lse required);
+ *   q, k, v, offsets: the forward's inputs;  lse: the forward's lse output (required);
  *   dout [N][heads][dh] I/O type;
  *   dq, dk, dv [N][heads][dh] I/O type (written);  doffsets [heads][N][3] fp32 (written);
  *   workspace: device scratch of workspace_bytes bytes (contents on entry are ignored).
  * The offset gradient is the derivative of the trilinear weights within the cell [i, i+1]; the
- * mask and the integer part of the offset are held fixed.
+ * mask and the integer part of the offset are held fixed.  The softmax Jacobian's row term
+ * D = sum_tau P_tau dP_tau is recomputed (it equals dout . out for the unrounded out), so the
+ * forward's out is not an input.
  */
 dsa3d_status_t dsa3d_backward(const void *q, const void *k, const void *v, const float *offsets,
-                              const void *out, const float *lse, const void *dout, void *dq,
+                              const float *lse, const void *dout, void *dq,
                               void *dk, void *dv, float *doffsets, void *workspace,
                               size_t workspace_bytes, int F, int Hp, int Wp, int heads, int dh,
                               int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
@@ -119,7 +135,7 @@ dsa3d_status_t dsa3d_backward(const void *q, const void *k, const void *v, const
 #define DSA3D_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 
 dsa3d_status_t dsa3d_backward_noalloc(const void *q, const void *k, const void *v,
-                                      const float *offsets, const void *out, const float *lse,
+                                      const float *offsets, const float *lse,
                                       const void *dout, void *dq, void *dk, void *dv,
                                       float *doffsets, int F, int Hp, int Wp, int heads, int dh,
                                       int kt, int kh, int kw, dsa3d_dtype_t dtype,

@@ -36,8 +36,8 @@
  *   R6  Values are sampled at the same positions as keys.  No causal mask.
  *   R7  Backward: exact derivative of the above with the validity pattern and the integer
  *       part held fixed; d/d(delta) is the derivative of the trilinear weights inside the cell
- *       [i, i+1] (the +f side at exact integers).  D = dO . out uses out rounded to the I/O
- *       type, as a caller's backward receives it.
+ *       [i, i+1] (the +f side at exact integers).  The softmax Jacobian's D = sum_tau P dP
+ *       equals dO . out for the exact out (no rounding to the I/O type).
  *
  * Layouts: q, k, v, dout: [N][heads][dh] (token n = (t*Hp + y)*Wp + x), in fp32 or bf16 bits.
  * offsets: [heads][N][3] fp32, order (dt, dy, dx).  A query or key "item" is h*N + n.
@@ -71,21 +71,6 @@ static double rd(const void *base, int io, int64_t idx) {
     float x;
     memcpy(&x, &u, 4);
     return (double)x;
-}
-
-/* Round to the I/O type, round-to-nearest-even (double -> fp32 -> bf16). */
-static double round_io(double x, int io) {
-    float f = (float)x;
-    if (io == IO_F32) return (double)f;
-    uint32_t u;
-    memcpy(&u, &f, 4);
-    if ((u & 0x7f800000u) != 0x7f800000u) {
-        uint32_t lsb = (u >> 16) & 1u;
-        u += 0x7fffu + lsb;
-    }
-    u &= 0xffff0000u;
-    memcpy(&f, &u, 4);
-    return (double)f;
 }
 
 static decode_t decode(const prob_t *P, int h, int64_t n) {
@@ -336,7 +321,7 @@ static int query_backward(const prob_t *P, int h, int64_t n, scratch_t *S, doubl
         S->dO[e] = rd(P->dout, P->io, row + e);
     }
     double D = 0.0;
-    for (int e = 0; e < dh; e++) D += S->dO[e] * round_io(S->out[e], P->io);
+    for (int e = 0; e < dh; e++) D += S->dO[e] * S->out[e];
     for (int tau = 0; tau < K; tau++) {
         if (S->s[tau] == -INFINITY) continue;
         tap_base(P, p, &d, tau, b);

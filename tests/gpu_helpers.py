@@ -21,8 +21,8 @@ def gpu_forward(d, dims, window):
     return out, lse
 
 
-def gpu_backward(d, out, lse, dims, window):
-    grads = abi.backward(d["q"], d["k"], d["v"], d["offsets"], out, lse, d["dout"], dims, window)
+def gpu_backward(d, lse, dims, window):
+    grads = abi.backward(d["q"], d["k"], d["v"], d["offsets"], lse, d["dout"], dims, window)
     torch.cuda.synchronize()
     return grads
 
@@ -60,16 +60,28 @@ def assert_close(name, got, ref, tol):
     return err
 
 
+def has_mma_path(d, dims, window):
+    heads, dh = d["q"].shape[1], d["q"].shape[2]
+    code = abi.DSA3D_BF16 if d["q"].dtype == torch.bfloat16 else abi.DSA3D_F32
+    return abi.dsa3d_forward_workspace_bytes(*dims, heads, dh, *window, code) > 0
+
+
 def full_parity(inp, dims, window, dtype, backward=True):
-    """Element-by-element comparison of every output with the oracle."""
+    """Element-by-element comparison of every output with the oracle.  Where the shape has a
+    tensor-core forward, the general CUDA-core forward (no workspace) is checked as well."""
     tol = TOL[dtype]
     d = to_cuda(inp)
     out, lse = gpu_forward(d, dims, window)
     r_out, r_lse = oracle.full_forward(inp["q"], inp["k"], inp["v"], inp["offsets"], dims, window)
     errs = {"out": assert_close("out", f64(out), r_out, tol),
             "lse": assert_close("lse", f64(lse), r_lse, max(tol, 1e-5))}
+    if has_mma_path(d, dims, window):
+        out_cc, lse_cc = abi.forward(d["q"], d["k"], d["v"], d["offsets"], dims, window, workspace=None)
+        torch.cuda.synchronize()
+        errs["out_cc"] = assert_close("out (CUDA-core)", f64(out_cc), r_out, tol)
+        errs["lse_cc"] = assert_close("lse (CUDA-core)", f64(lse_cc), r_lse, max(tol, 1e-5))
     if backward:
-        dq, dk, dv, doff = gpu_backward(d, out, lse, dims, window)
+        dq, dk, dv, doff = gpu_backward(d, lse, dims, window)
         r = oracle.full_backward(inp["q"], inp["k"], inp["v"], inp["offsets"], inp["dout"], dims,
                                  window)
         for name, got, ref in (("dq", dq, r[0]), ("doff", doff, r[1]), ("dk", dk, r[2]),

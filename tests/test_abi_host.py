@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings():
-    assert abi.dsa3d_abi_version() == 1
+    assert abi.dsa3d_abi_version() == 2
     for s in range(6):
         assert abi.dsa3d_status_string(s)
     assert abi.dsa3d_status_string(0) == "ok"
@@ -49,8 +49,9 @@ P = 1 << 20  # a fake 16-byte-aligned address; validation fails before any devic
 def fwd(**kw):
     a = {**ARGS, **kw}
     ptrs = [kw.get(n, P * (i + 1)) for i, n in enumerate(["q", "k", "v", "off", "out", "lse"])]
-    return abi.dsa3d_forward(*ptrs, a["F"], a["Hp"], a["Wp"], a["heads"], a["dh"], a["kt"], a["kh"],
-                             a["kw"], kw.get("dtype", abi.DSA3D_BF16), 0)
+    return abi.dsa3d_forward(*ptrs, kw.get("ws", 0), kw.get("wsb", 0), a["F"], a["Hp"], a["Wp"],
+                             a["heads"], a["dh"], a["kt"], a["kh"], a["kw"],
+                             kw.get("dtype", abi.DSA3D_BF16), 0)
 
 
 def test_forward_rejects_bad_arguments():
@@ -66,6 +67,22 @@ def test_forward_rejects_bad_arguments():
     assert fwd(kh=17) == UNS      # larger than 2*Hp-1
     # out overlapping q
     assert fwd(q=P, out=P + 4096) == INV
+    # a workspace smaller than one head's sort, and one overlapping an input
+    assert fwd(ws=P * 64, wsb=1024) == 3
+    need = abi.dsa3d_forward_workspace_bytes(4, 8, 8, 1, 64, 3, 3, 3, abi.DSA3D_BF16)
+    assert fwd(ws=P, wsb=need) == INV
+
+
+def test_forward_workspace_bytes():
+    # per head: 4 * ((F+kt)(Hp+kh)(Wp+kw) + 1) bytes of buckets + 4 * 4N bytes, 16-byte aligned
+    one = abi.dsa3d_forward_workspace_bytes(4, 8, 8, 1, 64, 3, 3, 3, abi.DSA3D_BF16)
+    buckets = (4 + 3) * (8 + 3) * (8 + 3) + 1
+    assert one >= 4 * buckets + 4 * 4 * 256
+    assert abi.dsa3d_forward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_BF16) > one
+    # no tensor-core path: fp32, dh 32, kw > 15
+    assert abi.dsa3d_forward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_F32) == 0
+    assert abi.dsa3d_forward_workspace_bytes(4, 8, 8, 2, 32, 3, 3, 3, abi.DSA3D_BF16) == 0
+    assert abi.dsa3d_forward_workspace_bytes(4, 8, 16, 2, 64, 3, 3, 17, abi.DSA3D_BF16) == 0
 
 
 def test_backward_workspace_bytes():
@@ -76,7 +93,7 @@ def test_backward_workspace_bytes():
 
 
 def test_backward_rejects_bad_arguments():
-    ptr = [P * (i + 1) for i in range(12)]
+    ptr = [P * (i + 1) for i in range(11)]
     a = ARGS
     call = lambda ptrs, wsb=0, dtype=abi.DSA3D_BF16, **kw: abi.dsa3d_backward(
         *ptrs, wsb, kw.get("F", a["F"]), a["Hp"], a["Wp"], a["heads"], a["dh"], a["kt"], a["kh"],
@@ -88,5 +105,5 @@ def test_backward_rejects_bad_arguments():
     assert call(ptr, wsb=1000) == 3
     # dk aliasing q
     alias = list(ptr)
-    alias[8] = ptr[0]
+    alias[7] = ptr[0]
     assert call(alias, wsb=1 << 30) == 1

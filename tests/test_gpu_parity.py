@@ -5,6 +5,7 @@ compare every output element; the 720p workloads compare a seeded sample of quer
 dq, doffsets) and of keys (dk, dv), which the oracle computes one by one.
 """
 import dataclasses
+import math
 
 import numpy as np
 import pytest
@@ -84,6 +85,44 @@ def test_invalid_offsets_and_carry():
     full_parity(inp, dims, window, "f32")
 
 
+@pytest.mark.parametrize("window", [(3, 3, 15), (1, 1, 13), (5, 3, 11)])
+def test_widest_tensor_core_windows(window):
+    dims = (6, 9, 37)
+    _, inp = inputs.custom(*dims, 2, 128, window, "bf16", seed=300 + window[2], scale=3.0)
+    full_parity(inp, dims, window, "bf16")
+
+
+def test_tensor_core_path_sparse_and_invalid_queries():
+    # large offsets: many queries leave the volume, bucket rows are sparse and ragged
+    dims, window = (4, 7, 9), (3, 3, 3)
+    _, inp = inputs.custom(*dims, 3, 64, window, "bf16", seed=13, offsets="normal", scale=5.0)
+    inp["offsets"][0, 5, 1] = float("nan")
+    inp["offsets"][2, 9, 2] = 2.0 ** 30
+    full_parity(inp, dims, window, "bf16")
+
+
+def test_tensor_core_path_dense_buckets():
+    # all queries of a head share one origin (many queries per bucket, long chunks of equal x)
+    dims, window = (3, 6, 20), (3, 5, 7)
+    _, inp = inputs.custom(*dims, 2, 128, window, "bf16", seed=14)
+    t, y, x = [torch.arange(math.prod(dims)) // (6 * 20), (torch.arange(math.prod(dims)) // 20) % 6,
+               torch.arange(math.prod(dims)) % 20]
+    inp["offsets"][0] = torch.stack([1.25 - t, 2.5 - y, 7.75 - x], -1).float()
+    full_parity(inp, dims, window, "bf16")
+
+
+def test_forward_workspace_head_groups():
+    dims, window = (4, 6, 7), (3, 3, 5)
+    _, inp = inputs.custom(*dims, 5, 64, window, "bf16", seed=15, with_dout=False)
+    d = to_cuda(inp)
+    full, _ = abi.forward(d["q"], d["k"], d["v"], d["offsets"], dims, window)
+    one = abi.dsa3d_forward_workspace_bytes(*dims, 1, 64, *window, abi.DSA3D_BF16)
+    ws = torch.empty(one + 100, dtype=torch.uint8, device="cuda")
+    part, _ = abi.forward(d["q"], d["k"], d["v"], d["offsets"], dims, window, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(full, part)
+
+
 def test_small_bf16_workload_forward_full():
     w = inputs.BY_NAME["small-bf16"]
     inp = inputs.make(w, "cpu", with_dout=False)
@@ -104,7 +143,7 @@ def _sampled(w, n_q, n_k, seed, backward):
     assert_close("lse", f64(lse).reshape(-1)[qi], r_lse, tol)
     if not backward:
         return
-    dq, dk, dv, doff = gpu_backward(d, out, lse, w.dims, w.window)
+    dq, dk, dv, doff = gpu_backward(d, lse, w.dims, w.window)
     ki = items_of(w.heads, N, n_k, seed + 1)
     r_dq, r_doff, r_dk, r_dv = oracle.backward(inp["q"], inp["k"], inp["v"], inp["offsets"],
                                                inp["dout"], w.dims, w.window, qi, ki)
@@ -142,10 +181,10 @@ def test_workspace_smaller_than_all_heads():
     _, inp = inputs.custom(*dims, 4, 64, window, "bf16", seed=12)
     d = to_cuda(inp)
     out, lse = gpu_forward(d, dims, window)
-    full = gpu_backward(d, out, lse, dims, window)
+    full = gpu_backward(d, lse, dims, window)
     one = abi.dsa3d_backward_workspace_bytes(*dims, 1, 64, *window, abi.DSA3D_BF16)
     ws = torch.empty(one, dtype=torch.uint8, device="cuda")
-    part = abi.backward(d["q"], d["k"], d["v"], d["offsets"], out, lse, d["dout"], dims, window,
+    part = abi.backward(d["q"], d["k"], d["v"], d["offsets"], lse, d["dout"], dims, window,
                         workspace=ws)
     torch.cuda.synchronize()
     for a, b in zip(full, part):

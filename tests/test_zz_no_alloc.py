@@ -16,14 +16,14 @@ from tests.gpu_helpers import TOL, to_cuda
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gpu_lib")]
 
 
-def _noalloc(d, out, lse, dims, window, dtype_code):
+def _noalloc(d, lse, dims, window, dtype_code):
     N = dims[0] * dims[1] * dims[2]
     heads, dh = d["q"].shape[1], d["q"].shape[2]
     grads = (torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"]),
              torch.empty_like(d["offsets"]))
     st = abi.dsa3d_backward_noalloc(
         d["q"].data_ptr(), d["k"].data_ptr(), d["v"].data_ptr(), d["offsets"].data_ptr(),
-        out.data_ptr(), lse.data_ptr(), d["dout"].data_ptr(), *(g.data_ptr() for g in grads),
+        lse.data_ptr(), d["dout"].data_ptr(), *(g.data_ptr() for g in grads),
         *dims, heads, dh, *window, dtype_code, torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert st == 0, abi.dsa3d_status_string(st)
@@ -39,10 +39,10 @@ def test_noalloc_matches_workspace_backward_twice(dims, heads, dh, window):
     _, inp = inputs.custom(*dims, heads, dh, window, "bf16", seed=41, scale=2.0)
     d = to_cuda(inp)
     out, lse = abi.forward(d["q"], d["k"], d["v"], d["offsets"], dims, window)
-    ref = abi.backward(d["q"], d["k"], d["v"], d["offsets"], out, lse, d["dout"], dims, window)
+    ref = abi.backward(d["q"], d["k"], d["v"], d["offsets"], lse, d["dout"], dims, window)
     torch.cuda.synchronize()
     for _ in range(2):
-        got = _noalloc(d, out, lse, dims, window, abi.DSA3D_BF16)
+        got = _noalloc(d, lse, dims, window, abi.DSA3D_BF16)
         for name, a, b in zip(("dq", "dk", "dv", "doffsets"), got, ref):
             err = (a.float() - b.float()).abs().max().item()
             assert err <= TOL["bf16"], f"{name}: {err:.3e}"
@@ -55,6 +55,6 @@ def test_noalloc_refuses_problem_larger_than_its_scratch():
     t = torch.zeros(16, dtype=torch.uint8, device="cuda")  # never dereferenced: refused on the host
     p = t.data_ptr()
     st = abi.dsa3d_backward_noalloc(p, p + 1024, p + 2048, p + 3072, p + 4096, p + 5120, p + 6144,
-                                    p + 7168, p + 8192, p + 9216, p + 10240, *dims, heads, dh,
+                                    p + 7168, p + 8192, p + 9216, *dims, heads, dh,
                                     *window, abi.DSA3D_BF16, torch.cuda.current_stream().cuda_stream)
     assert st == 3  # DSA3D_ERR_WORKSPACE_TOO_SMALL
