@@ -10,6 +10,7 @@
 
 #include "dsa3d.h"
 #include "dsa3d_bwd.cuh"
+#include "dsa3d_bwd_mma.cuh"
 #include "dsa3d_fwd.cuh"
 #include "dsa3d_fwd_mma.cuh"
 #include "dsa3d_sort.cuh"
@@ -224,7 +225,7 @@ dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const
   {
     TimedLaunch tl(kKernSortCount, st);
     dsa3d_sort_count_kernel<__nv_bfloat16, DH><<<grid_for(items, 256, 16), 256, 0, st>>>(
-        off, g, sg, h0, hg, w.cnt, w.qkey, w.qrank, static_cast<__nv_bfloat16*>(out), lse);
+        off, g, sg, h0, hg, w.cnt, w.qkey, w.qrank, static_cast<__nv_bfloat16*>(out), lse, nullptr);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
   {
@@ -266,6 +267,87 @@ struct BwdArgs {
   float *acc_k, *acc_v;
   int acc_heads, h0, hc;
 };
+
+// --- sorted tensor-core backward -------------------------------------------------------------
+BoxGeo make_box_geo(const Shape& s) {
+  BoxGeo bg;
+  bg.rows = s.kt * (s.kh + 1);
+  bg.width = s.kw + 1;
+  bg.per_q = bg.rows * bg.width;
+  return bg;
+}
+// Workspace for hg heads: the sort's | gamma' boxes | beta boxes | (D, f_t) per sorted query.
+size_t mma_bwd_ws_bytes(const Shape& s, int hg) {
+  const BoxGeo bg = make_box_geo(s);
+  const size_t boxes = align16((size_t)hg * s.N * bg.per_q * 2);
+  return sort_ws_bytes(s, hg) + 2 * boxes + align16((size_t)hg * s.N * 8);
+}
+
+template <int DH>
+dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const void* v,
+                             const float* off, const float* lse, const void* dout, void* dq, void* dk,
+                             void* dv, float* doff, void* ws, int h0, int hg, cudaStream_t st) {
+  const Geo g = make_geo(s);
+  const SortGeo sg = make_sort_geo(s);
+  const BoxGeo bg = make_box_geo(s);
+  const SortWs w = carve_sort_ws(s, hg, ws);
+  char* p = static_cast<char*>(ws) + sort_ws_bytes(s, hg);
+  const size_t boxes = align16((size_t)hg * s.N * bg.per_q * 2);
+  unsigned short* gbox = reinterpret_cast<unsigned short*>(p);
+  unsigned short* bbox = reinterpret_cast<unsigned short*>(p + boxes);
+  float2* dft = reinterpret_cast<float2*>(p + 2 * boxes);
+  using bf = __nv_bfloat16;
+  const bf* qb = static_cast<const bf*>(q);
+  const bf* kb = static_cast<const bf*>(k);
+  const bf* vb = static_cast<const bf*>(v);
+  const bf* ob = static_cast<const bf*>(dout);
+
+  dsa3d_status_t rc = zero16(w.cnt, align16(w.cnt_elems * 4) / 16, st);
+  if (rc != DSA3D_OK) return rc;
+  const int64_t items = (int64_t)hg * s.N;
+  {
+    TimedLaunch tl(kKernSortCount, st);
+    dsa3d_sort_count_kernel<bf, DH><<<grid_for(items, 256, 16), 256, 0, st>>>(
+        off, g, sg, h0, hg, w.cnt, w.qkey, w.qrank, static_cast<bf*>(dq), nullptr, doff);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    TimedLaunch tl(kKernScan, st);
+    dsa3d_scan_blocks_kernel<<<(unsigned)w.nb, kScanThreads, 0, st>>>(w.cnt, w.cnt_elems, w.bsum);
+    dsa3d_scan_sums_kernel<<<1, kScanThreads, 0, st>>>(w.bsum, (int)w.nb);
+    dsa3d_scan_apply_kernel<<<(unsigned)w.nb, kScanThreads, 0, st>>>(w.cnt, w.cnt_elems, w.bsum);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    TimedLaunch tl(kKernSortFill, st);
+    dsa3d_sort_fill_kernel<<<grid_for(items, 256, 16), 256, 0, st>>>(w.cnt, w.qkey, w.qrank, g, sg, hg,
+                                                                     w.sorted_n, w.sorted_ex);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
+  {
+    TimedLaunch tl(kKernBwdQ, st);
+    dsa3d_bwd_q_kernel<DH><<<grid_for(rows, 4, 1 << 20), 128, 0, st>>>(
+        qb, kb, vb, ob, off, lse, doff, w.cnt, w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg,
+        h0, hg);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    TimedLaunch tl(kKernBwdDq, st);
+    dsa3d_bwd_dq_kernel<DH><<<grid_for(rows, 4, 1 << 20), 128, 0, st>>>(
+        kb, static_cast<bf*>(dq), w.cnt, w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg, h0, hg);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    const int64_t tasks = (int64_t)hg * s.F * s.Hp * ((s.Wp + 15) / 16) * 2;
+    TimedLaunch tl(kKernBwdKv, st);
+    dsa3d_bwd_kv_kernel<DH><<<grid_for(tasks, 4, 1 << 20), 128, 0, st>>>(
+        qb, ob, static_cast<bf*>(dk), static_cast<bf*>(dv), w.cnt, w.sorted_n, w.sorted_ex, gbox,
+        bbox, dft, g, sg, bg, h0, hg);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  return DSA3D_OK;
+}
 
 template <typename T, int DH, int W>
 dsa3d_status_t bwd_launch(const Shape& s, const BwdArgs& a, cudaStream_t st) {
@@ -449,6 +531,7 @@ size_t dsa3d_backward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, 
   const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
   if (check_shape(s, dtype, 0) != DSA3D_OK) return 0;
   if (dtype == DSA3D_F32) return 0;
+  if (mma_forward_ok(s, dtype)) return mma_bwd_ws_bytes(s, heads);
   return acc_bytes_per_head(s) * (size_t)heads;
 }
 
@@ -477,6 +560,25 @@ dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const
       if (overlap(r, outs[i])) return DSA3D_ERR_INVALID_ARGUMENT;
     for (int j = i + 1; j < 4; j++)
       if (overlap(outs[i], outs[j])) return DSA3D_ERR_INVALID_ARGUMENT;
+  }
+
+  if (mma_forward_ok(s, dtype) && workspace && workspace_bytes >= mma_bwd_ws_bytes(s, 1)) {
+    if (!aligned16(workspace)) return DSA3D_ERR_INVALID_ARGUMENT;
+    const Range rw = range_of(workspace, workspace_bytes);
+    for (const Range& r : ins)
+      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+    for (const Range& r : outs)
+      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+    int hg = heads;
+    while (hg > 1 && mma_bwd_ws_bytes(s, hg) > workspace_bytes) hg = (hg + 1) / 2;
+    for (int h0 = 0; h0 < heads; h0 += hg) {
+      const int n = (heads - h0 < hg) ? heads - h0 : hg;
+      const dsa3d_status_t r =
+          (dh == 128) ? bwd_mma_group<128>(s, q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace, h0, n, stream)
+                      : bwd_mma_group<64>(s, q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace, h0, n, stream);
+      if (r != DSA3D_OK) return r;
+    }
+    return DSA3D_OK;
   }
 
   const size_t per_head = acc_bytes_per_head(s);

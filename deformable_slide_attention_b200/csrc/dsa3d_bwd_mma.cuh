@@ -1,0 +1,632 @@
+// dsa3d_bwd_mma.cuh -- 3D-DSA backward on tensor cores (bf16 I/O, dh 64 or 128, k_w <= 15).
+//
+// Exact derivative of the forward (MegaSlide-DiT, arXiv 2607.22696, Eq. 1) with the tap mask and
+// the integer offset parts held fixed; D = sum_tau P_tau dP_tau (dout . out for the exact out).
+// Queries are sorted by window origin and cut into the forward's chunks (<= 16 queries of one
+// bucket row whose x-origins span <= 16, 32-key segment per box row).  Three passes, no global
+// atomics:
+//
+//  1. query side (dsa3d_bwd_q_kernel): per tap plane u and box row, Q.K and dO.V of box planes
+//     u and u+1 on tensor cores; per tap: P = exp2(s - lse2), dP, their derivatives along the
+//     three fractional coordinates; per query D = sum P dP and
+//        doff_a = scale (sum P dP ds_a - D sum P ds_a) + sum P dp_a.
+//     It stores, per query and tap plane, the y/x-transposed splats of P (beta) and of P dP
+//     (gamma') onto the box rows, in bf16: box[pos][u][by][bx], and D, f_t per query.
+//  2. dq (dsa3d_bwd_dq_kernel): dq = scale sum_j gamma[j] K[j], gamma = gamma' - D beta and the
+//     t-mix of the two tap planes feeding each box plane, as tensor-core products per box row.
+//  3. key side (dsa3d_bwd_kv_kernel): one warp owns 16 keys x 64 dims of one key row and
+//     gathers, from the bucket ranges of the queries whose boxes cover those keys, the stored
+//     gamma/beta rows: dK += scale Gamma^T Q, dV += Beta^T dO on tensor cores, written once.
+#pragma once
+
+#include "dsa3d_fwd_mma.cuh"
+
+namespace dsa3d {
+
+// Geometry of the stored per-query splats.
+struct BoxGeo {
+  int rows;      // kt * (kh + 1) box rows per query (tap plane u, box row by)
+  int width;     // kw + 1
+  int per_q;     // rows * width bf16 values per query and array
+};
+
+__device__ __forceinline__ unsigned short bf16_bits(float x) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(x);
+  return *reinterpret_cast<const unsigned short*>(&b);
+}
+__device__ __forceinline__ float bf16_val(unsigned short u) { return __uint_as_float((unsigned)u << 16); }
+
+// One 16 x 32 raw-dot block: acc[jt] (n-tile jt, keys X0 + 8jt + [0,8)) = A . src[t, y, seg]^T,
+// A = 16 rows given as k-step fragments af (dims as laid out by MmaShape).
+template <int DH>
+__device__ __forceinline__ void raw_block(float (&acc)[4][4], const unsigned (&af)[MmaShape<DH>::KS][4],
+                                          const __nv_bfloat16* src_h, int t, int y, int X0, int segw,
+                                          int64_t rs, const Geo& g, int gq, int qq) {
+  using S = MmaShape<DH>;
+#pragma unroll
+  for (int jt = 0; jt < 4; jt++) acc[jt][0] = acc[jt][1] = acc[jt][2] = acc[jt][3] = 0.f;
+  if (t < 0 || t >= g.F || y < 0 || y >= g.Hp) return;
+#pragma unroll
+  for (int jt = 0; jt < 4; jt++) {
+    const int col = 8 * jt + gq;
+    const int x = X0 + col;
+    const bool ok = col < segw && x >= 0 && x < g.Wp;
+    const __nv_bfloat16* r = src_h + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + qq * (DH / 4);
+    unsigned w[S::QW];
+#pragma unroll
+    for (int c = 0; c < S::QW / 4; c++) {
+      const uint4 a = ok ? ldg16(r + c * 8) : make_uint4(0, 0, 0, 0);
+      w[4 * c] = a.x; w[4 * c + 1] = a.y; w[4 * c + 2] = a.z; w[4 * c + 3] = a.w;
+    }
+#pragma unroll
+    for (int s = 0; s < S::KS; s++)
+      mma_bf16_16816(acc[jt], af[s][0], af[s][1], af[s][2], af[s][3], w[2 * s], w[2 * s + 1]);
+  }
+}
+
+template <int DH>
+__device__ __forceinline__ void load_afrags(unsigned (&af)[MmaShape<DH>::KS][4], const __nv_bfloat16* base,
+                                            const MmaRow (&R)[2], int h, int heads, int qq) {
+  using S = MmaShape<DH>;
+  unsigned w0[S::QW], w1[S::QW];
+#pragma unroll
+  for (int c = 0; c < S::QW / 4; c++) {
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    if (R[0].live) a = ldg16(base + ((int64_t)R[0].n * heads + h) * DH + qq * (DH / 4) + c * 8);
+    if (R[1].live) b = ldg16(base + ((int64_t)R[1].n * heads + h) * DH + qq * (DH / 4) + c * 8);
+    w0[4 * c] = a.x; w0[4 * c + 1] = a.y; w0[4 * c + 2] = a.z; w0[4 * c + 3] = a.w;
+    w1[4 * c] = b.x; w1[4 * c + 1] = b.y; w1[4 * c + 2] = b.z; w1[4 * c + 3] = b.w;
+  }
+#pragma unroll
+  for (int s = 0; s < S::KS; s++) {
+    af[s][0] = w0[2 * s];
+    af[s][1] = w1[2 * s];
+    af[s][2] = w0[2 * s + 1];
+    af[s][3] = w1[2 * s + 1];
+  }
+}
+
+// Decode the rows of a chunk starting at sorted position pos (cnt rows).
+__device__ __forceinline__ void chunk_rows(MmaRow (&R)[2], const Geo& g, const float* off, int h,
+                                           const int* sorted_n, int pos, int cnt, int X0, int gq) {
+#pragma unroll
+  for (int hf = 0; hf < 2; hf++) {
+    const int r = gq + 8 * hf;
+    R[hf].live = r < cnt;
+    R[hf].n = R[hf].live ? sorted_n[pos + r] : 0;
+    const Query Qd = decode_query(g, off, h, R[hf].n);
+    R[hf].ox = Qd.o[2] - X0;
+#pragma unroll
+    for (int a = 0; a < 3; a++) {
+      R[hf].f[a] = Qd.f[a];
+      R[hf].lo[a] = Qd.lo[a];
+      R[hf].hi[a] = R[hf].live ? Qd.hi[a] : -1;
+    }
+  }
+}
+
+// Chunk of the bucket row [pos, qend): count of rows, X0.
+__device__ __forceinline__ int chunk_len(const int* sorted_ex, int pos, int qend, int kw, int lane, int& X0) {
+  const int ex_l = (lane < 16 && pos + lane < qend) ? sorted_ex[pos + lane] : 0x7fffffff;
+  const int ex0 = __shfl_sync(kFull, ex_l, 0);
+  const unsigned bal = __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 < 16);
+  X0 = ex0 - kw;
+  return __popc(bal);
+}
+
+// Store one box row of a row-half: values v_e/v_o at columns 8jt+2q(+1) -> box x = col - ox.
+__device__ __forceinline__ void store_box_row(unsigned short* dst, const float (&ve)[4], const float (&vo)[4],
+                                              int ox, int width, int qq) {
+#pragma unroll
+  for (int jt = 0; jt < 4; jt++) {
+    const int x0 = 8 * jt + 2 * qq - ox;
+    if (x0 >= 0 && x0 < width) dst[x0] = bf16_bits(ve[jt]);
+    if (x0 + 1 >= 0 && x0 + 1 < width) dst[x0 + 1] = bf16_bits(vo[jt]);
+  }
+}
+
+// ---- pass 1: query side ---------------------------------------------------------------------
+template <int DH>
+__global__ void __launch_bounds__(128)
+    dsa3d_bwd_q_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                       const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
+                       const float* __restrict__ off, const float* __restrict__ lse,
+                       float* __restrict__ doff, const int* __restrict__ start,
+                       const int* __restrict__ sorted_n, const int* __restrict__ sorted_ex,
+                       unsigned short* __restrict__ gbox, unsigned short* __restrict__ bbox,
+                       float2* __restrict__ dft, const Geo g, const SortGeo sg, const BoxGeo bg,
+                       const int h0, const int hg) {
+  using S = MmaShape<DH>;
+  __shared__ float prev_sh[4][4 * 16 * 32];  // per warp: st, bd, dpt, dbd of the previous box row
+  __shared__ float bxp_sh[4][2 * 16 * 32];   // per warp: x-transposed P and P dP of the previous tap row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, qq = lane & 3;
+  float* prev = prev_sh[warp];
+  float* bxp = bxp_sh[warp];
+  const int64_t rs = (int64_t)g.heads * DH;
+  const float sc = g.scale * kLog2e;
+  const int segw = 16 + g.kw;
+  const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
+
+  for (int64_t row = (int64_t)blockIdx.x * 4 + warp; row < rows; row += (int64_t)gridDim.x * 4) {
+    const int hh = (int)(row / ((int64_t)sg.Et * sg.Ey));
+    const int rem = (int)(row - (int64_t)hh * sg.Et * sg.Ey);
+    const int et = rem / sg.Ey, ey = rem % sg.Ey;
+    const int h = h0 + hh;
+    const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)et * sg.Ey + ey) * sg.Ex;
+    const int qbeg = start[b0], qend = start[b0 + sg.Ex];
+    const int ot = et - g.kt, oy = ey - g.kh;
+    const __nv_bfloat16* kh_ = k + (int64_t)h * DH;
+    const __nv_bfloat16* vh_ = v + (int64_t)h * DH;
+
+    for (int pos = qbeg; pos < qend;) {
+      int X0;
+      const int cnt = chunk_len(sorted_ex, pos, qend, g.kw, lane, X0);
+      MmaRow R[2];
+      chunk_rows(R, g, off, h, sorted_n, pos, cnt, X0, gq);
+      float lse2[2];
+#pragma unroll
+      for (int hf = 0; hf < 2; hf++)
+        lse2[hf] = R[hf].live ? __ldg(lse + (int64_t)h * g.N + R[hf].n) * kLog2e : 0.f;
+      unsigned qa[S::KS][4], ga[S::KS][4];
+      load_afrags<DH>(qa, q, R, h, g.heads, qq);
+      load_afrags<DH>(ga, dout, R, h, g.heads, qq);
+
+      float Dp[2] = {0.f, 0.f};
+      float A[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+      float Bs[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+      float C[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+
+      for (int u = 0; u < g.kt; u++) {
+        for (int i = lane; i < 4 * 16 * 32; i += 32) prev[i] = 0.f;
+        for (int i = lane; i < 2 * 16 * 32; i += 32) bxp[i] = 0.f;
+        __syncwarp();
+        for (int by = 0; by <= g.kh; by++) {
+          const int y = oy + by;
+          // raw blocks of box row by on planes u (0) and u+1 (1); blend and t-difference
+          float cur[4][4][4];  // [st, bd, dpt, dbd][jt][e]
+          {
+            float s0[4][4], s1[4][4];
+            raw_block<DH>(s0, qa, kh_, ot + u, y, X0, segw, rs, g, gq, qq);
+            raw_block<DH>(s1, qa, kh_, ot + u + 1, y, X0, segw, rs, g, gq, qq);
+#pragma unroll
+            for (int jt = 0; jt < 4; jt++)
+#pragma unroll
+              for (int e = 0; e < 4; e++) {
+                const float ft = R[e >> 1].f[0];
+                cur[1][jt][e] = s1[jt][e] - s0[jt][e];
+                cur[0][jt][e] = fmaf(ft, cur[1][jt][e], s0[jt][e]);
+              }
+            raw_block<DH>(s0, ga, vh_, ot + u, y, X0, segw, rs, g, gq, qq);
+            raw_block<DH>(s1, ga, vh_, ot + u + 1, y, X0, segw, rs, g, gq, qq);
+#pragma unroll
+            for (int jt = 0; jt < 4; jt++)
+#pragma unroll
+              for (int e = 0; e < 4; e++) {
+                const float ft = R[e >> 1].f[0];
+                cur[3][jt][e] = s1[jt][e] - s0[jt][e];
+                cur[2][jt][e] = fmaf(ft, cur[3][jt][e], s0[jt][e]);
+              }
+          }
+          if (by >= 1) {
+            const int ty = by - 1;
+            float pe[2][4], po[2][4], ge[2][4], go[2][4];  // P and P dP of tap row ty
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+              const float fx = R[hf].f[1 + 1], fy = R[hf].f[1];
+              // y-lerps (value, y-derivative) of the four blocks, even/odd columns
+              float ye[4][4], yo[4][4], dye[2][4], dyo[2][4];
+#pragma unroll
+              for (int b = 0; b < 4; b++)
+#pragma unroll
+                for (int jt = 0; jt < 4; jt++) {
+                  const float pe_ = prev[(b * 16 + jt * 4 + 2 * hf) * 32 + lane];
+                  const float po_ = prev[(b * 16 + jt * 4 + 2 * hf + 1) * 32 + lane];
+                  const float ce = cur[b][jt][2 * hf], co = cur[b][jt][2 * hf + 1];
+                  ye[b][jt] = fmaf(fy, ce - pe_, pe_);
+                  yo[b][jt] = fmaf(fy, co - po_, po_);
+                  if (b == 0 || b == 2) {
+                    dye[b >> 1][jt] = ce - pe_;
+                    dyo[b >> 1][jt] = co - po_;
+                  }
+                }
+              // x-neighbours of the y-lerped blends and of the y-derivatives
+              float ns_e[4], ns_o[4], np_e[4], np_o[4], nds_e[4], nds_o[4], ndp_e[4], ndp_o[4];
+              float nbs_e[4], nbs_o[4], nbp_e[4], nbp_o[4];
+              col_next(ye[0], yo[0], qq, lane, ns_e, ns_o);
+              col_next(ye[2], yo[2], qq, lane, np_e, np_o);
+              col_next(dye[0], dyo[0], qq, lane, nds_e, nds_o);
+              col_next(dye[1], dyo[1], qq, lane, ndp_e, ndp_o);
+              col_next(ye[1], yo[1], qq, lane, nbs_e, nbs_o);
+              col_next(ye[3], yo[3], qq, lane, nbp_e, nbp_o);
+              const bool row_ok = R[hf].lo[0] <= u && u <= R[hf].hi[0] && R[hf].lo[1] <= ty && ty <= R[hf].hi[1];
+#pragma unroll
+              for (int jt = 0; jt < 4; jt++) {
+#pragma unroll
+                for (int od = 0; od < 2; od++) {
+                  const int wx = 8 * jt + 2 * qq + od - R[hf].ox;
+                  const bool valid = row_ok && wx >= R[hf].lo[2] && wx <= R[hf].hi[2];
+                  const float sy = od ? yo[0][jt] : ye[0][jt], sn = od ? ns_o[jt] : ns_e[jt];
+                  const float py = od ? yo[2][jt] : ye[2][jt], pn = od ? np_o[jt] : np_e[jt];
+                  const float dsy = od ? dyo[0][jt] : dye[0][jt], dsn = od ? nds_o[jt] : nds_e[jt];
+                  const float dpy = od ? dyo[1][jt] : dye[1][jt], dpn = od ? ndp_o[jt] : ndp_e[jt];
+                  const float bsy = od ? yo[1][jt] : ye[1][jt], bsn = od ? nbs_o[jt] : nbs_e[jt];
+                  const float bpy = od ? yo[3][jt] : ye[3][jt], bpn = od ? nbp_o[jt] : nbp_e[jt];
+                  const float s = fmaf(fx, sn - sy, sy);      // raw score of the tap
+                  const float dpv = fmaf(fx, pn - py, py);    // dP of the tap
+                  float P = 0.f, PdP = 0.f;
+                  if (valid) {
+                    P = exp2f(fmaf(s, sc, -lse2[hf]));
+                    PdP = P * dpv;
+                    const float ds[3] = {fmaf(fx, bsn - bsy, bsy), fmaf(fx, dsn - dsy, dsy), sn - sy};
+                    const float dp[3] = {fmaf(fx, bpn - bpy, bpy), fmaf(fx, dpn - dpy, dpy), pn - py};
+                    Dp[hf] += PdP;
+#pragma unroll
+                    for (int ax = 0; ax < 3; ax++) {
+                      A[hf][ax] = fmaf(PdP, ds[ax], A[hf][ax]);
+                      Bs[hf][ax] = fmaf(P, ds[ax], Bs[hf][ax]);
+                      C[hf][ax] = fmaf(P, dp[ax], C[hf][ax]);
+                    }
+                  }
+                  if (od) { po[hf][jt] = P; go[hf][jt] = PdP; } else { pe[hf][jt] = P; ge[hf][jt] = PdP; }
+                }
+              }
+            }
+            // splats onto box row ty: x-transpose, then y-mix with the previous tap row
+#pragma unroll
+            for (int hf = 0; hf < 2; hf++) {
+              const float fx = R[hf].f[2], fy = R[hf].f[1];
+              float pv_e[4], pv_o[4], gv_e[4], gv_o[4];
+              col_prev(pe[hf], po[hf], qq, lane, pv_e, pv_o);
+              col_prev(ge[hf], go[hf], qq, lane, gv_e, gv_o);
+              float be[4], bo[4], gme[4], gmo[4];
+#pragma unroll
+              for (int jt = 0; jt < 4; jt++) {
+                const float bxe = fmaf(fx, pv_e[jt] - pe[hf][jt], pe[hf][jt]);
+                const float bxo = fmaf(fx, pv_o[jt] - po[hf][jt], po[hf][jt]);
+                const float gxe = fmaf(fx, gv_e[jt] - ge[hf][jt], ge[hf][jt]);
+                const float gxo = fmaf(fx, gv_o[jt] - go[hf][jt], go[hf][jt]);
+                float* bp = bxp + (jt * 4 + 2 * hf) * 32 + lane;
+                be[jt] = fmaf(fy, bp[0] - bxe, bxe);
+                bo[jt] = fmaf(fy, bp[32] - bxo, bxo);
+                gme[jt] = fmaf(fy, bp[16 * 32] - gxe, gxe);
+                gmo[jt] = fmaf(fy, bp[16 * 32 + 32] - gxo, gxo);
+                bp[0] = bxe;
+                bp[32] = bxo;
+                bp[16 * 32] = gxe;
+                bp[16 * 32 + 32] = gxo;
+              }
+              if (R[hf].live) {
+                const int64_t o = ((int64_t)(pos + gq + 8 * hf) * bg.rows + u * (g.kh + 1) + ty) * bg.width;
+                store_box_row(bbox + o, be, bo, R[hf].ox, bg.width, qq);
+                store_box_row(gbox + o, gme, gmo, R[hf].ox, bg.width, qq);
+              }
+            }
+          }
+          // this box row becomes the previous one
+#pragma unroll
+          for (int b = 0; b < 4; b++)
+#pragma unroll
+            for (int jt = 0; jt < 4; jt++)
+#pragma unroll
+              for (int e = 0; e < 4; e++) prev[(b * 16 + jt * 4 + e) * 32 + lane] = cur[b][jt][e];
+          __syncwarp();
+        }
+        // box row kh takes only the y-carry of tap row kh-1
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++) {
+          const float fy = R[hf].f[1];
+          float be[4], bo[4], gme[4], gmo[4];
+#pragma unroll
+          for (int jt = 0; jt < 4; jt++) {
+            const float* bp = bxp + (jt * 4 + 2 * hf) * 32 + lane;
+            be[jt] = fy * bp[0];
+            bo[jt] = fy * bp[32];
+            gme[jt] = fy * bp[16 * 32];
+            gmo[jt] = fy * bp[16 * 32 + 32];
+          }
+          if (R[hf].live) {
+            const int64_t o = ((int64_t)(pos + gq + 8 * hf) * bg.rows + u * (g.kh + 1) + g.kh) * bg.width;
+            store_box_row(bbox + o, be, bo, R[hf].ox, bg.width, qq);
+            store_box_row(gbox + o, gme, gmo, R[hf].ox, bg.width, qq);
+          }
+        }
+        __syncwarp();
+      }
+
+      // per-query totals: reduce over the quad, then D, doff, (D, f_t)
+#pragma unroll
+      for (int hf = 0; hf < 2; hf++) {
+        float d = Dp[hf];
+        d += __shfl_xor_sync(kFull, d, 1);
+        d += __shfl_xor_sync(kFull, d, 2);
+        float res[3];
+#pragma unroll
+        for (int ax = 0; ax < 3; ax++) {
+          float a = A[hf][ax], b = Bs[hf][ax], c = C[hf][ax];
+          a += __shfl_xor_sync(kFull, a, 1);
+          a += __shfl_xor_sync(kFull, a, 2);
+          b += __shfl_xor_sync(kFull, b, 1);
+          b += __shfl_xor_sync(kFull, b, 2);
+          c += __shfl_xor_sync(kFull, c, 1);
+          c += __shfl_xor_sync(kFull, c, 2);
+          res[ax] = fmaf(g.scale, fmaf(-d, b, a), c);
+        }
+        if (R[hf].live && qq == 0) {
+          float* od = doff + ((int64_t)h * g.N + R[hf].n) * 3;
+          od[0] = res[0];
+          od[1] = res[1];
+          od[2] = res[2];
+          dft[pos + gq + 8 * hf] = make_float2(d, R[hf].f[0]);
+        }
+      }
+      pos += cnt;
+    }
+  }
+}
+
+// ---- shared helpers of passes 2 and 3 ----------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(unsigned (&r)[4], const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+
+// gamma and beta of one query at box plane bt, box row by, column bx (t-mix of the stored tap
+// planes bt and bt-1; gamma = gamma' - D beta).
+__device__ __forceinline__ void box_value(const unsigned short* gbox, const unsigned short* bbox,
+                                          int64_t pos, const BoxGeo& bg, int kt, int kh, int bt,
+                                          int by, int bx, float D, float ft, float& gam, float& bet) {
+  gam = 0.f;
+  bet = 0.f;
+  if (bt < kt) {
+    const int64_t o = (pos * bg.rows + bt * (kh + 1) + by) * bg.width + bx;
+    const float b = bf16_val(bbox[o]), gp = bf16_val(gbox[o]);
+    bet = (1.f - ft) * b;
+    gam = (1.f - ft) * fmaf(-D, b, gp);
+  }
+  if (bt >= 1) {
+    const int64_t o = (pos * bg.rows + (bt - 1) * (kh + 1) + by) * bg.width + bx;
+    const float b = bf16_val(bbox[o]), gp = bf16_val(gbox[o]);
+    bet = fmaf(ft, b, bet);
+    gam = fmaf(ft, fmaf(-D, b, gp), gam);
+  }
+}
+
+// ---- pass 2: dq = scale * sum_j gamma[j] K[j] ----------------------------------------------------
+template <int DH>
+__global__ void __launch_bounds__(128)
+    dsa3d_bwd_dq_kernel(const __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ dq,
+                        const int* __restrict__ start, const int* __restrict__ sorted_n,
+                        const int* __restrict__ sorted_ex, const unsigned short* __restrict__ gbox,
+                        const unsigned short* __restrict__ bbox, const float2* __restrict__ dft,
+                        const Geo g, const SortGeo sg, const BoxGeo bg, const int h0, const int hg) {
+  using S = MmaShape<DH>;
+  constexpr int TS = 40;  // tile row stride (bf16), conflict-free for ldmatrix
+  __shared__ __align__(16) unsigned short tile_sh[4][16 * TS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, qq = lane & 3;
+  unsigned short* tile = tile_sh[warp];
+  const int64_t rs = (int64_t)g.heads * DH;
+  const int segw = 16 + g.kw;
+  const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
+
+  for (int64_t row = (int64_t)blockIdx.x * 4 + warp; row < rows; row += (int64_t)gridDim.x * 4) {
+    const int hh = (int)(row / ((int64_t)sg.Et * sg.Ey));
+    const int rem = (int)(row - (int64_t)hh * sg.Et * sg.Ey);
+    const int et = rem / sg.Ey, ey = rem % sg.Ey;
+    const int h = h0 + hh;
+    const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)et * sg.Ey + ey) * sg.Ex;
+    const int qbeg = start[b0], qend = start[b0 + sg.Ex];
+    const int ot = et - g.kt, oy = ey - g.kh;
+    const __nv_bfloat16* kh_ = k + (int64_t)h * DH;
+
+    for (int pos = qbeg; pos < qend;) {
+      int X0;
+      const int cnt = chunk_len(sorted_ex, pos, qend, g.kw, lane, X0);
+      float acc[S::NT][4];
+#pragma unroll
+      for (int j = 0; j < S::NT; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+
+      for (int bt = 0; bt <= g.kt; bt++) {
+        const int t = ot + bt;
+        if (t < 0 || t >= g.F) continue;
+        for (int by = 0; by <= g.kh; by++) {
+          const int y = oy + by;
+          if (y < 0 || y >= g.Hp) continue;
+          // gamma tile: rows = queries, cols = segment keys
+          for (int i = lane; i < 16 * TS / 8; i += 32) reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
+          __syncwarp();
+          for (int idx = lane; idx < 16 * bg.width; idx += 32) {
+            const int r = idx / bg.width, bx = idx - r * bg.width;
+            if (r >= cnt) continue;
+            const float2 d = dft[pos + r];
+            float ga, be;
+            box_value(gbox, bbox, pos + r, bg, g.kt, g.kh, bt, by, bx, d.x, d.y, ga, be);
+            const int col = sorted_ex[pos + r] - g.kw - X0 + bx;
+            tile[r * TS + col] = bf16_bits(ga);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int kk = 0; kk < 2; kk++) {
+            unsigned a[4];
+            const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4) + 16 * kk;
+            ldsm_x4(a, tile + rr * TS + cc);
+            unsigned vw[4][S::VW];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+              const int key = 16 * kk + 2 * qq + (i & 1) + 8 * (i >> 1);
+              const int x = X0 + key;
+              const bool ok = key < segw && x >= 0 && x < g.Wp;
+              const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + gq * S::NT;
+#pragma unroll
+              for (int c = 0; c < S::VW / 4; c++) {
+                const uint4 w = ok ? ldg16(kr + c * 8) : make_uint4(0, 0, 0, 0);
+                vw[i][4 * c] = w.x; vw[i][4 * c + 1] = w.y; vw[i][4 * c + 2] = w.z; vw[i][4 * c + 3] = w.w;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < S::NT; j++) {
+              const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
+              const unsigned b0_ = __byte_perm(vw[0][j >> 1], vw[1][j >> 1], sel);
+              const unsigned b1_ = __byte_perm(vw[2][j >> 1], vw[3][j >> 1], sel);
+              mma_bf16_16816(acc[j], a[0], a[1], a[2], a[3], b0_, b1_);
+            }
+          }
+          __syncwarp();
+        }
+      }
+#pragma unroll
+      for (int hf = 0; hf < 2; hf++) {
+        const int r = gq + 8 * hf;
+        if (r >= cnt) continue;
+        const int n = sorted_n[pos + r];
+        __nv_bfloat16* drow = dq + ((int64_t)n * g.heads + h) * DH + qq * (DH / 4);
+        float vals[S::NT * 2];
+#pragma unroll
+        for (int j = 0; j < S::NT; j++) {
+          vals[j] = acc[j][2 * hf] * g.scale;
+          vals[S::NT + j] = acc[j][2 * hf + 1] * g.scale;
+        }
+#pragma unroll
+        for (int c = 0; c < S::NT * 2 / 8; c++) store16(drow + c * 8, vals + c * 8);
+      }
+      pos += cnt;
+    }
+  }
+}
+
+// ---- pass 3: key side ------------------------------------------------------------------------
+// Task = (head, key row (tk, yk), 16-key block b, dim half).  Contributing queries: origins with
+// o_t in [tk - kt, tk], o_y in [yk - kh, yk], o_x in [16b - kw, 16b + 15], i.e. bucket rows
+// e_t = tk - bt + kt, e_y = yk - by + kh and the e_x range [16b, 16b + 16 + kw).
+template <int DH>
+__global__ void __launch_bounds__(128)
+    dsa3d_bwd_kv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
+                        __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                        const int* __restrict__ start, const int* __restrict__ sorted_n,
+                        const int* __restrict__ sorted_ex, const unsigned short* __restrict__ gbox,
+                        const unsigned short* __restrict__ bbox, const float2* __restrict__ dft,
+                        const Geo g, const SortGeo sg, const BoxGeo bg, const int h0, const int hg) {
+  constexpr int HALF = DH / 2;     // dims per task
+  constexpr int NTH = HALF / 8;    // n-tiles per task
+  constexpr int SL = NTH;          // dims of a lane's B slice
+  constexpr int TS = 24;           // tile row stride (bf16)
+  __shared__ __align__(16) unsigned short tg_sh[4][16 * TS];
+  __shared__ __align__(16) unsigned short tb_sh[4][16 * TS];
+  __shared__ int tok_sh[4][16];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, qq = lane & 3;
+  unsigned short* tg = tg_sh[warp];
+  unsigned short* tb = tb_sh[warp];
+  int* tok = tok_sh[warp];
+  const int NB = (g.Wp + 15) / 16;
+  const int64_t tasks = (int64_t)hg * g.F * g.Hp * NB * 2;
+
+  for (int64_t task = (int64_t)blockIdx.x * 4 + warp; task < tasks; task += (int64_t)gridDim.x * 4) {
+    const int half = (int)(task & 1);
+    int64_t r = task >> 1;
+    const int b = (int)(r % NB);
+    r /= NB;
+    const int yk = (int)(r % g.Hp);
+    r /= g.Hp;
+    const int tk = (int)(r % g.F);
+    const int hh = (int)(r / g.F);
+    const int h = h0 + hh;
+    const int x_lo = 16 * b;
+
+    float ak[NTH][4], av[NTH][4];
+#pragma unroll
+    for (int j = 0; j < NTH; j++) ak[j][0] = ak[j][1] = ak[j][2] = ak[j][3] = av[j][0] = av[j][1] = av[j][2] = av[j][3] = 0.f;
+
+    for (int bt = 0; bt <= g.kt; bt++) {
+      const int et = tk - bt + g.kt;
+      for (int by = 0; by <= g.kh; by++) {
+        const int ey = yk - by + g.kh;
+        const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)et * sg.Ey + ey) * sg.Ex;
+        const int qs = start[b0 + x_lo];
+        const int qe = start[b0 + min(x_lo + 16 + g.kw, sg.Ex)];
+        for (int pos = qs; pos < qe; pos += 16) {
+          const int cnt = min(16, qe - pos);
+          for (int i = lane; i < 16 * TS / 8; i += 32) {
+            reinterpret_cast<uint4*>(tg)[i] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4*>(tb)[i] = make_uint4(0, 0, 0, 0);
+          }
+          if (lane < 16) tok[lane] = (lane < cnt) ? sorted_n[pos + lane] : -1;
+          __syncwarp();
+          for (int idx = lane; idx < 16 * bg.width; idx += 32) {
+            const int m = idx / bg.width, bx = idx - m * bg.width;
+            if (m >= cnt) continue;
+            const int key = sorted_ex[pos + m] - g.kw + bx - x_lo;
+            if (key < 0 || key >= 16) continue;
+            const float2 d = dft[pos + m];
+            float ga, be;
+            box_value(gbox, bbox, pos + m, bg, g.kt, g.kh, bt, by, bx, d.x, d.y, ga, be);
+            tg[key * TS + m] = bf16_bits(ga);
+            tb[key * TS + m] = bf16_bits(be);
+          }
+          __syncwarp();
+          unsigned agm[4], abt[4];
+          const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4);
+          ldsm_x4(agm, tg + rr * TS + cc);
+          ldsm_x4(abt, tb + rr * TS + cc);
+          // B fragments: queries 2q, 2q+1, 2q+8, 2q+9; lane gq owns dims half*HALF + gq*SL + [0, SL)
+          unsigned qw[4][SL / 2], ow[4][SL / 2];
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            const int m = 2 * qq + (i & 1) + 8 * (i >> 1);
+            const int n = tok[m];
+            const int64_t off_e = ((int64_t)max(n, 0) * g.heads + h) * DH + half * HALF + gq * SL;
+            if constexpr (SL >= 8) {
+#pragma unroll
+              for (int c = 0; c < SL / 8; c++) {
+                const uint4 a = (n >= 0) ? ldg16(q + off_e + c * 8) : make_uint4(0, 0, 0, 0);
+                const uint4 e = (n >= 0) ? ldg16(dout + off_e + c * 8) : make_uint4(0, 0, 0, 0);
+                qw[i][4 * c] = a.x; qw[i][4 * c + 1] = a.y; qw[i][4 * c + 2] = a.z; qw[i][4 * c + 3] = a.w;
+                ow[i][4 * c] = e.x; ow[i][4 * c + 1] = e.y; ow[i][4 * c + 2] = e.z; ow[i][4 * c + 3] = e.w;
+              }
+            } else {
+              const uint2 a = (n >= 0) ? __ldg(reinterpret_cast<const uint2*>(q + off_e)) : make_uint2(0, 0);
+              const uint2 e = (n >= 0) ? __ldg(reinterpret_cast<const uint2*>(dout + off_e)) : make_uint2(0, 0);
+              qw[i][0] = a.x; qw[i][1] = a.y;
+              ow[i][0] = e.x; ow[i][1] = e.y;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < NTH; j++) {
+            const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
+            mma_bf16_16816(ak[j], agm[0], agm[1], agm[2], agm[3], __byte_perm(qw[0][j >> 1], qw[1][j >> 1], sel),
+                           __byte_perm(qw[2][j >> 1], qw[3][j >> 1], sel));
+            mma_bf16_16816(av[j], abt[0], abt[1], abt[2], abt[3], __byte_perm(ow[0][j >> 1], ow[1][j >> 1], sel),
+                           __byte_perm(ow[2][j >> 1], ow[3][j >> 1], sel));
+          }
+          __syncwarp();
+        }
+      }
+    }
+    // write: key rows g, g+8 of the block; lane dims half*HALF + 2q*NTH + [0, 2*NTH)
+#pragma unroll
+    for (int hf = 0; hf < 2; hf++) {
+      const int x = x_lo + gq + 8 * hf;
+      if (x >= g.Wp) continue;
+      const int64_t tokk = ((int64_t)tk * g.Hp + yk) * g.Wp + x;
+      const int64_t base = (tokk * g.heads + h) * DH + half * HALF + 2 * qq * NTH;
+      float vk[2 * NTH], vv[2 * NTH];
+#pragma unroll
+      for (int j = 0; j < NTH; j++) {
+        vk[j] = ak[j][2 * hf] * g.scale;
+        vk[NTH + j] = ak[j][2 * hf + 1] * g.scale;
+        vv[j] = av[j][2 * hf];
+        vv[NTH + j] = av[j][2 * hf + 1];
+      }
+#pragma unroll
+      for (int c = 0; c < 2 * NTH / 8; c++) {
+        store16(dk + base + c * 8, vk + c * 8);
+        store16(dv + base + c * 8, vv + c * 8);
+      }
+    }
+  }
+}
+
+}  // namespace dsa3d

@@ -22,12 +22,14 @@ struct SortGeo {
 };
 
 // Per query of heads [h0, h0 + hg): bucket and rank; queries without a valid tap get key -1.
-// If out != nullptr, such queries' out rows are zeroed and their lse set to -inf here.
+// Such queries' rows of `out` (the forward's out, or the backward's dq) are zeroed here when out
+// is given, their lse set to -inf when lse is given and their offset gradient zeroed when doff is.
 template <typename T, int DH>
 __global__ void dsa3d_sort_count_kernel(const float* __restrict__ off, const Geo g, const SortGeo sg,
                                         const int h0, const int hg, int* __restrict__ cnt,
                                         int* __restrict__ qkey, int* __restrict__ qrank,
-                                        T* __restrict__ out, float* __restrict__ lse) {
+                                        T* __restrict__ out, float* __restrict__ lse,
+                                        float* __restrict__ doff) {
   const int64_t items = (int64_t)hg * g.N;
   for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
        it += (int64_t)gridDim.x * blockDim.x) {
@@ -44,7 +46,11 @@ __global__ void dsa3d_sort_count_kernel(const float* __restrict__ off, const Geo
         for (int e = 0; e < Elems<T>::kPerLoad; e++) z[e] = 0.f;
 #pragma unroll
         for (int c = 0; c < DH / Elems<T>::kPerLoad; c++) store16(row + c * Elems<T>::kPerLoad, z);
-        if (lse) lse[(int64_t)h * g.N + n] = -INFINITY;
+      }
+      if (lse) lse[(int64_t)h * g.N + n] = -INFINITY;
+      if (doff) {
+        float* od = doff + ((int64_t)h * g.N + n) * 3;
+        od[0] = od[1] = od[2] = 0.f;
       }
       continue;
     }

@@ -20,13 +20,17 @@ enum KernelId {
   kKernSortCount,
   kKernScan,
   kKernSortFill,
+  kKernBwdQ,
+  kKernBwdDq,
+  kKernBwdKv,
   kKernCount
 };
 inline const char* kernel_name(int id) {
   static const char* names[kKernCount] = {
       "dsa3d_fwd_kernel",      "dsa3d_bwd_kernel",        "dsa3d_bwd_finalize_kernel",
       "dsa3d_zero_kernel",     "dsa3d_fwd_mma_kernel",    "dsa3d_sort_count_kernel",
-      "dsa3d_scan_kernels",    "dsa3d_sort_fill_kernel"};
+      "dsa3d_scan_kernels",    "dsa3d_sort_fill_kernel",  "dsa3d_bwd_q_kernel",
+      "dsa3d_bwd_dq_kernel",   "dsa3d_bwd_kv_kernel"};
   return names[id];
 }
 
