@@ -59,19 +59,32 @@ def measured_peaks():
 
 
 # --- algorithmic units -------------------------------------------------------------------------
+# Per (token, head), each tensor the kernel must touch read or written once; s = element size.
+# Whole path: forward 4 dh s + 16, backward 8 dh s + 28 (q, k, v, dO read; dq, dk, dv written;
+# offsets, lse read; doffsets written).  Per kernel, the backward's three passes each re-read
+# some inputs, so their sum (10 dh s + 28) exceeds the backward's figure.
 def alg_bytes_per_item(w, kernel):
-    """Algorithmic HBM bytes per (token, head): each tensor read or written once."""
     s = 4 if w.dtype == "f32" else 2
-    if kernel == "fwd":
-        return 4 * w.dh * s + 12 + 4            # q, k, v read, out written; offsets, lse
-    return 8 * w.dh * s + 12 + 4 + 12           # q, k, v, out, dO read; dq, dk, dv written;
-    #                                             offsets, lse read; doffsets written
+    table = {
+        "dsa3d_fwd_kernel": 4 * w.dh * s + 16,        # q, k, v -> out; offsets, lse
+        "dsa3d_fwd_mma_kernel": 4 * w.dh * s + 16,
+        "dsa3d_bwd_kernel": 8 * w.dh * s + 28,        # the CUDA-core backward does it all
+        "dsa3d_bwd_q_kernel": 4 * w.dh * s + 28,      # q, k, v, dO; offsets, lse -> doffsets
+        "dsa3d_bwd_dq_kernel": 2 * w.dh * s,          # k -> dq
+        "dsa3d_bwd_kv_kernel": 4 * w.dh * s,          # q, dO -> dk, dv
+        "fwd": 4 * w.dh * s + 16,
+        "bwd": 8 * w.dh * s + 28,
+    }
+    return table.get(kernel, 0)
 
 
 def alg_flop_per_item(w, kernel):
-    """Factorised fp32 work per (token, head): box dots and box axpys of length dh."""
+    """Factorised fp32 work per (token, head): dots and axpys of length dh over the B box tokens."""
     B = (w.window[0] + 1) * (w.window[1] + 1) * (w.window[2] + 1)
-    return (4 if kernel == "fwd" else 10) * w.dh * B
+    per = {"dsa3d_fwd_kernel": 4, "dsa3d_fwd_mma_kernel": 4, "dsa3d_bwd_kernel": 10,
+           "dsa3d_bwd_q_kernel": 4, "dsa3d_bwd_dq_kernel": 2, "dsa3d_bwd_kv_kernel": 4,
+           "fwd": 4, "bwd": 10}
+    return per.get(kernel, 0) * w.dh * B
 
 
 # --- clocks ------------------------------------------------------------------------------------
@@ -148,8 +161,9 @@ def head_inputs_for_oracle(w, inp, head=0):
 
 
 def calibrated_items(w, hin, threads, budget_s):
-    t1 = oracle_sample(w, hin, max(threads, 1), 12345, threads)
-    per_round = t1  # one item per thread
+    oracle_sample(w, hin, max(threads, 1), 12344, threads)  # warm the inputs' pages
+    t1 = oracle_sample(w, hin, 4 * max(threads, 1), 12345, threads)
+    per_round = t1 / 4  # one item per thread
     rounds = max(1, int(budget_s / max(per_round, 1e-6)))
     return rounds * max(threads, 1)
 
@@ -298,10 +312,9 @@ def main(argv=None):
     if dominant:
         kname, (n, tot) = dominant
         avg_ms = tot / n
-        kind = "fwd" if "fwd" in kname else "bwd"
         launches_per_step = n / args.steps
         items_per_launch = w.heads * w.N / launches_per_step
-        alg = alg_bytes_per_item(w, kind) * items_per_launch
+        alg = alg_bytes_per_item(w, kname) * items_per_launch
         achieved = alg / (avg_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": None, "kernel": kname,
@@ -309,7 +322,7 @@ def main(argv=None):
                                if peak_src == "measured" else "fallback 6.65 TB/s"}
         mhz = clocks["sm_mhz"] or float(peaks.get("sm_max_mhz", 1965.0))
         fp32_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
-        flops = alg_flop_per_item(w, kind) * items_per_launch
+        flops = alg_flop_per_item(w, kname) * items_per_launch
         alu = {"bound": "alu", "achieved": flops / (avg_ms / 1000.0) / 1e12, "unit": "TFLOP/s",
                "peak": fp32_peak, "frac": flops / (avg_ms / 1000.0) / 1e12 / fp32_peak,
                "peak_basis": f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {mhz:.0f} MHz"}

@@ -127,7 +127,7 @@ __device__ __forceinline__ void store_box_row(unsigned short* dst, const float (
 
 // ---- pass 1: query side ---------------------------------------------------------------------
 template <int DH>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
     dsa3d_bwd_q_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                        const float* __restrict__ off, const float* __restrict__ lse,
@@ -396,7 +396,7 @@ __device__ __forceinline__ void box_value(const unsigned short* gbox, const unsi
 
 // ---- pass 2: dq = scale * sum_j gamma[j] K[j] ----------------------------------------------------
 template <int DH>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
     dsa3d_bwd_dq_kernel(const __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ dq,
                         const int* __restrict__ start, const int* __restrict__ sorted_n,
                         const int* __restrict__ sorted_ex, const unsigned short* __restrict__ gbox,
@@ -498,134 +498,157 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---- pass 3: key side ------------------------------------------------------------------------
-// Task = (head, key row (tk, yk), 16-key block b, dim half).  Contributing queries: origins with
-// o_t in [tk - kt, tk], o_y in [yk - kh, yk], o_x in [16b - kw, 16b + 15], i.e. bucket rows
-// e_t = tk - bt + kt, e_y = yk - by + kh and the e_x range [16b, 16b + 16 + kw).
+// One CTA of 8 warps owns a key tile of 4 consecutive key rows (yk0..yk0+3) x 16 keys
+// (x in [16b, 16b+16)) of one frame tk and head; warp w takes key row w/2 and half w%2 of the
+// head dims, with dK and dV in registers.  The queries whose windows cover the tile have origins
+// o_t = tk - bt, o_y in [yk0 - kh, yk0 + 3], o_x in [16b - kw, 16b + 15], i.e. bucket rows
+// e_t = tk - bt + kt, e_y in [yk0, yk0 + 3 + kh] and the e_x range [16b, 16b + 16 + kw).  Per
+// step (<= 16 such queries of one bucket row) the CTA stages their q and dO rows and the four key
+// rows' Gamma^T / Beta^T tiles (key x query, gathered from the stored splats) in shared memory;
+// each warp then adds Gamma^T q and Beta^T dO for its key row with m16n8k16 MMAs (B fragments by
+// ldmatrix.trans of the staged rows).  A query row is loaded once per tile, not once per key row.
+constexpr int kKvRows = 4;
+
 template <int DH>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256, DSA3D_KV_MINB)
     dsa3d_bwd_kv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
                         __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                         const int* __restrict__ start, const int* __restrict__ sorted_n,
                         const int* __restrict__ sorted_ex, const unsigned short* __restrict__ gbox,
                         const unsigned short* __restrict__ bbox, const float2* __restrict__ dft,
                         const Geo g, const SortGeo sg, const BoxGeo bg, const int h0, const int hg) {
-  constexpr int HALF = DH / 2;     // dims per task
-  constexpr int NTH = HALF / 8;    // n-tiles per task
-  constexpr int SL = NTH;          // dims of a lane's B slice
-  constexpr int TS = 24;           // tile row stride (bf16)
-  __shared__ __align__(16) unsigned short tg_sh[4][16 * TS];
-  __shared__ __align__(16) unsigned short tb_sh[4][16 * TS];
-  __shared__ int tok_sh[4][16];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int HALF = DH / 2;  // dims per warp
+  constexpr int NTH = HALF / 8; // n-tiles per warp
+  constexpr int TS = 24;        // Gamma/Beta tile row stride (bf16): conflict-free ldmatrix
+  constexpr int RS = DH + 8;    // staged q/dO row stride (bf16): conflict-free ldmatrix.trans
+  __shared__ __align__(16) unsigned short tg[kKvRows][16 * TS];
+  __shared__ __align__(16) unsigned short tb[kKvRows][16 * TS];
+  __shared__ __align__(16) unsigned short qs[16 * RS];
+  __shared__ __align__(16) unsigned short os[16 * RS];
+  __shared__ int m_tok[16], m_ox[16];
+  __shared__ float2 m_dft[16];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, qq = lane & 3;
-  unsigned short* tg = tg_sh[warp];
-  unsigned short* tb = tb_sh[warp];
-  int* tok = tok_sh[warp];
+  const int wr = warp >> 1, half = warp & 1;
   const int NB = (g.Wp + 15) / 16;
-  const int64_t tasks = (int64_t)hg * g.F * g.Hp * NB * 2;
+  const int NY = (g.Hp + kKvRows - 1) / kKvRows;
+  const int64_t tiles = (int64_t)hg * g.F * NY * NB;
 
-  for (int64_t task = (int64_t)blockIdx.x * 4 + warp; task < tasks; task += (int64_t)gridDim.x * 4) {
-    const int half = (int)(task & 1);
-    int64_t r = task >> 1;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    int64_t r = tile;
     const int b = (int)(r % NB);
     r /= NB;
-    const int yk = (int)(r % g.Hp);
-    r /= g.Hp;
+    const int yb = (int)(r % NY);
+    r /= NY;
     const int tk = (int)(r % g.F);
     const int hh = (int)(r / g.F);
     const int h = h0 + hh;
-    const int x_lo = 16 * b;
+    const int x_lo = 16 * b, yk0 = kKvRows * yb;
+    const int myk = yk0 + wr;  // this warp's key row
 
     float ak[NTH][4], av[NTH][4];
 #pragma unroll
-    for (int j = 0; j < NTH; j++) ak[j][0] = ak[j][1] = ak[j][2] = ak[j][3] = av[j][0] = av[j][1] = av[j][2] = av[j][3] = 0.f;
+    for (int j = 0; j < NTH; j++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) ak[j][e] = av[j][e] = 0.f;
 
     for (int bt = 0; bt <= g.kt; bt++) {
       const int et = tk - bt + g.kt;
-      for (int by = 0; by <= g.kh; by++) {
-        const int ey = yk - by + g.kh;
+      const int ey_hi = min(yk0 + kKvRows - 1 + g.kh, sg.Ey - 1);
+      for (int ey = yk0; ey <= ey_hi; ey++) {
         const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)et * sg.Ey + ey) * sg.Ex;
-        const int qs = start[b0 + x_lo];
-        const int qe = start[b0 + min(x_lo + 16 + g.kw, sg.Ex)];
-        for (int pos = qs; pos < qe; pos += 16) {
-          const int cnt = min(16, qe - pos);
-          for (int i = lane; i < 16 * TS / 8; i += 32) {
-            reinterpret_cast<uint4*>(tg)[i] = make_uint4(0, 0, 0, 0);
-            reinterpret_cast<uint4*>(tb)[i] = make_uint4(0, 0, 0, 0);
+        const int qbeg = start[b0 + x_lo];
+        const int qend = start[b0 + min(x_lo + 16 + g.kw, sg.Ex)];
+        for (int pos = qbeg; pos < qend; pos += 16) {
+          const int cnt = min(16, qend - pos);
+          __syncthreads();  // the previous step's tiles are consumed
+          // zero the tiles, load the step's per-query data
+          for (int i = tid; i < 2 * kKvRows * 16 * TS / 8; i += 256)
+            reinterpret_cast<uint4*>(i < kKvRows * 16 * TS / 8 ? &tg[0][0] : &tb[0][0])
+                [i < kKvRows * 16 * TS / 8 ? i : i - kKvRows * 16 * TS / 8] = make_uint4(0, 0, 0, 0);
+          if (tid < 16) {
+            const bool live = tid < cnt;
+            m_tok[tid] = live ? sorted_n[pos + tid] : -1;
+            m_ox[tid] = live ? sorted_ex[pos + tid] - g.kw - x_lo : 0;
+            m_dft[tid] = live ? dft[pos + tid] : make_float2(0.f, 0.f);
           }
-          if (lane < 16) tok[lane] = (lane < cnt) ? sorted_n[pos + lane] : -1;
-          __syncwarp();
-          for (int idx = lane; idx < 16 * bg.width; idx += 32) {
-            const int m = idx / bg.width, bx = idx - m * bg.width;
+          __syncthreads();
+          // stage q and dO rows (zeros for missing queries)
+          for (int i = tid; i < 2 * 16 * (DH / 8); i += 256) {
+            const int which = i / (16 * (DH / 8));
+            const int rem = i - which * 16 * (DH / 8);
+            const int m = rem / (DH / 8), c = rem - m * (DH / 8);
+            const int n = m_tok[m];
+            const __nv_bfloat16* src = which ? dout : q;
+            const uint4 val = (n >= 0) ? ldg16(src + ((int64_t)n * g.heads + h) * DH + c * 8)
+                                       : make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>((which ? os : qs) + m * RS + c * 8) = val;
+          }
+          // gather Gamma^T / Beta^T tiles of the 4 key rows: (query m, key row kr, column bx)
+          const int by_base = kKvRows - 1;  // by = yk0 + kr - ey + kh
+          for (int i = tid; i < 16 * kKvRows * bg.width; i += 256) {
+            const int m = i / (kKvRows * bg.width);
+            const int rem = i - m * (kKvRows * bg.width);
+            const int kr = rem / bg.width, bx = rem - kr * bg.width;
             if (m >= cnt) continue;
-            const int key = sorted_ex[pos + m] - g.kw + bx - x_lo;
+            const int by = yk0 + kr - ey + g.kh;
+            if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
+            const int key = m_ox[m] + bx;
             if (key < 0 || key >= 16) continue;
-            const float2 d = dft[pos + m];
+            const float2 d = m_dft[m];
             float ga, be;
             box_value(gbox, bbox, pos + m, bg, g.kt, g.kh, bt, by, bx, d.x, d.y, ga, be);
-            tg[key * TS + m] = bf16_bits(ga);
-            tb[key * TS + m] = bf16_bits(be);
+            tg[kr][key * TS + m] = bf16_bits(ga);
+            tb[kr][key * TS + m] = bf16_bits(be);
           }
-          __syncwarp();
-          unsigned agm[4], abt[4];
-          const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4);
-          ldsm_x4(agm, tg + rr * TS + cc);
-          ldsm_x4(abt, tb + rr * TS + cc);
-          // B fragments: queries 2q, 2q+1, 2q+8, 2q+9; lane gq owns dims half*HALF + gq*SL + [0, SL)
-          unsigned qw[4][SL / 2], ow[4][SL / 2];
+          (void)by_base;
+          __syncthreads();
+          const int by_w = myk - ey + g.kh;
+          if (myk < g.Hp && by_w >= 0 && by_w <= g.kh) {
+            unsigned agm[4], abt[4];
+            const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4);
+            ldsm_x4(agm, &tg[wr][rr * TS + cc]);
+            ldsm_x4(abt, &tb[wr][rr * TS + cc]);
 #pragma unroll
-          for (int i = 0; i < 4; i++) {
-            const int m = 2 * qq + (i & 1) + 8 * (i >> 1);
-            const int n = tok[m];
-            const int64_t off_e = ((int64_t)max(n, 0) * g.heads + h) * DH + half * HALF + gq * SL;
-            if constexpr (SL >= 8) {
-#pragma unroll
-              for (int c = 0; c < SL / 8; c++) {
-                const uint4 a = (n >= 0) ? ldg16(q + off_e + c * 8) : make_uint4(0, 0, 0, 0);
-                const uint4 e = (n >= 0) ? ldg16(dout + off_e + c * 8) : make_uint4(0, 0, 0, 0);
-                qw[i][4 * c] = a.x; qw[i][4 * c + 1] = a.y; qw[i][4 * c + 2] = a.z; qw[i][4 * c + 3] = a.w;
-                ow[i][4 * c] = e.x; ow[i][4 * c + 1] = e.y; ow[i][4 * c + 2] = e.z; ow[i][4 * c + 3] = e.w;
-              }
-            } else {
-              const uint2 a = (n >= 0) ? __ldg(reinterpret_cast<const uint2*>(q + off_e)) : make_uint2(0, 0);
-              const uint2 e = (n >= 0) ? __ldg(reinterpret_cast<const uint2*>(dout + off_e)) : make_uint2(0, 0);
-              qw[i][0] = a.x; qw[i][1] = a.y;
-              ow[i][0] = e.x; ow[i][1] = e.y;
+            for (int j2 = 0; j2 < NTH / 2; j2++) {
+              // B fragments of n-tiles 2*j2, 2*j2+1: rows = queries (k), cols = dims (n)
+              const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);
+              const int dcol = half * HALF + 16 * j2 + 8 * (lane >> 4);
+              unsigned bq[4], bo[4];
+              const unsigned aq = (unsigned)__cvta_generic_to_shared(qs + mrow * RS + dcol);
+              const unsigned ao = (unsigned)__cvta_generic_to_shared(os + mrow * RS + dcol);
+              asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                           : "=r"(bq[0]), "=r"(bq[1]), "=r"(bq[2]), "=r"(bq[3]) : "r"(aq));
+              asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                           : "=r"(bo[0]), "=r"(bo[1]), "=r"(bo[2]), "=r"(bo[3]) : "r"(ao));
+              mma_bf16_16816(ak[2 * j2], agm[0], agm[1], agm[2], agm[3], bq[0], bq[1]);
+              mma_bf16_16816(ak[2 * j2 + 1], agm[0], agm[1], agm[2], agm[3], bq[2], bq[3]);
+              mma_bf16_16816(av[2 * j2], abt[0], abt[1], abt[2], abt[3], bo[0], bo[1]);
+              mma_bf16_16816(av[2 * j2 + 1], abt[0], abt[1], abt[2], abt[3], bo[2], bo[3]);
             }
           }
-#pragma unroll
-          for (int j = 0; j < NTH; j++) {
-            const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
-            mma_bf16_16816(ak[j], agm[0], agm[1], agm[2], agm[3], __byte_perm(qw[0][j >> 1], qw[1][j >> 1], sel),
-                           __byte_perm(qw[2][j >> 1], qw[3][j >> 1], sel));
-            mma_bf16_16816(av[j], abt[0], abt[1], abt[2], abt[3], __byte_perm(ow[0][j >> 1], ow[1][j >> 1], sel),
-                           __byte_perm(ow[2][j >> 1], ow[3][j >> 1], sel));
-          }
-          __syncwarp();
         }
       }
     }
-    // write: key rows g, g+8 of the block; lane dims half*HALF + 2q*NTH + [0, 2*NTH)
+    // write this warp's key row: keys g, g+8 of the block; n-tile j col c -> dim half*HALF + 8j + c
+    if (myk < g.Hp) {
 #pragma unroll
-    for (int hf = 0; hf < 2; hf++) {
-      const int x = x_lo + gq + 8 * hf;
-      if (x >= g.Wp) continue;
-      const int64_t tokk = ((int64_t)tk * g.Hp + yk) * g.Wp + x;
-      const int64_t base = (tokk * g.heads + h) * DH + half * HALF + 2 * qq * NTH;
-      float vk[2 * NTH], vv[2 * NTH];
+      for (int hf = 0; hf < 2; hf++) {
+        const int x = x_lo + gq + 8 * hf;
+        if (x >= g.Wp) continue;
+        const int64_t tokk = ((int64_t)tk * g.Hp + myk) * g.Wp + x;
+        __nv_bfloat16* dkr = dk + (tokk * g.heads + h) * DH + half * HALF;
+        __nv_bfloat16* dvr = dv + (tokk * g.heads + h) * DH + half * HALF;
 #pragma unroll
-      for (int j = 0; j < NTH; j++) {
-        vk[j] = ak[j][2 * hf] * g.scale;
-        vk[NTH + j] = ak[j][2 * hf + 1] * g.scale;
-        vv[j] = av[j][2 * hf];
-        vv[NTH + j] = av[j][2 * hf + 1];
-      }
-#pragma unroll
-      for (int c = 0; c < 2 * NTH / 8; c++) {
-        store16(dk + base + c * 8, vk + c * 8);
-        store16(dv + base + c * 8, vv + c * 8);
+        for (int j = 0; j < NTH; j++) {
+          *reinterpret_cast<__nv_bfloat162*>(dkr + 8 * j + 2 * qq) =
+              __floats2bfloat162_rn(ak[j][2 * hf] * g.scale, ak[j][2 * hf + 1] * g.scale);
+          *reinterpret_cast<__nv_bfloat162*>(dvr + 8 * j + 2 * qq) =
+              __floats2bfloat162_rn(av[j][2 * hf], av[j][2 * hf + 1]);
+        }
       }
     }
+    __syncthreads();
   }
 }
 

@@ -11,6 +11,21 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+// Minimum resident CTAs per SM requested from the compiler for the tensor-core kernels
+// (trades registers for occupancy).
+#ifndef DSA3D_MMA_MINB
+#define DSA3D_MMA_MINB 2
+#endif
+#ifndef DSA3D_BWDQ_MINB
+#define DSA3D_BWDQ_MINB 2
+#endif
+#ifndef DSA3D_DQ_MINB
+#define DSA3D_DQ_MINB 3
+#endif
+#ifndef DSA3D_KV_MINB
+#define DSA3D_KV_MINB 2
+#endif
+
 namespace dsa3d {
 
 constexpr unsigned kFull = 0xffffffffu;

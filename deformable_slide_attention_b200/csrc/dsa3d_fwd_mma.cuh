@@ -130,7 +130,7 @@ __device__ __forceinline__ void dsa3d_pv_rows(float (&o)[MmaShape<DH>::NT][4], c
 }
 
 template <int DH>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
     dsa3d_fwd_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                          const __nv_bfloat16* __restrict__ v, const float* __restrict__ off,
                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse,

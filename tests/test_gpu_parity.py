@@ -193,3 +193,28 @@ def test_workspace_smaller_than_all_heads():
 
 def test_device_check_clean():
     assert abi.dsa3d_check_device(torch.cuda.current_stream().cuda_stream) == 0
+
+
+def test_cuda_core_backward_when_workspace_only_fits_its_accumulators():
+    """bf16 shapes with a tensor-core backward fall back to the CUDA-core backward when the
+    workspace holds one head's fp32 dK/dV accumulators but not the tensor-core pass's splats."""
+    dims, window, heads, dh = (4, 9, 10), (3, 9, 9), 2, 64
+    _, inp = inputs.custom(*dims, heads, dh, window, "bf16", seed=16, scale=2.0)
+    d = to_cuda(inp)
+    out, lse = gpu_forward(d, dims, window)
+    N = math.prod(dims)
+    acc_one = 2 * N * dh * 4
+    mma_one = abi.dsa3d_backward_workspace_bytes(*dims, 1, dh, *window, abi.DSA3D_BF16)
+    assert mma_one > acc_one
+    ws = torch.empty(acc_one, dtype=torch.uint8, device="cuda")
+    abi.dsa3d_timing_reset()
+    abi.dsa3d_timing_enable(True)
+    grads = abi.backward(d["q"], d["k"], d["v"], d["offsets"], lse, d["dout"], dims, window, workspace=ws)
+    torch.cuda.synchronize()
+    abi.dsa3d_timing_enable(False)
+    launched = abi.dsa3d_timing_read()
+    assert "dsa3d_bwd_kernel" in launched and "dsa3d_bwd_q_kernel" not in launched
+    r = oracle.full_backward(inp["q"], inp["k"], inp["v"], inp["offsets"], inp["dout"], dims, window)
+    for name, got, ref in (("dq", grads[0], r[0]), ("doff", grads[3], r[1]), ("dk", grads[1], r[2]),
+                           ("dv", grads[2], r[3])):
+        assert_close(name, f64(got), ref, TOL["bf16"])
