@@ -86,10 +86,20 @@ def test_forward_workspace_bytes():
 
 
 def test_backward_workspace_bytes():
-    ws = abi.dsa3d_backward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_BF16)
-    assert ws == 2 * 256 * 64 * 4 * 2
-    assert abi.dsa3d_backward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_F32) == 0
-    assert abi.dsa3d_backward_workspace_bytes(4, 8, 8, 2, 48, 3, 3, 3, abi.DSA3D_BF16) == 0
+    a16 = lambda b: (b + 15) // 16 * 16
+    F, Hp, Wp, H, kt, kh, kw = 4, 8, 8, 2, 3, 3, 3
+    N = F * Hp * Wp
+    # tensor-core backward (bf16, dh 64/128, kw <= 15): the sort's arrays, the bf16 splats of P and
+    # P dP per query and tap plane (kt (kh+1) (kw+1) each), and (D, f_t) per query
+    E1 = (F + kt) * (Hp + kh) * (Wp + kw) + 1
+    nb = (H * E1 + 2047) // 2048
+    sort = a16(4 * H * E1) + 4 * a16(4 * H * N) + a16(4 * nb)
+    splats = 2 * a16(H * N * kt * (kh + 1) * (kw + 1) * 2) + a16(H * N * 8)
+    assert abi.dsa3d_backward_workspace_bytes(F, Hp, Wp, H, 64, kt, kh, kw, abi.DSA3D_BF16) == sort + splats
+    # CUDA-core backward (bf16, dh 32): fp32 dK and dV accumulators of every head
+    assert abi.dsa3d_backward_workspace_bytes(F, Hp, Wp, H, 32, kt, kh, kw, abi.DSA3D_BF16) == 2 * N * 32 * 4 * H
+    assert abi.dsa3d_backward_workspace_bytes(F, Hp, Wp, H, 64, kt, kh, kw, abi.DSA3D_F32) == 0
+    assert abi.dsa3d_backward_workspace_bytes(F, Hp, Wp, H, 48, kt, kh, kw, abi.DSA3D_BF16) == 0
 
 
 def test_backward_rejects_bad_arguments():
