@@ -126,6 +126,20 @@ __device__ __forceinline__ void store_box_row(unsigned short* dst, const float (
 }
 
 // ---- pass 1: query side ---------------------------------------------------------------------
+// Per warp and chunk, per tap plane u and box row by: the MMA blocks of box planes u and u+1 for
+// q.K and dO.V are blended in registers to (st = S0 + f_t (S1 - S0), bd = S1 - S0) and
+// (dpt, dbd), and stored in a two-row ring in shared memory.  Then a compact epilogue: two lanes
+// per query, each taking every other tap of tap row by-1 (only the query's kw taps, not all 32
+// segment columns), forms the tap's score, dP, their derivatives along (t, y, x), P and the
+// per-query sums; the taps' P and P dP go to a two-row ring, from which box row by-1's splats
+// (x-transpose, then y-mix with the previous tap row) are stored.
+constexpr int kRawStride = 33;  // floats per row of a raw block (odd: conflict-free columns)
+constexpr int kTapStride = 16;  // floats per row of a tap-row buffer (kw <= 15)
+
+__host__ __device__ constexpr int bwdq_warp_floats() {
+  return 2 * 4 * 16 * kRawStride + 2 * 2 * 16 * kTapStride;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
     dsa3d_bwd_q_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -137,12 +151,12 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
                        float2* __restrict__ dft, const Geo g, const SortGeo sg, const BoxGeo bg,
                        const int h0, const int hg) {
   using S = MmaShape<DH>;
-  __shared__ float prev_sh[4][4 * 16 * 32];  // per warp: st, bd, dpt, dbd of the previous box row
-  __shared__ float bxp_sh[4][2 * 16 * 32];   // per warp: x-transposed P and P dP of the previous tap row
+  extern __shared__ __align__(16) float dyn_sh[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, qq = lane & 3;
-  float* prev = prev_sh[warp];
-  float* bxp = bxp_sh[warp];
+  float* raw = dyn_sh + warp * bwdq_warp_floats();         // [ring 2][block 4][16 rows][stride]
+  float* tapb = raw + 2 * 4 * 16 * kRawStride;              // [ring 2][P, PdP][16 rows][stride]
+  const int er = lane >> 1, side = lane & 1;                // epilogue: query row, tap parity
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
   const int segw = 16 + g.kw;
@@ -162,29 +176,27 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
     for (int pos = qbeg; pos < qend;) {
       int X0;
       const int cnt = chunk_len(sorted_ex, pos, qend, g.kw, lane, X0);
-      MmaRow R[2];
+      MmaRow R[2];  // fragment rows g, g+8 (for the MMA operands and the t-blend)
       chunk_rows(R, g, off, h, sorted_n, pos, cnt, X0, gq);
-      float lse2[2];
-#pragma unroll
-      for (int hf = 0; hf < 2; hf++)
-        lse2[hf] = R[hf].live ? __ldg(lse + (int64_t)h * g.N + R[hf].n) * kLog2e : 0.f;
       unsigned qa[S::KS][4], ga[S::KS][4];
       load_afrags<DH>(qa, q, R, h, g.heads, qq);
       load_afrags<DH>(ga, dout, R, h, g.heads, qq);
-
-      float Dp[2] = {0.f, 0.f};
-      float A[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
-      float Bs[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
-      float C[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+      // epilogue row er
+      const bool elive = er < cnt;
+      const int en = elive ? sorted_n[pos + er] : 0;
+      const Query EQ = decode_query(g, off, h, en);
+      const int eox = EQ.o[2] - X0;
+      const float ft = EQ.f[0], fy = EQ.f[1], fx = EQ.f[2];
+      const int lo_t = EQ.lo[0], hi_t = elive ? EQ.hi[0] : -1;
+      const float lse2 = elive ? __ldg(lse + (int64_t)h * g.N + en) * kLog2e : 0.f;
+      float Dp = 0.f, A[3] = {0.f, 0.f, 0.f}, Bs[3] = {0.f, 0.f, 0.f}, C[3] = {0.f, 0.f, 0.f};
 
       for (int u = 0; u < g.kt; u++) {
-        for (int i = lane; i < 4 * 16 * 32; i += 32) prev[i] = 0.f;
-        for (int i = lane; i < 2 * 16 * 32; i += 32) bxp[i] = 0.f;
-        __syncwarp();
+        const bool eplane = lo_t <= u && u <= hi_t;
+        for (int i = lane; i < 2 * 2 * 16 * kTapStride; i += 32) tapb[i] = 0.f;
         for (int by = 0; by <= g.kh; by++) {
           const int y = oy + by;
-          // raw blocks of box row by on planes u (0) and u+1 (1); blend and t-difference
-          float cur[4][4][4];  // [st, bd, dpt, dbd][jt][e]
+          float* rc = raw + (by & 1) * 4 * 16 * kRawStride;
           {
             float s0[4][4], s1[4][4];
             raw_block<DH>(s0, qa, kh_, ot + u, y, X0, segw, rs, g, gq, qq);
@@ -193,9 +205,10 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
             for (int jt = 0; jt < 4; jt++)
 #pragma unroll
               for (int e = 0; e < 4; e++) {
-                const float ft = R[e >> 1].f[0];
-                cur[1][jt][e] = s1[jt][e] - s0[jt][e];
-                cur[0][jt][e] = fmaf(ft, cur[1][jt][e], s0[jt][e]);
+                const int rr = gq + 8 * (e >> 1), cc = 8 * jt + 2 * qq + (e & 1);
+                const float d = s1[jt][e] - s0[jt][e];
+                rc[(0 * 16 + rr) * kRawStride + cc] = fmaf(R[e >> 1].f[0], d, s0[jt][e]);
+                rc[(1 * 16 + rr) * kRawStride + cc] = d;
               }
             raw_block<DH>(s0, ga, vh_, ot + u, y, X0, segw, rs, g, gq, qq);
             raw_block<DH>(s1, ga, vh_, ot + u + 1, y, X0, segw, rs, g, gq, qq);
@@ -203,162 +216,109 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
             for (int jt = 0; jt < 4; jt++)
 #pragma unroll
               for (int e = 0; e < 4; e++) {
-                const float ft = R[e >> 1].f[0];
-                cur[3][jt][e] = s1[jt][e] - s0[jt][e];
-                cur[2][jt][e] = fmaf(ft, cur[3][jt][e], s0[jt][e]);
+                const int rr = gq + 8 * (e >> 1), cc = 8 * jt + 2 * qq + (e & 1);
+                const float d = s1[jt][e] - s0[jt][e];
+                rc[(2 * 16 + rr) * kRawStride + cc] = fmaf(R[e >> 1].f[0], d, s0[jt][e]);
+                rc[(3 * 16 + rr) * kRawStride + cc] = d;
               }
           }
+          __syncwarp();
           if (by >= 1) {
             const int ty = by - 1;
-            float pe[2][4], po[2][4], ge[2][4], go[2][4];  // P and P dP of tap row ty
+            const float* rp = raw + ((by - 1) & 1) * 4 * 16 * kRawStride;
+            float* tp = tapb + (ty & 1) * 2 * 16 * kTapStride;
+            const bool erow = eplane && EQ.lo[1] <= ty && ty <= EQ.hi[1];
+            for (int wx = side; wx < g.kw; wx += 2) {
+              float P = 0.f, PdP = 0.f;
+              if (erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
+                const int c = eox + wx;
+                float yl[4][2], dy[2][2];
 #pragma unroll
-            for (int hf = 0; hf < 2; hf++) {
-              const float fx = R[hf].f[1 + 1], fy = R[hf].f[1];
-              // y-lerps (value, y-derivative) of the four blocks, even/odd columns
-              float ye[4][4], yo[4][4], dye[2][4], dyo[2][4];
+                for (int b = 0; b < 4; b++)
 #pragma unroll
-              for (int b = 0; b < 4; b++)
-#pragma unroll
-                for (int jt = 0; jt < 4; jt++) {
-                  const float pe_ = prev[(b * 16 + jt * 4 + 2 * hf) * 32 + lane];
-                  const float po_ = prev[(b * 16 + jt * 4 + 2 * hf + 1) * 32 + lane];
-                  const float ce = cur[b][jt][2 * hf], co = cur[b][jt][2 * hf + 1];
-                  ye[b][jt] = fmaf(fy, ce - pe_, pe_);
-                  yo[b][jt] = fmaf(fy, co - po_, po_);
-                  if (b == 0 || b == 2) {
-                    dye[b >> 1][jt] = ce - pe_;
-                    dyo[b >> 1][jt] = co - po_;
+                  for (int o = 0; o < 2; o++) {
+                    const float pv = rp[(b * 16 + er) * kRawStride + c + o];
+                    const float cv = rc[(b * 16 + er) * kRawStride + c + o];
+                    yl[b][o] = fmaf(fy, cv - pv, pv);
+                    if (b == 0 || b == 2) dy[b >> 1][o] = cv - pv;
                   }
-                }
-              // x-neighbours of the y-lerped blends and of the y-derivatives
-              float ns_e[4], ns_o[4], np_e[4], np_o[4], nds_e[4], nds_o[4], ndp_e[4], ndp_o[4];
-              float nbs_e[4], nbs_o[4], nbp_e[4], nbp_o[4];
-              col_next(ye[0], yo[0], qq, lane, ns_e, ns_o);
-              col_next(ye[2], yo[2], qq, lane, np_e, np_o);
-              col_next(dye[0], dyo[0], qq, lane, nds_e, nds_o);
-              col_next(dye[1], dyo[1], qq, lane, ndp_e, ndp_o);
-              col_next(ye[1], yo[1], qq, lane, nbs_e, nbs_o);
-              col_next(ye[3], yo[3], qq, lane, nbp_e, nbp_o);
-              const bool row_ok = R[hf].lo[0] <= u && u <= R[hf].hi[0] && R[hf].lo[1] <= ty && ty <= R[hf].hi[1];
+                const float s = fmaf(fx, yl[0][1] - yl[0][0], yl[0][0]);
+                const float dpv = fmaf(fx, yl[2][1] - yl[2][0], yl[2][0]);
+                const float ds[3] = {fmaf(fx, yl[1][1] - yl[1][0], yl[1][0]),
+                                     fmaf(fx, dy[0][1] - dy[0][0], dy[0][0]), yl[0][1] - yl[0][0]};
+                const float dp[3] = {fmaf(fx, yl[3][1] - yl[3][0], yl[3][0]),
+                                     fmaf(fx, dy[1][1] - dy[1][0], dy[1][0]), yl[2][1] - yl[2][0]};
+                P = exp2f(fmaf(s, sc, -lse2));
+                PdP = P * dpv;
+                Dp += PdP;
 #pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-#pragma unroll
-                for (int od = 0; od < 2; od++) {
-                  const int wx = 8 * jt + 2 * qq + od - R[hf].ox;
-                  const bool valid = row_ok && wx >= R[hf].lo[2] && wx <= R[hf].hi[2];
-                  const float sy = od ? yo[0][jt] : ye[0][jt], sn = od ? ns_o[jt] : ns_e[jt];
-                  const float py = od ? yo[2][jt] : ye[2][jt], pn = od ? np_o[jt] : np_e[jt];
-                  const float dsy = od ? dyo[0][jt] : dye[0][jt], dsn = od ? nds_o[jt] : nds_e[jt];
-                  const float dpy = od ? dyo[1][jt] : dye[1][jt], dpn = od ? ndp_o[jt] : ndp_e[jt];
-                  const float bsy = od ? yo[1][jt] : ye[1][jt], bsn = od ? nbs_o[jt] : nbs_e[jt];
-                  const float bpy = od ? yo[3][jt] : ye[3][jt], bpn = od ? nbp_o[jt] : nbp_e[jt];
-                  const float s = fmaf(fx, sn - sy, sy);      // raw score of the tap
-                  const float dpv = fmaf(fx, pn - py, py);    // dP of the tap
-                  float P = 0.f, PdP = 0.f;
-                  if (valid) {
-                    P = exp2f(fmaf(s, sc, -lse2[hf]));
-                    PdP = P * dpv;
-                    const float ds[3] = {fmaf(fx, bsn - bsy, bsy), fmaf(fx, dsn - dsy, dsy), sn - sy};
-                    const float dp[3] = {fmaf(fx, bpn - bpy, bpy), fmaf(fx, dpn - dpy, dpy), pn - py};
-                    Dp[hf] += PdP;
-#pragma unroll
-                    for (int ax = 0; ax < 3; ax++) {
-                      A[hf][ax] = fmaf(PdP, ds[ax], A[hf][ax]);
-                      Bs[hf][ax] = fmaf(P, ds[ax], Bs[hf][ax]);
-                      C[hf][ax] = fmaf(P, dp[ax], C[hf][ax]);
-                    }
-                  }
-                  if (od) { po[hf][jt] = P; go[hf][jt] = PdP; } else { pe[hf][jt] = P; ge[hf][jt] = PdP; }
+                for (int ax = 0; ax < 3; ax++) {
+                  A[ax] = fmaf(PdP, ds[ax], A[ax]);
+                  Bs[ax] = fmaf(P, ds[ax], Bs[ax]);
+                  C[ax] = fmaf(P, dp[ax], C[ax]);
                 }
               }
+              tp[(0 * 16 + er) * kTapStride + wx] = P;
+              tp[(1 * 16 + er) * kTapStride + wx] = PdP;
             }
-            // splats onto box row ty: x-transpose, then y-mix with the previous tap row
+            __syncwarp();
+            // splat onto box row ty: columns bx of this lane's parity
+            const float* tq = tapb + ((ty + 1) & 1) * 2 * 16 * kTapStride;  // tap row ty-1
+            if (elive) {
+              const int64_t o = ((int64_t)(pos + er) * bg.rows + u * (g.kh + 1) + ty) * bg.width;
+              for (int bx = side; bx <= g.kw; bx += 2) {
+                float vb[2], vg[2];
 #pragma unroll
-            for (int hf = 0; hf < 2; hf++) {
-              const float fx = R[hf].f[2], fy = R[hf].f[1];
-              float pv_e[4], pv_o[4], gv_e[4], gv_o[4];
-              col_prev(pe[hf], po[hf], qq, lane, pv_e, pv_o);
-              col_prev(ge[hf], go[hf], qq, lane, gv_e, gv_o);
-              float be[4], bo[4], gme[4], gmo[4];
-#pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-                const float bxe = fmaf(fx, pv_e[jt] - pe[hf][jt], pe[hf][jt]);
-                const float bxo = fmaf(fx, pv_o[jt] - po[hf][jt], po[hf][jt]);
-                const float gxe = fmaf(fx, gv_e[jt] - ge[hf][jt], ge[hf][jt]);
-                const float gxo = fmaf(fx, gv_o[jt] - go[hf][jt], go[hf][jt]);
-                float* bp = bxp + (jt * 4 + 2 * hf) * 32 + lane;
-                be[jt] = fmaf(fy, bp[0] - bxe, bxe);
-                bo[jt] = fmaf(fy, bp[32] - bxo, bxo);
-                gme[jt] = fmaf(fy, bp[16 * 32] - gxe, gxe);
-                gmo[jt] = fmaf(fy, bp[16 * 32 + 32] - gxo, gxo);
-                bp[0] = bxe;
-                bp[32] = bxo;
-                bp[16 * 32] = gxe;
-                bp[16 * 32 + 32] = gxo;
-              }
-              if (R[hf].live) {
-                const int64_t o = ((int64_t)(pos + gq + 8 * hf) * bg.rows + u * (g.kh + 1) + ty) * bg.width;
-                store_box_row(bbox + o, be, bo, R[hf].ox, bg.width, qq);
-                store_box_row(gbox + o, gme, gmo, R[hf].ox, bg.width, qq);
+                for (int w = 0; w < 2; w++) {
+                  const float* src = w ? tq : tp;
+                  const float p0 = (bx < g.kw) ? src[er * kTapStride + bx] : 0.f;
+                  const float p1 = (bx >= 1) ? src[er * kTapStride + bx - 1] : 0.f;
+                  const float g0 = (bx < g.kw) ? src[(16 + er) * kTapStride + bx] : 0.f;
+                  const float g1 = (bx >= 1) ? src[(16 + er) * kTapStride + bx - 1] : 0.f;
+                  vb[w] = fmaf(fx, p1 - p0, p0);
+                  vg[w] = fmaf(fx, g1 - g0, g0);
+                }
+                bbox[o + bx] = bf16_bits(fmaf(fy, vb[1] - vb[0], vb[0]));
+                gbox[o + bx] = bf16_bits(fmaf(fy, vg[1] - vg[0], vg[0]));
               }
             }
+            __syncwarp();
           }
-          // this box row becomes the previous one
-#pragma unroll
-          for (int b = 0; b < 4; b++)
-#pragma unroll
-            for (int jt = 0; jt < 4; jt++)
-#pragma unroll
-              for (int e = 0; e < 4; e++) prev[(b * 16 + jt * 4 + e) * 32 + lane] = cur[b][jt][e];
-          __syncwarp();
         }
         // box row kh takes only the y-carry of tap row kh-1
-#pragma unroll
-        for (int hf = 0; hf < 2; hf++) {
-          const float fy = R[hf].f[1];
-          float be[4], bo[4], gme[4], gmo[4];
-#pragma unroll
-          for (int jt = 0; jt < 4; jt++) {
-            const float* bp = bxp + (jt * 4 + 2 * hf) * 32 + lane;
-            be[jt] = fy * bp[0];
-            bo[jt] = fy * bp[32];
-            gme[jt] = fy * bp[16 * 32];
-            gmo[jt] = fy * bp[16 * 32 + 32];
-          }
-          if (R[hf].live) {
-            const int64_t o = ((int64_t)(pos + gq + 8 * hf) * bg.rows + u * (g.kh + 1) + g.kh) * bg.width;
-            store_box_row(bbox + o, be, bo, R[hf].ox, bg.width, qq);
-            store_box_row(gbox + o, gme, gmo, R[hf].ox, bg.width, qq);
+        {
+          const float* tq = tapb + ((g.kh - 1) & 1) * 2 * 16 * kTapStride;
+          if (elive) {
+            const int64_t o = ((int64_t)(pos + er) * bg.rows + u * (g.kh + 1) + g.kh) * bg.width;
+            for (int bx = side; bx <= g.kw; bx += 2) {
+              const float p0 = (bx < g.kw) ? tq[er * kTapStride + bx] : 0.f;
+              const float p1 = (bx >= 1) ? tq[er * kTapStride + bx - 1] : 0.f;
+              const float g0 = (bx < g.kw) ? tq[(16 + er) * kTapStride + bx] : 0.f;
+              const float g1 = (bx >= 1) ? tq[(16 + er) * kTapStride + bx - 1] : 0.f;
+              bbox[o + bx] = bf16_bits(fy * fmaf(fx, p1 - p0, p0));
+              gbox[o + bx] = bf16_bits(fy * fmaf(fx, g1 - g0, g0));
+            }
           }
         }
         __syncwarp();
       }
 
-      // per-query totals: reduce over the quad, then D, doff, (D, f_t)
+      // per-query totals: combine the two lanes of the row, then D, doff, (D, f_t)
+      Dp += __shfl_xor_sync(kFull, Dp, 1);
+      float res[3];
 #pragma unroll
-      for (int hf = 0; hf < 2; hf++) {
-        float d = Dp[hf];
-        d += __shfl_xor_sync(kFull, d, 1);
-        d += __shfl_xor_sync(kFull, d, 2);
-        float res[3];
-#pragma unroll
-        for (int ax = 0; ax < 3; ax++) {
-          float a = A[hf][ax], b = Bs[hf][ax], c = C[hf][ax];
-          a += __shfl_xor_sync(kFull, a, 1);
-          a += __shfl_xor_sync(kFull, a, 2);
-          b += __shfl_xor_sync(kFull, b, 1);
-          b += __shfl_xor_sync(kFull, b, 2);
-          c += __shfl_xor_sync(kFull, c, 1);
-          c += __shfl_xor_sync(kFull, c, 2);
-          res[ax] = fmaf(g.scale, fmaf(-d, b, a), c);
-        }
-        if (R[hf].live && qq == 0) {
-          float* od = doff + ((int64_t)h * g.N + R[hf].n) * 3;
-          od[0] = res[0];
-          od[1] = res[1];
-          od[2] = res[2];
-          dft[pos + gq + 8 * hf] = make_float2(d, R[hf].f[0]);
-        }
+      for (int ax = 0; ax < 3; ax++) {
+        A[ax] += __shfl_xor_sync(kFull, A[ax], 1);
+        Bs[ax] += __shfl_xor_sync(kFull, Bs[ax], 1);
+        C[ax] += __shfl_xor_sync(kFull, C[ax], 1);
+        res[ax] = fmaf(g.scale, fmaf(-Dp, Bs[ax], A[ax]), C[ax]);
+      }
+      if (elive && side == 0) {
+        float* od = doff + ((int64_t)h * g.N + en) * 3;
+        od[0] = res[0];
+        od[1] = res[1];
+        od[2] = res[2];
+        dft[pos + er] = make_float2(Dp, ft);
       }
       pos += cnt;
     }
