@@ -243,14 +243,13 @@ dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const
   }
   {
     auto kern = dsa3d_fwd_mma_kernel<DH>;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 128, 0) != cudaSuccess)
+    const int smem = 4 * fwd_mma_warp_bytes();
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return DSA3D_ERR_CUDA;
-    if (per_sm < 1) return DSA3D_ERR_UNSUPPORTED;
     const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
     const int grid = grid_for(rows, 4, 1 << 20);  // one row per warp; the scheduler balances rows
     TimedLaunch tl(kKernFwdMma, st);
-    kern<<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+    kern<<<grid, 128, smem, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                static_cast<const __nv_bfloat16*>(v), off,
                                static_cast<__nv_bfloat16*>(out), lse, w.cnt, w.sorted_n, w.sorted_ex, g,
                                sg, h0, hg);

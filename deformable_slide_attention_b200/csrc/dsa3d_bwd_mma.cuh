@@ -30,10 +30,6 @@ struct BoxGeo {
   int per_q;     // rows * width bf16 values per query and array
 };
 
-__device__ __forceinline__ unsigned short bf16_bits(float x) {
-  const __nv_bfloat16 b = __float2bfloat16_rn(x);
-  return *reinterpret_cast<const unsigned short*>(&b);
-}
 __device__ __forceinline__ float bf16_val(unsigned short u) { return __uint_as_float((unsigned)u << 16); }
 
 // One 16 x 32 raw-dot block: acc[jt] (n-tile jt, keys X0 + 8jt + [0,8)) = A . src[t, y, seg]^T,
@@ -326,13 +322,6 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
 }
 
 // ---- shared helpers of passes 2 and 3 ----------------------------------------------------------
-__device__ __forceinline__ void ldsm_x4(unsigned (&r)[4], const void* p) {
-  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(a));
-}
-
 // gamma and beta of one query at box plane bt, box row by, column bx (t-mix of the stored tap
 // planes bt and bt-1; gamma = gamma' - D beta).
 __device__ __forceinline__ void box_value(const unsigned short* gbox, const unsigned short* bbox,

@@ -10,9 +10,11 @@
 //   online softmax (base 2) over the taps, P = exp2(s - m)
 //   value weights of box row ty: beta = y-mix of the x-transposed P of tap rows ty and ty-1
 //   O += [(1-f_t) beta | f_t beta] . [V[u, ty]; V[u+1, ty]]     (MMAs, beta as bf16 A operand)
-// The MMA accumulator layout of S is the A-operand layout of P.V (lanes hold rows g and g+8,
-// column pairs), so the whole per-query epilogue stays in registers; x-neighbours come from the
-// neighbouring lane of the quad.  Only rows of valid queries exist here (the sort drops the rest).
+// The blended raw scores of each box row go to a two-row ring in shared memory; two lanes per
+// query then evaluate only that query's taps (online softmax per query), keep the taps' P in a
+// two-row ring, and write the value weights of the box row as two bf16 tiles (scaled by 1-f_t and
+// f_t), which ldmatrix turns back into A operands of the P.V MMAs.  Only rows of valid queries
+// exist here (the sort drops the rest).
 //
 // Operand layouts.  S = Q.K^T contracts dh: in k-step s, lane quad position q supplies the dims
 // of its slice [q*DH/4, (q+1)*DH/4) at words 2s and 2s+1, for the Q rows (A) and the key rows
@@ -129,6 +131,69 @@ __device__ __forceinline__ void dsa3d_pv_rows(float (&o)[MmaShape<DH>::NT][4], c
   }
 }
 
+__device__ __forceinline__ unsigned short bf16_bits(float x) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(x);
+  return *reinterpret_cast<const unsigned short*>(&b);
+}
+
+__device__ __forceinline__ void ldsm_x4(unsigned (&r)[4], const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+
+// O += tile0 . V[t0, y, seg] + tile1 . V[t0+1, y, seg]: the two bf16 value-weight tiles
+// (16 queries x 32 segment keys, row stride 40) as A operands (ldmatrix), V by byte permutes.
+template <int DH>
+__device__ __forceinline__ void dsa3d_pv_tile(float (&o)[MmaShape<DH>::NT][4], const unsigned short* tile,
+                                              int t0, int y, int X0, int segw, const __nv_bfloat16* vh,
+                                              int64_t rs, const Geo& g, int lane) {
+  using S = MmaShape<DH>;
+  const int gq = lane >> 2, qq = lane & 3;
+  if (y < 0 || y >= g.Hp) return;
+#pragma unroll
+  for (int pl = 0; pl < 2; pl++) {
+    const int t = t0 + pl;
+    if (t < 0 || t >= g.F) continue;
+#pragma unroll
+    for (int kk = 0; kk < 2; kk++) {
+      unsigned a[4];
+      const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4) + 16 * kk;
+      ldsm_x4(a, tile + (pl * 16 + rr) * 40 + cc);
+      unsigned vw[4][S::VW];
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const int key = 16 * kk + 2 * qq + (i & 1) + 8 * (i >> 1);
+        const int x = X0 + key;
+        const bool ok = key < segw && x >= 0 && x < g.Wp;
+        const __nv_bfloat16* vr = vh + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + gq * S::NT;
+#pragma unroll
+        for (int c = 0; c < S::VW / 4; c++) {
+          const uint4 w = ok ? ldg16(vr + c * 8) : make_uint4(0, 0, 0, 0);
+          vw[i][4 * c] = w.x; vw[i][4 * c + 1] = w.y; vw[i][4 * c + 2] = w.z; vw[i][4 * c + 3] = w.w;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < S::NT; j++) {
+        const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
+        const unsigned b0 = __byte_perm(vw[0][j >> 1], vw[1][j >> 1], sel);
+        const unsigned b1 = __byte_perm(vw[2][j >> 1], vw[3][j >> 1], sel);
+        mma_bf16_16816(o[j], a[0], a[1], a[2], a[3], b0, b1);
+      }
+    }
+  }
+}
+
+// Shared memory per warp of the forward: raw-score ring [2][16][kFwdRaw], tap ring
+// [2][16][kFwdTap] (P of tap rows ty, ty-1) and two bf16 value-weight tiles [2][16][kFwdTile].
+constexpr int kFwdRaw = 33;
+constexpr int kFwdTap = 16;
+constexpr int kFwdTile = 40;  // bf16 per row: 32 columns + pad (conflict-free ldmatrix)
+__host__ __device__ constexpr int fwd_mma_warp_bytes() {
+  return (2 * 16 * kFwdRaw + 2 * 16 * kFwdTap) * 4 + 2 * 16 * kFwdTile * 2;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
     dsa3d_fwd_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -138,11 +203,16 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
                          const int* __restrict__ sorted_ex, const Geo g, const SortGeo sg,
                          const int h0, const int hg) {
   using S = MmaShape<DH>;
+  extern __shared__ __align__(16) unsigned char fwd_sh[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, qq = lane & 3;  // fragment row group / quad position
+  float* raw = reinterpret_cast<float*>(fwd_sh + warp * fwd_mma_warp_bytes());
+  float* tapb = raw + 2 * 16 * kFwdRaw;
+  unsigned short* tile = reinterpret_cast<unsigned short*>(tapb + 2 * 16 * kFwdTap);
+  const int er = lane >> 1, side = lane & 1;  // epilogue: query row, tap parity
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
-  const int segw = 16 + g.kw;  // keys of the segment that can carry weight
+  const int segw = 16 + g.kw;
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
 
   for (int64_t row = (int64_t)blockIdx.x * 4 + warp; row < rows; row += (int64_t)gridDim.x * 4) {
@@ -164,32 +234,25 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
       const int cnt = __popc(bal);
       const int X0 = ex0 - g.kw;
 
-      MmaRow R[2];
+      // fragment rows g, g+8: their tokens and f_t (for the Q operand and the t-blend)
+      int fn[2];
+      float fft[2];
+      bool flive[2];
 #pragma unroll
       for (int hf = 0; hf < 2; hf++) {
         const int r = gq + 8 * hf;
-        R[hf].live = r < cnt;
-        R[hf].n = R[hf].live ? sorted_n[pos + r] : 0;
-        const Query Qd = decode_query(g, off, h, R[hf].n);
-        R[hf].ox = Qd.o[2] - X0;
-#pragma unroll
-        for (int a = 0; a < 3; a++) {
-          R[hf].f[a] = Qd.f[a];
-          R[hf].lo[a] = Qd.lo[a];
-          R[hf].hi[a] = R[hf].live ? Qd.hi[a] : -1;  // dead rows: no valid tap
-        }
-        DSA3D_DEVICE_CHECK(!R[hf].live || (Qd.ok && Qd.o[0] == ot && Qd.o[1] == oy && R[hf].ox >= 0 && R[hf].ox < 16));
+        flive[hf] = r < cnt;
+        fn[hf] = flive[hf] ? sorted_n[pos + r] : 0;
+        fft[hf] = flive[hf] ? decode_query(g, off, h, fn[hf]).f[0] : 0.f;
       }
-
-      // ---- Q fragments
       unsigned qa[S::KS][4];
       {
         unsigned w0[S::QW], w1[S::QW];
 #pragma unroll
         for (int c = 0; c < S::QW / 4; c++) {
           uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-          if (R[0].live) a = ldg16(q + ((int64_t)R[0].n * g.heads + h) * DH + qq * (DH / 4) + c * 8);
-          if (R[1].live) b = ldg16(q + ((int64_t)R[1].n * g.heads + h) * DH + qq * (DH / 4) + c * 8);
+          if (flive[0]) a = ldg16(q + ((int64_t)fn[0] * g.heads + h) * DH + qq * (DH / 4) + c * 8);
+          if (flive[1]) b = ldg16(q + ((int64_t)fn[1] * g.heads + h) * DH + qq * (DH / 4) + c * 8);
           w0[4 * c] = a.x; w0[4 * c + 1] = a.y; w0[4 * c + 2] = a.z; w0[4 * c + 3] = a.w;
           w1[4 * c] = b.x; w1[4 * c + 1] = b.y; w1[4 * c + 2] = b.z; w1[4 * c + 3] = b.w;
         }
@@ -201,171 +264,167 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
           qa[s][3] = w1[2 * s + 1];
         }
       }
+      // epilogue row er
+      const bool elive = er < cnt;
+      const int en = elive ? sorted_n[pos + er] : 0;
+      const Query EQ = decode_query(g, off, h, en);
+      DSA3D_DEVICE_CHECK(!elive || (EQ.ok && EQ.o[0] == ot && EQ.o[1] == oy && EQ.o[2] - X0 >= 0 && EQ.o[2] - X0 < 16));
+      const int eox = EQ.o[2] - X0;
+      const float eft = EQ.f[0], efy = EQ.f[1], efx = EQ.f[2];
+      const int hi_t = elive ? EQ.hi[0] : -1;
 
       float o[S::NT][4];
 #pragma unroll
       for (int j = 0; j < S::NT; j++) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      float m = -INFINITY, l = 0.f;  // running max (base 2) and partial sum of row er
 
       for (int u = 0; u < g.kt; u++) {
-        const bool plane_live = (R[0].lo[0] <= u && u <= R[0].hi[0]) || (R[1].lo[0] <= u && u <= R[1].hi[0]);
-        if (!__any_sync(kFull, plane_live)) continue;
-        const float ft[2] = {R[0].f[0], R[1].f[0]};
-        float st_prev[4][4];
-        float bx_prev[4][4];
-#pragma unroll
-        for (int jt = 0; jt < 4; jt++)
-#pragma unroll
-          for (int e = 0; e < 4; e++) st_prev[jt][e] = bx_prev[jt][e] = 0.f;
-
+        const bool eplane = EQ.lo[0] <= u && u <= hi_t;
+        if (!__any_sync(kFull, eplane)) continue;
+        for (int i = lane; i < 2 * 16 * kFwdTap; i += 32) tapb[i] = 0.f;
         for (int by = 0; by <= g.kh; by++) {
-          // --- t-blended raw scores of box row by
-          float st[4][4];
-#pragma unroll
-          for (int jt = 0; jt < 4; jt++) st[jt][0] = st[jt][1] = st[jt][2] = st[jt][3] = 0.f;
           const int y = oy + by;
+          float* rc = raw + (by & 1) * 16 * kFwdRaw;
+          // t-blended raw scores of box row by -> ring
+          {
+            float st[4][4];
 #pragma unroll
-          for (int pl = 0; pl < 2; pl++) {
-            const int t = ot + u + pl;
-            if (t < 0 || t >= g.F || y < 0 || y >= g.Hp) continue;
-            float acc[4][4];
+            for (int jt = 0; jt < 4; jt++) st[jt][0] = st[jt][1] = st[jt][2] = st[jt][3] = 0.f;
 #pragma unroll
-            for (int jt = 0; jt < 4; jt++) {
-              acc[jt][0] = acc[jt][1] = acc[jt][2] = acc[jt][3] = 0.f;
-              const int col = 8 * jt + gq;
-              const int x = X0 + col;
-              unsigned kw_[S::QW];
-              const bool ok = col < segw && x >= 0 && x < g.Wp;
-              const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + qq * (DH / 4);
+            for (int pl = 0; pl < 2; pl++) {
+              const int t = ot + u + pl;
+              if (t < 0 || t >= g.F || y < 0 || y >= g.Hp) continue;
 #pragma unroll
-              for (int c = 0; c < S::QW / 4; c++) {
-                const uint4 a = ok ? ldg16(kr + c * 8) : make_uint4(0, 0, 0, 0);
-                kw_[4 * c] = a.x; kw_[4 * c + 1] = a.y; kw_[4 * c + 2] = a.z; kw_[4 * c + 3] = a.w;
+              for (int jt = 0; jt < 4; jt++) {
+                const int col = 8 * jt + gq;
+                const int x = X0 + col;
+                const bool ok = col < segw && x >= 0 && x < g.Wp;
+                const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + qq * (DH / 4);
+                unsigned kw_[S::QW];
+#pragma unroll
+                for (int c = 0; c < S::QW / 4; c++) {
+                  const uint4 a = ok ? ldg16(kr + c * 8) : make_uint4(0, 0, 0, 0);
+                  kw_[4 * c] = a.x; kw_[4 * c + 1] = a.y; kw_[4 * c + 2] = a.z; kw_[4 * c + 3] = a.w;
+                }
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int s = 0; s < S::KS; s++)
+                  mma_bf16_16816(acc, qa[s][0], qa[s][1], qa[s][2], qa[s][3], kw_[2 * s], kw_[2 * s + 1]);
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                  const float w = pl ? fft[e >> 1] : 1.f - fft[e >> 1];
+                  st[jt][e] = fmaf(w, acc[e], st[jt][e]);
+                }
               }
-#pragma unroll
-              for (int s = 0; s < S::KS; s++)
-                mma_bf16_16816(acc[jt], qa[s][0], qa[s][1], qa[s][2], qa[s][3], kw_[2 * s], kw_[2 * s + 1]);
             }
 #pragma unroll
-            for (int jt = 0; jt < 4; jt++) {
-              const float w0 = pl ? ft[0] : 1.f - ft[0], w1 = pl ? ft[1] : 1.f - ft[1];
-              st[jt][0] = fmaf(w0, acc[jt][0], st[jt][0]);
-              st[jt][1] = fmaf(w0, acc[jt][1], st[jt][1]);
-              st[jt][2] = fmaf(w1, acc[jt][2], st[jt][2]);
-              st[jt][3] = fmaf(w1, acc[jt][3], st[jt][3]);
-            }
+            for (int jt = 0; jt < 4; jt++)
+#pragma unroll
+              for (int e = 0; e < 4; e++)
+                rc[(gq + 8 * (e >> 1)) * kFwdRaw + 8 * jt + 2 * qq + (e & 1)] = st[jt][e];
           }
-
+          __syncwarp();
           if (by >= 1) {
             const int ty = by - 1;
-            // --- tap scores of tap row ty: y-lerp then x-lerp
-            float sy_e[2][4], sy_o[2][4];
+            const float* rp = raw + ((by - 1) & 1) * 16 * kFwdRaw;
+            float* tp = tapb + (ty & 1) * 16 * kFwdTap;
+            float* tq = tapb + ((ty + 1) & 1) * 16 * kFwdTap;  // tap row ty-1
+            const bool erow = eplane && EQ.lo[1] <= ty && ty <= EQ.hi[1];
+            // scores of this lane's taps, row max
+            float sv[8];
+            float mx = -INFINITY;
 #pragma unroll
-            for (int hf = 0; hf < 2; hf++) {
-              const float fy = R[hf].f[1];
-#pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-                sy_e[hf][jt] = fmaf(fy, st[jt][2 * hf] - st_prev[jt][2 * hf], st_prev[jt][2 * hf]);
-                sy_o[hf][jt] = fmaf(fy, st[jt][2 * hf + 1] - st_prev[jt][2 * hf + 1], st_prev[jt][2 * hf + 1]);
+            for (int i = 0; i < 8; i++) {
+              const int wx = side + 2 * i;
+              sv[i] = -INFINITY;
+              if (wx < g.kw && erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
+                const int c = eox + wx;
+                const float p0 = rp[er * kFwdRaw + c], p1 = rp[er * kFwdRaw + c + 1];
+                const float c0 = rc[er * kFwdRaw + c], c1 = rc[er * kFwdRaw + c + 1];
+                const float y0 = fmaf(efy, c0 - p0, p0), y1 = fmaf(efy, c1 - p1, p1);
+                sv[i] = fmaf(efx, y1 - y0, y0) * sc;
+                mx = fmaxf(mx, sv[i]);
               }
             }
-            float p_e[2][4], p_o[2][4];
-            float alpha[2];
-#pragma unroll
-            for (int hf = 0; hf < 2; hf++) {
-              float nx_e[4], nx_o[4];
-              col_next(sy_e[hf], sy_o[hf], qq, lane, nx_e, nx_o);
-              const float fx = R[hf].f[2];
-              const bool row_ok = R[hf].lo[0] <= u && u <= R[hf].hi[0] && R[hf].lo[1] <= ty && ty <= R[hf].hi[1];
-              float mx = -INFINITY;
-#pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-                const int wx0 = 8 * jt + 2 * qq - R[hf].ox;
-                const bool v0 = row_ok && wx0 >= R[hf].lo[2] && wx0 <= R[hf].hi[2];
-                const bool v1 = row_ok && wx0 + 1 >= R[hf].lo[2] && wx0 + 1 <= R[hf].hi[2];
-                const float s0 = fmaf(fx, nx_e[jt] - sy_e[hf][jt], sy_e[hf][jt]) * sc;
-                const float s1 = fmaf(fx, nx_o[jt] - sy_o[hf][jt], sy_o[hf][jt]) * sc;
-                p_e[hf][jt] = v0 ? s0 : -INFINITY;
-                p_o[hf][jt] = v1 ? s1 : -INFINITY;
-                mx = fmaxf(mx, fmaxf(p_e[hf][jt], p_o[hf][jt]));
-              }
-              mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-              mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-              alpha[hf] = 1.f;
-              if (mx != -INFINITY) {
-                const float mn = fmaxf(m[hf], mx);
-                alpha[hf] = exp2f(m[hf] - mn);  // 0 when m was -inf
-                m[hf] = mn;
-              }
-              float ls = 0.f;
-#pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-                p_e[hf][jt] = (p_e[hf][jt] == -INFINITY) ? 0.f : exp2f(p_e[hf][jt] - m[hf]);
-                p_o[hf][jt] = (p_o[hf][jt] == -INFINITY) ? 0.f : exp2f(p_o[hf][jt] - m[hf]);
-                ls += p_e[hf][jt] + p_o[hf][jt];
-              }
-              l[hf] = fmaf(l[hf], alpha[hf], ls);
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            float alpha = 1.f;
+            if (mx > m) {
+              alpha = exp2f(m - mx);  // 0 when m was -inf
+              m = mx;
             }
-            if (__any_sync(kFull, alpha[0] != 1.f || alpha[1] != 1.f)) {
+            float ls = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+              const int wx = side + 2 * i;
+              if (wx < g.kw) {
+                const float p = (sv[i] == -INFINITY) ? 0.f : exp2f(sv[i] - m);
+                tp[er * kFwdTap + wx] = p;
+                ls += p;
+                if (alpha != 1.f) tq[er * kFwdTap + wx] *= alpha;  // rescale tap row ty-1
+              }
+            }
+            l = fmaf(l, alpha, ls);
+            // O rows g, g+8 rescale (alpha of row r is held by lanes 2r, 2r+1)
+            const float a0 = __shfl_sync(kFull, alpha, 2 * gq), a1 = __shfl_sync(kFull, alpha, 2 * (gq + 8));
+            if (__any_sync(kFull, a0 != 1.f || a1 != 1.f)) {
 #pragma unroll
               for (int j = 0; j < S::NT; j++) {
-                o[j][0] *= alpha[0]; o[j][1] *= alpha[0];
-                o[j][2] *= alpha[1]; o[j][3] *= alpha[1];
-              }
-#pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-                bx_prev[jt][0] *= alpha[0]; bx_prev[jt][1] *= alpha[0];
-                bx_prev[jt][2] *= alpha[1]; bx_prev[jt][3] *= alpha[1];
+                o[j][0] *= a0; o[j][1] *= a0;
+                o[j][2] *= a1; o[j][3] *= a1;
               }
             }
-            // --- value weights: x-transpose of P (this tap row), y-mix with the previous one
-            float beta[4][4];
-#pragma unroll
-            for (int hf = 0; hf < 2; hf++) {
-              float pv_e[4], pv_o[4];
-              col_prev(p_e[hf], p_o[hf], qq, lane, pv_e, pv_o);
-              const float fx = R[hf].f[2], fy = R[hf].f[1];
-#pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-                const float bxe = fmaf(fx, pv_e[jt] - p_e[hf][jt], p_e[hf][jt]);
-                const float bxo = fmaf(fx, pv_o[jt] - p_o[hf][jt], p_o[hf][jt]);
-                beta[jt][2 * hf] = fmaf(fy, bx_prev[jt][2 * hf] - bxe, bxe);
-                beta[jt][2 * hf + 1] = fmaf(fy, bx_prev[jt][2 * hf + 1] - bxo, bxo);
-                bx_prev[jt][2 * hf] = bxe;
-                bx_prev[jt][2 * hf + 1] = bxo;
+            __syncwarp();
+            // value weights of box row ty, scaled for box planes u (1-f_t) and u+1 (f_t)
+            for (int i = lane; i < 2 * 16 * kFwdTile / 8; i += 32)
+              reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
+            __syncwarp();
+            if (elive) {
+              for (int bx = side; bx <= g.kw; bx += 2) {
+                const float q0 = (bx < g.kw) ? tp[er * kFwdTap + bx] : 0.f;
+                const float q1 = (bx >= 1) ? tp[er * kFwdTap + bx - 1] : 0.f;
+                const float r0 = (bx < g.kw) ? tq[er * kFwdTap + bx] : 0.f;
+                const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
+                const float bxc = fmaf(efx, q1 - q0, q0), bxp = fmaf(efx, r1 - r0, r0);
+                const float beta = fmaf(efy, bxp - bxc, bxc);
+                tile[er * kFwdTile + eox + bx] = bf16_bits((1.f - eft) * beta);
+                tile[(16 + er) * kFwdTile + eox + bx] = bf16_bits(eft * beta);
               }
             }
-            // --- O += beta . V over box row ty of planes u, u+1
-            dsa3d_pv_rows<DH>(o, beta, ft, ot + u, oy + ty, X0, segw, vh_, rs, g, gq, qq);
+            __syncwarp();
+            dsa3d_pv_tile<DH>(o, tile, ot + u, oy + ty, X0, segw, vh_, rs, g, lane);
+            __syncwarp();
           }
-#pragma unroll
-          for (int jt = 0; jt < 4; jt++)
-#pragma unroll
-            for (int e = 0; e < 4; e++) st_prev[jt][e] = st[jt][e];
         }
-        // box row kh takes only the y-carry of tap row kh-1
+        // box row kh: only the y-carry (weight f_y) of tap row kh-1
         {
-          float beta[4][4];
-#pragma unroll
-          for (int jt = 0; jt < 4; jt++) {
-            beta[jt][0] = R[0].f[1] * bx_prev[jt][0];
-            beta[jt][1] = R[0].f[1] * bx_prev[jt][1];
-            beta[jt][2] = R[1].f[1] * bx_prev[jt][2];
-            beta[jt][3] = R[1].f[1] * bx_prev[jt][3];
+          const float* tq = tapb + ((g.kh - 1) & 1) * 16 * kFwdTap;
+          for (int i = lane; i < 2 * 16 * kFwdTile / 8; i += 32)
+            reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
+          __syncwarp();
+          if (elive) {
+            for (int bx = side; bx <= g.kw; bx += 2) {
+              const float r0 = (bx < g.kw) ? tq[er * kFwdTap + bx] : 0.f;
+              const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
+              const float beta = efy * fmaf(efx, r1 - r0, r0);
+              tile[er * kFwdTile + eox + bx] = bf16_bits((1.f - eft) * beta);
+              tile[(16 + er) * kFwdTile + eox + bx] = bf16_bits(eft * beta);
+            }
           }
-          dsa3d_pv_rows<DH>(o, beta, ft, ot + u, oy + g.kh, X0, segw, vh_, rs, g, gq, qq);
+          __syncwarp();
+          dsa3d_pv_tile<DH>(o, tile, ot + u, oy + g.kh, X0, segw, vh_, rs, g, lane);
+          __syncwarp();
         }
       }
 
-      // ---- normalise and store
+      // ---- normalise and store (row sums from the epilogue lanes)
+      const float lt_e = l + __shfl_xor_sync(kFull, l, 1);
+      if (elive && side == 0 && lse) lse[(int64_t)h * g.N + en] = (m + log2f(lt_e)) * kLn2;
 #pragma unroll
       for (int hf = 0; hf < 2; hf++) {
-        float lt = l[hf];
-        lt += __shfl_xor_sync(kFull, lt, 1);
-        lt += __shfl_xor_sync(kFull, lt, 2);
-        if (!R[hf].live) continue;
+        const float lt = __shfl_sync(kFull, lt_e, 2 * (gq + 8 * hf));
+        if (!flive[hf]) continue;
         const float inv = 1.f / lt;
-        __nv_bfloat16* orow = out + ((int64_t)R[hf].n * g.heads + h) * DH + qq * (DH / 4);
+        __nv_bfloat16* orow = out + ((int64_t)fn[hf] * g.heads + h) * DH + qq * (DH / 4);
         float vals[S::NT * 2];
 #pragma unroll
         for (int j = 0; j < S::NT; j++) {
@@ -374,7 +433,6 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
         }
 #pragma unroll
         for (int c = 0; c < S::NT * 2 / 8; c++) store16(orow + c * 8, vals + c * 8);
-        if (qq == 0 && lse) lse[(int64_t)h * g.N + R[hf].n] = (m[hf] + log2f(lt)) * kLn2;
       }
       pos += cnt;
     }
