@@ -343,6 +343,37 @@ __device__ __forceinline__ void box_value(const unsigned short* gbox, const unsi
   }
 }
 
+// gamma and beta of one query at box plane bt, box row by, columns 2w and 2w+1 (one 32-bit word
+// of each stored row; rows hold an even number of bf16 values, so words are 4-byte aligned).
+__device__ __forceinline__ void box_word(const unsigned short* gbox, const unsigned short* bbox,
+                                         int64_t pos, const BoxGeo& bg, int kt, int kh, int bt,
+                                         int by, int w, float D, float ft, float (&gam)[2],
+                                         float (&bet)[2]) {
+  gam[0] = gam[1] = bet[0] = bet[1] = 0.f;
+  if (bt < kt) {
+    const int64_t o = (pos * bg.rows + bt * (kh + 1) + by) * bg.width + 2 * w;
+    const unsigned bw = *reinterpret_cast<const unsigned*>(bbox + o);
+    const unsigned gw = *reinterpret_cast<const unsigned*>(gbox + o);
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+      const float b = bf16_val((unsigned short)(bw >> (16 * e))), gp = bf16_val((unsigned short)(gw >> (16 * e)));
+      bet[e] = (1.f - ft) * b;
+      gam[e] = (1.f - ft) * fmaf(-D, b, gp);
+    }
+  }
+  if (bt >= 1) {
+    const int64_t o = (pos * bg.rows + (bt - 1) * (kh + 1) + by) * bg.width + 2 * w;
+    const unsigned bw = *reinterpret_cast<const unsigned*>(bbox + o);
+    const unsigned gw = *reinterpret_cast<const unsigned*>(gbox + o);
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+      const float b = bf16_val((unsigned short)(bw >> (16 * e))), gp = bf16_val((unsigned short)(gw >> (16 * e)));
+      bet[e] = fmaf(ft, b, bet[e]);
+      gam[e] = fmaf(ft, fmaf(-D, b, gp), gam[e]);
+    }
+  }
+}
+
 // ---- pass 2: dq = scale * sum_j gamma[j] K[j] ----------------------------------------------------
 template <int DH>
 __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
@@ -387,14 +418,18 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
           // gamma tile: rows = queries, cols = segment keys
           for (int i = lane; i < 16 * TS / 8; i += 32) reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
           __syncwarp();
-          for (int idx = lane; idx < 16 * bg.width; idx += 32) {
-            const int r = idx / bg.width, bx = idx - r * bg.width;
-            if (r >= cnt) continue;
-            const float2 d = dft[pos + r];
-            float ga, be;
-            box_value(gbox, bbox, pos + r, bg, g.kt, g.kh, bt, by, bx, d.x, d.y, ga, be);
-            const int col = sorted_ex[pos + r] - g.kw - X0 + bx;
-            tile[r * TS + col] = bf16_bits(ga);
+          {
+            const int r = lane >> 1;
+            if (r < cnt) {
+              const float2 d = dft[pos + r];
+              const int col0 = sorted_ex[pos + r] - g.kw - X0;
+              for (int w = lane & 1; 2 * w < bg.width; w += 2) {
+                float ga[2], be[2];
+                box_word(gbox, bbox, pos + r, bg, g.kt, g.kh, bt, by, w, d.x, d.y, ga, be);
+                tile[r * TS + col0 + 2 * w] = bf16_bits(ga[0]);
+                tile[r * TS + col0 + 2 * w + 1] = bf16_bits(ga[1]);
+              }
+            }
           }
           __syncwarp();
 #pragma unroll
@@ -534,23 +569,30 @@ __global__ void __launch_bounds__(256, DSA3D_KV_MINB)
             *reinterpret_cast<uint4*>((which ? os : qs) + m * RS + c * 8) = val;
           }
           // gather Gamma^T / Beta^T tiles of the 4 key rows: (query m, key row kr, column bx)
-          const int by_base = kKvRows - 1;  // by = yk0 + kr - ey + kh
-          for (int i = tid; i < 16 * kKvRows * bg.width; i += 256) {
-            const int m = i / (kKvRows * bg.width);
-            const int rem = i - m * (kKvRows * bg.width);
-            const int kr = rem / bg.width, bx = rem - kr * bg.width;
-            if (m >= cnt) continue;
-            const int by = yk0 + kr - ey + g.kh;
-            if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
-            const int key = m_ox[m] + bx;
-            if (key < 0 || key >= 16) continue;
-            const float2 d = m_dft[m];
-            float ga, be;
-            box_value(gbox, bbox, pos + m, bg, g.kt, g.kh, bt, by, bx, d.x, d.y, ga, be);
-            tg[kr][key * TS + m] = bf16_bits(ga);
-            tb[kr][key * TS + m] = bf16_bits(be);
+          {
+            const int m = tid >> 4, w = tid & 15;
+            if (m < cnt && 2 * w < bg.width) {
+              const float2 d = m_dft[m];
+              const int key0 = m_ox[m] + 2 * w;
+              if (key0 + 1 >= 0 && key0 < 16) {
+#pragma unroll
+                for (int kr = 0; kr < kKvRows; kr++) {
+                  const int by = yk0 + kr - ey + g.kh;
+                  if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
+                  float ga[2], be[2];
+                  box_word(gbox, bbox, pos + m, bg, g.kt, g.kh, bt, by, w, d.x, d.y, ga, be);
+#pragma unroll
+                  for (int e = 0; e < 2; e++) {
+                    const int key = key0 + e;
+                    if (key >= 0 && key < 16) {
+                      tg[kr][key * TS + m] = bf16_bits(ga[e]);
+                      tb[kr][key * TS + m] = bf16_bits(be[e]);
+                    }
+                  }
+                }
+              }
+            }
           }
-          (void)by_base;
           __syncthreads();
           const int by_w = myk - ey + g.kh;
           if (myk < g.Hp && by_w >= 0 && by_w <= g.kh) {
