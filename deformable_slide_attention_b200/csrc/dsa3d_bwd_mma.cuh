@@ -47,11 +47,11 @@ __device__ __forceinline__ void raw_block(float (&acc)[4][4], const unsigned (&a
     const int col = 8 * jt + gq;
     const int x = X0 + col;
     const bool ok = col < segw && x >= 0 && x < g.Wp;
-    const __nv_bfloat16* r = src_h + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + qq * (DH / 4);
+    const __nv_bfloat16* r = src_h + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
     unsigned w[S::QW];
 #pragma unroll
     for (int c = 0; c < S::QW / 4; c++) {
-      const uint4 a = ok ? ldg16(r + c * 8) : make_uint4(0, 0, 0, 0);
+      const uint4 a = ok ? ldg16(r + qk_off(c, qq)) : make_uint4(0, 0, 0, 0);
       w[4 * c] = a.x; w[4 * c + 1] = a.y; w[4 * c + 2] = a.z; w[4 * c + 3] = a.w;
     }
 #pragma unroll
@@ -68,8 +68,8 @@ __device__ __forceinline__ void load_afrags(unsigned (&af)[MmaShape<DH>::KS][4],
 #pragma unroll
   for (int c = 0; c < S::QW / 4; c++) {
     uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-    if (R[0].live) a = ldg16(base + ((int64_t)R[0].n * heads + h) * DH + qq * (DH / 4) + c * 8);
-    if (R[1].live) b = ldg16(base + ((int64_t)R[1].n * heads + h) * DH + qq * (DH / 4) + c * 8);
+    if (R[0].live) a = ldg16(base + ((int64_t)R[0].n * heads + h) * DH + qk_off(c, qq));
+    if (R[1].live) b = ldg16(base + ((int64_t)R[1].n * heads + h) * DH + qk_off(c, qq));
     w0[4 * c] = a.x; w0[4 * c + 1] = a.y; w0[4 * c + 2] = a.z; w0[4 * c + 3] = a.w;
     w1[4 * c] = b.x; w1[4 * c + 1] = b.y; w1[4 * c + 2] = b.z; w1[4 * c + 3] = b.w;
   }
@@ -108,17 +108,6 @@ __device__ __forceinline__ int chunk_len(const int* sorted_ex, int pos, int qend
   const unsigned bal = __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 < 16);
   X0 = ex0 - kw;
   return __popc(bal);
-}
-
-// Store one box row of a row-half: values v_e/v_o at columns 8jt+2q(+1) -> box x = col - ox.
-__device__ __forceinline__ void store_box_row(unsigned short* dst, const float (&ve)[4], const float (&vo)[4],
-                                              int ox, int width, int qq) {
-#pragma unroll
-  for (int jt = 0; jt < 4; jt++) {
-    const int x0 = 8 * jt + 2 * qq - ox;
-    if (x0 >= 0 && x0 < width) dst[x0] = bf16_bits(ve[jt]);
-    if (x0 + 1 >= 0 && x0 + 1 < width) dst[x0 + 1] = bf16_bits(vo[jt]);
-  }
 }
 
 // ---- pass 1: query side ---------------------------------------------------------------------
@@ -322,27 +311,6 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
 }
 
 // ---- shared helpers of passes 2 and 3 ----------------------------------------------------------
-// gamma and beta of one query at box plane bt, box row by, column bx (t-mix of the stored tap
-// planes bt and bt-1; gamma = gamma' - D beta).
-__device__ __forceinline__ void box_value(const unsigned short* gbox, const unsigned short* bbox,
-                                          int64_t pos, const BoxGeo& bg, int kt, int kh, int bt,
-                                          int by, int bx, float D, float ft, float& gam, float& bet) {
-  gam = 0.f;
-  bet = 0.f;
-  if (bt < kt) {
-    const int64_t o = (pos * bg.rows + bt * (kh + 1) + by) * bg.width + bx;
-    const float b = bf16_val(bbox[o]), gp = bf16_val(gbox[o]);
-    bet = (1.f - ft) * b;
-    gam = (1.f - ft) * fmaf(-D, b, gp);
-  }
-  if (bt >= 1) {
-    const int64_t o = (pos * bg.rows + (bt - 1) * (kh + 1) + by) * bg.width + bx;
-    const float b = bf16_val(bbox[o]), gp = bf16_val(gbox[o]);
-    bet = fmaf(ft, b, bet);
-    gam = fmaf(ft, fmaf(-D, b, gp), gam);
-  }
-}
-
 // gamma and beta of one query at box plane bt, box row by, columns 2w and 2w+1 (one 32-bit word
 // of each stored row; rows hold an even number of bf16 values, so words are 4-byte aligned).
 __device__ __forceinline__ void box_word(const unsigned short* gbox, const unsigned short* bbox,
@@ -443,18 +411,19 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
               const int key = 16 * kk + 2 * qq + (i & 1) + 8 * (i >> 1);
               const int x = X0 + key;
               const bool ok = key < segw && x >= 0 && x < g.Wp;
-              const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + gq * S::NT;
+              const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
 #pragma unroll
               for (int c = 0; c < S::VW / 4; c++) {
-                const uint4 w = ok ? ldg16(kr + c * 8) : make_uint4(0, 0, 0, 0);
+                const uint4 w = ok ? ldg16(kr + pv_off(c, gq)) : make_uint4(0, 0, 0, 0);
                 vw[i][4 * c] = w.x; vw[i][4 * c + 1] = w.y; vw[i][4 * c + 2] = w.z; vw[i][4 * c + 3] = w.w;
               }
             }
 #pragma unroll
             for (int j = 0; j < S::NT; j++) {
+              const int wi = 4 * (j >> 3) + ((j & 7) >> 1);
               const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
-              const unsigned b0_ = __byte_perm(vw[0][j >> 1], vw[1][j >> 1], sel);
-              const unsigned b1_ = __byte_perm(vw[2][j >> 1], vw[3][j >> 1], sel);
+              const unsigned b0_ = __byte_perm(vw[0][wi], vw[1][wi], sel);
+              const unsigned b1_ = __byte_perm(vw[2][wi], vw[3][wi], sel);
               mma_bf16_16816(acc[j], a[0], a[1], a[2], a[3], b0_, b1_);
             }
           }
@@ -466,15 +435,18 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
         const int r = gq + 8 * hf;
         if (r >= cnt) continue;
         const int n = sorted_n[pos + r];
-        __nv_bfloat16* drow = dq + ((int64_t)n * g.heads + h) * DH + qq * (DH / 4);
-        float vals[S::NT * 2];
+        __nv_bfloat16* drow = dq + ((int64_t)n * g.heads + h) * DH;
 #pragma unroll
-        for (int j = 0; j < S::NT; j++) {
-          vals[j] = acc[j][2 * hf] * g.scale;
-          vals[S::NT + j] = acc[j][2 * hf + 1] * g.scale;
+        for (int c = 0; c < DH / 64; c++) {
+          float vals[16];
+#pragma unroll
+          for (int e = 0; e < 8; e++) {
+            vals[e] = acc[8 * c + e][2 * hf] * g.scale;
+            vals[8 + e] = acc[8 * c + e][2 * hf + 1] * g.scale;
+          }
+          store16(drow + 64 * c + 16 * qq, vals);
+          store16(drow + 64 * c + 16 * qq + 8, vals + 8);
         }
-#pragma unroll
-        for (int c = 0; c < S::NT * 2 / 8; c++) store16(drow + c * 8, vals + c * 8);
       }
       pos += cnt;
     }

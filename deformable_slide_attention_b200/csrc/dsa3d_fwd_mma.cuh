@@ -16,11 +16,11 @@
 // f_t), which ldmatrix turns back into A operands of the P.V MMAs.  Only rows of valid queries
 // exist here (the sort drops the rest).
 //
-// Operand layouts.  S = Q.K^T contracts dh: in k-step s, lane quad position q supplies the dims
-// of its slice [q*DH/4, (q+1)*DH/4) at words 2s and 2s+1, for the Q rows (A) and the key rows
-// (B) alike, so every lane reads contiguous 16-byte chunks.  O = P.V maps output column n of
-// n-tile j to dim n*NT + j, so lane g reads the contiguous dims [g*NT, (g+1)*NT) of each value
-// row and lane (g, q) ends up owning the contiguous output dims [2q*NT, 2q*NT + 2*NT).
+// Operand layouts.  S = Q.K^T contracts dh: in k-step s, lane quad position q supplies words 2s
+// and 2s+1 of its dim slice (qk_off), for the Q rows (A) and the key rows (B) alike -- any fixed
+// permutation of dh applied to both operands leaves the dot products unchanged.  O = P.V maps
+// output column n of n-tile j = 8c + e to dim 64c + 8n + e (pv_off), so lane g reads 16-byte
+// chunks of each value row and lane (g, q) owns output dims 64c + 16q + [0, 16).
 #pragma once
 
 #include "dsa3d_common.cuh"
@@ -35,11 +35,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], unsigned a0, unsig
       "{%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
-  const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const unsigned*>(&b);
 }
 
 __device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
@@ -61,75 +56,13 @@ struct MmaShape {
   static constexpr int VW = NT / 2;    // 32-bit words in a lane's dim slice of a V row
 };
 
-// x-neighbour helpers over the 4 n-tiles of one row-half (values v[jt][e], e = 0 even, 1 odd col).
-// next[c] = v[c + 1]; prev[c] = v[c - 1] (0 outside the segment).
-__device__ __forceinline__ void col_next(const float (&ev)[4], const float (&od)[4], int q, int lane,
-                                         float (&nx_ev)[4], float (&nx_od)[4]) {
-  const int src = (lane & ~3) | ((q + 1) & 3);
-#pragma unroll
-  for (int jt = 0; jt < 4; jt++) {
-    const float send = (q == 0) ? ((jt + 1 < 4) ? ev[jt + 1] : 0.f) : ev[jt];
-    const float r = __shfl_sync(kFull, send, src);
-    nx_ev[jt] = od[jt];  // col 2q -> 2q+1 in the same lane
-    nx_od[jt] = r;       // col 2q+1 -> 2q+2 (lane q+1, or next n-tile's q = 0)
-  }
-}
-__device__ __forceinline__ void col_prev(const float (&ev)[4], const float (&od)[4], int q, int lane,
-                                         float (&pv_ev)[4], float (&pv_od)[4]) {
-  const int src = (lane & ~3) | ((q + 3) & 3);
-#pragma unroll
-  for (int jt = 0; jt < 4; jt++) {
-    // receiver q = 0 wants lane 3's odd value of n-tile jt-1; receivers q > 0 want lane q-1's of jt
-    const float send = (q == 3) ? ((jt > 0) ? od[jt - 1] : 0.f) : od[jt];
-    pv_ev[jt] = __shfl_sync(kFull, send, src);
-    pv_od[jt] = ev[jt];  // col 2q+1 -> 2q in the same lane
-  }
-}
-
-// O += [(1-f_t) beta | f_t beta] . [V[t0, y, seg]; V[t0+1, y, seg]] for the 32-key segment at X0.
-// beta is in accumulator layout (n-tile jt: row g cols 8jt+2q, 8jt+2q+1 in [0],[1]; row g+8 in
-// [2],[3]), which is the A-operand layout of k-step kk = n-tiles 2kk, 2kk+1.
-template <int DH>
-__device__ __forceinline__ void dsa3d_pv_rows(float (&o)[MmaShape<DH>::NT][4], const float (&beta)[4][4],
-                                              const float (&ft)[2], int t0, int y, int X0, int segw,
-                                              const __nv_bfloat16* vh, int64_t rs, const Geo& g,
-                                              int gq, int qq) {
-  using S = MmaShape<DH>;
-  if (y < 0 || y >= g.Hp) return;
-#pragma unroll
-  for (int pl = 0; pl < 2; pl++) {
-    const int t = t0 + pl;
-    if (t < 0 || t >= g.F) continue;
-    const float w0 = pl ? ft[0] : 1.f - ft[0], w1 = pl ? ft[1] : 1.f - ft[1];
-#pragma unroll
-    for (int kk = 0; kk < 2; kk++) {
-      const unsigned a0 = pack_bf16(w0 * beta[2 * kk][0], w0 * beta[2 * kk][1]);
-      const unsigned a1 = pack_bf16(w1 * beta[2 * kk][2], w1 * beta[2 * kk][3]);
-      const unsigned a2 = pack_bf16(w0 * beta[2 * kk + 1][0], w0 * beta[2 * kk + 1][1]);
-      const unsigned a3 = pack_bf16(w1 * beta[2 * kk + 1][2], w1 * beta[2 * kk + 1][3]);
-      unsigned vw[4][S::VW];
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const int key = 16 * kk + 2 * qq + (i & 1) + 8 * (i >> 1);
-        const int x = X0 + key;
-        const bool ok = key < segw && x >= 0 && x < g.Wp;
-        const __nv_bfloat16* vr = vh + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + gq * S::NT;
-#pragma unroll
-        for (int c = 0; c < S::VW / 4; c++) {
-          const uint4 a = ok ? ldg16(vr + c * 8) : make_uint4(0, 0, 0, 0);
-          vw[i][4 * c] = a.x; vw[i][4 * c + 1] = a.y; vw[i][4 * c + 2] = a.z; vw[i][4 * c + 3] = a.w;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < S::NT; j++) {
-        const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
-        const unsigned b0 = __byte_perm(vw[0][j >> 1], vw[1][j >> 1], sel);
-        const unsigned b1 = __byte_perm(vw[2][j >> 1], vw[3][j >> 1], sel);
-        mma_bf16_16816(o[j], a0, a1, a2, a3, b0, b1);
-      }
-    }
-  }
-}
+// Dim slices, chosen so that one 16-byte load instruction of a warp touches as few cache lines
+// as possible.  Q.K^T operands: quad position q holds dims {32c + 8q + [0, 8)}, c < DH/32 (the
+// four q lanes of a key read one contiguous 64-byte span per instruction).  P.V operands and
+// outputs: lane group g holds dims {64c + 8g + [0, 8)}, c < DH/64 (eight g lanes read one
+// 128-byte line per instruction); n-tile j = 8c + e, column n maps to dim 64c + 8n + e.
+__device__ __forceinline__ int qk_off(int c, int qq) { return 32 * c + 8 * qq; }
+__device__ __forceinline__ int pv_off(int c, int gq) { return 64 * c + 8 * gq; }
 
 __device__ __forceinline__ unsigned short bf16_bits(float x) {
   const __nv_bfloat16 b = __float2bfloat16_rn(x);
@@ -167,18 +100,20 @@ __device__ __forceinline__ void dsa3d_pv_tile(float (&o)[MmaShape<DH>::NT][4], c
         const int key = 16 * kk + 2 * qq + (i & 1) + 8 * (i >> 1);
         const int x = X0 + key;
         const bool ok = key < segw && x >= 0 && x < g.Wp;
-        const __nv_bfloat16* vr = vh + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + gq * S::NT;
+        const __nv_bfloat16* vr = vh + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
 #pragma unroll
         for (int c = 0; c < S::VW / 4; c++) {
-          const uint4 w = ok ? ldg16(vr + c * 8) : make_uint4(0, 0, 0, 0);
+          const uint4 w = ok ? ldg16(vr + pv_off(c, gq)) : make_uint4(0, 0, 0, 0);
           vw[i][4 * c] = w.x; vw[i][4 * c + 1] = w.y; vw[i][4 * c + 2] = w.z; vw[i][4 * c + 3] = w.w;
         }
       }
 #pragma unroll
       for (int j = 0; j < S::NT; j++) {
+        // n-tile j = 8c + e: element e of chunk c is word 4c + e/2, half e & 1
+        const int wi = 4 * (j >> 3) + ((j & 7) >> 1);
         const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
-        const unsigned b0 = __byte_perm(vw[0][j >> 1], vw[1][j >> 1], sel);
-        const unsigned b1 = __byte_perm(vw[2][j >> 1], vw[3][j >> 1], sel);
+        const unsigned b0 = __byte_perm(vw[0][wi], vw[1][wi], sel);
+        const unsigned b1 = __byte_perm(vw[2][wi], vw[3][wi], sel);
         mma_bf16_16816(o[j], a[0], a[1], a[2], a[3], b0, b1);
       }
     }
@@ -251,8 +186,8 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
 #pragma unroll
         for (int c = 0; c < S::QW / 4; c++) {
           uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-          if (flive[0]) a = ldg16(q + ((int64_t)fn[0] * g.heads + h) * DH + qq * (DH / 4) + c * 8);
-          if (flive[1]) b = ldg16(q + ((int64_t)fn[1] * g.heads + h) * DH + qq * (DH / 4) + c * 8);
+          if (flive[0]) a = ldg16(q + ((int64_t)fn[0] * g.heads + h) * DH + qk_off(c, qq));
+          if (flive[1]) b = ldg16(q + ((int64_t)fn[1] * g.heads + h) * DH + qk_off(c, qq));
           w0[4 * c] = a.x; w0[4 * c + 1] = a.y; w0[4 * c + 2] = a.z; w0[4 * c + 3] = a.w;
           w1[4 * c] = b.x; w1[4 * c + 1] = b.y; w1[4 * c + 2] = b.z; w1[4 * c + 3] = b.w;
         }
@@ -299,11 +234,11 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
                 const int col = 8 * jt + gq;
                 const int x = X0 + col;
                 const bool ok = col < segw && x >= 0 && x < g.Wp;
-                const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs + qq * (DH / 4);
+                const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
                 unsigned kw_[S::QW];
 #pragma unroll
                 for (int c = 0; c < S::QW / 4; c++) {
-                  const uint4 a = ok ? ldg16(kr + c * 8) : make_uint4(0, 0, 0, 0);
+                  const uint4 a = ok ? ldg16(kr + qk_off(c, qq)) : make_uint4(0, 0, 0, 0);
                   kw_[4 * c] = a.x; kw_[4 * c + 1] = a.y; kw_[4 * c + 2] = a.z; kw_[4 * c + 3] = a.w;
                 }
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -424,15 +359,18 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
         const float lt = __shfl_sync(kFull, lt_e, 2 * (gq + 8 * hf));
         if (!flive[hf]) continue;
         const float inv = 1.f / lt;
-        __nv_bfloat16* orow = out + ((int64_t)fn[hf] * g.heads + h) * DH + qq * (DH / 4);
-        float vals[S::NT * 2];
+        __nv_bfloat16* orow = out + ((int64_t)fn[hf] * g.heads + h) * DH;
 #pragma unroll
-        for (int j = 0; j < S::NT; j++) {
-          vals[j] = o[j][2 * hf] * inv;
-          vals[S::NT + j] = o[j][2 * hf + 1] * inv;
+        for (int c = 0; c < DH / 64; c++) {
+          float vals[16];  // dims 64c + 16q + [0, 16): columns 2q then 2q+1 of n-tiles 8c..8c+7
+#pragma unroll
+          for (int e = 0; e < 8; e++) {
+            vals[e] = o[8 * c + e][2 * hf] * inv;
+            vals[8 + e] = o[8 * c + e][2 * hf + 1] * inv;
+          }
+          store16(orow + 64 * c + 16 * qq, vals);
+          store16(orow + 64 * c + 16 * qq + 8, vals + 8);
         }
-#pragma unroll
-        for (int c = 0; c < S::NT * 2 / 8; c++) store16(orow + c * 8, vals + c * 8);
       }
       pos += cnt;
     }
