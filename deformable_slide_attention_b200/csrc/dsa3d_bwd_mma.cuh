@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 }
 
 // ---- pass 3: key side ------------------------------------------------------------------------
-// One CTA of 8 warps owns a key tile of 4 consecutive key rows (yk0..yk0+3) x 16 keys
+// One CTA owns a key tile of kKvRows consecutive key rows x 16 keys
 // (x in [16b, 16b+16)) of one frame tk and head; warp w takes key row w/2 and half w%2 of the
 // head dims, with dK and dV in registers.  The queries whose windows cover the tile have origins
 // o_t = tk - bt, o_y in [yk0 - kh, yk0 + 3], o_x in [16b - kw, 16b + 15], i.e. bucket rows
@@ -463,10 +463,14 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 // rows' Gamma^T / Beta^T tiles (key x query, gathered from the stored splats) in shared memory;
 // each warp then adds Gamma^T q and Beta^T dO for its key row with m16n8k16 MMAs (B fragments by
 // ldmatrix.trans of the staged rows).  A query row is loaded once per tile, not once per key row.
-constexpr int kKvRows = 4;
+#ifndef DSA3D_KV_ROWS
+#define DSA3D_KV_ROWS 2
+#endif
+constexpr int kKvRows = DSA3D_KV_ROWS;  // key rows per CTA (2 warps each)
+constexpr int kKvThreads = 64 * kKvRows;
 
 template <int DH>
-__global__ void __launch_bounds__(256, DSA3D_KV_MINB)
+__global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
     dsa3d_bwd_kv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
                         __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                         const int* __restrict__ start, const int* __restrict__ sorted_n,
@@ -519,7 +523,7 @@ __global__ void __launch_bounds__(256, DSA3D_KV_MINB)
           const int cnt = min(16, qend - pos);
           __syncthreads();  // the previous step's tiles are consumed
           // zero the tiles, load the step's per-query data
-          for (int i = tid; i < 2 * kKvRows * 16 * TS / 8; i += 256)
+          for (int i = tid; i < 2 * kKvRows * 16 * TS / 8; i += kKvThreads)
             reinterpret_cast<uint4*>(i < kKvRows * 16 * TS / 8 ? &tg[0][0] : &tb[0][0])
                 [i < kKvRows * 16 * TS / 8 ? i : i - kKvRows * 16 * TS / 8] = make_uint4(0, 0, 0, 0);
           if (tid < 16) {
@@ -530,7 +534,7 @@ __global__ void __launch_bounds__(256, DSA3D_KV_MINB)
           }
           __syncthreads();
           // stage q and dO rows (zeros for missing queries)
-          for (int i = tid; i < 2 * 16 * (DH / 8); i += 256) {
+          for (int i = tid; i < 2 * 16 * (DH / 8); i += kKvThreads) {
             const int which = i / (16 * (DH / 8));
             const int rem = i - which * 16 * (DH / 8);
             const int m = rem / (DH / 8), c = rem - m * (DH / 8);
@@ -541,9 +545,10 @@ __global__ void __launch_bounds__(256, DSA3D_KV_MINB)
             *reinterpret_cast<uint4*>((which ? os : qs) + m * RS + c * 8) = val;
           }
           // gather Gamma^T / Beta^T tiles of the 4 key rows: (query m, key row kr, column bx)
-          {
-            const int m = tid >> 4, w = tid & 15;
-            if (m < cnt && 2 * w < bg.width) {
+          constexpr int WT = kKvThreads / 16;  // threads per query
+          for (int w = tid % WT; 2 * w < bg.width; w += WT) {
+            const int m = tid / WT;
+            if (m < cnt) {
               const float2 d = m_dft[m];
               const int key0 = m_ox[m] + 2 * w;
               if (key0 + 1 >= 0 && key0 < 16) {
