@@ -121,12 +121,16 @@ __device__ __forceinline__ void dsa3d_pv_tile(float (&o)[MmaShape<DH>::NT][4], c
 }
 
 // Shared memory per warp of the forward: raw-score ring [2][16][kFwdRaw], tap ring
-// [2][16][kFwdTap] (P of tap rows ty, ty-1) and two bf16 value-weight tiles [2][16][kFwdTile].
+// [2][16][kFwdTap] (P of tap rows ty, ty-1), two bf16 value-weight tiles [2][16][kFwdTile], and
+// the raw scores of box plane u+1 of the first kFwdCacheRows box rows, in fragment order
+// [row][16 values][32 lanes] (computed for tap plane u and reused as the lower plane of tap plane
+// u+1, so those rows' Q.K^T runs once per box plane; rows beyond the cache recompute).
 constexpr int kFwdRaw = 33;
 constexpr int kFwdTap = 16;
 constexpr int kFwdTile = 40;  // bf16 per row: 32 columns + pad (conflict-free ldmatrix)
+constexpr int kFwdCacheRows = 9;  // keeps two 4-warp CTAs per SM within 228 KB
 __host__ __device__ constexpr int fwd_mma_warp_bytes() {
-  return (2 * 16 * kFwdRaw + 2 * 16 * kFwdTap) * 4 + 2 * 16 * kFwdTile * 2;
+  return (2 * 16 * kFwdRaw + 2 * 16 * kFwdTap + kFwdCacheRows * 16 * 32) * 4 + 2 * 16 * kFwdTile * 2;
 }
 
 template <int DH>
@@ -143,7 +147,8 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
   const int gq = lane >> 2, qq = lane & 3;  // fragment row group / quad position
   float* raw = reinterpret_cast<float*>(fwd_sh + warp * fwd_mma_warp_bytes());
   float* tapb = raw + 2 * 16 * kFwdRaw;
-  unsigned short* tile = reinterpret_cast<unsigned short*>(tapb + 2 * 16 * kFwdTap);
+  float* scache = tapb + 2 * 16 * kFwdTap;
+  unsigned short* tile = reinterpret_cast<unsigned short*>(scache + kFwdCacheRows * 16 * 32);
   const int er = lane >> 1, side = lane & 1;  // epilogue: query row, tap parity
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
@@ -213,14 +218,18 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
       for (int j = 0; j < S::NT; j++) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
       float m = -INFINITY, l = 0.f;  // running max (base 2) and partial sum of row er
 
+      int cached_plane = -1;  // box plane whose raw scores scache holds
       for (int u = 0; u < g.kt; u++) {
         const bool eplane = EQ.lo[0] <= u && u <= hi_t;
         if (!__any_sync(kFull, eplane)) continue;
+        const bool have_u = cached_plane == u;
         for (int i = lane; i < 2 * 16 * kFwdTap; i += 32) tapb[i] = 0.f;
         for (int by = 0; by <= g.kh; by++) {
           const int y = oy + by;
           float* rc = raw + (by & 1) * 16 * kFwdRaw;
-          // t-blended raw scores of box row by -> ring
+          const bool cache_row = by < kFwdCacheRows;
+          float* cr = scache + (cache_row ? by : 0) * 16 * 32 + lane;  // + 32 * (4 * jt + e)
+          // t-blended raw scores of box row by -> ring; raw scores of plane u+1 -> cache
           {
             float st[4][4];
 #pragma unroll
@@ -228,7 +237,20 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
 #pragma unroll
             for (int pl = 0; pl < 2; pl++) {
               const int t = ot + u + pl;
-              if (t < 0 || t >= g.F || y < 0 || y >= g.Hp) continue;
+              if (pl == 0 && have_u && cache_row) {  // plane u was computed for tap plane u-1
+#pragma unroll
+                for (int jt = 0; jt < 4; jt++)
+#pragma unroll
+                  for (int e = 0; e < 4; e++) st[jt][e] = (1.f - fft[e >> 1]) * cr[32 * (4 * jt + e)];
+                continue;
+              }
+              if (t < 0 || t >= g.F || y < 0 || y >= g.Hp) {
+                if (pl == 1 && cache_row) {
+#pragma unroll
+                  for (int i = 0; i < 16; i++) cr[32 * i] = 0.f;
+                }
+                continue;
+              }
 #pragma unroll
               for (int jt = 0; jt < 4; jt++) {
                 const int col = 8 * jt + gq;
@@ -249,6 +271,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
                 for (int e = 0; e < 4; e++) {
                   const float w = pl ? fft[e >> 1] : 1.f - fft[e >> 1];
                   st[jt][e] = fmaf(w, acc[e], st[jt][e]);
+                  if (pl == 1 && cache_row) cr[32 * (4 * jt + e)] = acc[e];
                 }
               }
             }
@@ -349,6 +372,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
           dsa3d_pv_tile<DH>(o, tile, ot + u, oy + g.kh, X0, segw, vh_, rs, g, lane);
           __syncwarp();
         }
+        cached_plane = u + 1;
       }
 
       // ---- normalise and store (row sums from the epilogue lanes)
