@@ -14,7 +14,7 @@
 //     (gamma') onto the box rows, in bf16: box[pos][u][by][bx], and D, f_t per query.
 //  2. dq (dsa3d_bwd_dq_kernel): dq = scale sum_j gamma[j] K[j], gamma = gamma' - D beta and the
 //     t-mix of the two tap planes feeding each box plane, as tensor-core products per box row.
-//  3. key side (dsa3d_bwd_kv_kernel): one warp owns 16 keys x 64 dims of one key row and
+//  3. key side (dsa3d_bwd_kv_kernel): one warp owns 16 keys x dh/2 dims of one key row and
 //     gathers, from the bucket ranges of the queries whose boxes cover those keys, the stored
 //     gamma/beta rows: dK += scale Gamma^T Q, dV += Beta^T dO on tensor cores, written once.
 #pragma once
@@ -457,17 +457,18 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 // One CTA owns a key tile of kKvRows consecutive key rows x 16 keys
 // (x in [16b, 16b+16)) of one frame tk and head; warp w takes key row w/2 and half w%2 of the
 // head dims, with dK and dV in registers.  The queries whose windows cover the tile have origins
-// o_t = tk - bt, o_y in [yk0 - kh, yk0 + 3], o_x in [16b - kw, 16b + 15], i.e. bucket rows
-// e_t = tk - bt + kt, e_y in [yk0, yk0 + 3 + kh] and the e_x range [16b, 16b + 16 + kw).  Per
-// step (<= 16 such queries of one bucket row) the CTA stages their q and dO rows and the four key
-// rows' Gamma^T / Beta^T tiles (key x query, gathered from the stored splats) in shared memory;
-// each warp then adds Gamma^T q and Beta^T dO for its key row with m16n8k16 MMAs (B fragments by
+// o_t = tk - bt, o_y in [yk0 - kh, yk0 + kKvRows - 1], o_x in [16b - kw, 16b + 15], i.e. bucket
+// rows e_t = tk - bt + kt, e_y in [yk0, yk0 + kKvRows - 1 + kh] and the e_x range
+// [16b, 16b + 16 + kw).  Per step (16 such queries, in sorted order across those bucket rows)
+// the CTA stages their q and dO rows and its key rows' Gamma^T / Beta^T tiles (key x query,
+// gathered from the stored splats) in shared memory; each warp then adds Gamma^T q and Beta^T dO for its key row with m16n8k16 MMAs (B fragments by
 // ldmatrix.trans of the staged rows).  A query row is loaded once per tile, not once per key row.
 #ifndef DSA3D_KV_ROWS
 #define DSA3D_KV_ROWS 2
 #endif
 constexpr int kKvRows = DSA3D_KV_ROWS;  // key rows per CTA (2 warps each)
 constexpr int kKvThreads = 64 * kKvRows;
+constexpr int kKvRanges = 64;  // bucket-row ranges per batch (two per lane of warp 0)
 
 template <int DH>
 __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
@@ -485,8 +486,9 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
   __shared__ __align__(16) unsigned short tb[kKvRows][16 * TS];
   __shared__ __align__(16) unsigned short qs[16 * RS];
   __shared__ __align__(16) unsigned short os[16 * RS];
-  __shared__ int m_tok[16], m_ox[16];
+  __shared__ int m_tok[16], m_ox[16], m_pos[16], m_bt[16], m_by0[16];
   __shared__ float2 m_dft[16];
+  __shared__ int r_beg[kKvRanges], r_pre[kKvRanges + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, qq = lane & 3;
   const int wr = warp >> 1, half = warp & 1;
@@ -512,88 +514,130 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
 #pragma unroll
       for (int e = 0; e < 4; e++) ak[j][e] = av[j][e] = 0.f;
 
-    for (int bt = 0; bt <= g.kt; bt++) {
-      const int et = tk - bt + g.kt;
-      const int ey_hi = min(yk0 + kKvRows - 1 + g.kh, sg.Ey - 1);
-      for (int ey = yk0; ey <= ey_hi; ey++) {
-        const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)et * sg.Ey + ey) * sg.Ex;
-        const int qbeg = start[b0 + x_lo];
-        const int qend = start[b0 + min(x_lo + 16 + g.kw, sg.Ex)];
-        for (int pos = qbeg; pos < qend; pos += 16) {
-          const int cnt = min(16, qend - pos);
-          __syncthreads();  // the previous step's tiles are consumed
-          // zero the tiles, load the step's per-query data
-          for (int i = tid; i < 2 * kKvRows * 16 * TS / 8; i += kKvThreads)
-            reinterpret_cast<uint4*>(i < kKvRows * 16 * TS / 8 ? &tg[0][0] : &tb[0][0])
-                [i < kKvRows * 16 * TS / 8 ? i : i - kKvRows * 16 * TS / 8] = make_uint4(0, 0, 0, 0);
-          if (tid < 16) {
-            const bool live = tid < cnt;
-            m_tok[tid] = live ? sorted_n[pos + tid] : -1;
-            m_ox[tid] = live ? sorted_ex[pos + tid] - g.kw - x_lo : 0;
-            m_dft[tid] = live ? dft[pos + tid] : make_float2(0.f, 0.f);
-          }
-          __syncthreads();
-          // stage q and dO rows (zeros for missing queries)
-          for (int i = tid; i < 2 * 16 * (DH / 8); i += kKvThreads) {
-            const int which = i / (16 * (DH / 8));
-            const int rem = i - which * 16 * (DH / 8);
-            const int m = rem / (DH / 8), c = rem - m * (DH / 8);
-            const int n = m_tok[m];
-            const __nv_bfloat16* src = which ? dout : q;
-            const uint4 val = (n >= 0) ? ldg16(src + ((int64_t)n * g.heads + h) * DH + c * 8)
-                                       : make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>((which ? os : qs) + m * RS + c * 8) = val;
-          }
-          // gather Gamma^T / Beta^T tiles of the 4 key rows: (query m, key row kr, column bx)
-          constexpr int WT = kKvThreads / 16;  // threads per query
-          for (int w = tid % WT; 2 * w < bg.width; w += WT) {
-            const int m = tid / WT;
-            if (m < cnt) {
-              const float2 d = m_dft[m];
-              const int key0 = m_ox[m] + 2 * w;
-              if (key0 + 1 >= 0 && key0 < 16) {
+    // The queries covering the tile lie in (kt + 1) x ney bucket-row ranges of the sorted order
+    // (range r: bt = r / ney, ey = yk0 + r % ney).  They are taken in batches of up to kKvRanges
+    // ranges, concatenated, and consumed 16 at a time, so a step mixes queries of several bucket
+    // rows and only the last step of a batch is partly empty.
+    const int ney = min(yk0 + kKvRows - 1 + g.kh, sg.Ey - 1) - yk0 + 1;
+    const int nranges = (g.kt + 1) * ney;
+    for (int rb = 0; rb < nranges; rb += kKvRanges) {
+      const int nr = min(kKvRanges, nranges - rb);
+      __syncthreads();  // the previous batch's ranges are consumed
+      if (warp == 0) {
+        int len[2];
 #pragma unroll
-                for (int kr = 0; kr < kKvRows; kr++) {
-                  const int by = yk0 + kr - ey + g.kh;
-                  if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
-                  float ga[2], be[2];
-                  box_word(gbox, bbox, pos + m, bg, g.kt, g.kh, bt, by, w, d.x, d.y, ga, be);
+        for (int e = 0; e < 2; e++) {
+          const int r = 2 * lane + e;
+          len[e] = 0;
+          if (r < nr) {
+            const int bt = (rb + r) / ney, ey = yk0 + (rb + r) - bt * ney;
+            const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)(tk - bt + g.kt) * sg.Ey + ey) * sg.Ex;
+            const int qb = start[b0 + x_lo];
+            r_beg[r] = qb;
+            len[e] = start[b0 + min(x_lo + 16 + g.kw, sg.Ex)] - qb;
+          }
+        }
+        const int pair = len[0] + len[1];
+        int incl = pair;
 #pragma unroll
-                  for (int e = 0; e < 2; e++) {
-                    const int key = key0 + e;
-                    if (key >= 0 && key < 16) {
-                      tg[kr][key * TS + m] = bf16_bits(ga[e]);
-                      tb[kr][key * TS + m] = bf16_bits(be[e]);
-                    }
+        for (int d = 1; d < 32; d <<= 1) {
+          const int y = __shfl_up_sync(kFull, incl, d);
+          if (lane >= d) incl += y;
+        }
+        r_pre[2 * lane] = incl - pair;
+        r_pre[2 * lane + 1] = incl - pair + len[0];
+        if (lane == 31) r_pre[kKvRanges] = incl;
+      }
+      __syncthreads();
+      const int total = r_pre[kKvRanges];
+      for (int s0 = 0; s0 < total; s0 += 16) {
+        const int cnt = min(16, total - s0);
+        __syncthreads();  // the previous step's tiles are consumed
+        // zero the tiles, locate the step's queries
+        for (int i = tid; i < 2 * kKvRows * 16 * TS / 8; i += kKvThreads)
+          reinterpret_cast<uint4*>(i < kKvRows * 16 * TS / 8 ? &tg[0][0] : &tb[0][0])
+              [i < kKvRows * 16 * TS / 8 ? i : i - kKvRows * 16 * TS / 8] = make_uint4(0, 0, 0, 0);
+        if (tid < 16) {
+          if (tid < cnt) {
+            const int i = s0 + tid;
+            int lo = 0, hi = kKvRanges;  // largest r with r_pre[r] <= i (a non-empty range)
+            while (hi - lo > 1) {
+              const int mid = (lo + hi) >> 1;
+              if (r_pre[mid] <= i) lo = mid; else hi = mid;
+            }
+            const int pos = r_beg[lo] + (i - r_pre[lo]);
+            const int bt = (rb + lo) / ney;
+            m_pos[tid] = pos;
+            m_bt[tid] = bt;
+            m_by0[tid] = yk0 - (yk0 + (rb + lo) - bt * ney) + g.kh;  // box row of key row yk0
+            m_tok[tid] = sorted_n[pos];
+            m_ox[tid] = sorted_ex[pos] - g.kw - x_lo;
+            m_dft[tid] = dft[pos];
+          } else {
+            m_tok[tid] = -1;
+          }
+        }
+        __syncthreads();
+        // stage q and dO rows (zeros for missing queries)
+        for (int i = tid; i < 2 * 16 * (DH / 8); i += kKvThreads) {
+          const int which = i / (16 * (DH / 8));
+          const int rem = i - which * 16 * (DH / 8);
+          const int m = rem / (DH / 8), c = rem - m * (DH / 8);
+          const int n = m_tok[m];
+          const __nv_bfloat16* src = which ? dout : q;
+          const uint4 val = (n >= 0) ? ldg16(src + ((int64_t)n * g.heads + h) * DH + c * 8)
+                                     : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>((which ? os : qs) + m * RS + c * 8) = val;
+        }
+        // gather Gamma^T / Beta^T tiles of the key rows: (query m, key row kr, column bx)
+        constexpr int WT = kKvThreads / 16;  // threads per query
+        for (int w = tid % WT; 2 * w < bg.width; w += WT) {
+          const int m = tid / WT;
+          if (m < cnt) {
+            const float2 d = m_dft[m];
+            const int key0 = m_ox[m] + 2 * w;
+            if (key0 + 1 >= 0 && key0 < 16) {
+              const int pos = m_pos[m], bt = m_bt[m], by0 = m_by0[m];
+#pragma unroll
+              for (int kr = 0; kr < kKvRows; kr++) {
+                const int by = by0 + kr;
+                if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
+                float ga[2], be[2];
+                box_word(gbox, bbox, pos, bg, g.kt, g.kh, bt, by, w, d.x, d.y, ga, be);
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                  const int key = key0 + e;
+                  if (key >= 0 && key < 16) {
+                    tg[kr][key * TS + m] = bf16_bits(ga[e]);
+                    tb[kr][key * TS + m] = bf16_bits(be[e]);
                   }
                 }
               }
             }
           }
-          __syncthreads();
-          const int by_w = myk - ey + g.kh;
-          if (myk < g.Hp && by_w >= 0 && by_w <= g.kh) {
-            unsigned agm[4], abt[4];
-            const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4);
-            ldsm_x4(agm, &tg[wr][rr * TS + cc]);
-            ldsm_x4(abt, &tb[wr][rr * TS + cc]);
+        }
+        __syncthreads();
+        if (myk < g.Hp) {
+          unsigned agm[4], abt[4];
+          const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4);
+          ldsm_x4(agm, &tg[wr][rr * TS + cc]);
+          ldsm_x4(abt, &tb[wr][rr * TS + cc]);
 #pragma unroll
-            for (int j2 = 0; j2 < NTH / 2; j2++) {
-              // B fragments of n-tiles 2*j2, 2*j2+1: rows = queries (k), cols = dims (n)
-              const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);
-              const int dcol = half * HALF + 16 * j2 + 8 * (lane >> 4);
-              unsigned bq[4], bo[4];
-              const unsigned aq = (unsigned)__cvta_generic_to_shared(qs + mrow * RS + dcol);
-              const unsigned ao = (unsigned)__cvta_generic_to_shared(os + mrow * RS + dcol);
-              asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                           : "=r"(bq[0]), "=r"(bq[1]), "=r"(bq[2]), "=r"(bq[3]) : "r"(aq));
-              asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                           : "=r"(bo[0]), "=r"(bo[1]), "=r"(bo[2]), "=r"(bo[3]) : "r"(ao));
-              mma_bf16_16816(ak[2 * j2], agm[0], agm[1], agm[2], agm[3], bq[0], bq[1]);
-              mma_bf16_16816(ak[2 * j2 + 1], agm[0], agm[1], agm[2], agm[3], bq[2], bq[3]);
-              mma_bf16_16816(av[2 * j2], abt[0], abt[1], abt[2], abt[3], bo[0], bo[1]);
-              mma_bf16_16816(av[2 * j2 + 1], abt[0], abt[1], abt[2], abt[3], bo[2], bo[3]);
-            }
+          for (int j2 = 0; j2 < NTH / 2; j2++) {
+            // B fragments of n-tiles 2*j2, 2*j2+1: rows = queries (k), cols = dims (n)
+            const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);
+            const int dcol = half * HALF + 16 * j2 + 8 * (lane >> 4);
+            unsigned bq[4], bo[4];
+            const unsigned aq = (unsigned)__cvta_generic_to_shared(qs + mrow * RS + dcol);
+            const unsigned ao = (unsigned)__cvta_generic_to_shared(os + mrow * RS + dcol);
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(bq[0]), "=r"(bq[1]), "=r"(bq[2]), "=r"(bq[3]) : "r"(aq));
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                         : "=r"(bo[0]), "=r"(bo[1]), "=r"(bo[2]), "=r"(bo[3]) : "r"(ao));
+            mma_bf16_16816(ak[2 * j2], agm[0], agm[1], agm[2], agm[3], bq[0], bq[1]);
+            mma_bf16_16816(ak[2 * j2 + 1], agm[0], agm[1], agm[2], agm[3], bq[2], bq[3]);
+            mma_bf16_16816(av[2 * j2], abt[0], abt[1], abt[2], abt[3], bo[0], bo[1]);
+            mma_bf16_16816(av[2 * j2 + 1], abt[0], abt[1], abt[2], abt[3], bo[2], bo[3]);
           }
         }
       }

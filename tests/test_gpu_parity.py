@@ -92,6 +92,14 @@ def test_widest_tensor_core_windows(window):
     full_parity(inp, dims, window, "bf16")
 
 
+def test_tall_windows_many_bucket_rows_per_key_tile():
+    # a key tile of the key-side pass is covered by (k_t + 1) x (rows + k_h) bucket rows of queries:
+    # 10 x 18 = 180 here, more than one batch of the per-tile range list
+    dims, window = (6, 12, 10), (9, 17, 5)
+    _, inp = inputs.custom(*dims, 2, 64, window, "bf16", seed=17, scale=2.5)
+    full_parity(inp, dims, window, "bf16")
+
+
 def test_tensor_core_path_sparse_and_invalid_queries():
     # large offsets: many queries leave the volume, bucket rows are sparse and ragged
     dims, window = (4, 7, 9), (3, 3, 3)
