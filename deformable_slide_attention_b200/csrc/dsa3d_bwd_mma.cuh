@@ -470,6 +470,16 @@ constexpr int kKvRows = DSA3D_KV_ROWS;  // key rows per CTA (2 warps each)
 constexpr int kKvThreads = 64 * kKvRows;
 constexpr int kKvRanges = 64;  // bucket-row ranges per batch (two per lane of warp 0)
 
+// One query slot of a key-side step.
+struct KvSlot {
+  int tok;     // token, -1 for an empty slot
+  int pos;     // sorted position (index of the stored splats)
+  int bt;      // box plane of the tile's frame in the query's box
+  int by0;     // box row of the tile's first key row (may lie outside [0, kh])
+  int ox;      // x-origin minus the tile's first key x
+  float2 d;    // (D, f_t)
+};
+
 template <int DH>
 __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
     dsa3d_bwd_kv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
@@ -482,16 +492,19 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
   constexpr int NTH = HALF / 8; // n-tiles per warp
   constexpr int TS = 24;        // Gamma/Beta tile row stride (bf16): conflict-free ldmatrix
   constexpr int RS = DH + 8;    // staged q/dO row stride (bf16): conflict-free ldmatrix.trans
-  __shared__ __align__(16) unsigned short tg[kKvRows][16 * TS];
-  __shared__ __align__(16) unsigned short tb[kKvRows][16 * TS];
-  __shared__ __align__(16) unsigned short qs[16 * RS];
-  __shared__ __align__(16) unsigned short os[16 * RS];
-  __shared__ int m_tok[16], m_ox[16], m_pos[16], m_bt[16], m_by0[16];
-  __shared__ float2 m_dft[16];
+  constexpr int TILE = kKvRows * 16 * TS;  // one stage of Gamma^T (or Beta^T) tiles
+  constexpr int WT = kKvThreads / 16;      // gather threads per query slot
+  static_assert(WT >= 8, "a query's stored row (<= 8 words) is gathered by one pass of its threads");
+  __shared__ __align__(16) unsigned short tg[3][TILE];
+  __shared__ __align__(16) unsigned short tb[3][TILE];
+  __shared__ __align__(16) unsigned short qs[2][16 * RS];
+  __shared__ __align__(16) unsigned short os[2][16 * RS];
+  __shared__ KvSlot meta[2][16];
   __shared__ int r_beg[kKvRanges], r_pre[kKvRanges + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, qq = lane & 3;
   const int wr = warp >> 1, half = warp & 1;
+  const int gm = tid / WT, gw = tid % WT;  // gather: query slot, stored word
   const int NB = (g.Wp + 15) / 16;
   const int NY = (g.Hp + kKvRows - 1) / kKvRows;
   const int64_t tiles = (int64_t)hg * g.F * NY * NB;
@@ -522,18 +535,18 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
     const int nranges = (g.kt + 1) * ney;
     for (int rb = 0; rb < nranges; rb += kKvRanges) {
       const int nr = min(kKvRanges, nranges - rb);
-      __syncthreads();  // the previous batch's ranges are consumed
+      __syncthreads();  // the previous batch's ranges and buffers are consumed
       if (warp == 0) {
         int len[2];
 #pragma unroll
         for (int e = 0; e < 2; e++) {
-          const int r = 2 * lane + e;
+          const int rr = 2 * lane + e;
           len[e] = 0;
-          if (r < nr) {
-            const int bt = (rb + r) / ney, ey = yk0 + (rb + r) - bt * ney;
+          if (rr < nr) {
+            const int bt = (rb + rr) / ney, ey = yk0 + (rb + rr) - bt * ney;
             const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)(tk - bt + g.kt) * sg.Ey + ey) * sg.Ex;
             const int qb = start[b0 + x_lo];
-            r_beg[r] = qb;
+            r_beg[rr] = qb;
             len[e] = start[b0 + min(x_lo + 16 + g.kw, sg.Ex)] - qb;
           }
         }
@@ -550,96 +563,159 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
       }
       __syncthreads();
       const int total = r_pre[kKvRanges];
-      for (int s0 = 0; s0 < total; s0 += 16) {
-        const int cnt = min(16, total - s0);
-        __syncthreads();  // the previous step's tiles are consumed
-        // zero the tiles, locate the step's queries
-        for (int i = tid; i < 2 * kKvRows * 16 * TS / 8; i += kKvThreads)
-          reinterpret_cast<uint4*>(i < kKvRows * 16 * TS / 8 ? &tg[0][0] : &tb[0][0])
-              [i < kKvRows * 16 * TS / 8 ? i : i - kKvRows * 16 * TS / 8] = make_uint4(0, 0, 0, 0);
-        if (tid < 16) {
-          if (tid < cnt) {
-            const int i = s0 + tid;
-            int lo = 0, hi = kKvRanges;  // largest r with r_pre[r] <= i (a non-empty range)
-            while (hi - lo > 1) {
-              const int mid = (lo + hi) >> 1;
-              if (r_pre[mid] <= i) lo = mid; else hi = mid;
-            }
-            const int pos = r_beg[lo] + (i - r_pre[lo]);
-            const int bt = (rb + lo) / ney;
-            m_pos[tid] = pos;
-            m_bt[tid] = bt;
-            m_by0[tid] = yk0 - (yk0 + (rb + lo) - bt * ney) + g.kh;  // box row of key row yk0
-            m_tok[tid] = sorted_n[pos];
-            m_ox[tid] = sorted_ex[pos] - g.kw - x_lo;
-            m_dft[tid] = dft[pos];
-          } else {
-            m_tok[tid] = -1;
+      const int nsteps = (total + 15) / 16;
+      if (nsteps == 0) continue;
+
+      // slot tid (< 16) of step s: the query's sorted position, box plane, box row of key row
+      // yk0, token, x-origin relative to the tile and (D, f_t); tok = -1 for an empty slot
+      auto load_slot = [&](int s) {
+        KvSlot m;
+        m.tok = -1;
+        const int i = 16 * s + tid;
+        if (i < total) {
+          int lo = 0, hi = kKvRanges;  // largest r with r_pre[r] <= i (a non-empty range)
+          while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (r_pre[mid] <= i) lo = mid; else hi = mid;
           }
+          const int pos = r_beg[lo] + (i - r_pre[lo]);
+          const int bt = (rb + lo) / ney;
+          m.pos = pos;
+          m.bt = bt;
+          m.by0 = g.kh - ((rb + lo) - bt * ney);  // yk0 - ey + kh
+          m.tok = sorted_n[pos];
+          m.ox = sorted_ex[pos] - g.kw - x_lo;
+          m.d = dft[pos];
         }
-        __syncthreads();
-        // stage q and dO rows (zeros for missing queries)
+        return m;
+      };
+      // q and dO rows of step s into buffer s & 1 (zero-filled for empty slots)
+      auto stage_rows = [&](int s) {
+        const KvSlot* ms = meta[s & 1];
         for (int i = tid; i < 2 * 16 * (DH / 8); i += kKvThreads) {
           const int which = i / (16 * (DH / 8));
           const int rem = i - which * 16 * (DH / 8);
           const int m = rem / (DH / 8), c = rem - m * (DH / 8);
-          const int n = m_tok[m];
-          const __nv_bfloat16* src = which ? dout : q;
-          const uint4 val = (n >= 0) ? ldg16(src + ((int64_t)n * g.heads + h) * DH + c * 8)
-                                     : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>((which ? os : qs) + m * RS + c * 8) = val;
+          const int n = ms[m].tok;
+          const __nv_bfloat16* src = (which ? dout : q) + ((int64_t)max(n, 0) * g.heads + h) * DH + c * 8;
+          cp_async16_zfill((which ? os[s & 1] : qs[s & 1]) + m * RS + c * 8, src, n >= 0);
         }
-        // gather Gamma^T / Beta^T tiles of the key rows: (query m, key row kr, column bx)
-        constexpr int WT = kKvThreads / 16;  // threads per query
-        for (int w = tid % WT; 2 * w < bg.width; w += WT) {
-          const int m = tid / WT;
-          if (m < cnt) {
-            const float2 d = m_dft[m];
-            const int key0 = m_ox[m] + 2 * w;
-            if (key0 + 1 >= 0 && key0 < 16) {
-              const int pos = m_pos[m], bt = m_bt[m], by0 = m_by0[m];
+        cp_async_commit();
+      };
+      // the stored words of step s this thread gathers: per key row, planes bt and bt-1
+      struct Words { unsigned g0[kKvRows], b0[kKvRows], g1[kKvRows], b1[kKvRows]; };
+      auto gather_load = [&](int s, Words& wd, KvSlot& m) {
+        m = meta[s & 1][gm];
 #pragma unroll
-              for (int kr = 0; kr < kKvRows; kr++) {
-                const int by = by0 + kr;
-                if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
-                float ga[2], be[2];
-                box_word(gbox, bbox, pos, bg, g.kt, g.kh, bt, by, w, d.x, d.y, ga, be);
+        for (int kr = 0; kr < kKvRows; kr++) wd.g0[kr] = wd.b0[kr] = wd.g1[kr] = wd.b1[kr] = 0u;
+        const int key0 = m.ox + 2 * gw;
+        if (m.tok < 0 || 2 * gw >= bg.width || key0 + 1 < 0 || key0 >= 16) return;
 #pragma unroll
-                for (int e = 0; e < 2; e++) {
-                  const int key = key0 + e;
-                  if (key >= 0 && key < 16) {
-                    tg[kr][key * TS + m] = bf16_bits(ga[e]);
-                    tb[kr][key * TS + m] = bf16_bits(be[e]);
-                  }
-                }
-              }
-            }
+        for (int kr = 0; kr < kKvRows; kr++) {
+          const int by = m.by0 + kr;
+          if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
+          if (m.bt < g.kt) {
+            const int64_t o = ((int64_t)m.pos * bg.rows + m.bt * (g.kh + 1) + by) * bg.width + 2 * gw;
+            wd.g0[kr] = *reinterpret_cast<const unsigned*>(gbox + o);
+            wd.b0[kr] = *reinterpret_cast<const unsigned*>(bbox + o);
+          }
+          if (m.bt >= 1) {
+            const int64_t o = ((int64_t)m.pos * bg.rows + (m.bt - 1) * (g.kh + 1) + by) * bg.width + 2 * gw;
+            wd.g1[kr] = *reinterpret_cast<const unsigned*>(gbox + o);
+            wd.b1[kr] = *reinterpret_cast<const unsigned*>(bbox + o);
           }
         }
-        __syncthreads();
+      };
+      // gamma = t-mix of (gamma' - D beta), beta = t-mix of beta, into the stage's tiles
+      auto gather_store = [&](int stage, const Words& wd, const KvSlot& m) {
+        const int key0 = m.ox + 2 * gw;
+        if (m.tok < 0 || 2 * gw >= bg.width || key0 + 1 < 0 || key0 >= 16) return;
+        const float D = m.d.x, ft = m.d.y;
+#pragma unroll
+        for (int kr = 0; kr < kKvRows; kr++) {
+#pragma unroll
+          for (int e = 0; e < 2; e++) {
+            const int key = key0 + e;
+            if (key < 0 || key >= 16) continue;
+            const float bb0 = bf16_val((unsigned short)(wd.b0[kr] >> (16 * e)));
+            const float gg0 = bf16_val((unsigned short)(wd.g0[kr] >> (16 * e)));
+            const float bb1 = bf16_val((unsigned short)(wd.b1[kr] >> (16 * e)));
+            const float gg1 = bf16_val((unsigned short)(wd.g1[kr] >> (16 * e)));
+            const float be = fmaf(ft, bb1 - bb0, bb0);
+            const float c0 = fmaf(-D, bb0, gg0), c1 = fmaf(-D, bb1, gg1);
+            const float ga = fmaf(ft, c1 - c0, c0);
+            tg[stage][kr * 16 * TS + key * TS + gm] = bf16_bits(ga);
+            tb[stage][kr * 16 * TS + key * TS + gm] = bf16_bits(be);
+          }
+        }
+      };
+      auto zero_stage = [&](int stage) {
+        for (int i = tid; i < TILE / 8; i += kKvThreads) {
+          reinterpret_cast<uint4*>(tg[stage])[i] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(tb[stage])[i] = make_uint4(0, 0, 0, 0);
+        }
+      };
+
+      // prologue: slots of steps 0 and 1, step 0's rows and tiles
+      if (tid < 16) {
+        meta[0][tid] = load_slot(0);
+        meta[1][tid] = load_slot(1);
+      }
+      zero_stage(0);
+      zero_stage(1);
+      __syncthreads();
+      {
+        stage_rows(0);
+        Words wd;
+        KvSlot m;
+        gather_load(0, wd, m);
+        gather_store(0, wd, m);
+        cp_async_wait_all();
+      }
+      __syncthreads();
+
+      // step s: prefetch step s+1 (rows by cp.async, stored words into registers) and the slots
+      // of step s+2, run step s's MMAs, then complete step s+1's tiles; one barrier per step
+      for (int s = 0; s < nsteps; s++) {
+        const bool more = s + 1 < nsteps;
+        zero_stage((s + 2) % 3);
+        Words wd;
+        KvSlot m;
+        if (more) {
+          stage_rows(s + 1);
+          gather_load(s + 1, wd, m);
+        }
+        KvSlot next;
+        next.tok = -1;
+        if (tid < 16 && s + 2 < nsteps) next = load_slot(s + 2);
+
         if (myk < g.Hp) {
+          const unsigned short* tgs = tg[s % 3] + wr * 16 * TS;
+          const unsigned short* tbs = tb[s % 3] + wr * 16 * TS;
+          const unsigned short* qsb = qs[s & 1];
+          const unsigned short* osb = os[s & 1];
           unsigned agm[4], abt[4];
           const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4);
-          ldsm_x4(agm, &tg[wr][rr * TS + cc]);
-          ldsm_x4(abt, &tb[wr][rr * TS + cc]);
+          ldsm_x4(agm, tgs + rr * TS + cc);
+          ldsm_x4(abt, tbs + rr * TS + cc);
 #pragma unroll
           for (int j2 = 0; j2 < NTH / 2; j2++) {
             // B fragments of n-tiles 2*j2, 2*j2+1: rows = queries (k), cols = dims (n)
-            const int mrow = (lane & 7) + 8 * ((lane >> 3) & 1);
             const int dcol = half * HALF + 16 * j2 + 8 * (lane >> 4);
             unsigned bq[4], bo[4];
-            const unsigned aq = (unsigned)__cvta_generic_to_shared(qs + mrow * RS + dcol);
-            const unsigned ao = (unsigned)__cvta_generic_to_shared(os + mrow * RS + dcol);
-            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                         : "=r"(bq[0]), "=r"(bq[1]), "=r"(bq[2]), "=r"(bq[3]) : "r"(aq));
-            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                         : "=r"(bo[0]), "=r"(bo[1]), "=r"(bo[2]), "=r"(bo[3]) : "r"(ao));
+            ldsm_x4_trans(bq, qsb + rr * RS + dcol);
+            ldsm_x4_trans(bo, osb + rr * RS + dcol);
             mma_bf16_16816(ak[2 * j2], agm[0], agm[1], agm[2], agm[3], bq[0], bq[1]);
             mma_bf16_16816(ak[2 * j2 + 1], agm[0], agm[1], agm[2], agm[3], bq[2], bq[3]);
             mma_bf16_16816(av[2 * j2], abt[0], abt[1], abt[2], abt[3], bo[0], bo[1]);
             mma_bf16_16816(av[2 * j2 + 1], abt[0], abt[1], abt[2], abt[3], bo[2], bo[3]);
           }
         }
+
+        if (more) gather_store((s + 1) % 3, wd, m);
+        if (tid < 16 && s + 2 < nsteps) meta[s & 1][tid] = next;
+        cp_async_wait_all();
+        __syncthreads();
       }
     }
     // write this warp's key row: keys g, g+8 of the block; n-tile j col c -> dim half*HALF + 8j + c
@@ -660,7 +736,6 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
         }
       }
     }
-    __syncthreads();
   }
 }
 
