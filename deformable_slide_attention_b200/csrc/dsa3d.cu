@@ -336,8 +336,12 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
   {
+    const int smem = 4 * dq_warp_bytes<DH>();
+    if (cudaFuncSetAttribute(dsa3d_bwd_dq_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return DSA3D_ERR_CUDA;
     TimedLaunch tl(kKernBwdDq, st);
-    dsa3d_bwd_dq_kernel<DH><<<grid_for(rows, 4, 1 << 20), 128, 0, st>>>(
+    dsa3d_bwd_dq_kernel<DH><<<grid_for(rows, 4, 1 << 20), 128, smem, st>>>(
         kb, static_cast<bf*>(dq), w.cnt, w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg, h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }

@@ -13,7 +13,8 @@
 //     It stores, per query and tap plane, the y/x-transposed splats of P (beta) and of P dP
 //     (gamma') onto the box rows, in bf16: box[pos][u][by][bx], and D, f_t per query.
 //  2. dq (dsa3d_bwd_dq_kernel): dq = scale sum_j gamma[j] K[j], gamma = gamma' - D beta and the
-//     t-mix of the two tap planes feeding each box plane, as tensor-core products per box row.
+//     t-mix of the two tap planes feeding each box plane, as tensor-core products per box row
+//     (K segments staged in shared memory by cp.async, one step ahead).
 //  3. key side (dsa3d_bwd_kv_kernel): one warp owns 16 keys x dh/2 dims of one key row and
 //     gathers, from the bucket ranges of the queries whose boxes cover those keys, the stored
 //     gamma/beta rows: dK += scale Gamma^T Q, dV += Beta^T dO on tensor cores, written once.
@@ -118,8 +119,8 @@ __device__ __forceinline__ int chunk_len(const int* sorted_ex, int pos, int qend
 // segment columns), forms the tap's score, dP, their derivatives along (t, y, x), P and the
 // per-query sums; the taps' P and P dP go to a two-row ring, from which box row by-1's splats
 // (x-transpose, then y-mix with the previous tap row) are stored.
-constexpr int kRawStride = 33;  // floats per row of a raw block (odd: conflict-free columns)
-constexpr int kTapStride = 16;  // floats per row of a tap-row buffer (kw <= 15)
+constexpr int kRawStride = 40;  // floats per row of a raw block (conflict-free float2 fragment stores)
+constexpr int kTapStride = 18;  // floats per row of a tap-row buffer (kw <= 15; 18: conflict-free per-query lanes)
 
 __host__ __device__ constexpr int bwdq_warp_floats() {
   return 2 * 4 * 16 * kRawStride + 2 * 2 * 16 * kTapStride;
@@ -189,22 +190,24 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
 #pragma unroll
             for (int jt = 0; jt < 4; jt++)
 #pragma unroll
-              for (int e = 0; e < 4; e++) {
-                const int rr = gq + 8 * (e >> 1), cc = 8 * jt + 2 * qq + (e & 1);
-                const float d = s1[jt][e] - s0[jt][e];
-                rc[(0 * 16 + rr) * kRawStride + cc] = fmaf(R[e >> 1].f[0], d, s0[jt][e]);
-                rc[(1 * 16 + rr) * kRawStride + cc] = d;
+              for (int hf = 0; hf < 2; hf++) {
+                const int rr = gq + 8 * hf, cc = 8 * jt + 2 * qq;
+                const float d0 = s1[jt][2 * hf] - s0[jt][2 * hf], d1 = s1[jt][2 * hf + 1] - s0[jt][2 * hf + 1];
+                *reinterpret_cast<float2*>(rc + (0 * 16 + rr) * kRawStride + cc) =
+                    make_float2(fmaf(R[hf].f[0], d0, s0[jt][2 * hf]), fmaf(R[hf].f[0], d1, s0[jt][2 * hf + 1]));
+                *reinterpret_cast<float2*>(rc + (1 * 16 + rr) * kRawStride + cc) = make_float2(d0, d1);
               }
             raw_block<DH>(s0, ga, vh_, ot + u, y, X0, segw, rs, g, gq, qq);
             raw_block<DH>(s1, ga, vh_, ot + u + 1, y, X0, segw, rs, g, gq, qq);
 #pragma unroll
             for (int jt = 0; jt < 4; jt++)
 #pragma unroll
-              for (int e = 0; e < 4; e++) {
-                const int rr = gq + 8 * (e >> 1), cc = 8 * jt + 2 * qq + (e & 1);
-                const float d = s1[jt][e] - s0[jt][e];
-                rc[(2 * 16 + rr) * kRawStride + cc] = fmaf(R[e >> 1].f[0], d, s0[jt][e]);
-                rc[(3 * 16 + rr) * kRawStride + cc] = d;
+              for (int hf = 0; hf < 2; hf++) {
+                const int rr = gq + 8 * hf, cc = 8 * jt + 2 * qq;
+                const float d0 = s1[jt][2 * hf] - s0[jt][2 * hf], d1 = s1[jt][2 * hf + 1] - s0[jt][2 * hf + 1];
+                *reinterpret_cast<float2*>(rc + (2 * 16 + rr) * kRawStride + cc) =
+                    make_float2(fmaf(R[hf].f[0], d0, s0[jt][2 * hf]), fmaf(R[hf].f[0], d1, s0[jt][2 * hf + 1]));
+                *reinterpret_cast<float2*>(rc + (3 * 16 + rr) * kRawStride + cc) = make_float2(d0, d1);
               }
           }
           __syncwarp();
@@ -343,6 +346,18 @@ __device__ __forceinline__ void box_word(const unsigned short* gbox, const unsig
 }
 
 // ---- pass 2: dq = scale * sum_j gamma[j] K[j] ----------------------------------------------------
+// Per warp and chunk, per box plane bt and box row by (the box's in-volume rectangle, in order):
+// the chunk's gamma tile (16 queries x 32 segment keys, bf16) and the K segment of key row
+// (o_t + bt, o_y + by) in shared memory, then acc += gamma . K_seg on tensor cores (A by ldmatrix,
+// B by ldmatrix.trans of the staged key rows).  Software pipeline: the next step's K segment is
+// copied by cp.async into the other of two buffers and its stored splat words are loaded into
+// registers while the current step's MMAs run.
+constexpr int kDqTile = 40;  // gamma tile row stride (bf16): conflict-free ldmatrix
+template <int DH>
+__host__ __device__ constexpr int dq_warp_bytes() {
+  return (2 * 32 * (DH + 8) + 16 * kDqTile) * 2;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
     dsa3d_bwd_dq_kernel(const __nv_bfloat16* __restrict__ k, __nv_bfloat16* __restrict__ dq,
@@ -350,15 +365,18 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
                         const int* __restrict__ sorted_ex, const unsigned short* __restrict__ gbox,
                         const unsigned short* __restrict__ bbox, const float2* __restrict__ dft,
                         const Geo g, const SortGeo sg, const BoxGeo bg, const int h0, const int hg) {
-  using S = MmaShape<DH>;
-  constexpr int TS = 40;  // tile row stride (bf16), conflict-free for ldmatrix
-  __shared__ __align__(16) unsigned short tile_sh[4][16 * TS];
+  constexpr int NT = DH / 8;       // n-tiles of dq
+  constexpr int KR = DH + 8;       // staged key row stride (bf16): conflict-free ldmatrix.trans
+  constexpr int CH = DH / 8;       // 16-byte chunks per key row
+  extern __shared__ __align__(16) unsigned char dq_sh[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, qq = lane & 3;
-  unsigned short* tile = tile_sh[warp];
+  unsigned short* kbuf = reinterpret_cast<unsigned short*>(dq_sh + warp * dq_warp_bytes<DH>());
+  unsigned short* tile = kbuf + 2 * 32 * KR;
   const int64_t rs = (int64_t)g.heads * DH;
   const int segw = 16 + g.kw;
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
+  const int r = lane >> 1;  // gather: query row of this lane, stored words (lane & 1) + 2i
 
   for (int64_t row = (int64_t)blockIdx.x * 4 + warp; row < rows; row += (int64_t)gridDim.x * 4) {
     const int hh = (int)(row / ((int64_t)sg.Et * sg.Ey));
@@ -369,84 +387,118 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
     const int qbeg = start[b0], qend = start[b0 + sg.Ex];
     const int ot = et - g.kt, oy = ey - g.kh;
     const __nv_bfloat16* kh_ = k + (int64_t)h * DH;
+    // the box's planes and rows inside the volume
+    const int bt0 = max(0, -ot), bt1 = min(g.kt, g.F - 1 - ot);
+    const int by0 = max(0, -oy), by1 = min(g.kh, g.Hp - 1 - oy);
+    const int nby = by1 - by0 + 1;
+    const int nsteps = (bt1 >= bt0 && by1 >= by0) ? (bt1 - bt0 + 1) * nby : 0;
 
     for (int pos = qbeg; pos < qend;) {
       int X0;
       const int cnt = chunk_len(sorted_ex, pos, qend, g.kw, lane, X0);
-      float acc[S::NT][4];
+      const bool rlive = r < cnt;
+      const float2 d = rlive ? dft[pos + r] : make_float2(0.f, 0.f);
+      const int col0 = rlive ? sorted_ex[pos + r] - g.kw - X0 : 0;
+      float acc[NT][4];
 #pragma unroll
-      for (int j = 0; j < S::NT; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      for (int j = 0; j < NT; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 
-      for (int bt = 0; bt <= g.kt; bt++) {
-        const int t = ot + bt;
-        if (t < 0 || t >= g.F) continue;
-        for (int by = 0; by <= g.kh; by++) {
-          const int y = oy + by;
-          if (y < 0 || y >= g.Hp) continue;
-          // gamma tile: rows = queries, cols = segment keys
-          for (int i = lane; i < 16 * TS / 8; i += 32) reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
-          __syncwarp();
-          {
-            const int r = lane >> 1;
-            if (r < cnt) {
-              const float2 d = dft[pos + r];
-              const int col0 = sorted_ex[pos + r] - g.kw - X0;
-              for (int w = lane & 1; 2 * w < bg.width; w += 2) {
-                float ga[2], be[2];
-                box_word(gbox, bbox, pos + r, bg, g.kt, g.kh, bt, by, w, d.x, d.y, ga, be);
-                tile[r * TS + col0 + 2 * w] = bf16_bits(ga[0]);
-                tile[r * TS + col0 + 2 * w + 1] = bf16_bits(ga[1]);
-              }
-            }
-          }
-          __syncwarp();
-#pragma unroll
-          for (int kk = 0; kk < 2; kk++) {
-            unsigned a[4];
-            const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4) + 16 * kk;
-            ldsm_x4(a, tile + rr * TS + cc);
-            unsigned vw[4][S::VW];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-              const int key = 16 * kk + 2 * qq + (i & 1) + 8 * (i >> 1);
-              const int x = X0 + key;
-              const bool ok = key < segw && x >= 0 && x < g.Wp;
-              const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
-#pragma unroll
-              for (int c = 0; c < S::VW / 4; c++) {
-                const uint4 w = ok ? ldg16(kr + pv_off(c, gq)) : make_uint4(0, 0, 0, 0);
-                vw[i][4 * c] = w.x; vw[i][4 * c + 1] = w.y; vw[i][4 * c + 2] = w.z; vw[i][4 * c + 3] = w.w;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < S::NT; j++) {
-              const int wi = 4 * (j >> 3) + ((j & 7) >> 1);
-              const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
-              const unsigned b0_ = __byte_perm(vw[0][wi], vw[1][wi], sel);
-              const unsigned b1_ = __byte_perm(vw[2][wi], vw[3][wi], sel);
-              mma_bf16_16816(acc[j], a[0], a[1], a[2], a[3], b0_, b1_);
-            }
-          }
-          __syncwarp();
+      // K segment of step i -> buffer b (zero-filled outside the row and the segment)
+      auto issue_k = [&](int i, int b) {
+        const int bt = bt0 + i / nby, by = by0 + i % nby;
+        const __nv_bfloat16* krow = kh_ + (int64_t)((ot + bt) * g.Hp + oy + by) * g.Wp * rs;
+        unsigned short* dst = kbuf + b * 32 * KR;
+#pragma unroll 4
+        for (int c = lane; c < 32 * CH; c += 32) {
+          const int key = c / CH, ch = c - key * CH;
+          const int x = X0 + key;
+          const bool ok = key < segw && x >= 0 && x < g.Wp;
+          cp_async16_zfill(dst + key * KR + ch * 8, krow + (int64_t)min(max(x, 0), g.Wp - 1) * rs + ch * 8, ok);
         }
+        cp_async_commit();
+      };
+      // stored gamma'/beta words of step i for this lane's row: [word][plane bt, bt-1][gamma', beta]
+      unsigned wd[4][4];
+      auto gather_load = [&](int i) {
+        const int bt = bt0 + i / nby, by = by0 + i % nby;
+#pragma unroll
+        for (int ii = 0; ii < 4; ii++) {
+          const int w = (lane & 1) + 2 * ii;
+          wd[ii][0] = wd[ii][1] = wd[ii][2] = wd[ii][3] = 0u;
+          if (!rlive || 2 * w >= bg.width) continue;
+          if (bt < g.kt) {
+            const int64_t o = ((int64_t)(pos + r) * bg.rows + bt * (g.kh + 1) + by) * bg.width + 2 * w;
+            wd[ii][0] = *reinterpret_cast<const unsigned*>(gbox + o);
+            wd[ii][1] = *reinterpret_cast<const unsigned*>(bbox + o);
+          }
+          if (bt >= 1) {
+            const int64_t o = ((int64_t)(pos + r) * bg.rows + (bt - 1) * (g.kh + 1) + by) * bg.width + 2 * w;
+            wd[ii][2] = *reinterpret_cast<const unsigned*>(gbox + o);
+            wd[ii][3] = *reinterpret_cast<const unsigned*>(bbox + o);
+          }
+        }
+      };
+
+      if (nsteps > 0) {
+        issue_k(0, 0);
+        gather_load(0);
       }
+      for (int s = 0; s < nsteps; s++) {
+        // gamma tile of step s: t-mix of (gamma' - D beta) of the tap planes bt and bt-1
+        for (int i = lane; i < 16 * kDqTile / 8; i += 32) reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
+        __syncwarp();
+        if (rlive) {
+#pragma unroll
+          for (int ii = 0; ii < 4; ii++) {
+            const int w = (lane & 1) + 2 * ii;
+            if (2 * w >= bg.width) continue;
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+              const float g0 = bf16_val((unsigned short)(wd[ii][0] >> (16 * e)));
+              const float b0_ = bf16_val((unsigned short)(wd[ii][1] >> (16 * e)));
+              const float g1 = bf16_val((unsigned short)(wd[ii][2] >> (16 * e)));
+              const float b1_ = bf16_val((unsigned short)(wd[ii][3] >> (16 * e)));
+              const float c0 = fmaf(-d.x, b0_, g0), c1 = fmaf(-d.x, b1_, g1);
+              tile[r * kDqTile + col0 + 2 * w + e] = bf16_bits(fmaf(d.y, c1 - c0, c0));
+            }
+          }
+        }
+        const bool more = s + 1 < nsteps;
+        if (more) {
+          issue_k(s + 1, (s + 1) & 1);
+          gather_load(s + 1);
+          cp_async_wait_group1();
+        } else {
+          cp_async_wait_all();
+        }
+        __syncwarp();
+        const unsigned short* kb_ = kbuf + (s & 1) * 32 * KR;
+        const int rr = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+        for (int kk = 0; kk < 2; kk++) {
+          unsigned a[4];
+          ldsm_x4(a, tile + rr * kDqTile + 8 * (lane >> 4) + 16 * kk);
+#pragma unroll
+          for (int j2 = 0; j2 < NT / 2; j2++) {
+            unsigned bq[4];
+            ldsm_x4_trans(bq, kb_ + (16 * kk + rr) * KR + 16 * j2 + 8 * (lane >> 4));
+            mma_bf16_16816(acc[2 * j2], a[0], a[1], a[2], a[3], bq[0], bq[1]);
+            mma_bf16_16816(acc[2 * j2 + 1], a[0], a[1], a[2], a[3], bq[2], bq[3]);
+          }
+        }
+        __syncwarp();
+      }
+      // n-tile j, columns 2q, 2q+1 -> dims 8j + 2q, 8j + 2q + 1
 #pragma unroll
       for (int hf = 0; hf < 2; hf++) {
-        const int r = gq + 8 * hf;
-        if (r >= cnt) continue;
-        const int n = sorted_n[pos + r];
+        const int rq = gq + 8 * hf;
+        if (rq >= cnt) continue;
+        const int n = sorted_n[pos + rq];
         __nv_bfloat16* drow = dq + ((int64_t)n * g.heads + h) * DH;
 #pragma unroll
-        for (int c = 0; c < DH / 64; c++) {
-          float vals[16];
-#pragma unroll
-          for (int e = 0; e < 8; e++) {
-            vals[e] = acc[8 * c + e][2 * hf] * g.scale;
-            vals[8 + e] = acc[8 * c + e][2 * hf + 1] * g.scale;
-          }
-          store16(drow + 64 * c + 16 * qq, vals);
-          store16(drow + 64 * c + 16 * qq + 8, vals + 8);
-        }
+        for (int j = 0; j < NT; j++)
+          *reinterpret_cast<__nv_bfloat162*>(drow + 8 * j + 2 * qq) =
+              __floats2bfloat162_rn(acc[j][2 * hf] * g.scale, acc[j][2 * hf + 1] * g.scale);
       }
       pos += cnt;
     }
@@ -461,8 +513,9 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 // rows e_t = tk - bt + kt, e_y in [yk0, yk0 + kKvRows - 1 + kh] and the e_x range
 // [16b, 16b + 16 + kw).  Per step (16 such queries, in sorted order across those bucket rows)
 // the CTA stages their q and dO rows and its key rows' Gamma^T / Beta^T tiles (key x query,
-// gathered from the stored splats) in shared memory; each warp then adds Gamma^T q and Beta^T dO for its key row with m16n8k16 MMAs (B fragments by
-// ldmatrix.trans of the staged rows).  A query row is loaded once per tile, not once per key row.
+// gathered from the stored splats) in shared memory; each warp then adds Gamma^T q and Beta^T dO
+// for its key row with m16n8k16 MMAs (B fragments by ldmatrix.trans of the staged rows).  A query
+// row is loaded once per tile, not once per key row.
 #ifndef DSA3D_KV_ROWS
 #define DSA3D_KV_ROWS 2
 #endif

@@ -91,6 +91,8 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, boo
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+// wait until at most the most recent commit group is still in flight
+__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // O += tile0 . V[t0, y, seg] + tile1 . V[t0+1, y, seg]: the two bf16 value-weight tiles
 // (16 queries x 32 segment keys, row stride 40) as A operands (ldmatrix), V by byte permutes.
@@ -141,8 +143,8 @@ __device__ __forceinline__ void dsa3d_pv_tile(float (&o)[MmaShape<DH>::NT][4], c
 // the raw scores of box plane u+1 of the first kFwdCacheRows box rows, in fragment order
 // [row][16 values][32 lanes] (computed for tap plane u and reused as the lower plane of tap plane
 // u+1, so those rows' Q.K^T runs once per box plane; rows beyond the cache recompute).
-constexpr int kFwdRaw = 33;
-constexpr int kFwdTap = 16;
+constexpr int kFwdRaw = 40;  // conflict-free float2 stores of MMA fragments
+constexpr int kFwdTap = 18;  // kw <= 15; 18 keeps the two lanes per query row on distinct banks
 constexpr int kFwdTile = 40;  // bf16 per row: 32 columns + pad (conflict-free ldmatrix)
 constexpr int kFwdCacheRows = 9;  // keeps two 4-warp CTAs per SM within 228 KB
 __host__ __device__ constexpr int fwd_mma_warp_bytes() {
@@ -294,8 +296,9 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
 #pragma unroll
             for (int jt = 0; jt < 4; jt++)
 #pragma unroll
-              for (int e = 0; e < 4; e++)
-                rc[(gq + 8 * (e >> 1)) * kFwdRaw + 8 * jt + 2 * qq + (e & 1)] = st[jt][e];
+              for (int hf = 0; hf < 2; hf++)
+                *reinterpret_cast<float2*>(rc + (gq + 8 * hf) * kFwdRaw + 8 * jt + 2 * qq) =
+                    make_float2(st[jt][2 * hf], st[jt][2 * hf + 1]);
           }
           __syncwarp();
           if (by >= 1) {
