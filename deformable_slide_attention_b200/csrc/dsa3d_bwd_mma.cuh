@@ -403,38 +403,51 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 #pragma unroll
       for (int j = 0; j < NT; j++) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 
+      // This lane's part of a K segment copy: keys lane / CH + KPI * i (i < CH), 16-byte chunk
+      // lane % CH.  The segment's x-range is fixed for the chunk, so the per-key source offsets
+      // and the in-row mask are set once here; a step only adds its key row's base.
+      constexpr int KPI = 32 / CH;
+      const int key_l = lane / CH, ch_l = lane % CH;
+      const int64_t src0 = (int64_t)(X0 + key_l) * rs + ch_l * 8;
+      unsigned vmask = 0;
+#pragma unroll
+      for (int i = 0; i < CH; i++) {
+        const int key = key_l + KPI * i, x = X0 + key;
+        vmask |= (key < segw && x >= 0 && x < g.Wp) ? (1u << i) : 0u;
+      }
       // K segment of step i -> buffer b (zero-filled outside the row and the segment)
       auto issue_k = [&](int i, int b) {
         const int bt = bt0 + i / nby, by = by0 + i % nby;
         const __nv_bfloat16* krow = kh_ + (int64_t)((ot + bt) * g.Hp + oy + by) * g.Wp * rs;
-        unsigned short* dst = kbuf + b * 32 * KR;
-#pragma unroll 4
-        for (int c = lane; c < 32 * CH; c += 32) {
-          const int key = c / CH, ch = c - key * CH;
-          const int x = X0 + key;
-          const bool ok = key < segw && x >= 0 && x < g.Wp;
-          cp_async16_zfill(dst + key * KR + ch * 8, krow + (int64_t)min(max(x, 0), g.Wp - 1) * rs + ch * 8, ok);
+        const __nv_bfloat16* src = krow + src0;
+        unsigned short* dst = kbuf + b * 32 * KR + key_l * KR + ch_l * 8;
+#pragma unroll
+        for (int c = 0; c < CH; c++) {
+          const bool ok = (vmask >> c) & 1u;
+          cp_async16_zfill(dst + c * KPI * KR, ok ? src + (int64_t)c * KPI * rs : krow, ok);
         }
         cp_async_commit();
       };
       // stored gamma'/beta words of step i for this lane's row: [word][plane bt, bt-1][gamma', beta]
+      const int64_t gofs = (int64_t)(rlive ? pos + r : pos) * bg.per_q + 2 * (lane & 1);
+      const unsigned short* grow = gbox + gofs;
+      const unsigned short* brow = bbox + gofs;
       unsigned wd[4][4];
       auto gather_load = [&](int i) {
         const int bt = bt0 + i / nby, by = by0 + i % nby;
+        const int o0 = (bt * (g.kh + 1) + by) * bg.width, o1 = o0 - (g.kh + 1) * bg.width;
 #pragma unroll
         for (int ii = 0; ii < 4; ii++) {
           const int w = (lane & 1) + 2 * ii;
           wd[ii][0] = wd[ii][1] = wd[ii][2] = wd[ii][3] = 0u;
           if (!rlive || 2 * w >= bg.width) continue;
           if (bt < g.kt) {
-            const int64_t o = ((int64_t)(pos + r) * bg.rows + bt * (g.kh + 1) + by) * bg.width + 2 * w;
-            wd[ii][0] = *reinterpret_cast<const unsigned*>(gbox + o);
-            wd[ii][1] = *reinterpret_cast<const unsigned*>(bbox + o);
+            wd[ii][0] = *reinterpret_cast<const unsigned*>(grow + o0 + 4 * ii);
+            wd[ii][1] = *reinterpret_cast<const unsigned*>(brow + o0 + 4 * ii);
           }
           if (bt >= 1) {
-            const int64_t o = ((int64_t)(pos + r) * bg.rows + (bt - 1) * (g.kh + 1) + by) * bg.width + 2 * w;
-            wd[ii][2] = *reinterpret_cast<const unsigned*>(gbox + o);
-            wd[ii][3] = *reinterpret_cast<const unsigned*>(bbox + o);
+            wd[ii][2] = *reinterpret_cast<const unsigned*>(grow + o1 + 4 * ii);
+            wd[ii][3] = *reinterpret_cast<const unsigned*>(brow + o1 + 4 * ii);
           }
         }
       };
@@ -525,8 +538,9 @@ constexpr int kKvRanges = 64;  // bucket-row ranges per batch (two per lane of w
 
 // One query slot of a key-side step.
 struct KvSlot {
+  int64_t row;   // element offset of the query's q / dO row
+  int64_t box;   // element offset of the query's stored splats
   int tok;     // token, -1 for an empty slot
-  int pos;     // sorted position (index of the stored splats)
   int bt;      // box plane of the tile's frame in the query's box
   int by0;     // box row of the tile's first key row (may lie outside [0, kh])
   int ox;      // x-origin minus the tile's first key x
@@ -633,10 +647,11 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
           }
           const int pos = r_beg[lo] + (i - r_pre[lo]);
           const int bt = (rb + lo) / ney;
-          m.pos = pos;
           m.bt = bt;
+          m.box = (int64_t)pos * bg.per_q;
           m.by0 = g.kh - ((rb + lo) - bt * ney);  // yk0 - ey + kh
           m.tok = sorted_n[pos];
+          m.row = ((int64_t)m.tok * g.heads + h) * DH;
           m.ox = sorted_ex[pos] - g.kw - x_lo;
           m.d = dft[pos];
         }
@@ -645,13 +660,16 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
       // q and dO rows of step s into buffer s & 1 (zero-filled for empty slots)
       auto stage_rows = [&](int s) {
         const KvSlot* ms = meta[s & 1];
-        for (int i = tid; i < 2 * 16 * (DH / 8); i += kKvThreads) {
-          const int which = i / (16 * (DH / 8));
-          const int rem = i - which * 16 * (DH / 8);
-          const int m = rem / (DH / 8), c = rem - m * (DH / 8);
-          const int n = ms[m].tok;
-          const __nv_bfloat16* src = (which ? dout : q) + ((int64_t)max(n, 0) * g.heads + h) * DH + c * 8;
-          cp_async16_zfill((which ? os[s & 1] : qs[s & 1]) + m * RS + c * 8, src, n >= 0);
+        constexpr int CH = DH / 8;  // 16-byte chunks per row
+        static_assert((2 * 16 * CH) % kKvThreads == 0, "whole copy rounds");
+#pragma unroll
+        for (int k = 0; k < 2 * 16 * CH / kKvThreads; k++) {
+          const int i = tid + k * kKvThreads;
+          const int which = i / (16 * CH);
+          const int m = (i / CH) % 16, c = i % CH;
+          const bool ok = ms[m].tok >= 0;
+          const __nv_bfloat16* src = (which ? dout : q) + (ok ? ms[m].row + c * 8 : 0);
+          cp_async16_zfill((which ? os[s & 1] : qs[s & 1]) + m * RS + c * 8, src, ok);
         }
         cp_async_commit();
       };
@@ -663,19 +681,20 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
         for (int kr = 0; kr < kKvRows; kr++) wd.g0[kr] = wd.b0[kr] = wd.g1[kr] = wd.b1[kr] = 0u;
         const int key0 = m.ox + 2 * gw;
         if (m.tok < 0 || 2 * gw >= bg.width || key0 + 1 < 0 || key0 >= 16) return;
+        const unsigned short* grow = gbox + m.box + 2 * gw;
+        const unsigned short* brow = bbox + m.box + 2 * gw;
+        const int o0 = (m.bt * (g.kh + 1) + m.by0) * bg.width, o1 = o0 - (g.kh + 1) * bg.width;
 #pragma unroll
         for (int kr = 0; kr < kKvRows; kr++) {
           const int by = m.by0 + kr;
           if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
           if (m.bt < g.kt) {
-            const int64_t o = ((int64_t)m.pos * bg.rows + m.bt * (g.kh + 1) + by) * bg.width + 2 * gw;
-            wd.g0[kr] = *reinterpret_cast<const unsigned*>(gbox + o);
-            wd.b0[kr] = *reinterpret_cast<const unsigned*>(bbox + o);
+            wd.g0[kr] = *reinterpret_cast<const unsigned*>(grow + o0 + kr * bg.width);
+            wd.b0[kr] = *reinterpret_cast<const unsigned*>(brow + o0 + kr * bg.width);
           }
           if (m.bt >= 1) {
-            const int64_t o = ((int64_t)m.pos * bg.rows + (m.bt - 1) * (g.kh + 1) + by) * bg.width + 2 * gw;
-            wd.g1[kr] = *reinterpret_cast<const unsigned*>(gbox + o);
-            wd.b1[kr] = *reinterpret_cast<const unsigned*>(bbox + o);
+            wd.g1[kr] = *reinterpret_cast<const unsigned*>(grow + o1 + kr * bg.width);
+            wd.b1[kr] = *reinterpret_cast<const unsigned*>(brow + o1 + kr * bg.width);
           }
         }
       };
