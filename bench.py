@@ -72,6 +72,7 @@ def alg_bytes_per_item(w, kernel):
         "dsa3d_bwd_q_kernel": 4 * w.dh * s + 28,      # q, k, v, dO; offsets, lse -> doffsets
         "dsa3d_bwd_dq_kernel": 2 * w.dh * s,          # k -> dq
         "dsa3d_bwd_kv_kernel": 4 * w.dh * s,          # q, dO -> dk, dv
+        "dsa3d_pair_v_kernel": 2 * w.dh * s,          # v -> paired value rows (workspace)
         "fwd": 4 * w.dh * s + 16,
         "bwd": 8 * w.dh * s + 28,
     }
@@ -253,18 +254,24 @@ def main(argv=None):
     out = torch.empty_like(q)
     lse = torch.empty((w.heads, w.N), dtype=torch.float32, device=dev)
     dq, dk, dv, doff = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(off)
+    # one workspace serves the forward and the backward (they run one after the other on the
+    # stream): all heads at once when that fits in free memory minus a margin, else head groups
     fws_bytes = abi.dsa3d_forward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
-    fws = torch.empty(fws_bytes, dtype=torch.uint8, device=dev) if fws_bytes else None
     full_ws = abi.dsa3d_backward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
     per_head = full_ws // w.heads if full_ws else 0
     free, _ = torch.cuda.mem_get_info(dev)
     margin = 6 << 30
-    heads_per_pass = w.heads if not per_head else max(1, min(w.heads, (free - margin) // per_head))
-    ws = torch.empty(max(per_head * heads_per_pass, 16), dtype=torch.uint8, device=dev)
+    ws_bytes = max(16, min(max(fws_bytes, full_ws), free - margin))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    heads_per_pass = w.heads if not per_head else max(1, min(w.heads, ws_bytes // per_head))
+    fwd_heads = w.heads
+    while fwd_heads > 1 and abi.dsa3d_forward_workspace_bytes(*w.dims, fwd_heads, w.dh, *w.window,
+                                                              code) > ws_bytes:
+        fwd_heads = (fwd_heads + 1) // 2
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        abi.forward(q, k, v, off, w.dims, w.window, out=out, lse=lse, workspace=fws)
+        abi.forward(q, k, v, off, w.dims, w.window, out=out, lse=lse, workspace=ws)
         abi.backward(q, k, v, off, lse, do, w.dims, w.window, workspace=ws, grads=(dq, dk, dv, doff))
 
     def barrier():
@@ -334,7 +341,7 @@ def main(argv=None):
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_leg(args, w, inp, abi, torch, dev, (fws, ws), world, (out, lse, dq, dk, dv, doff))
+        e2e = e2e_leg(args, w, inp, abi, torch, dev, (ws, ws), world, (out, lse, dq, dk, dv, doff))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -346,6 +353,7 @@ def main(argv=None):
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "frames": w.F, "grid": [w.Hp, w.Wp], "tokens": w.N,
                    "heads": w.heads, "dh": w.dh, "window": list(w.window),
+                   "heads_per_forward_pass": fwd_heads,
                    "heads_per_backward_pass": heads_per_pass,
                    "l2": "inputs larger than L2 (each tensor > 126 MB); no flush",
                    "parallelism": f"independent clip per GPU x{world}"},

@@ -181,6 +181,13 @@ size_t sort_ws_bytes(const Shape& s, int hg) {
   const int64_t nb = (cnt + kScanTile - 1) / kScanTile;
   return align16(cnt * 4) + 4 * align16((size_t)hg * s.N * 4) + align16(nb * 4);
 }
+// Forward workspace of a head group: the sort arrays, then the paired value rows
+// (F * Hp * ceil(Wp / 2) pairs of keys x hg heads x dh words).
+int pair_width(const Shape& s) { return (s.Wp + 1) / 2; }
+size_t vpair_bytes(const Shape& s, int hg) {
+  return align16((size_t)s.F * s.Hp * pair_width(s) * hg * s.dh * 4);
+}
+size_t fwd_ws_bytes(const Shape& s, int hg) { return sort_ws_bytes(s, hg) + vpair_bytes(s, hg); }
 SortWs carve_sort_ws(const Shape& s, int hg, void* base) {
   const SortGeo sg = make_sort_geo(s);
   SortWs w;
@@ -215,13 +222,21 @@ dsa3d_status_t zero16(void* p, size_t n16, cudaStream_t st);
 
 template <int DH>
 dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const void* v,
-                             const float* off, void* out, float* lse, const SortWs& w, int h0,
-                             int hg, cudaStream_t st) {
+                             const float* off, void* out, float* lse, const SortWs& w,
+                             unsigned* vp, int h0, int hg, cudaStream_t st) {
   const Geo g = make_geo(s);
   const SortGeo sg = make_sort_geo(s);
+  const int Wp2 = pair_width(s);
   dsa3d_status_t rc = zero16(w.cnt, align16(w.cnt_elems * 4) / 16, st);
   if (rc != DSA3D_OK) return rc;
   const int64_t items = (int64_t)hg * s.N;
+  {
+    TimedLaunch tl(kKernPairV, st);
+    const int64_t pitems = (int64_t)s.F * s.Hp * Wp2 * hg * (DH / 8);
+    dsa3d_pair_v_kernel<DH><<<grid_for(pitems, 256, 16), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(v), vp, g, Wp2, h0, hg);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
   {
     TimedLaunch tl(kKernSortCount, st);
     dsa3d_sort_count_kernel<__nv_bfloat16, DH><<<grid_for(items, 256, 16), 256, 0, st>>>(
@@ -251,8 +266,8 @@ dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const
     TimedLaunch tl(kKernFwdMma, st);
     kern<<<grid, 128, smem, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                static_cast<const __nv_bfloat16*>(v), off,
-                               static_cast<__nv_bfloat16*>(out), lse, w.cnt, w.sorted_n, w.sorted_ex, g,
-                               sg, h0, hg);
+                               static_cast<__nv_bfloat16*>(out), lse, w.cnt, w.sorted_n, w.sorted_ex, vp,
+                               Wp2, g, sg, h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
   return DSA3D_OK;
@@ -497,7 +512,7 @@ dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const 
   if (lse && overlap(ro, rl)) return DSA3D_ERR_INVALID_ARGUMENT;
 
   if (workspace && workspace_bytes > 0 && mma_forward_ok(s, dtype)) {
-    const size_t one = sort_ws_bytes(s, 1);
+    const size_t one = fwd_ws_bytes(s, 1);
     if (workspace_bytes < one) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
     if (!aligned16(workspace)) return DSA3D_ERR_INVALID_ARGUMENT;
     const Range rw = range_of(workspace, workspace_bytes);
@@ -505,13 +520,14 @@ dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const 
       if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
     if (overlap(ro, rw) || (lse && overlap(rl, rw))) return DSA3D_ERR_INVALID_ARGUMENT;
     int hg = heads;
-    while (hg > 1 && sort_ws_bytes(s, hg) > workspace_bytes) hg = (hg + 1) / 2;
+    while (hg > 1 && fwd_ws_bytes(s, hg) > workspace_bytes) hg = (hg + 1) / 2;
     for (int h0 = 0; h0 < heads; h0 += hg) {
       const int n = (heads - h0 < hg) ? heads - h0 : hg;
       const SortWs wn = carve_sort_ws(s, n, workspace);
-      const dsa3d_status_t r = (dh == 128)
-                                   ? fwd_mma_group<128>(s, q, k, v, offsets, out, lse, wn, h0, n, stream)
-                                   : fwd_mma_group<64>(s, q, k, v, offsets, out, lse, wn, h0, n, stream);
+      unsigned* vp = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + sort_ws_bytes(s, n));
+      const dsa3d_status_t r =
+          (dh == 128) ? fwd_mma_group<128>(s, q, k, v, offsets, out, lse, wn, vp, h0, n, stream)
+                      : fwd_mma_group<64>(s, q, k, v, offsets, out, lse, wn, vp, h0, n, stream);
       if (r != DSA3D_OK) return r;
     }
     return DSA3D_OK;
@@ -530,7 +546,7 @@ size_t dsa3d_forward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, i
                                      int kw, dsa3d_dtype_t dtype) {
   const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
   if (check_shape(s, dtype, 0) != DSA3D_OK || !mma_forward_ok(s, dtype)) return 0;
-  return sort_ws_bytes(s, heads);
+  return fwd_ws_bytes(s, heads);
 }
 
 size_t dsa3d_backward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,

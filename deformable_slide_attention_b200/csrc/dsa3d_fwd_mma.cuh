@@ -18,9 +18,9 @@
 //
 // Operand layouts.  S = Q.K^T contracts dh: in k-step s, lane quad position q supplies words 2s
 // and 2s+1 of its dim slice (qk_off), for the Q rows (A) and the key rows (B) alike -- any fixed
-// permutation of dh applied to both operands leaves the dot products unchanged.  O = P.V maps
-// output column n of n-tile j = 8c + e to dim 64c + 8n + e (pv_off), so lane g reads 16-byte
-// chunks of each value row and lane (g, q) owns output dims 64c + 16q + [0, 16).
+// permutation of dh applied to both operands leaves the dot products unchanged.  O = P.V reads
+// the value rows in key pairs (dsa3d_pair_v_kernel) and maps output column n of n-tile j to dim
+// 32 (j / 4) + 4n + j % 4 (pv_word), so lane (g, q) owns output dims 32c + 8q + [0, 8).
 #pragma once
 
 #include "dsa3d_common.cuh"
@@ -56,13 +56,10 @@ struct MmaShape {
   static constexpr int VW = NT / 2;    // 32-bit words in a lane's dim slice of a V row
 };
 
-// Dim slices, chosen so that one 16-byte load instruction of a warp touches as few cache lines
-// as possible.  Q.K^T operands: quad position q holds dims {32c + 8q + [0, 8)}, c < DH/32 (the
-// four q lanes of a key read one contiguous 64-byte span per instruction).  P.V operands and
-// outputs: lane group g holds dims {64c + 8g + [0, 8)}, c < DH/64 (eight g lanes read one
-// 128-byte line per instruction); n-tile j = 8c + e, column n maps to dim 64c + 8n + e.
+// Dim slices of the Q.K^T operands, chosen so that one 16-byte load instruction of a warp
+// touches as few cache lines as possible: quad position q holds dims {32c + 8q + [0, 8)},
+// c < DH/32 (the four q lanes of a key read one contiguous 64-byte span per instruction).
 __device__ __forceinline__ int qk_off(int c, int qq) { return 32 * c + 8 * qq; }
-__device__ __forceinline__ int pv_off(int c, int gq) { return 64 * c + 8 * gq; }
 
 __device__ __forceinline__ unsigned short bf16_bits(float x) {
   const __nv_bfloat16 b = __float2bfloat16_rn(x);
@@ -94,46 +91,80 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // wait until at most the most recent commit group is still in flight
 __device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
+// Paired value rows.  The P.V products take V as the B operand with the keys as the contraction
+// dimension, so each B register holds two consecutive keys of one dim.  The forward first copies
+// the value rows of its head group into that form:
+//   vp[((t * Hp + y) * Wp2 + xp) * hg + hh][d] = (V[(t, y, 2xp)][h0 + hh][d], V[(t, y, 2xp + 1)][..][d])
+// as bf16 pairs (32-bit words), Wp2 = ceil(Wp / 2), zero where 2xp + 1 == Wp.  One thread moves
+// 8 dims of one pair of keys: two 16-byte loads, two 16-byte stores.
+template <int DH>
+__global__ void dsa3d_pair_v_kernel(const __nv_bfloat16* __restrict__ v, unsigned* __restrict__ vp,
+                                    const Geo g, const int Wp2, const int h0, const int hg) {
+  constexpr int CH = DH / 8;
+  const int64_t items = (int64_t)g.F * g.Hp * Wp2 * hg * CH;
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
+       it += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(it % CH);
+    int64_t r = it / CH;
+    const int hh = (int)(r % hg);
+    r /= hg;
+    const int xp = (int)(r % Wp2);
+    const int64_t ty = r / Wp2;  // t * Hp + y
+    const int64_t n0 = ty * g.Wp + 2 * xp;
+    const uint4 a = ldg16(v + (n0 * g.heads + h0 + hh) * DH + 8 * c);
+    const uint4 b = (2 * xp + 1 < g.Wp) ? ldg16(v + ((n0 + 1) * g.heads + h0 + hh) * DH + 8 * c)
+                                        : make_uint4(0, 0, 0, 0);
+    uint4 lo, hi;
+    lo.x = __byte_perm(a.x, b.x, 0x5410); lo.y = __byte_perm(a.x, b.x, 0x7632);
+    lo.z = __byte_perm(a.y, b.y, 0x5410); lo.w = __byte_perm(a.y, b.y, 0x7632);
+    hi.x = __byte_perm(a.z, b.z, 0x5410); hi.y = __byte_perm(a.z, b.z, 0x7632);
+    hi.z = __byte_perm(a.w, b.w, 0x5410); hi.w = __byte_perm(a.w, b.w, 0x7632);
+    uint4* dst = reinterpret_cast<uint4*>(vp + (r * hg + hh) * DH + 8 * c);
+    dst[0] = lo;
+    dst[1] = hi;
+  }
+}
+
+// P.V n-tile j, column n <-> dim 32 (j / 4) + 4 n + j % 4: lane group g then reads words
+// 32c + 4g + [0, 4) of a paired row (eight lanes cover 128 contiguous bytes per instruction), and
+// lane (g, q) owns output dims 32c + 8q + [0, 8).
+__device__ __forceinline__ int pv_word(int c, int gq) { return 32 * c + 4 * gq; }
+
 // O += tile0 . V[t0, y, seg] + tile1 . V[t0+1, y, seg]: the two bf16 value-weight tiles
-// (16 queries x 32 segment keys, row stride 40) as A operands (ldmatrix), V by byte permutes.
+// (16 queries x 32 segment keys from the even key X0e, row stride 40) as A operands (ldmatrix),
+// the paired value rows as B operands (one 16-byte load per four n-tiles).
 template <int DH>
 __device__ __forceinline__ void dsa3d_pv_tile(float (&o)[MmaShape<DH>::NT][4], const unsigned short* tile,
-                                              int t0, int y, int X0, int segw, const __nv_bfloat16* vh,
-                                              int64_t rs, const Geo& g, int lane) {
+                                              int t0, int y, int X0e, const unsigned* vph, int Wp2,
+                                              int hg, const Geo& g, int lane) {
   using S = MmaShape<DH>;
   const int gq = lane >> 2, qq = lane & 3;
   if (y < 0 || y >= g.Hp) return;
+  const int64_t prs = (int64_t)hg * DH;  // words per pair of keys
 #pragma unroll
   for (int pl = 0; pl < 2; pl++) {
     const int t = t0 + pl;
     if (t < 0 || t >= g.F) continue;
+    const unsigned* rowp = vph + (int64_t)(t * g.Hp + y) * Wp2 * prs;
 #pragma unroll
     for (int kk = 0; kk < 2; kk++) {
       unsigned a[4];
       const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4) + 16 * kk;
       ldsm_x4(a, tile + (pl * 16 + rr) * 40 + cc);
-      unsigned vw[4][S::VW];
+      unsigned vw[2][S::NT];  // [keys 2q, 2q+1 | keys 2q+8, 2q+9][n-tile]
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const int key = 16 * kk + 2 * qq + (i & 1) + 8 * (i >> 1);
-        const int x = X0 + key;
-        const bool ok = key < segw && x >= 0 && x < g.Wp;
-        const __nv_bfloat16* vr = vh + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
+      for (int hb = 0; hb < 2; hb++) {
+        const int xp = (X0e >> 1) + 8 * kk + qq + 4 * hb;
+        const bool ok = xp >= 0 && xp < Wp2;
+        const unsigned* src = rowp + (int64_t)max(xp, 0) * prs;
 #pragma unroll
-        for (int c = 0; c < S::VW / 4; c++) {
-          const uint4 w = ok ? ldg16(vr + pv_off(c, gq)) : make_uint4(0, 0, 0, 0);
-          vw[i][4 * c] = w.x; vw[i][4 * c + 1] = w.y; vw[i][4 * c + 2] = w.z; vw[i][4 * c + 3] = w.w;
+        for (int c = 0; c < DH / 32; c++) {
+          const uint4 w = ok ? ldg16(src + pv_word(c, gq)) : make_uint4(0, 0, 0, 0);
+          vw[hb][4 * c] = w.x; vw[hb][4 * c + 1] = w.y; vw[hb][4 * c + 2] = w.z; vw[hb][4 * c + 3] = w.w;
         }
       }
 #pragma unroll
-      for (int j = 0; j < S::NT; j++) {
-        // n-tile j = 8c + e: element e of chunk c is word 4c + e/2, half e & 1
-        const int wi = 4 * (j >> 3) + ((j & 7) >> 1);
-        const unsigned sel = (j & 1) ? 0x7632u : 0x5410u;
-        const unsigned b0 = __byte_perm(vw[0][wi], vw[1][wi], sel);
-        const unsigned b1 = __byte_perm(vw[2][wi], vw[3][wi], sel);
-        mma_bf16_16816(o[j], a[0], a[1], a[2], a[3], b0, b1);
-      }
+      for (int j = 0; j < S::NT; j++) mma_bf16_16816(o[j], a[0], a[1], a[2], a[3], vw[0][j], vw[1][j]);
     }
   }
 }
@@ -157,8 +188,8 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
                          const __nv_bfloat16* __restrict__ v, const float* __restrict__ off,
                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                          const int* __restrict__ start, const int* __restrict__ sorted_n,
-                         const int* __restrict__ sorted_ex, const Geo g, const SortGeo sg,
-                         const int h0, const int hg) {
+                         const int* __restrict__ sorted_ex, const unsigned* __restrict__ vp,
+                         const int Wp2, const Geo g, const SortGeo sg, const int h0, const int hg) {
   using S = MmaShape<DH>;
   extern __shared__ __align__(16) unsigned char fwd_sh[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -182,7 +213,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
     const int qbeg = start[b0], qend = start[b0 + sg.Ex];
     const int ot = et - g.kt, oy = ey - g.kh;
     const __nv_bfloat16* kh_ = k + (int64_t)h * DH;
-    const __nv_bfloat16* vh_ = v + (int64_t)h * DH;
+    const unsigned* vph = vp + (int64_t)hh * DH;
 
     for (int pos = qbeg; pos < qend;) {
       // ---- chunk: <= 16 consecutive queries whose x-origins span <= 16
@@ -191,6 +222,8 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
       const unsigned bal = __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 < 16);
       const int cnt = __popc(bal);
       const int X0 = ex0 - g.kw;
+      const int X0e = X0 - (X0 & 1);  // even start of the value segment (covers [X0, X0 + 16 + kw))
+      const int vsh = X0 - X0e;       // value-tile columns are shifted by this
 
       // fragment rows g, g+8: their tokens and f_t (for the Q operand and the t-blend)
       int fn[2];
@@ -363,12 +396,12 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
                 const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
                 const float bxc = fmaf(efx, q1 - q0, q0), bxp = fmaf(efx, r1 - r0, r0);
                 const float beta = fmaf(efy, bxp - bxc, bxc);
-                tile[er * kFwdTile + eox + bx] = bf16_bits((1.f - eft) * beta);
-                tile[(16 + er) * kFwdTile + eox + bx] = bf16_bits(eft * beta);
+                tile[er * kFwdTile + vsh + eox + bx] = bf16_bits((1.f - eft) * beta);
+                tile[(16 + er) * kFwdTile + vsh + eox + bx] = bf16_bits(eft * beta);
               }
             }
             __syncwarp();
-            dsa3d_pv_tile<DH>(o, tile, ot + u, oy + ty, X0, segw, vh_, rs, g, lane);
+            dsa3d_pv_tile<DH>(o, tile, ot + u, oy + ty, X0e, vph, Wp2, hg, g, lane);
             __syncwarp();
           }
         }
@@ -383,12 +416,12 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
               const float r0 = (bx < g.kw) ? tq[er * kFwdTap + bx] : 0.f;
               const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
               const float beta = efy * fmaf(efx, r1 - r0, r0);
-              tile[er * kFwdTile + eox + bx] = bf16_bits((1.f - eft) * beta);
-              tile[(16 + er) * kFwdTile + eox + bx] = bf16_bits(eft * beta);
+              tile[er * kFwdTile + vsh + eox + bx] = bf16_bits((1.f - eft) * beta);
+              tile[(16 + er) * kFwdTile + vsh + eox + bx] = bf16_bits(eft * beta);
             }
           }
           __syncwarp();
-          dsa3d_pv_tile<DH>(o, tile, ot + u, oy + g.kh, X0, segw, vh_, rs, g, lane);
+          dsa3d_pv_tile<DH>(o, tile, ot + u, oy + g.kh, X0e, vph, Wp2, hg, g, lane);
           __syncwarp();
         }
         cached_plane = u + 1;
@@ -404,15 +437,14 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
         const float inv = 1.f / lt;
         __nv_bfloat16* orow = out + ((int64_t)fn[hf] * g.heads + h) * DH;
 #pragma unroll
-        for (int c = 0; c < DH / 64; c++) {
-          float vals[16];  // dims 64c + 16q + [0, 16): columns 2q then 2q+1 of n-tiles 8c..8c+7
+        for (int c = 0; c < DH / 32; c++) {
+          float vals[8];  // dims 32c + 8q + [0, 8): column 2q then 2q+1 of n-tiles 4c..4c+3
 #pragma unroll
-          for (int e = 0; e < 8; e++) {
-            vals[e] = o[8 * c + e][2 * hf] * inv;
-            vals[8 + e] = o[8 * c + e][2 * hf + 1] * inv;
+          for (int i = 0; i < 4; i++) {
+            vals[i] = o[4 * c + i][2 * hf] * inv;
+            vals[4 + i] = o[4 * c + i][2 * hf + 1] * inv;
           }
-          store16(orow + 64 * c + 16 * qq, vals);
-          store16(orow + 64 * c + 16 * qq + 8, vals + 8);
+          store16(orow + 32 * c + 8 * qq, vals);
         }
       }
       pos += cnt;

@@ -83,7 +83,9 @@ dsa3d_status_t dsa3d_forward(const void *q, const void *k, const void *v, const 
 
 /*
  * Bytes of forward workspace for all heads in one pass (0 if the shape has no tensor-core path,
- * or is invalid).  Per head: 4 * ((F+kt)(Hp+kh)(Wp+kw) + 1 + 4N) bytes, plus scan scratch.
+ * or is invalid).  Per head: 4 * ((F+kt)(Hp+kh)(Wp+kw) + 1 + 4N) bytes for the sort, plus scan
+ * scratch, plus 4 * F * Hp * ceil(Wp/2) * dh bytes for a copy of the head's value rows arranged
+ * in pairs of adjacent keys (the operand form of the tensor-core value products).
  */
 size_t dsa3d_forward_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,
                                      int kw, dsa3d_dtype_t dtype);

@@ -74,10 +74,17 @@ def test_forward_rejects_bad_arguments():
 
 
 def test_forward_workspace_bytes():
-    # per head: 4 * ((F+kt)(Hp+kh)(Wp+kw) + 1) bytes of buckets + 4 * 4N bytes, 16-byte aligned
+    # the sort's arrays (buckets, then key, rank, sorted token and x-origin per query, then the
+    # scan's block sums) and the paired value rows: F Hp ceil(Wp/2) pairs x heads x dh words
+    a16 = lambda b: (b + 15) // 16 * 16
+    for (F, Hp, Wp, H, dh, kt, kh, kw) in ((4, 8, 8, 1, 64, 3, 3, 3), (4, 8, 9, 2, 128, 3, 5, 7)):
+        N = F * Hp * Wp
+        E1 = (F + kt) * (Hp + kh) * (Wp + kw) + 1
+        nb = (H * E1 + 2047) // 2048
+        sort = a16(4 * H * E1) + 4 * a16(4 * H * N) + a16(4 * nb)
+        pairs = a16(F * Hp * ((Wp + 1) // 2) * H * dh * 4)
+        assert abi.dsa3d_forward_workspace_bytes(F, Hp, Wp, H, dh, kt, kh, kw, abi.DSA3D_BF16) == sort + pairs
     one = abi.dsa3d_forward_workspace_bytes(4, 8, 8, 1, 64, 3, 3, 3, abi.DSA3D_BF16)
-    buckets = (4 + 3) * (8 + 3) * (8 + 3) + 1
-    assert one >= 4 * buckets + 4 * 4 * 256
     assert abi.dsa3d_forward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_BF16) > one
     # no tensor-core path: fp32, dh 32, kw > 15
     assert abi.dsa3d_forward_workspace_bytes(4, 8, 8, 2, 64, 3, 3, 3, abi.DSA3D_F32) == 0

@@ -25,16 +25,14 @@ def test_1080p_workload_full_size():
     inp = inputs.make(w, dev, with_dout=True)
     q, k, v, off, do = (inp[n] for n in ("q", "k", "v", "offsets", "dout"))
     code = abi.DSA3D_BF16
-    fws = torch.empty(abi.dsa3d_forward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code),
-                      dtype=torch.uint8, device=dev)
-    out, lse = abi.forward(q, k, v, off, w.dims, w.window, workspace=fws)
-    del fws
-    full_ws = abi.dsa3d_backward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
-    per_head = full_ws // w.heads
+    out, lse = torch.empty_like(q), torch.empty((w.heads, w.N), dtype=torch.float32, device=dev)
     grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(off))
+    # one workspace for both calls, sized as bench.py sizes it
+    fws = abi.dsa3d_forward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
+    full_ws = abi.dsa3d_backward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
     free, _ = torch.cuda.mem_get_info(dev)
-    hpp = max(1, min(w.heads, (free - (6 << 30)) // per_head))
-    ws = torch.empty(per_head * hpp, dtype=torch.uint8, device=dev)
+    ws = torch.empty(max(16, min(max(fws, full_ws), free - (6 << 30))), dtype=torch.uint8, device=dev)
+    out, lse = abi.forward(q, k, v, off, w.dims, w.window, out=out, lse=lse, workspace=ws)
     dq, dk, dv, doff = abi.backward(q, k, v, off, lse, do, w.dims, w.window, workspace=ws, grads=grads)
     torch.cuda.synchronize()
     del ws
