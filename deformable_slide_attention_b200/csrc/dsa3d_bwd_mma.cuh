@@ -6,8 +6,8 @@
 // bucket row whose x-origins span <= 16, 32-key segment per box row).  Three passes, no global
 // atomics:
 //
-//  1. query side (dsa3d_bwd_q_kernel): per tap plane u and box row, Q.K and dO.V of box planes
-//     u and u+1 on tensor cores; per tap: P = exp2(s - lse2), dP, their derivatives along the
+//  1. query side (dsa3d_bwd_q_kernel, two warps per chunk): per tap plane u and box row, Q.K and
+//     dO.V of box planes u and u+1 on tensor cores; per tap: P = exp2(s - lse2), dP, their derivatives along the
 //     three fractional coordinates; per query D = sum P dP and
 //        doff_a = scale (sum P dP ds_a - D sum P ds_a) + sum P dp_a.
 //     It stores, per query and tap plane, the y/x-transposed splats of P (beta) and of P dP
@@ -112,18 +112,22 @@ __device__ __forceinline__ int chunk_len(const int* sorted_ex, int pos, int qend
 }
 
 // ---- pass 1: query side ---------------------------------------------------------------------
-// Per warp and chunk, per tap plane u and box row by: the MMA blocks of box planes u and u+1 for
-// q.K and dO.V are blended in registers to (st = S0 + f_t (S1 - S0), bd = S1 - S0) and
-// (dpt, dbd), and stored in a two-row ring in shared memory.  Then a compact epilogue: two lanes
-// per query, each taking every other tap of tap row by-1 (only the query's kw taps, not all 32
-// segment columns), forms the tap's score, dP, their derivatives along (t, y, x), P and the
-// per-query sums; the taps' P and P dP go to a two-row ring, from which box row by-1's splats
-// (x-transpose, then y-mix with the previous tap row) are stored.
+// Two warps per chunk.  Per tap plane u and box row by, warp 0 of the pair computes the Q.K MMA
+// blocks of box planes u and u+1 and warp 1 the dO.V blocks; each blends its two blocks in
+// registers -- (st = S0 + f_t (S1 - S0), bd = S1 - S0), resp. (dpt, dbd) -- and stores them in a
+// three-slot ring in shared memory, with one pair barrier per box row (a slot is rewritten two
+// box rows after it was read).  Then each warp evaluates eight of the chunk's queries, four lanes
+// per query, each lane taking every fourth tap of tap row by-1 (only the query's kw taps, not the
+// 32 segment columns): the tap's score, dP, their derivatives along (t, y, x), P and the
+// per-query sums.  The taps' P and P dP go to the warp's rows of a two-row tap ring, from which
+// box row by-1's splats (x-transpose, then y-mix with the previous tap row) are stored.
 constexpr int kRawStride = 40;  // floats per row of a raw block (conflict-free float2 fragment stores)
-constexpr int kTapStride = 18;  // floats per row of a tap-row buffer (kw <= 15; 18: conflict-free per-query lanes)
+constexpr int kTapStride = 20;  // floats per row of a tap-row buffer (kw <= 15; 20: four lanes per row
+                                // of eight rows fall on distinct banks)
+constexpr int kBwdqSlots = 3;
 
-__host__ __device__ constexpr int bwdq_warp_floats() {
-  return 2 * 4 * 16 * kRawStride + 2 * 2 * 16 * kTapStride;
+__host__ __device__ constexpr int bwdq_pair_floats() {
+  return kBwdqSlots * 4 * 16 * kRawStride + 2 * 2 * 16 * kTapStride;
 }
 
 template <int DH>
@@ -139,16 +143,20 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
   using S = MmaShape<DH>;
   extern __shared__ __align__(16) float dyn_sh[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = warp >> 1, role = warp & 1;  // role 0: Q.K blocks, role 1: dO.V blocks
   const int gq = lane >> 2, qq = lane & 3;
-  float* raw = dyn_sh + warp * bwdq_warp_floats();         // [ring 2][block 4][16 rows][stride]
-  float* tapb = raw + 2 * 4 * 16 * kRawStride;              // [ring 2][P, PdP][16 rows][stride]
-  const int er = lane >> 1, side = lane & 1;                // epilogue: query row, tap parity
+  float* raw = dyn_sh + pair * bwdq_pair_floats();     // [slot 3][block 4][16 rows][stride]
+  float* tapb = raw + kBwdqSlots * 4 * 16 * kRawStride;  // [ring 2][P, PdP][16 rows][stride]
+  const int er = 8 * role + (lane >> 2), s4 = lane & 3;  // epilogue: query row, tap phase
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
   const int segw = 16 + g.kw;
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
+  const unsigned bar_id = 1 + pair;
+  const __nv_bfloat16* asrc = role ? dout : q;  // A operand rows of this warp
+  int sidx = 0;                                  // box-row steps so far (ring slot = sidx % 3)
 
-  for (int64_t row = (int64_t)blockIdx.x * 4 + warp; row < rows; row += (int64_t)gridDim.x * 4) {
+  for (int64_t row = (int64_t)blockIdx.x * 2 + pair; row < rows; row += (int64_t)gridDim.x * 2) {
     const int hh = (int)(row / ((int64_t)sg.Et * sg.Ey));
     const int rem = (int)(row - (int64_t)hh * sg.Et * sg.Ey);
     const int et = rem / sg.Ey, ey = rem % sg.Ey;
@@ -156,17 +164,15 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
     const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)et * sg.Ey + ey) * sg.Ex;
     const int qbeg = start[b0], qend = start[b0 + sg.Ex];
     const int ot = et - g.kt, oy = ey - g.kh;
-    const __nv_bfloat16* kh_ = k + (int64_t)h * DH;
-    const __nv_bfloat16* vh_ = v + (int64_t)h * DH;
+    const __nv_bfloat16* bsrc = (role ? v : k) + (int64_t)h * DH;  // B operand rows
 
     for (int pos = qbeg; pos < qend;) {
       int X0;
       const int cnt = chunk_len(sorted_ex, pos, qend, g.kw, lane, X0);
       MmaRow R[2];  // fragment rows g, g+8 (for the MMA operands and the t-blend)
       chunk_rows(R, g, off, h, sorted_n, pos, cnt, X0, gq);
-      unsigned qa[S::KS][4], ga[S::KS][4];
-      load_afrags<DH>(qa, q, R, h, g.heads, qq);
-      load_afrags<DH>(ga, dout, R, h, g.heads, qq);
+      unsigned af[S::KS][4];
+      load_afrags<DH>(af, asrc, R, h, g.heads, qq);
       // epilogue row er
       const bool elive = er < cnt;
       const int en = elive ? sorted_n[pos + er] : 0;
@@ -176,47 +182,42 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
       const int lo_t = EQ.lo[0], hi_t = elive ? EQ.hi[0] : -1;
       const float lse2 = elive ? __ldg(lse + (int64_t)h * g.N + en) * kLog2e : 0.f;
       float Dp = 0.f, A[3] = {0.f, 0.f, 0.f}, Bs[3] = {0.f, 0.f, 0.f}, C[3] = {0.f, 0.f, 0.f};
+      const int64_t qbox = (int64_t)(elive ? pos + er : pos) * bg.per_q;
 
       for (int u = 0; u < g.kt; u++) {
         const bool eplane = lo_t <= u && u <= hi_t;
-        for (int i = lane; i < 2 * 2 * 16 * kTapStride; i += 32) tapb[i] = 0.f;
-        for (int by = 0; by <= g.kh; by++) {
+        for (int sk = 0; sk < 4; sk++)
+          for (int c = s4; c < kTapStride; c += 4) tapb[(sk * 16 + er) * kTapStride + c] = 0.f;
+        __syncwarp();
+        for (int by = 0; by <= g.kh; by++, sidx++) {
           const int y = oy + by;
-          float* rc = raw + (by & 1) * 4 * 16 * kRawStride;
+          float* rc = raw + (sidx % kBwdqSlots) * 4 * 16 * kRawStride;
           {
             float s0[4][4], s1[4][4];
-            raw_block<DH>(s0, qa, kh_, ot + u, y, X0, segw, rs, g, gq, qq);
-            raw_block<DH>(s1, qa, kh_, ot + u + 1, y, X0, segw, rs, g, gq, qq);
+            raw_block<DH>(s0, af, bsrc, ot + u, y, X0, segw, rs, g, gq, qq);
+            raw_block<DH>(s1, af, bsrc, ot + u + 1, y, X0, segw, rs, g, gq, qq);
+            float* blk = rc + (2 * role) * 16 * kRawStride;
 #pragma unroll
             for (int jt = 0; jt < 4; jt++)
 #pragma unroll
               for (int hf = 0; hf < 2; hf++) {
                 const int rr = gq + 8 * hf, cc = 8 * jt + 2 * qq;
                 const float d0 = s1[jt][2 * hf] - s0[jt][2 * hf], d1 = s1[jt][2 * hf + 1] - s0[jt][2 * hf + 1];
-                *reinterpret_cast<float2*>(rc + (0 * 16 + rr) * kRawStride + cc) =
+                *reinterpret_cast<float2*>(blk + rr * kRawStride + cc) =
                     make_float2(fmaf(R[hf].f[0], d0, s0[jt][2 * hf]), fmaf(R[hf].f[0], d1, s0[jt][2 * hf + 1]));
-                *reinterpret_cast<float2*>(rc + (1 * 16 + rr) * kRawStride + cc) = make_float2(d0, d1);
-              }
-            raw_block<DH>(s0, ga, vh_, ot + u, y, X0, segw, rs, g, gq, qq);
-            raw_block<DH>(s1, ga, vh_, ot + u + 1, y, X0, segw, rs, g, gq, qq);
-#pragma unroll
-            for (int jt = 0; jt < 4; jt++)
-#pragma unroll
-              for (int hf = 0; hf < 2; hf++) {
-                const int rr = gq + 8 * hf, cc = 8 * jt + 2 * qq;
-                const float d0 = s1[jt][2 * hf] - s0[jt][2 * hf], d1 = s1[jt][2 * hf + 1] - s0[jt][2 * hf + 1];
-                *reinterpret_cast<float2*>(rc + (2 * 16 + rr) * kRawStride + cc) =
-                    make_float2(fmaf(R[hf].f[0], d0, s0[jt][2 * hf]), fmaf(R[hf].f[0], d1, s0[jt][2 * hf + 1]));
-                *reinterpret_cast<float2*>(rc + (3 * 16 + rr) * kRawStride + cc) = make_float2(d0, d1);
+                *reinterpret_cast<float2*>(blk + (16 + rr) * kRawStride + cc) = make_float2(d0, d1);
               }
           }
-          __syncwarp();
+          asm volatile("bar.sync %0, 64;\n" ::"r"(bar_id) : "memory");
           if (by >= 1) {
             const int ty = by - 1;
-            const float* rp = raw + ((by - 1) & 1) * 4 * 16 * kRawStride;
+            const float* rp = raw + ((sidx + kBwdqSlots - 1) % kBwdqSlots) * 4 * 16 * kRawStride;
             float* tp = tapb + (ty & 1) * 2 * 16 * kTapStride;
             const bool erow = eplane && EQ.lo[1] <= ty && ty <= EQ.hi[1];
-            for (int wx = side; wx < g.kw; wx += 2) {
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+              const int wx = s4 + 4 * i;
+              if (wx >= g.kw) break;
               float P = 0.f, PdP = 0.f;
               if (erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
                 const int c = eox + wx;
@@ -250,24 +251,34 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
               tp[(1 * 16 + er) * kTapStride + wx] = PdP;
             }
             __syncwarp();
-            // splat onto box row ty: columns bx of this lane's parity
+            // splat onto box row ty: this lane's column pairs (2w, 2w+1), w = s4, s4 + 4
             const float* tq = tapb + ((ty + 1) & 1) * 2 * 16 * kTapStride;  // tap row ty-1
             if (elive) {
-              const int64_t o = ((int64_t)(pos + er) * bg.rows + u * (g.kh + 1) + ty) * bg.width;
-              for (int bx = side; bx <= g.kw; bx += 2) {
+              const int64_t o = qbox + (u * (g.kh + 1) + ty) * bg.width;
+#pragma unroll
+              for (int j = 0; j < 2; j++) {
+                const int w = s4 + 4 * j;
+                if (2 * w > g.kw) break;
                 float vb[2], vg[2];
 #pragma unroll
-                for (int w = 0; w < 2; w++) {
-                  const float* src = w ? tq : tp;
-                  const float p0 = (bx < g.kw) ? src[er * kTapStride + bx] : 0.f;
-                  const float p1 = (bx >= 1) ? src[er * kTapStride + bx - 1] : 0.f;
-                  const float g0 = (bx < g.kw) ? src[(16 + er) * kTapStride + bx] : 0.f;
-                  const float g1 = (bx >= 1) ? src[(16 + er) * kTapStride + bx - 1] : 0.f;
-                  vb[w] = fmaf(fx, p1 - p0, p0);
-                  vg[w] = fmaf(fx, g1 - g0, g0);
+                for (int e = 0; e < 2; e++) {
+                  const int bx = 2 * w + e;
+                  float cb[2], cg[2];
+#pragma unroll
+                  for (int rw = 0; rw < 2; rw++) {
+                    const float* src = rw ? tq : tp;
+                    const float p0 = (bx < g.kw) ? src[er * kTapStride + bx] : 0.f;
+                    const float p1 = (bx >= 1) ? src[er * kTapStride + bx - 1] : 0.f;
+                    const float g0 = (bx < g.kw) ? src[(16 + er) * kTapStride + bx] : 0.f;
+                    const float g1 = (bx >= 1) ? src[(16 + er) * kTapStride + bx - 1] : 0.f;
+                    cb[rw] = fmaf(fx, p1 - p0, p0);
+                    cg[rw] = fmaf(fx, g1 - g0, g0);
+                  }
+                  vb[e] = fmaf(fy, cb[1] - cb[0], cb[0]);
+                  vg[e] = fmaf(fy, cg[1] - cg[0], cg[0]);
                 }
-                bbox[o + bx] = bf16_bits(fmaf(fy, vb[1] - vb[0], vb[0]));
-                gbox[o + bx] = bf16_bits(fmaf(fy, vg[1] - vg[0], vg[0]));
+                *reinterpret_cast<unsigned*>(bbox + o + 2 * w) = bf16x2_bits(vb[0], vb[1]);
+                *reinterpret_cast<unsigned*>(gbox + o + 2 * w) = bf16x2_bits(vg[0], vg[1]);
               }
             }
             __syncwarp();
@@ -277,35 +288,45 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
         {
           const float* tq = tapb + ((g.kh - 1) & 1) * 2 * 16 * kTapStride;
           if (elive) {
-            const int64_t o = ((int64_t)(pos + er) * bg.rows + u * (g.kh + 1) + g.kh) * bg.width;
-            for (int bx = side; bx <= g.kw; bx += 2) {
-              const float p0 = (bx < g.kw) ? tq[er * kTapStride + bx] : 0.f;
-              const float p1 = (bx >= 1) ? tq[er * kTapStride + bx - 1] : 0.f;
-              const float g0 = (bx < g.kw) ? tq[(16 + er) * kTapStride + bx] : 0.f;
-              const float g1 = (bx >= 1) ? tq[(16 + er) * kTapStride + bx - 1] : 0.f;
-              bbox[o + bx] = bf16_bits(fy * fmaf(fx, p1 - p0, p0));
-              gbox[o + bx] = bf16_bits(fy * fmaf(fx, g1 - g0, g0));
+            const int64_t o = qbox + (u * (g.kh + 1) + g.kh) * bg.width;
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+              const int w = s4 + 4 * j;
+              if (2 * w > g.kw) break;
+              float vb[2], vg[2];
+#pragma unroll
+              for (int e = 0; e < 2; e++) {
+                const int bx = 2 * w + e;
+                const float p0 = (bx < g.kw) ? tq[er * kTapStride + bx] : 0.f;
+                const float p1 = (bx >= 1) ? tq[er * kTapStride + bx - 1] : 0.f;
+                const float g0 = (bx < g.kw) ? tq[(16 + er) * kTapStride + bx] : 0.f;
+                const float g1 = (bx >= 1) ? tq[(16 + er) * kTapStride + bx - 1] : 0.f;
+                vb[e] = fy * fmaf(fx, p1 - p0, p0);
+                vg[e] = fy * fmaf(fx, g1 - g0, g0);
+              }
+              *reinterpret_cast<unsigned*>(bbox + o + 2 * w) = bf16x2_bits(vb[0], vb[1]);
+              *reinterpret_cast<unsigned*>(gbox + o + 2 * w) = bf16x2_bits(vg[0], vg[1]);
             }
           }
         }
         __syncwarp();
       }
 
-      // per-query totals: combine the two lanes of the row, then D, doff, (D, f_t)
-      Dp += __shfl_xor_sync(kFull, Dp, 1);
-      float res[3];
+      // per-query totals: combine the row's four lanes, then D, doff, (D, f_t)
 #pragma unroll
-      for (int ax = 0; ax < 3; ax++) {
-        A[ax] += __shfl_xor_sync(kFull, A[ax], 1);
-        Bs[ax] += __shfl_xor_sync(kFull, Bs[ax], 1);
-        C[ax] += __shfl_xor_sync(kFull, C[ax], 1);
-        res[ax] = fmaf(g.scale, fmaf(-Dp, Bs[ax], A[ax]), C[ax]);
+      for (int d = 1; d <= 2; d <<= 1) {
+        Dp += __shfl_xor_sync(kFull, Dp, d);
+#pragma unroll
+        for (int ax = 0; ax < 3; ax++) {
+          A[ax] += __shfl_xor_sync(kFull, A[ax], d);
+          Bs[ax] += __shfl_xor_sync(kFull, Bs[ax], d);
+          C[ax] += __shfl_xor_sync(kFull, C[ax], d);
+        }
       }
-      if (elive && side == 0) {
+      if (elive && s4 == 0) {
         float* od = doff + ((int64_t)h * g.N + en) * 3;
-        od[0] = res[0];
-        od[1] = res[1];
-        od[2] = res[2];
+#pragma unroll
+        for (int ax = 0; ax < 3; ax++) od[ax] = fmaf(g.scale, fmaf(-Dp, Bs[ax], A[ax]), C[ax]);
         dft[pos + er] = make_float2(Dp, ft);
       }
       pos += cnt;

@@ -17,7 +17,7 @@
 #define DSA3D_MMA_MINB 2
 #endif
 #ifndef DSA3D_BWDQ_MINB
-#define DSA3D_BWDQ_MINB 2
+#define DSA3D_BWDQ_MINB 3
 #endif
 #ifndef DSA3D_DQ_MINB
 #define DSA3D_DQ_MINB 3

@@ -66,6 +66,12 @@ __device__ __forceinline__ unsigned short bf16_bits(float x) {
   return *reinterpret_cast<const unsigned short*>(&b);
 }
 
+// two floats as packed bf16 (round to nearest even), x in the low half
+__device__ __forceinline__ unsigned bf16x2_bits(float x, float y) {
+  const __nv_bfloat162 b = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<const unsigned*>(&b);
+}
+
 __device__ __forceinline__ void ldsm_x4(unsigned (&r)[4], const void* p) {
   const unsigned a = (unsigned)__cvta_generic_to_shared(p);
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
