@@ -49,6 +49,35 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
+# DRAM traffic per (token, head) of each kernel, dram__bytes_read.sum + dram__bytes_write.sum
+# from one ncu capture on the 720p training workload (16 heads x 115,200 tokens per launch),
+# valid while the kernel sources hash to "sources"; the traffic of a launch is this times the
+# (token, head) items it processes (the kernels' traffic grows in proportion to the items).
+NCU_TRAFFIC = {
+    "sources": "49c8ea9acd4717c5",
+    "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
+    "bytes_per_item": {
+        "dsa3d_fwd_mma_kernel": 1081.2,
+        "dsa3d_bwd_q_kernel": 2235.3,
+        "dsa3d_bwd_dq_kernel": 1635.0,
+        "dsa3d_bwd_kv_kernel": 2185.8,
+    },
+}
+
+
+def sources_digest():
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "deformable_slide_attention_b200", "csrc", "*")) +
+                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -162,11 +191,18 @@ def head_inputs_for_oracle(w, inp, head=0):
 
 
 def calibrated_items(w, hin, threads, budget_s):
-    oracle_sample(w, hin, max(threads, 1), 12344, threads)  # warm the inputs' pages
-    t1 = oracle_sample(w, hin, 4 * max(threads, 1), 12345, threads)
-    per_round = t1 / 4  # one item per thread
-    rounds = max(1, int(budget_s / max(per_round, 1e-6)))
-    return rounds * max(threads, 1)
+    """Items (a multiple of the thread count) that take about budget_s: time growing samples until
+    one lasts half a second, so the per-call overhead does not distort the estimate."""
+    threads = max(threads, 1)
+    oracle_sample(w, hin, threads, 12344, threads)  # warm the inputs' pages
+    rounds = 4
+    while True:
+        t = oracle_sample(w, hin, rounds * threads, 12345, threads)
+        if t >= 0.5 or rounds >= (1 << 20):
+            break
+        rounds *= 4
+    per_round = t / rounds  # one item per thread
+    return max(1, int(budget_s / max(per_round, 1e-9))) * threads
 
 
 def cpu_baseline(w, inp, budget_s):
@@ -323,8 +359,13 @@ def main(argv=None):
         items_per_launch = w.heads * w.N / launches_per_step
         alg = alg_bytes_per_item(w, kname) * items_per_launch
         achieved = alg / (avg_ms / 1000.0) / 1e9
+        per_item = NCU_TRAFFIC["bytes_per_item"].get(kname)
+        traffic = (per_item * items_per_launch
+                   if per_item is not None and sources_digest() == NCU_TRAFFIC["sources"] else None)
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": None, "kernel": kname,
+                "frac": achieved / hbm, "traffic": traffic, "traffic_unit": "bytes per launch",
+                "traffic_source": NCU_TRAFFIC["capture"] if traffic is not None else None,
+                "kernel": kname,
                 "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"
                                if peak_src == "measured" else "fallback 6.65 TB/s"}
         mhz = clocks["sm_mhz"] or float(peaks.get("sm_max_mhz", 1965.0))
