@@ -258,11 +258,11 @@ dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const
   }
   {
     auto kern = dsa3d_fwd_mma_kernel<DH>;
-    const int smem = 4 * fwd_mma_warp_bytes();
+    const int smem = 2 * fwd_pair_bytes();  // two warp pairs per CTA
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return DSA3D_ERR_CUDA;
     const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
-    const int grid = grid_for(rows, 4, 1 << 20);  // one row per warp; the scheduler balances rows
+    const int grid = grid_for(rows, 2, 1 << 20);  // one row per warp pair; the scheduler balances rows
     TimedLaunch tl(kKernFwdMma, st);
     kern<<<grid, 128, smem, st>>>(static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                static_cast<const __nv_bfloat16*>(v), off,

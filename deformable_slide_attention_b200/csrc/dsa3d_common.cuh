@@ -14,7 +14,7 @@
 // Minimum resident CTAs per SM requested from the compiler for the tensor-core kernels
 // (trades registers for occupancy).
 #ifndef DSA3D_MMA_MINB
-#define DSA3D_MMA_MINB 2
+#define DSA3D_MMA_MINB 3
 #endif
 #ifndef DSA3D_BWDQ_MINB
 #define DSA3D_BWDQ_MINB 3

@@ -175,19 +175,39 @@ __device__ __forceinline__ void dsa3d_pv_tile(float (&o)[MmaShape<DH>::NT][4], c
   }
 }
 
-// Shared memory per warp of the forward: raw-score ring [2][16][kFwdRaw], tap ring
-// [2][16][kFwdTap] (P of tap rows ty, ty-1), two bf16 value-weight tiles [2][16][kFwdTile], and
-// the raw scores of box plane u+1 of the first kFwdCacheRows box rows, in fragment order
-// [row][16 values][32 lanes] (computed for tap plane u and reused as the lower plane of tap plane
-// u+1, so those rows' Q.K^T runs once per box plane; rows beyond the cache recompute).
-constexpr int kFwdRaw = 40;  // conflict-free float2 stores of MMA fragments
-constexpr int kFwdTap = 18;  // kw <= 15; 18 keeps the two lanes per query row on distinct banks
+// Shared memory of one warp pair of the forward (scores warp S, values warp P):
+//   S only:  raw-score ring [2][16][kFwdRaw]; raw scores of box plane u+1 of the first
+//            kFwdCacheRows box rows in fragment order [row][16 values][32 lanes] (computed for tap
+//            plane u and reused as the lower plane of tap plane u+1, so those rows' Q.K^T runs
+//            once per box plane; rows beyond the cache recompute)
+//   shared:  tap ring [kFwdSlots][16 rows][kFwdTap] of P, each slot followed by 16 floats: the
+//            rows' rescale factors of that tap row, or, in a chunk's last entry, the row sums
+//   P only:  two bf16 value-weight tiles [2][16][kFwdTile]
+constexpr int kFwdRaw = 40;   // conflict-free float2 stores of MMA fragments
+constexpr int kFwdTap = 18;   // kw <= 15; 18 keeps the two lanes per query row on distinct banks
 constexpr int kFwdTile = 40;  // bf16 per row: 32 columns + pad (conflict-free ldmatrix)
-constexpr int kFwdCacheRows = 9;  // keeps two 4-warp CTAs per SM within 228 KB
-__host__ __device__ constexpr int fwd_mma_warp_bytes() {
-  return (2 * 16 * kFwdRaw + 2 * 16 * kFwdTap + kFwdCacheRows * 16 * 32) * 4 + 2 * 16 * kFwdTile * 2;
+constexpr int kFwdCacheRows = 9;
+constexpr int kFwdSlots = 3;  // tap-ring entries: P holds two (tap rows ty-1, ty), S fills the third
+constexpr int kFwdSlotFloats = 16 * kFwdTap + 16;
+__host__ __device__ constexpr int fwd_pair_bytes() {
+  return (2 * 16 * kFwdRaw + kFwdCacheRows * 16 * 32 + kFwdSlots * kFwdSlotFloats) * 4 +
+         2 * 16 * kFwdTile * 2;
 }
 
+__device__ __forceinline__ void named_sync(unsigned id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void named_arrive(unsigned id) {
+  __threadfence_block();
+  asm volatile("bar.arrive %0, 64;\n" ::"r"(id) : "memory");
+}
+
+// Two warps per chunk, specialised.  The scores warp S computes the t-blended raw scores of each
+// box row (Q.K^T on tensor cores, the plane cache above), then the taps of the previous tap row:
+// y/x blends, the online softmax (base 2) and P, which it hands to the values warp P through the
+// tap ring together with the rows' rescale factors.  P rescales O, forms the value weights of the
+// box row (x-splat of the tap row, y-mix with the previous one scaled by the factor) as two bf16
+// tiles and adds [(1-f_t) beta | f_t beta] . [V[u, ty]; V[u+1, ty]] on tensor cores.  Ring entry n
+// lives in slot n % kFwdSlots; named barriers full[s] (S arrives, P waits) and empty[s] (P
+// arrives, S waits) order them.  Both warps walk the same chunks and skip the same planes.
 template <int DH>
 __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
     dsa3d_fwd_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -199,18 +219,21 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
   using S = MmaShape<DH>;
   extern __shared__ __align__(16) unsigned char fwd_sh[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, qq = lane & 3;  // fragment row group / quad position
-  float* raw = reinterpret_cast<float*>(fwd_sh + warp * fwd_mma_warp_bytes());
-  float* tapb = raw + 2 * 16 * kFwdRaw;
-  float* scache = tapb + 2 * 16 * kFwdTap;
-  unsigned short* tile = reinterpret_cast<unsigned short*>(scache + kFwdCacheRows * 16 * 32);
-  const int er = lane >> 1, side = lane & 1;  // epilogue: query row, tap parity
+  const int pair = warp >> 1, role = warp & 1;  // role 0: scores warp, role 1: values warp
+  const int gq = lane >> 2, qq = lane & 3;      // fragment row group / quad position
+  float* raw = reinterpret_cast<float*>(fwd_sh + pair * fwd_pair_bytes());
+  float* scache = raw + 2 * 16 * kFwdRaw;
+  float* ring = scache + kFwdCacheRows * 16 * 32;
+  unsigned short* tile = reinterpret_cast<unsigned short*>(ring + kFwdSlots * kFwdSlotFloats);
+  const unsigned full0 = 1 + 2 * kFwdSlots * pair, empty0 = full0 + kFwdSlots;
+  const int er = lane >> 1, side = lane & 1;  // epilogue / tile rows: query row, tap parity
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
   const int segw = 16 + g.kw;
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
+  int n = 0;  // tap-ring entries of this pair so far
 
-  for (int64_t row = (int64_t)blockIdx.x * 4 + warp; row < rows; row += (int64_t)gridDim.x * 4) {
+  for (int64_t row = (int64_t)blockIdx.x * 2 + pair; row < rows; row += (int64_t)gridDim.x * 2) {
     const int hh = (int)(row / ((int64_t)sg.Et * sg.Ey));
     const int rem = (int)(row - (int64_t)hh * sg.Et * sg.Ey);
     const int et = rem / sg.Ey, ey = rem % sg.Ey;
@@ -218,8 +241,6 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
     const int64_t b0 = (int64_t)hh * sg.E1 + ((int64_t)et * sg.Ey + ey) * sg.Ex;
     const int qbeg = start[b0], qend = start[b0 + sg.Ex];
     const int ot = et - g.kt, oy = ey - g.kh;
-    const __nv_bfloat16* kh_ = k + (int64_t)h * DH;
-    const unsigned* vph = vp + (int64_t)hh * DH;
 
     for (int pos = qbeg; pos < qend;) {
       // ---- chunk: <= 16 consecutive queries whose x-origins span <= 16
@@ -228,234 +249,265 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
       const unsigned bal = __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 < 16);
       const int cnt = __popc(bal);
       const int X0 = ex0 - g.kw;
-      const int X0e = X0 - (X0 & 1);  // even start of the value segment (covers [X0, X0 + 16 + kw))
-      const int vsh = X0 - X0e;       // value-tile columns are shifted by this
 
-      // fragment rows g, g+8: their tokens and f_t (for the Q operand and the t-blend)
+      // fragment rows g, g+8: token, f_t and tap-plane range (the same in both warps)
       int fn[2];
       float fft[2];
       bool flive[2];
+      int flo_t[2], fhi_t[2];
 #pragma unroll
       for (int hf = 0; hf < 2; hf++) {
         const int r = gq + 8 * hf;
         flive[hf] = r < cnt;
         fn[hf] = flive[hf] ? sorted_n[pos + r] : 0;
-        fft[hf] = flive[hf] ? decode_query(g, off, h, fn[hf]).f[0] : 0.f;
+        const Query Fq = decode_query(g, off, h, fn[hf]);
+        fft[hf] = flive[hf] ? Fq.f[0] : 0.f;
+        flo_t[hf] = Fq.lo[0];
+        fhi_t[hf] = flive[hf] ? Fq.hi[0] : -1;
       }
-      unsigned qa[S::KS][4];
-      {
-        unsigned w0[S::QW], w1[S::QW];
-#pragma unroll
-        for (int c = 0; c < S::QW / 4; c++) {
-          uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-          if (flive[0]) a = ldg16(q + ((int64_t)fn[0] * g.heads + h) * DH + qk_off(c, qq));
-          if (flive[1]) b = ldg16(q + ((int64_t)fn[1] * g.heads + h) * DH + qk_off(c, qq));
-          w0[4 * c] = a.x; w0[4 * c + 1] = a.y; w0[4 * c + 2] = a.z; w0[4 * c + 3] = a.w;
-          w1[4 * c] = b.x; w1[4 * c + 1] = b.y; w1[4 * c + 2] = b.z; w1[4 * c + 3] = b.w;
-        }
-#pragma unroll
-        for (int s = 0; s < S::KS; s++) {
-          qa[s][0] = w0[2 * s];
-          qa[s][1] = w1[2 * s];
-          qa[s][2] = w0[2 * s + 1];
-          qa[s][3] = w1[2 * s + 1];
-        }
-      }
-      // epilogue row er
+      // epilogue / tile row er
       const bool elive = er < cnt;
       const int en = elive ? sorted_n[pos + er] : 0;
       const Query EQ = decode_query(g, off, h, en);
       DSA3D_DEVICE_CHECK(!elive || (EQ.ok && EQ.o[0] == ot && EQ.o[1] == oy && EQ.o[2] - X0 >= 0 && EQ.o[2] - X0 < 16));
       const int eox = EQ.o[2] - X0;
       const float eft = EQ.f[0], efy = EQ.f[1], efx = EQ.f[2];
-      const int hi_t = elive ? EQ.hi[0] : -1;
 
-      float o[S::NT][4];
+      if (role == 0) {
+        // ================= scores warp =================
+        const __nv_bfloat16* kh_ = k + (int64_t)h * DH;
+        unsigned qa[S::KS][4];
+        {
+          unsigned w0[S::QW], w1[S::QW];
 #pragma unroll
-      for (int j = 0; j < S::NT; j++) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-      float m = -INFINITY, l = 0.f;  // running max (base 2) and partial sum of row er
-
-      int cached_plane = -1;  // box plane whose raw scores scache holds
-      for (int u = 0; u < g.kt; u++) {
-        const bool eplane = EQ.lo[0] <= u && u <= hi_t;
-        if (!__any_sync(kFull, eplane)) continue;
-        const bool have_u = cached_plane == u;
-        for (int i = lane; i < 2 * 16 * kFwdTap; i += 32) tapb[i] = 0.f;
-        for (int by = 0; by <= g.kh; by++) {
-          const int y = oy + by;
-          float* rc = raw + (by & 1) * 16 * kFwdRaw;
-          const bool cache_row = by < kFwdCacheRows;
-          float* cr = scache + (cache_row ? by : 0) * 16 * 32 + lane;  // + 32 * (4 * jt + e)
-          // t-blended raw scores of box row by -> ring; raw scores of plane u+1 -> cache
-          {
-            float st[4][4];
-#pragma unroll
-            for (int jt = 0; jt < 4; jt++) st[jt][0] = st[jt][1] = st[jt][2] = st[jt][3] = 0.f;
-#pragma unroll
-            for (int pl = 0; pl < 2; pl++) {
-              const int t = ot + u + pl;
-              if (pl == 0 && have_u && cache_row) {  // plane u was computed for tap plane u-1
-#pragma unroll
-                for (int jt = 0; jt < 4; jt++)
-#pragma unroll
-                  for (int e = 0; e < 4; e++) st[jt][e] = (1.f - fft[e >> 1]) * cr[32 * (4 * jt + e)];
-                continue;
-              }
-              if (t < 0 || t >= g.F || y < 0 || y >= g.Hp) {
-                if (pl == 1 && cache_row) {
-#pragma unroll
-                  for (int i = 0; i < 16; i++) cr[32 * i] = 0.f;
-                }
-                continue;
-              }
-#pragma unroll
-              for (int jt = 0; jt < 4; jt++) {
-                const int col = 8 * jt + gq;
-                const int x = X0 + col;
-                const bool ok = col < segw && x >= 0 && x < g.Wp;
-                const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
-                unsigned kw_[S::QW];
-#pragma unroll
-                for (int c = 0; c < S::QW / 4; c++) {
-                  const uint4 a = ok ? ldg16(kr + qk_off(c, qq)) : make_uint4(0, 0, 0, 0);
-                  kw_[4 * c] = a.x; kw_[4 * c + 1] = a.y; kw_[4 * c + 2] = a.z; kw_[4 * c + 3] = a.w;
-                }
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int s = 0; s < S::KS; s++)
-                  mma_bf16_16816(acc, qa[s][0], qa[s][1], qa[s][2], qa[s][3], kw_[2 * s], kw_[2 * s + 1]);
-#pragma unroll
-                for (int e = 0; e < 4; e++) {
-                  const float w = pl ? fft[e >> 1] : 1.f - fft[e >> 1];
-                  st[jt][e] = fmaf(w, acc[e], st[jt][e]);
-                  if (pl == 1 && cache_row) cr[32 * (4 * jt + e)] = acc[e];
-                }
-              }
-            }
-#pragma unroll
-            for (int jt = 0; jt < 4; jt++)
-#pragma unroll
-              for (int hf = 0; hf < 2; hf++)
-                *reinterpret_cast<float2*>(rc + (gq + 8 * hf) * kFwdRaw + 8 * jt + 2 * qq) =
-                    make_float2(st[jt][2 * hf], st[jt][2 * hf + 1]);
+          for (int c = 0; c < S::QW / 4; c++) {
+            uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+            if (flive[0]) a = ldg16(q + ((int64_t)fn[0] * g.heads + h) * DH + qk_off(c, qq));
+            if (flive[1]) b = ldg16(q + ((int64_t)fn[1] * g.heads + h) * DH + qk_off(c, qq));
+            w0[4 * c] = a.x; w0[4 * c + 1] = a.y; w0[4 * c + 2] = a.z; w0[4 * c + 3] = a.w;
+            w1[4 * c] = b.x; w1[4 * c + 1] = b.y; w1[4 * c + 2] = b.z; w1[4 * c + 3] = b.w;
           }
-          __syncwarp();
-          if (by >= 1) {
-            const int ty = by - 1;
-            const float* rp = raw + ((by - 1) & 1) * 16 * kFwdRaw;
-            float* tp = tapb + (ty & 1) * 16 * kFwdTap;
-            float* tq = tapb + ((ty + 1) & 1) * 16 * kFwdTap;  // tap row ty-1
-            const bool erow = eplane && EQ.lo[1] <= ty && ty <= EQ.hi[1];
-            // scores of this lane's taps, row max
-            float sv[8];
-            float mx = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-              const int wx = side + 2 * i;
-              sv[i] = -INFINITY;
-              if (wx < g.kw && erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
-                const int c = eox + wx;
-                const float p0 = rp[er * kFwdRaw + c], p1 = rp[er * kFwdRaw + c + 1];
-                const float c0 = rc[er * kFwdRaw + c], c1 = rc[er * kFwdRaw + c + 1];
-                const float y0 = fmaf(efy, c0 - p0, p0), y1 = fmaf(efy, c1 - p1, p1);
-                sv[i] = fmaf(efx, y1 - y0, y0) * sc;
-                mx = fmaxf(mx, sv[i]);
-              }
-            }
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-            float alpha = 1.f;
-            if (mx > m) {
-              alpha = exp2f(m - mx);  // 0 when m was -inf
-              m = mx;
-            }
-            float ls = 0.f;
+          for (int s = 0; s < S::KS; s++) {
+            qa[s][0] = w0[2 * s];
+            qa[s][1] = w1[2 * s];
+            qa[s][2] = w0[2 * s + 1];
+            qa[s][3] = w1[2 * s + 1];
+          }
+        }
+        const int hi_t = elive ? EQ.hi[0] : -1;
+        float m = -INFINITY, l = 0.f;  // running max (base 2) and partial sum of row er
+        int cached_plane = -1;         // box plane whose raw scores scache holds
+        for (int u = 0; u < g.kt; u++) {
+          const bool fpl = (flo_t[0] <= u && u <= fhi_t[0]) || (flo_t[1] <= u && u <= fhi_t[1]);
+          if (!__any_sync(kFull, fpl)) continue;
+          const bool eplane = EQ.lo[0] <= u && u <= hi_t;
+          const bool have_u = cached_plane == u;
+          for (int by = 0; by <= g.kh; by++) {
+            const int y = oy + by;
+            float* rc = raw + (by & 1) * 16 * kFwdRaw;
+            const bool cache_row = by < kFwdCacheRows;
+            float* cr = scache + (cache_row ? by : 0) * 16 * 32 + lane;  // + 32 * (4 * jt + e)
+            // t-blended raw scores of box row by -> ring; raw scores of plane u+1 -> cache
+            {
+              float st[4][4];
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-              const int wx = side + 2 * i;
-              if (wx < g.kw) {
-                const float p = (sv[i] == -INFINITY) ? 0.f : exp2f(sv[i] - m);
-                tp[er * kFwdTap + wx] = p;
-                ls += p;
-                if (alpha != 1.f) tq[er * kFwdTap + wx] *= alpha;  // rescale tap row ty-1
-              }
-            }
-            l = fmaf(l, alpha, ls);
-            // O rows g, g+8 rescale (alpha of row r is held by lanes 2r, 2r+1)
-            const float a0 = __shfl_sync(kFull, alpha, 2 * gq), a1 = __shfl_sync(kFull, alpha, 2 * (gq + 8));
-            if (__any_sync(kFull, a0 != 1.f || a1 != 1.f)) {
+              for (int jt = 0; jt < 4; jt++) st[jt][0] = st[jt][1] = st[jt][2] = st[jt][3] = 0.f;
 #pragma unroll
-              for (int j = 0; j < S::NT; j++) {
-                o[j][0] *= a0; o[j][1] *= a0;
-                o[j][2] *= a1; o[j][3] *= a1;
+              for (int pl = 0; pl < 2; pl++) {
+                const int t = ot + u + pl;
+                if (pl == 0 && have_u && cache_row) {  // plane u was computed for tap plane u-1
+#pragma unroll
+                  for (int jt = 0; jt < 4; jt++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) st[jt][e] = (1.f - fft[e >> 1]) * cr[32 * (4 * jt + e)];
+                  continue;
+                }
+                if (t < 0 || t >= g.F || y < 0 || y >= g.Hp) {
+                  if (pl == 1 && cache_row) {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) cr[32 * i] = 0.f;
+                  }
+                  continue;
+                }
+#pragma unroll
+                for (int jt = 0; jt < 4; jt++) {
+                  const int col = 8 * jt + gq;
+                  const int x = X0 + col;
+                  const bool ok = col < segw && x >= 0 && x < g.Wp;
+                  const __nv_bfloat16* kr = kh_ + ((int64_t)(t * g.Hp + y) * g.Wp + max(x, 0)) * rs;
+                  unsigned kw_[S::QW];
+#pragma unroll
+                  for (int c = 0; c < S::QW / 4; c++) {
+                    const uint4 a = ok ? ldg16(kr + qk_off(c, qq)) : make_uint4(0, 0, 0, 0);
+                    kw_[4 * c] = a.x; kw_[4 * c + 1] = a.y; kw_[4 * c + 2] = a.z; kw_[4 * c + 3] = a.w;
+                  }
+                  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                  for (int s = 0; s < S::KS; s++)
+                    mma_bf16_16816(acc, qa[s][0], qa[s][1], qa[s][2], qa[s][3], kw_[2 * s], kw_[2 * s + 1]);
+#pragma unroll
+                  for (int e = 0; e < 4; e++) {
+                    const float w = pl ? fft[e >> 1] : 1.f - fft[e >> 1];
+                    st[jt][e] = fmaf(w, acc[e], st[jt][e]);
+                    if (pl == 1 && cache_row) cr[32 * (4 * jt + e)] = acc[e];
+                  }
+                }
               }
+#pragma unroll
+              for (int jt = 0; jt < 4; jt++)
+#pragma unroll
+                for (int hf = 0; hf < 2; hf++)
+                  *reinterpret_cast<float2*>(rc + (gq + 8 * hf) * kFwdRaw + 8 * jt + 2 * qq) =
+                      make_float2(st[jt][2 * hf], st[jt][2 * hf + 1]);
             }
             __syncwarp();
-            // value weights of box row ty, scaled for box planes u (1-f_t) and u+1 (f_t)
+            if (by >= 1) {
+              const int ty = by - 1;
+              const float* rp = raw + ((by - 1) & 1) * 16 * kFwdRaw;
+              const int slot = n % kFwdSlots;
+              if (n >= kFwdSlots) named_sync(empty0 + slot);  // P is done with entry n - slots
+              float* tp = ring + slot * kFwdSlotFloats;
+              const bool erow = eplane && EQ.lo[1] <= ty && ty <= EQ.hi[1];
+              // scores of this lane's taps, row max
+              float sv[8];
+              float mx = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < 8; i++) {
+                const int wx = side + 2 * i;
+                sv[i] = -INFINITY;
+                if (wx < g.kw && erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
+                  const int c = eox + wx;
+                  const float p0 = rp[er * kFwdRaw + c], p1 = rp[er * kFwdRaw + c + 1];
+                  const float c0 = rc[er * kFwdRaw + c], c1 = rc[er * kFwdRaw + c + 1];
+                  const float y0 = fmaf(efy, c0 - p0, p0), y1 = fmaf(efy, c1 - p1, p1);
+                  sv[i] = fmaf(efx, y1 - y0, y0) * sc;
+                  mx = fmaxf(mx, sv[i]);
+                }
+              }
+              mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+              float alpha = 1.f;
+              if (mx > m) {
+                alpha = exp2f(m - mx);  // 0 when m was -inf
+                m = mx;
+              }
+              float ls = 0.f;
+#pragma unroll
+              for (int i = 0; i < 8; i++) {
+                const int wx = side + 2 * i;
+                if (wx < g.kw) {
+                  const float p = (sv[i] == -INFINITY) ? 0.f : exp2f(sv[i] - m);
+                  tp[er * kFwdTap + wx] = p;
+                  ls += p;
+                }
+              }
+              l = fmaf(l, alpha, ls);
+              if (side == 0) tp[16 * kFwdTap + er] = alpha;
+              __syncwarp();
+              named_arrive(full0 + slot);
+              n++;
+            }
+          }
+          cached_plane = u + 1;
+        }
+        // the chunk's last entry: row sums (and lse)
+        const float lt_e = l + __shfl_xor_sync(kFull, l, 1);
+        if (elive && side == 0 && lse) lse[(int64_t)h * g.N + en] = (m + log2f(lt_e)) * kLn2;
+        const int slot = n % kFwdSlots;
+        if (n >= kFwdSlots) named_sync(empty0 + slot);
+        if (side == 0) ring[slot * kFwdSlotFloats + 16 * kFwdTap + er] = lt_e;
+        __syncwarp();
+        named_arrive(full0 + slot);
+        n++;
+      } else {
+        // ================= values warp =================
+        const unsigned* vph = vp + (int64_t)hh * DH;
+        const int X0e = X0 - (X0 & 1);  // even start of the value segment (covers [X0, X0 + 16 + kw))
+        const int vcol = X0 - X0e + eox;  // value-tile column of box column 0 of row er
+        float o[S::NT][4];
+#pragma unroll
+        for (int j = 0; j < S::NT; j++) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        for (int u = 0; u < g.kt; u++) {
+          const bool fpl = (flo_t[0] <= u && u <= fhi_t[0]) || (flo_t[1] <= u && u <= fhi_t[1]);
+          if (!__any_sync(kFull, fpl)) continue;
+          for (int ty = 0; ty <= g.kh; ty++) {
+            // box row ty: tap rows ty (entry n, none for ty == kh) and ty-1 (entry n-1, none for ty == 0)
+            const bool has_cur = ty < g.kh;
+            const float* tp = ring + (n % kFwdSlots) * kFwdSlotFloats;
+            const float* tq = ring + ((n + kFwdSlots - 1) % kFwdSlots) * kFwdSlotFloats;
+            float a_er = 1.f;
+            if (has_cur) {
+              named_sync(full0 + n % kFwdSlots);
+              // O rows g, g+8 rescale by the tap row's factors
+              const float a0 = tp[16 * kFwdTap + gq], a1 = tp[16 * kFwdTap + gq + 8];
+              if (__any_sync(kFull, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+                for (int j = 0; j < S::NT; j++) {
+                  o[j][0] *= a0; o[j][1] *= a0;
+                  o[j][2] *= a1; o[j][3] *= a1;
+                }
+              }
+              a_er = tp[16 * kFwdTap + er];
+            }
+            // value weights of box row ty, scaled for box planes u (1 - f_t) and u+1 (f_t)
             for (int i = lane; i < 2 * 16 * kFwdTile / 8; i += 32)
               reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
             __syncwarp();
             if (elive) {
               for (int bx = side; bx <= g.kw; bx += 2) {
-                const float q0 = (bx < g.kw) ? tp[er * kFwdTap + bx] : 0.f;
-                const float q1 = (bx >= 1) ? tp[er * kFwdTap + bx - 1] : 0.f;
-                const float r0 = (bx < g.kw) ? tq[er * kFwdTap + bx] : 0.f;
-                const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
-                const float bxc = fmaf(efx, q1 - q0, q0), bxp = fmaf(efx, r1 - r0, r0);
+                float bxc = 0.f, bxp = 0.f;
+                if (has_cur) {
+                  const float q0 = (bx < g.kw) ? tp[er * kFwdTap + bx] : 0.f;
+                  const float q1 = (bx >= 1) ? tp[er * kFwdTap + bx - 1] : 0.f;
+                  bxc = fmaf(efx, q1 - q0, q0);
+                }
+                if (ty >= 1) {
+                  const float r0 = (bx < g.kw) ? tq[er * kFwdTap + bx] : 0.f;
+                  const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
+                  bxp = a_er * fmaf(efx, r1 - r0, r0);
+                }
                 const float beta = fmaf(efy, bxp - bxc, bxc);
-                tile[er * kFwdTile + vsh + eox + bx] = bf16_bits((1.f - eft) * beta);
-                tile[(16 + er) * kFwdTile + vsh + eox + bx] = bf16_bits(eft * beta);
+                tile[er * kFwdTile + vcol + bx] = bf16_bits((1.f - eft) * beta);
+                tile[(16 + er) * kFwdTile + vcol + bx] = bf16_bits(eft * beta);
               }
             }
             __syncwarp();
+            if (ty >= 1) named_arrive(empty0 + (n + kFwdSlots - 1) % kFwdSlots);  // tap row ty-1 done
+            if (has_cur) n++;
             dsa3d_pv_tile<DH>(o, tile, ot + u, oy + ty, X0e, vph, Wp2, hg, g, lane);
             __syncwarp();
           }
         }
-        // box row kh: only the y-carry (weight f_y) of tap row kh-1
-        {
-          const float* tq = tapb + ((g.kh - 1) & 1) * 16 * kFwdTap;
-          for (int i = lane; i < 2 * 16 * kFwdTile / 8; i += 32)
-            reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
-          __syncwarp();
-          if (elive) {
-            for (int bx = side; bx <= g.kw; bx += 2) {
-              const float r0 = (bx < g.kw) ? tq[er * kFwdTap + bx] : 0.f;
-              const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
-              const float beta = efy * fmaf(efx, r1 - r0, r0);
-              tile[er * kFwdTile + vsh + eox + bx] = bf16_bits((1.f - eft) * beta);
-              tile[(16 + er) * kFwdTile + vsh + eox + bx] = bf16_bits(eft * beta);
+        // the chunk's last entry: row sums; normalise and store
+        const int slot = n % kFwdSlots;
+        named_sync(full0 + slot);
+        const float* lsum = ring + slot * kFwdSlotFloats + 16 * kFwdTap;
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++) {
+          if (!flive[hf]) continue;
+          const float inv = 1.f / lsum[gq + 8 * hf];
+          __nv_bfloat16* orow = out + ((int64_t)fn[hf] * g.heads + h) * DH;
+#pragma unroll
+          for (int c = 0; c < DH / 32; c++) {
+            float vals[8];  // dims 32c + 8q + [0, 8): column 2q then 2q+1 of n-tiles 4c..4c+3
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+              vals[i] = o[4 * c + i][2 * hf] * inv;
+              vals[4 + i] = o[4 * c + i][2 * hf + 1] * inv;
             }
+            store16(orow + 32 * c + 8 * qq, vals);
           }
-          __syncwarp();
-          dsa3d_pv_tile<DH>(o, tile, ot + u, oy + g.kh, X0e, vph, Wp2, hg, g, lane);
-          __syncwarp();
         }
-        cached_plane = u + 1;
-      }
-
-      // ---- normalise and store (row sums from the epilogue lanes)
-      const float lt_e = l + __shfl_xor_sync(kFull, l, 1);
-      if (elive && side == 0 && lse) lse[(int64_t)h * g.N + en] = (m + log2f(lt_e)) * kLn2;
-#pragma unroll
-      for (int hf = 0; hf < 2; hf++) {
-        const float lt = __shfl_sync(kFull, lt_e, 2 * (gq + 8 * hf));
-        if (!flive[hf]) continue;
-        const float inv = 1.f / lt;
-        __nv_bfloat16* orow = out + ((int64_t)fn[hf] * g.heads + h) * DH;
-#pragma unroll
-        for (int c = 0; c < DH / 32; c++) {
-          float vals[8];  // dims 32c + 8q + [0, 8): column 2q then 2q+1 of n-tiles 4c..4c+3
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            vals[i] = o[4 * c + i][2 * hf] * inv;
-            vals[4 + i] = o[4 * c + i][2 * hf + 1] * inv;
-          }
-          store16(orow + 32 * c + 8 * qq, vals);
-        }
+        __syncwarp();
+        named_arrive(empty0 + slot);
+        n++;
       }
       pos += cnt;
     }
   }
+  // the scores warp takes the values warp's last releases, so every barrier phase completes
+  if (role == 0)
+    for (int m = max(0, n - kFwdSlots); m < n; m++) named_sync(empty0 + m % kFwdSlots);
 }
 
 }  // namespace dsa3d
