@@ -221,9 +221,9 @@ def cpu_baseline(w, inp, budget_s):
 
 def run_reference(args):
     """--impl reference: the CPU oracle, K timed steps of a bounded sample each."""
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return 0
+    from deformable_slide_attention_b200 import ranks
+    if ranks.rank_info().rank != 0:
+        return 0  # rank 0 alone times the oracle; the other ranks exit without work
     import torch
     from deformable_slide_attention_b200 import inputs
     import oracle
@@ -268,11 +268,10 @@ def main(argv=None):
         return run_reference(args)
     import torch
     import torch.distributed as dist
-    from deformable_slide_attention_b200 import abi, build, inputs
+    from deformable_slide_attention_b200 import abi, build, inputs, ranks
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    ri = ranks.rank_info()
+    world, rank, local = ri.world, ri.rank, ri.local
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     torch.cuda.set_device(local)
@@ -283,7 +282,7 @@ def main(argv=None):
     build.build()
 
     base = inputs.BY_NAME[args.workload]
-    w = dataclasses.replace(base, seed=base.seed + 1000 * rank)
+    w = ranks.clip_workload(base, rank)
     inp = inputs.make(w, dev, with_dout=True)
     code = abi.DSA3D_BF16 if w.dtype == "bf16" else abi.DSA3D_F32
     q, k, v, off, do = (inp[n] for n in ("q", "k", "v", "offsets", "dout"))
@@ -337,12 +336,8 @@ def main(argv=None):
     abi.dsa3d_timing_enable(False)
     ktimes = abi.dsa3d_timing_read()
     clocks = sampler.stop()
-    ms = t0.elapsed_time(t1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = w.N * world / (ms / 1000.0)
+    ms = ranks.max_over_ranks(t0.elapsed_time(t1) / args.steps, dev)
+    value = ranks.job_rate(w.N, world, ms)
     launches = sum(n for n, _ in ktimes.values())
 
     peaks, peak_src = measured_peaks()
@@ -461,15 +456,11 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
         step()
     t1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = t0.elapsed_time(t1) / steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    from deformable_slide_attention_b200 import ranks
+    ms = ranks.max_over_ranks(t0.elapsed_time(t1) / steps, dev)
     bi = sum(t.numel() * t.element_size() for t in h_in.values())
     bo = sum(t.numel() * t.element_size() for t in h_out.values())
-    return {"value": w.N * world / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+    return {"value": ranks.job_rate(w.N, world, ms), "unit": UNIT, "ms_per_step": ms, "steps": steps,
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "read_back": sorted(h_out)}
 
 
