@@ -214,71 +214,94 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
             const float* rp = raw + ((sidx + kBwdqSlots - 1) % kBwdqSlots) * 4 * 16 * kRawStride;
             float* tp = tapb + (ty & 1) * 2 * 16 * kTapStride;
             const bool erow = eplane && EQ.lo[1] <= ty && ty <= EQ.hi[1];
+            // this lane's taps form a run [t0, t1) of tap row ty; tap wx blends columns wx and
+            // wx+1, so each column's four blocks are read and y-blended once and kept for the
+            // next tap: Y = y-lerps of blocks 0..3, then the y-differences of blocks 0 and 2
+            {
+              const int run = (g.kw + 3) >> 2;
+              const int t0 = s4 * run, t1 = min(t0 + run, g.kw);
+              float Yp[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-              const int wx = s4 + 4 * i;
-              if (wx >= g.kw) break;
-              float P = 0.f, PdP = 0.f;
-              if (erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
-                const int c = eox + wx;
-                float yl[4][2], dy[2][2];
+              for (int jj = 0; jj <= 4; jj++) {  // run <= 4 taps (kw <= 15): at most 5 columns
+                const int j = t0 + jj;
+                if (j > t1 || t0 >= t1) break;
+                const int c = er * kRawStride + eox + j;
+                float Y[6];
 #pragma unroll
-                for (int b = 0; b < 4; b++)
-#pragma unroll
-                  for (int o = 0; o < 2; o++) {
-                    const float pv = rp[(b * 16 + er) * kRawStride + c + o];
-                    const float cv = rc[(b * 16 + er) * kRawStride + c + o];
-                    yl[b][o] = fmaf(fy, cv - pv, pv);
-                    if (b == 0 || b == 2) dy[b >> 1][o] = cv - pv;
-                  }
-                const float s = fmaf(fx, yl[0][1] - yl[0][0], yl[0][0]);
-                const float dpv = fmaf(fx, yl[2][1] - yl[2][0], yl[2][0]);
-                const float ds[3] = {fmaf(fx, yl[1][1] - yl[1][0], yl[1][0]),
-                                     fmaf(fx, dy[0][1] - dy[0][0], dy[0][0]), yl[0][1] - yl[0][0]};
-                const float dp[3] = {fmaf(fx, yl[3][1] - yl[3][0], yl[3][0]),
-                                     fmaf(fx, dy[1][1] - dy[1][0], dy[1][0]), yl[2][1] - yl[2][0]};
-                P = exp2f(fmaf(s, sc, -lse2));
-                PdP = P * dpv;
-                Dp += PdP;
-#pragma unroll
-                for (int ax = 0; ax < 3; ax++) {
-                  A[ax] = fmaf(PdP, ds[ax], A[ax]);
-                  Bs[ax] = fmaf(P, ds[ax], Bs[ax]);
-                  C[ax] = fmaf(P, dp[ax], C[ax]);
+                for (int b = 0; b < 4; b++) {
+                  const float pv = rp[b * 16 * kRawStride + c], cv = rc[b * 16 * kRawStride + c];
+                  Y[b] = fmaf(fy, cv - pv, pv);
+                  if (b == 0) Y[4] = cv - pv;
+                  if (b == 2) Y[5] = cv - pv;
                 }
+                if (j > t0) {
+                  const int wx = j - 1;
+                  float P = 0.f, PdP = 0.f;
+                  if (erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
+                    const float s = fmaf(fx, Y[0] - Yp[0], Yp[0]);
+                    const float dpv = fmaf(fx, Y[2] - Yp[2], Yp[2]);
+                    const float ds[3] = {fmaf(fx, Y[1] - Yp[1], Yp[1]), fmaf(fx, Y[4] - Yp[4], Yp[4]),
+                                         Y[0] - Yp[0]};
+                    const float dp[3] = {fmaf(fx, Y[3] - Yp[3], Yp[3]), fmaf(fx, Y[5] - Yp[5], Yp[5]),
+                                         Y[2] - Yp[2]};
+                    P = exp2f(fmaf(s, sc, -lse2));
+                    PdP = P * dpv;
+                    Dp += PdP;
+#pragma unroll
+                    for (int ax = 0; ax < 3; ax++) {
+                      A[ax] = fmaf(PdP, ds[ax], A[ax]);
+                      Bs[ax] = fmaf(P, ds[ax], Bs[ax]);
+                      C[ax] = fmaf(P, dp[ax], C[ax]);
+                    }
+                  }
+                  tp[(0 * 16 + er) * kTapStride + wx] = P;
+                  tp[(1 * 16 + er) * kTapStride + wx] = PdP;
+                }
+#pragma unroll
+                for (int e = 0; e < 6; e++) Yp[e] = Y[e];
               }
-              tp[(0 * 16 + er) * kTapStride + wx] = P;
-              tp[(1 * 16 + er) * kTapStride + wx] = PdP;
             }
             __syncwarp();
-            // splat onto box row ty: this lane's column pairs (2w, 2w+1), w = s4, s4 + 4
+            // splat onto box row ty: this lane's run of column pairs [w0, w1); column bx takes
+            // taps bx and bx-1 of each tap row, so tap values roll from one column to the next
             const float* tq = tapb + ((ty + 1) & 1) * 2 * 16 * kTapStride;  // tap row ty-1
-            if (elive) {
-              const int64_t o = qbox + (u * (g.kh + 1) + ty) * bg.width;
-#pragma unroll
-              for (int j = 0; j < 2; j++) {
-                const int w = s4 + 4 * j;
-                if (2 * w > g.kw) break;
-                float vb[2], vg[2];
-#pragma unroll
-                for (int e = 0; e < 2; e++) {
-                  const int bx = 2 * w + e;
-                  float cb[2], cg[2];
-#pragma unroll
-                  for (int rw = 0; rw < 2; rw++) {
-                    const float* src = rw ? tq : tp;
-                    const float p0 = (bx < g.kw) ? src[er * kTapStride + bx] : 0.f;
-                    const float p1 = (bx >= 1) ? src[er * kTapStride + bx - 1] : 0.f;
-                    const float g0 = (bx < g.kw) ? src[(16 + er) * kTapStride + bx] : 0.f;
-                    const float g1 = (bx >= 1) ? src[(16 + er) * kTapStride + bx - 1] : 0.f;
-                    cb[rw] = fmaf(fx, p1 - p0, p0);
-                    cg[rw] = fmaf(fx, g1 - g0, g0);
-                  }
-                  vb[e] = fmaf(fy, cb[1] - cb[0], cb[0]);
-                  vg[e] = fmaf(fy, cg[1] - cg[0], cg[0]);
+            {
+              const int words = bg.width >> 1, wrun = (words + 3) >> 2;
+              const int w0 = s4 * wrun, w1 = min(w0 + wrun, words);
+              if (elive && w0 < w1) {
+                const int64_t o = qbox + (u * (g.kh + 1) + ty) * bg.width;
+                float prv[4];  // taps at bx - 1: tap row ty (P, P dP), tap row ty-1 (P, P dP)
+                {
+                  const int x = 2 * w0 - 1;
+                  const bool in = x >= 0;
+                  prv[0] = in ? tp[er * kTapStride + x] : 0.f;
+                  prv[1] = in ? tp[(16 + er) * kTapStride + x] : 0.f;
+                  prv[2] = in ? tq[er * kTapStride + x] : 0.f;
+                  prv[3] = in ? tq[(16 + er) * kTapStride + x] : 0.f;
                 }
-                *reinterpret_cast<unsigned*>(bbox + o + 2 * w) = bf16x2_bits(vb[0], vb[1]);
-                *reinterpret_cast<unsigned*>(gbox + o + 2 * w) = bf16x2_bits(vg[0], vg[1]);
+#pragma unroll
+                for (int ww = 0; ww < 2; ww++) {  // wrun <= 2 (kw <= 15)
+                  const int w = w0 + ww;
+                  if (w >= w1) break;
+                  float vb[2], vg[2];
+#pragma unroll
+                  for (int e = 0; e < 2; e++) {
+                    const int bx = 2 * w + e;
+                    const bool in = bx < g.kw;
+                    const float cur[4] = {in ? tp[er * kTapStride + bx] : 0.f,
+                                          in ? tp[(16 + er) * kTapStride + bx] : 0.f,
+                                          in ? tq[er * kTapStride + bx] : 0.f,
+                                          in ? tq[(16 + er) * kTapStride + bx] : 0.f};
+                    const float cb0 = fmaf(fx, prv[0] - cur[0], cur[0]), cg0 = fmaf(fx, prv[1] - cur[1], cur[1]);
+                    const float cb1 = fmaf(fx, prv[2] - cur[2], cur[2]), cg1 = fmaf(fx, prv[3] - cur[3], cur[3]);
+                    vb[e] = fmaf(fy, cb1 - cb0, cb0);
+                    vg[e] = fmaf(fy, cg1 - cg0, cg0);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) prv[i] = cur[i];
+                  }
+                  *reinterpret_cast<unsigned*>(bbox + o + 2 * w) = bf16x2_bits(vb[0], vb[1]);
+                  *reinterpret_cast<unsigned*>(gbox + o + 2 * w) = bf16x2_bits(vg[0], vg[1]);
+                }
               }
             }
             __syncwarp();
@@ -287,22 +310,26 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
         // box row kh takes only the y-carry of tap row kh-1
         {
           const float* tq = tapb + ((g.kh - 1) & 1) * 2 * 16 * kTapStride;
-          if (elive) {
+          const int words = bg.width >> 1, wrun = (words + 3) >> 2;
+          const int w0 = s4 * wrun, w1 = min(w0 + wrun, words);
+          if (elive && w0 < w1) {
             const int64_t o = qbox + (u * (g.kh + 1) + g.kh) * bg.width;
+            const int x = 2 * w0 - 1;
+            float prv[2] = {x >= 0 ? tq[er * kTapStride + x] : 0.f, x >= 0 ? tq[(16 + er) * kTapStride + x] : 0.f};
 #pragma unroll
-            for (int j = 0; j < 2; j++) {
-              const int w = s4 + 4 * j;
-              if (2 * w > g.kw) break;
+            for (int ww = 0; ww < 2; ww++) {
+              const int w = w0 + ww;
+              if (w >= w1) break;
               float vb[2], vg[2];
 #pragma unroll
               for (int e = 0; e < 2; e++) {
                 const int bx = 2 * w + e;
-                const float p0 = (bx < g.kw) ? tq[er * kTapStride + bx] : 0.f;
-                const float p1 = (bx >= 1) ? tq[er * kTapStride + bx - 1] : 0.f;
-                const float g0 = (bx < g.kw) ? tq[(16 + er) * kTapStride + bx] : 0.f;
-                const float g1 = (bx >= 1) ? tq[(16 + er) * kTapStride + bx - 1] : 0.f;
-                vb[e] = fy * fmaf(fx, p1 - p0, p0);
-                vg[e] = fy * fmaf(fx, g1 - g0, g0);
+                const bool in = bx < g.kw;
+                const float c0 = in ? tq[er * kTapStride + bx] : 0.f, c1 = in ? tq[(16 + er) * kTapStride + bx] : 0.f;
+                vb[e] = fy * fmaf(fx, prv[0] - c0, c0);
+                vg[e] = fy * fmaf(fx, prv[1] - c1, c1);
+                prv[0] = c0;
+                prv[1] = c1;
               }
               *reinterpret_cast<unsigned*>(bbox + o + 2 * w) = bf16x2_bits(vb[0], vb[1]);
               *reinterpret_cast<unsigned*>(gbox + o + 2 * w) = bf16x2_bits(vg[0], vg[1]);

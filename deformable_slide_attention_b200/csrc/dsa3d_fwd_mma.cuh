@@ -369,20 +369,28 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
               if (n >= kFwdSlots) named_sync(empty0 + slot);  // P is done with entry n - slots
               float* tp = ring + slot * kFwdSlotFloats;
               const bool erow = eplane && EQ.lo[1] <= ty && ty <= EQ.hi[1];
-              // scores of this lane's taps, row max
+              // scores of this lane's taps, a run [t0, t1) of the tap row (tap wx blends columns
+              // wx and wx+1, so each column is read and y-blended once), and the row max
+              const int t0 = side ? (g.kw + 1) >> 1 : 0, t1 = side ? g.kw : (g.kw + 1) >> 1;
               float sv[8];
               float mx = -INFINITY;
+              float Yp;
+              {
+                const int c = er * kFwdRaw + eox + t0;
+                Yp = fmaf(efy, rc[c] - rp[c], rp[c]);
+              }
 #pragma unroll
               for (int i = 0; i < 8; i++) {
-                const int wx = side + 2 * i;
+                const int wx = t0 + i;
                 sv[i] = -INFINITY;
-                if (wx < g.kw && erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
-                  const int c = eox + wx;
-                  const float p0 = rp[er * kFwdRaw + c], p1 = rp[er * kFwdRaw + c + 1];
-                  const float c0 = rc[er * kFwdRaw + c], c1 = rc[er * kFwdRaw + c + 1];
-                  const float y0 = fmaf(efy, c0 - p0, p0), y1 = fmaf(efy, c1 - p1, p1);
-                  sv[i] = fmaf(efx, y1 - y0, y0) * sc;
-                  mx = fmaxf(mx, sv[i]);
+                if (wx < t1) {
+                  const int c = er * kFwdRaw + eox + wx + 1;
+                  const float Y = fmaf(efy, rc[c] - rp[c], rp[c]);
+                  if (erow && wx >= EQ.lo[2] && wx <= EQ.hi[2]) {
+                    sv[i] = fmaf(efx, Y - Yp, Yp) * sc;
+                    mx = fmaxf(mx, sv[i]);
+                  }
+                  Yp = Y;
                 }
               }
               mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
@@ -394,8 +402,8 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
               float ls = 0.f;
 #pragma unroll
               for (int i = 0; i < 8; i++) {
-                const int wx = side + 2 * i;
-                if (wx < g.kw) {
+                const int wx = t0 + i;
+                if (wx < t1) {
                   const float p = (sv[i] == -INFINITY) ? 0.f : exp2f(sv[i] - m);
                   tp[er * kFwdTap + wx] = p;
                   ls += p;
@@ -454,21 +462,24 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
               reinterpret_cast<uint4*>(tile)[i] = make_uint4(0, 0, 0, 0);
             __syncwarp();
             if (elive) {
-              for (int bx = side; bx <= g.kw; bx += 2) {
-                float bxc = 0.f, bxp = 0.f;
-                if (has_cur) {
-                  const float q0 = (bx < g.kw) ? tp[er * kFwdTap + bx] : 0.f;
-                  const float q1 = (bx >= 1) ? tp[er * kFwdTap + bx - 1] : 0.f;
-                  bxc = fmaf(efx, q1 - q0, q0);
-                }
-                if (ty >= 1) {
-                  const float r0 = (bx < g.kw) ? tq[er * kFwdTap + bx] : 0.f;
-                  const float r1 = (bx >= 1) ? tq[er * kFwdTap + bx - 1] : 0.f;
-                  bxp = a_er * fmaf(efx, r1 - r0, r0);
-                }
+              // this lane's run [b0, b1) of the kw + 1 box columns; column bx takes taps bx and
+              // bx-1 of each tap row, so tap values roll from one column to the next
+              const int hb = (g.kw + 2) >> 1;
+              const int b0 = side ? hb : 0, b1 = side ? g.kw + 1 : hb;
+              const bool prev_in = b0 >= 1;
+              float pq = (has_cur && prev_in) ? tp[er * kFwdTap + b0 - 1] : 0.f;
+              float pr = (ty >= 1 && prev_in) ? tq[er * kFwdTap + b0 - 1] : 0.f;
+              for (int bx = b0; bx < b1; bx++) {
+                const bool in = bx < g.kw;
+                const float cq = (has_cur && in) ? tp[er * kFwdTap + bx] : 0.f;
+                const float cr = (ty >= 1 && in) ? tq[er * kFwdTap + bx] : 0.f;
+                const float bxc = fmaf(efx, pq - cq, cq);
+                const float bxp = a_er * fmaf(efx, pr - cr, cr);
                 const float beta = fmaf(efy, bxp - bxc, bxc);
                 tile[er * kFwdTile + vcol + bx] = bf16_bits((1.f - eft) * beta);
                 tile[(16 + er) * kFwdTile + vcol + bx] = bf16_bits(eft * beta);
+                pq = cq;
+                pr = cr;
               }
             }
             __syncwarp();
