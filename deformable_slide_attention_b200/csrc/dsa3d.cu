@@ -362,8 +362,12 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
   }
   {
     const int64_t tiles = (int64_t)hg * s.F * ((s.Hp + kKvRows - 1) / kKvRows) * ((s.Wp + 15) / 16);
+    const int smem = kv_dyn_bytes<DH>();
+    if (cudaFuncSetAttribute(dsa3d_bwd_kv_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return DSA3D_ERR_CUDA;
     TimedLaunch tl(kKernBwdKv, st);
-    dsa3d_bwd_kv_kernel<DH><<<grid_for(tiles, 1, 1 << 20), kKvThreads, 0, st>>>(
+    dsa3d_bwd_kv_kernel<DH><<<grid_for(tiles, 1, 1 << 20), kKvThreads, smem, st>>>(
         qb, ob, static_cast<bf*>(dk), static_cast<bf*>(dv), w.cnt, w.sorted_n, w.sorted_ex, gbox,
         bbox, dft, g, sg, bg, h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;

@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 // head dims, with dK and dV in registers.  The queries whose windows cover the tile have origins
 // o_t = tk - bt, o_y in [yk0 - kh, yk0 + kKvRows - 1], o_x in [16b - kw, 16b + 15], i.e. bucket
 // rows e_t = tk - bt + kt, e_y in [yk0, yk0 + kKvRows - 1 + kh] and the e_x range
-// [16b, 16b + 16 + kw).  Per step (16 such queries, in sorted order across those bucket rows)
+// [16b, 16b + 16 + kw).  Per step (kKvQ such queries, in sorted order across those bucket rows)
 // the CTA stages their q and dO rows and its key rows' Gamma^T / Beta^T tiles (key x query,
 // gathered from the stored splats) in shared memory; each warp then adds Gamma^T q and Beta^T dO
 // for its key row with m16n8k16 MMAs (B fragments by ldmatrix.trans of the staged rows).  A query
@@ -583,6 +583,11 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 constexpr int kKvRows = DSA3D_KV_ROWS;  // key rows per CTA (2 warps each)
 constexpr int kKvThreads = 64 * kKvRows;
 constexpr int kKvRanges = 64;  // bucket-row ranges per batch (two per lane of warp 0)
+#ifndef DSA3D_KV_QPS
+#define DSA3D_KV_QPS 32
+#endif
+constexpr int kKvQ = DSA3D_KV_QPS;  // queries per step (the MMAs' k dimension: 16 per k-step)
+static_assert(kKvQ % 16 == 0 && kKvQ <= 32, "whole k-steps; one warp locates a step's slots");
 
 // One query slot of a key-side step.
 struct KvSlot {
@@ -596,6 +601,11 @@ struct KvSlot {
 };
 
 template <int DH>
+__host__ __device__ constexpr int kv_dyn_bytes() {
+  return (6 * kKvRows * 16 * (kKvQ + 8) + 4 * kKvQ * (DH + 8)) * 2;
+}
+
+template <int DH>
 __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
     dsa3d_bwd_kv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ dout,
                         __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
@@ -605,16 +615,18 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
                         const Geo g, const SortGeo sg, const BoxGeo bg, const int h0, const int hg) {
   constexpr int HALF = DH / 2;  // dims per warp
   constexpr int NTH = HALF / 8; // n-tiles per warp
-  constexpr int TS = 24;        // Gamma/Beta tile row stride (bf16): conflict-free ldmatrix
+  constexpr int TS = kKvQ + 8;  // Gamma/Beta tile row stride (bf16): conflict-free ldmatrix
   constexpr int RS = DH + 8;    // staged q/dO row stride (bf16): conflict-free ldmatrix.trans
   constexpr int TILE = kKvRows * 16 * TS;  // one stage of Gamma^T (or Beta^T) tiles
-  constexpr int WT = kKvThreads / 16;      // gather threads per query slot
-  static_assert(WT >= 8, "a query's stored row (<= 8 words) is gathered by one pass of its threads");
-  __shared__ __align__(16) unsigned short tg[3][TILE];
-  __shared__ __align__(16) unsigned short tb[3][TILE];
-  __shared__ __align__(16) unsigned short qs[2][16 * RS];
-  __shared__ __align__(16) unsigned short os[2][16 * RS];
-  __shared__ KvSlot meta[2][16];
+  constexpr int WT = kKvThreads / kKvQ;    // gather threads per query slot
+  constexpr int NW = (8 + WT - 1) / WT;    // stored words per gather thread (a row has <= 8)
+  // dynamic shared memory: Gamma^T and Beta^T tiles [3 stages][TILE], q and dO rows [2][kKvQ][RS]
+  extern __shared__ __align__(16) unsigned short kv_sh[];
+  unsigned short (*tg)[TILE] = reinterpret_cast<unsigned short (*)[TILE]>(kv_sh);
+  unsigned short (*tb)[TILE] = reinterpret_cast<unsigned short (*)[TILE]>(kv_sh + 3 * TILE);
+  unsigned short (*qs)[kKvQ * RS] = reinterpret_cast<unsigned short (*)[kKvQ * RS]>(kv_sh + 6 * TILE);
+  unsigned short (*os)[kKvQ * RS] = reinterpret_cast<unsigned short (*)[kKvQ * RS]>(kv_sh + 6 * TILE + 2 * kKvQ * RS);
+  __shared__ KvSlot meta[2][kKvQ];
   __shared__ int r_beg[kKvRanges], r_pre[kKvRanges + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, qq = lane & 3;
@@ -644,7 +656,7 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
 
     // The queries covering the tile lie in (kt + 1) x ney bucket-row ranges of the sorted order
     // (range r: bt = r / ney, ey = yk0 + r % ney).  They are taken in batches of up to kKvRanges
-    // ranges, concatenated, and consumed 16 at a time, so a step mixes queries of several bucket
+    // ranges, concatenated, and consumed kKvQ at a time, so a step mixes queries of several bucket
     // rows and only the last step of a batch is partly empty.
     const int ney = min(yk0 + kKvRows - 1 + g.kh, sg.Ey - 1) - yk0 + 1;
     const int nranges = (g.kt + 1) * ney;
@@ -678,15 +690,15 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
       }
       __syncthreads();
       const int total = r_pre[kKvRanges];
-      const int nsteps = (total + 15) / 16;
+      const int nsteps = (total + kKvQ - 1) / kKvQ;
       if (nsteps == 0) continue;
 
-      // slot tid (< 16) of step s: the query's sorted position, box plane, box row of key row
+      // slot tid (< kKvQ) of step s: the query's sorted position, box plane, box row of key row
       // yk0, token, x-origin relative to the tile and (D, f_t); tok = -1 for an empty slot
       auto load_slot = [&](int s) {
         KvSlot m;
         m.tok = -1;
-        const int i = 16 * s + tid;
+        const int i = kKvQ * s + tid;
         if (i < total) {
           int lo = 0, hi = kKvRanges;  // largest r with r_pre[r] <= i (a non-empty range)
           while (hi - lo > 1) {
@@ -709,63 +721,76 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
       auto stage_rows = [&](int s) {
         const KvSlot* ms = meta[s & 1];
         constexpr int CH = DH / 8;  // 16-byte chunks per row
-        static_assert((2 * 16 * CH) % kKvThreads == 0, "whole copy rounds");
+        static_assert((2 * kKvQ * CH) % kKvThreads == 0, "whole copy rounds");
 #pragma unroll
-        for (int k = 0; k < 2 * 16 * CH / kKvThreads; k++) {
+        for (int k = 0; k < 2 * kKvQ * CH / kKvThreads; k++) {
           const int i = tid + k * kKvThreads;
-          const int which = i / (16 * CH);
-          const int m = (i / CH) % 16, c = i % CH;
+          const int which = i / (kKvQ * CH);
+          const int m = (i / CH) % kKvQ, c = i % CH;
           const bool ok = ms[m].tok >= 0;
           const __nv_bfloat16* src = (which ? dout : q) + (ok ? ms[m].row + c * 8 : 0);
           cp_async16_zfill((which ? os[s & 1] : qs[s & 1]) + m * RS + c * 8, src, ok);
         }
         cp_async_commit();
       };
-      // the stored words of step s this thread gathers: per key row, planes bt and bt-1
-      struct Words { unsigned g0[kKvRows], b0[kKvRows], g1[kKvRows], b1[kKvRows]; };
+      // the stored words of step s this thread gathers (words gw + WT iw of the query's rows):
+      // per key row, planes bt and bt-1
+      struct Words { unsigned g0[NW][kKvRows], b0[NW][kKvRows], g1[NW][kKvRows], b1[NW][kKvRows]; };
       auto gather_load = [&](int s, Words& wd, KvSlot& m) {
         m = meta[s & 1][gm];
 #pragma unroll
-        for (int kr = 0; kr < kKvRows; kr++) wd.g0[kr] = wd.b0[kr] = wd.g1[kr] = wd.b1[kr] = 0u;
-        const int key0 = m.ox + 2 * gw;
-        if (m.tok < 0 || 2 * gw >= bg.width || key0 + 1 < 0 || key0 >= 16) return;
-        const unsigned short* grow = gbox + m.box + 2 * gw;
-        const unsigned short* brow = bbox + m.box + 2 * gw;
+        for (int iw = 0; iw < NW; iw++)
+#pragma unroll
+          for (int kr = 0; kr < kKvRows; kr++) wd.g0[iw][kr] = wd.b0[iw][kr] = wd.g1[iw][kr] = wd.b1[iw][kr] = 0u;
+        if (m.tok < 0) return;
         const int o0 = (m.bt * (g.kh + 1) + m.by0) * bg.width, o1 = o0 - (g.kh + 1) * bg.width;
 #pragma unroll
-        for (int kr = 0; kr < kKvRows; kr++) {
-          const int by = m.by0 + kr;
-          if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
-          if (m.bt < g.kt) {
-            wd.g0[kr] = *reinterpret_cast<const unsigned*>(grow + o0 + kr * bg.width);
-            wd.b0[kr] = *reinterpret_cast<const unsigned*>(brow + o0 + kr * bg.width);
-          }
-          if (m.bt >= 1) {
-            wd.g1[kr] = *reinterpret_cast<const unsigned*>(grow + o1 + kr * bg.width);
-            wd.b1[kr] = *reinterpret_cast<const unsigned*>(brow + o1 + kr * bg.width);
+        for (int iw = 0; iw < NW; iw++) {
+          const int w = gw + WT * iw;
+          const int key0 = m.ox + 2 * w;
+          if (2 * w >= bg.width || key0 + 1 < 0 || key0 >= 16) continue;
+          const unsigned short* grow = gbox + m.box + 2 * w;
+          const unsigned short* brow = bbox + m.box + 2 * w;
+#pragma unroll
+          for (int kr = 0; kr < kKvRows; kr++) {
+            const int by = m.by0 + kr;
+            if (by < 0 || by > g.kh || yk0 + kr >= g.Hp) continue;
+            if (m.bt < g.kt) {
+              wd.g0[iw][kr] = *reinterpret_cast<const unsigned*>(grow + o0 + kr * bg.width);
+              wd.b0[iw][kr] = *reinterpret_cast<const unsigned*>(brow + o0 + kr * bg.width);
+            }
+            if (m.bt >= 1) {
+              wd.g1[iw][kr] = *reinterpret_cast<const unsigned*>(grow + o1 + kr * bg.width);
+              wd.b1[iw][kr] = *reinterpret_cast<const unsigned*>(brow + o1 + kr * bg.width);
+            }
           }
         }
       };
       // gamma = t-mix of (gamma' - D beta), beta = t-mix of beta, into the stage's tiles
       auto gather_store = [&](int stage, const Words& wd, const KvSlot& m) {
-        const int key0 = m.ox + 2 * gw;
-        if (m.tok < 0 || 2 * gw >= bg.width || key0 + 1 < 0 || key0 >= 16) return;
+        if (m.tok < 0) return;
         const float D = m.d.x, ft = m.d.y;
 #pragma unroll
-        for (int kr = 0; kr < kKvRows; kr++) {
+        for (int iw = 0; iw < NW; iw++) {
+          const int w = gw + WT * iw;
+          const int key0 = m.ox + 2 * w;
+          if (2 * w >= bg.width || key0 + 1 < 0 || key0 >= 16) continue;
 #pragma unroll
-          for (int e = 0; e < 2; e++) {
-            const int key = key0 + e;
-            if (key < 0 || key >= 16) continue;
-            const float bb0 = bf16_val((unsigned short)(wd.b0[kr] >> (16 * e)));
-            const float gg0 = bf16_val((unsigned short)(wd.g0[kr] >> (16 * e)));
-            const float bb1 = bf16_val((unsigned short)(wd.b1[kr] >> (16 * e)));
-            const float gg1 = bf16_val((unsigned short)(wd.g1[kr] >> (16 * e)));
-            const float be = fmaf(ft, bb1 - bb0, bb0);
-            const float c0 = fmaf(-D, bb0, gg0), c1 = fmaf(-D, bb1, gg1);
-            const float ga = fmaf(ft, c1 - c0, c0);
-            tg[stage][kr * 16 * TS + key * TS + gm] = bf16_bits(ga);
-            tb[stage][kr * 16 * TS + key * TS + gm] = bf16_bits(be);
+          for (int kr = 0; kr < kKvRows; kr++) {
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+              const int key = key0 + e;
+              if (key < 0 || key >= 16) continue;
+              const float bb0 = bf16_val((unsigned short)(wd.b0[iw][kr] >> (16 * e)));
+              const float gg0 = bf16_val((unsigned short)(wd.g0[iw][kr] >> (16 * e)));
+              const float bb1 = bf16_val((unsigned short)(wd.b1[iw][kr] >> (16 * e)));
+              const float gg1 = bf16_val((unsigned short)(wd.g1[iw][kr] >> (16 * e)));
+              const float be = fmaf(ft, bb1 - bb0, bb0);
+              const float c0 = fmaf(-D, bb0, gg0), c1 = fmaf(-D, bb1, gg1);
+              const float ga = fmaf(ft, c1 - c0, c0);
+              tg[stage][kr * 16 * TS + key * TS + gm] = bf16_bits(ga);
+              tb[stage][kr * 16 * TS + key * TS + gm] = bf16_bits(be);
+            }
           }
         }
       };
@@ -777,7 +802,7 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
       };
 
       // prologue: slots of steps 0 and 1, step 0's rows and tiles
-      if (tid < 16) {
+      if (tid < kKvQ) {
         meta[0][tid] = load_slot(0);
         meta[1][tid] = load_slot(1);
       }
@@ -807,33 +832,36 @@ __global__ void __launch_bounds__(kKvThreads, DSA3D_KV_MINB)
         }
         KvSlot next;
         next.tok = -1;
-        if (tid < 16 && s + 2 < nsteps) next = load_slot(s + 2);
+        if (tid < kKvQ && s + 2 < nsteps) next = load_slot(s + 2);
 
         if (myk < g.Hp) {
           const unsigned short* tgs = tg[s % 3] + wr * 16 * TS;
           const unsigned short* tbs = tb[s % 3] + wr * 16 * TS;
           const unsigned short* qsb = qs[s & 1];
           const unsigned short* osb = os[s & 1];
-          unsigned agm[4], abt[4];
           const int rr = (lane & 7) + 8 * ((lane >> 3) & 1), cc = 8 * (lane >> 4);
-          ldsm_x4(agm, tgs + rr * TS + cc);
-          ldsm_x4(abt, tbs + rr * TS + cc);
 #pragma unroll
-          for (int j2 = 0; j2 < NTH / 2; j2++) {
-            // B fragments of n-tiles 2*j2, 2*j2+1: rows = queries (k), cols = dims (n)
-            const int dcol = half * HALF + 16 * j2 + 8 * (lane >> 4);
-            unsigned bq[4], bo[4];
-            ldsm_x4_trans(bq, qsb + rr * RS + dcol);
-            ldsm_x4_trans(bo, osb + rr * RS + dcol);
-            mma_bf16_16816(ak[2 * j2], agm[0], agm[1], agm[2], agm[3], bq[0], bq[1]);
-            mma_bf16_16816(ak[2 * j2 + 1], agm[0], agm[1], agm[2], agm[3], bq[2], bq[3]);
-            mma_bf16_16816(av[2 * j2], abt[0], abt[1], abt[2], abt[3], bo[0], bo[1]);
-            mma_bf16_16816(av[2 * j2 + 1], abt[0], abt[1], abt[2], abt[3], bo[2], bo[3]);
+          for (int kq = 0; kq < kKvQ / 16; kq++) {  // k-steps over the step's queries
+            unsigned agm[4], abt[4];
+            ldsm_x4(agm, tgs + rr * TS + 16 * kq + cc);
+            ldsm_x4(abt, tbs + rr * TS + 16 * kq + cc);
+#pragma unroll
+            for (int j2 = 0; j2 < NTH / 2; j2++) {
+              // B fragments of n-tiles 2*j2, 2*j2+1: rows = queries (k), cols = dims (n)
+              const int dcol = half * HALF + 16 * j2 + 8 * (lane >> 4);
+              unsigned bq[4], bo[4];
+              ldsm_x4_trans(bq, qsb + (16 * kq + rr) * RS + dcol);
+              ldsm_x4_trans(bo, osb + (16 * kq + rr) * RS + dcol);
+              mma_bf16_16816(ak[2 * j2], agm[0], agm[1], agm[2], agm[3], bq[0], bq[1]);
+              mma_bf16_16816(ak[2 * j2 + 1], agm[0], agm[1], agm[2], agm[3], bq[2], bq[3]);
+              mma_bf16_16816(av[2 * j2], abt[0], abt[1], abt[2], abt[3], bo[0], bo[1]);
+              mma_bf16_16816(av[2 * j2 + 1], abt[0], abt[1], abt[2], abt[3], bo[2], bo[3]);
+            }
           }
         }
 
         if (more) gather_store((s + 1) % 3, wd, m);
-        if (tid < 16 && s + 2 < nsteps) meta[s & 1][tid] = next;
+        if (tid < kKvQ && s + 2 < nsteps) meta[s & 1][tid] = next;
         cp_async_wait_all();
         __syncthreads();
       }
