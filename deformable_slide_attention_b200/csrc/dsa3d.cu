@@ -257,7 +257,8 @@ dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
   {
-    auto kern = dsa3d_fwd_mma_kernel<DH>;
+    // the scores warp's tap loops sized for the window: two lanes per query, ceil(kw / 2) taps each
+    auto kern = (s.kw <= 9) ? dsa3d_fwd_mma_kernel<DH, 5> : dsa3d_fwd_mma_kernel<DH, 8>;
     const int smem = 2 * fwd_pair_bytes();  // two warp pairs per CTA
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return DSA3D_ERR_CUDA;

@@ -208,7 +208,8 @@ __device__ __forceinline__ void named_arrive(unsigned id) {
 // tiles and adds [(1-f_t) beta | f_t beta] . [V[u, ty]; V[u+1, ty]] on tensor cores.  Ring entry n
 // lives in slot n % kFwdSlots; named barriers full[s] (S arrives, P waits) and empty[s] (P
 // arrives, S waits) order them.  Both warps walk the same chunks and skip the same planes.
-template <int DH>
+// RUN: the longest run of taps a lane of the scores warp evaluates, ceil(kw / 2) <= RUN
+template <int DH, int RUN>
 __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
     dsa3d_fwd_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                          const __nv_bfloat16* __restrict__ v, const float* __restrict__ off,
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
               // scores of this lane's taps, a run [t0, t1) of the tap row (tap wx blends columns
               // wx and wx+1, so each column is read and y-blended once), and the row max
               const int t0 = side ? (g.kw + 1) >> 1 : 0, t1 = side ? g.kw : (g.kw + 1) >> 1;
-              float sv[8];
+              float sv[RUN];
               float mx = -INFINITY;
               float Yp;
               {
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
                 Yp = fmaf(efy, rc[c] - rp[c], rp[c]);
               }
 #pragma unroll
-              for (int i = 0; i < 8; i++) {
+              for (int i = 0; i < RUN; i++) {
                 const int wx = t0 + i;
                 sv[i] = -INFINITY;
                 if (wx < t1) {
@@ -401,7 +402,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
               }
               float ls = 0.f;
 #pragma unroll
-              for (int i = 0; i < 8; i++) {
+              for (int i = 0; i < RUN; i++) {
                 const int wx = t0 + i;
                 if (wx < t1) {
                   const float p = (sv[i] == -INFINITY) ? 0.f : exp2f(sv[i] - m);
