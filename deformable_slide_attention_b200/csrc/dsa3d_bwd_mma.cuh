@@ -3,8 +3,8 @@
 // Exact derivative of the forward (MegaSlide-DiT, arXiv 2607.22696, Eq. 1) with the tap mask and
 // the integer offset parts held fixed; D = sum_tau P_tau dP_tau (dout . out for the exact out).
 // Queries are sorted by window origin and cut into the forward's chunks (<= 16 queries of one
-// bucket row whose x-origins span <= 16, 32-key segment per box row).  Three passes, no global
-// atomics:
+// bucket row whose x-origins differ by <= chunk_span(kw), 32-key segment per box row).  Three
+// passes, no global atomics:
 //
 //  1. query side (dsa3d_bwd_q_kernel, two warps per chunk): per tap plane u and box row, Q.K and
 //     dO.V of box planes u and u+1 on tensor cores; per tap: P = exp2(s - lse2), dP, their derivatives along the
@@ -106,7 +106,7 @@ __device__ __forceinline__ void chunk_rows(MmaRow (&R)[2], const Geo& g, const f
 __device__ __forceinline__ int chunk_len(const int* sorted_ex, int pos, int qend, int kw, int lane, int& X0) {
   const int ex_l = (lane < 16 && pos + lane < qend) ? sorted_ex[pos + lane] : 0x7fffffff;
   const int ex0 = __shfl_sync(kFull, ex_l, 0);
-  const unsigned bal = __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 < 16);
+  const unsigned bal = __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 <= chunk_span(kw));
   X0 = ex0 - kw;
   return __popc(bal);
 }
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
   const int er = 8 * role + (lane >> 2), s4 = lane & 3;  // epilogue: query row, tap phase
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
-  const int segw = 16 + g.kw;
+  const int segw = segment_keys(g.kw);
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
   const unsigned bar_id = 1 + pair;
   const __nv_bfloat16* asrc = role ? dout : q;  // A operand rows of this warp
@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
   unsigned short* kbuf = reinterpret_cast<unsigned short*>(dq_sh + warp * dq_warp_bytes<DH>());
   unsigned short* tile = kbuf + 2 * 32 * KR;
   const int64_t rs = (int64_t)g.heads * DH;
-  const int segw = 16 + g.kw;
+  const int segw = segment_keys(g.kw);
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
   const int r = lane >> 1;  // gather: query row of this lane, stored words (lane & 1) + 2i
 

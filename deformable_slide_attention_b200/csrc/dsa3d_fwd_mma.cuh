@@ -2,9 +2,10 @@
 //
 // Input: queries sorted by box origin (dsa3d_sort.cuh).  One warp takes one bucket row (all
 // queries sharing the origin's t and y) and cuts it into chunks of at most 16 queries whose
-// x-origins span at most 16.  For a chunk, box row (bt, by) of every query lies in key row
-// (o_t + bt, o_y + by) inside the 32-key segment [X0, X0 + 32), X0 = the chunk's smallest
-// x-origin.  Per tap plane u and box row by:
+// x-origins differ by at most chunk_span(kw) = 30 - kw.  For a chunk, box row (bt, by) of every
+// query lies in key row (o_t + bt, o_y + by) inside the 32-key segment [X0, X0 + 32), X0 = the
+// chunk's smallest x-origin (and inside the 32 keys from the even key at or below X0, which the
+// value products use).  Per tap plane u and box row by:
 //   S_t  = (1-f_t) * Q.K[u, by]^T + f_t * Q.K[u+1, by]^T        (m16n8k16 MMAs, fp32 blend)
 //   taps of row ty = by-1:  s = x-lerp(y-lerp(S_t[by-1], S_t[by]))  masked per query
 //   online softmax (base 2) over the taps, P = exp2(s - m)
@@ -39,11 +40,17 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], unsigned a0, unsig
 
 __device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
+// Largest difference of x-origins within a chunk: box columns ox - X0 + [0, kw] then stay below
+// 31, so they fit the 32-key segment from X0 and, shifted by X0's parity, the one from the even key
+// below it.  segment_keys(kw) = keys of the segment any box column can reach.
+__host__ __device__ constexpr int chunk_span(int kw) { return 30 - kw; }
+__host__ __device__ constexpr int segment_keys(int kw) { return chunk_span(kw) + kw + 1; }
+
 // Per-row state of a chunk (rows g and g+8 of the lane).
 struct MmaRow {
   bool live;        // row holds a query
   int n;            // token
-  int ox;           // x-origin minus X0, in [0, 16)
+  int ox;           // x-origin minus X0, in [0, chunk_span(kw)]
   float f[3];
   int lo[3], hi[3];
 };
@@ -230,7 +237,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
   const int er = lane >> 1, side = lane & 1;  // epilogue / tile rows: query row, tap parity
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
-  const int segw = 16 + g.kw;
+  const int segw = segment_keys(g.kw);
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
   int n = 0;  // tap-ring entries of this pair so far
 
@@ -244,10 +251,11 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
     const int ot = et - g.kt, oy = ey - g.kh;
 
     for (int pos = qbeg; pos < qend;) {
-      // ---- chunk: <= 16 consecutive queries whose x-origins span <= 16
+      // ---- chunk: <= 16 consecutive queries whose x-origins differ by <= chunk_span(kw)
       const int ex_l = (lane < 16 && pos + lane < qend) ? sorted_ex[pos + lane] : 0x7fffffff;
       const int ex0 = __shfl_sync(kFull, ex_l, 0);
-      const unsigned bal = __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 < 16);
+      const unsigned bal =
+          __ballot_sync(kFull, lane < 16 && pos + lane < qend && ex_l - ex0 <= chunk_span(g.kw));
       const int cnt = __popc(bal);
       const int X0 = ex0 - g.kw;
 
@@ -270,7 +278,7 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
       const bool elive = er < cnt;
       const int en = elive ? sorted_n[pos + er] : 0;
       const Query EQ = decode_query(g, off, h, en);
-      DSA3D_DEVICE_CHECK(!elive || (EQ.ok && EQ.o[0] == ot && EQ.o[1] == oy && EQ.o[2] - X0 >= 0 && EQ.o[2] - X0 < 16));
+      DSA3D_DEVICE_CHECK(!elive || (EQ.ok && EQ.o[0] == ot && EQ.o[1] == oy && EQ.o[2] - X0 >= 0 && EQ.o[2] - X0 <= chunk_span(g.kw)));
       const int eox = EQ.o[2] - X0;
       const float eft = EQ.f[0], efy = EQ.f[1], efx = EQ.f[2];
 
