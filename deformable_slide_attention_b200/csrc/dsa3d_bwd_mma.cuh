@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(128, DSA3D_DQ_MINB)
 // for its key row with m16n8k16 MMAs (B fragments by ldmatrix.trans of the staged rows).  A query
 // row is loaded once per tile, not once per key row.
 #ifndef DSA3D_KV_ROWS
-#define DSA3D_KV_ROWS 2
+#define DSA3D_KV_ROWS 4
 #endif
 constexpr int kKvRows = DSA3D_KV_ROWS;  // key rows per CTA (2 warps each)
 constexpr int kKvThreads = 64 * kKvRows;

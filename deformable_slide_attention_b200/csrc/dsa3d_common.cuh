@@ -23,7 +23,7 @@
 #define DSA3D_DQ_MINB 3
 #endif
 #ifndef DSA3D_KV_MINB
-#define DSA3D_KV_MINB 4
+#define DSA3D_KV_MINB 2
 #endif
 
 namespace dsa3d {
