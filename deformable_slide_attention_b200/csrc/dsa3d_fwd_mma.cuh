@@ -193,8 +193,15 @@ __device__ __forceinline__ void dsa3d_pv_tile(float (&o)[MmaShape<DH>::NT][4], c
 constexpr int kFwdRaw = 40;   // conflict-free float2 stores of MMA fragments
 constexpr int kFwdTap = 18;   // kw <= 15; 18 keeps the two lanes per query row on distinct banks
 constexpr int kFwdTile = 40;  // bf16 per row: 32 columns + pad (conflict-free ldmatrix)
-constexpr int kFwdCacheRows = 9;
-constexpr int kFwdSlots = 3;  // tap-ring entries: P holds two (tap rows ty-1, ty), S fills the third
+#ifndef DSA3D_FWD_CACHE_ROWS
+#define DSA3D_FWD_CACHE_ROWS 10
+#endif
+#ifndef DSA3D_FWD_SLOTS
+#define DSA3D_FWD_SLOTS 4
+#endif
+constexpr int kFwdCacheRows = DSA3D_FWD_CACHE_ROWS;
+constexpr int kFwdSlots = DSA3D_FWD_SLOTS;  // tap-ring entries: P holds two (tap rows ty-1, ty)
+static_assert(kFwdSlots >= 3 && 2 * 2 * kFwdSlots <= 16, "two pairs' full and empty barriers fit the 16 ids");
 constexpr int kFwdSlotFloats = 16 * kFwdTap + 16;
 __host__ __device__ constexpr int fwd_pair_bytes() {
   return (2 * 16 * kFwdRaw + kFwdCacheRows * 16 * 32 + kFwdSlots * kFwdSlotFloats) * 4 +
@@ -233,7 +240,8 @@ __global__ void __launch_bounds__(128, DSA3D_MMA_MINB)
   float* scache = raw + 2 * 16 * kFwdRaw;
   float* ring = scache + kFwdCacheRows * 16 * 32;
   unsigned short* tile = reinterpret_cast<unsigned short*>(ring + kFwdSlots * kFwdSlotFloats);
-  const unsigned full0 = 1 + 2 * kFwdSlots * pair, empty0 = full0 + kFwdSlots;
+  // named barrier ids (this kernel uses no __syncthreads, so id 0 is free when 16 ids are needed)
+  const unsigned full0 = (2 * 2 * kFwdSlots < 16 ? 1 : 0) + 2 * kFwdSlots * pair, empty0 = full0 + kFwdSlots;
   const int er = lane >> 1, side = lane & 1;  // epilogue / tile rows: query row, tap parity
   const int64_t rs = (int64_t)g.heads * DH;
   const float sc = g.scale * kLog2e;
