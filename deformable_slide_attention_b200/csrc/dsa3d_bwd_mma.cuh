@@ -7,17 +7,18 @@
 // passes, no global atomics:
 //
 //  1. query side (dsa3d_bwd_q_kernel, two warps per chunk): per tap plane u and box row, Q.K and
-//     dO.V of box planes u and u+1 on tensor cores; per tap: P = exp2(s - lse2), dP, their derivatives along the
-//     three fractional coordinates; per query D = sum P dP and
+//     dO.V of box planes u and u+1 on tensor cores; per tap: P = exp2(s - lse2), dP, their
+//     derivatives along the three fractional coordinates; per query D = sum P dP and
 //        doff_a = scale (sum P dP ds_a - D sum P ds_a) + sum P dp_a.
 //     It stores, per query and tap plane, the y/x-transposed splats of P (beta) and of P dP
 //     (gamma') onto the box rows, in bf16: box[pos][u][by][bx], and D, f_t per query.
 //  2. dq (dsa3d_bwd_dq_kernel): dq = scale sum_j gamma[j] K[j], gamma = gamma' - D beta and the
 //     t-mix of the two tap planes feeding each box plane, as tensor-core products per box row
 //     (K segments staged in shared memory by cp.async, one step ahead).
-//  3. key side (dsa3d_bwd_kv_kernel): one warp owns 16 keys x dh/2 dims of one key row and
-//     gathers, from the bucket ranges of the queries whose boxes cover those keys, the stored
-//     gamma/beta rows: dK += scale Gamma^T Q, dV += Beta^T dO on tensor cores, written once.
+//  3. key side (dsa3d_bwd_kv_kernel): one warp owns 16 keys x dh/2 dims of one key row (a CTA
+//     owns kKvRows rows) and gathers, from the bucket ranges of the queries whose boxes cover
+//     those keys, the stored gamma/beta rows, kKvQ queries per step: dK += scale Gamma^T Q,
+//     dV += Beta^T dO on tensor cores, written once.
 #pragma once
 
 #include "dsa3d_fwd_mma.cuh"

@@ -1,6 +1,6 @@
 // dsa3d_fwd_mma.cuh -- 3D-DSA forward on tensor cores (bf16 I/O, dh 64 or 128, k_w <= 15).
 //
-// Input: queries sorted by box origin (dsa3d_sort.cuh).  One warp takes one bucket row (all
+// Input: queries sorted by box origin (dsa3d_sort.cuh).  One warp pair takes one bucket row (all
 // queries sharing the origin's t and y) and cuts it into chunks of at most 16 queries whose
 // x-origins differ by at most chunk_span(kw) = 30 - kw.  For a chunk, box row (bt, by) of every
 // query lies in key row (o_t + bt, o_y + by) inside the 32-key segment [X0, X0 + 32), X0 = the
@@ -11,11 +11,12 @@
 //   online softmax (base 2) over the taps, P = exp2(s - m)
 //   value weights of box row ty: beta = y-mix of the x-transposed P of tap rows ty and ty-1
 //   O += [(1-f_t) beta | f_t beta] . [V[u, ty]; V[u+1, ty]]     (MMAs, beta as bf16 A operand)
-// The blended raw scores of each box row go to a two-row ring in shared memory; two lanes per
-// query then evaluate only that query's taps (online softmax per query), keep the taps' P in a
-// two-row ring, and write the value weights of the box row as two bf16 tiles (scaled by 1-f_t and
-// f_t), which ldmatrix turns back into A operands of the P.V MMAs.  Only rows of valid queries
-// exist here (the sort drops the rest).
+// The pair is warp-specialised (see dsa3d_fwd_mma_kernel): the scores warp writes the blended
+// raw scores of each box row to a two-row ring in shared memory, and two of its lanes per query
+// evaluate only that query's taps (online softmax per query); the taps' P go through a tap ring
+// to the values warp, which writes the value weights of the box row as two bf16 tiles (scaled by
+// 1-f_t and f_t) that ldmatrix turns back into A operands of the P.V MMAs.  Only rows of valid
+// queries exist here (the sort drops the rest).
 //
 // Operand layouts.  S = Q.K^T contracts dh: in k-step s, lane quad position q supplies words 2s
 // and 2s+1 of its dim slice (qk_off), for the Q rows (A) and the key rows (B) alike -- any fixed

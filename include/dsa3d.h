@@ -29,7 +29,8 @@
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; 0 = the legacy default
  *     stream).  The returned status covers argument validation and launch errors only; a later
  *     device-side failure surfaces through CUDA's own error reporting or dsa3d_check_device.
- *   - The library allocates no device memory.  The backward takes a caller-owned workspace.
+ *   - The library allocates no device memory.  The forward (for its tensor-core path) and the
+ *     backward take a caller-owned workspace.
  *   - Supported: dh in {32, 64, 128}; odd window sizes 1 <= k <= 2*dim - 1 on each axis;
  *     every extent >= 1; N*heads*dh < 2^62.  Other shapes return DSA3D_ERR_UNSUPPORTED.
  *   - Thread safety: calls on different streams may run concurrently.
@@ -123,11 +124,13 @@ dsa3d_status_t dsa3d_backward(const void *q, const void *k, const void *v, const
  * with no workspace argument, and steps that must not pay cudaMalloc's device-wide
  * synchronisation.  Arguments, results and errors are those of dsa3d_backward.
  *
- * Its scratch (the fp32 dK/dV accumulators of one head group) is a file-scope device array of
- * DSA3D_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the library holds
- * until the process exits.  Heads are processed in groups that fit; a problem whose single head
- * needs more than the array (2 * N * dh * 4 bytes with bf16 I/O; fp32 I/O needs none) is
- * rejected with DSA3D_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ * Its scratch is a file-scope device array of DSA3D_NOALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits, passed to dsa3d_backward
+ * as the workspace: the tensor-core path runs when one head's sort and stored splats fit it, the
+ * general path when one head's fp32 dK/dV accumulators fit; heads are processed in groups that
+ * fit.  A problem whose single head needs more than the array for the accumulators
+ * (2 * N * dh * 4 bytes with bf16 I/O; fp32 I/O needs none) is rejected with
+ * DSA3D_ERR_WORKSPACE_TOO_SMALL before anything is launched.
  * The first call on each device looks up the array's device address (on the current device) and
  * caches it; make that first call before any stream capture.  The array is shared by every call
  * and keeps the previous call's contents (the accumulators are cleared before use): calls that
