@@ -54,13 +54,13 @@ def parse_args(argv=None):
 # valid while the kernel sources hash to "sources"; the traffic of a launch is this times the
 # (token, head) items it processes (the kernels' traffic grows in proportion to the items).
 NCU_TRAFFIC = {
-    "sources": "a823319245b7d97e",
+    "sources": "ade4806829a0e1b6",
     "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
     "bytes_per_item": {
-        "dsa3d_fwd_mma_kernel": 1084.7,
-        "dsa3d_bwd_q_kernel": 2259.0,
-        "dsa3d_bwd_dq_kernel": 1649.2,
-        "dsa3d_bwd_kv_kernel": 2211.8,
+        "dsa3d_fwd_mma_kernel": 1086.2,
+        "dsa3d_bwd_q_kernel": 2260.3,
+        "dsa3d_bwd_dq_kernel": 1652.0,
+        "dsa3d_bwd_kv_kernel": 2213.6,
     },
 }
 
