@@ -11,7 +11,6 @@
 #include "dsa3d.h"
 #include "dsa3d_bwd.cuh"
 #include "dsa3d_bwd_mma.cuh"
-#include "dsa3d_dq_tc.cuh"
 #include "dsa3d_fwd.cuh"
 #include "dsa3d_fwd_mma.cuh"
 #include "dsa3d_sort.cuh"
@@ -352,17 +351,7 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
         h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
-  if constexpr (DH == 128) {
-    // tcgen05 UMMA with the accumulator in tensor memory: one chunk per CTA at a time
-    const int smem = dq_tc_smem_bytes();
-    if (cudaFuncSetAttribute(dsa3d_bwd_dq_tc_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return DSA3D_ERR_CUDA;
-    TimedLaunch tl(kKernBwdDq, st);
-    dsa3d_bwd_dq_tc_kernel<DH><<<grid_for(rows, 1, kTcCtasPerSm), 128, smem, st>>>(
-        kb, static_cast<bf*>(dq), w.cnt, w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg, h0, hg);
-    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
-  } else {
+  {
     const int smem = 4 * dq_warp_bytes<DH>();
     if (cudaFuncSetAttribute(dsa3d_bwd_dq_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
