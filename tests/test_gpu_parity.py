@@ -85,10 +85,12 @@ def test_invalid_offsets_and_carry():
     full_parity(inp, dims, window, "f32")
 
 
-@pytest.mark.parametrize("window", [(3, 3, 15), (1, 1, 13), (5, 3, 11)])
-def test_widest_tensor_core_windows(window):
+@pytest.mark.parametrize("window,dh", [((3, 3, 15), 128), ((1, 1, 13), 128), ((5, 3, 11), 128),
+                                       ((3, 5, 15), 64), ((3, 3, 11), 64)])
+def test_widest_tensor_core_windows(window, dh):
+    # k_w > 9 selects the forward's longer tap runs; k_w = 15 is the widest window of the path
     dims = (6, 9, 37)
-    _, inp = inputs.custom(*dims, 2, 128, window, "bf16", seed=300 + window[2], scale=3.0)
+    _, inp = inputs.custom(*dims, 2, dh, window, "bf16", seed=300 + window[2] + dh, scale=3.0)
     full_parity(inp, dims, window, "bf16")
 
 
