@@ -416,11 +416,22 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
         avail = psutil.virtual_memory().available
     except ImportError:
         avail = 0
-    # pinned host memory: all inputs, and every output if that stays under 60% of free RAM;
-    # otherwise the step's read-back is the offset gradient and lse only
+    # every rank on this node pins its own buffers at about the same time: each may use its share
+    # of the free RAM only
+    local_ranks = max(1, int(os.environ.get("LOCAL_WORLD_SIZE", str(world))))
+    avail //= local_ranks
+    # pinned host memory: all inputs, and every output if that stays under 60% of this rank's share
+    # of free RAM; otherwise the step's read-back is the offset gradient and lse only
     read_all = in_bytes + out_bytes < 0.6 * avail
-    if in_bytes > 0.6 * avail:
-        return {"value": None, "unit": UNIT, "skipped": f"host RAM {avail >> 30} GiB too small"}
+    skip = in_bytes > 0.6 * avail
+    if world > 1:
+        # the ranks must agree on running the leg (it contains collectives)
+        from deformable_slide_attention_b200 import ranks
+        skip = ranks.max_over_ranks(1.0 if skip else 0.0, dev) > 0.5
+        read_all = ranks.max_over_ranks(0.0 if read_all else 1.0, dev) < 0.5
+    if skip:
+        return {"value": None, "unit": UNIT,
+                "skipped": f"host RAM share {avail >> 30} GiB per rank too small for {in_bytes >> 30} GiB"}
     h_in = {}
     try:
         for n in names_in:
@@ -432,7 +443,18 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
             for n in ("out", "dq", "dk", "dv"):
                 h_out[n] = torch.empty(inp["q"].shape, dtype=inp["q"].dtype, pin_memory=True)
     except RuntimeError as e:
-        return {"value": None, "unit": UNIT, "skipped": f"pinned host buffers unavailable: {e}"[:200]}
+        err = str(e)
+    else:
+        err = None
+    failed = err is not None
+    if world > 1:  # every rank runs the leg or none does
+        from deformable_slide_attention_b200 import ranks
+        failed = ranks.max_over_ranks(1.0 if failed else 0.0, dev) > 0.5
+    if failed:
+        h_in.clear()
+        h_out = {}
+        return {"value": None, "unit": UNIT,
+                "skipped": f"pinned host buffers unavailable: {err or 'on another rank'}"[:200]}
     d_in = {n: inp[n] for n in names_in}
     stream = torch.cuda.current_stream(dev)
 
