@@ -8,7 +8,7 @@ module compiles it with gcc on first use and marshals numpy/torch CPU arrays thr
 
 Source of the operator: MegaSlide-DiT (arXiv 2607.22696), the 3D-DSA definition (Eq. 1 and the
 softmax over the k_t x k_h x k_w neighbourhood that follows it).  The readings the paper leaves
-open are listed in the C file's header (R1..R7).
+open are listed in the C file's header (R1..R8).
 
 Parity pins: every routine here is pinned by ``tests/test_oracle_pins.py`` against brute-force
 dense attention, torch's ``grid_sample``, finite differences and an independent torch autograd
@@ -61,6 +61,10 @@ def _load():
             lib.dsa3d_oracle_backward.argtypes = [ctypes.c_int, vp, vp, vp, vp, vp, *dims, i64p,
                                                   ctypes.c_int64, vp, vp, i64p, ctypes.c_int64,
                                                   vp, vp, ctypes.c_int]
+            lib.dsa3d_oracle_forward_taps.restype = ctypes.c_int64
+            lib.dsa3d_oracle_forward_taps.argtypes = lib.dsa3d_oracle_forward.argtypes
+            lib.dsa3d_oracle_backward_taps.restype = ctypes.c_int
+            lib.dsa3d_oracle_backward_taps.argtypes = lib.dsa3d_oracle_backward.argtypes
             lib.dsa3d_oracle_tap.restype = ctypes.c_int
             lib.dsa3d_oracle_tap.argtypes = [ctypes.c_int, vp, vp, *dims, ctypes.c_int,
                                              ctypes.c_int64, ctypes.c_int, i64p, vp, vp, vp]
@@ -114,10 +118,12 @@ def _threads(n):
     return int(n) if n else (os.cpu_count() or 1)
 
 
-def forward(q, k, v, offsets, dims, window, items=None, threads=None, return_reads=False):
+def forward(q, k, v, offsets, dims, window, items=None, threads=None, return_reads=False,
+            per_tap=False):
     """Forward of 3D-DSA.
 
-    q, k, v: [N][heads][dh] (fp32 or bf16); offsets: [heads][N][3] fp32; dims = (F, Hp, Wp);
+    q, k, v: [N][heads][dh] (fp32 or bf16); offsets: [heads][N][3] fp32, or with ``per_tap``
+    [heads][N][K][3] (one offset per window tap, K = kt*kh*kw, reading R8); dims = (F, Hp, Wp);
     window = (kt, kh, kw).  ``items`` lists h*N + n; None means every (h, n), head-major.
     Returns (out [n_items][dh] float64, lse [n_items] float64).
     """
@@ -132,20 +138,23 @@ def forward(q, k, v, offsets, dims, window, items=None, threads=None, return_rea
     it, itp = _items(items, N * heads)
     out = np.zeros((len(it), dh), np.float64)
     lse = np.zeros(len(it), np.float64)
-    reads = _load().dsa3d_oracle_forward(io, _ptr(qa), _ptr(ka), _ptr(va), _ptr(off), *dims, heads,
-                                         dh, *window, itp, len(it), _ptr(out), _ptr(lse),
-                                         _threads(threads))
+    _check_offsets(off, heads, N, window, per_tap)
+    fn = _load().dsa3d_oracle_forward_taps if per_tap else _load().dsa3d_oracle_forward
+    reads = fn(io, _ptr(qa), _ptr(ka), _ptr(va), _ptr(off), *dims, heads, dh, *window, itp, len(it),
+               _ptr(out), _ptr(lse), _threads(threads))
     if reads < 0:
         raise ValueError("oracle forward rejected its arguments")
     return (out, lse, reads) if return_reads else (out, lse)
 
 
-def backward(q, k, v, offsets, dout, dims, window, q_items=None, k_items=None, threads=None):
+def backward(q, k, v, offsets, dout, dims, window, q_items=None, k_items=None, threads=None,
+             per_tap=False):
     """Backward of 3D-DSA.
 
-    Returns (dq [n_q][dh], doff [n_q][3], dk [n_k][dh], dv [n_k][dh]) in float64.  ``q_items``
-    and ``k_items`` list h*N + n; None means every item.  dk/dv at a key gather the contributions
-    of every query of that head.
+    Returns (dq [n_q][dh], doff [n_q][3], dk [n_k][dh], dv [n_k][dh]) in float64; with
+    ``per_tap`` (offsets [heads][N][K][3]) doff is [n_q][K][3].  ``q_items`` and ``k_items`` list
+    h*N + n; None means every item.  dk/dv at a key gather the contributions of every query of
+    that head.
     """
     qa, io = _as_io(q)
     ka, _ = _as_io(k)
@@ -158,16 +167,25 @@ def backward(q, k, v, offsets, dout, dims, window, q_items=None, k_items=None, t
     heads, dh = qa.shape[-2], qa.shape[-1]
     qi, qip = _items(q_items, N * heads)
     ki, kip = _items(k_items, N * heads)
+    _check_offsets(off, heads, N, window, per_tap)
+    K = window[0] * window[1] * window[2]
     dq = np.zeros((len(qi), dh), np.float64)
-    doff = np.zeros((len(qi), 3), np.float64)
+    doff = np.zeros((len(qi), K, 3) if per_tap else (len(qi), 3), np.float64)
     dk = np.zeros((len(ki), dh), np.float64)
     dv = np.zeros((len(ki), dh), np.float64)
-    rc = _load().dsa3d_oracle_backward(io, _ptr(qa), _ptr(ka), _ptr(va), _ptr(off), _ptr(da), *dims,
-                                       heads, dh, *window, qip, len(qi), _ptr(dq), _ptr(doff), kip,
-                                       len(ki), _ptr(dk), _ptr(dv), _threads(threads))
+    fn = _load().dsa3d_oracle_backward_taps if per_tap else _load().dsa3d_oracle_backward
+    rc = fn(io, _ptr(qa), _ptr(ka), _ptr(va), _ptr(off), _ptr(da), *dims, heads, dh, *window, qip,
+            len(qi), _ptr(dq), _ptr(doff), kip, len(ki), _ptr(dk), _ptr(dv), _threads(threads))
     if rc != 0:
         raise ValueError("oracle backward rejected its arguments")
     return dq, doff, dk, dv
+
+
+def _check_offsets(off, heads, N, window, per_tap):
+    K = window[0] * window[1] * window[2]
+    want = heads * N * (K if per_tap else 1) * 3
+    if off.size != want:
+        raise ValueError(f"offsets hold {off.size} values, expected {want}")
 
 
 def tap(src, offsets, dims, window, h, n, tau):
@@ -187,19 +205,21 @@ def tap(src, offsets, dims, window, h, n, tau):
     return bool(rc), base, frac, samp, dsamp
 
 
-def full_forward(q, k, v, offsets, dims, window, threads=None):
+def full_forward(q, k, v, offsets, dims, window, threads=None, per_tap=False):
     """Forward over every (n, h), returned in the [N][heads][dh] / [heads][N] layouts."""
     N = dims[0] * dims[1] * dims[2]
     heads, dh = q.shape[-2], q.shape[-1]
-    out, lse = forward(q, k, v, offsets, dims, window, None, threads)
+    out, lse = forward(q, k, v, offsets, dims, window, None, threads, per_tap=per_tap)
     out = out.reshape(heads, N, dh).transpose(1, 0, 2).copy()
     return out, lse.reshape(heads, N)
 
 
-def full_backward(q, k, v, offsets, dout, dims, window, threads=None):
-    """Backward over every item, returned as dq/dk/dv [N][heads][dh] and doff [heads][N][3]."""
+def full_backward(q, k, v, offsets, dout, dims, window, threads=None, per_tap=False):
+    """Backward over every item, returned as dq/dk/dv [N][heads][dh] and doff [heads][N][3]
+    (per_tap: [heads][N][K][3])."""
     N = dims[0] * dims[1] * dims[2]
     heads, dh = q.shape[-2], q.shape[-1]
-    dq, doff, dk, dv = backward(q, k, v, offsets, dout, dims, window, None, None, threads)
+    dq, doff, dk, dv = backward(q, k, v, offsets, dout, dims, window, None, None, threads,
+                                per_tap=per_tap)
     r = lambda a: a.reshape(heads, N, dh).transpose(1, 0, 2).copy()
-    return r(dq), doff.reshape(heads, N, 3), r(dk), r(dv)
+    return r(dq), doff.reshape((heads, N, -1, 3) if per_tap else (heads, N, 3)), r(dk), r(dv)

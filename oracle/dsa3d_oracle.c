@@ -38,6 +38,12 @@
  *       part held fixed; d/d(delta) is the derivative of the trilinear weights inside the cell
  *       [i, i+1] (the +f side at exact integers).  The softmax Jacobian's D = sum_tau P dP
  *       equals dO . out for the exact out (no rounding to the I/O type).
+ *   R8  Per-tap offsets (the *_taps entry points): the paper's offset tensor with one 3-vector
+ *       per window tap, offsets [heads][N][K][3] with K = kt*kh*kw in tap order (u outermost).
+ *       Tap tau samples at p + tau + delta_tau; each tap's offset is decoded as in R4 on its
+ *       own, and a non-finite or too large offset masks only that tap (R5 applies per tap).
+ *       The offset gradient is per tap, [heads][N][K][3].  With every tap's offset equal to one
+ *       per-token offset the result is that of R1.
  *
  * Layouts: q, k, v, dout: [N][heads][dh] (token n = (t*Hp + y)*Wp + x), in fp32 or bf16 bits.
  * offsets: [heads][N][3] fp32, order (dt, dy, dx).  A query or key "item" is h*N + n.
@@ -53,6 +59,7 @@
 
 typedef struct {
     int F, Hp, Wp, heads, dh, kt, kh, kw, io;
+    int n_off;       /* offsets per (token, head): 1 (R1) or K (R8) */
     int64_t N;
     const void *q, *k, *v, *dout;
     const float *off;
@@ -73,10 +80,10 @@ static double rd(const void *base, int io, int64_t idx) {
     return (double)x;
 }
 
-static decode_t decode(const prob_t *P, int h, int64_t n) {
+/* Decode one offset 3-vector o (R4). */
+static decode_t decode_vec(const float *o) {
     decode_t d;
     d.ok = 1;
-    const float *o = P->off + ((int64_t)h * P->N + n) * 3;
     for (int a = 0; a < 3; a++) {
         volatile float delta = o[a];
         if (!isfinite(delta) || fabsf(delta) > 16777216.0f) {
@@ -96,6 +103,17 @@ static decode_t decode(const prob_t *P, int h, int64_t n) {
         d.f[a] = fr;
     }
     return d;
+}
+
+/* The per-token offset of query n (R1). */
+static decode_t decode(const prob_t *P, int h, int64_t n) {
+    return decode_vec(P->off + ((int64_t)h * P->N + n) * 3);
+}
+
+/* The decoded offset of tap tau of query n: the query's own d (R1), or the tap's (R8). */
+static decode_t tap_decode(const prob_t *P, int h, int64_t n, int tau, const decode_t *d) {
+    if (P->n_off == 1) return *d;
+    return decode_vec(P->off + (((int64_t)h * P->N + n) * P->n_off + tau) * 3);
 }
 
 /* Token coordinates of token n. */
@@ -202,11 +220,12 @@ static double query_forward(const prob_t *P, int h, int64_t n, double *out, doub
     double m = -INFINITY;
     int any = 0;
     for (int tau = 0; tau < K; tau++) {
-        if (!tap_base(P, p, &d, tau, b)) {
+        const decode_t dt = tap_decode(P, h, n, tau, &d);
+        if (!tap_base(P, p, &dt, tau, b)) {
             s[tau] = -INFINITY;
             continue;
         }
-        sample(P, P->k, h, b, d.f, ktil, NULL, reads);
+        sample(P, P->k, h, b, dt.f, ktil, NULL, reads);
         s[tau] = scale * dot_row(P, P->q, h, n, ktil);
         if (s[tau] > m) m = s[tau];
         any = 1;
@@ -218,8 +237,9 @@ static double query_forward(const prob_t *P, int h, int64_t n, double *out, doub
         if (s[tau] == -INFINITY) continue;
         double pt = exp(s[tau] - m);
         l += pt;
-        tap_base(P, p, &d, tau, b);
-        sample(P, P->v, h, b, d.f, vtil, NULL, reads);
+        const decode_t dt = tap_decode(P, h, n, tau, &d);
+        tap_base(P, p, &dt, tau, b);
+        sample(P, P->v, h, b, dt.f, vtil, NULL, reads);
         for (int e = 0; e < dh; e++) out[e] += pt * vtil[e];
     }
     for (int e = 0; e < dh; e++) out[e] /= l;
@@ -234,6 +254,7 @@ static prob_t make_prob(int io, const void *q, const void *k, const void *v, con
     P.kt = kt; P.kh = kh; P.kw = kw; P.io = io;
     P.N = (int64_t)F * Hp * Wp;
     P.q = q; P.k = k; P.v = v; P.off = off; P.dout = dout;
+    P.n_off = 1;
     return P;
 }
 
@@ -247,14 +268,16 @@ static int check_args(int F, int Hp, int Wp, int heads, int dh, int kt, int kh, 
 /*
  * Forward for a list of query items (h*N + n).  out: [n_items][dh], lse: [n_items].
  * Returns the number of corner-token reads performed (a work counter), or -1 on bad arguments.
+ * per_tap selects the offset layout: 0 = [heads][N][3] (R1), 1 = [heads][N][K][3] (R8).
  */
-int64_t dsa3d_oracle_forward(int io, const void *q, const void *k, const void *v, const float *off,
-                             int F, int Hp, int Wp, int heads, int dh, int kt, int kh, int kw,
-                             const int64_t *items, int64_t n_items, double *out, double *lse,
-                             int n_threads) {
+static int64_t forward_impl(int io, const void *q, const void *k, const void *v, const float *off,
+                            int F, int Hp, int Wp, int heads, int dh, int kt, int kh, int kw,
+                            const int64_t *items, int64_t n_items, double *out, double *lse,
+                            int n_threads, int per_tap) {
     if (check_args(F, Hp, Wp, heads, dh, kt, kh, kw, io)) return -1;
     prob_t P = make_prob(io, q, k, v, off, NULL, F, Hp, Wp, heads, dh, kt, kh, kw);
     int K = kt * kh * kw;
+    P.n_off = per_tap ? K : 1;
     for (int64_t it = 0; it < n_items; it++)
         if (items[it] < 0 || items[it] >= P.N * heads) return -1;
     int64_t total_reads = 0;
@@ -274,6 +297,23 @@ int64_t dsa3d_oracle_forward(int io, const void *q, const void *k, const void *v
         free(s); free(kt_); free(vt_);
     }
     return total_reads;
+}
+
+int64_t dsa3d_oracle_forward(int io, const void *q, const void *k, const void *v, const float *off,
+                             int F, int Hp, int Wp, int heads, int dh, int kt, int kh, int kw,
+                             const int64_t *items, int64_t n_items, double *out, double *lse,
+                             int n_threads) {
+    return forward_impl(io, q, k, v, off, F, Hp, Wp, heads, dh, kt, kh, kw, items, n_items, out, lse,
+                        n_threads, 0);
+}
+
+/* Forward with per-tap offsets [heads][N][K][3] (R8); otherwise as dsa3d_oracle_forward. */
+int64_t dsa3d_oracle_forward_taps(int io, const void *q, const void *k, const void *v,
+                                  const float *off, int F, int Hp, int Wp, int heads, int dh, int kt,
+                                  int kh, int kw, const int64_t *items, int64_t n_items, double *out,
+                                  double *lse, int n_threads) {
+    return forward_impl(io, q, k, v, off, F, Hp, Wp, heads, dh, kt, kh, kw, items, n_items, out, lse,
+                        n_threads, 1);
 }
 
 /* Per-thread work arrays of the backward. */
@@ -304,14 +344,15 @@ static void scratch_free(scratch_t *S) {
  * Softmax backward of one query: P[tau], dS[tau] (zero for masked taps), and dq, doff.
  * Returns 0 if the query has no valid tap (everything zero).
  */
-static int query_backward(const prob_t *P, int h, int64_t n, scratch_t *S, double *dq, double *doff) {
+static int query_backward(const prob_t *P, int h, int64_t n, scratch_t *S, double *dq,
+                          double *doff_all) {
     int K = P->kt * P->kh * P->kw, dh = P->dh;
     double scale = 1.0 / sqrt((double)dh);
     int64_t p[3], b[3];
     coords(P, n, p);
     decode_t d = decode(P, h, n);
     for (int e = 0; e < dh; e++) dq[e] = 0.0;
-    doff[0] = doff[1] = doff[2] = 0.0;
+    for (int e = 0; e < 3 * P->n_off; e++) doff_all[e] = 0.0;
     for (int tau = 0; tau < K; tau++) S->P[tau] = S->dS[tau] = 0.0;
     double lse = query_forward(P, h, n, S->out, S->s, S->ktil, S->vtil, NULL);
     if (lse == -INFINITY) return 0;
@@ -324,9 +365,11 @@ static int query_backward(const prob_t *P, int h, int64_t n, scratch_t *S, doubl
     for (int e = 0; e < dh; e++) D += S->dO[e] * S->out[e];
     for (int tau = 0; tau < K; tau++) {
         if (S->s[tau] == -INFINITY) continue;
-        tap_base(P, p, &d, tau, b);
-        sample(P, P->k, h, b, d.f, S->ktil, S->dk_t, NULL);
-        sample(P, P->v, h, b, d.f, S->vtil, S->dv_t, NULL);
+        const decode_t dt = tap_decode(P, h, n, tau, &d);
+        double *doff = doff_all + (P->n_off > 1 ? 3 * tau : 0); /* per query (R1) or tap (R8) */
+        tap_base(P, p, &dt, tau, b);
+        sample(P, P->k, h, b, dt.f, S->ktil, S->dk_t, NULL);
+        sample(P, P->v, h, b, dt.f, S->vtil, S->dv_t, NULL);
         double Pt = exp(S->s[tau] - lse);
         double dP = 0.0;
         for (int e = 0; e < dh; e++) dP += S->dO[e] * S->vtil[e];
@@ -349,16 +392,18 @@ static int query_backward(const prob_t *P, int h, int64_t n, scratch_t *S, doubl
 /*
  * Backward.  dq/doff are reported for the query items q_items ([n_q][dh], [n_q][3]).
  * dk/dv are reported for the key items k_items ([n_k][dh]); each gathers the contributions of
- * every query of its head whose taps touch it.  Returns 0, or -1 on bad arguments.
+ * every query of its head whose taps touch it.  Returns 0, or -1 on bad arguments.  With
+ * per_tap (R8) the offsets are [heads][N][K][3] and doff is [n_q][K][3].
  */
-int dsa3d_oracle_backward(int io, const void *q, const void *k, const void *v, const float *off,
-                          const void *dout, int F, int Hp, int Wp, int heads, int dh, int kt,
-                          int kh, int kw, const int64_t *q_items, int64_t n_q, double *dq,
-                          double *doff, const int64_t *k_items, int64_t n_k, double *dk,
-                          double *dv, int n_threads) {
+static int backward_impl(int io, const void *q, const void *k, const void *v, const float *off,
+                         const void *dout, int F, int Hp, int Wp, int heads, int dh, int kt,
+                         int kh, int kw, const int64_t *q_items, int64_t n_q, double *dq,
+                         double *doff, const int64_t *k_items, int64_t n_k, double *dk,
+                         double *dv, int n_threads, int per_tap) {
     if (check_args(F, Hp, Wp, heads, dh, kt, kh, kw, io)) return -1;
     prob_t P = make_prob(io, q, k, v, off, dout, F, Hp, Wp, heads, dh, kt, kh, kw);
     int K = kt * kh * kw;
+    P.n_off = per_tap ? K : 1;
     int nt = n_threads > 0 ? n_threads : 1;
     double scale = 1.0 / sqrt((double)dh);
     for (int64_t it = 0; it < n_q; it++)
@@ -373,7 +418,7 @@ int dsa3d_oracle_backward(int io, const void *q, const void *k, const void *v, c
         for (int64_t it = 0; it < n_q; it++) {
             int h = (int)(q_items[it] / P.N);
             int64_t n = q_items[it] % P.N;
-            query_backward(&P, h, n, &S, dq + it * dh, doff + it * 3);
+            query_backward(&P, h, n, &S, dq + it * dh, doff + it * 3 * P.n_off);
         }
         scratch_free(&S);
     }
@@ -393,7 +438,7 @@ int dsa3d_oracle_backward(int io, const void *q, const void *k, const void *v, c
     {
         scratch_t S = scratch_new(K, dh);
         double *dq_tmp = malloc(sizeof(double) * dh);
-        double doff_tmp[3];
+        double *doff_tmp = malloc(sizeof(double) * 3 * P.n_off);
 #pragma omp for schedule(dynamic, 1)
         for (int h = 0; h < heads; h++) {
             if (!head_used[h]) continue;
@@ -403,10 +448,11 @@ int dsa3d_oracle_backward(int io, const void *q, const void *k, const void *v, c
                 int64_t p[3], b[3];
                 coords(&P, n, p);
                 decode_t d = decode(&P, h, n);
-                if (!d.ok) continue;
+                if (P.n_off == 1 && !d.ok) continue;
                 int touches = 0;
                 for (int tau = 0; tau < K && !touches; tau++) {
-                    if (!tap_base(&P, p, &d, tau, b)) continue;
+                    const decode_t dt = tap_decode(&P, h, n, tau, &d);
+                    if (!tap_base(&P, p, &dt, tau, b)) continue;
                     for (int c = 0; c < 8; c++) {
                         int64_t tok = corner_tok(&P, b, c);
                         if (tok >= 0 && map[tok] >= 0) { touches = 1; break; }
@@ -416,11 +462,12 @@ int dsa3d_oracle_backward(int io, const void *q, const void *k, const void *v, c
                 if (!query_backward(&P, h, n, &S, dq_tmp, doff_tmp)) continue;
                 for (int tau = 0; tau < K; tau++) {
                     if (S.P[tau] == 0.0 && S.dS[tau] == 0.0) continue;
-                    tap_base(&P, p, &d, tau, b);
+                    const decode_t dt = tap_decode(&P, h, n, tau, &d);
+                    tap_base(&P, p, &dt, tau, b);
                     for (int c = 0; c < 8; c++) {
                         int64_t tok = corner_tok(&P, b, c);
                         if (tok < 0 || map[tok] < 0) continue;
-                        double w = corner_w(d.f, c);
+                        double w = corner_w(dt.f, c);
                         double gk = w * scale * S.dS[tau];
                         double gv = w * S.P[tau];
                         double *dkr = dk + map[tok] * dh, *dvr = dv + map[tok] * dh;
@@ -433,11 +480,31 @@ int dsa3d_oracle_backward(int io, const void *q, const void *k, const void *v, c
             }
         }
         free(dq_tmp);
+        free(doff_tmp);
         scratch_free(&S);
     }
     free(rowmap);
     free(head_used);
     return 0;
+}
+
+int dsa3d_oracle_backward(int io, const void *q, const void *k, const void *v, const float *off,
+                          const void *dout, int F, int Hp, int Wp, int heads, int dh, int kt,
+                          int kh, int kw, const int64_t *q_items, int64_t n_q, double *dq,
+                          double *doff, const int64_t *k_items, int64_t n_k, double *dk,
+                          double *dv, int n_threads) {
+    return backward_impl(io, q, k, v, off, dout, F, Hp, Wp, heads, dh, kt, kh, kw, q_items, n_q, dq,
+                         doff, k_items, n_k, dk, dv, n_threads, 0);
+}
+
+/* Backward with per-tap offsets (R8): offsets [heads][N][K][3], doff [n_q][K][3]. */
+int dsa3d_oracle_backward_taps(int io, const void *q, const void *k, const void *v,
+                               const float *off, const void *dout, int F, int Hp, int Wp, int heads,
+                               int dh, int kt, int kh, int kw, const int64_t *q_items, int64_t n_q,
+                               double *dq, double *doff, const int64_t *k_items, int64_t n_k,
+                               double *dk, double *dv, int n_threads) {
+    return backward_impl(io, q, k, v, off, dout, F, Hp, Wp, heads, dh, kt, kh, kw, q_items, n_q, dq,
+                         doff, k_items, n_k, dk, dv, n_threads, 1);
 }
 
 /*

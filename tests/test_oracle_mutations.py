@@ -29,6 +29,9 @@ MUTANTS = {
     "no_carry": ("if (fr == 1.0f) {", "if (0) {"),
     "dv_uses_dS": ("double gv = w * S.P[tau];", "double gv = w * S.dS[tau];"),
     "dq_uses_vtil": ("dq[e] += scale * dS * S->ktil[e];", "dq[e] += scale * dS * S->vtil[e];"),
+    "per_tap_offsets_read_tap_0": ("* P->n_off + tau) * 3);", "* P->n_off + 0) * 3);"),
+    "per_tap_gradient_not_per_tap": ("double *doff = doff_all + (P->n_off > 1 ? 3 * tau : 0);",
+                                     "double *doff = doff_all;"),
 }
 
 

@@ -17,6 +17,12 @@ Each pin is chosen so that a plausible mistake in the oracle fails at least one 
      lse >= max tap score
   P9 work counter scales linearly in N
   P10 heads are independent; permuting heads permutes the result
+Per-tap offsets (the paper's offset tensor with one 3-vector per window tap, reading R8):
+  P11 every tap carrying the query's offset == the per-token oracle (exactly); the per-tap offset
+      gradients sum to the per-token one
+  P12 torch float64 autograd of the grid_sample restatement with per-tap offsets == the oracle
+  P13 central finite differences along single taps' offsets == the per-tap offset gradient
+  P14 a tap with a non-finite offset is masked alone (== the same tap moved out of the volume)
 """
 import math
 
@@ -340,3 +346,95 @@ def test_golden_regression_snapshot():
                                        w.dims, w.window, ITEMS, ITEMS)
     for name, got in (("out", out), ("lse", lse), ("dq", dq), ("doff", doff), ("dk", dk), ("dv", dv)):
         assert np.allclose(got, np.array(rec[name]), atol=1e-12, rtol=0), name
+
+
+# ---------------------------------------------------------------------------------------------
+# per-tap offsets (R8)
+def _taps_problem(seed):
+    """The P6/P7 problem with one offset per window tap: coarse binary fractions away from integers,
+    so the finite differences below stay exact and never cross a cell or a box face."""
+    dims, window, q, k, v, do, _ = _fd_problem(seed)
+    H, N, K = q.shape[1], q.shape[0], math.prod(window)
+    g = torch.Generator().manual_seed(seed + 1000)
+    off = torch.empty(H, N, K, 3).uniform_(-1.4, 1.4, generator=g)
+    frac = off - off.floor()
+    off = torch.where(frac < 0.01, off + 0.02, off)
+    off = torch.where(frac > 0.99, off - 0.02, off)
+    off = (torch.round(off * 1024) / 1024).float()
+    return dims, window, q, k, v, do, off
+
+
+def _loss_taps(q, k, v, off, do, dims, window):
+    out, _ = oracle.full_forward(q, k, v, off, dims, window, per_tap=True)
+    return float((out * do.double().numpy()).sum())
+
+
+def test_p11_shared_tap_offsets_equal_per_token():
+    dims, window, q, k, v, do, off = _fd_problem(31)
+    K = math.prod(window)
+    taps = off[:, :, None, :].expand(-1, -1, K, -1).contiguous()
+    o1, l1 = oracle.full_forward(q, k, v, off, dims, window)
+    o2, l2 = oracle.full_forward(q, k, v, taps, dims, window, per_tap=True)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    g1 = oracle.full_backward(q, k, v, off, do, dims, window)
+    g2 = oracle.full_backward(q, k, v, taps, do, dims, window, per_tap=True)
+    for name, a, b in (("dq", g1[0], g2[0]), ("dk", g1[2], g2[2]), ("dv", g1[3], g2[3])):
+        assert np.array_equal(a, b), name
+    assert g2[1].shape == off.shape[:2] + (K, 3)
+    assert np.allclose(g2[1].sum(axis=2), g1[1], atol=1e-12, rtol=0)
+
+
+def test_p12_per_tap_matches_torch_autograd_restatement():
+    dims, window, q, k, v, do, off = _taps_problem(32)
+    q64, k64, v64, off64 = (x.double().clone().requires_grad_(True) for x in (q, k, v, off))
+    out, lse = tr.dsa3d(q64, k64, v64, off64, dims, window)
+    (out * do.double()).sum().backward()
+    o_out, o_lse = oracle.full_forward(q, k, v, off, dims, window, per_tap=True)
+    assert np.allclose(o_out, out.detach().numpy(), atol=1e-12, rtol=0)
+    fin = torch.isfinite(lse).numpy()
+    assert np.array_equal(np.isfinite(o_lse), fin)
+    assert np.allclose(o_lse[fin], lse.detach().numpy()[fin], atol=1e-12, rtol=0)
+    dq, doff, dk, dv = oracle.full_backward(q, k, v, off, do, dims, window, per_tap=True)
+    for name, a, b in (("dq", dq, q64.grad), ("dk", dk, k64.grad), ("dv", dv, v64.grad),
+                       ("doff", doff, off64.grad)):
+        assert np.allclose(a, b.numpy(), atol=1e-10, rtol=0), name
+
+
+def test_p13_per_tap_finite_differences():
+    dims, window, q, k, v, do, off = _taps_problem(33)
+    H, N, K = off.shape[0], off.shape[1], off.shape[2]
+    _, doff, _, _ = oracle.full_backward(q, k, v, off, do, dims, window, per_tap=True)
+    g = torch.Generator().manual_seed(5)
+    eps = 2.0 ** -14
+    checked = 0
+    for _ in range(48):
+        h, n = int(torch.randint(0, H, (1,), generator=g)), int(torch.randint(0, N, (1,), generator=g))
+        tau, a = int(torch.randint(0, K, (1,), generator=g)), int(torch.randint(0, 3, (1,), generator=g))
+        op, om = off.clone(), off.clone()
+        op[h, n, tau, a] += eps
+        om[h, n, tau, a] -= eps
+        fd = (_loss_taps(q, k, v, op, do, dims, window) - _loss_taps(q, k, v, om, do, dims, window)) / (2 * eps)
+        an = doff[h, n, tau, a]
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (h, n, tau, a, fd, an)
+        checked += an != 0.0
+    assert checked >= 8  # enough of the sampled taps lie inside the small volume
+
+
+def test_p14_non_finite_tap_offset_masks_that_tap_only():
+    dims, window, q, k, v, _, off = _taps_problem(34)
+    K = off.shape[2]
+    o_ref, l_ref = oracle.forward(q, k, v, off, dims, window, items=np.array([7]), per_tap=True)
+    bad, far = off.clone(), off.clone()
+    # a tap of query 7 (head 0) whose sample position lies inside the volume
+    pos = tr.token_coords(dims)[7][None] + tr.tap_offsets(window) + off[0, 7].double()
+    ext = torch.tensor([d - 1 for d in dims], dtype=torch.float64)
+    inside = ((pos >= 0) & (pos <= ext)).all(-1)
+    assert inside.sum() >= 2
+    tau0 = int(torch.nonzero(inside)[0])
+    bad[0, 7, tau0] = float("nan")
+    far[0, 7, tau0, 0] = 1.0e6
+    o_bad, l_bad = oracle.forward(q, k, v, bad, dims, window, items=np.array([7]), per_tap=True)
+    o_far, l_far = oracle.forward(q, k, v, far, dims, window, items=np.array([7]), per_tap=True)
+    assert np.isfinite(l_bad).all()
+    assert np.array_equal(o_bad, o_far) and np.array_equal(l_bad, l_far)
+    assert not np.array_equal(o_bad, o_ref)

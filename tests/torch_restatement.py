@@ -31,11 +31,13 @@ def token_coords(dims):
 
 
 def dsa3d(q, k, v, off, dims, window):
-    """q, k, v: [N][H][dh] float64; off: [H][N][3] float64.  Returns out [N][H][dh], lse [H][N]."""
+    """q, k, v: [N][H][dh] float64; off: [H][N][3] float64 (one offset per query), or [H][N][K][3]
+    (one per window tap).  Returns out [N][H][dh], lse [H][N]."""
     F, Hp, Wp = dims
     N, H, dh = q.shape
     assert min(dims) >= 2, "grid_sample normalisation needs every extent >= 2"
-    pos = token_coords(dims)[None, :, None, :] + tap_offsets(window)[None, None] + off[:, :, None, :]
+    per_tap = off if off.dim() == 4 else off[:, :, None, :]
+    pos = token_coords(dims)[None, :, None, :] + tap_offsets(window)[None, None] + per_tap
     ext = torch.tensor([F - 1, Hp - 1, Wp - 1], dtype=torch.float64)
     valid = ((pos >= 0) & (pos <= ext)).all(-1)  # [H][N][K]
     g = 2.0 * pos / ext - 1.0
