@@ -11,7 +11,8 @@ so no extra L2 flush is needed between steps.  Multi-GPU runs (torchrun) are wea
 rank processes its own independent clip (seed + rank); 3D-DSA has no exchange step.
 
 ``--impl reference`` times the CPU oracle (the only other implementation) on a bounded sample.
-Prints one JSON line (rank 0).
+``--workload 720p-train-taps-bf16`` measures the per-tap offset entry points (one offset 3-vector
+per window tap) on the 720p training shapes instead.  Prints one JSON line (rank 0).
 """
 from __future__ import annotations
 
@@ -31,6 +32,15 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "3D-DSA fwd+bwd tokens/s at N≈2.1M (1 B200) and % of HBM roofline"
+DEFAULT_WORKLOAD = "1080p-long-bf16"
+
+
+def metric_of(w):
+    """The headline metric on the default workload; other workloads name themselves."""
+    if w.name.startswith(DEFAULT_WORKLOAD):
+        return METRIC
+    kind = "per-tap offsets, " if w.per_tap else ""
+    return f"3D-DSA fwd+bwd tokens/s ({kind}{w.name}, N={w.N}, 1 B200) and % of HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FP32_LANES_PER_SM = 128
@@ -41,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="1080p-long-bf16")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -91,9 +101,16 @@ def measured_peaks():
 # Per (token, head), each tensor the kernel must touch read or written once; s = element size.
 # Whole path: forward 4 dh s + 16, backward 8 dh s + 28 (q, k, v, dO read; dq, dk, dv written;
 # offsets, lse read; doffsets written).  Per kernel, the backward's three passes each re-read
-# some inputs, so their sum (10 dh s + 28) exceeds the backward's figure.
+# some inputs, so their sum (10 dh s + 28) exceeds the backward's figure.  With per-tap offsets
+# the offsets and their gradient are K 3-vectors per (token, head): 12 K bytes each.
 def alg_bytes_per_item(w, kernel):
     s = 4 if w.dtype == "f32" else 2
+    if w.per_tap:
+        ob = 12 * w.K
+        return {"dsa3d_fwd_taps_kernel": 4 * w.dh * s + ob + 4,     # q, k, v, offsets -> out, lse
+                "dsa3d_bwd_taps_kernel": 8 * w.dh * s + 2 * ob + 4,  # + dO, lse -> dq, dk, dv, doffsets
+                "fwd": 4 * w.dh * s + ob + 4,
+                "bwd": 8 * w.dh * s + 2 * ob + 4}.get(kernel, 0)
     table = {
         "dsa3d_fwd_kernel": 4 * w.dh * s + 16,        # q, k, v -> out; offsets, lse
         "dsa3d_fwd_mma_kernel": 4 * w.dh * s + 16,
@@ -109,7 +126,13 @@ def alg_bytes_per_item(w, kernel):
 
 
 def alg_flop_per_item(w, kernel):
-    """Factorised fp32 work per (token, head): dots and axpys of length dh over the B box tokens."""
+    """Factorised fp32 work per (token, head): dots and axpys of length dh over the B box tokens.
+    Per-tap offsets have no shared box: 8 corners per tap, 36 dh K forward (sampling k~ and v~,
+    one dot, one axpy) and 64 dh K backward (per-corner dots with q and dO, then dq and the dK/dV
+    scatter)."""
+    if w.per_tap:
+        return {"dsa3d_fwd_taps_kernel": 36, "dsa3d_bwd_taps_kernel": 64,
+                "fwd": 36, "bwd": 64}.get(kernel, 0) * w.dh * w.K
     B = (w.window[0] + 1) * (w.window[1] + 1) * (w.window[2] + 1)
     per = {"dsa3d_fwd_kernel": 4, "dsa3d_fwd_mma_kernel": 4, "dsa3d_bwd_kernel": 10,
            "dsa3d_bwd_q_kernel": 4, "dsa3d_bwd_dq_kernel": 2, "dsa3d_bwd_kv_kernel": 4,
@@ -178,13 +201,13 @@ def oracle_sample(w, head_inputs, n_items, seed, threads):
     items = np.sort(rng.choice(w.N, size=n_items, replace=False)).astype(np.int64)
     q, k, v, off, do = head_inputs
     t0 = time.perf_counter()
-    oracle.forward(q, k, v, off, w.dims, w.window, items, threads)
-    oracle.backward(q, k, v, off, do, w.dims, w.window, items, [], threads)
+    oracle.forward(q, k, v, off, w.dims, w.window, items, threads, per_tap=w.per_tap)
+    oracle.backward(q, k, v, off, do, w.dims, w.window, items, [], threads, per_tap=w.per_tap)
     return time.perf_counter() - t0
 
 
 def head_inputs_for_oracle(w, inp, head=0):
-    """One head's inputs as contiguous CPU tensors ([N][1][dh] and [1][N][3])."""
+    """One head's inputs as contiguous CPU tensors ([N][1][dh] and [1][N][3] or [1][N][K][3])."""
     pick = lambda t: t[:, head:head + 1, :].contiguous().cpu()
     return (pick(inp["q"]), pick(inp["k"]), pick(inp["v"]),
             inp["offsets"][head:head + 1].contiguous().cpu(), pick(inp["dout"]))
@@ -246,7 +269,7 @@ def run_reference(args):
     tokens_per_step = n_items / w.heads
     value = tokens_per_step * args.steps / total
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_of(w), "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
@@ -262,6 +285,16 @@ def run_reference(args):
 
 
 # --- GPU leg -----------------------------------------------------------------------------------
+def path_of(w, abi):
+    """The public forward and backward calls of the workload: per-token or per-tap offsets."""
+    if not w.per_tap:
+        return abi.forward, abi.backward
+
+    def fwd(q, k, v, off, dims, window, out=None, lse=None, workspace=None):
+        return abi.forward_taps(q, k, v, off, dims, window, out=out, lse=lse)
+    return fwd, abi.backward_taps
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
@@ -291,8 +324,12 @@ def main(argv=None):
     dq, dk, dv, doff = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(off)
     # one workspace serves the forward and the backward (they run one after the other on the
     # stream): all heads at once when that fits in free memory minus a margin, else head groups
-    fws_bytes = abi.dsa3d_forward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
-    full_ws = abi.dsa3d_backward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
+    if w.per_tap:  # the per-tap forward takes no workspace
+        fws_bytes = 0
+        full_ws = abi.dsa3d_backward_taps_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
+    else:
+        fws_bytes = abi.dsa3d_forward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
+        full_ws = abi.dsa3d_backward_workspace_bytes(*w.dims, w.heads, w.dh, *w.window, code)
     per_head = full_ws // w.heads if full_ws else 0
     free, _ = torch.cuda.mem_get_info(dev)
     margin = 6 << 30
@@ -300,14 +337,15 @@ def main(argv=None):
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     heads_per_pass = w.heads if not per_head else max(1, min(w.heads, ws_bytes // per_head))
     fwd_heads = w.heads
-    while fwd_heads > 1 and abi.dsa3d_forward_workspace_bytes(*w.dims, fwd_heads, w.dh, *w.window,
-                                                              code) > ws_bytes:
+    while not w.per_tap and fwd_heads > 1 and abi.dsa3d_forward_workspace_bytes(
+            *w.dims, fwd_heads, w.dh, *w.window, code) > ws_bytes:
         fwd_heads = (fwd_heads + 1) // 2
     stream = torch.cuda.current_stream(dev)
+    fwd_fn, bwd_fn = path_of(w, abi)
 
     def step():
-        abi.forward(q, k, v, off, w.dims, w.window, out=out, lse=lse, workspace=ws)
-        abi.backward(q, k, v, off, lse, do, w.dims, w.window, workspace=ws, grads=(dq, dk, dv, doff))
+        fwd_fn(q, k, v, off, w.dims, w.window, out=out, lse=lse, workspace=ws)
+        bwd_fn(q, k, v, off, lse, do, w.dims, w.window, workspace=ws, grads=(dq, dk, dv, doff))
 
     def barrier():
         if world > 1:
@@ -384,11 +422,12 @@ def main(argv=None):
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": metric_of(w), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "frames": w.F, "grid": [w.Hp, w.Wp], "tokens": w.N,
                    "heads": w.heads, "dh": w.dh, "window": list(w.window),
+                   "offsets": "per tap [heads][N][K][3]" if w.per_tap else "per token [heads][N][3]",
                    "heads_per_forward_pass": fwd_heads,
                    "heads_per_backward_pass": heads_per_pass,
                    "l2": "inputs larger than L2 (each tensor > 126 MB); no flush",
@@ -410,7 +449,7 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
     the inputs host->device and reads back every output (out, lse, dq, dk, dv, doffsets)."""
     names_in = ("q", "k", "v", "offsets", "dout")
     in_bytes = sum(inp[n].numel() * inp[n].element_size() for n in names_in)
-    out_bytes = in_bytes - inp["offsets"].numel() * 4 + (w.heads * w.N * 4) * 4
+    out_bytes = in_bytes + w.heads * w.N * 4  # out, dq, dk, dv, doffsets mirror the inputs; + lse
     try:
         import psutil
         avail = psutil.virtual_memory().available
@@ -457,14 +496,15 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
                 "skipped": f"pinned host buffers unavailable: {err or 'on another rank'}"[:200]}
     d_in = {n: inp[n] for n in names_in}
     stream = torch.cuda.current_stream(dev)
+    fwd_fn, bwd_fn = path_of(w, abi)
 
     def step():
         for n in names_in:
             d_in[n].copy_(h_in[n], non_blocking=True)
-        out, lse = abi.forward(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], w.dims, w.window,
-                               out=outs[0], lse=outs[1], workspace=ws[0])
-        dq, dk, dv, doff = abi.backward(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], lse,
-                                        d_in["dout"], w.dims, w.window, workspace=ws[1], grads=outs[2:])
+        out, lse = fwd_fn(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], w.dims, w.window,
+                          out=outs[0], lse=outs[1], workspace=ws[0])
+        dq, dk, dv, doff = bwd_fn(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], lse,
+                                  d_in["dout"], w.dims, w.window, workspace=ws[1], grads=outs[2:])
         for n, t in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("doffsets", doff)):
             if n in h_out:
                 h_out[n].copy_(t, non_blocking=True)

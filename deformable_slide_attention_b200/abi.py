@@ -61,6 +61,12 @@ def _load():
         lib.dsa3d_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
         lib.dsa3d_backward_noalloc.restype = I
         lib.dsa3d_backward_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, *dims, I, P]
+        lib.dsa3d_forward_taps.restype = I
+        lib.dsa3d_forward_taps.argtypes = [P, P, P, P, P, P, *dims, I, P]
+        lib.dsa3d_backward_taps_workspace_bytes.restype = Z
+        lib.dsa3d_backward_taps_workspace_bytes.argtypes = [*dims, I]
+        lib.dsa3d_backward_taps.restype = I
+        lib.dsa3d_backward_taps.argtypes = [P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
         lib.dsa3d_check_device.restype = I
         lib.dsa3d_check_device.argtypes = [P]
         lib.dsa3d_timing_enable.restype = I
@@ -118,6 +124,25 @@ def dsa3d_backward_noalloc(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, F,
                                           F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream)
 
 
+def dsa3d_forward_taps(q, k, v, offsets, out, lse, F, Hp, Wp, heads, dh, kt, kh, kw, dtype,
+                       stream) -> int:
+    """Forward with per-tap offsets ([heads][N][K][3])."""
+    return _load().dsa3d_forward_taps(q, k, v, offsets, out, lse, F, Hp, Wp, heads, dh, kt, kh, kw,
+                                      dtype, stream)
+
+
+def dsa3d_backward_taps_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype) -> int:
+    return _load().dsa3d_backward_taps_workspace_bytes(F, Hp, Wp, heads, dh, kt, kh, kw, dtype)
+
+
+def dsa3d_backward_taps(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace,
+                        workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype, stream) -> int:
+    """Backward with per-tap offsets; doffsets is [heads][N][K][3]."""
+    return _load().dsa3d_backward_taps(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace,
+                                       workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype,
+                                       stream)
+
+
 def dsa3d_check_device(stream) -> int:
     return _load().dsa3d_check_device(stream)
 
@@ -163,14 +188,16 @@ def _check(status, what):
         raise Dsa3dError(status, what)
 
 
-def _shapes(q, offsets, dims):
+def _shapes(q, offsets, dims, taps=None):
+    """N, heads, dh; offsets must be [heads][N][3], or [heads][N][taps][3] when taps is given."""
     F, Hp, Wp = dims
     N = F * Hp * Wp
     if q.dim() != 3 or q.shape[0] != N:
         raise ValueError(f"q must be [N={N}][heads][dh], got {tuple(q.shape)}")
     heads, dh = q.shape[1], q.shape[2]
-    if tuple(offsets.shape) != (heads, N, 3):
-        raise ValueError(f"offsets must be [heads][N][3] = {(heads, N, 3)}, got {tuple(offsets.shape)}")
+    want = (heads, N, 3) if taps is None else (heads, N, taps, 3)
+    if tuple(offsets.shape) != want:
+        raise ValueError(f"offsets must be {want}, got {tuple(offsets.shape)}")
     return N, heads, dh
 
 
@@ -221,4 +248,49 @@ def backward(q, k, v, offsets, lse, dout, dims, window, workspace=None, stream=N
                           lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                           doff.data_ptr(), ws_ptr, ws_bytes, *dims, heads, dh, *window, code,
                           _stream_handle(stream)), "dsa3d_backward")
+    return dq, dk, dv, doff
+
+
+def _taps(window):
+    kt, kh, kw = window
+    return kt * kh * kw
+
+
+def forward_taps(q, k, v, offsets, dims, window, out=None, lse=None, stream=None, want_lse=True):
+    """3D-DSA forward with per-tap offsets ([heads][N][kt*kh*kw][3]) on CUDA tensors.
+    Returns (out [N][heads][dh], lse [heads][N] or None)."""
+    torch = _torch()
+    N, heads, dh = _shapes(q, offsets, dims, _taps(window))
+    for t in (q, k, v, offsets):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((heads, N), dtype=torch.float32, device=q.device)
+    _check(dsa3d_forward_taps(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(),
+                              out.data_ptr(), lse.data_ptr() if lse is not None else None, *dims,
+                              heads, dh, *window, code, _stream_handle(stream)), "dsa3d_forward_taps")
+    return out, lse
+
+
+def backward_taps(q, k, v, offsets, lse, dout, dims, window, workspace=None, stream=None, grads=None):
+    """3D-DSA backward with per-tap offsets.  Returns (dq, dk, dv, doffsets [heads][N][K][3])."""
+    torch = _torch()
+    N, heads, dh = _shapes(q, offsets, dims, _taps(window))
+    code = _dtype_code(q)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty_like(offsets))
+    dq, dk, dv, doff = grads
+    need = dsa3d_backward_taps_workspace_bytes(*dims, heads, dh, *window, code)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(dsa3d_backward_taps(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(),
+                               lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), doff.data_ptr(), ws_ptr, ws_bytes, *dims, heads, dh,
+                               *window, code, _stream_handle(stream)), "dsa3d_backward_taps")
     return dq, dk, dv, doff

@@ -1,6 +1,6 @@
 // dsa3d.cu -- C ABI of the 3D-DSA library: argument validation, launch configuration and the
 // extern "C" entry points declared in include/dsa3d.h.  All device work is in the kernels of
-// dsa3d_fwd.cuh / dsa3d_bwd.cuh; this file allocates no device memory.
+// dsa3d_*.cuh headers; this file allocates no device memory.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -14,6 +14,7 @@
 #include "dsa3d_fwd.cuh"
 #include "dsa3d_fwd_mma.cuh"
 #include "dsa3d_sort.cuh"
+#include "dsa3d_taps.cuh"
 #include "dsa3d_timing.cuh"
 
 namespace dsa3d {
@@ -216,6 +217,71 @@ int grid_for(int64_t work, int threads, int per_sm_cap) {
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   return (int)grid;
+}
+
+// Argument checks of the forward entry points (after check_shape): pointers present and aligned,
+// outputs disjoint from the inputs and from each other.  off_bytes: size of the offsets.
+dsa3d_status_t check_forward_args(const Shape& s, dsa3d_dtype_t dtype, const void* q, const void* k,
+                                  const void* v, const float* offsets, size_t off_bytes,
+                                  const void* out, const float* lse) {
+  if (!q || !k || !v || !offsets || !out) return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al[] = {q, k, v, offsets, out};
+  for (const void* p : al)
+    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DSA3D_ERR_INVALID_ARGUMENT;
+  const size_t tb = (size_t)s.N * s.heads * s.dh * elem_size(dtype);
+  const Range in[] = {range_of(q, tb), range_of(k, tb), range_of(v, tb), range_of(offsets, off_bytes)};
+  const Range ro = range_of(out, tb);
+  const Range rl = range_of(lse, lse ? (size_t)s.heads * s.N * 4 : 0);
+  for (const Range& r : in)
+    if (overlap(r, ro) || (lse && overlap(r, rl))) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (lse && overlap(ro, rl)) return DSA3D_ERR_INVALID_ARGUMENT;
+  return DSA3D_OK;
+}
+
+// The same for the backward entry points; fills the input and output ranges for the workspace
+// checks.  off_bytes: size of the offsets (and of their gradient).
+dsa3d_status_t check_backward_args(const Shape& s, dsa3d_dtype_t dtype, const void* q, const void* k,
+                                   const void* v, const float* offsets, const float* lse,
+                                   const void* dout, const void* dq, const void* dk, const void* dv,
+                                   const float* doffsets, size_t off_bytes, Range ins[6],
+                                   Range outs[4]) {
+  if (!q || !k || !v || !offsets || !lse || !dout || !dq || !dk || !dv || !doffsets)
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al[] = {q, k, v, offsets, dout, dq, dk, dv, doffsets};
+  for (const void* p : al)
+    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return DSA3D_ERR_INVALID_ARGUMENT;
+  const size_t tb = (size_t)s.N * s.heads * s.dh * elem_size(dtype);
+  ins[0] = range_of(q, tb);
+  ins[1] = range_of(k, tb);
+  ins[2] = range_of(v, tb);
+  ins[3] = range_of(offsets, off_bytes);
+  ins[4] = range_of(lse, (size_t)s.heads * s.N * 4);
+  ins[5] = range_of(dout, tb);
+  outs[0] = range_of(dq, tb);
+  outs[1] = range_of(dk, tb);
+  outs[2] = range_of(dv, tb);
+  outs[3] = range_of(doffsets, off_bytes);
+  for (int i = 0; i < 4; i++) {
+    for (int j = 0; j < 6; j++)
+      if (overlap(ins[j], outs[i])) return DSA3D_ERR_INVALID_ARGUMENT;
+    for (int j = i + 1; j < 4; j++)
+      if (overlap(outs[i], outs[j])) return DSA3D_ERR_INVALID_ARGUMENT;
+  }
+  return DSA3D_OK;
+}
+
+// A caller workspace must be aligned and disjoint from every tensor argument.
+dsa3d_status_t check_workspace(const void* ws, size_t bytes, const Range* ins, int n_in,
+                               const Range* outs, int n_out) {
+  if (!aligned16(ws)) return DSA3D_ERR_INVALID_ARGUMENT;
+  const Range rw = range_of(ws, bytes);
+  for (int i = 0; i < n_in; i++)
+    if (overlap(ins[i], rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < n_out; i++)
+    if (overlap(outs[i], rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+  return DSA3D_OK;
 }
 
 dsa3d_status_t zero16(void* p, size_t n16, cudaStream_t st);
@@ -437,6 +503,89 @@ dsa3d_status_t bwd_dispatch(const Shape& s, int warps, const BwdArgs& a, cudaStr
   }
 }
 
+// --- per-tap offsets (CUDA cores) -----------------------------------------------------------------
+template <typename T, int DH>
+dsa3d_status_t fwd_taps_launch(const Shape& s, const void* q, const void* k, const void* v,
+                               const float* off, void* out, float* lse, cudaStream_t st) {
+  const Geo g = make_geo(s);
+  constexpr int W = kTapsFwdWarps;
+  auto kern = dsa3d_fwd_taps_kernel<T, DH, W>;
+  int grid = 0;
+  const int64_t items = (int64_t)s.heads * s.N;
+  dsa3d_status_t rc = launch_persistent(kern, W, 0, items, st, grid);
+  if (rc != DSA3D_OK) return rc;
+  TimedLaunch tl(kKernFwdTaps, st);
+  kern<<<grid, W * 32, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                     static_cast<const T*>(v), off, static_cast<T*>(out), lse, g, items);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+template <typename T>
+dsa3d_status_t fwd_taps_dispatch(const Shape& s, const void* q, const void* k, const void* v,
+                                 const float* off, void* out, float* lse, cudaStream_t st) {
+  switch (s.dh) {
+    case 32: return fwd_taps_launch<T, 32>(s, q, k, v, off, out, lse, st);
+    case 64: return fwd_taps_launch<T, 64>(s, q, k, v, off, out, lse, st);
+    case 128: return fwd_taps_launch<T, 128>(s, q, k, v, off, out, lse, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+// Warps per CTA of the per-tap backward: its per-warp shared memory grows with K.
+int pick_taps_warps(const Geo& g, int max_smem) {
+  for (int w = kWarps; w >= 1; w >>= 1)
+    if ((int64_t)w * bwd_taps_warp_bytes(g.K) + w * 32 * 20 <= max_smem) return w;
+  return 0;
+}
+
+template <typename T, int DH, int W>
+dsa3d_status_t bwd_taps_launch(const Shape& s, const BwdArgs& a, cudaStream_t st) {
+  const Geo g = make_geo(s);
+  const int smem = W * bwd_taps_warp_bytes(g.K);
+  auto kern = dsa3d_bwd_taps_kernel<T, DH, W>;
+  int grid = 0;
+  const int64_t items = (int64_t)a.hc * s.N;
+  dsa3d_status_t rc = launch_persistent(kern, W, smem, items, st, grid);
+  if (rc != DSA3D_OK) return rc;
+  TimedLaunch tl(kKernBwdTaps, st);
+  kern<<<grid, W * 32, smem, st>>>(
+      static_cast<const T*>(a.q), static_cast<const T*>(a.k), static_cast<const T*>(a.v), a.off,
+      a.lse, static_cast<const T*>(a.dout), static_cast<T*>(a.dq), a.doff, a.acc_k, a.acc_v,
+      a.acc_heads, a.h0, g, items);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+template <typename T, int DH>
+dsa3d_status_t bwd_taps_dispatch_w(const Shape& s, int warps, const BwdArgs& a, cudaStream_t st) {
+  switch (warps) {
+    case 4: return bwd_taps_launch<T, DH, 4>(s, a, st);
+    case 2: return bwd_taps_launch<T, DH, 2>(s, a, st);
+    case 1: return bwd_taps_launch<T, DH, 1>(s, a, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename T>
+dsa3d_status_t bwd_taps_dispatch(const Shape& s, int warps, const BwdArgs& a, cudaStream_t st,
+                                 bool finalize) {
+  dsa3d_status_t rc;
+  switch (s.dh) {
+    case 32: rc = bwd_taps_dispatch_w<T, 32>(s, warps, a, st); break;
+    case 64: rc = bwd_taps_dispatch_w<T, 64>(s, warps, a, st); break;
+    case 128: rc = bwd_taps_dispatch_w<T, 128>(s, warps, a, st); break;
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+  if (rc != DSA3D_OK || !finalize) return rc;
+  switch (s.dh) {
+    case 32: return bwd_finalize<T, 32>(s, a, st);
+    case 64: return bwd_finalize<T, 64>(s, a, st);
+    case 128: return bwd_finalize<T, 128>(s, a, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
 // Zero n16 16-byte words at p (the backward's fp32 accumulators).
 dsa3d_status_t zero16(void* p, size_t n16, cudaStream_t st) {
   const DeviceInfo d = device_info();
@@ -502,28 +651,16 @@ dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const 
   const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
   dsa3d_status_t rc = check_shape(s, dtype, 0);
   if (rc != DSA3D_OK) return rc;
-  if (!q || !k || !v || !offsets || !out) return DSA3D_ERR_INVALID_ARGUMENT;
-  const void* al[] = {q, k, v, offsets, out};
-  for (const void* p : al)
-    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return DSA3D_ERR_INVALID_ARGUMENT;
-  const size_t tb = (size_t)s.N * heads * dh * elem_size(dtype);
-  const Range in[] = {range_of(q, tb), range_of(k, tb), range_of(v, tb),
-                      range_of(offsets, (size_t)heads * s.N * 12)};
-  const Range ro = range_of(out, tb);
-  const Range rl = range_of(lse, lse ? (size_t)heads * s.N * 4 : 0);
-  for (const Range& r : in)
-    if (overlap(r, ro) || (lse && overlap(r, rl))) return DSA3D_ERR_INVALID_ARGUMENT;
-  if (lse && overlap(ro, rl)) return DSA3D_ERR_INVALID_ARGUMENT;
+  const size_t ob = (size_t)heads * s.N * 12;
+  if ((rc = check_forward_args(s, dtype, q, k, v, offsets, ob, out, lse)) != DSA3D_OK) return rc;
 
   if (workspace && workspace_bytes > 0 && mma_forward_ok(s, dtype)) {
     const size_t one = fwd_ws_bytes(s, 1);
     if (workspace_bytes < one) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
-    if (!aligned16(workspace)) return DSA3D_ERR_INVALID_ARGUMENT;
-    const Range rw = range_of(workspace, workspace_bytes);
-    for (const Range& r : in)
-      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
-    if (overlap(ro, rw) || (lse && overlap(rl, rw))) return DSA3D_ERR_INVALID_ARGUMENT;
+    const size_t tb = (size_t)s.N * heads * dh * elem_size(dtype);
+    const Range ins[] = {range_of(q, tb), range_of(k, tb), range_of(v, tb), range_of(offsets, ob)};
+    const Range outs[] = {range_of(out, tb), range_of(lse, lse ? (size_t)heads * s.N * 4 : 0)};
+    if ((rc = check_workspace(workspace, workspace_bytes, ins, 4, outs, 2)) != DSA3D_OK) return rc;
     int hg = heads;
     while (hg > 1 && fwd_ws_bytes(s, hg) > workspace_bytes) hg = (hg + 1) / 2;
     for (int h0 = 0; h0 < heads; h0 += hg) {
@@ -571,32 +708,14 @@ dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const
   const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
   dsa3d_status_t rc = check_shape(s, dtype, 0);
   if (rc != DSA3D_OK) return rc;
-  if (!q || !k || !v || !offsets || !lse || !dout || !dq || !dk || !dv || !doffsets)
-    return DSA3D_ERR_INVALID_ARGUMENT;
-  const void* al[] = {q, k, v, offsets, dout, dq, dk, dv, doffsets};
-  for (const void* p : al)
-    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
-  if (reinterpret_cast<uintptr_t>(lse) & 3u) return DSA3D_ERR_INVALID_ARGUMENT;
+  Range ins[6], outs[4];
+  rc = check_backward_args(s, dtype, q, k, v, offsets, lse, dout, dq, dk, dv, doffsets,
+                           (size_t)heads * s.N * 12, ins, outs);
+  if (rc != DSA3D_OK) return rc;
   const size_t tb = (size_t)s.N * heads * dh * elem_size(dtype);
-  const size_t ob = (size_t)heads * s.N * 12;
-  const Range ins[] = {range_of(q, tb), range_of(k, tb), range_of(v, tb), range_of(offsets, ob),
-                       range_of(lse, (size_t)heads * s.N * 4), range_of(dout, tb)};
-  const Range outs[] = {range_of(dq, tb), range_of(dk, tb), range_of(dv, tb),
-                        range_of(doffsets, ob)};
-  for (int i = 0; i < 4; i++) {
-    for (const Range& r : ins)
-      if (overlap(r, outs[i])) return DSA3D_ERR_INVALID_ARGUMENT;
-    for (int j = i + 1; j < 4; j++)
-      if (overlap(outs[i], outs[j])) return DSA3D_ERR_INVALID_ARGUMENT;
-  }
 
   if (mma_forward_ok(s, dtype) && workspace && workspace_bytes >= mma_bwd_ws_bytes(s, 1)) {
-    if (!aligned16(workspace)) return DSA3D_ERR_INVALID_ARGUMENT;
-    const Range rw = range_of(workspace, workspace_bytes);
-    for (const Range& r : ins)
-      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
-    for (const Range& r : outs)
-      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+    if ((rc = check_workspace(workspace, workspace_bytes, ins, 6, outs, 4)) != DSA3D_OK) return rc;
     int hg = heads;
     while (hg > 1 && mma_bwd_ws_bytes(s, hg) > workspace_bytes) hg = (hg + 1) / 2;
     for (int h0 = 0; h0 < heads; h0 += hg) {
@@ -612,12 +731,7 @@ dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const
   const size_t per_head = acc_bytes_per_head(s);
   if (dtype == DSA3D_BF16) {
     if (!workspace || workspace_bytes < per_head) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
-    if (!aligned16(workspace)) return DSA3D_ERR_INVALID_ARGUMENT;
-    const Range rw = range_of(workspace, workspace_bytes);
-    for (const Range& r : ins)
-      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
-    for (const Range& r : outs)
-      if (overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+    if ((rc = check_workspace(workspace, workspace_bytes, ins, 6, outs, 4)) != DSA3D_OK) return rc;
   }
 
   const Geo g = make_geo(s);
@@ -676,6 +790,76 @@ dsa3d_status_t dsa3d_backward_noalloc(const void* q, const void* k, const void* 
   return dsa3d_backward(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, scratch,
                         DSA3D_NOALLOC_SCRATCH_BYTES, F, Hp, Wp, heads, dh, kt, kh, kw, dtype,
                         stream);
+}
+
+dsa3d_status_t dsa3d_forward_taps(const void* q, const void* k, const void* v, const float* offsets,
+                                  void* out, float* lse, int F, int Hp, int Wp, int heads, int dh,
+                                  int kt, int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  dsa3d_status_t rc = check_shape(s, dtype, 0);
+  if (rc != DSA3D_OK) return rc;
+  const size_t ob = (size_t)heads * s.N * kt * kh * kw * 12;
+  if ((rc = check_forward_args(s, dtype, q, k, v, offsets, ob, out, lse)) != DSA3D_OK) return rc;
+  if (dtype == DSA3D_F32) return fwd_taps_dispatch<float>(s, q, k, v, offsets, out, lse, stream);
+  return fwd_taps_dispatch<__nv_bfloat16>(s, q, k, v, offsets, out, lse, stream);
+}
+
+size_t dsa3d_backward_taps_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt, int kh,
+                                           int kw, dsa3d_dtype_t dtype) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  if (check_shape(s, dtype, 0) != DSA3D_OK || dtype == DSA3D_F32) return 0;
+  return acc_bytes_per_head(s) * (size_t)heads;
+}
+
+dsa3d_status_t dsa3d_backward_taps(const void* q, const void* k, const void* v, const float* offsets,
+                                   const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                   float* doffsets, void* workspace, size_t workspace_bytes, int F,
+                                   int Hp, int Wp, int heads, int dh, int kt, int kh, int kw,
+                                   dsa3d_dtype_t dtype, cudaStream_t stream) {
+  const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
+  dsa3d_status_t rc = check_shape(s, dtype, 0);
+  if (rc != DSA3D_OK) return rc;
+  Range ins[6], outs[4];
+  rc = check_backward_args(s, dtype, q, k, v, offsets, lse, dout, dq, dk, dv, doffsets,
+                           (size_t)heads * s.N * kt * kh * kw * 12, ins, outs);
+  if (rc != DSA3D_OK) return rc;
+  const size_t per_head = acc_bytes_per_head(s);
+  if (dtype == DSA3D_BF16) {
+    if (!workspace || workspace_bytes < per_head) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+    if ((rc = check_workspace(workspace, workspace_bytes, ins, 6, outs, 4)) != DSA3D_OK) return rc;
+  }
+  const Geo g = make_geo(s);
+  const int warps = pick_taps_warps(g, device_info().max_smem);
+  if (warps == 0) return DSA3D_ERR_UNSUPPORTED;
+
+  BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.off = offsets; a.lse = lse;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.doff = doffsets;
+  if (dtype == DSA3D_F32) {
+    const size_t tb = (size_t)s.N * heads * dh * 4;
+    if ((rc = zero16(dk, tb / 16, stream)) != DSA3D_OK) return rc;
+    if ((rc = zero16(dv, tb / 16, stream)) != DSA3D_OK) return rc;
+    a.acc_k = static_cast<float*>(dk);
+    a.acc_v = static_cast<float*>(dv);
+    a.acc_heads = heads;
+    a.h0 = 0;
+    a.hc = heads;
+    return bwd_taps_dispatch<float>(s, warps, a, stream, false);
+  }
+  int hc_max = (int)(workspace_bytes / per_head);
+  if (hc_max > heads) hc_max = heads;
+  for (int h0 = 0; h0 < heads; h0 += hc_max) {
+    const int hc = (heads - h0 < hc_max) ? heads - h0 : hc_max;
+    const size_t half = (size_t)s.N * hc * dh;
+    a.acc_k = static_cast<float*>(workspace);
+    a.acc_v = a.acc_k + half;
+    a.acc_heads = hc;
+    a.h0 = h0;
+    a.hc = hc;
+    if ((rc = zero16(workspace, 2 * half * sizeof(float) / 16, stream)) != DSA3D_OK) return rc;
+    if ((rc = bwd_taps_dispatch<__nv_bfloat16>(s, warps, a, stream, true)) != DSA3D_OK) return rc;
+  }
+  return DSA3D_OK;
 }
 
 dsa3d_status_t dsa3d_timing_enable(int enable) {

@@ -56,8 +56,24 @@ struct Query {
 __device__ __forceinline__ int dim_of(const Geo& g, int a) { return a == 0 ? g.F : (a == 1 ? g.Hp : g.Wp); }
 __device__ __forceinline__ int win_of(const Geo& g, int a) { return a == 0 ? g.kt : (a == 1 ? g.kh : g.kw); }
 
-// Offset decode: i = floor(delta), f = delta - i in fp32 round-to-nearest, f == 1 carries.
-// Non-finite or |delta| > 2^24 makes the query invalid.  Then the per-axis tap and corner ranges.
+// One offset component: i = floor(delta), f = delta - i in fp32 round-to-nearest, f == 1 carries
+// into i.  Returns false (i = 0, f = 0) for a non-finite delta or |delta| > 2^24.
+__device__ __forceinline__ bool decode_delta(float d, int& ii, float& fr) {
+  ii = 0;
+  fr = 0.f;
+  if (!(fabsf(d) <= 16777216.f)) return false;  // also false for NaN
+  const float fl = floorf(d);
+  fr = __fsub_rn(d, fl);
+  ii = (int)fl;
+  if (fr == 1.0f) {
+    ii += 1;
+    fr = 0.f;
+  }
+  return true;
+}
+
+// Offset decode of a per-token offset (decode_delta on each axis; an invalid component makes
+// the query invalid), then the per-axis tap and corner ranges.
 // The forward reads only corners with a nonzero weight (the +1 plane only when f != 0).  With
 // for_grad the +1 plane is read whenever it lies in the volume: at f == 0 its weight is zero but
 // the derivative of the weight along that axis is not.
@@ -72,20 +88,9 @@ __device__ __forceinline__ Query decode_query(const Geo& g, const float* __restr
   const int p[3] = {t, y, x};
 #pragma unroll
   for (int a = 0; a < 3; a++) {
-    const float d = __ldg(o + a);
-    int ii = 0;
-    float fr = 0.f;
-    if (!(fabsf(d) <= 16777216.f)) {  // also false for NaN
-      Q.ok = false;
-    } else {
-      const float fl = floorf(d);
-      fr = __fsub_rn(d, fl);
-      ii = (int)fl;
-      if (fr == 1.0f) {
-        ii += 1;
-        fr = 0.f;
-      }
-    }
+    int ii;
+    float fr;
+    if (!decode_delta(__ldg(o + a), ii, fr)) Q.ok = false;
     const int k = win_of(g, a), D = dim_of(g, a);
     const int org = p[a] + ii - (k - 1) / 2;
     const int up = (fr != 0.f) ? 1 : 0;

@@ -24,6 +24,8 @@ enum KernelId {
   kKernBwdDq,
   kKernBwdKv,
   kKernPairV,
+  kKernFwdTaps,
+  kKernBwdTaps,
   kKernCount
 };
 inline const char* kernel_name(int id) {
@@ -31,7 +33,8 @@ inline const char* kernel_name(int id) {
       "dsa3d_fwd_kernel",      "dsa3d_bwd_kernel",        "dsa3d_bwd_finalize_kernel",
       "dsa3d_zero_kernel",     "dsa3d_fwd_mma_kernel",    "dsa3d_sort_count_kernel",
       "dsa3d_scan_kernels",    "dsa3d_sort_fill_kernel",  "dsa3d_bwd_q_kernel",
-      "dsa3d_bwd_dq_kernel",   "dsa3d_bwd_kv_kernel",     "dsa3d_pair_v_kernel"};
+      "dsa3d_bwd_dq_kernel",   "dsa3d_bwd_kv_kernel",     "dsa3d_pair_v_kernel",
+      "dsa3d_fwd_taps_kernel", "dsa3d_bwd_taps_kernel"};
   return names[id];
 }
 

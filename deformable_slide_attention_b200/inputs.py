@@ -19,9 +19,14 @@ Workloads (draw order q, k, v, offsets, dO from one torch.Generator seeded per w
                    + N(0, 0.5^2) with kt, ky, kx in {1, 2} and phi ~ U(0, 2 pi) drawn per
                    (head, axis), A = sqrt(2 * 15.75) so the total std is 4; seed 4; forward +
                    backward.  Generated on the device (its tensors are 17 GB each).
+  720p-train-taps-bf16  the 720p-train-bf16 shapes with per-tap offsets: one offset 3-vector per
+                   (head, token, window tap), [heads][N][243][3] (5.4 GB), each component
+                   N(0, 3^2) unclamped like the per-token 720p offsets; dO ~ N(0,1); seed 5;
+                   forward + backward.  Generated on the device.
 
 q, k, v and dO are N(0,1), rounded to bf16 (round to nearest even) for the bf16 workloads.
-Layouts: q/k/v/dO [N][heads][dh]; offsets [heads][N][3] fp32 in (dt, dy, dx) order.
+Layouts: q/k/v/dO [N][heads][dh]; offsets [heads][N][3] fp32 in (dt, dy, dx) order, or
+[heads][N][K][3] (K = kt*kh*kw, tap order u, v, w with w fastest) for per-tap workloads.
 """
 from __future__ import annotations
 
@@ -46,6 +51,7 @@ class Workload:
     scale: float = 0.0  # offset range / std
     backward: bool = False
     device_generated: bool = False
+    per_tap: bool = False  # offsets per (head, token, tap) instead of per (head, token)
     extra: dict = field(default_factory=dict)
 
     @property
@@ -55,6 +61,10 @@ class Workload:
     @property
     def N(self):
         return self.F * self.Hp * self.Wp
+
+    @property
+    def K(self):
+        return self.window[0] * self.window[1] * self.window[2]
 
     @property
     def torch_dtype(self):
@@ -68,6 +78,8 @@ WORKLOADS = [
     Workload("720p-train-bf16", 32, 45, 80, 16, 128, (3, 9, 9), "bf16", 3, "normal", 3.0, backward=True),
     Workload("1080p-long-bf16", 256, 68, 120, 32, 128, (3, 9, 9), "bf16", 4, "smooth", 4.0,
              backward=True, device_generated=True),
+    Workload("720p-train-taps-bf16", 32, 45, 80, 16, 128, (3, 9, 9), "bf16", 5, "normal", 3.0,
+             backward=True, device_generated=True, per_tap=True),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS}
 
@@ -97,14 +109,18 @@ def _coords(F, Hp, Wp, device):
     return t, y, x
 
 
-def offsets_uniform(gen, heads, N, half_range, device="cpu"):
-    u = torch.empty((heads, N, 3), dtype=torch.float32, device=device)
+def _offset_shape(heads, N, taps):
+    return (heads, N, 3) if taps is None else (heads, N, taps, 3)
+
+
+def offsets_uniform(gen, heads, N, half_range, device="cpu", taps=None):
+    u = torch.empty(_offset_shape(heads, N, taps), dtype=torch.float32, device=device)
     u.uniform_(-half_range, half_range, generator=gen)
     return u
 
 
-def offsets_normal(gen, heads, N, std, device="cpu"):
-    o = torch.empty((heads, N, 3), dtype=torch.float32, device=device)
+def offsets_normal(gen, heads, N, std, device="cpu", taps=None):
+    o = torch.empty(_offset_shape(heads, N, taps), dtype=torch.float32, device=device)
     o.normal_(0.0, std, generator=gen)
     return o
 
@@ -168,10 +184,13 @@ def make(w: Workload, device="cpu", with_dout=None):
     else:
         for name in ("q", "k", "v"):
             out[name] = _normal(shape, gen, "cpu", w.torch_dtype)
+    taps = w.K if w.per_tap else None
     if w.offsets == "uniform":
-        off = offsets_uniform(gen, w.heads, N, w.scale, gen_device)
+        off = offsets_uniform(gen, w.heads, N, w.scale, gen_device, taps)
     elif w.offsets == "normal":
-        off = offsets_normal(gen, w.heads, N, w.scale, gen_device)
+        off = offsets_normal(gen, w.heads, N, w.scale, gen_device, taps)
+    elif w.per_tap:
+        raise ValueError(f"per-tap offsets are drawn uniform or normal, not {w.offsets}")
     elif w.offsets == "normal_clamped_zero_blocks":
         off = offsets_normal_clamped_zero_blocks(gen, w.F, w.Hp, w.Wp, w.heads, w.scale)
     elif w.offsets == "smooth":
@@ -192,8 +211,8 @@ def make(w: Workload, device="cpu", with_dout=None):
 
 
 def custom(F, Hp, Wp, heads, dh, window, dtype="f32", seed=0, offsets="uniform", scale=1.5,
-           with_dout=True):
+           with_dout=True, per_tap=False):
     """A small ad-hoc workload (CPU tensors) for tests; same draw order as the named ones."""
     w = Workload(f"custom-{F}x{Hp}x{Wp}", F, Hp, Wp, heads, dh, tuple(window), dtype, seed, offsets,
-                 scale, backward=with_dout)
+                 scale, backward=with_dout, per_tap=per_tap)
     return w, make(w, "cpu", with_dout)

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define DSA3D_ABI_VERSION 2
+#define DSA3D_ABI_VERSION 3
 
 typedef enum {
     DSA3D_OK = 0,
@@ -145,6 +145,50 @@ dsa3d_status_t dsa3d_backward_noalloc(const void *q, const void *k, const void *
                                       float *doffsets, int F, int Hp, int Wp, int heads, int dh,
                                       int kt, int kh, int kw, dsa3d_dtype_t dtype,
                                       cudaStream_t stream);
+
+/*
+ * Per-tap offsets: the offset tensor of the 3D-DSA definition (MegaSlide-DiT, Eq. 1) taken
+ * literally, one 3-vector per (head, query, window tap) instead of one per (head, query).
+ *   offsets, doffsets: [heads][N][K][3] fp32, K = kt*kh*kw, taps in (u, v, w) order with u (the
+ *   temporal tap) outermost and w fastest; components (dt, dy, dx).
+ * Tap tau of query p samples K and V at p + tau + delta[h,p,tau] (trilinear, align_corners=True).
+ * Each tap's offset is decoded on its own as above (floor, fp32 fraction, carry); a non-finite
+ * component or |component| > 2^24 masks that tap only, and a tap whose sample position leaves the
+ * closed box [0, dim-1] is masked.  A query with no valid tap gets out = 0, lse = -inf and zero
+ * gradients.  With every tap's offset equal to one per-token offset the results equal those of
+ * dsa3d_forward / dsa3d_backward.  The other arguments, layouts and errors are those of
+ * dsa3d_forward and dsa3d_backward.  These entry points always run the general CUDA-core kernels
+ * (every tap reads its own 8 corners, so the shared-box tensor-core form does not apply).
+ */
+dsa3d_status_t dsa3d_forward_taps(const void *q, const void *k, const void *v,
+                                  const float *offsets, void *out, float *lse, int F, int Hp,
+                                  int Wp, int heads, int dh, int kt, int kh, int kw,
+                                  dsa3d_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * Workspace of dsa3d_backward_taps for all heads in one pass: the fp32 dK/dV accumulators,
+ * 2 * N * dh * 4 bytes per head with bf16 I/O (any multiple of one head's share works; heads are
+ * then processed in groups), 0 with fp32 I/O (the gradients accumulate in dk/dv themselves) and
+ * for invalid shapes.
+ */
+size_t dsa3d_backward_taps_workspace_bytes(int F, int Hp, int Wp, int heads, int dh, int kt,
+                                           int kh, int kw, dsa3d_dtype_t dtype);
+
+/*
+ * Backward with per-tap offsets: gradients of sum(out * dout) with respect to q, k, v and the
+ * per-tap offsets (doffsets [heads][N][K][3], the derivative of each tap's trilinear weights
+ * within its cell, masks and integer parts held fixed).  Needs the lse of dsa3d_forward_taps;
+ * the softmax Jacobian's row term D = sum_tau P dP is recomputed exactly, as in dsa3d_backward.
+ * The other arguments and errors are those of dsa3d_backward, with offsets and doffsets
+ * [heads][N][K][3].  Its shared memory grows with the tap count (20 bytes per tap per warp):
+ * windows of more than about 11,000 taps return DSA3D_ERR_UNSUPPORTED.
+ */
+dsa3d_status_t dsa3d_backward_taps(const void *q, const void *k, const void *v,
+                                   const float *offsets, const float *lse, const void *dout,
+                                   void *dq, void *dk, void *dv, float *doffsets, void *workspace,
+                                   size_t workspace_bytes, int F, int Hp, int Wp, int heads,
+                                   int dh, int kt, int kh, int kw, dsa3d_dtype_t dtype,
+                                   cudaStream_t stream);
 
 /*
  * Synchronises `stream` and reports DSA3D_ERR_DEVICE_CHECK if any kernel of this library on the

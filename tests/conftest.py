@@ -27,5 +27,5 @@ def gpu_lib():
     from deformable_slide_attention_b200 import abi, build
     build.build()
     assert torch.cuda.is_available(), "GPU test run without a CUDA device"
-    assert abi.dsa3d_abi_version() == 2
+    assert abi.dsa3d_abi_version() == 3
     return abi

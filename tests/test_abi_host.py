@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings():
-    assert abi.dsa3d_abi_version() == 2
+    assert abi.dsa3d_abi_version() == 3
     for s in range(6):
         assert abi.dsa3d_status_string(s)
     assert abi.dsa3d_status_string(0) == "ok"
@@ -124,3 +124,56 @@ def test_backward_rejects_bad_arguments():
     alias = list(ptr)
     alias[7] = ptr[0]
     assert call(alias, wsb=1 << 30) == 1
+
+
+def fwd_taps(**kw):
+    a = {**ARGS, **kw}
+    ptrs = [kw.get(n, P * (i + 1)) for i, n in enumerate(["q", "k", "v", "off", "out", "lse"])]
+    return abi.dsa3d_forward_taps(*ptrs, a["F"], a["Hp"], a["Wp"], a["heads"], a["dh"], a["kt"],
+                                  a["kh"], a["kw"], kw.get("dtype", abi.DSA3D_BF16), 0)
+
+
+def test_forward_taps_rejects_bad_arguments():
+    INV, UNS = 1, 2
+    assert fwd_taps(v=0) == INV
+    assert fwd_taps(off=P * 4 + 4) == INV   # misaligned
+    assert fwd_taps(kh=4) == INV            # even window
+    assert fwd_taps(dtype=3) == INV
+    assert fwd_taps(dh=96) == UNS
+    assert fwd_taps(kw=17) == UNS           # larger than 2*Wp-1
+    # the per-tap offsets are K = 27 times the per-token size (2 * 256 * 27 * 12 bytes): an
+    # output placed 100 KB after their start overlaps them
+    assert fwd_taps(off=P * 8, out=P * 8 + 100_000) == INV
+
+
+def test_backward_taps_workspace_bytes_and_rejections():
+    F, Hp, Wp, H, kt, kh, kw = 4, 8, 8, 2, 3, 3, 3
+    N = F * Hp * Wp
+    # fp32 dK/dV accumulators of every head with bf16 I/O (no tensor-core path for per-tap
+    # offsets), none with fp32 I/O
+    for dh in (32, 64, 128):
+        assert abi.dsa3d_backward_taps_workspace_bytes(F, Hp, Wp, H, dh, kt, kh, kw, abi.DSA3D_BF16) == 2 * N * dh * 4 * H
+        assert abi.dsa3d_backward_taps_workspace_bytes(F, Hp, Wp, H, dh, kt, kh, kw, abi.DSA3D_F32) == 0
+    assert abi.dsa3d_backward_taps_workspace_bytes(F, Hp, Wp, H, 48, kt, kh, kw, abi.DSA3D_BF16) == 0
+    # q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace
+    ptr = [P * (i + 1) for i in range(11)]
+    a = ARGS
+    call = lambda ptrs, wsb=0, dtype=abi.DSA3D_BF16: abi.dsa3d_backward_taps(
+        *ptrs, wsb, a["F"], a["Hp"], a["Wp"], a["heads"], a["dh"], a["kt"], a["kh"], a["kw"], dtype, 0)
+    for i in (4, 5):  # lse, dout
+        bad = list(ptr)
+        bad[i] = 0
+        assert call(bad, wsb=1 << 30) == 1
+    misaligned = list(ptr)
+    misaligned[5] += 8
+    assert call(misaligned, wsb=1 << 30) == 1
+    assert call(ptr, wsb=1000) == 3  # smaller than one head's accumulators
+    alias = list(ptr)
+    alias[9] = ptr[3] + 16 * 4096  # doffsets inside the per-tap offsets
+    assert call(alias, wsb=1 << 30) == 1
+    alias = list(ptr)
+    alias[6] = ptr[5]  # dq on top of dout
+    assert call(alias, wsb=1 << 30) == 1
+    overlap_ws = list(ptr)
+    overlap_ws[10] = ptr[2]  # workspace on top of v
+    assert call(overlap_ws, wsb=1 << 20) == 1
