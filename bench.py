@@ -56,30 +56,57 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only this many of the workload's heads (small profiling captures); "
+                         "0 = all")
     return ap.parse_args(argv)
 
 
 # DRAM traffic per (token, head) of each kernel, dram__bytes_read.sum + dram__bytes_write.sum
-# from one ncu capture on the 720p training workload (16 heads x 115,200 tokens per launch),
-# valid while the kernel sources hash to "sources"; the traffic of a launch is this times the
-# (token, head) items it processes (the kernels' traffic grows in proportion to the items).
-NCU_TRAFFIC = {
-    "sources": "ade4806829a0e1b6",
-    "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
-    "bytes_per_item": {
-        "dsa3d_fwd_mma_kernel": 1086.2,
-        "dsa3d_bwd_q_kernel": 2260.3,
-        "dsa3d_bwd_dq_kernel": 1652.0,
-        "dsa3d_bwd_kv_kernel": 2213.6,
-    },
-}
+# from ncu captures (the file named by "capture" gives the command and workload), valid while the
+# files that define those kernels and their launches ("files", under the package's csrc/) hash to
+# "sources"; the traffic of a launch is this times the (token, head) items it processes (the
+# kernels' traffic grows in proportion to the items).
+TENSOR_CORE_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_fwd_mma.cuh", "dsa3d_bwd_mma.cuh",
+                     "dsa3d_sort.cuh"]
+PER_TAP_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_taps.cuh", "dsa3d_bwd.cuh", "dsa3d_fwd.cuh"]
+NCU_TRAFFIC = [
+    {"files": TENSOR_CORE_FILES, "sources": "8eaed48778e074f4",
+     "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
+     "bytes_per_item": {
+         "dsa3d_fwd_mma_kernel": 1084.2,
+         "dsa3d_bwd_q_kernel": 2254.5,
+         "dsa3d_bwd_dq_kernel": 1650.5,
+         "dsa3d_bwd_kv_kernel": 2206.3,
+     }},
+    {"files": PER_TAP_FILES, "sources": "df10cf32e12d6270",
+     "capture": "profiles/per_tap_kernels_720p-train-taps-bf16.md",
+     "bytes_per_item": {
+         "dsa3d_fwd_taps_kernel": 18471.7,
+         "dsa3d_bwd_taps_kernel": 191471.2,
+     }},
+]
 
 
-def sources_digest():
+def traffic_per_item(kernel):
+    """(DRAM bytes per item, capture file) of a kernel from a capture of the current sources, or
+    (None, None)."""
+    for cap in NCU_TRAFFIC:
+        if kernel in cap["bytes_per_item"] and cap["sources"] == sources_digest(cap["files"]):
+            return cap["bytes_per_item"][kernel], cap["capture"]
+    return None, None
+
+
+def sources_digest(names=None):
+    """Digest of the named csrc files (all of csrc/ and include/ when names is None)."""
     import glob
     import hashlib
-    files = sorted(glob.glob(os.path.join(ROOT, "deformable_slide_attention_b200", "csrc", "*")) +
-                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    csrc = os.path.join(ROOT, "deformable_slide_attention_b200", "csrc")
+    if names is None:
+        files = sorted(glob.glob(os.path.join(csrc, "*")) +
+                       glob.glob(os.path.join(ROOT, "include", "*.h")))
+    else:
+        files = sorted(os.path.join(csrc, n) for n in names)
     h = hashlib.sha256()
     for f in files:
         h.update(os.path.basename(f).encode())
@@ -217,15 +244,17 @@ def calibrated_items(w, hin, threads, budget_s):
     """Items (a multiple of the thread count) that take about budget_s: time growing samples until
     one lasts half a second, so the per-call overhead does not distort the estimate."""
     threads = max(threads, 1)
-    oracle_sample(w, hin, threads, 12344, threads)  # warm the inputs' pages
+    oracle_sample(w, hin, min(w.N, threads), 12344, threads)  # warm the inputs' pages
     rounds = 4
     while True:
-        t = oracle_sample(w, hin, rounds * threads, 12345, threads)
-        if t >= 0.5 or rounds >= (1 << 20):
+        t = oracle_sample(w, hin, min(w.N, rounds * threads), 12345, threads)
+        if t >= 0.5 or rounds >= (1 << 20) or rounds * threads >= w.N:
             break
         rounds *= 4
+    rounds = min(rounds * threads, w.N) / threads
     per_round = t / rounds  # one item per thread
-    return max(1, int(budget_s / max(per_round, 1e-9))) * threads
+    # at most one head's queries (a sample is drawn without replacement from them)
+    return min(w.N, max(1, int(budget_s / max(per_round, 1e-9))) * threads)
 
 
 def cpu_baseline(w, inp, budget_s):
@@ -315,6 +344,8 @@ def main(argv=None):
     build.build()
 
     base = inputs.BY_NAME[args.workload]
+    if args.heads:
+        base = dataclasses.replace(base, heads=args.heads)
     w = ranks.clip_workload(base, rank)
     inp = inputs.make(w, dev, with_dout=True)
     code = abi.DSA3D_BF16 if w.dtype == "bf16" else abi.DSA3D_F32
@@ -392,12 +423,11 @@ def main(argv=None):
         items_per_launch = w.heads * w.N / launches_per_step
         alg = alg_bytes_per_item(w, kname) * items_per_launch
         achieved = alg / (avg_ms / 1000.0) / 1e9
-        per_item = NCU_TRAFFIC["bytes_per_item"].get(kname)
-        traffic = (per_item * items_per_launch
-                   if per_item is not None and sources_digest() == NCU_TRAFFIC["sources"] else None)
+        per_item, capture = traffic_per_item(kname)
+        traffic = per_item * items_per_launch if per_item is not None else None
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic, "traffic_unit": "bytes per launch",
-                "traffic_source": NCU_TRAFFIC["capture"] if traffic is not None else None,
+                "traffic_source": capture,
                 "kernel": kname,
                 "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)"
                                if peak_src == "measured" else "fallback 6.65 TB/s"}
