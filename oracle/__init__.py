@@ -8,11 +8,16 @@ module compiles it with gcc on first use and marshals numpy/torch CPU arrays thr
 
 Source of the operator: MegaSlide-DiT (arXiv 2607.22696), the 3D-DSA definition (Eq. 1 and the
 softmax over the k_t x k_h x k_w neighbourhood that follows it).  The readings the paper leaves
-open are listed in the C file's header (R1..R8).
+open are listed in the C file's header (R1..R10).  Besides the attention term, the module holds
+the other two parts of Eq. 1's layer: the DWConv3D term (a depthwise 3-D convolution, R9) and the
+offset network (a depthwise 3-D convolution and a pointwise linear layer, R10).
 
-Parity pins: every routine here is pinned by ``tests/test_oracle_pins.py`` against brute-force
-dense attention, torch's ``grid_sample``, finite differences and an independent torch autograd
-restatement.  The one unpinned reading is the score scale (R3, 1/sqrt(dh)).
+Parity pins: every routine here is pinned, the attention by ``tests/test_oracle_pins.py``
+against brute-force dense attention, torch's ``grid_sample``, finite differences and an
+independent torch autograd restatement, and the convolution and offset network by
+``tests/test_oracle_layer_pins.py`` against torch's conv3d and autograd, closed forms and
+finite differences through the whole layer.  The one unpinned reading is the score scale (R3,
+1/sqrt(dh)); the convolution's kernel extent (R9, R10) is a reading the pins take as given.
 """
 from __future__ import annotations
 
@@ -65,6 +70,12 @@ def _load():
             lib.dsa3d_oracle_forward_taps.argtypes = lib.dsa3d_oracle_forward.argtypes
             lib.dsa3d_oracle_backward_taps.restype = ctypes.c_int
             lib.dsa3d_oracle_backward_taps.argtypes = lib.dsa3d_oracle_backward.argtypes
+            cdims = [ctypes.c_int] * 7  # F, Hp, Wp, C, kt, kh, kw
+            lib.dsa3d_oracle_dwconv3d.restype = ctypes.c_int
+            lib.dsa3d_oracle_dwconv3d.argtypes = [ctypes.c_int, vp, vp, vp, *cdims, vp, ctypes.c_int]
+            lib.dsa3d_oracle_dwconv3d_backward.restype = ctypes.c_int
+            lib.dsa3d_oracle_dwconv3d_backward.argtypes = [ctypes.c_int, vp, vp, vp, *cdims, vp,
+                                                           vp, vp, ctypes.c_int]
             lib.dsa3d_oracle_tap.restype = ctypes.c_int
             lib.dsa3d_oracle_tap.argtypes = [ctypes.c_int, vp, vp, *dims, ctypes.c_int,
                                              ctypes.c_int64, ctypes.c_int, i64p, vp, vp, vp]
@@ -223,3 +234,84 @@ def full_backward(q, k, v, offsets, dout, dims, window, threads=None, per_tap=Fa
                                 per_tap=per_tap)
     r = lambda a: a.reshape(heads, N, dh).transpose(1, 0, 2).copy()
     return r(dq), doff.reshape((heads, N, -1, 3) if per_tap else (heads, N, 3)), r(dk), r(dv)
+
+
+# --- the DWConv3D term and the offset network (R9, R10) ----------------------------------------
+def _conv_args(x, weight, bias, dims):
+    xa, io = _as_io(x)
+    F, Hp, Wp = dims
+    N = F * Hp * Wp
+    if xa.ndim != 2 or xa.shape[0] != N:
+        raise ValueError(f"x must be [N={N}][C], got {xa.shape}")
+    C = xa.shape[1]
+    w = _f32(weight)
+    if w.ndim != 4 or w.shape[0] != C:
+        raise ValueError(f"weight must be [C={C}][kt][kh][kw], got {w.shape}")
+    b = None if bias is None else _f32(bias).reshape(C)
+    return xa, io, w, b, C, w.shape[1:]
+
+
+def dwconv3d(x, weight, bias, dims, threads=None):
+    """Depthwise 3-D convolution (R9): x [N][C] (fp32 or bf16), weight [C][kt][kh][kw] fp32,
+    bias [C] fp32 or None.  Returns Y [N][C] float64 (zero padding, output grid = token grid)."""
+    xa, io, w, b, C, (kt, kh, kw) = _conv_args(x, weight, bias, dims)
+    y = np.zeros((xa.shape[0], C), np.float64)
+    rc = _load().dsa3d_oracle_dwconv3d(io, _ptr(xa), _ptr(w), _ptr(b), *dims, C, kt, kh, kw,
+                                       _ptr(y), _threads(threads))
+    if rc != 0:
+        raise ValueError("dsa3d_oracle_dwconv3d: bad arguments")
+    return y
+
+
+def dwconv3d_backward(x, weight, dy, dims, threads=None):
+    """Gradients of sum(Y * dy) for Y = dwconv3d(x, weight, bias): (dx [N][C], dweight
+    [C][kt][kh][kw], dbias [C]), all float64."""
+    xa, io, w, _, C, (kt, kh, kw) = _conv_args(x, weight, None, dims)
+    g = np.ascontiguousarray(dy, dtype=np.float64).reshape(xa.shape[0], C)
+    dx = np.zeros((xa.shape[0], C), np.float64)
+    dw = np.zeros(w.shape, np.float64)
+    db = np.zeros(C, np.float64)
+    rc = _load().dsa3d_oracle_dwconv3d_backward(io, _ptr(xa), _ptr(w), _ptr(g), *dims, C, kt, kh,
+                                                kw, _ptr(dx), _ptr(dw), _ptr(db), _threads(threads))
+    if rc != 0:
+        raise ValueError("dsa3d_oracle_dwconv3d_backward: bad arguments")
+    return dx, dw, db
+
+
+def _offset_layout(flat, heads, taps):
+    """[N][heads * (taps) * 3] -> [heads][N][3] or [heads][N][taps][3]."""
+    N = flat.shape[0]
+    if taps is None:
+        return np.ascontiguousarray(flat.reshape(N, heads, 3).transpose(1, 0, 2))
+    return np.ascontiguousarray(flat.reshape(N, heads, taps, 3).transpose(1, 0, 2, 3))
+
+
+def offset_head(x, dw_weight, dw_bias, pw_weight, pw_bias, dims, heads, taps=None, threads=None):
+    """The offset network (R10): Z = dwconv3d(x, dw_weight, dw_bias), then the pointwise layer
+    O = Z @ pw_weight + pw_bias with pw_weight [C][heads * 3] (per token) or [C][heads * taps * 3]
+    (per tap).  Returns the offsets in the attention's layout, [heads][N][3] or
+    [heads][N][taps][3], float64 (the attention takes them rounded to fp32)."""
+    z = dwconv3d(x, dw_weight, dw_bias, dims, threads)
+    pw = np.asarray(_f32(pw_weight), np.float64)
+    width = heads * 3 * (1 if taps is None else taps)
+    if pw.shape != (z.shape[1], width):
+        raise ValueError(f"pw_weight must be [C][{width}], got {pw.shape}")
+    flat = z @ pw + np.asarray(_f32(pw_bias), np.float64).reshape(width)
+    return _offset_layout(flat, heads, taps)
+
+
+def offset_head_backward(x, dw_weight, dw_bias, pw_weight, doffsets, dims, threads=None):
+    """Gradients of sum(offsets * doffsets) for offsets = offset_head(...): (dx [N][C],
+    d dw_weight, d dw_bias, d pw_weight [C][width], d pw_bias [width]), float64.  doffsets is in
+    the attention's layout ([heads][N][3] or [heads][N][taps][3])."""
+    z = dwconv3d(x, dw_weight, dw_bias, dims, threads)
+    g = np.asarray(doffsets, np.float64)
+    N = z.shape[0]
+    # back to the pointwise layer's [N][heads * (taps) * 3] order
+    g_flat = np.ascontiguousarray(np.moveaxis(g, 1, 0)).reshape(N, -1)
+    pw = np.asarray(_f32(pw_weight), np.float64)
+    d_pw = z.T @ g_flat
+    d_pb = g_flat.sum(axis=0)
+    dz = g_flat @ pw.T
+    dx, d_dw, d_db = dwconv3d_backward(x, dw_weight, dz, dims, threads)
+    return dx, d_dw, d_db, d_pw, d_pb

@@ -44,6 +44,18 @@
  *       own, and a non-finite or too large offset masks only that tap (R5 applies per tap).
  *       The offset gradient is per tap, [heads][N][K][3].  With every tap's offset equal to one
  *       per-token offset the result is that of R1.
+ *   R9  The DWConv3D term of Eq. 1 (dsa3d_oracle_dwconv3d): a depthwise 3-D convolution of the
+ *       layer input X [N][C], C = heads * dh, with a kernel of the window's extent
+ *       (kt x kh x kw: the paper names one neighbourhood size per layer), stride 1, zero
+ *       padding so the output grid equals the token grid, a bias per channel, and
+ *       cross-correlation (PyTorch's conv3d convention, which the paper's implementation
+ *       uses).  Its output adds to the attention output channel by channel, c = h * dh + e.
+ *   R10 The offset network ("a lightweight depthwise 3D convolution followed by a linear
+ *       layer"; nn.Conv3d with groups = hidden size, then pointwise convolutions): its own
+ *       depthwise convolution as in R9, then one pointwise linear layer C -> heads * 3 (per
+ *       token, R1) or heads * K * 3 (per tap, R8) with bias; output channel (h * 3 + a), or
+ *       ((h * K + tau) * 3 + a), is offset component a of head h (and tap tau).  The pointwise
+ *       layer is a matrix product and is composed in the Python module.
  *
  * Layouts: q, k, v, dout: [N][heads][dh] (token n = (t*Hp + y)*Wp + x), in fp32 or bf16 bits.
  * offsets: [heads][N][3] fp32, order (dt, dy, dx).  A query or key "item" is h*N + n.
@@ -524,4 +536,87 @@ int dsa3d_oracle_tap(int io, const void *src, const float *off, int F, int Hp, i
     frac[0] = d.f[0]; frac[1] = d.f[1]; frac[2] = d.f[2];
     sample(&P, src, h, base, d.f, samp, dsamp, NULL);
     return valid;
+}
+
+/*
+ * Depthwise 3-D convolution: the DWConv3D term of Eq. 1 and the first layer of the offset
+ * network (readings R9 and R10, MegaSlide-DiT, the 3D-DSA definition).  For every channel c of
+ * X [N][C] (token n = (t*Hp + y)*Wp + x) and every output token p = (t, y, x):
+ *
+ *   Y[p][c] = b[c] + sum_{u<kt, v<kh, w<kw} W[c][u][v][w] * X[(t + u - r_t, y + v - r_h, x + w - r_w)][c]
+ *
+ * with r = (k-1)/2 and X = 0 outside the volume (zero padding; the output grid is the input
+ * grid).  This is cross-correlation, the convention of PyTorch's conv3d with groups = C and
+ * padding k // 2.  W is [C][kt][kh][kw] fp32, b is [C] fp32 (may be NULL: no bias), X is fp32 or
+ * bf16 bits; Y is double.  Each output is summed directly over its window, tap by tap.
+ */
+static int conv_args(int F, int Hp, int Wp, int C, int kt, int kh, int kw, int io) {
+    if (F < 1 || Hp < 1 || Wp < 1 || C < 1) return -1;
+    if (kt < 1 || kh < 1 || kw < 1 || !(kt & 1) || !(kh & 1) || !(kw & 1)) return -1;
+    if (io != IO_F32 && io != IO_BF16) return -1;
+    return 0;
+}
+
+int dsa3d_oracle_dwconv3d(int io, const void *x, const float *w, const float *b, int F, int Hp,
+                          int Wp, int C, int kt, int kh, int kw, double *y, int n_threads) {
+    if (conv_args(F, Hp, Wp, C, kt, kh, kw, io)) return -1;
+    const int64_t N = (int64_t)F * Hp * Wp;
+    const int rt = (kt - 1) / 2, rh = (kh - 1) / 2, rw = (kw - 1) / 2;
+#pragma omp parallel for schedule(static) num_threads(n_threads > 0 ? n_threads : 1)
+    for (int64_t n = 0; n < N; n++) {
+        const int64_t x0 = n % Wp, y0 = (n / Wp) % Hp, t0 = n / ((int64_t)Wp * Hp);
+        for (int c = 0; c < C; c++) {
+            double acc = b ? (double)b[c] : 0.0;
+            for (int u = 0; u < kt; u++)
+                for (int v = 0; v < kh; v++)
+                    for (int ww = 0; ww < kw; ww++) {
+                        const int64_t ts = t0 + u - rt, ys = y0 + v - rh, xs = x0 + ww - rw;
+                        if (ts < 0 || ts >= F || ys < 0 || ys >= Hp || xs < 0 || xs >= Wp) continue;
+                        const int64_t src = (ts * Hp + ys) * Wp + xs;
+                        acc += (double)w[((int64_t)c * kt + u) * kh * kw + v * kw + ww] *
+                               rd(x, io, src * C + c);
+                    }
+            y[n * C + c] = acc;
+        }
+    }
+    return 0;
+}
+
+/*
+ * Backward of dsa3d_oracle_dwconv3d for an upstream gradient dY [N][C] (double):
+ *   dX[m][c]       = sum over outputs p and taps whose source is m of W[c][u][v][w] * dY[p][c]
+ *   dW[c][u][v][w] = sum_p dY[p][c] * X[p + (u - r_t, v - r_h, w - r_w)][c]   (in-volume sources)
+ *   db[c]          = sum_p dY[p][c]
+ * Written as the forward's loop with each product's contributions accumulated into its
+ * operands; threads own channels, so no two threads touch the same accumulator.
+ */
+int dsa3d_oracle_dwconv3d_backward(int io, const void *x, const float *w, const double *dy, int F,
+                                   int Hp, int Wp, int C, int kt, int kh, int kw, double *dx,
+                                   double *dw, double *db, int n_threads) {
+    if (conv_args(F, Hp, Wp, C, kt, kh, kw, io)) return -1;
+    const int64_t N = (int64_t)F * Hp * Wp;
+    const int K = kt * kh * kw;
+    const int rt = (kt - 1) / 2, rh = (kh - 1) / 2, rw = (kw - 1) / 2;
+    for (int64_t e = 0; e < N * C; e++) dx[e] = 0.0;
+    for (int64_t e = 0; e < (int64_t)C * K; e++) dw[e] = 0.0;
+    for (int c = 0; c < C; c++) db[c] = 0.0;
+#pragma omp parallel for schedule(static) num_threads(n_threads > 0 ? n_threads : 1)
+    for (int c = 0; c < C; c++) {
+        for (int64_t n = 0; n < N; n++) {
+            const int64_t x0 = n % Wp, y0 = (n / Wp) % Hp, t0 = n / ((int64_t)Wp * Hp);
+            const double g = dy[n * C + c];
+            db[c] += g;
+            for (int u = 0; u < kt; u++)
+                for (int v = 0; v < kh; v++)
+                    for (int ww = 0; ww < kw; ww++) {
+                        const int64_t ts = t0 + u - rt, ys = y0 + v - rh, xs = x0 + ww - rw;
+                        if (ts < 0 || ts >= F || ys < 0 || ys >= Hp || xs < 0 || xs >= Wp) continue;
+                        const int64_t src = (ts * Hp + ys) * Wp + xs;
+                        const int64_t wi = ((int64_t)c * kt + u) * kh * kw + v * kw + ww;
+                        dx[src * C + c] += (double)w[wi] * g;
+                        dw[wi] += g * rd(x, io, src * C + c);
+                    }
+        }
+    }
+    return 0;
 }

@@ -1,7 +1,8 @@
 """The oracle's pins must catch plausible mistakes.
 
 Each case below plants one mistake in a copy of ``oracle/dsa3d_oracle.c`` (on the CPU only),
-builds it, and runs the pin suite against that copy; the suite must fail.  This checks that the
+builds it, and runs the pin suites (attention, and the layer's convolution and offset network)
+against that copy; the suites must fail.  This checks that the
 pins fix the oracle rather than merely agreeing with it.
 """
 import os
@@ -32,7 +33,19 @@ MUTANTS = {
     "per_tap_offsets_read_tap_0": ("* P->n_off + tau) * 3);", "* P->n_off + 0) * 3);"),
     "per_tap_gradient_not_per_tap": ("double *doff = doff_all + (P->n_off > 1 ? 3 * tau : 0);",
                                      "double *doff = doff_all;"),
+    "dwconv_convolution_not_correlation": (
+        "const int64_t ts = t0 + u - rt, ys = y0 + v - rh, xs = x0 + ww - rw;\n"
+        "                        if (ts < 0 || ts >= F || ys < 0 || ys >= Hp || xs < 0 || xs >= Wp) continue;\n"
+        "                        const int64_t src = (ts * Hp + ys) * Wp + xs;\n                        acc",
+        "const int64_t ts = t0 - u + rt, ys = y0 - v + rh, xs = x0 - ww + rw;\n"
+        "                        if (ts < 0 || ts >= F || ys < 0 || ys >= Hp || xs < 0 || xs >= Wp) continue;\n"
+        "                        const int64_t src = (ts * Hp + ys) * Wp + xs;\n                        acc"),
+    "dwconv_bias_dropped": ("double acc = b ? (double)b[c] : 0.0;", "double acc = 0.0;"),
+    "dwconv_dw_wrong_source": ("dw[wi] += g * rd(x, io, src * C + c);", "dw[wi] += g * rd(x, io, n * C + c);"),
+    "dwconv_dx_wrong_target": ("dx[src * C + c] += (double)w[wi] * g;", "dx[n * C + c] += (double)w[wi] * g;"),
+    "dwconv_db_dropped": ("            db[c] += g;\n", ""),
 }
+PIN_FILES = ["test_oracle_pins.py", "test_oracle_layer_pins.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -47,6 +60,6 @@ def test_pins_reject_planted_mistake(name, tmp_path):
                     "-o", str(lib), str(mut), "-lm"], check=True)
     env = dict(os.environ, DSA3D_ORACLE_LIB=str(lib), OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        *(os.path.join(ROOT, "tests", f) for f in PIN_FILES)],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins accepted the planted mistake {name}:\n{r.stdout[-2000:]}"
