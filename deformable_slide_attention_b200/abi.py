@@ -67,6 +67,11 @@ def _load():
         lib.dsa3d_backward_taps_workspace_bytes.argtypes = [*dims, I]
         lib.dsa3d_backward_taps.restype = I
         lib.dsa3d_backward_taps.argtypes = [P, P, P, P, P, P, P, P, P, P, P, Z, *dims, I, P]
+        cdims = [I] * 7  # F, Hp, Wp, C, kt, kh, kw
+        lib.dsa3d_dwconv3d.restype = I
+        lib.dsa3d_dwconv3d.argtypes = [P, P, P, P, P, *cdims, I, P]
+        lib.dsa3d_dwconv3d_backward.restype = I
+        lib.dsa3d_dwconv3d_backward.argtypes = [P, P, P, P, P, P, *cdims, I, P]
         lib.dsa3d_check_device.restype = I
         lib.dsa3d_check_device.argtypes = [P]
         lib.dsa3d_timing_enable.restype = I
@@ -141,6 +146,17 @@ def dsa3d_backward_taps(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, works
     return _load().dsa3d_backward_taps(q, k, v, offsets, lse, dout, dq, dk, dv, doffsets, workspace,
                                        workspace_bytes, F, Hp, Wp, heads, dh, kt, kh, kw, dtype,
                                        stream)
+
+
+def dsa3d_dwconv3d(x, weight, bias, add, y, F, Hp, Wp, C, kt, kh, kw, dtype, stream) -> int:
+    """The DWConv3D term of Eq. 1 (depthwise 3-D convolution, optional fused add)."""
+    return _load().dsa3d_dwconv3d(x, weight, bias, add, y, F, Hp, Wp, C, kt, kh, kw, dtype, stream)
+
+
+def dsa3d_dwconv3d_backward(x, weight, dy, dx, dweight, dbias, F, Hp, Wp, C, kt, kh, kw, dtype,
+                            stream) -> int:
+    return _load().dsa3d_dwconv3d_backward(x, weight, dy, dx, dweight, dbias, F, Hp, Wp, C, kt, kh,
+                                           kw, dtype, stream)
 
 
 def dsa3d_check_device(stream) -> int:
@@ -294,3 +310,34 @@ def backward_taps(q, k, v, offsets, lse, dout, dims, window, workspace=None, str
                                dv.data_ptr(), doff.data_ptr(), ws_ptr, ws_bytes, *dims, heads, dh,
                                *window, code, _stream_handle(stream)), "dsa3d_backward_taps")
     return dq, dk, dv, doff
+
+
+def dwconv3d(x, weight, bias, dims, add=None, out=None, stream=None):
+    """Depthwise 3-D convolution of x [N][C] with weight [C][kt][kh][kw] (fp32) and bias [C]
+    (fp32 or None), plus add [N][C] if given (the attention output viewed as [N][C]; out may be
+    add itself).  Returns out [N][C]."""
+    torch = _torch()
+    code = _dtype_code(x)
+    if out is None:
+        out = torch.empty_like(x)
+    C = x.shape[1]
+    kt, kh, kw = weight.shape[1:]
+    _check(dsa3d_dwconv3d(x.data_ptr(), weight.data_ptr(), bias.data_ptr() if bias is not None else None,
+                          add.data_ptr() if add is not None else None, out.data_ptr(), *dims, C, kt,
+                          kh, kw, code, _stream_handle(stream)), "dsa3d_dwconv3d")
+    return out
+
+
+def dwconv3d_backward(x, weight, dy, dims, stream=None):
+    """Gradients of sum(dwconv3d(x, weight, bias) * dy): (dx [N][C], dweight, dbias [C] fp32)."""
+    torch = _torch()
+    code = _dtype_code(x)
+    dx = torch.empty_like(x)
+    dw = torch.empty_like(weight, dtype=torch.float32)
+    db = torch.empty(x.shape[1], dtype=torch.float32, device=x.device)
+    C = x.shape[1]
+    kt, kh, kw = weight.shape[1:]
+    _check(dsa3d_dwconv3d_backward(x.data_ptr(), weight.data_ptr(), dy.data_ptr(), dx.data_ptr(),
+                                   dw.data_ptr(), db.data_ptr(), *dims, C, kt, kh, kw, code,
+                                   _stream_handle(stream)), "dsa3d_dwconv3d_backward")
+    return dx, dw, db

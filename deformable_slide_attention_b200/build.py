@@ -23,7 +23,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
 def sources():
-    return [os.path.join(CSRC, "dsa3d.cu")]
+    # the attention's translation unit, and the DWConv3D term's
+    return [os.path.join(CSRC, "dsa3d.cu"), os.path.join(CSRC, "dsa3d_conv.cu")]
 
 
 def _stale(out):

@@ -1,0 +1,208 @@
+// dsa3d_conv.cu -- C ABI of the DWConv3D term of Eq. 1 (MegaSlide-DiT, the 3D-DSA definition):
+// argument validation, launch configuration and the extern "C" entry points dsa3d_dwconv3d and
+// dsa3d_dwconv3d_backward declared in include/dsa3d.h.  The kernels are in dsa3d_conv.cuh.  A
+// translation unit of its own, next to dsa3d.cu; this file allocates no device memory.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "dsa3d.h"
+#include "dsa3d_conv.cuh"
+#include "dsa3d_timing.cuh"
+
+namespace dsa3d {
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+Range range_of(const void* p, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return {a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+size_t elem_size(dsa3d_dtype_t t) { return t == DSA3D_F32 ? 4 : 2; }
+
+struct DeviceInfo {
+  int sms = 0;
+};
+DeviceInfo device_info() {
+  DeviceInfo d;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  return d;
+}
+
+// Blocks of `threads` for `work` items, at most per_sm_cap per SM (the kernels stride the rest).
+int grid_for(int64_t work, int threads, int per_sm_cap) {
+  const DeviceInfo d = device_info();
+  int64_t grid = (work + threads - 1) / threads;
+  const int64_t cap = (int64_t)(d.sms > 0 ? d.sms : 1) * per_sm_cap;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  return (int)grid;
+}
+
+// --- depthwise 3-D convolution (the DWConv3D term of Eq. 1) -----------------------------------------
+ConvGeo make_conv_geo(int F, int Hp, int Wp, int C, int kt, int kh, int kw) {
+  ConvGeo g;
+  g.F = F; g.Hp = Hp; g.Wp = Wp; g.C = C; g.kt = kt; g.kh = kh; g.kw = kw;
+  g.N = (int64_t)F * Hp * Wp;
+  return g;
+}
+
+dsa3d_status_t check_conv_shape(int F, int Hp, int Wp, int C, int kt, int kh, int kw,
+                                dsa3d_dtype_t dtype) {
+  if (dtype != DSA3D_F32 && dtype != DSA3D_BF16) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (F < 1 || Hp < 1 || Wp < 1 || C < 2) return DSA3D_ERR_INVALID_ARGUMENT;
+  const int dims[3] = {F, Hp, Wp}, win[3] = {kt, kh, kw};
+  for (int a = 0; a < 3; a++) {
+    if (win[a] < 1 || (win[a] & 1) == 0) return DSA3D_ERR_INVALID_ARGUMENT;
+    if ((int64_t)win[a] > 2 * (int64_t)dims[a] - 1) return DSA3D_ERR_UNSUPPORTED;
+  }
+  if (kw > 15 || (C & 1)) return DSA3D_ERR_UNSUPPORTED;  // kernel rows are unrolled; channel pairs
+  if ((int64_t)F * Hp * Wp >= (int64_t(1) << 31)) return DSA3D_ERR_UNSUPPORTED;
+  return DSA3D_OK;
+}
+
+template <typename T, int KW>
+dsa3d_status_t dwconv_launch_kw(const ConvGeo& g, const void* x, const float* w, const float* b,
+                                const void* add, void* y, int flip, cudaStream_t st) {
+  const int64_t items = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip) * (g.C / 2);
+  TimedLaunch tl(kKernDwconv, st);
+  dsa3d_dwconv3d_kernel<T, KW><<<grid_for(items, 256, 8), 256, 0, st>>>(
+      static_cast<const T*>(x), w, b, static_cast<const T*>(add), static_cast<T*>(y), g, flip);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+template <typename T>
+dsa3d_status_t dwconv_launch(const ConvGeo& g, const void* x, const float* w, const float* b,
+                             const void* add, void* y, int flip, cudaStream_t st) {
+  switch (g.kw) {
+    case 1: return dwconv_launch_kw<T, 1>(g, x, w, b, add, y, flip, st);
+    case 3: return dwconv_launch_kw<T, 3>(g, x, w, b, add, y, flip, st);
+    case 5: return dwconv_launch_kw<T, 5>(g, x, w, b, add, y, flip, st);
+    case 7: return dwconv_launch_kw<T, 7>(g, x, w, b, add, y, flip, st);
+    case 9: return dwconv_launch_kw<T, 9>(g, x, w, b, add, y, flip, st);
+    case 11: return dwconv_launch_kw<T, 11>(g, x, w, b, add, y, flip, st);
+    case 13: return dwconv_launch_kw<T, 13>(g, x, w, b, add, y, flip, st);
+    case 15: return dwconv_launch_kw<T, 15>(g, x, w, b, add, y, flip, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+// Strips per dW work item: enough items to fill the GPU (about 8 per SM-slot), each long enough
+// that its final atomics are a small share of its work.
+int dw_strips_per_item(const ConvGeo& g) {
+  const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
+  const int64_t lanes = (int64_t)(g.C / 2) * g.kt * g.kh;
+  const int64_t want_items = (int64_t)device_info().sms * 2048;
+  int64_t chunks = want_items / (lanes > 0 ? lanes : 1);
+  if (chunks < 1) chunks = 1;
+  int64_t spi = (strips + chunks - 1) / chunks;
+  if (spi < 1) spi = 1;
+  if (spi > (1 << 20)) spi = 1 << 20;
+  return (int)spi;
+}
+
+template <typename T, int KW>
+dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* dy, float* dw,
+                                   float* db, cudaStream_t st) {
+  const int spi = dw_strips_per_item(g);
+  const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
+  const int64_t items = (strips + spi - 1) / spi * g.kt * g.kh * (g.C / 2);
+  TimedLaunch tl(kKernDwconvDw, st);
+  dsa3d_dwconv3d_dw_kernel<T, KW><<<grid_for(items, 256, 8), 256, 0, st>>>(
+      static_cast<const T*>(x), static_cast<const T*>(dy), dw, db, g, spi);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+template <typename T>
+dsa3d_status_t dwconv_dw_launch(const ConvGeo& g, const void* x, const void* dy, float* dw,
+                                float* db, cudaStream_t st) {
+  switch (g.kw) {
+    case 1: return dwconv_dw_launch_kw<T, 1>(g, x, dy, dw, db, st);
+    case 3: return dwconv_dw_launch_kw<T, 3>(g, x, dy, dw, db, st);
+    case 5: return dwconv_dw_launch_kw<T, 5>(g, x, dy, dw, db, st);
+    case 7: return dwconv_dw_launch_kw<T, 7>(g, x, dy, dw, db, st);
+    case 9: return dwconv_dw_launch_kw<T, 9>(g, x, dy, dw, db, st);
+    case 11: return dwconv_dw_launch_kw<T, 11>(g, x, dy, dw, db, st);
+    case 13: return dwconv_dw_launch_kw<T, 13>(g, x, dy, dw, db, st);
+    case 15: return dwconv_dw_launch_kw<T, 15>(g, x, dy, dw, db, st);
+    default: return DSA3D_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace
+}  // namespace dsa3d
+
+using namespace dsa3d;
+
+extern "C" {
+
+dsa3d_status_t dsa3d_dwconv3d(const void* x, const float* weight, const float* bias,
+                              const void* add, void* y, int F, int Hp, int Wp, int C, int kt, int kh,
+                              int kw, dsa3d_dtype_t dtype, cudaStream_t stream) {
+  dsa3d_status_t rc = check_conv_shape(F, Hp, Wp, C, kt, kh, kw, dtype);
+  if (rc != DSA3D_OK) return rc;
+  if (!x || !weight || !y) return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al[] = {x, y};
+  for (const void* p : al)
+    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if ((add && !aligned16(add)) || (reinterpret_cast<uintptr_t>(weight) & 3u) ||
+      (bias && (reinterpret_cast<uintptr_t>(bias) & 7u)))
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  const ConvGeo g = make_conv_geo(F, Hp, Wp, C, kt, kh, kw);
+  const size_t tb = (size_t)g.N * C * elem_size(dtype);
+  const Range ry = range_of(y, tb);
+  // y is written while neighbouring rows of x are still read; add may be y itself
+  if (overlap(range_of(x, tb), ry) || overlap(range_of(weight, (size_t)C * kt * kh * kw * 4), ry) ||
+      (bias && overlap(range_of(bias, (size_t)C * 4), ry)))
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  if (add && add != y && overlap(range_of(add, tb), ry)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (dtype == DSA3D_F32) return dwconv_launch<float>(g, x, weight, bias, add, y, 0, stream);
+  return dwconv_launch<__nv_bfloat16>(g, x, weight, bias, add, y, 0, stream);
+}
+
+dsa3d_status_t dsa3d_dwconv3d_backward(const void* x, const float* weight, const void* dy, void* dx,
+                                       float* dweight, float* dbias, int F, int Hp, int Wp, int C,
+                                       int kt, int kh, int kw, dsa3d_dtype_t dtype,
+                                       cudaStream_t stream) {
+  dsa3d_status_t rc = check_conv_shape(F, Hp, Wp, C, kt, kh, kw, dtype);
+  if (rc != DSA3D_OK) return rc;
+  if (!x || !weight || !dy || !dx || !dweight || !dbias) return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al[] = {x, dy, dx};
+  for (const void* p : al)
+    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(weight) & 3u) || (reinterpret_cast<uintptr_t>(dweight) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dbias) & 7u))
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  const ConvGeo g = make_conv_geo(F, Hp, Wp, C, kt, kh, kw);
+  const size_t tb = (size_t)g.N * C * elem_size(dtype), wb = (size_t)C * kt * kh * kw * 4;
+  const Range ins[] = {range_of(x, tb), range_of(weight, wb), range_of(dy, tb)};
+  const Range outs[] = {range_of(dx, tb), range_of(dweight, wb), range_of(dbias, (size_t)C * 4)};
+  for (int i = 0; i < 3; i++) {
+    for (const Range& r : ins)
+      if (overlap(r, outs[i])) return DSA3D_ERR_INVALID_ARGUMENT;
+    for (int j = i + 1; j < 3; j++)
+      if (overlap(outs[i], outs[j])) return DSA3D_ERR_INVALID_ARGUMENT;
+  }
+  if (cudaMemsetAsync(dweight, 0, wb, stream) != cudaSuccess ||
+      cudaMemsetAsync(dbias, 0, (size_t)C * 4, stream) != cudaSuccess)
+    return DSA3D_ERR_CUDA;
+  if (dtype == DSA3D_F32) {
+    if ((rc = dwconv_launch<float>(g, dy, weight, nullptr, nullptr, dx, 1, stream)) != DSA3D_OK) return rc;
+    return dwconv_dw_launch<float>(g, x, dy, dweight, dbias, stream);
+  }
+  if ((rc = dwconv_launch<__nv_bfloat16>(g, dy, weight, nullptr, nullptr, dx, 1, stream)) != DSA3D_OK)
+    return rc;
+  return dwconv_dw_launch<__nv_bfloat16>(g, x, dy, dweight, dbias, stream);
+}
+
+}  // extern "C"

@@ -26,6 +26,8 @@ enum KernelId {
   kKernPairV,
   kKernFwdTaps,
   kKernBwdTaps,
+  kKernDwconv,
+  kKernDwconvDw,
   kKernCount
 };
 inline const char* kernel_name(int id) {
@@ -34,7 +36,8 @@ inline const char* kernel_name(int id) {
       "dsa3d_zero_kernel",     "dsa3d_fwd_mma_kernel",    "dsa3d_sort_count_kernel",
       "dsa3d_scan_kernels",    "dsa3d_sort_fill_kernel",  "dsa3d_bwd_q_kernel",
       "dsa3d_bwd_dq_kernel",   "dsa3d_bwd_kv_kernel",     "dsa3d_pair_v_kernel",
-      "dsa3d_fwd_taps_kernel", "dsa3d_bwd_taps_kernel"};
+      "dsa3d_fwd_taps_kernel", "dsa3d_bwd_taps_kernel", "dsa3d_dwconv3d_kernel",
+      "dsa3d_dwconv3d_dw_kernel"};
   return names[id];
 }
 

@@ -191,6 +191,33 @@ dsa3d_status_t dsa3d_backward_taps(const void *q, const void *k, const void *v,
                                    cudaStream_t stream);
 
 /*
+ * The DWConv3D term of Eq. 1 (MegaSlide-DiT, the 3D-DSA definition): a depthwise 3-D convolution
+ * of the layer input X, added to the attention output.
+ *   x    [N][C] I/O type (C = heads * dh in the layer; any even C >= 2 here);
+ *   weight [C][kt][kh][kw] fp32, bias [C] fp32 (may be NULL);
+ *   add  [N][C] I/O type or NULL: added element by element (the attention output
+ *        [N][heads][dh] viewed as [N][C]); may equal y (in place);
+ *   y    [N][C] I/O type (written):
+ *        y[(t,y,x)][c] = bias[c] + sum_{u,v,w} weight[c][u][v][w] * x[(t+u-r_t, y+v-r_h, x+w-r_w)][c]
+ *                        (+ add), with x = 0 outside the volume (zero padding, same grid).
+ * Cross-correlation (PyTorch's conv3d with groups = C and padding k // 2).  Kernel extents are
+ * odd, at most 2 * dim - 1, and kw <= 15.  y must not overlap x, weight or bias.
+ */
+dsa3d_status_t dsa3d_dwconv3d(const void *x, const float *weight, const float *bias,
+                              const void *add, void *y, int F, int Hp, int Wp, int C, int kt,
+                              int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * Backward of dsa3d_dwconv3d for the upstream gradient dy [N][C]: dx [N][C] I/O type (the
+ * convolution of dy with the flipped kernel), dweight [C][kt][kh][kw] and dbias [C] fp32 (both
+ * overwritten; summed over all tokens in fp32).  Outputs must not overlap the inputs or each other.
+ */
+dsa3d_status_t dsa3d_dwconv3d_backward(const void *x, const float *weight, const void *dy,
+                                       void *dx, float *dweight, float *dbias, int F, int Hp,
+                                       int Wp, int C, int kt, int kh, int kw, dsa3d_dtype_t dtype,
+                                       cudaStream_t stream);
+
+/*
  * Synchronises `stream` and reports DSA3D_ERR_DEVICE_CHECK if any kernel of this library on the
  * current device recorded a failed internal check since the last call (the record is then
  * cleared), DSA3D_ERR_CUDA if the stream reports an error, else DSA3D_OK.

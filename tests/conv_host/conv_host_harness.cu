@@ -1,0 +1,120 @@
+// conv_host_harness.cu -- runs the depthwise-convolution kernels' per-thread routines
+// (conv_strip, dw_row from the library's dsa3d_conv.cuh) on the CPU, over every work item the
+// GPU kernels would process, so that their indexing and arithmetic can be compared with the
+// oracle without a GPU.  Test infrastructure: built by tests/test_conv_host.py with nvcc as
+// host code; nothing here launches a kernel.
+#include <stdint.h>
+
+#include "dsa3d_conv.cuh"
+
+using namespace dsa3d;
+
+namespace {
+
+template <typename T, int KW>
+void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, int flip, float* y) {
+  const int pairs = g.C / 2, nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
+  for (int t = 0; t < g.F; t++)
+    for (int yy = 0; yy < g.Hp; yy++)
+      for (int sx = 0; sx < nxs; sx++)
+        for (int c2 = 0; c2 < pairs; c2++) {
+          float acc[kConvStrip][2];
+          for (int i = 0; i < kConvStrip; i++) {
+            acc[i][0] = b ? b[2 * c2] : 0.f;
+            acc[i][1] = b ? b[2 * c2 + 1] : 0.f;
+          }
+          const int x0 = sx * kConvStrip;
+          conv_strip<T, KW>(x, w, g, t, yy, x0, c2, flip != 0, acc);
+          for (int i = 0; i < kConvStrip && x0 + i < g.Wp; i++) {
+            const int64_t o = (((int64_t)t * g.Hp + yy) * g.Wp + x0 + i) * g.C + 2 * c2;
+            y[o] = acc[i][0];
+            y[o + 1] = acc[i][1];
+          }
+        }
+}
+
+template <typename T, int KW>
+void dw_all(const T* x, const T* dy, const ConvGeo& g, int strips_per_item, float* dw, float* db) {
+  const int pairs = g.C / 2, rows = g.kt * g.kh, nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
+  const int64_t strips = (int64_t)g.F * g.Hp * nxs, K = (int64_t)rows * KW;
+  const int64_t chunks = (strips + strips_per_item - 1) / strips_per_item;
+  for (int64_t chunk = 0; chunk < chunks; chunk++)
+    for (int r = 0; r < rows; r++)
+      for (int c2 = 0; c2 < pairs; c2++) {
+        float dwr[KW][2] = {};
+        float dbl[2] = {0.f, 0.f};
+        const int64_t s_end = (chunk + 1) * strips_per_item < strips ? (chunk + 1) * strips_per_item : strips;
+        for (int64_t s = chunk * strips_per_item; s < s_end; s++) {
+          const int x0 = (int)(s % nxs) * kConvStrip;
+          const int yy = (int)((s / nxs) % g.Hp);
+          const int t = (int)(s / ((int64_t)nxs * g.Hp));
+          dw_row<T, KW>(x, dy, g, t, yy, x0, c2, r / g.kh, r % g.kh, dwr, r == 0 ? dbl : nullptr);
+        }
+        for (int j = 0; j < KW; j++) {
+          dw[(int64_t)(2 * c2) * K + (int64_t)r * KW + j] += dwr[j][0];
+          dw[(int64_t)(2 * c2 + 1) * K + (int64_t)r * KW + j] += dwr[j][1];
+        }
+        if (r == 0) {
+          db[2 * c2] += dbl[0];
+          db[2 * c2 + 1] += dbl[1];
+        }
+      }
+}
+
+template <template <typename, int> class Fn, typename T, typename... A>
+int by_kw(int kw, A... a) {
+  switch (kw) {
+    case 1: Fn<T, 1>::run(a...); return 0;
+    case 3: Fn<T, 3>::run(a...); return 0;
+    case 5: Fn<T, 5>::run(a...); return 0;
+    case 7: Fn<T, 7>::run(a...); return 0;
+    case 9: Fn<T, 9>::run(a...); return 0;
+    case 11: Fn<T, 11>::run(a...); return 0;
+    case 13: Fn<T, 13>::run(a...); return 0;
+    case 15: Fn<T, 15>::run(a...); return 0;
+    default: return -1;
+  }
+}
+template <typename T, int KW>
+struct Fwd {
+  static void run(const void* x, const float* w, const float* b, ConvGeo g, int flip, float* y) {
+    forward_all<T, KW>(static_cast<const T*>(x), w, b, g, flip, y);
+  }
+};
+template <typename T, int KW>
+struct Dw {
+  static void run(const void* x, const void* dy, ConvGeo g, int spi, float* dw, float* db) {
+    dw_all<T, KW>(static_cast<const T*>(x), static_cast<const T*>(dy), g, spi, dw, db);
+  }
+};
+
+ConvGeo geo(int F, int Hp, int Wp, int C, int kt, int kh, int kw) {
+  ConvGeo g;
+  g.F = F; g.Hp = Hp; g.Wp = Wp; g.C = C; g.kt = kt; g.kh = kh; g.kw = kw;
+  g.N = (int64_t)F * Hp * Wp;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+// io: 0 = fp32, 1 = bf16.  y [N][C] fp32 (every element written).
+int conv_host_forward(int io, const void* x, const float* w, const float* b, int F, int Hp, int Wp,
+                      int C, int kt, int kh, int kw, int flip, float* y) {
+  if (C % 2) return -1;
+  const ConvGeo g = geo(F, Hp, Wp, C, kt, kh, kw);
+  return io ? by_kw<Fwd, __nv_bfloat16>(kw, x, w, b, g, flip, y)
+            : by_kw<Fwd, float>(kw, x, w, b, g, flip, y);
+}
+
+// dw [C][kt][kh][kw], db [C]: fp32, accumulated into (zero them first).
+int conv_host_dw(int io, const void* x, const void* dy, int F, int Hp, int Wp, int C, int kt, int kh,
+                 int kw, int strips_per_item, float* dw, float* db) {
+  if (C % 2 || strips_per_item < 1) return -1;
+  const ConvGeo g = geo(F, Hp, Wp, C, kt, kh, kw);
+  return io ? by_kw<Dw, __nv_bfloat16>(kw, x, dy, g, strips_per_item, dw, db)
+            : by_kw<Dw, float>(kw, x, dy, g, strips_per_item, dw, db);
+}
+
+}  // extern "C"

@@ -1,0 +1,119 @@
+"""The depthwise-convolution kernels' per-thread routines (conv_strip, dw_row in
+csrc/dsa3d_conv.cuh), run on the CPU by a host harness over every work item the GPU kernels
+process, against the oracle's convolution (reading R9).  This checks their indexing, boundary
+handling, kernel flip and weight-gradient accumulation without a GPU; the GPU parity tests call
+the same code through the C ABI.
+
+Tolerances: the routines accumulate in fp32 (the oracle in fp64): max-abs 1e-4 relative to the
+output scale for the forward and dX, 1e-4 relative for dW and db (sums over all tokens).
+"""
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+SRC = os.path.join(HERE, "conv_host", "conv_host_harness.cu")
+CSRC = os.path.join(ROOT, "deformable_slide_attention_b200", "csrc")
+LIB = os.path.join(HERE, "conv_host", "_build", "libconvhost.so")
+
+
+@pytest.fixture(scope="module")
+def harness():
+    deps = [SRC, os.path.join(CSRC, "dsa3d_conv.cuh")]
+    if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(d) for d in deps):
+        os.makedirs(os.path.dirname(LIB), exist_ok=True)
+        subprocess.run(["/usr/local/cuda/bin/nvcc", "-O2", "-std=c++17", "-x", "cu",
+                        "-gencode", "arch=compute_100a,code=sm_100a", "-Xcompiler", "-fPIC",
+                        "-shared", "-I", CSRC, "-o", LIB + ".tmp", SRC], check=True)
+        os.replace(LIB + ".tmp", LIB)
+    lib = ctypes.CDLL(LIB)
+    I, P = ctypes.c_int, ctypes.c_void_p
+    lib.conv_host_forward.argtypes = [I, P, P, P] + [I] * 7 + [I, P]
+    lib.conv_host_dw.argtypes = [I, P, P] + [I] * 7 + [I, P, P]
+    return lib
+
+
+def _io(x):
+    x = x.contiguous()
+    if x.dtype == torch.bfloat16:
+        return 1, x.view(torch.int16).numpy()
+    return 0, x.numpy()
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def host_forward(lib, x, w, b, dims, flip=False):
+    io, xa = _io(x)
+    C = x.shape[1]
+    wa = w.float().contiguous().numpy()
+    ba = None if b is None else b.float().contiguous().numpy()
+    y = np.zeros((x.shape[0], C), np.float32)
+    rc = lib.conv_host_forward(io, _ptr(xa), _ptr(wa), _ptr(ba), *dims, C, *w.shape[1:], int(flip),
+                               _ptr(y))
+    assert rc == 0
+    return y
+
+
+def host_dw(lib, x, dy, dims, window, strips_per_item):
+    io, xa = _io(x)
+    _, da = _io(dy)
+    C = x.shape[1]
+    dw = np.zeros((C, *window), np.float32)
+    db = np.zeros(C, np.float32)
+    rc = lib.conv_host_dw(io, _ptr(xa), _ptr(da), *dims, C, *window, strips_per_item, _ptr(dw), _ptr(db))
+    assert rc == 0
+    return dw, db
+
+
+CASES = [((3, 5, 6), 4, (3, 3, 3)), ((2, 7, 19), 6, (3, 5, 9)), ((4, 3, 11), 2, (1, 1, 15)),
+         ((1, 4, 9), 8, (1, 3, 1)), ((5, 2, 17), 4, (5, 3, 7)), ((2, 3, 8), 2, (3, 3, 13))]
+
+
+@pytest.mark.parametrize("dims,C,window", CASES)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_forward_and_dx_match_oracle(harness, dims, C, window, dtype):
+    g = torch.Generator().manual_seed(sum(dims) + C)
+    N = math.prod(dims)
+    x = torch.randn(N, C, generator=g).to(dtype)
+    w = torch.randn(C, *window, generator=g)
+    b = torch.randn(C, generator=g)
+    y = host_forward(harness, x, w, b, dims)
+    ref = oracle.dwconv3d(x, w, b, dims)
+    assert np.abs(y - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())
+    # dX = the forward on dY with the kernel flipped (no bias)
+    dy = torch.randn(N, C, generator=g).to(dtype)
+    dx = host_forward(harness, dy, w, None, dims, flip=True)
+    ref_dx, _, _ = oracle.dwconv3d_backward(x, w, dy.double().numpy(), dims)
+    assert np.abs(dx - ref_dx).max() <= 1e-4 * max(1.0, np.abs(ref_dx).max())
+
+
+@pytest.mark.parametrize("dims,C,window", CASES)
+@pytest.mark.parametrize("strips_per_item", [1, 3, 64])
+def test_weight_gradient_matches_oracle(harness, dims, C, window, strips_per_item):
+    g = torch.Generator().manual_seed(7 + sum(window))
+    N = math.prod(dims)
+    x = torch.randn(N, C, generator=g).to(torch.bfloat16)
+    dy = torch.randn(N, C, generator=g).to(torch.bfloat16)
+    w = torch.randn(C, *window, generator=g)
+    dw, db = host_dw(harness, x, dy, dims, window, strips_per_item)
+    _, ref_dw, ref_db = oracle.dwconv3d_backward(x, w, dy.double().numpy(), dims)
+    assert np.abs(dw - ref_dw).max() <= 1e-4 * max(1.0, np.abs(ref_dw).max())
+    assert np.abs(db - ref_db).max() <= 1e-4 * max(1.0, np.abs(ref_db).max())
+
+
+def test_unsupported_width_is_refused(harness):
+    x = torch.zeros(6, 2)
+    y = np.zeros((6, 2), np.float32)
+    w = np.zeros((2, 1, 1, 17), np.float32)
+    io, xa = _io(x)
+    assert harness.conv_host_forward(io, _ptr(xa), _ptr(w), None, 1, 1, 6, 2, 1, 1, 17, 0, _ptr(y)) == -1

@@ -1,0 +1,77 @@
+"""GPU parity of the DWConv3D term of Eq. 1 (dsa3d_dwconv3d / dsa3d_dwconv3d_backward) against
+the oracle's depthwise convolution (reading R9), through the C ABI.
+
+Weights are scaled by 1/sqrt(kt kh kw) so outputs are O(1); tolerances max-abs 1e-5 (fp32) and
+2e-2 (bf16 I/O, fp32 accumulation); dweight and dbias (fp32 sums over every token) relative 1e-4.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from deformable_slide_attention_b200 import abi
+from tests.gpu_helpers import TOL, assert_close, f64
+
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gpu_lib", "oracle_lib")]
+
+CASES = [((3, 5, 6), 4, (3, 3, 3)), ((2, 7, 19), 6, (3, 5, 9)), ((4, 3, 11), 2, (1, 1, 15)),
+         ((1, 4, 9), 8, (1, 3, 1)), ((5, 2, 17), 4, (5, 3, 7)), ((4, 9, 16), 64, (3, 9, 9))]
+
+
+def _problem(dims, C, window, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    N, K = math.prod(dims), math.prod(window)
+    x = torch.randn(N, C, generator=g).to(dtype)
+    w = torch.randn(C, *window, generator=g) / math.sqrt(K)
+    b = torch.randn(C, generator=g)
+    add = torch.randn(N, C, generator=g).to(dtype)
+    dy = torch.randn(N, C, generator=g).to(dtype)
+    return x, w, b, add, dy
+
+
+@pytest.mark.parametrize("dims,C,window", CASES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_forward_with_and_without_add(dims, C, window, dtype):
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    x, w, b, add, _ = _problem(dims, C, window, td, sum(dims) + C)
+    dx, dw_, db_, dadd = (t.cuda() for t in (x, w, b, add))
+    y = abi.dwconv3d(dx, dw_, db_, dims)
+    y_add = abi.dwconv3d(dx, dw_, db_, dims, add=dadd)
+    inplace = dadd.clone()
+    abi.dwconv3d(dx, dw_, db_, dims, add=inplace, out=inplace)  # y = conv + add, in place
+    torch.cuda.synchronize()
+    ref = oracle.dwconv3d(x, w, b, dims)
+    assert_close("y", f64(y), ref, TOL[dtype])
+    assert_close("y+add", f64(y_add), ref + f64(add), TOL[dtype])
+    assert torch.equal(inplace, y_add)
+
+
+@pytest.mark.parametrize("dims,C,window", CASES)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward(dims, C, window, dtype):
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    x, w, _, _, dy = _problem(dims, C, window, td, 3 * sum(dims) + C)
+    gx, gw, gb = abi.dwconv3d_backward(x.cuda(), w.cuda(), dy.cuda(), dims)
+    torch.cuda.synchronize()
+    rx, rw, rb = oracle.dwconv3d_backward(x, w, dy.double().numpy(), dims)
+    assert_close("dx", f64(gx), rx, TOL[dtype])
+    for name, got, ref in (("dweight", gw, rw), ("dbias", gb, rb)):
+        err = np.abs(f64(got) - ref).max()
+        assert err <= 1e-4 * max(1.0, np.abs(ref).max()), (name, err)
+
+
+def test_rejects_unsupported_and_overlapping():
+    x = torch.zeros(24, 4, device="cuda", dtype=torch.bfloat16)
+    w = torch.zeros(4, 1, 1, 17, device="cuda")
+    y = torch.empty_like(x)
+    st = torch.cuda.current_stream().cuda_stream
+    assert abi.dsa3d_dwconv3d(x.data_ptr(), w.data_ptr(), None, None, y.data_ptr(), 1, 1, 24, 4, 1, 1,
+                              17, abi.DSA3D_BF16, st) == 2  # kw > 15
+    w3 = torch.zeros(4, 1, 1, 3, device="cuda")
+    assert abi.dsa3d_dwconv3d(x.data_ptr(), w3.data_ptr(), None, None, x.data_ptr(), 1, 1, 24, 4, 1, 1,
+                              3, abi.DSA3D_BF16, st) == 1  # y on top of x
+    x3 = torch.zeros(24, 3, device="cuda", dtype=torch.bfloat16)
+    assert abi.dsa3d_dwconv3d(x3.data_ptr(), w3.data_ptr(), None, None, y.data_ptr(), 1, 1, 24, 3, 1, 1,
+                              3, abi.DSA3D_BF16, st) == 2  # odd channel count
