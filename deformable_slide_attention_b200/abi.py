@@ -204,6 +204,34 @@ def _check(status, what):
         raise Dsa3dError(status, what)
 
 
+def _need(t, name, shape, dtype):
+    """t must be a contiguous tensor of exactly this shape and dtype: the C ABI takes plain
+    pointers and reads sizes from the extents, so a mismatched tensor would be read past its end."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _on_device(ref, *ts):
+    """Every tensor given must be a CUDA tensor on ref's device."""
+    for t in (ref, *ts):
+        if t is not None and (not t.is_cuda or t.device != ref.device):
+            raise ValueError("tensors must be CUDA tensors on one device")
+
+
+def _workspace(ws):
+    if ws is not None:
+        torch = _torch()
+        if ws.dtype != torch.uint8 or not ws.is_contiguous() or ws.dim() != 1:
+            raise ValueError("workspace must be a contiguous 1-D uint8 tensor")
+    return ws
+
+
 def _shapes(q, offsets, dims, taps=None):
     """N, heads, dh; offsets must be [heads][N][3], or [heads][N][taps][3] when taps is given."""
     F, Hp, Wp = dims
@@ -227,17 +255,21 @@ def forward(q, k, v, offsets, dims, window, out=None, lse=None, stream=None, wan
     """
     torch = _torch()
     N, heads, dh = _shapes(q, offsets, dims)
-    for t in (q, k, v, offsets):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("inputs must be contiguous CUDA tensors")
     code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.shape, q.dtype)
+    _need(offsets, "offsets", offsets.shape, torch.float32)
     if out is None:
         out = torch.empty_like(q)
+    _need(out, "out", q.shape, q.dtype)
     if lse is None and want_lse:
         lse = torch.empty((heads, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", (heads, N), torch.float32)
     if isinstance(workspace, str):
         need = dsa3d_forward_workspace_bytes(*dims, heads, dh, *window, code)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device) if need else None
+    _on_device(q, k, v, offsets, out, lse, _workspace(workspace))
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(dsa3d_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(), out.data_ptr(),
@@ -251,13 +283,18 @@ def backward(q, k, v, offsets, lse, dout, dims, window, workspace=None, stream=N
     torch = _torch()
     N, heads, dh = _shapes(q, offsets, dims)
     code = _dtype_code(q)
+    _check_backward_tensors(q, k, v, offsets, lse, dout, heads, N)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
                  torch.empty_like(offsets))
     dq, dk, dv, doff = grads
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, name, q.shape, q.dtype)
+    _need(doff, "doffsets", offsets.shape, torch.float32)
     need = dsa3d_backward_workspace_bytes(*dims, heads, dh, *window, code)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _on_device(q, k, v, offsets, lse, dout, dq, dk, dv, doff, _workspace(workspace))
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(dsa3d_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(),
@@ -265,6 +302,14 @@ def backward(q, k, v, offsets, lse, dout, dims, window, workspace=None, stream=N
                           doff.data_ptr(), ws_ptr, ws_bytes, *dims, heads, dh, *window, code,
                           _stream_handle(stream)), "dsa3d_backward")
     return dq, dk, dv, doff
+
+
+def _check_backward_tensors(q, k, v, offsets, lse, dout, heads, N):
+    torch = _torch()
+    for name, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _need(t, name, q.shape, q.dtype)
+    _need(offsets, "offsets", offsets.shape, torch.float32)
+    _need(lse, "lse", (heads, N), torch.float32)
 
 
 def _taps(window):
@@ -277,14 +322,18 @@ def forward_taps(q, k, v, offsets, dims, window, out=None, lse=None, stream=None
     Returns (out [N][heads][dh], lse [heads][N] or None)."""
     torch = _torch()
     N, heads, dh = _shapes(q, offsets, dims, _taps(window))
-    for t in (q, k, v, offsets):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("inputs must be contiguous CUDA tensors")
     code = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.shape, q.dtype)
+    _need(offsets, "offsets", offsets.shape, torch.float32)
     if out is None:
         out = torch.empty_like(q)
+    _need(out, "out", q.shape, q.dtype)
     if lse is None and want_lse:
         lse = torch.empty((heads, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", (heads, N), torch.float32)
+    _on_device(q, k, v, offsets, out, lse)
     _check(dsa3d_forward_taps(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(),
                               out.data_ptr(), lse.data_ptr() if lse is not None else None, *dims,
                               heads, dh, *window, code, _stream_handle(stream)), "dsa3d_forward_taps")
@@ -296,13 +345,18 @@ def backward_taps(q, k, v, offsets, lse, dout, dims, window, workspace=None, str
     torch = _torch()
     N, heads, dh = _shapes(q, offsets, dims, _taps(window))
     code = _dtype_code(q)
+    _check_backward_tensors(q, k, v, offsets, lse, dout, heads, N)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
                  torch.empty_like(offsets))
     dq, dk, dv, doff = grads
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, name, q.shape, q.dtype)
+    _need(doff, "doffsets", offsets.shape, torch.float32)
     need = dsa3d_backward_taps_workspace_bytes(*dims, heads, dh, *window, code)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _on_device(q, k, v, offsets, lse, dout, dq, dk, dv, doff, _workspace(workspace))
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(dsa3d_backward_taps(q.data_ptr(), k.data_ptr(), v.data_ptr(), offsets.data_ptr(),
@@ -312,16 +366,36 @@ def backward_taps(q, k, v, offsets, lse, dout, dims, window, workspace=None, str
     return dq, dk, dv, doff
 
 
+def _conv_shapes(x, weight, dims):
+    """(C, kt, kh, kw) of a convolution call; x must be [N][C] with N = F*Hp*Wp and weight
+    [C][kt][kh][kw] fp32, both contiguous."""
+    torch = _torch()
+    N = dims[0] * dims[1] * dims[2]
+    if x.dim() != 2 or x.shape[0] != N:
+        raise ValueError(f"x must be [N={N}][C], got {tuple(x.shape)}")
+    _need(x, "x", x.shape, x.dtype)
+    C = x.shape[1]
+    if weight.dim() != 4 or weight.shape[0] != C:
+        raise ValueError(f"weight must be [C={C}][kt][kh][kw], got {tuple(weight.shape)}")
+    _need(weight, "weight", weight.shape, torch.float32)
+    return (C, *weight.shape[1:])
+
+
 def dwconv3d(x, weight, bias, dims, add=None, out=None, stream=None):
     """Depthwise 3-D convolution of x [N][C] with weight [C][kt][kh][kw] (fp32) and bias [C]
     (fp32 or None), plus add [N][C] if given (the attention output viewed as [N][C]; out may be
     add itself).  Returns out [N][C]."""
     torch = _torch()
     code = _dtype_code(x)
+    C, kt, kh, kw = _conv_shapes(x, weight, dims)
+    if bias is not None:
+        _need(bias, "bias", (C,), torch.float32)
+    if add is not None:
+        _need(add, "add", x.shape, x.dtype)
     if out is None:
         out = torch.empty_like(x)
-    C = x.shape[1]
-    kt, kh, kw = weight.shape[1:]
+    _need(out, "out", x.shape, x.dtype)
+    _on_device(x, weight, bias, add, out)
     _check(dsa3d_dwconv3d(x.data_ptr(), weight.data_ptr(), bias.data_ptr() if bias is not None else None,
                           add.data_ptr() if add is not None else None, out.data_ptr(), *dims, C, kt,
                           kh, kw, code, _stream_handle(stream)), "dsa3d_dwconv3d")
@@ -332,11 +406,12 @@ def dwconv3d_backward(x, weight, dy, dims, stream=None):
     """Gradients of sum(dwconv3d(x, weight, bias) * dy): (dx [N][C], dweight, dbias [C] fp32)."""
     torch = _torch()
     code = _dtype_code(x)
+    C, kt, kh, kw = _conv_shapes(x, weight, dims)
+    _need(dy, "dy", x.shape, x.dtype)
+    _on_device(x, weight, dy)
     dx = torch.empty_like(x)
     dw = torch.empty_like(weight, dtype=torch.float32)
     db = torch.empty(x.shape[1], dtype=torch.float32, device=x.device)
-    C = x.shape[1]
-    kt, kh, kw = weight.shape[1:]
     _check(dsa3d_dwconv3d_backward(x.data_ptr(), weight.data_ptr(), dy.data_ptr(), dx.data_ptr(),
                                    dw.data_ptr(), db.data_ptr(), *dims, C, kt, kh, kw, code,
                                    _stream_handle(stream)), "dsa3d_dwconv3d_backward")
