@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
     DSA3D_OK = 0,
     DSA3D_ERR_INVALID_ARGUMENT = 1,   /* null/misaligned pointer, bad extent, aliasing, bad dtype */
-    DSA3D_ERR_UNSUPPORTED = 2,        /* valid arguments this build does not handle (dh, window) */
+    DSA3D_ERR_UNSUPPORTED = 2,        /* valid arguments this library does not handle (dh, window) */
     DSA3D_ERR_WORKSPACE_TOO_SMALL = 3,
     DSA3D_ERR_CUDA = 4,               /* a CUDA runtime call or kernel launch failed */
     DSA3D_ERR_DEVICE_CHECK = 5        /* a kernel recorded a failed internal check */
