@@ -56,6 +56,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
+    ap.add_argument("--part", choices=["attention", "dwconv"], default="attention",
+                    help="attention: the operator's forward + backward (the default); dwconv: the "
+                         "DWConv3D term of Eq. 1 alone (forward with the fused add, backward) at "
+                         "the workload's shapes")
     ap.add_argument("--heads", type=int, default=0,
                     help="run only this many of the workload's heads (small profiling captures); "
                          "0 = all")
@@ -324,10 +328,97 @@ def path_of(w, abi):
     return fwd, abi.backward_taps
 
 
+def dwconv_units(w):
+    """Per token, the DWConv3D term over C = heads * dh channels with the window's kernel:
+    bytes: forward reads x and the attention output and writes the sum (3 C s), backward reads x
+    and dy and writes dx (3 C s); flop: 2 C K each for the forward and dX, 2 C K for dW."""
+    s = 4 if w.dtype == "f32" else 2
+    C, K = w.heads * w.dh, w.K
+    return {"fwd_bytes": 3 * C * s, "bwd_bytes": 3 * C * s,
+            "fwd_flop": 2 * C * K, "bwd_flop": 4 * C * K}
+
+
+def run_dwconv(args):
+    """--part dwconv: the DWConv3D term's forward (fused into an attention-shaped output) and
+    backward on one GPU, timed like the attention step; one JSON line."""
+    import torch
+    from deformable_slide_attention_b200 import abi, build, inputs
+    build.build()
+    w = inputs.BY_NAME[args.workload]
+    if args.heads:
+        w = dataclasses.replace(w, heads=args.heads)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    C, N = w.heads * w.dh, w.N
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    td = w.torch_dtype
+    x, y, dy = (torch.empty((N, C), dtype=td, device=dev) for _ in range(3))
+    for t in (x, y, dy):
+        inputs._fill_normal_chunked(t, gen)
+    weight = torch.empty((C, *w.window), dtype=torch.float32, device=dev)
+    weight.normal_(0.0, 1.0 / math.sqrt(w.K), generator=gen)
+    bias = torch.empty(C, dtype=torch.float32, device=dev)
+    bias.normal_(0.0, 1.0, generator=gen)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        abi.dwconv3d(x, weight, bias, w.dims, add=y, out=y)  # y += conv(x): the layer's sum
+        abi.dwconv3d_backward(x, weight, dy, w.dims)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(str(getattr(props, "uuid", "") or ""))
+    sampler.start()
+    time.sleep(0.5)
+    abi.dsa3d_timing_reset()
+    abi.dsa3d_timing_enable(True)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    abi.dsa3d_timing_enable(False)
+    ktimes = abi.dsa3d_timing_read()
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    u = dwconv_units(w)
+    peaks, peak_src = measured_peaks()
+    mhz = clocks["sm_mhz"] or float(peaks.get("sm_max_mhz", 1965.0))
+    fp32_peak = props.multi_processor_count * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    flop = N * (u["fwd_flop"] + u["bwd_flop"])
+    tflops = flop / (ms / 1000.0) / 1e12
+    line = {
+        "metric": f"3D-DSA DWConv3D term fwd+bwd tokens/s ({w.name} shapes, C={C}, 1 B200)",
+        "value": N / (ms / 1000.0), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "part": "dwconv", "tokens": N, "channels": C,
+                   "kernel": list(w.window), "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "alu", "achieved": tflops, "peak": fp32_peak, "unit": "TFLOP/s",
+                     "frac": tflops / fp32_peak, "traffic": None,
+                     "peak_basis": f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 x {mhz:.0f} MHz"},
+        "hbm": {"alg_bytes_per_step": N * (u["fwd_bytes"] + u["bwd_bytes"]),
+                "frac_of_hbm": N * (u["fwd_bytes"] + u["bwd_bytes"]) / (ms / 1000.0) / 1e9
+                               / float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))},
+        "kernels": {k: {"launches": n, "avg_ms": tot / n} for k, (n, tot) in ktimes.items()},
+        "gpu_launches": sum(n for n, _ in ktimes.values()), "clocks": clocks,
+        "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.part == "dwconv":
+        return run_dwconv(args)
     import torch
     import torch.distributed as dist
     from deformable_slide_attention_b200 import abi, build, inputs, ranks

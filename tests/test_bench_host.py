@@ -75,3 +75,12 @@ def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.traffic_per_item("dsa3d_bwd_taps_kernel") == (None, None)
     assert bench.traffic_per_item("dsa3d_bwd_q_kernel")[0] == before["dsa3d_bwd_q_kernel"]
+
+
+def test_dwconv_part_units_and_default():
+    assert bench.parse_args([]).part == "attention"  # the default step is the operator's
+    w = inputs.BY_NAME["1080p-long-bf16"]
+    u = bench.dwconv_units(w)
+    C, K = 32 * 128, 243
+    assert u["fwd_bytes"] == u["bwd_bytes"] == 3 * C * 2
+    assert u["fwd_flop"] == 2 * C * K and u["bwd_flop"] == 4 * C * K
