@@ -74,7 +74,7 @@ dsa3d_status_t dwconv_launch_kw(const ConvGeo& g, const void* x, const float* w,
                                 const void* add, void* y, int flip, cudaStream_t st) {
   const int64_t items = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip) * (g.C / 2);
   TimedLaunch tl(kKernDwconv, st);
-  dsa3d_dwconv3d_kernel<T, KW><<<grid_for(items, 256, 8), 256, 0, st>>>(
+  dsa3d_dwconv3d_kernel<T, KW><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
       static_cast<const T*>(x), w, b, static_cast<const T*>(add), static_cast<T*>(y), g, flip);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
@@ -117,7 +117,7 @@ dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* 
   const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
   const int64_t items = (strips + spi - 1) / spi * g.kt * g.kh * (g.C / 2);
   TimedLaunch tl(kKernDwconvDw, st);
-  dsa3d_dwconv3d_dw_kernel<T, KW><<<grid_for(items, 256, 8), 256, 0, st>>>(
+  dsa3d_dwconv3d_dw_kernel<T, KW><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
       static_cast<const T*>(x), static_cast<const T*>(dy), dw, db, g, spi);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;

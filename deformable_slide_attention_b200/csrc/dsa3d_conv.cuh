@@ -23,9 +23,19 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+// Threads per block of the convolution kernels, and the minimum resident blocks per SM asked of
+// the compiler (a register cap; 1 = none).
+#ifndef DSA3D_CONV_THREADS
+#define DSA3D_CONV_THREADS 256
+#endif
+#ifndef DSA3D_CONV_MINB
+#define DSA3D_CONV_MINB 1
+#endif
+
 namespace dsa3d {
 
 constexpr int kConvStrip = 8;  // outputs along x per thread
+constexpr int kConvThreads = DSA3D_CONV_THREADS;
 
 struct ConvGeo {
   int F, Hp, Wp, C;
@@ -160,7 +170,7 @@ __host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const T
 // Y = conv(X) (+ bias) (+ add): one thread per (strip, channel pair), channel pairs fastest.
 // add (nullable) is added element by element (the attention output of Eq. 1; may equal y).
 template <typename T, int KW>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(DSA3D_CONV_THREADS, DSA3D_CONV_MINB)
     dsa3d_dwconv3d_kernel(const T* __restrict__ x, const float* __restrict__ w,
                           const float* __restrict__ bias, const T* add, T* y, const ConvGeo g,
                           const int flip) {
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(256)
 // dW (and db): one thread per (channel pair, kernel row (u, v), range of strips); fp32 partial
 // sums reduced with atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).
 template <typename T, int KW>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(DSA3D_CONV_THREADS, DSA3D_CONV_MINB)
     dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const T* __restrict__ dy, float* dweight,
                              float* dbias, const ConvGeo g, const int strips_per_item) {
   const int pairs = g.C / 2;
