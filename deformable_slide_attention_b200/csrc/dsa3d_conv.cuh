@@ -23,13 +23,16 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-// Threads per block of the convolution kernels, and the minimum resident blocks per SM asked of
-// the compiler (a register cap; 1 = none).
+// Threads per block of the convolution kernels and, if DSA3D_CONV_MINB is defined, the minimum
+// resident blocks per SM asked of the compiler (a register cap).  Without it the launch bounds
+// name the block size alone (the compiler's own register choice).
 #ifndef DSA3D_CONV_THREADS
 #define DSA3D_CONV_THREADS 256
 #endif
-#ifndef DSA3D_CONV_MINB
-#define DSA3D_CONV_MINB 1
+#ifdef DSA3D_CONV_MINB
+#define DSA3D_CONV_BOUNDS __launch_bounds__(DSA3D_CONV_THREADS, DSA3D_CONV_MINB)
+#else
+#define DSA3D_CONV_BOUNDS __launch_bounds__(DSA3D_CONV_THREADS)
 #endif
 
 namespace dsa3d {
@@ -170,7 +173,7 @@ __host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const T
 // Y = conv(X) (+ bias) (+ add): one thread per (strip, channel pair), channel pairs fastest.
 // add (nullable) is added element by element (the attention output of Eq. 1; may equal y).
 template <typename T, int KW>
-__global__ void __launch_bounds__(DSA3D_CONV_THREADS, DSA3D_CONV_MINB)
+__global__ void DSA3D_CONV_BOUNDS
     dsa3d_dwconv3d_kernel(const T* __restrict__ x, const float* __restrict__ w,
                           const float* __restrict__ bias, const T* add, T* y, const ConvGeo g,
                           const int flip) {
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(DSA3D_CONV_THREADS, DSA3D_CONV_MINB)
 // dW (and db): one thread per (channel pair, kernel row (u, v), range of strips); fp32 partial
 // sums reduced with atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).
 template <typename T, int KW>
-__global__ void __launch_bounds__(DSA3D_CONV_THREADS, DSA3D_CONV_MINB)
+__global__ void DSA3D_CONV_BOUNDS
     dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const T* __restrict__ dy, float* dweight,
                              float* dbias, const ConvGeo g, const int strips_per_item) {
   const int pairs = g.C / 2;
