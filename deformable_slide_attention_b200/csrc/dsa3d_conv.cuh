@@ -172,11 +172,12 @@ __host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const T
 #ifdef __CUDACC__
 // Y = conv(X) (+ bias) (+ add): one thread per (strip, channel pair), channel pairs fastest.
 // add (nullable) is added element by element (the attention output of Eq. 1; may equal y).
-template <typename T, int KW>
+// OutT: the output type (the input's, or fp32 for the offset network's first layer).
+template <typename T, int KW, typename OutT = T>
 __global__ void DSA3D_CONV_BOUNDS
     dsa3d_dwconv3d_kernel(const T* __restrict__ x, const float* __restrict__ w,
-                          const float* __restrict__ bias, const T* add, T* y, const ConvGeo g,
-                          const int flip) {
+                          const float* __restrict__ bias, const OutT* add, OutT* y,
+                          const ConvGeo g, const int flip) {
   const int pairs = g.C / 2;
   const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
   const int64_t items = (int64_t)g.F * g.Hp * nxs * pairs;

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "dsa3d_conv.cuh"
+#include "dsa3d_pointwise.cuh"
 
 using namespace dsa3d;
 
@@ -115,6 +116,22 @@ int conv_host_dw(int io, const void* x, const void* dy, int F, int Hp, int Wp, i
   const ConvGeo g = geo(F, Hp, Wp, C, kt, kh, kw);
   return io ? by_kw<Dw, __nv_bfloat16>(kw, x, dy, g, strips_per_item, dw, db)
             : by_kw<Dw, float>(kw, x, dy, g, strips_per_item, dw, db);
+}
+
+// The offset network's pointwise layer over every (token tile, output channel) item:
+// z [N][C] fp32, wp [C][width], bp [width]; offsets [heads][N][taps3 / 3][3] (written).
+int pw_host_offsets(const float* z, const float* wp, const float* bp, int C, int width, int taps3,
+                    long long N, float* offsets) {
+  if (C % 4 || width % taps3) return -1;
+  const int64_t tiles = (N + kPwTokens - 1) / kPwTokens;
+  for (int64_t tile = 0; tile < tiles; tile++)
+    for (int o = 0; o < width; o++) {
+      float acc[kPwTokens];
+      pw_tile(z, wp, bp, C, width, N, tile * kPwTokens, o, acc);
+      for (int t = 0; t < kPwTokens && tile * kPwTokens + t < N; t++)
+        offsets[pw_out_index(N, taps3, tile * kPwTokens + t, o)] = acc[t];
+    }
+  return 0;
 }
 
 }  // extern "C"

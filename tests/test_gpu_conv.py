@@ -75,3 +75,30 @@ def test_rejects_unsupported_and_overlapping():
     x3 = torch.zeros(24, 3, device="cuda", dtype=torch.bfloat16)
     assert abi.dsa3d_dwconv3d(x3.data_ptr(), w3.data_ptr(), None, None, y.data_ptr(), 1, 1, 24, 3, 1, 1,
                               3, abi.DSA3D_BF16, st) == 2  # odd channel count
+
+
+@pytest.mark.parametrize("per_tap", [False, True])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_offset_network_forward(per_tap, dtype):
+    """dsa3d_offset_head against oracle.offset_head (relative 1e-4: fp32 throughout), and the
+    offsets it writes drive the attention exactly as the same offsets given by hand."""
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    C, N, K = heads * dh, math.prod(dims), math.prod(window)
+    g = torch.Generator().manual_seed(77 + int(per_tap))
+    x = torch.randn(N, C, generator=g).to(td)
+    dw_w, dw_b = torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g)
+    width = heads * 3 * (K if per_tap else 1)
+    pw_w, pw_b = torch.randn(C, width, generator=g) * 0.3, torch.randn(width, generator=g)
+    off = abi.offset_head(x.cuda(), dw_w.cuda(), dw_b.cuda(), pw_w.cuda(), pw_b.cuda(), dims, heads,
+                          per_tap=per_tap)
+    torch.cuda.synchronize()
+    ref = oracle.offset_head(x, dw_w, dw_b, pw_w, pw_b, dims, heads, K if per_tap else None)
+    err = np.abs(f64(off) - ref).max()
+    assert err <= 1e-4 * max(1.0, np.abs(ref).max()), err
+    q, k, v = (torch.randn(N, heads, dh, generator=g).to(td).cuda() for _ in range(3))
+    fwd = abi.forward_taps if per_tap else abi.forward
+    out1, lse1 = fwd(q, k, v, off, dims, window)
+    out2, lse2 = fwd(q, k, v, off.clone(), dims, window)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
