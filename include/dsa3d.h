@@ -230,6 +230,23 @@ dsa3d_status_t dsa3d_dwconv3d_backward(const void *x, const float *weight, const
  * after the input, since the offsets' integer parts are taken by a floor.
  */
 size_t dsa3d_offset_head_workspace_bytes(int F, int Hp, int Wp, int C);
+
+/*
+ * Backward of dsa3d_offset_head for the offsets' gradient doffsets (the layout of the offsets;
+ * dsa3d_backward / dsa3d_backward_taps write it): dx [N][C] I/O type (the offset network's part
+ * of the layer input's gradient), d_dw_weight [C][kt][kh][kw], d_dw_bias [C], d_pw_weight
+ * [C][heads*taps*3], d_pw_bias [heads*taps*3], all fp32 and overwritten.  The workspace holds Z
+ * (recomputed) and dZ in fp32: dsa3d_offset_head_backward_workspace_bytes = 2 N C 4 bytes.
+ * C must be a multiple of 16; the other rules are dsa3d_offset_head's.
+ */
+size_t dsa3d_offset_head_backward_workspace_bytes(int F, int Hp, int Wp, int C);
+dsa3d_status_t dsa3d_offset_head_backward(const void *x, const float *dw_weight,
+                                          const float *dw_bias, const float *pw_weight,
+                                          const float *doffsets, void *dx, float *d_dw_weight,
+                                          float *d_dw_bias, float *d_pw_weight, float *d_pw_bias,
+                                          void *workspace, size_t workspace_bytes, int F, int Hp,
+                                          int Wp, int C, int heads, int taps, int kt, int kh,
+                                          int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
 dsa3d_status_t dsa3d_offset_head(const void *x, const float *dw_weight, const float *dw_bias,
                                  const float *pw_weight, const float *pw_bias, float *offsets,
                                  void *workspace, size_t workspace_bytes, int F, int Hp, int Wp,

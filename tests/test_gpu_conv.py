@@ -102,3 +102,27 @@ def test_offset_network_forward(per_tap, dtype):
     out2, lse2 = fwd(q, k, v, off.clone(), dims, window)
     torch.cuda.synchronize()
     assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("per_tap", [False, True])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_offset_network_backward(per_tap, dtype):
+    """dsa3d_offset_head_backward against oracle.offset_head_backward: dx (the I/O tolerance) and
+    the fp32 weight gradients (relative 1e-4)."""
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    C, N, K = heads * dh, math.prod(dims), math.prod(window)
+    g = torch.Generator().manual_seed(91 + int(per_tap))
+    x = torch.randn(N, C, generator=g).to(td)
+    dw_w, dw_b = torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g)
+    width = heads * 3 * (K if per_tap else 1)
+    pw_w = torch.randn(C, width, generator=g) / math.sqrt(C)
+    doff = torch.randn((heads, N, K, 3) if per_tap else (heads, N, 3), generator=g) / math.sqrt(width)
+    got = abi.offset_head_backward(x.cuda(), dw_w.cuda(), dw_b.cuda(), pw_w.cuda(), doff.cuda(), dims,
+                                   heads, per_tap=per_tap)
+    torch.cuda.synchronize()
+    ref = oracle.offset_head_backward(x, dw_w, dw_b, pw_w, doff.double().numpy(), dims)
+    assert_close("dx", f64(got[0]), ref[0], TOL[dtype])
+    for name, a, b in zip(("d dw_weight", "d dw_bias", "d pw_weight", "d pw_bias"), got[1:], ref[1:]):
+        err = np.abs(f64(a) - b).max()
+        assert err <= 1e-4 * max(1.0, np.abs(b).max()), (name, err)
