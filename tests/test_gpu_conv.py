@@ -126,3 +126,33 @@ def test_offset_network_backward(per_tap, dtype):
     for name, a, b in zip(("d dw_weight", "d dw_bias", "d pw_weight", "d pw_bias"), got[1:], ref[1:]):
         err = np.abs(f64(a) - b).max()
         assert err <= 1e-4 * max(1.0, np.abs(b).max()), (name, err)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_layer_against_the_oracle_chain(dtype):
+    """layer.forward / backward (offset network, attention, fused convolution) against the oracle's
+    parts composed the same way, with the GPU's offsets fed to the oracle's attention (so that a
+    floor decision near an integer cannot differ between the two)."""
+    from deformable_slide_attention_b200 import layer
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    C, N, K = heads * dh, math.prod(dims), math.prod(window)
+    g = torch.Generator().manual_seed(123)
+    x = torch.randn(N, C, generator=g).to(td)
+    q, k, v, dout = (torch.randn(N, heads, dh, generator=g).to(td) for _ in range(4))
+    w = [torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g),
+         torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g),
+         torch.randn(C, heads * 3, generator=g) / math.sqrt(C), torch.randn(heads * 3, generator=g)]
+    wts = layer.LayerWeights(*(t.cuda() for t in w))
+    out, ctx = layer.forward(x.cuda(), q.cuda(), k.cuda(), v.cuda(), wts, dims, window)
+    grads = layer.backward(ctx, dout.cuda())
+    torch.cuda.synchronize()
+    off = ctx[4].float().cpu()
+    r_att, _ = oracle.full_forward(q, k, v, off, dims, window)
+    r_out = r_att + oracle.dwconv3d(x, w[0], w[1], dims).reshape(N, heads, dh)
+    assert_close("out", f64(out), r_out, 2 * TOL[dtype])  # attention and sum each rounded once
+    r_dq, r_doff, r_dk, r_dv = oracle.full_backward(q, k, v, off, dout, dims, window)
+    r_dx = (oracle.offset_head_backward(x, w[2], w[3], w[4], r_doff, dims)[0] +
+            oracle.dwconv3d_backward(x, w[0], dout.double().numpy().reshape(N, C), dims)[0])
+    assert_close("dx", f64(grads["x"]), r_dx, 2 * TOL[dtype])
+    assert_close("dq", f64(grads["q"]), r_dq, TOL[dtype])
