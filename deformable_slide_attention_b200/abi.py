@@ -72,6 +72,14 @@ def _load():
         lib.dsa3d_dwconv3d.argtypes = [P, P, P, P, P, *cdims, I, P]
         lib.dsa3d_dwconv3d_backward.restype = I
         lib.dsa3d_dwconv3d_backward.argtypes = [P, P, P, P, P, P, *cdims, I, P]
+        lib.dsa3d_offset_head_workspace_bytes.restype = Z
+        lib.dsa3d_offset_head_workspace_bytes.argtypes = [I, I, I, I]
+        lib.dsa3d_offset_head.restype = I
+        lib.dsa3d_offset_head.argtypes = [P, P, P, P, P, P, P, Z, I, I, I, I, I, I, I, I, I, I, P]
+        lib.dsa3d_offset_head_backward_workspace_bytes.restype = Z
+        lib.dsa3d_offset_head_backward_workspace_bytes.argtypes = [I, I, I, I]
+        lib.dsa3d_offset_head_backward.restype = I
+        lib.dsa3d_offset_head_backward.argtypes = [P] * 11 + [Z] + [I] * 10 + [P]
         lib.dsa3d_check_device.restype = I
         lib.dsa3d_check_device.argtypes = [P]
         lib.dsa3d_timing_enable.restype = I
@@ -157,6 +165,31 @@ def dsa3d_dwconv3d_backward(x, weight, dy, dx, dweight, dbias, F, Hp, Wp, C, kt,
                             stream) -> int:
     return _load().dsa3d_dwconv3d_backward(x, weight, dy, dx, dweight, dbias, F, Hp, Wp, C, kt, kh,
                                            kw, dtype, stream)
+
+
+def dsa3d_offset_head_workspace_bytes(F, Hp, Wp, C) -> int:
+    return _load().dsa3d_offset_head_workspace_bytes(F, Hp, Wp, C)
+
+
+def dsa3d_offset_head(x, dw_weight, dw_bias, pw_weight, pw_bias, offsets, workspace,
+                      workspace_bytes, F, Hp, Wp, C, heads, taps, kt, kh, kw, dtype, stream) -> int:
+    """The offset network's forward: depthwise conv then the pointwise layer, into offsets."""
+    return _load().dsa3d_offset_head(x, dw_weight, dw_bias, pw_weight, pw_bias, offsets, workspace,
+                                     workspace_bytes, F, Hp, Wp, C, heads, taps, kt, kh, kw, dtype,
+                                     stream)
+
+
+def dsa3d_offset_head_backward_workspace_bytes(F, Hp, Wp, C) -> int:
+    return _load().dsa3d_offset_head_backward_workspace_bytes(F, Hp, Wp, C)
+
+
+def dsa3d_offset_head_backward(x, dw_weight, dw_bias, pw_weight, doffsets, dx, d_dw_weight,
+                               d_dw_bias, d_pw_weight, d_pw_bias, workspace, workspace_bytes, F,
+                               Hp, Wp, C, heads, taps, kt, kh, kw, dtype, stream) -> int:
+    return _load().dsa3d_offset_head_backward(x, dw_weight, dw_bias, pw_weight, doffsets, dx,
+                                              d_dw_weight, d_dw_bias, d_pw_weight, d_pw_bias,
+                                              workspace, workspace_bytes, F, Hp, Wp, C, heads, taps,
+                                              kt, kh, kw, dtype, stream)
 
 
 def dsa3d_check_device(stream) -> int:
@@ -416,3 +449,58 @@ def dwconv3d_backward(x, weight, dy, dims, stream=None):
                                    dw.data_ptr(), db.data_ptr(), *dims, C, kt, kh, kw, code,
                                    _stream_handle(stream)), "dsa3d_dwconv3d_backward")
     return dx, dw, db
+
+
+def offset_head(x, dw_weight, dw_bias, pw_weight, pw_bias, dims, heads, per_tap=False, stream=None):
+    """The offset network's forward on CUDA tensors: offsets [heads][N][3] (or [heads][N][K][3]
+    with per_tap) from x [N][C], dw_weight [C][kt][kh][kw], dw_bias [C] or None, pw_weight
+    [C][heads * (K) * 3] and pw_bias (fp32)."""
+    torch = _torch()
+    code = _dtype_code(x)
+    C, kt, kh, kw = _conv_shapes(x, dw_weight, dims)
+    taps = kt * kh * kw if per_tap else 1
+    width = heads * taps * 3
+    if dw_bias is not None:
+        _need(dw_bias, "dw_bias", (C,), torch.float32)
+    _need(pw_weight, "pw_weight", (C, width), torch.float32)
+    _need(pw_bias, "pw_bias", (width,), torch.float32)
+    N = x.shape[0]
+    offsets = torch.empty((heads, N, taps, 3) if per_tap else (heads, N, 3), dtype=torch.float32,
+                          device=x.device)
+    ws = torch.empty(dsa3d_offset_head_workspace_bytes(*dims, C), dtype=torch.uint8, device=x.device)
+    _on_device(x, dw_weight, dw_bias, pw_weight, pw_bias)
+    _check(dsa3d_offset_head(x.data_ptr(), dw_weight.data_ptr(),
+                             dw_bias.data_ptr() if dw_bias is not None else None,
+                             pw_weight.data_ptr(), pw_bias.data_ptr(), offsets.data_ptr(),
+                             ws.data_ptr(), ws.numel(), *dims, C, heads, taps, kt, kh, kw, code,
+                             _stream_handle(stream)), "dsa3d_offset_head")
+    return offsets
+
+
+def offset_head_backward(x, dw_weight, dw_bias, pw_weight, doffsets, dims, heads, per_tap=False,
+                         stream=None):
+    """Gradients of sum(offsets * doffsets) for offsets = offset_head(...): (dx [N][C] in x's
+    dtype, d dw_weight, d dw_bias, d pw_weight, d pw_bias, all fp32 but dx)."""
+    torch = _torch()
+    code = _dtype_code(x)
+    C, kt, kh, kw = _conv_shapes(x, dw_weight, dims)
+    taps = kt * kh * kw if per_tap else 1
+    width = heads * taps * 3
+    N = x.shape[0]
+    if dw_bias is not None:
+        _need(dw_bias, "dw_bias", (C,), torch.float32)
+    _need(pw_weight, "pw_weight", (C, width), torch.float32)
+    _need(doffsets, "doffsets", (heads, N, taps, 3) if per_tap else (heads, N, 3), torch.float32)
+    _on_device(x, dw_weight, dw_bias, pw_weight, doffsets)
+    dx = torch.empty_like(x)
+    grads = (torch.empty_like(dw_weight), torch.empty(C, dtype=torch.float32, device=x.device),
+             torch.empty_like(pw_weight), torch.empty(width, dtype=torch.float32, device=x.device))
+    ws = torch.empty(dsa3d_offset_head_backward_workspace_bytes(*dims, C), dtype=torch.uint8,
+                     device=x.device)
+    _check(dsa3d_offset_head_backward(x.data_ptr(), dw_weight.data_ptr(),
+                                      dw_bias.data_ptr() if dw_bias is not None else None,
+                                      pw_weight.data_ptr(), doffsets.data_ptr(), dx.data_ptr(),
+                                      *(t.data_ptr() for t in grads), ws.data_ptr(), ws.numel(), *dims,
+                                      C, heads, taps, kt, kh, kw, code, _stream_handle(stream)),
+           "dsa3d_offset_head_backward")
+    return (dx, *grads)

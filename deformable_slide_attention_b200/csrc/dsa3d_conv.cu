@@ -8,6 +8,7 @@
 
 #include "dsa3d.h"
 #include "dsa3d_conv.cuh"
+#include "dsa3d_pointwise.cuh"
 #include "dsa3d_timing.cuh"
 
 namespace dsa3d {
@@ -69,29 +70,29 @@ dsa3d_status_t check_conv_shape(int F, int Hp, int Wp, int C, int kt, int kh, in
   return DSA3D_OK;
 }
 
-template <typename T, int KW>
+template <typename T, int KW, typename OutT = T>
 dsa3d_status_t dwconv_launch_kw(const ConvGeo& g, const void* x, const float* w, const float* b,
                                 const void* add, void* y, int flip, cudaStream_t st) {
   const int64_t items = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip) * (g.C / 2);
   TimedLaunch tl(kKernDwconv, st);
-  dsa3d_dwconv3d_kernel<T, KW><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
-      static_cast<const T*>(x), w, b, static_cast<const T*>(add), static_cast<T*>(y), g, flip);
+  dsa3d_dwconv3d_kernel<T, KW, OutT><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
+      static_cast<const T*>(x), w, b, static_cast<const OutT*>(add), static_cast<OutT*>(y), g, flip);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
 }
 
-template <typename T>
+template <typename T, typename OutT = T>
 dsa3d_status_t dwconv_launch(const ConvGeo& g, const void* x, const float* w, const float* b,
                              const void* add, void* y, int flip, cudaStream_t st) {
   switch (g.kw) {
-    case 1: return dwconv_launch_kw<T, 1>(g, x, w, b, add, y, flip, st);
-    case 3: return dwconv_launch_kw<T, 3>(g, x, w, b, add, y, flip, st);
-    case 5: return dwconv_launch_kw<T, 5>(g, x, w, b, add, y, flip, st);
-    case 7: return dwconv_launch_kw<T, 7>(g, x, w, b, add, y, flip, st);
-    case 9: return dwconv_launch_kw<T, 9>(g, x, w, b, add, y, flip, st);
-    case 11: return dwconv_launch_kw<T, 11>(g, x, w, b, add, y, flip, st);
-    case 13: return dwconv_launch_kw<T, 13>(g, x, w, b, add, y, flip, st);
-    case 15: return dwconv_launch_kw<T, 15>(g, x, w, b, add, y, flip, st);
+    case 1: return dwconv_launch_kw<T, 1, OutT>(g, x, w, b, add, y, flip, st);
+    case 3: return dwconv_launch_kw<T, 3, OutT>(g, x, w, b, add, y, flip, st);
+    case 5: return dwconv_launch_kw<T, 5, OutT>(g, x, w, b, add, y, flip, st);
+    case 7: return dwconv_launch_kw<T, 7, OutT>(g, x, w, b, add, y, flip, st);
+    case 9: return dwconv_launch_kw<T, 9, OutT>(g, x, w, b, add, y, flip, st);
+    case 11: return dwconv_launch_kw<T, 11, OutT>(g, x, w, b, add, y, flip, st);
+    case 13: return dwconv_launch_kw<T, 13, OutT>(g, x, w, b, add, y, flip, st);
+    case 15: return dwconv_launch_kw<T, 15, OutT>(g, x, w, b, add, y, flip, st);
     default: return DSA3D_ERR_UNSUPPORTED;
   }
 }
@@ -110,33 +111,37 @@ int dw_strips_per_item(const ConvGeo& g) {
   return (int)spi;
 }
 
-template <typename T, int KW>
+template <typename T, int KW, typename TD = T>
 dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* dy, float* dw,
                                    float* db, cudaStream_t st) {
   const int spi = dw_strips_per_item(g);
   const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
   const int64_t items = (strips + spi - 1) / spi * g.kt * g.kh * (g.C / 2);
   TimedLaunch tl(kKernDwconvDw, st);
-  dsa3d_dwconv3d_dw_kernel<T, KW><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
-      static_cast<const T*>(x), static_cast<const T*>(dy), dw, db, g, spi);
+  dsa3d_dwconv3d_dw_kernel<T, KW, TD><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
+      static_cast<const T*>(x), static_cast<const TD*>(dy), dw, db, g, spi);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
 }
 
-template <typename T>
+template <typename T, typename TD = T>
 dsa3d_status_t dwconv_dw_launch(const ConvGeo& g, const void* x, const void* dy, float* dw,
                                 float* db, cudaStream_t st) {
   switch (g.kw) {
-    case 1: return dwconv_dw_launch_kw<T, 1>(g, x, dy, dw, db, st);
-    case 3: return dwconv_dw_launch_kw<T, 3>(g, x, dy, dw, db, st);
-    case 5: return dwconv_dw_launch_kw<T, 5>(g, x, dy, dw, db, st);
-    case 7: return dwconv_dw_launch_kw<T, 7>(g, x, dy, dw, db, st);
-    case 9: return dwconv_dw_launch_kw<T, 9>(g, x, dy, dw, db, st);
-    case 11: return dwconv_dw_launch_kw<T, 11>(g, x, dy, dw, db, st);
-    case 13: return dwconv_dw_launch_kw<T, 13>(g, x, dy, dw, db, st);
-    case 15: return dwconv_dw_launch_kw<T, 15>(g, x, dy, dw, db, st);
+    case 1: return dwconv_dw_launch_kw<T, 1, TD>(g, x, dy, dw, db, st);
+    case 3: return dwconv_dw_launch_kw<T, 3, TD>(g, x, dy, dw, db, st);
+    case 5: return dwconv_dw_launch_kw<T, 5, TD>(g, x, dy, dw, db, st);
+    case 7: return dwconv_dw_launch_kw<T, 7, TD>(g, x, dy, dw, db, st);
+    case 9: return dwconv_dw_launch_kw<T, 9, TD>(g, x, dy, dw, db, st);
+    case 11: return dwconv_dw_launch_kw<T, 11, TD>(g, x, dy, dw, db, st);
+    case 13: return dwconv_dw_launch_kw<T, 13, TD>(g, x, dy, dw, db, st);
+    case 15: return dwconv_dw_launch_kw<T, 15, TD>(g, x, dy, dw, db, st);
     default: return DSA3D_ERR_UNSUPPORTED;
   }
+}
+
+size_t offset_head_ws_bytes(int F, int Hp, int Wp, int C) {
+  return ((size_t)F * Hp * Wp * C * 4 + 15) & ~size_t(15);
 }
 
 }  // namespace
@@ -203,6 +208,129 @@ dsa3d_status_t dsa3d_dwconv3d_backward(const void* x, const float* weight, const
   if ((rc = dwconv_launch<__nv_bfloat16>(g, dy, weight, nullptr, nullptr, dx, 1, stream)) != DSA3D_OK)
     return rc;
   return dwconv_dw_launch<__nv_bfloat16>(g, x, dy, dweight, dbias, stream);
+}
+
+size_t dsa3d_offset_head_workspace_bytes(int F, int Hp, int Wp, int C) {
+  if (F < 1 || Hp < 1 || Wp < 1 || C < 1) return 0;
+  return offset_head_ws_bytes(F, Hp, Wp, C);
+}
+
+dsa3d_status_t dsa3d_offset_head(const void* x, const float* dw_weight, const float* dw_bias,
+                                 const float* pw_weight, const float* pw_bias, float* offsets,
+                                 void* workspace, size_t workspace_bytes, int F, int Hp, int Wp,
+                                 int C, int heads, int taps, int kt, int kh, int kw,
+                                 dsa3d_dtype_t dtype, cudaStream_t stream) {
+  dsa3d_status_t rc = check_conv_shape(F, Hp, Wp, C, kt, kh, kw, dtype);
+  if (rc != DSA3D_OK) return rc;
+  if (heads < 1 || (taps != 1 && taps != kt * kh * kw)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (C % 4) return DSA3D_ERR_UNSUPPORTED;  // the pointwise layer reads 4 channels at a time
+  if (!x || !dw_weight || !pw_weight || !pw_bias || !offsets || !workspace)
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  if (!aligned16(x) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(offsets) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dw_weight) & 3u) || (reinterpret_cast<uintptr_t>(pw_weight) & 3u) ||
+      (reinterpret_cast<uintptr_t>(pw_bias) & 3u) || (dw_bias && (reinterpret_cast<uintptr_t>(dw_bias) & 7u)))
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < offset_head_ws_bytes(F, Hp, Wp, C)) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+  const ConvGeo g = make_conv_geo(F, Hp, Wp, C, kt, kh, kw);
+  const int width = heads * taps * 3;
+  const size_t tb = (size_t)g.N * C * elem_size(dtype);
+  const size_t ob = (size_t)g.N * width * 4;
+  const Range ins[] = {range_of(x, tb), range_of(dw_weight, (size_t)C * kt * kh * kw * 4),
+                       range_of(dw_bias, dw_bias ? (size_t)C * 4 : 0),
+                       range_of(pw_weight, (size_t)C * width * 4), range_of(pw_bias, (size_t)width * 4)};
+  const Range ro = range_of(offsets, ob), rw = range_of(workspace, workspace_bytes);
+  for (const Range& r : ins)
+    if (overlap(r, ro) || overlap(r, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (overlap(ro, rw)) return DSA3D_ERR_INVALID_ARGUMENT;
+  float* z = static_cast<float*>(workspace);
+  rc = (dtype == DSA3D_F32)
+           ? dwconv_launch<float, float>(g, x, dw_weight, dw_bias, nullptr, z, 0, stream)
+           : dwconv_launch<__nv_bfloat16, float>(g, x, dw_weight, dw_bias, nullptr, z, 0, stream);
+  if (rc != DSA3D_OK) return rc;
+  const int64_t items = (g.N + kPwTokens - 1) / kPwTokens * width;
+  TimedLaunch tl(kKernPointwise, stream);
+  dsa3d_pointwise_offsets_kernel<<<grid_for(items, 256, 8), 256, 0, stream>>>(
+      z, pw_weight, pw_bias, offsets, C, width, taps * 3, g.N);
+  const bool launched = cudaGetLastError() == cudaSuccess;
+  return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+size_t dsa3d_offset_head_backward_workspace_bytes(int F, int Hp, int Wp, int C) {
+  if (F < 1 || Hp < 1 || Wp < 1 || C < 1) return 0;
+  return 2 * offset_head_ws_bytes(F, Hp, Wp, C);
+}
+
+dsa3d_status_t dsa3d_offset_head_backward(const void* x, const float* dw_weight, const float* dw_bias,
+                                          const float* pw_weight, const float* doffsets, void* dx,
+                                          float* d_dw_weight, float* d_dw_bias, float* d_pw_weight,
+                                          float* d_pw_bias, void* workspace, size_t workspace_bytes,
+                                          int F, int Hp, int Wp, int C, int heads, int taps, int kt,
+                                          int kh, int kw, dsa3d_dtype_t dtype, cudaStream_t stream) {
+  dsa3d_status_t rc = check_conv_shape(F, Hp, Wp, C, kt, kh, kw, dtype);
+  if (rc != DSA3D_OK) return rc;
+  if (heads < 1 || (taps != 1 && taps != kt * kh * kw)) return DSA3D_ERR_INVALID_ARGUMENT;
+  if (C % kPwChannels) return DSA3D_ERR_UNSUPPORTED;  // 16-channel groups in the weight gradient
+  if (!x || !dw_weight || !pw_weight || !doffsets || !dx || !d_dw_weight || !d_dw_bias ||
+      !d_pw_weight || !d_pw_bias || !workspace)
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al16[] = {x, dx, workspace};
+  for (const void* p : al16)
+    if (!aligned16(p)) return DSA3D_ERR_INVALID_ARGUMENT;
+  const void* al4[] = {dw_weight, pw_weight, doffsets, d_dw_weight, d_pw_weight, d_pw_bias};
+  for (const void* p : al4)
+    if (reinterpret_cast<uintptr_t>(p) & 3u) return DSA3D_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(d_dw_bias) & 7u) || (dw_bias && (reinterpret_cast<uintptr_t>(dw_bias) & 7u)))
+    return DSA3D_ERR_INVALID_ARGUMENT;
+  const size_t zb = offset_head_ws_bytes(F, Hp, Wp, C);
+  if (workspace_bytes < 2 * zb) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+  const ConvGeo g = make_conv_geo(F, Hp, Wp, C, kt, kh, kw);
+  const int width = heads * taps * 3;
+  const size_t tb = (size_t)g.N * C * elem_size(dtype), wb = (size_t)C * kt * kh * kw * 4;
+  const size_t pwb = (size_t)C * width * 4, ob = (size_t)g.N * width * 4;
+  const Range ins[] = {range_of(x, tb), range_of(dw_weight, wb), range_of(dw_bias, dw_bias ? (size_t)C * 4 : 0),
+                       range_of(pw_weight, pwb), range_of(doffsets, ob)};
+  const Range outs[] = {range_of(dx, tb), range_of(d_dw_weight, wb), range_of(d_dw_bias, (size_t)C * 4),
+                        range_of(d_pw_weight, pwb), range_of(d_pw_bias, (size_t)width * 4),
+                        range_of(workspace, workspace_bytes)};
+  for (int i = 0; i < 6; i++) {
+    for (const Range& r : ins)
+      if (overlap(r, outs[i])) return DSA3D_ERR_INVALID_ARGUMENT;
+    for (int j = i + 1; j < 6; j++)
+      if (overlap(outs[i], outs[j])) return DSA3D_ERR_INVALID_ARGUMENT;
+  }
+  float* z = static_cast<float*>(workspace);
+  float* dz = reinterpret_cast<float*>(static_cast<char*>(workspace) + zb);
+  if (cudaMemsetAsync(d_dw_weight, 0, wb, stream) != cudaSuccess ||
+      cudaMemsetAsync(d_dw_bias, 0, (size_t)C * 4, stream) != cudaSuccess ||
+      cudaMemsetAsync(d_pw_weight, 0, pwb, stream) != cudaSuccess ||
+      cudaMemsetAsync(d_pw_bias, 0, (size_t)width * 4, stream) != cudaSuccess)
+    return DSA3D_ERR_CUDA;
+  const bool f32 = dtype == DSA3D_F32;
+  // Z again (the forward's convolution), then the pointwise layer's dZ and weight gradient
+  rc = f32 ? dwconv_launch<float, float>(g, x, dw_weight, dw_bias, nullptr, z, 0, stream)
+           : dwconv_launch<__nv_bfloat16, float>(g, x, dw_weight, dw_bias, nullptr, z, 0, stream);
+  if (rc != DSA3D_OK) return rc;
+  {
+    const int64_t items = (g.N + kPwTokens - 1) / kPwTokens * C;
+    TimedLaunch tl(kKernPointwiseDz, stream);
+    dsa3d_pointwise_dz_kernel<<<grid_for(items, 256, 8), 256, 0, stream>>>(doffsets, pw_weight, dz, C,
+                                                                          width, taps * 3, g.N);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  {
+    const int64_t per_item = 256;
+    const int64_t items = (g.N + per_item - 1) / per_item * (C / kPwChannels) * width;
+    TimedLaunch tl(kKernPointwiseDw, stream);
+    dsa3d_pointwise_dw_kernel<<<grid_for(items, 256, 8), 256, 0, stream>>>(
+        z, doffsets, d_pw_weight, d_pw_bias, C, width, taps * 3, g.N, per_item);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  // the depthwise convolution's backward for the fp32 dZ
+  rc = f32 ? dwconv_launch<float, float>(g, dz, dw_weight, nullptr, nullptr, dx, 1, stream)
+           : dwconv_launch<float, __nv_bfloat16>(g, dz, dw_weight, nullptr, nullptr, dx, 1, stream);
+  if (rc != DSA3D_OK) return rc;
+  return f32 ? dwconv_dw_launch<float, float>(g, x, dz, d_dw_weight, d_dw_bias, stream)
+             : dwconv_dw_launch<__nv_bfloat16, float>(g, x, dz, d_dw_weight, d_dw_bias, stream);
 }
 
 }  // extern "C"

@@ -134,14 +134,15 @@ __host__ __device__ __forceinline__ void conv_strip(const T* __restrict__ x, con
 // The contribution of one output strip (t, y, x0 .. x0 + kConvStrip - 1) to the weight gradient
 // of kernel row (u, v) of channel pair c2: dwr[j][k] += sum_i dY[(t, y, x0 + i)][2 c2 + k] *
 // X[(t + u - r_t, y + v - r_h, x0 + i + j - r_w)][2 c2 + k]; and, with db != nullptr, the bias
-// gradient db[k] += sum_i dY[...].  Outputs past the volume's last column are skipped.
-template <typename T, int KW>
-__host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const T* __restrict__ dy,
+// gradient db[k] += sum_i dY[...].  Outputs past the volume's last column are skipped.  TD: the
+// type of dY (the input's, or fp32 for the offset network's backward).
+template <typename T, int KW, typename TD = T>
+__host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const TD* __restrict__ dy,
                                                 const ConvGeo& g, int t, int y, int x0, int c2, int u,
                                                 int v, float (&dwr)[KW][2], float* db) {
   const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2, rw = (KW - 1) / 2;
   float ga[kConvStrip], gb[kConvStrip];
-  const T* dyrow = dy + ((int64_t)t * g.Hp + y) * g.Wp * g.C + 2 * c2;
+  const TD* dyrow = dy + ((int64_t)t * g.Hp + y) * g.Wp * g.C + 2 * c2;
 #pragma unroll
   for (int i = 0; i < kConvStrip; i++) {
     ga[i] = gb[i] = 0.f;
@@ -172,11 +173,12 @@ __host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const T
 #ifdef __CUDACC__
 // Y = conv(X) (+ bias) (+ add): one thread per (strip, channel pair), channel pairs fastest.
 // add (nullable) is added element by element (the attention output of Eq. 1; may equal y).
-template <typename T, int KW>
+// OutT: the output type (the input's, or fp32 for the offset network's first layer).
+template <typename T, int KW, typename OutT = T>
 __global__ void DSA3D_CONV_BOUNDS
     dsa3d_dwconv3d_kernel(const T* __restrict__ x, const float* __restrict__ w,
-                          const float* __restrict__ bias, const T* add, T* y, const ConvGeo g,
-                          const int flip) {
+                          const float* __restrict__ bias, const OutT* add, OutT* y,
+                          const ConvGeo g, const int flip) {
   const int pairs = g.C / 2;
   const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
   const int64_t items = (int64_t)g.F * g.Hp * nxs * pairs;
@@ -214,9 +216,9 @@ __global__ void DSA3D_CONV_BOUNDS
 
 // dW (and db): one thread per (channel pair, kernel row (u, v), range of strips); fp32 partial
 // sums reduced with atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).
-template <typename T, int KW>
+template <typename T, int KW, typename TD = T>
 __global__ void DSA3D_CONV_BOUNDS
-    dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const T* __restrict__ dy, float* dweight,
+    dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const TD* __restrict__ dy, float* dweight,
                              float* dbias, const ConvGeo g, const int strips_per_item) {
   const int pairs = g.C / 2;
   const int rows = g.kt * g.kh;
@@ -239,7 +241,7 @@ __global__ void DSA3D_CONV_BOUNDS
       const int x0 = (int)(s % nxs) * kConvStrip;
       const int yy = (int)((s / nxs) % g.Hp);
       const int t = (int)(s / ((int64_t)nxs * g.Hp));
-      dw_row<T, KW>(x, dy, g, t, yy, x0, c2, u, v, dwr, r == 0 ? db : nullptr);
+      dw_row<T, KW, TD>(x, dy, g, t, yy, x0, c2, u, v, dwr, r == 0 ? db : nullptr);
     }
     const int64_t K = (int64_t)rows * KW;
     float* d0 = dweight + (int64_t)(2 * c2) * K + (int64_t)r * KW;

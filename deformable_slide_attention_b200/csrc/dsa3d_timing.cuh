@@ -28,6 +28,9 @@ enum KernelId {
   kKernBwdTaps,
   kKernDwconv,
   kKernDwconvDw,
+  kKernPointwise,
+  kKernPointwiseDz,
+  kKernPointwiseDw,
   kKernCount
 };
 inline const char* kernel_name(int id) {
@@ -37,7 +40,8 @@ inline const char* kernel_name(int id) {
       "dsa3d_scan_kernels",    "dsa3d_sort_fill_kernel",  "dsa3d_bwd_q_kernel",
       "dsa3d_bwd_dq_kernel",   "dsa3d_bwd_kv_kernel",     "dsa3d_pair_v_kernel",
       "dsa3d_fwd_taps_kernel", "dsa3d_bwd_taps_kernel", "dsa3d_dwconv3d_kernel",
-      "dsa3d_dwconv3d_dw_kernel"};
+      "dsa3d_dwconv3d_dw_kernel", "dsa3d_pointwise_offsets_kernel", "dsa3d_pointwise_dz_kernel",
+      "dsa3d_pointwise_dw_kernel"};
   return names[id];
 }
 

@@ -218,6 +218,42 @@ dsa3d_status_t dsa3d_dwconv3d_backward(const void *x, const float *weight, const
                                        cudaStream_t stream);
 
 /*
+ * The offset network of 3D-DSA (MegaSlide-DiT, the 3D-DSA definition: offsets are predicted by a
+ * depthwise 3-D convolution followed by a linear layer), forward:
+ *   Z = depthwise conv of x (as dsa3d_dwconv3d, kernel dw_weight [C][kt][kh][kw], bias dw_bias or
+ *       NULL), in fp32 in the workspace (N * C * 4 bytes, dsa3d_offset_head_workspace_bytes);
+ *   O[n][o] = pw_bias[o] + sum_c Z[n][c] * pw_weight[c][o],  pw_weight [C][heads*taps*3] fp32;
+ *   offsets [heads][N][3] (taps = 1) or [heads][N][K][3] (taps = K = kt*kh*kw) fp32 (written),
+ *   element (h, n, tau, a) = O[n][(h*taps + tau)*3 + a]: the layouts dsa3d_forward and
+ *   dsa3d_forward_taps take.
+ * C must be a multiple of 4; the other shape rules are dsa3d_dwconv3d's.  Everything is fp32
+ * after the input, since the offsets' integer parts are taken by a floor.
+ */
+size_t dsa3d_offset_head_workspace_bytes(int F, int Hp, int Wp, int C);
+
+/*
+ * Backward of dsa3d_offset_head for the offsets' gradient doffsets (the layout of the offsets;
+ * dsa3d_backward / dsa3d_backward_taps write it): dx [N][C] I/O type (the offset network's part
+ * of the layer input's gradient), d_dw_weight [C][kt][kh][kw], d_dw_bias [C], d_pw_weight
+ * [C][heads*taps*3], d_pw_bias [heads*taps*3], all fp32 and overwritten.  The workspace holds Z
+ * (recomputed) and dZ in fp32: dsa3d_offset_head_backward_workspace_bytes = 2 N C 4 bytes.
+ * C must be a multiple of 16; the other rules are dsa3d_offset_head's.
+ */
+size_t dsa3d_offset_head_backward_workspace_bytes(int F, int Hp, int Wp, int C);
+dsa3d_status_t dsa3d_offset_head_backward(const void *x, const float *dw_weight,
+                                          const float *dw_bias, const float *pw_weight,
+                                          const float *doffsets, void *dx, float *d_dw_weight,
+                                          float *d_dw_bias, float *d_pw_weight, float *d_pw_bias,
+                                          void *workspace, size_t workspace_bytes, int F, int Hp,
+                                          int Wp, int C, int heads, int taps, int kt, int kh,
+                                          int kw, dsa3d_dtype_t dtype, cudaStream_t stream);
+dsa3d_status_t dsa3d_offset_head(const void *x, const float *dw_weight, const float *dw_bias,
+                                 const float *pw_weight, const float *pw_bias, float *offsets,
+                                 void *workspace, size_t workspace_bytes, int F, int Hp, int Wp,
+                                 int C, int heads, int taps, int kt, int kh, int kw,
+                                 dsa3d_dtype_t dtype, cudaStream_t stream);
+
+/*
  * Synchronises `stream` and reports DSA3D_ERR_DEVICE_CHECK if any kernel of this library on the
  * current device recorded a failed internal check since the last call (the record is then
  * cleared), DSA3D_ERR_CUDA if the stream reports an error, else DSA3D_OK.

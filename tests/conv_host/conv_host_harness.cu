@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "dsa3d_conv.cuh"
+#include "dsa3d_pointwise.cuh"
 
 using namespace dsa3d;
 
@@ -33,8 +34,8 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
         }
 }
 
-template <typename T, int KW>
-void dw_all(const T* x, const T* dy, const ConvGeo& g, int strips_per_item, float* dw, float* db) {
+template <typename T, int KW, typename TD = T>
+void dw_all(const T* x, const TD* dy, const ConvGeo& g, int strips_per_item, float* dw, float* db) {
   const int pairs = g.C / 2, rows = g.kt * g.kh, nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
   const int64_t strips = (int64_t)g.F * g.Hp * nxs, K = (int64_t)rows * KW;
   const int64_t chunks = (strips + strips_per_item - 1) / strips_per_item;
@@ -48,7 +49,7 @@ void dw_all(const T* x, const T* dy, const ConvGeo& g, int strips_per_item, floa
           const int x0 = (int)(s % nxs) * kConvStrip;
           const int yy = (int)((s / nxs) % g.Hp);
           const int t = (int)(s / ((int64_t)nxs * g.Hp));
-          dw_row<T, KW>(x, dy, g, t, yy, x0, c2, r / g.kh, r % g.kh, dwr, r == 0 ? dbl : nullptr);
+          dw_row<T, KW, TD>(x, dy, g, t, yy, x0, c2, r / g.kh, r % g.kh, dwr, r == 0 ? dbl : nullptr);
         }
         for (int j = 0; j < KW; j++) {
           dw[(int64_t)(2 * c2) * K + (int64_t)r * KW + j] += dwr[j][0];
@@ -79,6 +80,12 @@ template <typename T, int KW>
 struct Fwd {
   static void run(const void* x, const float* w, const float* b, ConvGeo g, int flip, float* y) {
     forward_all<T, KW>(static_cast<const T*>(x), w, b, g, flip, y);
+  }
+};
+template <typename T, int KW>
+struct DwMixed {  // dY in fp32 (the offset network's backward)
+  static void run(const void* x, const void* dy, ConvGeo g, int spi, float* dw, float* db) {
+    dw_all<T, KW, float>(static_cast<const T*>(x), static_cast<const float*>(dy), g, spi, dw, db);
   }
 };
 template <typename T, int KW>
@@ -115,6 +122,58 @@ int conv_host_dw(int io, const void* x, const void* dy, int F, int Hp, int Wp, i
   const ConvGeo g = geo(F, Hp, Wp, C, kt, kh, kw);
   return io ? by_kw<Dw, __nv_bfloat16>(kw, x, dy, g, strips_per_item, dw, db)
             : by_kw<Dw, float>(kw, x, dy, g, strips_per_item, dw, db);
+}
+
+// dW with x in the I/O type (io) and dY in fp32.
+int conv_host_dw_mixed(int io, const void* x, const float* dy, int F, int Hp, int Wp, int C, int kt,
+                       int kh, int kw, int strips_per_item, float* dw, float* db) {
+  if (C % 2 || strips_per_item < 1) return -1;
+  const ConvGeo g = geo(F, Hp, Wp, C, kt, kh, kw);
+  return io ? by_kw<DwMixed, __nv_bfloat16>(kw, x, (const void*)dy, g, strips_per_item, dw, db)
+            : by_kw<DwMixed, float>(kw, x, (const void*)dy, g, strips_per_item, dw, db);
+}
+
+// The pointwise layer's backward over every work item of its two kernels: dz [N][C] written;
+// dwp [C][width] and dbp [width] accumulated into (zero them first).
+int pw_host_backward(const float* z, const float* doff, const float* wp, int C, int width, int taps3,
+                     long long N, long long tokens_per_item, float* dz, float* dwp, float* dbp) {
+  if (C % kPwChannels || width % taps3 || tokens_per_item < 1) return -1;
+  const int64_t tiles = (N + kPwTokens - 1) / kPwTokens;
+  for (int64_t tile = 0; tile < tiles; tile++)
+    for (int c = 0; c < C; c++) {
+      float acc[kPwTokens];
+      pw_dz_tile(doff, wp, width, taps3, N, tile * kPwTokens, c, acc);
+      for (int t = 0; t < kPwTokens && tile * kPwTokens + t < N; t++) dz[(tile * kPwTokens + t) * C + c] = acc[t];
+    }
+  const int64_t chunks = (N + tokens_per_item - 1) / tokens_per_item;
+  for (int64_t chunk = 0; chunk < chunks; chunk++)
+    for (int grp = 0; grp < C / kPwChannels; grp++)
+      for (int o = 0; o < width; o++) {
+        float acc[kPwChannels] = {};
+        float db = 0.f;
+        const int64_t nbeg = chunk * tokens_per_item;
+        const int64_t nend = nbeg + tokens_per_item < N ? nbeg + tokens_per_item : N;
+        pw_dw_tile(z, doff, C, taps3, N, nbeg, nend, o, grp * kPwChannels, acc, grp == 0 ? &db : nullptr);
+        for (int i = 0; i < kPwChannels; i++) dwp[(int64_t)(grp * kPwChannels + i) * width + o] += acc[i];
+        if (grp == 0) dbp[o] += db;
+      }
+  return 0;
+}
+
+// The offset network's pointwise layer over every (token tile, output channel) item:
+// z [N][C] fp32, wp [C][width], bp [width]; offsets [heads][N][taps3 / 3][3] (written).
+int pw_host_offsets(const float* z, const float* wp, const float* bp, int C, int width, int taps3,
+                    long long N, float* offsets) {
+  if (C % 4 || width % taps3) return -1;
+  const int64_t tiles = (N + kPwTokens - 1) / kPwTokens;
+  for (int64_t tile = 0; tile < tiles; tile++)
+    for (int o = 0; o < width; o++) {
+      float acc[kPwTokens];
+      pw_tile(z, wp, bp, C, width, N, tile * kPwTokens, o, acc);
+      for (int t = 0; t < kPwTokens && tile * kPwTokens + t < N; t++)
+        offsets[pw_out_index(N, taps3, tile * kPwTokens + t, o)] = acc[t];
+    }
+  return 0;
 }
 
 }  // extern "C"

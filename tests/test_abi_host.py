@@ -177,3 +177,39 @@ def test_backward_taps_workspace_bytes_and_rejections():
     overlap_ws = list(ptr)
     overlap_ws[10] = ptr[2]  # workspace on top of v
     assert call(overlap_ws, wsb=1 << 20) == 1
+
+
+def test_offset_head_rejections():
+    a = dict(F=2, Hp=4, Wp=4, C=8, heads=2, kt=3, kh=3, kw=3)
+    need = abi.dsa3d_offset_head_workspace_bytes(a["F"], a["Hp"], a["Wp"], a["C"])
+    assert need == 2 * 4 * 4 * 8 * 4
+
+    def call(taps=1, C=8, wsb=need, ws=P * 20, x=P):
+        return abi.dsa3d_offset_head(x, P * 2, None, P * 4, P * 6, P * 8, ws, wsb, a["F"], a["Hp"],
+                                     a["Wp"], C, a["heads"], taps, a["kt"], a["kh"], a["kw"],
+                                     abi.DSA3D_BF16, 0)
+    assert call(taps=5) == 1          # neither 1 nor kt*kh*kw
+    assert call(C=6) == 2             # the pointwise layer reads 4 channels at a time
+    assert call(wsb=need - 16) == 3   # workspace too small
+    assert call(x=0) == 1
+    assert call(ws=P * 8) == 1        # workspace on top of the offsets
+
+
+def test_offset_head_backward_rejections():
+    F, Hp, Wp, C, heads = 2, 4, 4, 16, 2
+    need = abi.dsa3d_offset_head_backward_workspace_bytes(F, Hp, Wp, C)
+    assert need == 2 * F * Hp * Wp * C * 4
+    ptr = [P * (i + 1) for i in range(11)]  # x, dw_w, dw_b, pw_w, doff, dx, ddw, ddb, dpw, dpb, ws
+
+    def call(p=ptr, C=C, taps=1, wsb=need):
+        return abi.dsa3d_offset_head_backward(*p, wsb, F, Hp, Wp, C, heads, taps, 3, 3, 3,
+                                              abi.DSA3D_BF16, 0)
+    assert call(C=8) == 2          # 16-channel groups in the weight gradient
+    assert call(taps=4) == 1
+    assert call(wsb=need - 16) == 3
+    bad = list(ptr)
+    bad[5] = 0                     # dx
+    assert call(bad) == 1
+    alias = list(ptr)
+    alias[5] = ptr[0]              # dx on top of x
+    assert call(alias) == 1

@@ -25,10 +25,10 @@ def calls(monkeypatch):
         return f
 
     for name in ("dsa3d_forward", "dsa3d_backward", "dsa3d_forward_taps", "dsa3d_backward_taps",
-                 "dsa3d_dwconv3d", "dsa3d_dwconv3d_backward"):
+                 "dsa3d_dwconv3d", "dsa3d_dwconv3d_backward", "dsa3d_offset_head"):
         monkeypatch.setattr(abi, name, fake(name))
     for name in ("dsa3d_forward_workspace_bytes", "dsa3d_backward_workspace_bytes",
-                 "dsa3d_backward_taps_workspace_bytes"):
+                 "dsa3d_backward_taps_workspace_bytes", "dsa3d_offset_head_workspace_bytes"):
         monkeypatch.setattr(abi, name, lambda *a: 64)
     monkeypatch.setattr(abi, "_on_device", lambda *a: None)
     monkeypatch.setattr(abi, "_stream_handle", lambda s: 0)
@@ -61,8 +61,14 @@ def test_call_patterns_of_the_tests_and_the_bench_are_accepted(calls):
     y = abi.dwconv3d(x, w, b, DIMS)
     abi.dwconv3d(x, w, None, DIMS, add=y, out=y)  # in place into the attention output
     abi.dwconv3d_backward(x, w, y, DIMS)
+    off = abi.offset_head(x, w, b, torch.zeros(HEADS * DH, HEADS * 3), torch.zeros(HEADS * 3), DIMS, HEADS)
+    assert off.shape == (HEADS, N, 3)
+    off = abi.offset_head(x, w, None, torch.zeros(HEADS * DH, HEADS * K * 3), torch.zeros(HEADS * K * 3),
+                          DIMS, HEADS, per_tap=True)
+    assert off.shape == (HEADS, N, K, 3)
     assert calls == ["dsa3d_forward"] * 3 + ["dsa3d_backward"] * 2 + ["dsa3d_forward_taps"] * 2 + \
-        ["dsa3d_backward_taps"] * 2 + ["dsa3d_dwconv3d"] * 2 + ["dsa3d_dwconv3d_backward"]
+        ["dsa3d_backward_taps"] * 2 + ["dsa3d_dwconv3d"] * 2 + ["dsa3d_dwconv3d_backward"] + \
+        ["dsa3d_offset_head"] * 2
 
 
 def test_mismatched_tensors_are_refused_before_any_call(calls):
@@ -88,6 +94,10 @@ def test_mismatched_tensors_are_refused_before_any_call(calls):
         lambda: abi.dwconv3d(torch.zeros(N, 8), torch.zeros(8, *WINDOW), None, DIMS,
                              add=torch.zeros(N, 8, dtype=torch.bfloat16)),
         lambda: abi.dwconv3d_backward(torch.zeros(N, 8), torch.zeros(8, *WINDOW), torch.zeros(N, 4), DIMS),
+        lambda: abi.offset_head(torch.zeros(N, 8), torch.zeros(8, *WINDOW), None, torch.zeros(8, 5),
+                                torch.zeros(6), DIMS, 2),                             # pw width
+        lambda: abi.offset_head(torch.zeros(N, 8), torch.zeros(8, *WINDOW), None, torch.zeros(8, 6),
+                                torch.zeros(6, dtype=torch.float64), DIMS, 2),        # pw bias dtype
     ]
     for i, f in enumerate(bad):
         with pytest.raises(ValueError):

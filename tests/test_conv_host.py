@@ -1,5 +1,6 @@
 """The depthwise-convolution kernels' per-thread routines (conv_strip, dw_row in
-csrc/dsa3d_conv.cuh), run on the CPU by a host harness over every work item the GPU kernels
+csrc/dsa3d_conv.cuh) and the offset network's pointwise routine (pw_tile in
+csrc/dsa3d_pointwise.cuh), run on the CPU by a host harness over every work item the GPU kernels
 process, against the oracle's convolution (reading R9).  This checks their indexing, boundary
 handling, kernel flip and weight-gradient accumulation without a GPU; the GPU parity tests call
 the same code through the C ABI.
@@ -27,7 +28,7 @@ LIB = os.path.join(HERE, "conv_host", "_build", "libconvhost.so")
 
 @pytest.fixture(scope="module")
 def harness():
-    deps = [SRC, os.path.join(CSRC, "dsa3d_conv.cuh")]
+    deps = [SRC, os.path.join(CSRC, "dsa3d_conv.cuh"), os.path.join(CSRC, "dsa3d_pointwise.cuh")]
     if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(d) for d in deps):
         os.makedirs(os.path.dirname(LIB), exist_ok=True)
         subprocess.run(["/usr/local/cuda/bin/nvcc", "-O2", "-std=c++17", "-x", "cu",
@@ -38,6 +39,10 @@ def harness():
     I, P = ctypes.c_int, ctypes.c_void_p
     lib.conv_host_forward.argtypes = [I, P, P, P] + [I] * 7 + [I, P]
     lib.conv_host_dw.argtypes = [I, P, P] + [I] * 7 + [I, P, P]
+    lib.pw_host_offsets.argtypes = [P, P, P, I, I, I, ctypes.c_longlong, P]
+    lib.conv_host_dw_mixed.argtypes = [I, P, P] + [I] * 7 + [I, P, P]
+    L = ctypes.c_longlong
+    lib.pw_host_backward.argtypes = [P, P, P, I, I, I, L, L, P, P, P]
     return lib
 
 
@@ -117,3 +122,64 @@ def test_unsupported_width_is_refused(harness):
     w = np.zeros((2, 1, 1, 17), np.float32)
     io, xa = _io(x)
     assert harness.conv_host_forward(io, _ptr(xa), _ptr(w), None, 1, 1, 6, 2, 1, 1, 17, 0, _ptr(y)) == -1
+
+
+@pytest.mark.parametrize("taps", [None, 9])
+@pytest.mark.parametrize("dims,heads,dh,window", [((2, 5, 6), 2, 8, (1, 3, 3)),
+                                                  ((3, 4, 9), 3, 4, (3, 3, 5))])
+def test_offset_network_matches_oracle(harness, dims, heads, dh, window, taps):
+    """Z = the conv routine in fp32 (as the GPU writes it to its workspace), then the pointwise
+    routine into the attention's offset layout, against oracle.offset_head."""
+    if taps is not None:
+        taps = math.prod(window)
+    C, N = heads * dh, math.prod(dims)
+    g = torch.Generator().manual_seed(C + N)
+    x = torch.randn(N, C, generator=g).to(torch.bfloat16)
+    dw_w, dw_b = torch.randn(C, *window, generator=g), torch.randn(C, generator=g)
+    width = heads * 3 * (taps or 1)
+    pw_w = torch.randn(C, width, generator=g) * 0.2
+    pw_b = torch.randn(width, generator=g)
+    z = host_forward(harness, x, dw_w, dw_b, dims)
+    off = np.zeros((heads, N, taps, 3) if taps else (heads, N, 3), np.float32)
+    wa, ba = pw_w.contiguous().numpy(), pw_b.contiguous().numpy()
+    rc = harness.pw_host_offsets(_ptr(np.ascontiguousarray(z)), _ptr(wa), _ptr(ba), C, width,
+                                 3 * (taps or 1), N, _ptr(off))
+    assert rc == 0
+    ref = oracle.offset_head(x, dw_w, dw_b, pw_w, pw_b, dims, heads, taps)
+    assert np.abs(off - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max())
+
+
+@pytest.mark.parametrize("taps", [None, 9])
+@pytest.mark.parametrize("tokens_per_item", [7, 1000])
+def test_offset_network_backward_matches_oracle(harness, taps, tokens_per_item):
+    """The backward's pieces in the order the library runs them: Z (conv, fp32), dZ and dWp/dbp
+    (pointwise), dX (conv of the fp32 dZ with the flipped kernel), dW/db (x in bf16, dZ in fp32),
+    against oracle.offset_head_backward."""
+    dims, heads, dh, window = (2, 5, 6), 2, 16, (1, 3, 3)
+    if taps is not None:
+        taps = math.prod(window)
+    C, N = heads * dh, math.prod(dims)
+    g = torch.Generator().manual_seed(5 + C)
+    x = torch.randn(N, C, generator=g).to(torch.bfloat16)
+    dw_w, dw_b = torch.randn(C, *window, generator=g), torch.randn(C, generator=g)
+    width = heads * 3 * (taps or 1)
+    pw_w = torch.randn(C, width, generator=g) * 0.2
+    doff = torch.randn((heads, N, taps, 3) if taps else (heads, N, 3), generator=g)
+    z = np.ascontiguousarray(host_forward(harness, x, dw_w, dw_b, dims))
+    dz = np.zeros((N, C), np.float32)
+    dwp = np.zeros((C, width), np.float32)
+    dbp = np.zeros(width, np.float32)
+    wa, da = pw_w.contiguous().numpy(), doff.contiguous().numpy()
+    assert harness.pw_host_backward(_ptr(z), _ptr(da), _ptr(wa), C, width, 3 * (taps or 1), N,
+                                    tokens_per_item, _ptr(dz), _ptr(dwp), _ptr(dbp)) == 0
+    dx = host_forward(harness, torch.from_numpy(dz), dw_w, None, dims, flip=True)
+    ddw = np.zeros((C, *window), np.float32)
+    ddb = np.zeros(C, np.float32)
+    io, xa = _io(x)
+    assert harness.conv_host_dw_mixed(io, _ptr(xa), _ptr(dz), *dims, C, *window, 3, _ptr(ddw),
+                                      _ptr(ddb)) == 0
+    ref = oracle.offset_head_backward(x, dw_w, dw_b, pw_w, doff.double().numpy(), dims)
+    for name, got, want in (("dx", dx, ref[0]), ("d dw_weight", ddw, ref[1]), ("d dw_bias", ddb, ref[2]),
+                            ("d pw_weight", dwp, ref[3]), ("d pw_bias", dbp, ref[4])):
+        err = np.abs(got - want).max()
+        assert err <= 1e-4 * max(1.0, np.abs(want).max()), (name, err)

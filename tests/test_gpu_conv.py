@@ -75,3 +75,84 @@ def test_rejects_unsupported_and_overlapping():
     x3 = torch.zeros(24, 3, device="cuda", dtype=torch.bfloat16)
     assert abi.dsa3d_dwconv3d(x3.data_ptr(), w3.data_ptr(), None, None, y.data_ptr(), 1, 1, 24, 3, 1, 1,
                               3, abi.DSA3D_BF16, st) == 2  # odd channel count
+
+
+@pytest.mark.parametrize("per_tap", [False, True])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_offset_network_forward(per_tap, dtype):
+    """dsa3d_offset_head against oracle.offset_head (relative 1e-4: fp32 throughout), and the
+    offsets it writes drive the attention exactly as the same offsets given by hand."""
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    C, N, K = heads * dh, math.prod(dims), math.prod(window)
+    g = torch.Generator().manual_seed(77 + int(per_tap))
+    x = torch.randn(N, C, generator=g).to(td)
+    dw_w, dw_b = torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g)
+    width = heads * 3 * (K if per_tap else 1)
+    pw_w, pw_b = torch.randn(C, width, generator=g) * 0.3, torch.randn(width, generator=g)
+    off = abi.offset_head(x.cuda(), dw_w.cuda(), dw_b.cuda(), pw_w.cuda(), pw_b.cuda(), dims, heads,
+                          per_tap=per_tap)
+    torch.cuda.synchronize()
+    ref = oracle.offset_head(x, dw_w, dw_b, pw_w, pw_b, dims, heads, K if per_tap else None)
+    err = np.abs(f64(off) - ref).max()
+    assert err <= 1e-4 * max(1.0, np.abs(ref).max()), err
+    q, k, v = (torch.randn(N, heads, dh, generator=g).to(td).cuda() for _ in range(3))
+    fwd = abi.forward_taps if per_tap else abi.forward
+    out1, lse1 = fwd(q, k, v, off, dims, window)
+    out2, lse2 = fwd(q, k, v, off.clone(), dims, window)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("per_tap", [False, True])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_offset_network_backward(per_tap, dtype):
+    """dsa3d_offset_head_backward against oracle.offset_head_backward: dx (the I/O tolerance) and
+    the fp32 weight gradients (relative 1e-4)."""
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    C, N, K = heads * dh, math.prod(dims), math.prod(window)
+    g = torch.Generator().manual_seed(91 + int(per_tap))
+    x = torch.randn(N, C, generator=g).to(td)
+    dw_w, dw_b = torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g)
+    width = heads * 3 * (K if per_tap else 1)
+    pw_w = torch.randn(C, width, generator=g) / math.sqrt(C)
+    doff = torch.randn((heads, N, K, 3) if per_tap else (heads, N, 3), generator=g) / math.sqrt(width)
+    got = abi.offset_head_backward(x.cuda(), dw_w.cuda(), dw_b.cuda(), pw_w.cuda(), doff.cuda(), dims,
+                                   heads, per_tap=per_tap)
+    torch.cuda.synchronize()
+    ref = oracle.offset_head_backward(x, dw_w, dw_b, pw_w, doff.double().numpy(), dims)
+    assert_close("dx", f64(got[0]), ref[0], TOL[dtype])
+    for name, a, b in zip(("d dw_weight", "d dw_bias", "d pw_weight", "d pw_bias"), got[1:], ref[1:]):
+        err = np.abs(f64(a) - b).max()
+        assert err <= 1e-4 * max(1.0, np.abs(b).max()), (name, err)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_layer_against_the_oracle_chain(dtype):
+    """layer.forward / backward (offset network, attention, fused convolution) against the oracle's
+    parts composed the same way, with the GPU's offsets fed to the oracle's attention (so that a
+    floor decision near an integer cannot differ between the two)."""
+    from deformable_slide_attention_b200 import layer
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    C, N, K = heads * dh, math.prod(dims), math.prod(window)
+    g = torch.Generator().manual_seed(123)
+    x = torch.randn(N, C, generator=g).to(td)
+    q, k, v, dout = (torch.randn(N, heads, dh, generator=g).to(td) for _ in range(4))
+    w = [torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g),
+         torch.randn(C, *window, generator=g) / math.sqrt(K), torch.randn(C, generator=g),
+         torch.randn(C, heads * 3, generator=g) / math.sqrt(C), torch.randn(heads * 3, generator=g)]
+    wts = layer.LayerWeights(*(t.cuda() for t in w))
+    out, ctx = layer.forward(x.cuda(), q.cuda(), k.cuda(), v.cuda(), wts, dims, window)
+    grads = layer.backward(ctx, dout.cuda())
+    torch.cuda.synchronize()
+    off = ctx[4].float().cpu()
+    r_att, _ = oracle.full_forward(q, k, v, off, dims, window)
+    r_out = r_att + oracle.dwconv3d(x, w[0], w[1], dims).reshape(N, heads, dh)
+    assert_close("out", f64(out), r_out, 2 * TOL[dtype])  # attention and sum each rounded once
+    r_dq, r_doff, r_dk, r_dv = oracle.full_backward(q, k, v, off, dout, dims, window)
+    r_dx = (oracle.offset_head_backward(x, w[2], w[3], w[4], r_doff, dims)[0] +
+            oracle.dwconv3d_backward(x, w[0], dout.double().numpy().reshape(N, C), dims)[0])
+    assert_close("dx", f64(grads["x"]), r_dx, 2 * TOL[dtype])
+    assert_close("dq", f64(grads["q"]), r_dq, TOL[dtype])
