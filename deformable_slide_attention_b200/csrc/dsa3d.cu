@@ -286,27 +286,22 @@ dsa3d_status_t check_workspace(const void* ws, size_t bytes, const Range* ins, i
 
 dsa3d_status_t zero16(void* p, size_t n16, cudaStream_t st);
 
+// Sort the queries of heads [h0, h0 + hg) by window origin into w (dsa3d_sort.cuh): zero the
+// bucket counts, count, scan, fill, then order each bucket by token index so that the sorted
+// arrays are the same in every run.  Queries without a valid tap get zero rows of zrow (the
+// forward's out or the backward's dq), lse = -inf (when lse is given) and zero doff (when given).
 template <int DH>
-dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const void* v,
-                             const float* off, void* out, float* lse, const SortWs& w,
-                             unsigned* vp, int h0, int hg, cudaStream_t st) {
+dsa3d_status_t sort_queries(const Shape& s, const float* off, const SortWs& w, int h0, int hg,
+                            __nv_bfloat16* zrow, float* lse, float* doff, cudaStream_t st) {
   const Geo g = make_geo(s);
   const SortGeo sg = make_sort_geo(s);
-  const int Wp2 = pair_width(s);
   dsa3d_status_t rc = zero16(w.cnt, align16(w.cnt_elems * 4) / 16, st);
   if (rc != DSA3D_OK) return rc;
   const int64_t items = (int64_t)hg * s.N;
   {
-    TimedLaunch tl(kKernPairV, st);
-    const int64_t pitems = (int64_t)s.F * s.Hp * Wp2 * hg * (DH / 8);
-    dsa3d_pair_v_kernel<DH><<<grid_for(pitems, 256, 16), 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(v), vp, g, Wp2, h0, hg);
-    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
-  }
-  {
     TimedLaunch tl(kKernSortCount, st);
     dsa3d_sort_count_kernel<__nv_bfloat16, DH><<<grid_for(items, 256, 16), 256, 0, st>>>(
-        off, g, sg, h0, hg, w.cnt, w.qkey, w.qrank, static_cast<__nv_bfloat16*>(out), lse, nullptr);
+        off, g, sg, h0, hg, w.cnt, w.qkey, w.qrank, zrow, lse, doff);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
   {
@@ -322,6 +317,36 @@ dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const
                                                                      w.sorted_n, w.sorted_ex);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
+  // order: the scan's block sums are spent, so bsum[0] counts the large buckets (listed in qkey,
+  // whose keys are spent too) and qrank is the merge scratch of their runs
+  if ((rc = zero16(w.bsum, 1, st)) != DSA3D_OK) return rc;
+  {
+    TimedLaunch tl(kKernSortOrder, st);
+    dsa3d_sort_order_kernel<<<grid_for(w.cnt_elems - 1, 256, 16), 256, 0, st>>>(
+        w.cnt, w.cnt_elems - 1, w.sorted_n, w.qkey, w.bsum);
+    dsa3d_sort_order_big_kernel<<<device_info().sms, kBigThreads, 0, st>>>(w.cnt, w.qkey, w.bsum,
+                                                                           w.sorted_n, w.qrank);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  return DSA3D_OK;
+}
+
+template <int DH>
+dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const void* v,
+                             const float* off, void* out, float* lse, const SortWs& w,
+                             unsigned* vp, int h0, int hg, cudaStream_t st) {
+  const Geo g = make_geo(s);
+  const SortGeo sg = make_sort_geo(s);
+  const int Wp2 = pair_width(s);
+  {
+    TimedLaunch tl(kKernPairV, st);
+    const int64_t pitems = (int64_t)s.F * s.Hp * Wp2 * hg * (DH / 8);
+    dsa3d_pair_v_kernel<DH><<<grid_for(pitems, 256, 16), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(v), vp, g, Wp2, h0, hg);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  }
+  dsa3d_status_t rc = sort_queries<DH>(s, off, w, h0, hg, static_cast<__nv_bfloat16*>(out), lse, nullptr, st);
+  if (rc != DSA3D_OK) return rc;
   {
     // the scores warp's tap loops sized for the window: two lanes per query, ceil(kw / 2) taps each
     auto kern = (s.kw <= 9) ? dsa3d_fwd_mma_kernel<DH, 5> : dsa3d_fwd_mma_kernel<DH, 8>;
@@ -383,28 +408,8 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
   const bf* vb = static_cast<const bf*>(v);
   const bf* ob = static_cast<const bf*>(dout);
 
-  dsa3d_status_t rc = zero16(w.cnt, align16(w.cnt_elems * 4) / 16, st);
+  dsa3d_status_t rc = sort_queries<DH>(s, off, w, h0, hg, static_cast<bf*>(dq), nullptr, doff, st);
   if (rc != DSA3D_OK) return rc;
-  const int64_t items = (int64_t)hg * s.N;
-  {
-    TimedLaunch tl(kKernSortCount, st);
-    dsa3d_sort_count_kernel<bf, DH><<<grid_for(items, 256, 16), 256, 0, st>>>(
-        off, g, sg, h0, hg, w.cnt, w.qkey, w.qrank, static_cast<bf*>(dq), nullptr, doff);
-    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
-  }
-  {
-    TimedLaunch tl(kKernScan, st);
-    dsa3d_scan_blocks_kernel<<<(unsigned)w.nb, kScanThreads, 0, st>>>(w.cnt, w.cnt_elems, w.bsum);
-    dsa3d_scan_sums_kernel<<<1, kScanThreads, 0, st>>>(w.bsum, (int)w.nb);
-    dsa3d_scan_apply_kernel<<<(unsigned)w.nb, kScanThreads, 0, st>>>(w.cnt, w.cnt_elems, w.bsum);
-    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
-  }
-  {
-    TimedLaunch tl(kKernSortFill, st);
-    dsa3d_sort_fill_kernel<<<grid_for(items, 256, 16), 256, 0, st>>>(w.cnt, w.qkey, w.qrank, g, sg, hg,
-                                                                     w.sorted_n, w.sorted_ex);
-    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
-  }
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
   {
     const int smem = 2 * bwdq_pair_floats() * (int)sizeof(float);  // two warp pairs per CTA
@@ -677,6 +682,7 @@ dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const 
 
   const Geo g = make_geo(s);
   const DeviceInfo d = device_info();
+  if (d.sms == 0) return DSA3D_ERR_CUDA;  // no usable device
   const int warps = pick_warps(g, false, d.max_smem);
   if (warps == 0) return DSA3D_ERR_UNSUPPORTED;
   if (dtype == DSA3D_F32)
@@ -736,6 +742,7 @@ dsa3d_status_t dsa3d_backward(const void* q, const void* k, const void* v, const
 
   const Geo g = make_geo(s);
   const DeviceInfo d = device_info();
+  if (d.sms == 0) return DSA3D_ERR_CUDA;  // no usable device
   const int warps = pick_warps(g, true, d.max_smem);
   if (warps == 0) return DSA3D_ERR_UNSUPPORTED;
 
@@ -781,9 +788,12 @@ dsa3d_status_t dsa3d_backward_noalloc(const void* q, const void* k, const void* 
   const Shape s{F, Hp, Wp, heads, dh, kt, kh, kw, (int64_t)F * Hp * Wp};
   const dsa3d_status_t rc = check_shape(s, dtype, 0);
   if (rc != DSA3D_OK) return rc;
-  // reject, before any device work, a head that does not fit the fixed scratch
-  if (dtype == DSA3D_BF16 && acc_bytes_per_head(s) > DSA3D_NOALLOC_SCRATCH_BYTES)
-    return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+  // reject, before any device work, a problem whose single head fits neither path in the fixed
+  // scratch: the tensor-core path's sort and splats, or the general path's fp32 accumulators
+  if (dtype == DSA3D_BF16) {
+    const bool mma_fits = mma_forward_ok(s, dtype) && mma_bwd_ws_bytes(s, 1) <= DSA3D_NOALLOC_SCRATCH_BYTES;
+    if (!mma_fits && acc_bytes_per_head(s) > DSA3D_NOALLOC_SCRATCH_BYTES) return DSA3D_ERR_WORKSPACE_TOO_SMALL;
+  }
   void* scratch = nullptr;
   const dsa3d_status_t sc = noalloc_scratch(&scratch);
   if (sc != DSA3D_OK) return sc;

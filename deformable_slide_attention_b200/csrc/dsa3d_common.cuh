@@ -206,7 +206,8 @@ __device__ __forceinline__ void unpack3(int r, int& a, int& b, int& c) {
 }
 
 // Device-side check record (set by kernels built with DSA3D_DEBUG, read by dsa3d_check_device).
-// The library is one translation unit, so this is its only definition.
+// Of the library's two translation units only dsa3d.cu includes this header (the convolution's
+// dsa3d_conv.cu does not), so this is its only definition.
 __device__ int g_dsa3d_check;
 
 #ifdef DSA3D_DEBUG

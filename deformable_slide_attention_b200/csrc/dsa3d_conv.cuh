@@ -39,6 +39,8 @@ namespace dsa3d {
 
 constexpr int kConvStrip = 8;  // outputs along x per thread
 constexpr int kConvThreads = DSA3D_CONV_THREADS;
+static_assert(kConvThreads % 32 == 0 && kConvThreads >= 32 && kConvThreads <= 1024,
+              "DSA3D_CONV_THREADS: whole warps, at most 1024 threads per block");
 
 struct ConvGeo {
   int F, Hp, Wp, C;

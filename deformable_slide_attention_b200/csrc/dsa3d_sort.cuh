@@ -9,7 +9,9 @@
 //
 // Steps: count (per query: bucket and rank by atomicAdd), exclusive scan over all heads' bucket
 // counts (block sums, a single-block scan of those, block-local scans), fill (scatter token
-// index and e_x to the sorted position).  The order within one bucket follows the atomics.
+// index and e_x to the sorted position), order (sort each bucket's queries by token index).  The
+// fill's order within one bucket follows the atomics; the order step makes the sorted arrays,
+// and with them every kernel that reads them, the same from run to run.
 #pragma once
 
 #include "dsa3d_common.cuh"
@@ -161,6 +163,110 @@ __global__ void dsa3d_sort_fill_kernel(const int* __restrict__ start, const int*
     DSA3D_DEVICE_CHECK(pos >= 0 && pos < items);
     sorted_n[pos] = (int)n;
     sorted_ex[pos] = key % sg.Ex;
+  }
+}
+
+// ---- deterministic order within a bucket ---------------------------------------------------
+// dsa3d_sort_order_kernel sorts each bucket's run of sorted_n by token index: one thread per
+// bucket of at most kSmallBucket queries (insertion sort in place); larger buckets are listed in
+// big[] (count in *nbig, zero on entry) for dsa3d_sort_order_big_kernel, one CTA per listed
+// bucket: bitonic sorts of kBigChunk-query chunks in shared memory, then bottom-up merges of the
+// sorted runs between the run and a scratch array of the same positions.  sorted_ex is the same
+// for every query of a bucket, so it needs no reordering.  nb = buckets of the head group
+// (hg * E1 - 1: bucket b's run is [start[b], start[b+1])).
+constexpr int kSmallBucket = 32;
+constexpr int kBigThreads = 512;
+constexpr int kBigChunk = 4096;  // ints per shared-memory chunk (a power of two)
+
+__global__ void dsa3d_sort_order_kernel(const int* __restrict__ start, const int64_t nb,
+                                        int* __restrict__ sorted_n, int* __restrict__ big,
+                                        int* __restrict__ nbig) {
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nb;
+       b += (int64_t)gridDim.x * blockDim.x) {
+    const int lo = start[b], S = start[b + 1] - lo;
+    if (S < 2) continue;
+    if (S > kSmallBucket) {
+      big[atomicAdd(nbig, 1)] = (int)b;
+      continue;
+    }
+    int* a = sorted_n + lo;
+    for (int i = 1; i < S; i++) {
+      const int x = a[i];
+      int j = i - 1;
+      while (j >= 0 && a[j] > x) {
+        a[j + 1] = a[j];
+        j--;
+      }
+      a[j + 1] = x;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kBigThreads)
+    dsa3d_sort_order_big_kernel(const int* __restrict__ start, const int* __restrict__ big,
+                                const int* __restrict__ nbig, int* __restrict__ sorted_n,
+                                int* __restrict__ scratch) {
+  __shared__ int sh[kBigChunk];
+  const int count = *nbig;
+  for (int e = blockIdx.x; e < count; e += gridDim.x) {
+    const int b = big[e];
+    const int lo = start[b], S = start[b + 1] - lo;
+    int* a = sorted_n + lo;
+    // 1. sort each chunk (padded to a power of two with INT_MAX, larger than any token index)
+    for (int c0 = 0; c0 < S; c0 += kBigChunk) {
+      const int n = min(kBigChunk, S - c0);
+      int P = 1;
+      while (P < n) P <<= 1;
+      for (int i = threadIdx.x; i < P; i += blockDim.x) sh[i] = i < n ? a[c0 + i] : 0x7fffffff;
+      __syncthreads();
+      for (int k = 2; k <= P; k <<= 1)
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          for (int i = threadIdx.x; i < P; i += blockDim.x) {
+            const int l = i ^ j;
+            if (l > i) {
+              const bool up = (i & k) == 0;
+              const int x = sh[i], y = sh[l];
+              if ((x > y) == up) {
+                sh[i] = y;
+                sh[l] = x;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      for (int i = threadIdx.x; i < n; i += blockDim.x) a[c0 + i] = sh[i];
+      __syncthreads();
+    }
+    // 2. merge pairs of sorted runs of width w (token indices are distinct: no ties); output
+    //    element o of a pair takes the co-rank i (elements of the first run before it) by binary
+    //    search along the merge path
+    int* src = a;
+    int* dst = scratch + lo;
+    for (int w = kBigChunk; w < S; w <<= 1) {
+      for (int o = threadIdx.x; o < S; o += blockDim.x) {
+        const int p0 = (o / (2 * w)) * (2 * w);
+        const int n1 = min(w, S - p0), n2 = max(0, min(w, S - p0 - w));
+        const int* A = src + p0;
+        const int* B = A + n1;
+        const int k = o - p0;
+        int ilo = max(0, k - n2), ihi = min(k, n1);
+        while (ilo < ihi) {
+          const int i = (ilo + ihi) >> 1;
+          if (A[i] < B[k - i - 1]) ilo = i + 1;
+          else ihi = i;
+        }
+        const int i = ilo, j = k - ilo;
+        dst[o] = (i < n1 && (j >= n2 || A[i] < B[j])) ? A[i] : B[j];
+      }
+      __syncthreads();
+      int* tmp = src;
+      src = dst;
+      dst = tmp;
+    }
+    if (src != a) {
+      for (int i = threadIdx.x; i < S; i += blockDim.x) a[i] = src[i];
+    }
+    __syncthreads();
   }
 }
 

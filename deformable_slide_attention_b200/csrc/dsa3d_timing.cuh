@@ -31,6 +31,8 @@ enum KernelId {
   kKernPointwise,
   kKernPointwiseDz,
   kKernPointwiseDw,
+  kKernSortOrder,
+  kKernFwdTc,
   kKernCount
 };
 inline const char* kernel_name(int id) {
@@ -41,7 +43,7 @@ inline const char* kernel_name(int id) {
       "dsa3d_bwd_dq_kernel",   "dsa3d_bwd_kv_kernel",     "dsa3d_pair_v_kernel",
       "dsa3d_fwd_taps_kernel", "dsa3d_bwd_taps_kernel", "dsa3d_dwconv3d_kernel",
       "dsa3d_dwconv3d_dw_kernel", "dsa3d_pointwise_offsets_kernel", "dsa3d_pointwise_dz_kernel",
-      "dsa3d_pointwise_dw_kernel"};
+      "dsa3d_pointwise_dw_kernel", "dsa3d_sort_order_kernels", "dsa3d_fwd_tc_kernel"};
   return names[id];
 }
 

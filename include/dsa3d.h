@@ -76,6 +76,11 @@ const char *dsa3d_status_string(dsa3d_status_t status);
  * workspace).  Otherwise (no workspace, fp32, other shapes) it runs the general CUDA-core kernel;
  * both compute the same function.  A non-NULL workspace smaller than one head's need is
  * DSA3D_ERR_WORKSPACE_TOO_SMALL.  The backward needs lse; pass NULL only for inference.
+ * The workspace pair is an addition to the operator's plain signature (tensors, extents, window,
+ * dtype, stream): the library allocates no device memory, and the tensor-core path sorts the
+ * queries by window origin into caller-owned scratch.  A caller that cannot provide it passes
+ * NULL, 0 and gets the same results from the general kernel, several times slower on large
+ * problems (the sorted tensor-core forward is the fast path).
  */
 dsa3d_status_t dsa3d_forward(const void *q, const void *k, const void *v, const float *offsets,
                              void *out, float *lse, void *workspace, size_t workspace_bytes,
@@ -128,11 +133,14 @@ dsa3d_status_t dsa3d_backward(const void *q, const void *k, const void *v, const
  * which every GPU that loads the library holds until the process exits, passed to dsa3d_backward
  * as the workspace: the tensor-core path runs when one head's sort and stored splats fit it, the
  * general path when one head's fp32 dK/dV accumulators fit; heads are processed in groups that
- * fit.  A problem whose single head needs more than the array for the accumulators
- * (2 * N * dh * 4 bytes with bf16 I/O; fp32 I/O needs none) is rejected with
- * DSA3D_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ * fit.  A bf16 problem whose single head fits neither -- not the tensor-core path's workspace
+ * (dsa3d_backward_workspace_bytes with heads = 1, where that path applies) and not the fp32
+ * accumulators (2 * N * dh * 4 bytes) -- is rejected with DSA3D_ERR_WORKSPACE_TOO_SMALL before
+ * anything is launched; fp32 I/O needs no scratch.
  * The first call on each device looks up the array's device address (on the current device) and
- * caches it; make that first call before any stream capture.  The array is shared by every call
+ * caches it for the life of the process; make that first call before any stream capture.  The
+ * cached address belongs to the device's primary context (the one the CUDA runtime uses): after
+ * cudaDeviceReset, or under a different context, it is no longer valid.  The array is shared by every call
  * and keeps the previous call's contents (the accumulators are cleared before use): calls that
  * overlap on the GPU -- on different streams, or from different threads -- race on it.
  * The function calls no cudaMalloc, cudaFree or other allocating routine.

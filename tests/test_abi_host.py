@@ -73,6 +73,25 @@ def test_forward_rejects_bad_arguments():
     assert fwd(ws=P, wsb=need) == INV
 
 
+def test_forward_accepts_a_null_workspace():
+    """The forward's workspace is optional (a departure from the survey's workspace-free forward
+    signature, made because the library allocates nothing and the sort needs scratch): a NULL
+    workspace passes validation and runs the general CUDA-core kernels, a non-NULL one smaller than
+    one head's need is refused, and a large enough one selects the sorted tensor-core path.  Here,
+    without a GPU, a call that passes validation ends at the device with DSA3D_ERR_CUDA (the fake
+    pointers are never dereferenced); on a machine with a GPU the call would launch on them, so
+    the test does not run there."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("would launch kernels on fake device pointers")
+    assert fwd(ws=0, wsb=0) == 4          # validated, then no device: DSA3D_ERR_CUDA
+    assert fwd(ws=0, wsb=0, dtype=abi.DSA3D_F32) == 4
+    need = abi.dsa3d_forward_workspace_bytes(4, 8, 8, 1, 64, 3, 3, 3, abi.DSA3D_BF16)
+    assert need > 0
+    assert fwd(ws=P * 64, wsb=need - 16) == 3   # DSA3D_ERR_WORKSPACE_TOO_SMALL, before any launch
+    assert fwd(ws=P * 64, wsb=need) == 4        # the tensor-core path, then no device
+
+
 def test_forward_workspace_bytes():
     # the sort's arrays (buckets, then key, rank, sorted token and x-origin per query, then the
     # scan's block sums) and the paired value rows: F Hp ceil(Wp/2) pairs x heads x dh words

@@ -1,0 +1,83 @@
+"""Run-to-run determinism of the tensor-core path, and the sort's large-bucket ordering.
+
+The sort places the queries of one window-origin bucket in the order of its atomics and then
+sorts every bucket by token index, so the sorted arrays -- and with them the chunks, the tiles and
+the key side's summation order -- are the same in every run.  These tests run forward and backward
+twice on the same inputs and require bit-equal outputs, and check a degenerate offset field that
+sends every query of a head to one bucket (the shared-memory and merge paths of the large-bucket
+ordering) against the oracle.
+"""
+import pytest
+import torch
+
+import oracle
+from deformable_slide_attention_b200 import abi, inputs
+from tests.gpu_helpers import TOL, assert_close, f64, to_cuda
+
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gpu_lib", "oracle_lib")]
+
+
+def _run(d, dims, window):
+    out, lse = abi.forward(d["q"], d["k"], d["v"], d["offsets"], dims, window)
+    grads = abi.backward(d["q"], d["k"], d["v"], d["offsets"], lse, d["dout"], dims, window)
+    torch.cuda.synchronize()
+    return (out, lse) + tuple(grads)
+
+
+def _assert_bit_equal(a, b):
+    for name, x, y in zip(("out", "lse", "dq", "dk", "dv", "doffsets"), a, b):
+        assert torch.equal(x, y), f"{name} differs between two runs on the same inputs"
+
+
+@pytest.mark.parametrize("case", ["ragged", "720p-train-bf16"])
+def test_forward_backward_bit_equal_across_runs(case):
+    if case == "ragged":
+        dims, window = (5, 13, 21), (3, 5, 7)
+        _, inp = inputs.custom(*dims, 3, 64, window, "bf16", seed=77, scale=2.5)
+    else:
+        w = inputs.BY_NAME[case]
+        dims, window = w.dims, w.window
+        inp = inputs.make(w, "cpu", with_dout=True)
+    d = to_cuda(inp)
+    assert abi.dsa3d_forward_workspace_bytes(*dims, d["q"].shape[1], d["q"].shape[2], *window,
+                                             abi.DSA3D_BF16) > 0
+    first = _run(d, dims, window)
+    second = _run(d, dims, window)
+    _assert_bit_equal(first, second)
+
+
+def _one_origin_offsets(dims, heads, centre, frac):
+    """Offsets that send the window of every token p to the same place: delta = centre - p + frac,
+    so every query of a head has the same integer box origin (one bucket of N queries)."""
+    F, Hp, Wp = dims
+    t, y, x = torch.meshgrid(torch.arange(F), torch.arange(Hp), torch.arange(Wp), indexing="ij")
+    p = torch.stack([t, y, x], -1).reshape(-1, 3).float()
+    c = torch.tensor(centre, dtype=torch.float32) + torch.tensor(frac, dtype=torch.float32)
+    return (c - p).unsqueeze(0).expand(heads, -1, -1).contiguous()
+
+
+@pytest.mark.parametrize("dims", [(4, 12, 20), (8, 32, 40)])
+def test_one_bucket_for_every_query(dims):
+    # 960 queries per bucket (shared-memory sort of one chunk) and 10,240 (three chunks, merged)
+    heads, dh, window = 2, 64, (3, 3, 3)
+    _, inp = inputs.custom(*dims, heads, dh, window, "bf16", seed=88, scale=2.0)
+    centre = (dims[0] // 2, dims[1] // 2, dims[2] // 2)
+    inp["offsets"] = _one_origin_offsets(dims, heads, centre, (0.25, 0.5, 0.75))
+    d = to_cuda(inp)
+    first = _run(d, dims, window)
+    _assert_bit_equal(first, _run(d, dims, window))
+    out, lse, dq, dk, dv, doff = first
+    r_out, r_lse = oracle.full_forward(inp["q"], inp["k"], inp["v"], inp["offsets"], dims, window)
+    r_dq, r_doff, r_dk, r_dv = oracle.full_backward(inp["q"], inp["k"], inp["v"], inp["offsets"],
+                                                    inp["dout"], dims, window)
+    tol = TOL["bf16"]
+    assert_close("out", f64(out), r_out, tol)
+    assert_close("lse", f64(lse), r_lse, tol)
+    assert_close("dq", f64(dq), r_dq, tol)
+    assert_close("doffsets", f64(doff), r_doff, tol)
+    # every query adds into the same 4 x 4 x 4 keys, so dK and dV grow with N; their bf16
+    # rounding (2^-8 relative) then dominates the absolute bar
+    for name, got, ref in (("dk", dk, r_dk), ("dv", dv, r_dv)):
+        g, r = f64(got), ref
+        bound = tol + 2.0 ** -8 * abs(r)
+        assert (abs(g - r) <= bound).all(), f"{name}: max-abs error {abs(g - r).max():.3e}"

@@ -32,8 +32,12 @@ def _noalloc(d, lse, dims, window, dtype_code):
 
 
 @pytest.mark.parametrize("dims,heads,dh,window", [
-    ((16, 32, 32), 8, 64, (3, 7, 7)),    # all heads in one pass of the fixed scratch
-    ((16, 64, 64), 2, 128, (3, 5, 5)),   # one head fills the scratch: two passes
+    ((16, 32, 32), 8, 64, (3, 7, 7)),    # tensor-core path, all heads in one pass of the scratch
+    ((16, 64, 64), 2, 128, (3, 5, 5)),   # tensor-core path, both heads in one pass (~58 MiB)
+    ((32, 45, 80), 2, 128, (3, 3, 3)),   # tensor-core path: one head's sort and splats (~26 MB)
+                                         # fit, although its fp32 accumulators (118 MB) would not
+    ((16, 96, 96), 2, 32, (3, 3, 3)),    # dh 32: the general path; one head's accumulators
+                                         # (37.7 MB) fit, two do not: two passes of the scratch
 ])
 def test_noalloc_matches_workspace_backward_twice(dims, heads, dh, window):
     _, inp = inputs.custom(*dims, heads, dh, window, "bf16", seed=41, scale=2.0)
@@ -49,9 +53,12 @@ def test_noalloc_matches_workspace_backward_twice(dims, heads, dh, window):
 
 
 def test_noalloc_refuses_problem_larger_than_its_scratch():
-    dims, heads, dh, window = (32, 45, 80), 2, 128, (3, 3, 3)  # one head needs 118 MB > 64 MiB
+    # 720p at dh 128 with a 3x9x9 window: one head's stored splats alone take 138 MB and its fp32
+    # accumulators 118 MB, so neither path fits the 64 MiB scratch
+    dims, heads, dh, window = (32, 45, 80), 2, 128, (3, 9, 9)
     N = dims[0] * dims[1] * dims[2]
     assert 2 * N * dh * 4 > (64 << 20)
+    assert abi.dsa3d_backward_workspace_bytes(*dims, 1, dh, *window, abi.DSA3D_BF16) > (64 << 20)
     t = torch.zeros(16, dtype=torch.uint8, device="cuda")  # never dereferenced: refused on the host
     p = t.data_ptr()
     st = abi.dsa3d_backward_noalloc(p, p + 1024, p + 2048, p + 3072, p + 4096, p + 5120, p + 6144,
