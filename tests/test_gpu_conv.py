@@ -83,7 +83,7 @@ def test_offset_network_forward(per_tap, dtype):
     """dsa3d_offset_head against oracle.offset_head (relative 1e-4: fp32 throughout), and the
     offsets it writes drive the attention exactly as the same offsets given by hand."""
     td = torch.float32 if dtype == "f32" else torch.bfloat16
-    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    dims, heads, dh, window = (3, 5, 9), 2, 32, (3, 3, 3)  # dh 32: the smallest the attention takes
     C, N, K = heads * dh, math.prod(dims), math.prod(window)
     g = torch.Generator().manual_seed(77 + int(per_tap))
     x = torch.randn(N, C, generator=g).to(td)
@@ -110,7 +110,7 @@ def test_offset_network_backward(per_tap, dtype):
     """dsa3d_offset_head_backward against oracle.offset_head_backward: dx (the I/O tolerance) and
     the fp32 weight gradients (relative 1e-4)."""
     td = torch.float32 if dtype == "f32" else torch.bfloat16
-    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    dims, heads, dh, window = (3, 5, 9), 2, 32, (3, 3, 3)  # dh 32: the smallest the attention takes
     C, N, K = heads * dh, math.prod(dims), math.prod(window)
     g = torch.Generator().manual_seed(91 + int(per_tap))
     x = torch.randn(N, C, generator=g).to(td)
@@ -135,7 +135,7 @@ def test_layer_against_the_oracle_chain(dtype):
     floor decision near an integer cannot differ between the two)."""
     from deformable_slide_attention_b200 import layer
     td = torch.float32 if dtype == "f32" else torch.bfloat16
-    dims, heads, dh, window = (3, 5, 9), 2, 16, (3, 3, 3)
+    dims, heads, dh, window = (3, 5, 9), 2, 32, (3, 3, 3)  # dh 32: the smallest the attention takes
     C, N, K = heads * dh, math.prod(dims), math.prod(window)
     g = torch.Generator().manual_seed(123)
     x = torch.randn(N, C, generator=g).to(td)
