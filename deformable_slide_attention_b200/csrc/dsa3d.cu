@@ -2,8 +2,10 @@
 // extern "C" entry points declared in include/dsa3d.h.  All device work is in the kernels of
 // dsa3d_*.cuh headers; this file allocates no device memory.
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -13,6 +15,7 @@
 #include "dsa3d_bwd_mma.cuh"
 #include "dsa3d_fwd.cuh"
 #include "dsa3d_fwd_mma.cuh"
+#include "dsa3d_fwd_tc.cuh"
 #include "dsa3d_sort.cuh"
 #include "dsa3d_taps.cuh"
 #include "dsa3d_timing.cuh"
@@ -365,6 +368,88 @@ dsa3d_status_t fwd_mma_group(const Shape& s, const void* q, const void* k, const
   return DSA3D_OK;
 }
 
+// --- tcgen05 forward ---------------------------------------------------------------------------
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to the driver library).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a [T][H'][W'][heads][dh] bf16 tensor (k or v) viewed as the 5-D
+// (8 dims, x, y, t, heads * dh / 8 dim groups), box (8, 32 keys, 1 row, 2 planes, dh / 8): one TMA
+// copy brings a K or V "pair" (one row, two planes, 32 keys, one head's dims) into the layout the
+// tcgen05 forward's UMMAs read (dsa3d_fwd_tc.cuh).
+bool make_pair_map(CUtensorMap* m, const void* base, const Shape& s) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t row = (cuuint64_t)s.heads * s.dh * 2;  // bytes per token
+  const cuuint64_t dims[5] = {8, (cuuint64_t)s.Wp, (cuuint64_t)s.Hp, (cuuint64_t)s.F,
+                              (cuuint64_t)s.heads * s.dh / 8};
+  const cuuint64_t strides[4] = {row, row * s.Wp, row * s.Wp * s.Hp, 16};
+  const cuuint32_t box[5] = {8, (cuuint32_t)kTcSeg, 1, 2, (cuuint32_t)s.dh / 8};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Bucket rows per tile: about 96 queries per tile at the volume's average density (one query
+// per bucket, spread over (F+kt)(H'+kh)(W'+kw) buckets), 1..kTcRyMax; DSA3D_TC_RY overrides it.
+TcTileGeo make_tile_geo(const Shape& s, int hg) {
+  const SortGeo sg = make_sort_geo(s);
+  TcTileGeo tg;
+  tg.Wx = kTcSeg - s.kw;
+  const double dens = (double)s.N / ((double)sg.Et * sg.Ey * sg.Ex);
+  int ry = (int)std::lround(96.0 / (dens * tg.Wx));
+  if (const char* e = std::getenv("DSA3D_TC_RY")) ry = std::atoi(e);
+  tg.Ry = ry < 1 ? 1 : (ry > kTcRyMax ? kTcRyMax : ry);
+  tg.nYb = (sg.Ey + tg.Ry - 1) / tg.Ry;
+  tg.nXb = (sg.Ex + tg.Wx - 1) / tg.Wx;
+  tg.tiles = (int64_t)hg * sg.Et * tg.nYb * tg.nXb;
+  return tg;
+}
+
+// The tcgen05 forward runs unless DSA3D_FWD_KERNEL=mma selects the mma.sync forward.
+bool use_tc_forward() {
+  const char* e = std::getenv("DSA3D_FWD_KERNEL");
+  return !(e && std::strcmp(e, "mma") == 0);
+}
+
+template <int DH>
+dsa3d_status_t fwd_tc_group(const Shape& s, const void* q, const void* k, const void* v,
+                            const float* off, void* out, float* lse, const SortWs& w, int h0, int hg,
+                            cudaStream_t st) {
+  using C = FwdTcCfg<DH>;
+  const Geo g = make_geo(s);
+  const SortGeo sg = make_sort_geo(s);
+  CUtensorMap tmk, tmv;
+  if (!make_pair_map(&tmk, k, s) || !make_pair_map(&tmv, v, s)) return DSA3D_ERR_CUDA;
+  dsa3d_status_t rc = sort_queries<DH>(s, off, w, h0, hg, static_cast<__nv_bfloat16*>(out), lse, nullptr, st);
+  if (rc != DSA3D_OK) return rc;
+  const TcTileGeo tg = make_tile_geo(s, hg);
+  auto kern = dsa3d_fwd_tc_kernel<DH>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return DSA3D_ERR_CUDA;
+  const DeviceInfo d = device_info();
+  int64_t grid = d.sms;
+  if (grid > tg.tiles) grid = tg.tiles;
+  if (grid < 1) grid = 1;
+  TimedLaunch tl(kKernFwdTc, st);
+  kern<<<(int)grid, kTcThreads, C::SMEM_BYTES, st>>>(tmk, tmv, static_cast<const __nv_bfloat16*>(q), off,
+                                                     static_cast<__nv_bfloat16*>(out), lse, w.cnt, w.sorted_n,
+                                                     w.sorted_ex, g, sg, tg, h0);
+  if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  return DSA3D_OK;
+}
+
 struct BwdArgs {
   const void *q, *k, *v, *dout;
   const float *off, *lse;
@@ -672,9 +757,13 @@ dsa3d_status_t dsa3d_forward(const void* q, const void* k, const void* v, const 
       const int n = (heads - h0 < hg) ? heads - h0 : hg;
       const SortWs wn = carve_sort_ws(s, n, workspace);
       unsigned* vp = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + sort_ws_bytes(s, n));
-      const dsa3d_status_t r =
-          (dh == 128) ? fwd_mma_group<128>(s, q, k, v, offsets, out, lse, wn, vp, h0, n, stream)
-                      : fwd_mma_group<64>(s, q, k, v, offsets, out, lse, wn, vp, h0, n, stream);
+      dsa3d_status_t r;
+      if (use_tc_forward())
+        r = (dh == 128) ? fwd_tc_group<128>(s, q, k, v, offsets, out, lse, wn, h0, n, stream)
+                        : fwd_tc_group<64>(s, q, k, v, offsets, out, lse, wn, h0, n, stream);
+      else
+        r = (dh == 128) ? fwd_mma_group<128>(s, q, k, v, offsets, out, lse, wn, vp, h0, n, stream)
+                        : fwd_mma_group<64>(s, q, k, v, offsets, out, lse, wn, vp, h0, n, stream);
       if (r != DSA3D_OK) return r;
     }
     return DSA3D_OK;
@@ -882,6 +971,12 @@ int dsa3d_timing_read(dsa3d_kernel_time_t* out, int max_entries) {
 }
 
 void dsa3d_timing_reset(void) { Timing::get().reset(); }
+
+#ifdef DSA3D_TC_TRACE
+int dsa3d_tc_trace_read(float* host, int n) {
+  return cudaMemcpyFromSymbol(host, g_tc_trace, (size_t)n * sizeof(float)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 dsa3d_status_t dsa3d_check_device(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return DSA3D_ERR_CUDA;
