@@ -384,20 +384,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Tensor map over a [T][H'][W'][heads][dh] bf16 tensor (k or v) viewed as the 5-D
-// (8 dims, x, y, t, heads * dh / 8 dim groups), box (8, 32 keys, 1 row, 2 planes, dh / 8): one TMA
-// copy brings a K or V "pair" (one row, two planes, 32 keys, one head's dims) into the layout the
-// tcgen05 forward's UMMAs read (dsa3d_fwd_tc.cuh).
+// (64 dims, heads * dh / 64 head halves, x, y, t), box (64, 1, 32 keys, 1 row, 2 planes) with the
+// 128-byte swizzle: one TMA copy per 64 dims brings half of a K or V "pair" (one row, two planes,
+// 32 keys) into the layout the tcgen05 forward's UMMAs read (dsa3d_fwd_tc.cuh).
 bool make_pair_map(CUtensorMap* m, const void* base, const Shape& s) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t row = (cuuint64_t)s.heads * s.dh * 2;  // bytes per token
-  const cuuint64_t dims[5] = {8, (cuuint64_t)s.Wp, (cuuint64_t)s.Hp, (cuuint64_t)s.F,
-                              (cuuint64_t)s.heads * s.dh / 8};
-  const cuuint64_t strides[4] = {row, row * s.Wp, row * s.Wp * s.Hp, 16};
-  const cuuint32_t box[5] = {8, (cuuint32_t)kTcSeg, 1, 2, (cuuint32_t)s.dh / 8};
+  const cuuint64_t dims[5] = {64, (cuuint64_t)s.heads * s.dh / 64, (cuuint64_t)s.Wp, (cuuint64_t)s.Hp,
+                              (cuuint64_t)s.F};
+  const cuuint64_t strides[4] = {128, row, row * s.Wp, row * s.Wp * s.Hp};
+  const cuuint32_t box[5] = {64, 1, (cuuint32_t)kTcSeg, 1, 2};
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -975,6 +975,9 @@ void dsa3d_timing_reset(void) { Timing::get().reset(); }
 #ifdef DSA3D_TC_TRACE
 int dsa3d_tc_trace_read(float* host, int n) {
   return cudaMemcpyFromSymbol(host, g_tc_trace, (size_t)n * sizeof(float)) == cudaSuccess ? 0 : 1;
+}
+int dsa3d_tc_clk_read(unsigned* host, int n) {
+  return cudaMemcpyFromSymbol(host, g_tc_clk, (size_t)n * sizeof(unsigned)) == cudaSuccess ? 0 : 1;
 }
 #endif
 

@@ -26,13 +26,14 @@
 // share the max in use).  At the end of a pass each thread divides its row of O by the softmax
 // sum and writes out and lse.
 //
-// Roles (192 threads): warps 0-3 the epilogue (tensor-memory lane quarter w), warp 4 the TMA
-// producer (one lane), warp 5 the UMMA issuer (one lane; the warp also allocates tensor memory).
+// Roles (256 threads): warps 0-3 the epilogue (tensor-memory lane quarter w), warps 4 and 6 the TMA
+// producers of K and of V, warp 5 the UMMA issuer of the raw dots (the warp also allocates tensor
+// memory), warp 7 the UMMA issuer of the value products (one lane each).
 // Rings of shared-memory stages hold K and V "pairs" (one union row, two planes, 32 keys, dh):
-// a 5-D box (8 dims, 32 keys, 1 row, 2 planes, dh/8 dim groups) of the tensor map over
-// [T][H'][W'][heads * dh / 8][8], so the stage is [dim group][plane][key][8 dims] -- the no-swizzle
-// core-matrix layout the UMMA reads as K-major B (keys = N) for S and as MN-major B (dims = N,
-// keys = K) for P.V.  Out-of-volume keys, rows and planes read as zero.
+// per 64 dims, a 5-D box (64 dims, 1 head half, 32 keys, 1 row, 2 planes) of the tensor map over
+// [T][H'][W'][heads * dh / 64][64] with the 128-byte swizzle, so each half is 64 rows (plane-major
+// keys) of 128 bytes -- the layout the UMMA reads as K-major B (keys = N) for the dots and as
+// MN-major B (dims = N, keys = K) for P.V.  Out-of-volume keys, rows and planes read as zero.
 // mbarriers order everything; every wait is bounded (dsa3d_tc.cuh).
 #pragma once
 
@@ -42,7 +43,8 @@
 
 namespace dsa3d {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 256;  // 4 epilogue warps, K producer, dots issuer, V producer, P.V issuer
+constexpr int kTcKWarp = 4, kTcMmaWarp = 5, kTcVWarp = 6, kTcPvWarp = 7;
 constexpr int kTcSeg = 32;         // keys per segment
 constexpr int kTcRyMax = 8;        // bucket rows per tile (Ry <= kTcRyMax)
 constexpr int kTcKStages = 4;      // K pair ring
@@ -51,7 +53,7 @@ constexpr float kTcRescale = 8.f;  // lazy-rescale threshold (base-2 units)
 
 template <int DH>
 struct FwdTcCfg {
-  static constexpr int DG = DH / 8;                       // 16-byte dim groups per row
+  static constexpr int HALVES = DH / 64;                  // 128-byte row halves of a key
   static constexpr int PAIR_BYTES = 2 * kTcSeg * DH * 2;  // two planes x 32 keys x dh bf16
   static constexpr int KSTEPS = DH / 16;                  // UMMA K-steps of S
   static constexpr int A_COLS = DH / 2;                   // the query tile (bf16 pairs)
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto p_full = [&](int s) { return bx + 8u * (4 + s); };
   auto p_empty = [&](int s) { return bx + 8u * (6 + s); };
   const uint32_t a_full = bx + 8u * 8, o_full = bx + 8u * 9, o_empty = bx + 8u * 10;
-  const uint32_t m_done = bx + 8u * 11;  // the UMMA issuer's own exit drain
+  const uint32_t m_done = bx + 8u * 11, m_done2 = bx + 8u * 12;  // the UMMA issuers' own exit drains
   uint32_t* tslot = reinterpret_cast<uint32_t*>(stages + C::STAGE_BYTES + 8 * 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
 
@@ -158,30 +160,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(o_full, 1);
     mbar_init(o_empty, 4);
     mbar_init(m_done, 1);
+    mbar_init(m_done2, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 5) tmem_alloc(smem_u32(tslot), C::COLS);
+  if (warp == kTcMmaWarp) tmem_alloc(smem_u32(tslot), C::COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const int U = g.kh + tg.Ry;  // union rows per tile
 
-  if (warp == 4) {
-    // ===================== TMA producer =====================
+  if (warp == kTcKWarp || warp == kTcVWarp) {
+    // ===================== TMA producers: K pairs (warp kTcKWarp) and V pairs (warp kTcVWarp) ==
+    // Each ring has its own thread, so that neither waits behind the other's free slots.
     if (lane == 0) {
-      tma_prefetch_desc(&tmk);
-      tma_prefetch_desc(&tmv);
-      uint32_t kc = 0, vc = 0;
+      const bool is_k = warp == kTcKWarp;
+      const CUtensorMap* tm = is_k ? &tmk : &tmv;
+      const int nst = is_k ? kTcKStages : kTcVStages;
+      const uint32_t base = is_k ? kst : vst;
+      tma_prefetch_desc(tm);
+      uint32_t cnt = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* tm, uint32_t base, int stages_n, uint32_t& cnt, bool is_k, int t0,
-                      int y, int X, int hd) {
-        const int s = (int)(cnt % stages_n);
+      auto load = [&](int t0, int y, int X, int hd) {
+        const int s = (int)(cnt % nst);
         const uint32_t full = is_k ? k_full(s) : v_full(s), empty = is_k ? k_empty(s) : v_empty(s);
-        if (cnt >= (uint32_t)stages_n && !mbar_wait(empty, ((cnt / stages_n) - 1) & 1, abort_flag)) return false;
+        if (cnt >= (uint32_t)nst && !mbar_wait(empty, ((cnt / nst) - 1) & 1, abort_flag)) return false;
         mbar_arrive_expect_tx(full, C::PAIR_BYTES);
-        tma_load_5d(base + s * C::PAIR_BYTES, tm, full, 0, X, y, t0, hd);
+#pragma unroll
+        for (int hv = 0; hv < C::HALVES; hv++)
+          tma_load_5d(base + s * C::PAIR_BYTES + hv * (C::PAIR_BYTES / C::HALVES), tm, full, 0, hd + hv, X, y, t0);
         cnt++;
         return true;
       };
@@ -189,30 +197,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         TcTile T;
         tc_tile(tg, sg, start, t, T);
         const int passes = (T.cnt + 127) / 128;
-        const int ot = T.et - g.kt, Xs = T.X0 - g.kw, hd = (h0 + T.hh) * C::DG;
+        const int ot = T.et - g.kt, Xs = T.X0 - g.kw, hd = (h0 + T.hh) * C::HALVES;
+        // per tap plane u: the pairs (planes u, u+1) of union rows 0 .. U-1, in the order of use
         for (int ps = 0; ps < passes && ok; ps++)
-          for (int u = 0; u < g.kt && ok; u++) {
-            for (int j = 0; j < U && ok; j++) {
-              const int y = T.Y0 - g.kh + j;
-              ok = load(&tmk, kst, kTcKStages, kc, true, ot + u, y, Xs, hd);
-              if (ok && j >= 1) ok = load(&tmv, vst, kTcVStages, vc, false, ot + u, y - 1, Xs, hd);
-            }
-            if (ok) ok = load(&tmv, vst, kTcVStages, vc, false, ot + u, T.Y0 - g.kh + U - 1, Xs, hd);
-          }
+          for (int u = 0; u < g.kt && ok; u++)
+            for (int j = 0; j < U && ok; j++) ok = load(ot + u, T.Y0 - g.kh + j, Xs, hd);
       }
       // every issued copy has landed before the CTA can exit (bounded; the last copy of each
       // stage completes its phase last)
-      for (uint32_t i = (kc > kTcKStages ? kc - kTcKStages : 0); i < kc; i++)
-        mbar_drain(k_full(i % kTcKStages), (i / kTcKStages) & 1, abort_flag);
-      for (uint32_t i = (vc > kTcVStages ? vc - kTcVStages : 0); i < vc; i++)
-        mbar_drain(v_full(i % kTcVStages), (i / kTcVStages) & 1, abort_flag);
+      for (uint32_t i = (cnt > (uint32_t)nst ? cnt - nst : 0); i < cnt; i++)
+        mbar_drain(is_k ? k_full(i % nst) : v_full(i % nst), (i / nst) & 1, abort_flag);
     }
-  } else if (warp == 5) {
-    // ===================== UMMA issuer =====================
+  } else if (warp == kTcMmaWarp) {
+    // ===================== UMMA issuer of the raw dots =====================
+    // Raw dots of union row j, planes u and u+1 (K pair (u, j), released when done), into the
+    // S buffer j % 2 once the epilogue has read the row two back.
     if (lane == 0) {
-      uint32_t kc = 0, kwaited = 0, vc = 0, sc = 0, pc = 0, npass = 0;
+      uint32_t kc = 0, sc = 0, npass = 0;
       bool ok = true;
-      const uint32_t tA = tmem + C::COL_A, tS = tmem + C::COL_S, tP = tmem + C::COL_P, tO = tmem + C::COL_O;
+      const uint32_t tA = tmem + C::COL_A, tS = tmem + C::COL_S;
+      const uint64_t kd0 = umma_sdesc_sw128(kst, 16, 1024);
       for (int64_t t = blockIdx.x; t < tg.tiles && ok; t += gridDim.x) {
         TcTile T;
         tc_tile(tg, sg, start, t, T);
@@ -220,72 +224,76 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int ps = 0; ps < passes && ok; ps++, npass++) {
           ok = mbar_wait(a_full, npass & 1, abort_flag);
           if (!ok) break;
-          tc_fence_after();
-          const uint32_t kbase = kc;  // K pair (u, j) of this pass is kbase + u U + j
-          bool first_pv = true;
-          // raw dots of union row j, planes u and u+1: K pair (u, j), released when done
-          auto issue_s = [&](int u, int j) {
-            const uint32_t p0 = kbase + u * U + j;
-            while (kwaited <= p0) {
-              if (!mbar_wait(k_full(kwaited % kTcKStages), (kwaited / kTcKStages) & 1, abort_flag)) return false;
-              kwaited++;
+          const int rows = g.kt * U;
+          for (int r = 0; r < rows && ok; r++, kc++, sc++) {
+            const int ks_ = (int)(kc % kTcKStages), sb = (int)(sc & 1);
+            if (!mbar_wait(k_full(ks_), (kc / kTcKStages) & 1, abort_flag) ||
+                (sc >= 2 && !mbar_wait(s_empty(sb), ((sc - 2) >> 1) & 1, abort_flag))) {
+              ok = false;
+              break;
             }
-            const int sb = (int)(sc & 1);
-            if (sc >= 2 && !mbar_wait(s_empty(sb), ((sc - 2) >> 1) & 1, abort_flag)) return false;
             tc_fence_after();
-            const uint32_t kp = kst + (p0 % kTcKStages) * C::PAIR_BYTES;
+            // B, K-major: 64 keys (plane 0 then plane 1) = 64 rows of 128 bytes per 64-dim half;
+            // dims 16 ks .. 16 ks + 15 are 32 bytes into the rows of half ks / 4.  The descriptors
+            // differ only in their start address (bits 0-13, 16-byte units): constant adds.
+            const uint64_t bd0 = kd0 + (uint64_t)((ks_ * C::PAIR_BYTES) >> 4);
+            const uint32_t d = tS + sb * 64;
+            umma_ts_c<false>(d, tA, bd0, C::IDESC_S);
 #pragma unroll
-            for (int ks = 0; ks < C::KSTEPS; ks++) {
-              // B: 64 keys (plane 0 then plane 1, 8-key core matrices 128 bytes apart) x dims
-              // 16 ks .. 16 ks + 15 (two dim groups, 1024 bytes apart)
-              const uint64_t bd = umma_sdesc(kp + ks * 2 * (2 * kTcSeg * 16), 2 * kTcSeg * 16, 128);
-              umma_ts(tS + sb * 64, tA + ks * 8, bd, C::IDESC_S, ks ? 1u : 0u);
-            }
+            for (int ks = 1; ks < C::KSTEPS; ks++)
+              umma_ts_c<true>(d, tA + ks * 8, bd0 + (uint64_t)(((ks >> 2) * (C::PAIR_BYTES / C::HALVES) + (ks & 3) * 32) >> 4),
+                              C::IDESC_S);
             umma_commit(s_full(sb));
-            umma_commit(k_empty(p0 % kTcKStages));
-            sc++;
-            return true;
-          };
-          // O += [beta_a | beta_b] . [V[u, j]; V[u+1, j]]
-          auto issue_pv = [&](int u, int j) {
-            (void)u;
-            (void)j;
-            const int pb = (int)(pc & 1);
-            if (!mbar_wait(p_full(pb), (pc >> 1) & 1, abort_flag)) return false;
-            if (!mbar_wait(v_full(vc % kTcVStages), (vc / kTcVStages) & 1, abort_flag)) return false;
-            if (first_pv && npass > 0 && !mbar_wait(o_empty, (npass - 1) & 1, abort_flag)) return false;
+            umma_commit(k_empty(ks_));
+          }
+        }
+      }
+      // nothing of this thread's may still run when tensor memory is released
+      umma_commit(m_done);
+      mbar_drain(m_done, 0, abort_flag);
+    }
+  } else if (warp == kTcPvWarp) {
+    // ===================== UMMA issuer of the value products =====================
+    // O += [beta_a | beta_b] . [V[u, j]; V[u+1, j]] once the epilogue has written box row j's
+    // weights; the first product of a pass overwrites O (after the epilogue read the previous
+    // pass's), the last one signals o_full.
+    if (lane == 0) {
+      uint32_t vc = 0, pc = 0, npass = 0;
+      bool ok = true;
+      const uint32_t tP = tmem + C::COL_P, tO = tmem + C::COL_O;
+      const uint64_t vd0 = umma_sdesc_sw128(vst, C::PAIR_BYTES / C::HALVES, 1024);
+      for (int64_t t = blockIdx.x; t < tg.tiles && ok; t += gridDim.x) {
+        TcTile T;
+        tc_tile(tg, sg, start, t, T);
+        const int passes = (T.cnt + 127) / 128;
+        for (int ps = 0; ps < passes && ok; ps++, npass++) {
+          const int rows = g.kt * U;
+          for (int r = 0; r < rows && ok; r++, vc++, pc++) {
+            const int pb = (int)(pc & 1), vs = (int)(vc % kTcVStages);
+            if (!mbar_wait(p_full(pb), (pc >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(v_full(vs), (vc / kTcVStages) & 1, abort_flag) ||
+                (r == 0 && npass > 0 && !mbar_wait(o_empty, (npass - 1) & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
-            const uint32_t vp = vst + (vc % kTcVStages) * C::PAIR_BYTES;
+            // B, MN-major: keys 16 ks .. 16 ks + 15 are rows 16 ks ..; 64-dim halves apart by
+            // PAIR_BYTES / HALVES
+            const uint64_t bd0 = vd0 + (uint64_t)((vs * C::PAIR_BYTES) >> 4);
+            const uint32_t a = tP + pb * 32;
+            umma_ts(tO, a, bd0, C::IDESC_PV, r == 0 ? 0u : 1u);
 #pragma unroll
-            for (int ks = 0; ks < 4; ks++) {
-              const uint64_t bd = umma_sdesc(vp + ks * 256, 128, 2 * kTcSeg * 16);
-              umma_ts(tO, tP + pb * 32 + ks * 8, bd, C::IDESC_PV, (first_pv && ks == 0) ? 0u : 1u);
-            }
+            for (int ks = 1; ks < 4; ks++) umma_ts_c<true>(tO, a + ks * 8, bd0 + (uint64_t)((ks * 2048) >> 4), C::IDESC_PV);
             umma_commit(p_empty(pb));
-            umma_commit(v_empty(vc % kTcVStages));
-            vc++;
-            pc++;
-            first_pv = false;
-            return true;
-          };
-          // the raw dots run two rows ahead of the value products: box row j's weights need
-          // rows j and j+1
-          for (int u = 0; u < g.kt && ok; u++) {
-            ok = issue_s(u, 0);
-            if (ok && U > 1) ok = issue_s(u, 1);
-            for (int j = 0; j < U && ok; j++) {
-              if (j + 2 < U) ok = issue_s(u, j + 2);
-              if (ok) ok = issue_pv(u, j);
-            }
+            umma_commit(v_empty(vs));
           }
           if (ok) umma_commit(o_full);
-          kc = kbase + g.kt * U;
         }
       }
       // nothing of this thread's may still run when tensor memory is released (a barrier of its
       // own: a further phase of o_full could be mistaken by an epilogue warp still waiting on it)
-      umma_commit(m_done);
-      mbar_drain(m_done, 0, abort_flag);
+      umma_commit(m_done2);
+      mbar_drain(m_done2, 0, abort_flag);
     }
   } else {
     // ===================== epilogue: thread = tensor-memory lane = query of the pass =====================
@@ -402,9 +410,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               for (int c = 0; c < 31; c++) {
                 const float sv = fmaf(fx, yb[c + 1] - yb[c], yb[c]) * sc2;
                 p[c] = (c >= cmin && c <= cmax) ? sv : -INFINITY;
-                mx = fmaxf(mx, p[c]);
               }
               p[31] = -INFINITY;
+              float m16[16];
+#pragma unroll
+              for (int c = 0; c < 16; c++) m16[c] = fmaxf(p[c], p[c + 16]);
+#pragma unroll
+              for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; c++) m16[c] = fmaxf(m16[c], m16[c + w]);
+              mx = m16[0];
             } else {
 #pragma unroll
               for (int c = 0; c < 32; c++) p[c] = -INFINITY;
@@ -446,13 +461,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             // P, its sum, the x-splat, and the value weights of box row j-1
             const float mu = (m_used == -INFINITY) ? 0.f : m_used;  // no valid tap yet: every p is 0
-            float ls = 0.f;
 #pragma unroll
-            for (int c = 0; c < 32; c++) {
-              p[c] = ex2_approx(p[c] - mu);  // -inf -> 0
-              ls += p[c];
+            for (int c = 0; c < 32; c++) p[c] = ex2_approx(p[c] - mu);  // -inf -> 0
+            {
+              float s16[16];
+#pragma unroll
+              for (int c = 0; c < 16; c++) s16[c] = p[c] + p[c + 16];
+#pragma unroll
+              for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; c++) s16[c] += s16[c + w];
+              l += s16[0];
             }
-            l += ls;
             uint32_t pw[32];
             float prev = 0.f;
 #pragma unroll
@@ -518,7 +538,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // release tensor memory once no role can touch it
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kTcMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, C::COLS);
   }
