@@ -73,15 +73,21 @@ def parse_args(argv=None):
 # kernels' traffic grows in proportion to the items).
 TENSOR_CORE_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_fwd_mma.cuh", "dsa3d_bwd_mma.cuh",
                      "dsa3d_sort.cuh"]
+TC_FORWARD_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_tc.cuh", "dsa3d_fwd_tc.cuh",
+                    "dsa3d_sort.cuh", "dsa3d_bwd_mma.cuh", "dsa3d_fwd_mma.cuh"]
 PER_TAP_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_taps.cuh", "dsa3d_bwd.cuh", "dsa3d_fwd.cuh"]
 NCU_TRAFFIC = [
-    {"files": TENSOR_CORE_FILES, "sources": "8eaed48778e074f4",
+    {"files": TENSOR_CORE_FILES, "sources": "f439b4ef408f12c1",
      "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
      "bytes_per_item": {
-         "dsa3d_fwd_mma_kernel": 1084.2,
-         "dsa3d_bwd_q_kernel": 2254.5,
-         "dsa3d_bwd_dq_kernel": 1650.5,
-         "dsa3d_bwd_kv_kernel": 2206.3,
+         "dsa3d_bwd_q_kernel": 2257.4,
+         "dsa3d_bwd_dq_kernel": 1649.9,
+         "dsa3d_bwd_kv_kernel": 2211.1,
+     }},
+    {"files": TC_FORWARD_FILES, "sources": "5401473b888b9a33",
+     "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
+     "bytes_per_item": {
+         "dsa3d_fwd_tc_kernel": 1552.3,
      }},
     {"files": PER_TAP_FILES, "sources": "df10cf32e12d6270",
      "capture": "profiles/per_tap_kernels_720p-train-taps-bf16.md",
@@ -145,6 +151,7 @@ def alg_bytes_per_item(w, kernel):
     table = {
         "dsa3d_fwd_kernel": 4 * w.dh * s + 16,        # q, k, v -> out; offsets, lse
         "dsa3d_fwd_mma_kernel": 4 * w.dh * s + 16,
+        "dsa3d_fwd_tc_kernel": 4 * w.dh * s + 16,
         "dsa3d_bwd_kernel": 8 * w.dh * s + 28,        # the CUDA-core backward does it all
         "dsa3d_bwd_q_kernel": 4 * w.dh * s + 28,      # q, k, v, dO; offsets, lse -> doffsets
         "dsa3d_bwd_dq_kernel": 2 * w.dh * s,          # k -> dq
@@ -165,7 +172,7 @@ def alg_flop_per_item(w, kernel):
         return {"dsa3d_fwd_taps_kernel": 36, "dsa3d_bwd_taps_kernel": 64,
                 "fwd": 36, "bwd": 64}.get(kernel, 0) * w.dh * w.K
     B = (w.window[0] + 1) * (w.window[1] + 1) * (w.window[2] + 1)
-    per = {"dsa3d_fwd_kernel": 4, "dsa3d_fwd_mma_kernel": 4, "dsa3d_bwd_kernel": 10,
+    per = {"dsa3d_fwd_kernel": 4, "dsa3d_fwd_mma_kernel": 4, "dsa3d_fwd_tc_kernel": 4, "dsa3d_bwd_kernel": 10,
            "dsa3d_bwd_q_kernel": 4, "dsa3d_bwd_dq_kernel": 2, "dsa3d_bwd_kv_kernel": 4,
            "fwd": 4, "bwd": 10}
     return per.get(kernel, 0) * w.dh * B
@@ -566,11 +573,17 @@ def main(argv=None):
 
 
 def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
-    """Same step through the public API with pinned host inputs and results: every step copies
-    the inputs host->device and reads back every output (out, lse, dq, dk, dv, doffsets)."""
+    """Same step through the public API with host inputs and results: every step copies the
+    inputs host->device from pinned buffers and reads every output (out, lse, dq, dk, dv,
+    doffsets) back device->host.  The inputs of step i+1 cross on their own stream while the
+    outputs of step i come back on a third one (the two directions of the link overlap); compute
+    waits for its inputs and for the previous read-back (the device output buffers are reused).
+    Host RAM holds the pinned inputs and a pinned read-back area: lse and doffsets each their own,
+    and one [N][heads][dh] buffer that out, dq, dk and dv pass through in turn."""
     names_in = ("q", "k", "v", "offsets", "dout")
     in_bytes = sum(inp[n].numel() * inp[n].element_size() for n in names_in)
-    out_bytes = in_bytes + w.heads * w.N * 4  # out, dq, dk, dv, doffsets mirror the inputs; + lse
+    row_bytes = inp["q"].numel() * inp["q"].element_size()
+    host_out_bytes = row_bytes + w.heads * w.N * 4 + inp["offsets"].numel() * 4
     try:
         import psutil
         avail = psutil.virtual_memory().available
@@ -580,28 +593,23 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
     # of the free RAM only
     local_ranks = max(1, int(os.environ.get("LOCAL_WORLD_SIZE", str(world))))
     avail //= local_ranks
-    # pinned host memory: all inputs, and every output if that stays under 60% of this rank's share
-    # of free RAM; otherwise the step's read-back is the offset gradient and lse only
-    read_all = in_bytes + out_bytes < 0.6 * avail
-    skip = in_bytes > 0.6 * avail
+    skip = in_bytes + host_out_bytes > 0.75 * avail
     if world > 1:
         # the ranks must agree on running the leg (it contains collectives)
         from deformable_slide_attention_b200 import ranks
         skip = ranks.max_over_ranks(1.0 if skip else 0.0, dev) > 0.5
-        read_all = ranks.max_over_ranks(0.0 if read_all else 1.0, dev) < 0.5
     if skip:
         return {"value": None, "unit": UNIT,
-                "skipped": f"host RAM share {avail >> 30} GiB per rank too small for {in_bytes >> 30} GiB"}
+                "skipped": f"host RAM share {avail >> 30} GiB per rank too small for "
+                           f"{(in_bytes + host_out_bytes) >> 30} GiB"}
     h_in = {}
     try:
         for n in names_in:
             h_in[n] = torch.empty(inp[n].shape, dtype=inp[n].dtype, pin_memory=True)
             h_in[n].copy_(inp[n])
-        h_out = {"lse": torch.empty((w.heads, w.N), dtype=torch.float32, pin_memory=True),
-                 "doffsets": torch.empty(inp["offsets"].shape, dtype=torch.float32, pin_memory=True)}
-        if read_all:
-            for n in ("out", "dq", "dk", "dv"):
-                h_out[n] = torch.empty(inp["q"].shape, dtype=inp["q"].dtype, pin_memory=True)
+        h_rows = torch.empty(inp["q"].shape, dtype=inp["q"].dtype, pin_memory=True)
+        h_lse = torch.empty((w.heads, w.N), dtype=torch.float32, pin_memory=True)
+        h_doff = torch.empty(inp["offsets"].shape, dtype=torch.float32, pin_memory=True)
     except RuntimeError as e:
         err = str(e)
     else:
@@ -612,39 +620,68 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
         failed = ranks.max_over_ranks(1.0 if failed else 0.0, dev) > 0.5
     if failed:
         h_in.clear()
-        h_out = {}
         return {"value": None, "unit": UNIT,
                 "skipped": f"pinned host buffers unavailable: {err or 'on another rank'}"[:200]}
     d_in = {n: inp[n] for n in names_in}
-    stream = torch.cuda.current_stream(dev)
+    compute = torch.cuda.current_stream(dev)
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     fwd_fn, bwd_fn = path_of(w, abi)
+    state = {"computed": None, "read": None}
+    d2h_bytes = [0]
 
     def step():
-        for n in names_in:
-            d_in[n].copy_(h_in[n], non_blocking=True)
+        # inputs: after the previous step's compute has finished reading them
+        if state["computed"] is not None:
+            s_h2d.wait_event(state["computed"])
+        with torch.cuda.stream(s_h2d):
+            for n in names_in:
+                d_in[n].copy_(h_in[n], non_blocking=True)
+        arrived = torch.cuda.Event()
+        arrived.record(s_h2d)
+        compute.wait_event(arrived)
+        if state["read"] is not None:  # the output buffers are free again
+            compute.wait_event(state["read"])
         out, lse = fwd_fn(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], w.dims, w.window,
                           out=outs[0], lse=outs[1], workspace=ws[0])
         dq, dk, dv, doff = bwd_fn(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], lse,
                                   d_in["dout"], w.dims, w.window, workspace=ws[1], grads=outs[2:])
-        for n, t in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("doffsets", doff)):
-            if n in h_out:
-                h_out[n].copy_(t, non_blocking=True)
+        done = torch.cuda.Event()
+        done.record(compute)
+        state["computed"] = done
+        s_d2h.wait_event(done)
+        nb = 0
+        with torch.cuda.stream(s_d2h):
+            for t in (out, dq, dk, dv):
+                h_rows.copy_(t, non_blocking=True)
+                nb += t.numel() * t.element_size()
+            h_lse.copy_(lse, non_blocking=True)
+            h_doff.copy_(doff, non_blocking=True)
+            nb += lse.numel() * 4 + doff.numel() * 4
+        read = torch.cuda.Event()
+        read.record(s_d2h)
+        state["read"] = read
+        d2h_bytes[0] = nb
 
     step()
     torch.cuda.synchronize(dev)
     steps = max(1, min(args.steps, 3))
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
+    t0.record(compute)
+    begin = torch.cuda.Event()
+    begin.record(compute)
+    state["computed"] = begin  # the first timed copies start after t0
     for _ in range(steps):
         step()
-    t1.record(stream)
+    compute.wait_event(state["read"])  # the last read-back is inside the timed region
+    t1.record(compute)
     torch.cuda.synchronize(dev)
     from deformable_slide_attention_b200 import ranks
     ms = ranks.max_over_ranks(t0.elapsed_time(t1) / steps, dev)
     bi = sum(t.numel() * t.element_size() for t in h_in.values())
-    bo = sum(t.numel() * t.element_size() for t in h_out.values())
     return {"value": ranks.job_rate(w.N, world, ms), "unit": UNIT, "ms_per_step": ms, "steps": steps,
-            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "read_back": sorted(h_out)}
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": d2h_bytes[0],
+            "read_back": ["dk", "doffsets", "dq", "dv", "lse", "out"],
+            "overlap": "inputs of step i+1 (own stream) with the read-back of step i (own stream)"}
 
 
 if __name__ == "__main__":
