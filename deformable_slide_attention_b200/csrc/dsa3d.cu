@@ -401,16 +401,17 @@ bool make_pair_map(CUtensorMap* m, const void* base, const Shape& s) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Bucket rows per tile: about 130 queries per tile at the volume's average density (one query
+// Bucket rows per tile: about 225 queries per tile at the volume's average density (one query
 // per bucket, spread over (F+kt)(H'+kh)(W'+kw) buckets), 1..kTcRyMax; DSA3D_TC_RY overrides it.
-// A step costs about the same whatever the tile's query count, so fuller tiles win even where
-// some of them need a second pass (1080p: 347, 330, 326 ms at 5, 6, 7 rows).
+// A tile of more than 128 queries takes a second pass, but each pass walks only its own union
+// rows and each epilogue warp skips the rows none of its queries touch, so tall tiles still win
+// (1080p: 309, 293, 286, 277 ms at 6, 8, 10, 12 rows; 720p: 9.5, 8.8, 8.1, 8.3 ms).
 TcTileGeo make_tile_geo(const Shape& s, int hg) {
   const SortGeo sg = make_sort_geo(s);
   TcTileGeo tg;
   tg.Wx = kTcSeg - s.kw;
   const double dens = (double)s.N / ((double)sg.Et * sg.Ey * sg.Ex);
-  int ry = (int)std::lround(130.0 / (dens * tg.Wx));
+  int ry = (int)std::lround(225.0 / (dens * tg.Wx));
   if (const char* e = std::getenv("DSA3D_TC_RY")) ry = std::atoi(e);
   tg.Ry = ry < 1 ? 1 : (ry > kTcRyMax ? kTcRyMax : ry);
   tg.nYb = (sg.Ey + tg.Ry - 1) / tg.Ry;

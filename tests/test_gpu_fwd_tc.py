@@ -82,7 +82,7 @@ def test_every_tile_geometry_gives_the_same_bits(case):
     _, inp = inputs.custom(*dims, heads, dh, window, "bf16", seed=700 + case, scale=scale)
     d = to_cuda(inp)
     ref = _fwd(d, dims, window)
-    for ry in (1, 3, 8):
+    for ry in (1, 3, 8, 12):
         with _env(DSA3D_TC_RY=ry):
             got = _fwd(d, dims, window)
         assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[1]), f"Ry={ry}"
