@@ -156,6 +156,7 @@ def alg_bytes_per_item(w, kernel):
         "dsa3d_bwd_q_kernel": 4 * w.dh * s + 28,      # q, k, v, dO; offsets, lse -> doffsets
         "dsa3d_bwd_dq_kernel": 2 * w.dh * s,          # k -> dq
         "dsa3d_bwd_kv_kernel": 4 * w.dh * s,          # q, dO -> dk, dv
+        "dsa3d_bwd_kv_tc_kernel": 4 * w.dh * s,       # the same on tcgen05
         "dsa3d_pair_v_kernel": 2 * w.dh * s,          # v -> paired value rows (workspace)
         "fwd": 4 * w.dh * s + 16,
         "bwd": 8 * w.dh * s + 28,
@@ -174,6 +175,7 @@ def alg_flop_per_item(w, kernel):
     B = (w.window[0] + 1) * (w.window[1] + 1) * (w.window[2] + 1)
     per = {"dsa3d_fwd_kernel": 4, "dsa3d_fwd_mma_kernel": 4, "dsa3d_fwd_tc_kernel": 4, "dsa3d_bwd_kernel": 10,
            "dsa3d_bwd_q_kernel": 4, "dsa3d_bwd_dq_kernel": 2, "dsa3d_bwd_kv_kernel": 4,
+           "dsa3d_bwd_kv_tc_kernel": 4,
            "fwd": 4, "bwd": 10}
     return per.get(kernel, 0) * w.dh * B
 

@@ -12,6 +12,7 @@
 
 #include "dsa3d.h"
 #include "dsa3d_bwd.cuh"
+#include "dsa3d_bwd_kv_tc.cuh"
 #include "dsa3d_bwd_mma.cuh"
 #include "dsa3d_fwd.cuh"
 #include "dsa3d_fwd_mma.cuh"
@@ -453,6 +454,14 @@ dsa3d_status_t fwd_tc_group(const Shape& s, const void* q, const void* k, const 
   return DSA3D_OK;
 }
 
+// The tcgen05 key side runs unless DSA3D_KV_KERNEL=mma selects the mma.sync one, or a tile's
+// covering queries span more bucket-row ranges than it takes ((kt + 1)(4 + kh) > 128).
+bool use_tc_key_side(const Shape& s) {
+  const char* e = std::getenv("DSA3D_KV_KERNEL");
+  if (e && std::strcmp(e, "mma") == 0) return false;
+  return (s.kt + 1) * (kKvtRows + s.kh) <= kKvtRanges;
+}
+
 struct BwdArgs {
   const void *q, *k, *v, *dout;
   const float *off, *lse;
@@ -520,7 +529,21 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
         kb, static_cast<bf*>(dq), w.cnt, w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg, h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
-  {
+  if (use_tc_key_side(s)) {
+    using C = KvtCfg<DH>;
+    const int64_t tiles = (int64_t)hg * s.F * ((s.Hp + kKvtRows - 1) / kKvtRows) * ((s.Wp + kKvtKeys - 1) / kKvtKeys);
+    auto kern = dsa3d_bwd_kv_tc_kernel<DH>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return DSA3D_ERR_CUDA;
+    const DeviceInfo d = device_info();
+    int64_t grid = d.sms;
+    if (grid > tiles) grid = tiles;
+    if (grid < 1) grid = 1;
+    TimedLaunch tl(kKernBwdKvTc, st);
+    kern<<<(int)grid, kKvtThreads, C::SMEM_BYTES, st>>>(qb, ob, static_cast<bf*>(dk), static_cast<bf*>(dv), w.cnt,
+                                                       w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg, h0, hg);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  } else {
     const int64_t tiles = (int64_t)hg * s.F * ((s.Hp + kKvRows - 1) / kKvRows) * ((s.Wp + 15) / 16);
     const int smem = kv_dyn_bytes<DH>();
     if (cudaFuncSetAttribute(dsa3d_bwd_kv_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=

@@ -33,6 +33,7 @@ enum KernelId {
   kKernPointwiseDw,
   kKernSortOrder,
   kKernFwdTc,
+  kKernBwdKvTc,
   kKernCount
 };
 inline const char* kernel_name(int id) {
@@ -43,7 +44,8 @@ inline const char* kernel_name(int id) {
       "dsa3d_bwd_dq_kernel",   "dsa3d_bwd_kv_kernel",     "dsa3d_pair_v_kernel",
       "dsa3d_fwd_taps_kernel", "dsa3d_bwd_taps_kernel", "dsa3d_dwconv3d_kernel",
       "dsa3d_dwconv3d_dw_kernel", "dsa3d_pointwise_offsets_kernel", "dsa3d_pointwise_dz_kernel",
-      "dsa3d_pointwise_dw_kernel", "dsa3d_sort_order_kernels", "dsa3d_fwd_tc_kernel"};
+      "dsa3d_pointwise_dw_kernel", "dsa3d_sort_order_kernels", "dsa3d_fwd_tc_kernel",
+      "dsa3d_bwd_kv_tc_kernel"};
   return names[id];
 }
 
