@@ -539,9 +539,12 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
     int64_t grid = d.sms;
     if (grid > tiles) grid = tiles;
     if (grid < 1) grid = 1;
+    // the tile counter: the scan's block sums, dead once the sort is done (at least 16 bytes)
+    if (cudaMemsetAsync(w.bsum, 0, sizeof(int), st) != cudaSuccess) return DSA3D_ERR_CUDA;
     TimedLaunch tl(kKernBwdKvTc, st);
     kern<<<(int)grid, kKvtThreads, C::SMEM_BYTES, st>>>(qb, ob, static_cast<bf*>(dk), static_cast<bf*>(dv), w.cnt,
-                                                       w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg, h0, hg);
+                                                       w.sorted_n, w.sorted_ex, gbox, bbox, dft, w.bsum, g, sg,
+                                                       bg, h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   } else {
     const int64_t tiles = (int64_t)hg * s.F * ((s.Hp + kKvRows - 1) / kKvRows) * ((s.Wp + 15) / 16);

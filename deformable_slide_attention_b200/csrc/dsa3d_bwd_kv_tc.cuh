@@ -34,6 +34,7 @@ constexpr int kKvtRows = 4;        // key rows per tile
 constexpr int kKvtKeys = 32;       // keys per key row of a tile
 constexpr int kKvtQ = 64;          // queries per stage (K of the UMMAs: four K-steps of 16)
 constexpr int kKvtStages = 3;
+constexpr int kKvtTileRing = 4;    // tiles drawn ahead of the slowest role
 constexpr int kKvtRanges = 128;    // bucket-row ranges per tile: (kt + 1) (kKvtRows + kh) <= this
 constexpr int kKvtEpiWarp0 = 8, kKvtMmaWarp = 12;
 constexpr int kKvtThreads = 13 * 32;
@@ -107,8 +108,10 @@ struct KvtCfg {
   static constexpr int STAGE_BYTES = 2 * A_BYTES + 2 * B_BYTES;
   static constexpr int META_BYTES = kKvtStages * kKvtQ * (int)sizeof(KvtSlot);
   static constexpr int RANGE_BYTES = kKvtEpiWarp0 * (2 * kKvtRanges + 8) * 4;
+  static constexpr int SCRATCH_BYTES = 16 * kKvtEpiWarp0;  // a store target per builder warp
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = kKvtStages * STAGE_BYTES + META_BYTES + RANGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int SMEM_BYTES =
+      kKvtStages * STAGE_BYTES + META_BYTES + RANGE_BYTES + SCRATCH_BYTES + BAR_BYTES + 1024;
   static constexpr int COLS = (4 * DH <= 256) ? 256 : 512;  // two (dK, dV) pairs
   static constexpr uint32_t IDESC = umma_idesc_bf16(128, DH, false, true);
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -146,13 +149,15 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
                            const int* __restrict__ start, const int* __restrict__ sorted_n,
                            const int* __restrict__ sorted_ex, const unsigned short* __restrict__ gbox,
                            const unsigned short* __restrict__ bbox, const float2* __restrict__ dft,
-                           const Geo g, const SortGeo sg, const BoxGeo bg, const int h0, const int hg) {
+                           int* __restrict__ tile_counter, const Geo g, const SortGeo sg, const BoxGeo bg,
+                           const int h0, const int hg) {
   using C = KvtCfg<DH>;
   extern __shared__ __align__(1024) unsigned char kvt_smem[];
   unsigned char* stages = kvt_smem + ((1024 - (smem_u32(kvt_smem) & 1023)) & 1023);
   KvtSlot* meta = reinterpret_cast<KvtSlot*>(stages + kKvtStages * C::STAGE_BYTES);
   int* ranges = reinterpret_cast<int*>(stages + kKvtStages * C::STAGE_BYTES + C::META_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stages + kKvtStages * C::STAGE_BYTES + C::META_BYTES + C::RANGE_BYTES);
+  unsigned char* scratch = stages + kKvtStages * C::STAGE_BYTES + C::META_BYTES + C::RANGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scratch + C::SCRATCH_BYTES);
   const uint32_t st0 = smem_u32(stages);
   const uint32_t b0 = smem_u32(bars);
   auto full = [&](int s) { return b0 + 8u * s; };
@@ -160,9 +165,13 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
   auto acc_full = [&](int s) { return b0 + 8u * (2 * kKvtStages + s); };
   auto acc_empty = [&](int s) { return b0 + 8u * (2 * kKvtStages + 2 + s); };
   const uint32_t m_done = b0 + 8u * (2 * kKvtStages + 4);
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
+  auto tile_full = [&](int s) { return b0 + 8u * (2 * kKvtStages + 5 + s); };
+  auto tile_empty = [&](int s) { return b0 + 8u * (2 * kKvtStages + 5 + kKvtTileRing + s); };
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
-  static_assert((2 * kKvtStages + 5) * 8 <= 128 && 128 + 8 <= C::BAR_BYTES, "barrier slots");
+  volatile int* tile_ring = reinterpret_cast<volatile int*>(tslot + 2);  // kKvtTileRing tile indices
+  static_assert((2 * kKvtStages + 5 + 2 * kKvtTileRing) * 8 <= 192 && 192 + 8 + 4 * kKvtTileRing <= C::BAR_BYTES,
+                "barrier slots");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -175,6 +184,10 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
       mbar_init(acc_empty(s), 4);
     }
     mbar_init(m_done, 1);
+    for (int s = 0; s < kKvtTileRing; s++) {
+      mbar_init(tile_full(s), 1);
+      mbar_init(tile_empty(s), kKvtThreads / 32);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -185,6 +198,31 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
   const uint32_t tmem = *tslot;
   const int NB = (g.Wp + kKvtKeys - 1) / kKvtKeys, NY = (g.Hp + kKvtRows - 1) / kKvtRows;
   const int64_t tiles = (int64_t)hg * g.F * NY * NB;
+  // Tiles are taken in order from a counter shared by the CTAs (so that the tiles in flight stay
+  // close together and their query rows and splats stay in L2): builder warp 0's lane 0 draws the
+  // CTA's k-th tile into slot k % kKvtTileRing of a ring every warp reads (-1: no tile left).
+  auto next_tile = [&](uint32_t k, bool& ok) -> int64_t {
+    const int s = (int)(k % kKvtTileRing);
+    int64_t t = -1;
+    if (lane == 0) {
+      if (warp == 0) {
+        if (k >= (uint32_t)kKvtTileRing && !mbar_wait(tile_empty(s), ((k / kKvtTileRing) - 1) & 1, abort_flag)) ok = false;
+        if (ok) {
+          const int v = atomicAdd(tile_counter, 1);
+          tile_ring[s] = (v < tiles) ? v : -1;
+          mbar_arrive(tile_full(s));
+        }
+      }
+      if (ok && !mbar_wait(tile_full(s), (k / kKvtTileRing) & 1, abort_flag)) ok = false;
+      if (ok) {
+        t = tile_ring[s];
+        mbar_arrive(tile_empty(s));
+      }
+    }
+    ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
+    t = __shfl_sync(kFull, (int)t, 0);
+    return ok ? t : -1;
+  };
 
   if (warp < kKvtEpiWarp0) {
     // ===================== stage builders: warp w builds query columns 8w .. 8w + 7 of every stage =====================
@@ -196,7 +234,9 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
     KvtSlot* mw = meta;               // stage buffers' slots
     uint32_t gs = 0;                  // stages of the tiles before this one
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    for (uint32_t kt_ = 0; ok; kt_++) {
+      const int64_t t = next_tile(kt_, ok);
+      if (t < 0) break;
       const KvtTile T = kvt_tile(g, sg, t);
       const int h = h0 + T.hh;
       // ranges 4 lane .. 4 lane + 3 and their exclusive prefix
@@ -350,19 +390,20 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
         }
         __syncwarp();
         DSA3D_KV_CLK(5);
-        if (live) {
-          // key x of key row r, query k = 8 warp + kl: row r 32 + x of the A tile, whose 128-byte
-          // row starts at 128 (r 32 + x) and holds query chunk warp at chunk warp ^ (x & 7)
+        {
+          // key x of key row r is tile row mk = 4 x + r (the four key rows of a column sit in
+          // rows with different swizzle phases, so the four lanes of a slot store to different
+          // banks); query k = 8 warp + kl sits in chunk warp ^ (mk & 7) of the row.  A column
+          // outside the tile (or an item without a box row here) stores to the warp's scratch word.
           const float D = m.D, ft = m.ft;
-          unsigned char* ag_r = ag + r * 4096 + 2 * kl;
-          unsigned char* ab_r = ab + r * 4096 + 2 * kl;
+          const uint32_t dummy = (uint32_t)(scratch - ag) + 16u * warp;
 #pragma unroll
           for (int w = 0; w < 8; w++) {
             if (w >= words) break;
 #pragma unroll
             for (int e = 0; e < 2; e++) {
               const int x = m.ox + 2 * w + e;
-              if (x < 0 || x >= kKvtKeys) continue;
+              const bool in = live && x >= 0 && x < kKvtKeys;
               const float bb0 = __uint_as_float(e ? (ew0[w] & 0xffff0000u) : (ew0[w] << 16));
               const float gg0 = __uint_as_float(e ? (gw0[w] & 0xffff0000u) : (gw0[w] << 16));
               const float bb1 = __uint_as_float(e ? (ew1[w] & 0xffff0000u) : (ew1[w] << 16));
@@ -370,9 +411,10 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
               const float be = fmaf(ft, bb1 - bb0, bb0);
               const float c0 = fmaf(-D, bb0, gg0), c1 = fmaf(-D, bb1, gg1);
               const float ga = fmaf(ft, c1 - c0, c0);
-              const uint32_t off = (uint32_t)(x * 128 + ((warp ^ (x & 7)) << 4));
-              *reinterpret_cast<unsigned short*>(ag_r + off) = bf16_bits(ga);
-              *reinterpret_cast<unsigned short*>(ab_r + off) = bf16_bits(be);
+              const int mk = 4 * x + r;
+              const uint32_t off = in ? (uint32_t)(128 * mk + ((warp ^ (mk & 7)) << 4) + 2 * kl) : dummy;
+              *reinterpret_cast<unsigned short*>(ag + off) = bf16_bits(ga);
+              *reinterpret_cast<unsigned short*>(ag + off + (in ? C::A_BYTES : 0u)) = bf16_bits(be);
             }
           }
         }
@@ -388,11 +430,13 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
     }
   } else if (warp < kKvtMmaWarp) {
     // ===================== dK, dV out: thread = key =====================
-    const int quarter = warp - kKvtEpiWarp0;  // lanes 32 quarter ..; key row yk0 + quarter
+    const int quarter = warp - kKvtEpiWarp0;  // lanes 32 quarter ..: tile row mk = 32 quarter + lane
     const uint32_t lq = (uint32_t)(32 * quarter) << 16;
     uint32_t tc = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, tc++) {
+    for (; ok; tc++) {
+      const int64_t t = next_tile(tc, ok);
+      if (t < 0) break;
       const KvtTile T = kvt_tile(g, sg, t);
       const int total = kvt_total(g, sg, T, start, lane);
       const int buf = (int)(tc & 1);
@@ -402,7 +446,8 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
       if (!ok) break;
       if (quarter == 0 && lane == 0 && tc < 1000) TC_CLK(12288 + 2 * tc);
       tc_fence_after();
-      const int yk = T.yk0 + quarter, x = T.x_lo + lane;
+      const int mk = 32 * quarter + lane;  // key x = mk / 4 of key row mk % 4
+      const int yk = T.yk0 + (mk & 3), x = T.x_lo + (mk >> 2);
       const bool live = yk < g.Hp && x < g.Wp;
       const int64_t row = (((int64_t)(T.tk * g.Hp + yk) * g.Wp + x) * g.heads + (h0 + T.hh)) * DH;
       const uint32_t acc = tmem + lq + (uint32_t)(buf * 2 * DH);
@@ -441,7 +486,9 @@ __global__ void __launch_bounds__(kKvtThreads, 1)
     bool ok = true;
     const uint64_t d0 = umma_sdesc_sw128(st0, 16, 1024);                     // A: K-major, 8-row groups
     const uint64_t e0 = umma_sdesc_sw128(st0, C::HALF_BYTES, 1024);          // B: MN-major, 64-dim halves
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, tc++) {
+    for (; ok; tc++) {
+      const int64_t t = next_tile(tc, ok);
+      if (t < 0) break;
       const KvtTile T = kvt_tile(g, sg, t);
       const int total = kvt_total(g, sg, T, start, lane);
       const int nst = (total + kKvtQ - 1) / kKvtQ;
