@@ -446,10 +446,12 @@ dsa3d_status_t fwd_tc_group(const Shape& s, const void* q, const void* k, const 
   int64_t grid = d.sms;
   if (grid > tg.tiles) grid = tg.tiles;
   if (grid < 1) grid = 1;
+  // the tile counter: the scan's block sums, dead once the sort is done (at least 16 bytes)
+  if (cudaMemsetAsync(w.bsum, 0, sizeof(int), st) != cudaSuccess) return DSA3D_ERR_CUDA;
   TimedLaunch tl(kKernFwdTc, st);
   kern<<<(int)grid, kTcThreads, C::SMEM_BYTES, st>>>(tmk, tmv, static_cast<const __nv_bfloat16*>(q), off,
                                                      static_cast<__nv_bfloat16*>(out), lse, w.cnt, w.sorted_n,
-                                                     w.sorted_ex, g, sg, tg, h0);
+                                                     w.sorted_ex, w.bsum, g, sg, tg, h0);
   if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   return DSA3D_OK;
 }

@@ -54,6 +54,7 @@ constexpr int kTcSeg = 32;         // keys per segment
 constexpr int kTcRyMax = 12;       // bucket rows per tile (Ry <= kTcRyMax)
 constexpr int kTcKStages = 4;      // K pair ring
 constexpr int kTcVStages = 3;      // V pair ring
+constexpr int kTcTileRing = 4;     // tiles drawn ahead of the slowest role
 constexpr float kTcRescale = 8.f;  // lazy-rescale threshold (base-2 units)
 
 template <int DH>
@@ -69,7 +70,8 @@ struct FwdTcCfg {
   static constexpr int COL_OB = COL_OA + DH;              // O of keys 16 .. 31
   static constexpr int COLS = 512;                        // allocation (power of two >= COL_OB + DH)
   static_assert(COL_OB + DH <= COLS, "tensor memory budget");
-  static_assert((2 * kTcKStages + 2 * kTcVStages + 17) * 8 <= 256, "mbarriers below the allocation slot");
+  static_assert((2 * kTcKStages + 2 * kTcVStages + 17 + 2 * kTcTileRing) * 8 <= 448,
+                "mbarriers below the allocation slot");
   static constexpr int STAGE_BYTES = (kTcKStages + kTcVStages) * PAIR_BYTES;
   static constexpr int BAR_BYTES = 512;                   // mbarriers, then the allocation slot, abort flag
   static constexpr int XCH_BYTES = 2 * 2 * 128 * 8;       // (max, sum) per pass parity, half, lane
@@ -142,8 +144,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         const __nv_bfloat16* __restrict__ q, const float* __restrict__ off,
                         __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
                         const int* __restrict__ start, const int* __restrict__ sorted_n,
-                        const int* __restrict__ sorted_ex, const Geo g, const SortGeo sg,
-                        const TcTileGeo tg, const int h0) {
+                        const int* __restrict__ sorted_ex, int* __restrict__ tile_counter, const Geo g,
+                        const SortGeo sg, const TcTileGeo tg, const int h0) {
   using C = FwdTcCfg<DH>;
   extern __shared__ __align__(1024) unsigned char tc_smem[];
   unsigned char* stages = tc_smem + ((1024 - (smem_u32(tc_smem) & 1023)) & 1023);
@@ -164,8 +166,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t a_full = bx + 8u * 8, o_full = bx + 8u * 9, o_empty = bx + 8u * 10;
   const uint32_t m_done = bx + 8u * 11, m_done2 = bx + 8u * 12;  // the UMMA issuers' own exit drains
   auto x_bar = [&](int qtr) { return bx + 8u * (13 + qtr); };       // end-of-pass exchange of a lane quarter
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(stages + C::STAGE_BYTES + 8 * 32);
+  auto tile_full = [&](int s) { return bx + 8u * (17 + s); };
+  auto tile_empty = [&](int s) { return bx + 8u * (17 + kTcTileRing + s); };
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(stages + C::STAGE_BYTES + 448);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  volatile int* tile_ring = reinterpret_cast<volatile int*>(tslot + 2);  // kTcTileRing tile indices
   float2* xch = reinterpret_cast<float2*>(stages + C::STAGE_BYTES + C::BAR_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -190,6 +195,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(m_done, 1);
     mbar_init(m_done2, 1);
     for (int qtr = 0; qtr < 4; qtr++) mbar_init(x_bar(qtr), 2);
+    for (int s = 0; s < kTcTileRing; s++) {
+      mbar_init(tile_full(s), 1);
+      mbar_init(tile_empty(s), kTcThreads / 32);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -198,6 +207,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // Tiles are taken in order from a counter shared by the CTAs, so that the tiles in flight stay
+  // close together and their K and V rows stay in L2: the K producer draws the CTA's k-th tile into
+  // slot k % kTcTileRing of a ring that one thread of every warp reads (-1: no tile left).
+  auto tile_at = [&](uint32_t k, bool fetch, bool& ok) -> int64_t {
+    const int s = (int)(k % kTcTileRing);
+    if (fetch) {
+      if (k >= (uint32_t)kTcTileRing && !mbar_wait(tile_empty(s), ((k / kTcTileRing) - 1) & 1, abort_flag)) {
+        ok = false;
+        return -1;
+      }
+      const int v = atomicAdd(tile_counter, 1);
+      tile_ring[s] = (v < tg.tiles) ? v : -1;
+      mbar_arrive(tile_full(s));
+    }
+    if (!mbar_wait(tile_full(s), (k / kTcTileRing) & 1, abort_flag)) {
+      ok = false;
+      return -1;
+    }
+    const int t = tile_ring[s];
+    mbar_arrive(tile_empty(s));
+    return t;
+  };
 
   if (warp == kTcKWarp || warp == kTcVWarp) {
     // ===================== TMA producers: K pairs (warp kTcKWarp) and V pairs (warp kTcVWarp) ==
@@ -223,7 +254,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         cnt++;
         return true;
       };
-      for (int64_t t = blockIdx.x; t < tg.tiles && ok; t += gridDim.x) {
+      for (uint32_t k = 0; ok; k++) {
+        const int64_t t = tile_at(k, is_k, ok);
+        if (t < 0) break;
         TcTile T;
         tc_tile(tg, sg, start, t, T);
         const int passes = (T.cnt + 127) / 128;
@@ -251,7 +284,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       const uint32_t tA = tmem + C::COL_A, tS = tmem + C::COL_S;
       const uint64_t kd0 = umma_sdesc_sw128(kst, 16, 1024);
-      for (int64_t t = blockIdx.x; t < tg.tiles && ok; t += gridDim.x) {
+      for (uint32_t k = 0; ok; k++) {
+        const int64_t t = tile_at(k, false, ok);
+        if (t < 0) break;
         TcTile T;
         tc_tile(tg, sg, start, t, T);
         const int passes = (T.cnt + 127) / 128;
@@ -301,7 +336,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       const uint32_t tP = tmem + C::COL_P, tOa = tmem + C::COL_OA, tOb = tmem + C::COL_OB;
       const uint64_t vd0 = umma_sdesc_sw128(vst, C::PAIR_BYTES / C::HALVES, 1024);
-      for (int64_t t = blockIdx.x; t < tg.tiles && ok; t += gridDim.x) {
+      for (uint32_t k = 0; ok; k++) {
+        const int64_t t = tile_at(k, false, ok);
+        if (t < 0) break;
         TcTile T;
         tc_tile(tg, sg, start, t, T);
         const int passes = (T.cnt + 127) / 128;
@@ -368,7 +405,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) r = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
       return __shfl_sync(kFull, r, 0) != 0;
     };
-    for (int64_t t = blockIdx.x; t < tg.tiles && ok; t += gridDim.x) {
+    for (uint32_t k = 0; ok; k++) {
+      int tv = -1, okv = 1;
+      if (lane == 0) {
+        bool o = true;
+        tv = (int)tile_at(k, false, o);
+        okv = o ? 1 : 0;
+      }
+      ok = __shfl_sync(kFull, okv, 0) != 0;
+      const int64_t t = __shfl_sync(kFull, tv, 0);
+      if (!ok || t < 0) break;
       TcTile T;
       tc_tile(tg, sg, start, t, T);
       const int passes = (T.cnt + 127) / 128;
