@@ -12,6 +12,7 @@
 
 #include "dsa3d.h"
 #include "dsa3d_bwd.cuh"
+#include "dsa3d_bwd_dq_tc.cuh"
 #include "dsa3d_bwd_kv_tc.cuh"
 #include "dsa3d_bwd_mma.cuh"
 #include "dsa3d_fwd.cuh"
@@ -456,6 +457,12 @@ dsa3d_status_t fwd_tc_group(const Shape& s, const void* q, const void* k, const 
   return DSA3D_OK;
 }
 
+// The tcgen05 dq pass runs unless DSA3D_DQ_KERNEL=mma selects the mma.sync one.
+bool use_tc_dq() {
+  const char* e = std::getenv("DSA3D_DQ_KERNEL");
+  return !(e && std::strcmp(e, "mma") == 0);
+}
+
 // The tcgen05 key side runs unless DSA3D_KV_KERNEL=mma selects the mma.sync one, or a tile's
 // covering queries span more bucket-row ranges than it takes ((kt + 1)(4 + kh) > 128).
 bool use_tc_key_side(const Shape& s) {
@@ -521,7 +528,25 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
         h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
   }
-  {
+  if (use_tc_dq()) {
+    using C = DqtCfg<DH>;
+    CUtensorMap tmk;
+    if (!make_pair_map(&tmk, k, s)) return DSA3D_ERR_CUDA;
+    const TcTileGeo tg = make_tile_geo(s, hg);
+    auto kern = dsa3d_bwd_dq_tc_kernel<DH>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return DSA3D_ERR_CUDA;
+    const DeviceInfo d = device_info();
+    int64_t grid = 2 * (int64_t)d.sms;
+    if (grid > tg.tiles) grid = tg.tiles;
+    if (grid < 1) grid = 1;
+    // the tile counter: the scan's block sums, dead once the sort is done
+    if (cudaMemsetAsync(w.bsum, 0, sizeof(int), st) != cudaSuccess) return DSA3D_ERR_CUDA;
+    TimedLaunch tl(kKernBwdDqTc, st);
+    kern<<<(int)grid, kDqtThreads, C::SMEM_BYTES, st>>>(tmk, static_cast<bf*>(dq), w.cnt, w.sorted_n, w.sorted_ex,
+                                                        gbox, bbox, dft, w.bsum, g, sg, bg, tg, h0);
+    if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;
+  } else {
     const int smem = 4 * dq_warp_bytes<DH>();
     if (cudaFuncSetAttribute(dsa3d_bwd_dq_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)

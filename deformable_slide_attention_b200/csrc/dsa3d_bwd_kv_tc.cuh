@@ -126,20 +126,6 @@ __device__ __forceinline__ uint32_t kvt_b_off(int k, int hv, int c) {
   return (uint32_t)(hv * (kKvtQ * 128) + k * 128 + ((c ^ (k & 7)) << 4));
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem] . B[smem], both shared-memory descriptors.  Issued by one thread.
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t .reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 
 template <int DH>

@@ -1,11 +1,11 @@
-"""The tcgen05 key side of the backward (dK, dV in tensor memory) against the oracle and against
-the mma.sync key side it replaces.
+"""The tcgen05 passes of the backward -- the key side (dK, dV in tensor memory) and dq (dq in
+tensor memory) -- against the oracle and against the mma.sync passes they replace.
 
-DSA3D_KV_KERNEL=mma selects the mma.sync key side (the library reads it at every call).  Both
-sum, per key, the same bf16 products in fp32; their results agree to the oracle's tolerance, and
-each is bit-for-bit repeatable (tests/test_gpu_determinism.py).  A window whose tiles span more
-bucket-row ranges than the tcgen05 kernel takes ((kt + 1)(4 + kh) > 128) falls back to the
-mma.sync kernel.
+DSA3D_KV_KERNEL=mma and DSA3D_DQ_KERNEL=mma select the mma.sync passes (the library reads them at
+every call).  Both forms sum the same bf16 products in fp32, in different orders; their results
+agree to the oracle's tolerance, and each is bit-for-bit repeatable
+(tests/test_gpu_determinism.py).  A window whose key tiles span more bucket-row ranges than the
+tcgen05 key side takes ((kt + 1)(4 + kh) > 128) falls back to the mma.sync key side.
 """
 import os
 
@@ -71,19 +71,25 @@ def test_key_side_matches_the_oracle_and_the_mma_key_side(case):
     # the two key sides sum the same bf16 products of each key in fp32, in different orders
     assert abs(f64(dk) - f64(dk_m)).max() <= tol
     assert abs(f64(dv) - f64(dv_m)).max() <= tol
+    with _env(DSA3D_DQ_KERNEL="mma"):
+        dq_q, dk_q, dv_q, doff_q = _bwd(d, lse, dims, window)
+    assert_close("dq (mma.sync)", f64(dq_q), r_dq, tol)
+    assert abs(f64(dq) - f64(dq_q)).max() <= tol
+    assert torch.equal(dk, dk_q) and torch.equal(dv, dv_q) and torch.equal(doff, doff_q), \
+        "the dq pass must not change the other gradients"
 
 
-def test_720p_train_key_side_agrees_with_the_mma_key_side():
-    # the full 720p training workload (16 heads x 115,200 tokens): every key of every head,
-    # against the mma.sync key side, to the bf16 output rounding of the two summation orders
+def test_720p_train_tc_passes_agree_with_the_mma_passes():
+    # the full 720p training workload (16 heads x 115,200 tokens): every key and query of every
+    # head, against the mma.sync passes, to the bf16 output rounding of the two summation orders
     w = inputs.BY_NAME["720p-train-bf16"]
     inp = inputs.make(w, "cpu", with_dout=True)
     d = to_cuda(inp)
     _, lse = abi.forward(d["q"], d["k"], d["v"], d["offsets"], w.dims, w.window)
-    _, dk, dv, _ = _bwd(d, lse, w.dims, w.window)
-    with _env(DSA3D_KV_KERNEL="mma"):
-        _, dk_m, dv_m, _ = _bwd(d, lse, w.dims, w.window)
-    for name, a, b in (("dk", dk, dk_m), ("dv", dv, dv_m)):
+    dq, dk, dv, _ = _bwd(d, lse, w.dims, w.window)
+    with _env(DSA3D_KV_KERNEL="mma", DSA3D_DQ_KERNEL="mma"):
+        dq_m, dk_m, dv_m, _ = _bwd(d, lse, w.dims, w.window)
+    for name, a, b in (("dq", dq, dq_m), ("dk", dk, dk_m), ("dv", dv, dv_m)):
         a, b = a.float(), b.float()
         err = (a - b).abs()
         bound = 2e-2 + 2.0 ** -7 * torch.maximum(a.abs(), b.abs())
