@@ -32,8 +32,8 @@ namespace dsa3d {
 
 constexpr int kDqtThreads = 192;
 constexpr int kDqtKWarp = 4, kDqtMmaWarp = 5;
-constexpr int kDqtKStages = 4;  // K pair ring
-constexpr int kDqtABufs = 2;    // A tiles
+constexpr int kDqtKStages = 3;  // K pair ring
+constexpr int kDqtABufs = 3;    // A tiles
 
 template <int DH>
 struct DqtCfg {
@@ -66,17 +66,18 @@ __global__ void __launch_bounds__(kDqtThreads, 2)
   const uint32_t b0 = smem_u32(bars);
   auto k_full = [&](int s) { return b0 + 8u * s; };
   auto k_empty = [&](int s) { return b0 + 8u * (kDqtKStages + s); };
-  auto a_full = [&](int s) { return b0 + 8u * (2 * kDqtKStages + s); };
-  auto a_empty = [&](int s) { return b0 + 8u * (2 * kDqtKStages + 2 + s); };
-  auto acc_full = [&](int s) { return b0 + 8u * (2 * kDqtKStages + 4 + s); };
-  auto acc_empty = [&](int s) { return b0 + 8u * (2 * kDqtKStages + 6 + s); };
-  const uint32_t m_done = b0 + 8u * (2 * kDqtKStages + 8);
-  auto tile_full = [&](int s) { return b0 + 8u * (2 * kDqtKStages + 9 + s); };
-  auto tile_empty = [&](int s) { return b0 + 8u * (2 * kDqtKStages + 9 + kTcTileRing + s); };
+  constexpr int BA = 2 * kDqtKStages, BC = BA + 2 * kDqtABufs;  // first A, first accumulator barrier
+  auto a_full = [&](int s) { return b0 + 8u * (BA + s); };
+  auto a_empty = [&](int s) { return b0 + 8u * (BA + kDqtABufs + s); };
+  auto acc_full = [&](int s) { return b0 + 8u * (BC + s); };
+  auto acc_empty = [&](int s) { return b0 + 8u * (BC + 2 + s); };
+  const uint32_t m_done = b0 + 8u * (BC + 4);
+  auto tile_full = [&](int s) { return b0 + 8u * (BC + 5 + s); };
+  auto tile_empty = [&](int s) { return b0 + 8u * (BC + 5 + kTcTileRing + s); };
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 28);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   volatile int* tile_ring = reinterpret_cast<volatile int*>(tslot + 2);
-  static_assert((2 * kDqtKStages + 9 + 2 * kTcTileRing) * 8 <= 224 && 232 + 4 * kTcTileRing <= C::BAR_BYTES,
+  static_assert((BC + 5 + 2 * kTcTileRing) * 8 <= 224 && 232 + 4 * kTcTileRing <= C::BAR_BYTES,
                 "barrier slots");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -85,9 +86,11 @@ __global__ void __launch_bounds__(kDqtThreads, 2)
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
     }
-    for (int s = 0; s < 2; s++) {
+    for (int s = 0; s < kDqtABufs; s++) {
       mbar_init(a_full(s), 128);
       mbar_init(a_empty(s), 1);
+    }
+    for (int s = 0; s < 2; s++) {
       mbar_init(acc_full(s), 1);
       mbar_init(acc_empty(s), 4);
     }
@@ -185,9 +188,9 @@ __global__ void __launch_bounds__(kDqtThreads, 2)
             break;
           }
           for (int r = 0; r < rows && ok; r++, kc++, ac++) {
-            const int ks_ = (int)(kc % kDqtKStages), as_ = (int)(ac & 1);
+            const int ks_ = (int)(kc % kDqtKStages), as_ = (int)(ac % kDqtABufs);
             if (!mbar_wait(k_full(ks_), (kc / kDqtKStages) & 1, abort_flag) ||
-                !mbar_wait(a_full(as_), (ac >> 1) & 1, abort_flag)) {
+                !mbar_wait(a_full(as_), (ac / kDqtABufs) & 1, abort_flag)) {
               ok = false;
               break;
             }
@@ -285,9 +288,9 @@ __global__ void __launch_bounds__(kDqtThreads, 2)
               const int nu = (jj + 1 < up) ? u : u + 1, nj = (jj + 1 < up) ? jj + 1 : 0;
               if (nu < g.kt) load_row(nu, nj, gn, bn);
             }
-            const int as_ = (int)(ac & 1);
-            if (ac >= 2) {
-              ok = wwait(a_empty(as_), ((ac >> 1) - 1) & 1);
+            const int as_ = (int)(ac % kDqtABufs);
+            if (ac >= (uint32_t)kDqtABufs) {
+              ok = wwait(a_empty(as_), ((ac / kDqtABufs) - 1) & 1);
               if (!ok) break;
             }
             unsigned char* arow = abuf + as_ * C::A_BYTES;
@@ -321,6 +324,7 @@ __global__ void __launch_bounds__(kDqtThreads, 2)
                 *reinterpret_cast<unsigned*>(arow + a_off(32 + key)) = bf16x2_bits(ft * a, ft * b);
               }
             }
+            // this thread's stores become visible to the tensor cores, then it arrives
             fence_proxy_async_smem();
             mbar_arrive(a_full(as_));
           }
