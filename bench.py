@@ -71,23 +71,17 @@ def parse_args(argv=None):
 # files that define those kernels and their launches ("files", under the package's csrc/) hash to
 # "sources"; the traffic of a launch is this times the (token, head) items it processes (the
 # kernels' traffic grows in proportion to the items).
-TENSOR_CORE_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_fwd_mma.cuh", "dsa3d_bwd_mma.cuh",
-                     "dsa3d_sort.cuh"]
-TC_FORWARD_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_tc.cuh", "dsa3d_fwd_tc.cuh",
-                    "dsa3d_sort.cuh", "dsa3d_bwd_mma.cuh", "dsa3d_fwd_mma.cuh"]
+TENSOR_CORE_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_tc.cuh", "dsa3d_sort.cuh", "dsa3d_fwd_tc.cuh",
+                     "dsa3d_fwd_mma.cuh", "dsa3d_bwd_mma.cuh", "dsa3d_bwd_dq_tc.cuh", "dsa3d_bwd_kv_tc.cuh"]
 PER_TAP_FILES = ["dsa3d.cu", "dsa3d_common.cuh", "dsa3d_taps.cuh", "dsa3d_bwd.cuh", "dsa3d_fwd.cuh"]
 NCU_TRAFFIC = [
-    {"files": TENSOR_CORE_FILES, "sources": "f439b4ef408f12c1",
+    {"files": TENSOR_CORE_FILES, "sources": "415297fb73f643fa",
      "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
      "bytes_per_item": {
-         "dsa3d_bwd_q_kernel": 2257.4,
-         "dsa3d_bwd_dq_kernel": 1649.9,
-         "dsa3d_bwd_kv_kernel": 2211.1,
-     }},
-    {"files": TC_FORWARD_FILES, "sources": "5401473b888b9a33",
-     "capture": "profiles/tensor_core_kernels_720p-train-bf16.md",
-     "bytes_per_item": {
-         "dsa3d_fwd_tc_kernel": 1552.3,
+         "dsa3d_fwd_tc_kernel": 1020.1,
+         "dsa3d_bwd_q_kernel": 2256.4,
+         "dsa3d_bwd_dq_tc_kernel": 1701.6,
+         "dsa3d_bwd_kv_tc_kernel": 2136.1,
      }},
     {"files": PER_TAP_FILES, "sources": "df10cf32e12d6270",
      "capture": "profiles/per_tap_kernels_720p-train-taps-bf16.md",
@@ -155,6 +149,7 @@ def alg_bytes_per_item(w, kernel):
         "dsa3d_bwd_kernel": 8 * w.dh * s + 28,        # the CUDA-core backward does it all
         "dsa3d_bwd_q_kernel": 4 * w.dh * s + 28,      # q, k, v, dO; offsets, lse -> doffsets
         "dsa3d_bwd_dq_kernel": 2 * w.dh * s,          # k -> dq
+        "dsa3d_bwd_dq_tc_kernel": 2 * w.dh * s,       # the same on tcgen05
         "dsa3d_bwd_kv_kernel": 4 * w.dh * s,          # q, dO -> dk, dv
         "dsa3d_bwd_kv_tc_kernel": 4 * w.dh * s,       # the same on tcgen05
         "dsa3d_pair_v_kernel": 2 * w.dh * s,          # v -> paired value rows (workspace)
@@ -175,7 +170,7 @@ def alg_flop_per_item(w, kernel):
     B = (w.window[0] + 1) * (w.window[1] + 1) * (w.window[2] + 1)
     per = {"dsa3d_fwd_kernel": 4, "dsa3d_fwd_mma_kernel": 4, "dsa3d_fwd_tc_kernel": 4, "dsa3d_bwd_kernel": 10,
            "dsa3d_bwd_q_kernel": 4, "dsa3d_bwd_dq_kernel": 2, "dsa3d_bwd_kv_kernel": 4,
-           "dsa3d_bwd_kv_tc_kernel": 4,
+           "dsa3d_bwd_kv_tc_kernel": 4, "dsa3d_bwd_dq_tc_kernel": 2,
            "fwd": 4, "bwd": 10}
     return per.get(kernel, 0) * w.dh * B
 
