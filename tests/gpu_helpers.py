@@ -41,6 +41,28 @@ def items_of(heads, N, n_sample, seed, include_edges=True):
     return np.array(sorted(items), dtype=np.int64)
 
 
+def edge_keys(dims, heads, seed, n_random=0):
+    """Key items h*N + n on the edges the key-side kernels tile by, for each head in ``heads``:
+    the first, second, middle and last two frames, the first and last rows, rows 3 and 4 (a
+    4-row tile boundary) and the middle row, and the columns 0, 31, 32 (a 32-key tile boundary),
+    the middle and the last -- every combination -- plus n_random seeded keys per head."""
+    F, Hp, Wp = dims
+    N = F * Hp * Wp
+    pick = lambda vals, hi: sorted({min(max(v, 0), hi - 1) for v in vals})
+    ts = pick([0, 1, F // 2, F - 2, F - 1], F)
+    ys = pick([0, 3, 4, Hp // 2, Hp - 1], Hp)
+    xs = pick([0, 31, 32, Wp // 2, Wp - 1], Wp)
+    g = np.random.default_rng(seed)
+    items = set()
+    for h in heads:
+        for t in ts:
+            for y in ys:
+                for x in xs:
+                    items.add(h * N + (t * Hp + y) * Wp + x)
+        items.update((h * N + g.integers(0, N, size=n_random)).tolist())
+    return np.array(sorted(items), dtype=np.int64)
+
+
 def gather_rows(t, items, N):
     """t [N][heads][dh] -> rows [len(items)][dh] for items h*N + n."""
     h, n = items // N, items % N

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from deformable_slide_attention_b200 import abi, inputs
-from tests.gpu_helpers import TOL, assert_close, items_of
+from tests.gpu_helpers import TOL, assert_close, edge_keys, items_of
 
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gpu_lib", "oracle_lib")]
 
@@ -53,7 +53,8 @@ def test_1080p_workload_full_size():
         hq, hk, hv, hdo = pick(q), pick(k), pick(v), pick(do)
         hoff = off[h:h + 1].contiguous().cpu()
         qi = items_of(1, w.N, 96, seed=40 + h)           # query tokens (head index 0 of the slice)
-        ki = items_of(1, w.N, 6, seed=50 + h)            # key tokens
+        # key tokens: the key tiles' frame, row and segment edges, and a few at random
+        ki = edge_keys(w.dims, (0,), seed=50 + h, n_random=8)
         r_out, r_lse = oracle.forward(hq, hk, hv, hoff, w.dims, w.window, qi)
         assert_close("out", out[qi, h].float().cpu().double().numpy(), r_out, tol)
         assert_close("lse", lse[h, qi].cpu().double().numpy(), r_lse, tol)

@@ -13,8 +13,8 @@ import torch
 
 import oracle
 from deformable_slide_attention_b200 import abi, inputs
-from tests.gpu_helpers import (TOL, assert_close, f64, full_parity, gather_rows, gpu_backward,
-                               gpu_forward, items_of, to_cuda)
+from tests.gpu_helpers import (TOL, assert_close, edge_keys, f64, full_parity, gather_rows,
+                               gpu_backward, gpu_forward, items_of, to_cuda)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gpu_lib", "oracle_lib")]
 
@@ -141,7 +141,7 @@ def test_small_bf16_workload_forward_full():
     full_parity(inp, w.dims, w.window, "bf16", backward=False)
 
 
-def _sampled(w, n_q, n_k, seed, backward):
+def _sampled(w, n_q, n_k, seed, backward, key_edges=False):
     inp = inputs.make(w, "cpu", with_dout=backward)
     d = to_cuda(inp)
     out, lse = gpu_forward(d, w.dims, w.window)
@@ -155,6 +155,8 @@ def _sampled(w, n_q, n_k, seed, backward):
         return
     dq, dk, dv, doff = gpu_backward(d, lse, w.dims, w.window)
     ki = items_of(w.heads, N, n_k, seed + 1)
+    if key_edges:  # the key tiles' frame, row and segment edges on the first and last heads
+        ki = np.union1d(ki, edge_keys(w.dims, (0, w.heads - 1), seed + 2))
     r_dq, r_doff, r_dk, r_dv = oracle.backward(inp["q"], inp["k"], inp["v"], inp["offsets"],
                                                inp["dout"], w.dims, w.window, qi, ki)
     assert_close("dq", gather_rows(dq, qi, N), r_dq, tol)
@@ -173,7 +175,7 @@ def test_720p_workload_forward_sampled():
 
 
 def test_720p_train_workload_sampled():
-    _sampled(inputs.BY_NAME["720p-train-bf16"], 256, 24, 33, True)
+    _sampled(inputs.BY_NAME["720p-train-bf16"], 256, 24, 33, True, key_edges=True)
 
 
 def test_forward_without_lse_matches():
