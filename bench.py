@@ -537,14 +537,23 @@ def main(argv=None):
                  "achieved_gbs": step_bytes / (ms / 1000.0) / 1e9,
                  "frac_of_hbm": step_bytes / (ms / 1000.0) / 1e9 / hbm}
 
-    # end to end through the public API with pinned host buffers
-    e2e = None
-    if not args.no_e2e:
-        e2e = e2e_leg(args, w, inp, abi, torch, dev, (ws, ws), world, (out, lse, dq, dk, dv, doff))
-
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
+
+    # end to end through the public API with pinned host buffers: the host copies are taken from
+    # the device inputs, then the device leg's tensors are released for the leg's own buffers
+    e2e = None
+    if not args.no_e2e:
+        host, why = e2e_host(w, inp, torch, dev, world)
+        del step
+        inp = q = k = v = off = do = out = lse = dq = dk = dv = doff = ws = None
+        torch.cuda.empty_cache()
+        if host is None:
+            e2e = {"value": None, "unit": UNIT, "skipped": why}
+        else:
+            e2e = e2e_leg(args, w, host, abi, torch, dev, world, code)
+            host.clear()
 
     line = {
         "metric": metric_of(w), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -569,14 +578,25 @@ def main(argv=None):
     return 0
 
 
-def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
-    """Same step through the public API with host inputs and results: every step copies the
-    inputs host->device from pinned buffers and reads every output (out, lse, dq, dk, dv,
-    doffsets) back device->host.  The inputs of step i+1 cross on their own stream while the
-    outputs of step i come back on a third one (the two directions of the link overlap); compute
-    waits for its inputs and for the previous read-back (the device output buffers are reused).
-    Host RAM holds the pinned inputs and a pinned read-back area: lse and doffsets each their own,
-    and one [N][heads][dh] buffer that out, dq, dk and dv pass through in turn."""
+def _cudart():
+    """The CUDA runtime library torch has loaded (for 2-D copies between pitched host and device
+    rows, which torch's copy_ does not issue)."""
+    import ctypes
+    lib = None
+    with open("/proc/self/maps") as f:
+        for line in f:
+            if "libcudart.so" in line:
+                lib = line.split()[-1]
+                break
+    rt = ctypes.CDLL(lib or "libcudart.so.12")
+    rt.cudaMemcpy2DAsync.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t,
+                                     ctypes.c_size_t, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+    rt.cudaMemcpy2DAsync.restype = ctypes.c_int
+    return rt
+
+
+def e2e_host(w, inp, torch, dev, world):
+    """Pinned host copies of the step's inputs and a pinned read-back area, or (None, reason)."""
     names_in = ("q", "k", "v", "offsets", "dout")
     in_bytes = sum(inp[n].numel() * inp[n].element_size() for n in names_in)
     row_bytes = inp["q"].numel() * inp["q"].element_size()
@@ -596,17 +616,16 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
         from deformable_slide_attention_b200 import ranks
         skip = ranks.max_over_ranks(1.0 if skip else 0.0, dev) > 0.5
     if skip:
-        return {"value": None, "unit": UNIT,
-                "skipped": f"host RAM share {avail >> 30} GiB per rank too small for "
-                           f"{(in_bytes + host_out_bytes) >> 30} GiB"}
-    h_in = {}
+        return None, (f"host RAM share {avail >> 30} GiB per rank too small for "
+                      f"{(in_bytes + host_out_bytes) >> 30} GiB")
+    host = {}
     try:
         for n in names_in:
-            h_in[n] = torch.empty(inp[n].shape, dtype=inp[n].dtype, pin_memory=True)
-            h_in[n].copy_(inp[n])
-        h_rows = torch.empty(inp["q"].shape, dtype=inp["q"].dtype, pin_memory=True)
-        h_lse = torch.empty((w.heads, w.N), dtype=torch.float32, pin_memory=True)
-        h_doff = torch.empty(inp["offsets"].shape, dtype=torch.float32, pin_memory=True)
+            host[n] = torch.empty(inp[n].shape, dtype=inp[n].dtype, pin_memory=True)
+            host[n].copy_(inp[n])
+        host["rows"] = torch.empty(inp["q"].shape, dtype=inp["q"].dtype, pin_memory=True)
+        host["lse"] = torch.empty((w.heads, w.N), dtype=torch.float32, pin_memory=True)
+        host["doff"] = torch.empty(inp["offsets"].shape, dtype=torch.float32, pin_memory=True)
     except RuntimeError as e:
         err = str(e)
     else:
@@ -616,48 +635,110 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
         from deformable_slide_attention_b200 import ranks
         failed = ranks.max_over_ranks(1.0 if failed else 0.0, dev) > 0.5
     if failed:
-        h_in.clear()
-        return {"value": None, "unit": UNIT,
-                "skipped": f"pinned host buffers unavailable: {err or 'on another rank'}"[:200]}
-    d_in = {n: inp[n] for n in names_in}
+        host.clear()
+        return None, f"pinned host buffers unavailable: {err or 'on another rank'}"[:200]
+    return host, None
+
+
+def e2e_leg(args, w, host, abi, torch, dev, world, code):
+    """The step through the public API with host inputs and results: every step copies all inputs
+    host->device from pinned buffers and reads every output (out, lse, dq, dk, dv, doffsets) back
+    device->host.  The step runs as G head groups (heads are independent), each a forward and a
+    backward call on [N][g][dh] tensors, through two slots of device buffers: group i+1's inputs
+    cross on their own stream (pitched 2-D copies out of the [N][heads][dh] host arrays) while
+    group i computes, and group i-1's outputs come back on a third stream, so both directions of
+    the link and the compute overlap.  Host RAM holds the pinned inputs and a read-back area: lse
+    and doffsets each their own, one [N][heads][dh] buffer that out, dq, dk and dv pass through in
+    turn."""
+    from deformable_slide_attention_b200 import ranks
+    s = 4 if w.dtype == "f32" else 2
+    H, N, dh = w.heads, w.N, w.dh
+    off_per_head = host["offsets"][0].numel()  # N*3, or N*K*3 with per-tap offsets
+
+    def ws_bytes(g):
+        if w.per_tap:
+            return abi.dsa3d_backward_taps_workspace_bytes(*w.dims, g, dh, *w.window, code)
+        return max(abi.dsa3d_forward_workspace_bytes(*w.dims, g, dh, *w.window, code),
+                   abi.dsa3d_backward_workspace_bytes(*w.dims, g, dh, *w.window, code))
+
+    def slot_bytes(g):
+        return 8 * N * g * dh * s + 2 * g * off_per_head * 4 + g * N * 4
+
+    free, _ = torch.cuda.mem_get_info(dev)
+    budget = free - (6 << 30)
+    # the largest group that fits, with four groups or more where the heads allow it (the first
+    # group's inputs and the last one's outputs are the pipeline's fill and drain)
+    g = 1
+    for cand in list(range(H // 4, 0, -1)) + list(range(H // 2, H // 4, -1)):
+        if cand >= 1 and H % cand == 0 and 2 * slot_bytes(cand) + ws_bytes(cand) <= budget:
+            g = cand
+            break
+    G = H // g
+    slots = []
+    for _ in range(2):
+        t = {n: torch.empty((N, g, dh), dtype=host["q"].dtype, device=dev)
+             for n in ("q", "k", "v", "dout", "out", "dq", "dk", "dv")}
+        t["offsets"] = torch.empty((g,) + tuple(host["offsets"].shape[1:]), dtype=torch.float32, device=dev)
+        t["doff"] = torch.empty_like(t["offsets"])
+        t["lse"] = torch.empty((g, N), dtype=torch.float32, device=dev)
+        slots.append(t)
+    ws = torch.empty(max(16, ws_bytes(g)), dtype=torch.uint8, device=dev)
+    rt = _cudart()
+    row_src, row_dst = H * dh * s, g * dh * s  # bytes per token row: host arrays, group slices
     compute = torch.cuda.current_stream(dev)
     s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     fwd_fn, bwd_fn = path_of(w, abi)
-    state = {"computed": None, "read": None}
-    d2h_bytes = [0]
+    ev = {"comp": [None, None], "out": [None, None]}
+    state = {"k": 0, "start": None, "last": None}
+    nbytes = {"h2d": 0, "d2h": 0}
 
-    def step():
-        # inputs: after the previous step's compute has finished reading them
-        if state["computed"] is not None:
-            s_h2d.wait_event(state["computed"])
+    def copy2d(dst, dpitch, src, spitch, width, stream, kind):
+        rc = rt.cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, N, kind, stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(f"cudaMemcpy2DAsync failed ({rc})")
+
+    def group(h0):
+        sl = state["k"] % 2
+        state["k"] += 1
+        t = slots[sl]
+        # inputs: the slot's previous group must have finished reading them
+        if ev["comp"][sl] is not None:
+            s_h2d.wait_event(ev["comp"][sl])
+        elif state["start"] is not None:
+            s_h2d.wait_event(state["start"])
+        for n in ("q", "k", "v", "dout"):
+            copy2d(t[n].data_ptr(), row_dst, host[n].data_ptr() + h0 * dh * s, row_src, row_dst, s_h2d, 1)
+            nbytes["h2d"] += N * row_dst
         with torch.cuda.stream(s_h2d):
-            for n in names_in:
-                d_in[n].copy_(h_in[n], non_blocking=True)
+            t["offsets"].copy_(host["offsets"][h0:h0 + g], non_blocking=True)
+        nbytes["h2d"] += t["offsets"].numel() * 4
         arrived = torch.cuda.Event()
         arrived.record(s_h2d)
         compute.wait_event(arrived)
-        if state["read"] is not None:  # the output buffers are free again
-            compute.wait_event(state["read"])
-        out, lse = fwd_fn(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], w.dims, w.window,
-                          out=outs[0], lse=outs[1], workspace=ws[0])
-        dq, dk, dv, doff = bwd_fn(d_in["q"], d_in["k"], d_in["v"], d_in["offsets"], lse,
-                                  d_in["dout"], w.dims, w.window, workspace=ws[1], grads=outs[2:])
+        if ev["out"][sl] is not None:  # the slot's outputs have been read back
+            compute.wait_event(ev["out"][sl])
+        fwd_fn(t["q"], t["k"], t["v"], t["offsets"], w.dims, w.window, out=t["out"], lse=t["lse"], workspace=ws)
+        bwd_fn(t["q"], t["k"], t["v"], t["offsets"], t["lse"], t["dout"], w.dims, w.window, workspace=ws,
+               grads=(t["dq"], t["dk"], t["dv"], t["doff"]))
         done = torch.cuda.Event()
         done.record(compute)
-        state["computed"] = done
+        ev["comp"][sl] = done
         s_d2h.wait_event(done)
-        nb = 0
+        for n in ("out", "dq", "dk", "dv"):
+            copy2d(host["rows"].data_ptr() + h0 * dh * s, row_src, t[n].data_ptr(), row_dst, row_dst, s_d2h, 2)
+            nbytes["d2h"] += N * row_dst
         with torch.cuda.stream(s_d2h):
-            for t in (out, dq, dk, dv):
-                h_rows.copy_(t, non_blocking=True)
-                nb += t.numel() * t.element_size()
-            h_lse.copy_(lse, non_blocking=True)
-            h_doff.copy_(doff, non_blocking=True)
-            nb += lse.numel() * 4 + doff.numel() * 4
+            host["lse"][h0:h0 + g].copy_(t["lse"], non_blocking=True)
+            host["doff"][h0:h0 + g].copy_(t["doff"], non_blocking=True)
+        nbytes["d2h"] += t["lse"].numel() * 4 + t["doff"].numel() * 4
         read = torch.cuda.Event()
         read.record(s_d2h)
-        state["read"] = read
-        d2h_bytes[0] = nb
+        ev["out"][sl] = read
+        state["last"] = read
+
+    def step():
+        for gi in range(G):
+            group(gi * g)
 
     step()
     torch.cuda.synchronize(dev)
@@ -666,19 +747,20 @@ def e2e_leg(args, w, inp, abi, torch, dev, ws, world, outs):
     t0.record(compute)
     begin = torch.cuda.Event()
     begin.record(compute)
-    state["computed"] = begin  # the first timed copies start after t0
+    ev["comp"] = [begin, begin]  # the first timed copies start after t0
+    nbytes["h2d"] = nbytes["d2h"] = 0
     for _ in range(steps):
         step()
-    compute.wait_event(state["read"])  # the last read-back is inside the timed region
+    compute.wait_event(state["last"])  # the last read-back is inside the timed region
     t1.record(compute)
     torch.cuda.synchronize(dev)
-    from deformable_slide_attention_b200 import ranks
     ms = ranks.max_over_ranks(t0.elapsed_time(t1) / steps, dev)
-    bi = sum(t.numel() * t.element_size() for t in h_in.values())
     return {"value": ranks.job_rate(w.N, world, ms), "unit": UNIT, "ms_per_step": ms, "steps": steps,
-            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": d2h_bytes[0],
+            "h2d_bytes_per_step": nbytes["h2d"] // steps, "d2h_bytes_per_step": nbytes["d2h"] // steps,
             "read_back": ["dk", "doffsets", "dq", "dv", "lse", "out"],
-            "overlap": "inputs of step i+1 (own stream) with the read-back of step i (own stream)"}
+            "head_groups": G, "heads_per_group": g,
+            "overlap": "per head group: inputs of group i+1 and outputs of group i-1 (own streams) "
+                       "while group i computes"}
 
 
 if __name__ == "__main__":
