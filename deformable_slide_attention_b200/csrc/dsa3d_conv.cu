@@ -4,6 +4,8 @@
 // translation unit of its own, next to dsa3d.cu; this file allocates no device memory.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <climits>
 #include <cstdint>
 
 #include "dsa3d.h"
@@ -70,13 +72,33 @@ dsa3d_status_t check_conv_shape(int F, int Hp, int Wp, int C, int kt, int kh, in
   return DSA3D_OK;
 }
 
+// The forward (and dX, flip = 1): the staged kernel when the kernel's taps fit in shared memory
+// and its grid in one dimension, else the global-memory one.
 template <typename T, int KW, typename OutT = T>
 dsa3d_status_t dwconv_launch_kw(const ConvGeo& g, const void* x, const float* w, const float* b,
                                 const void* add, void* y, int flip, cudaStream_t st) {
-  const int64_t items = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip) * (g.C / 2);
+  const int64_t units = (int64_t)g.F * ((g.Hp + 1) / 2) * ((g.Wp + kConvStrip - 1) / kConvStrip);
+  const int64_t groups = (g.C / 2 + kConvGroupPairs - 1) / kConvGroupPairs;
+  const int64_t sw_blocks = (units + kConvSwUnits - 1) / kConvSwUnits * groups;
+  const int K = g.kt * g.kh * KW;
+  const T* xt = static_cast<const T*>(x);
+  const OutT* at = static_cast<const OutT*>(add);
+  OutT* yt = static_cast<OutT*>(y);
+  if (K <= kConvSwMaxTaps && sw_blocks <= INT_MAX) {
+    // the staged kernel may take up to conv_sw_bytes(kConvSwMaxTaps) of dynamic shared memory
+    if (cudaFuncSetAttribute(dsa3d_dwconv3d_sw_kernel<T, KW, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)conv_sw_bytes(kConvSwMaxTaps)) != cudaSuccess)
+      return DSA3D_ERR_CUDA;
+    TimedLaunch tl(kKernDwconvSw, st);
+    dsa3d_dwconv3d_sw_kernel<T, KW, OutT><<<(unsigned)sw_blocks, kConvSwWarps * 32, conv_sw_bytes(K), st>>>(
+        xt, w, b, at, yt, g, flip);
+    const bool launched = cudaGetLastError() == cudaSuccess;
+    return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+  }
+  const int64_t items = units * (g.C / 2);
   TimedLaunch tl(kKernDwconv, st);
-  dsa3d_dwconv3d_kernel<T, KW, OutT><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
-      static_cast<const T*>(x), w, b, static_cast<const OutT*>(add), static_cast<OutT*>(y), g, flip);
+  dsa3d_dwconv3d_kernel<T, KW, OutT><<<grid_for(items, kConvFwdThreads, 8), kConvFwdThreads, 0, st>>>(
+      xt, w, b, at, yt, g, flip);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
 }
@@ -97,12 +119,13 @@ dsa3d_status_t dwconv_launch(const ConvGeo& g, const void* x, const float* w, co
   }
 }
 
-// Strips per dW work item: enough items to fill the GPU (about 8 per SM-slot), each long enough
-// that its final atomics are a small share of its work.
-int dw_strips_per_item(const ConvGeo& g) {
+// Strips per dW work item: about 8 items per resident thread (resident = the threads the GPU
+// holds at once), so that the items' last round leaves little of the GPU idle, each item long
+// enough that its final atomics are a small share of its work.
+int dw_strips_per_item(const ConvGeo& g, int64_t resident) {
   const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
   const int64_t lanes = (int64_t)(g.C / 2) * g.kt * g.kh;
-  const int64_t want_items = (int64_t)device_info().sms * 2048;
+  const int64_t want_items = resident * 8;
   int64_t chunks = want_items / (lanes > 0 ? lanes : 1);
   if (chunks < 1) chunks = 1;
   int64_t spi = (strips + chunks - 1) / chunks;
@@ -111,14 +134,21 @@ int dw_strips_per_item(const ConvGeo& g) {
   return (int)spi;
 }
 
+// dW and db: a grid of exactly the blocks the GPU holds at once, striding over the items.
 template <typename T, int KW, typename TD = T>
 dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* dy, float* dw,
                                    float* db, cudaStream_t st) {
-  const int spi = dw_strips_per_item(g);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dsa3d_dwconv3d_dw_kernel<T, KW, TD>,
+                                                    kConvDwThreads, 0) != cudaSuccess)
+    return DSA3D_ERR_CUDA;
+  if (per_sm < 1) per_sm = 1;
+  const int sms = std::max(device_info().sms, 1);
+  const int spi = dw_strips_per_item(g, (int64_t)sms * per_sm * kConvDwThreads);
   const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
   const int64_t items = (strips + spi - 1) / spi * g.kt * g.kh * (g.C / 2);
   TimedLaunch tl(kKernDwconvDw, st);
-  dsa3d_dwconv3d_dw_kernel<T, KW, TD><<<grid_for(items, kConvThreads, 8), kConvThreads, 0, st>>>(
+  dsa3d_dwconv3d_dw_kernel<T, KW, TD><<<grid_for(items, kConvDwThreads, per_sm), kConvDwThreads, 0, st>>>(
       static_cast<const T*>(x), static_cast<const TD*>(dy), dw, db, g, spi);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;

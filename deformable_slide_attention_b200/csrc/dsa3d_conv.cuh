@@ -10,37 +10,39 @@
 //
 // At the window's extent (3 x 9 x 9) the convolution does 2 C K flop per token for 4 C bytes of
 // bf16 traffic: about 120 flop per byte, so it is bound by the fp32 FMA pipes, not by HBM.  The
-// kernels block registers along x: a thread owns one channel pair (a 4-byte bf16x2 or 8-byte
-// float2 load, consecutive threads on consecutive pairs, so a warp's loads are one coalesced
-// 128- or 256-byte row segment) and a strip of kConvStrip outputs along x.  Per kernel row
-// (u, v) it loads the kConvStrip + KW - 1 input values of the row once and the KW weights of
-// the row once, and does kConvStrip * KW FMAs per channel from registers.
+// kernels block registers along x and y: a thread owns one channel pair (a 4-byte bf16x2 or
+// 8-byte float2 load, consecutive threads on consecutive pairs, so a warp's loads are one
+// coalesced 128- or 256-byte row segment) and, in the forward, two strips of kConvStrip outputs
+// along x in consecutive rows.  Per kernel plane u it loads each of the kh + 1 input rows'
+// kConvStrip + KW - 1 values once and each kernel row's KW weights once, and does
+// 2 kConvStrip KW FMAs per channel per kernel row from registers.
 //
-// The per-thread arithmetic (conv_strip, dw_row) is __host__ __device__ code so that a host
+// The per-thread arithmetic (conv_strip2, dw_row) is __host__ __device__ code so that a host
 // harness can run exactly these routines on the CPU.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-// Threads per block of the convolution kernels and, if DSA3D_CONV_MINB is defined, the minimum
-// resident blocks per SM asked of the compiler (a register cap).  Without it the launch bounds
-// name the block size alone (the compiler's own register choice).
-#ifndef DSA3D_CONV_THREADS
-#define DSA3D_CONV_THREADS 256
+// Threads per block of the two convolution kernels.  The forward/dX kernel holds two strips of
+// accumulators per thread (about 140 registers) and runs fastest in 128-thread blocks (at 1080p,
+// 68 x 120 x 256 tokens, 64 channels, 3 x 9 x 9: 326 ms at 128 threads, 412 ms at 256); the dW
+// kernel's per-thread work is lighter and 256 threads suit it (593 ms against 659 ms at 128).
+#ifndef DSA3D_CONV_FWD_THREADS
+#define DSA3D_CONV_FWD_THREADS 128
 #endif
-#ifdef DSA3D_CONV_MINB
-#define DSA3D_CONV_BOUNDS __launch_bounds__(DSA3D_CONV_THREADS, DSA3D_CONV_MINB)
-#else
-#define DSA3D_CONV_BOUNDS __launch_bounds__(DSA3D_CONV_THREADS)
+#ifndef DSA3D_CONV_DW_THREADS
+#define DSA3D_CONV_DW_THREADS 256
 #endif
 
 namespace dsa3d {
 
 constexpr int kConvStrip = 8;  // outputs along x per thread
-constexpr int kConvThreads = DSA3D_CONV_THREADS;
-static_assert(kConvThreads % 32 == 0 && kConvThreads >= 32 && kConvThreads <= 1024,
-              "DSA3D_CONV_THREADS: whole warps, at most 1024 threads per block");
+constexpr int kConvFwdThreads = DSA3D_CONV_FWD_THREADS;
+constexpr int kConvDwThreads = DSA3D_CONV_DW_THREADS;
+static_assert(kConvFwdThreads % 32 == 0 && kConvFwdThreads >= 32 && kConvFwdThreads <= 1024 &&
+                  kConvDwThreads % 32 == 0 && kConvDwThreads >= 32 && kConvDwThreads <= 1024,
+              "convolution blocks: whole warps, at most 1024 threads");
 
 struct ConvGeo {
   int F, Hp, Wp, C;
@@ -87,47 +89,135 @@ __host__ __device__ __forceinline__ float conv_ldw(const float* p) {
 #endif
 }
 
-// Convolution sums of channel pair c2 (channels 2 c2 and 2 c2 + 1) for the outputs
-// (t, y, x0 + i), i < kConvStrip, added into acc[i][0..1].  flip: use W[c][kt-1-u][kh-1-v][kw-1-w]
-// (the backward's dX).  KW = the kernel's width kw (a compile-time constant).
+// Where conv_strip2 reads the kernel: tap k (flattened (u, v, w)) of channel pair c2's two
+// channels.  ConvWGlobal reads W [C][kt][kh][kw] where it lies; its channels are K floats apart,
+// so a warp's 32 pairs touch 32 cache lines per tap.  ConvWShared reads a block's staged copy of
+// its channel group, tap-major (conv_sw_index), where a warp's pairs read one 256-byte row.
+struct ConvWGlobal {
+  const float* w0;  // W[2 c2][0][0][0]
+  int64_t K;        // taps per channel
+  __host__ __device__ __forceinline__ float2 operator()(int64_t k) const {
+    return make_float2(conv_ldw(w0 + k), conv_ldw(w0 + K + k));
+  }
+};
+
+constexpr int kConvGroupPairs = 32;                        // channel pairs per staged group: one per lane
+constexpr int kConvGroupStride = 2 * kConvGroupPairs + 2;  // floats per staged tap row (2 of padding)
+constexpr int kConvSwWarps = 4;                            // warps per block of the staged kernel
+constexpr int kConvSwUnits = 32;                           // (t, row pair, strip) units per block
+// Most taps staged: 387 x 66 x 4 B = 102 KB, two blocks per SM (3 x 9 x 9 = 243 taps take 64 KB:
+// three).  A larger kernel runs from global memory.
+constexpr int kConvSwMaxTaps = 387;
+static_assert(kConvSwUnits % kConvSwWarps == 0, "whole steps of the staged kernel's warps");
+
+// Channel cc (of the group's 2 kConvGroupPairs) at tap k in the staged copy.
+__host__ __device__ __forceinline__ int conv_sw_index(int k, int cc) { return k * kConvGroupStride + cc; }
+__host__ __device__ __forceinline__ size_t conv_sw_bytes(int K) {
+  return (size_t)K * kConvGroupStride * sizeof(float);
+}
+struct ConvWShared {
+  const float* s;  // the staged group + 2 * lane (8-byte aligned: the stride is even)
+  __host__ __device__ __forceinline__ float2 operator()(int64_t k) const {
+    return *reinterpret_cast<const float2*>(s + (int)k * kConvGroupStride);
+  }
+};
+
+// Unit (t, y0, x0) of the forward's work: output rows y0, y0 + 1 from column x0, strips fastest,
+// then row pairs, then frames.
+__host__ __device__ __forceinline__ void conv_unit(int64_t unit, int nxs, int nyp, int& t, int& y0,
+                                                   int& x0) {
+  x0 = (int)(unit % nxs) * kConvStrip;
+  const int64_t r = unit / nxs;
+  y0 = 2 * (int)(r % nyp);
+  t = (int)(r / nyp);
+}
+
+// The i-th unit (i < kConvSwUnits / kConvSwWarps) of warp `warp` in the staged kernel's block
+// slot `slot` of `slots` (= ceil(units / kConvSwUnits)).  The slots' units interleave: at step i
+// the resident blocks, whose slots are consecutive, work on one run of consecutive units (the
+// rows they read stay in L2), and every unit below slots * kConvSwUnits is visited once.
+__host__ __device__ __forceinline__ int64_t conv_sw_unit(int64_t slot, int64_t slots, int warp, int i) {
+  return ((int64_t)i * slots + slot) * kConvSwWarps + warp;
+}
+
+// Convolution sums of channel pair c2 (channels 2 c2 and 2 c2 + 1) for the two output strips
+// (t, y0 + r, x0 + i), r < 2, i < kConvStrip, added into acc[r][i][0..1].  For kernel plane u the
+// input rows y0 - r_h .. y0 + 1 + r_h are loaded once each, and kernel row v's weights once for
+// both outputs: output row y0 takes input row y0 + v - r_h, output row y0 + 1 the next one, so
+// the row loaded for one v is carried to the next.  flip: use W[c][kt-1-u][kh-1-v][kw-1-w] (the
+// backward's dX).  An output row past the volume (y0 + 1 = Hp) is computed and not stored.  KW =
+// the kernel's width kw (a compile-time constant); wget: where the weights are read
+// (ConvWGlobal, ConvWShared).
 template <typename T, int KW>
-__host__ __device__ __forceinline__ void conv_strip(const T* __restrict__ x, const float* __restrict__ w,
-                                                    const ConvGeo& g, int t, int y, int x0, int c2,
-                                                    bool flip, float (&acc)[kConvStrip][2]) {
-  const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2, rw = (KW - 1) / 2;
-  const int64_t K = (int64_t)g.kt * g.kh * KW;
-  const float* w0 = w + (int64_t)(2 * c2) * K;
-  const float* w1 = w0 + K;
+__host__ __device__ __forceinline__ void conv_load_row(const T* __restrict__ row, const ConvGeo& g, int x0,
+                                                       float (&a)[kConvStrip + KW - 1],
+                                                       float (&b)[kConvStrip + KW - 1]) {
+  const int rw = (KW - 1) / 2;
+#pragma unroll
+  for (int j = 0; j < kConvStrip + KW - 1; j++) {
+    const int xs = x0 - rw + j;
+    a[j] = b[j] = 0.f;
+    if (xs >= 0 && xs < g.Wp) conv_load2(row + (int64_t)xs * g.C, a[j], b[j]);
+  }
+}
+
+template <typename T, int KW, typename WGet>
+__host__ __device__ __forceinline__ void conv_strip2(const T* __restrict__ x, const WGet& wget,
+                                                     const ConvGeo& g, int t, int y0, int x0, int c2,
+                                                     bool flip, float (&acc)[2][kConvStrip][2]) {
+  constexpr int NJ = kConvStrip + KW - 1;
+  const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2;
+  const int64_t rstride = (int64_t)g.Wp * g.C;  // one token row
   for (int u = 0; u < g.kt; u++) {
     const int ts = t + u - rt;
     if (ts < 0 || ts >= g.F) continue;
+    const T* plane = x + (int64_t)ts * g.Hp * rstride + 2 * c2;
+    // the row under output row y0 for kernel row v (pa, pb), and the one under y0 + 1 (ca, cb)
+    float pa[NJ], pb[NJ], ca[NJ], cb[NJ];
+    {
+      const int ys = y0 - rh;
+      if (ys >= 0 && ys < g.Hp) {
+        conv_load_row<T, KW>(plane + ys * rstride, g, x0, pa, pb);
+      } else {
+#pragma unroll
+        for (int j = 0; j < NJ; j++) pa[j] = pb[j] = 0.f;
+      }
+    }
     for (int v = 0; v < g.kh; v++) {
-      const int ys = y + v - rh;
-      if (ys < 0 || ys >= g.Hp) continue;
+      const int ys = y0 + 1 + v - rh;
+      if (ys >= 0 && ys < g.Hp) {
+        conv_load_row<T, KW>(plane + ys * rstride, g, x0, ca, cb);
+      } else {
+#pragma unroll
+        for (int j = 0; j < NJ; j++) ca[j] = cb[j] = 0.f;
+      }
       // the kernel row's weights (flipped for the transposed convolution)
       const int64_t wrow = flip ? ((int64_t)(g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW
                                 : ((int64_t)u * g.kh + v) * KW;
       float wa[KW], wb[KW];
 #pragma unroll
       for (int j = 0; j < KW; j++) {
-        const int jj = flip ? KW - 1 - j : j;
-        wa[j] = conv_ldw(w0 + wrow + jj);
-        wb[j] = conv_ldw(w1 + wrow + jj);
+        const float2 p = wget(wrow + (flip ? KW - 1 - j : j));
+        wa[j] = p.x;
+        wb[j] = p.y;
       }
-      const T* row = x + ((int64_t)ts * g.Hp + ys) * g.Wp * g.C + 2 * c2;
       // input column x0 - rw + j feeds output x0 + i through tap j - i
 #pragma unroll
-      for (int j = 0; j < kConvStrip + KW - 1; j++) {
-        const int xs = x0 - rw + j;
-        float a = 0.f, b = 0.f;
-        if (xs >= 0 && xs < g.Wp) conv_load2(row + (int64_t)xs * g.C, a, b);
+      for (int j = 0; j < NJ; j++) {
 #pragma unroll
         for (int i = 0; i < kConvStrip; i++) {
           if (j - i >= 0 && j - i < KW) {
-            acc[i][0] = fmaf(wa[j - i], a, acc[i][0]);
-            acc[i][1] = fmaf(wb[j - i], b, acc[i][1]);
+            acc[0][i][0] = fmaf(wa[j - i], pa[j], acc[0][i][0]);
+            acc[0][i][1] = fmaf(wb[j - i], pb[j], acc[0][i][1]);
+            acc[1][i][0] = fmaf(wa[j - i], ca[j], acc[1][i][0]);
+            acc[1][i][1] = fmaf(wb[j - i], cb[j], acc[1][i][1]);
           }
         }
+      }
+#pragma unroll
+      for (int j = 0; j < NJ; j++) {
+        pa[j] = ca[j];
+        pb[j] = cb[j];
       }
     }
   }
@@ -135,13 +225,14 @@ __host__ __device__ __forceinline__ void conv_strip(const T* __restrict__ x, con
 
 // The contribution of one output strip (t, y, x0 .. x0 + kConvStrip - 1) to the weight gradient
 // of kernel row (u, v) of channel pair c2: dwr[j][k] += sum_i dY[(t, y, x0 + i)][2 c2 + k] *
-// X[(t + u - r_t, y + v - r_h, x0 + i + j - r_w)][2 c2 + k]; and, with db != nullptr, the bias
+// X[(t + u - r_t, y + v - r_h, x0 + i + j - r_w)][2 c2 + k]; and, if with_db, the bias
 // gradient db[k] += sum_i dY[...].  Outputs past the volume's last column are skipped.  TD: the
 // type of dY (the input's, or fp32 for the offset network's backward).
 template <typename T, int KW, typename TD = T>
 __host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const TD* __restrict__ dy,
                                                 const ConvGeo& g, int t, int y, int x0, int c2, int u,
-                                                int v, float (&dwr)[KW][2], float* db) {
+                                                int v, float (&dwr)[KW][2], bool with_db,
+                                                float (&db)[2]) {
   const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2, rw = (KW - 1) / 2;
   float ga[kConvStrip], gb[kConvStrip];
   const TD* dyrow = dy + ((int64_t)t * g.Hp + y) * g.Wp * g.C + 2 * c2;
@@ -149,7 +240,7 @@ __host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const T
   for (int i = 0; i < kConvStrip; i++) {
     ga[i] = gb[i] = 0.f;
     if (x0 + i < g.Wp) conv_load2(dyrow + (int64_t)(x0 + i) * g.C, ga[i], gb[i]);
-    if (db) {
+    if (with_db) {
       db[0] += ga[i];
       db[1] += gb[i];
     }
@@ -172,39 +263,47 @@ __host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const T
   }
 }
 
-#ifdef __CUDACC__
-// Y = conv(X) (+ bias) (+ add): one thread per (strip, channel pair), channel pairs fastest.
-// add (nullable) is added element by element (the attention output of Eq. 1; may equal y).
-// OutT: the output type (the input's, or fp32 for the offset network's first layer).
-template <typename T, int KW, typename OutT = T>
-__global__ void DSA3D_CONV_BOUNDS
-    dsa3d_dwconv3d_kernel(const T* __restrict__ x, const float* __restrict__ w,
-                          const float* __restrict__ bias, const OutT* add, OutT* y,
-                          const ConvGeo g, const int flip) {
-  const int pairs = g.C / 2;
+// One dW work item: kernel row r = u kh + v of channel pair c2 over strips [s0, s1) (strips
+// (t, y, x0) in token order, x0 fastest), added into dwr and, if with_db, db.  The strip
+// position advances by counters, with no division per strip.
+template <typename T, int KW, typename TD = T>
+__host__ __device__ __forceinline__ void dw_item(const T* __restrict__ x, const TD* __restrict__ dy,
+                                                 const ConvGeo& g, int64_t s0, int64_t s1, int r, int c2,
+                                                 float (&dwr)[KW][2], bool with_db, float (&db)[2]) {
+  if (s0 >= s1) return;
   const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
-  const int64_t items = (int64_t)g.F * g.Hp * nxs * pairs;
-  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
-       it += (int64_t)gridDim.x * blockDim.x) {
-    const int c2 = (int)(it % pairs);
-    const int64_t s = it / pairs;
-    const int x0 = (int)(s % nxs) * kConvStrip;
-    const int yy = (int)((s / nxs) % g.Hp);
-    const int t = (int)(s / ((int64_t)nxs * g.Hp));
-    float acc[kConvStrip][2];
-    const float b0 = bias ? __ldg(bias + 2 * c2) : 0.f, b1 = bias ? __ldg(bias + 2 * c2 + 1) : 0.f;
-#pragma unroll
-    for (int i = 0; i < kConvStrip; i++) {
-      acc[i][0] = b0;
-      acc[i][1] = b1;
+  const int u = r / g.kh, v = r % g.kh;
+  int xs = (int)(s0 % nxs);
+  const int64_t row = s0 / nxs;
+  int yy = (int)(row % g.Hp), t = (int)(row / g.Hp);
+  for (int64_t s = s0; s < s1; s++) {
+    dw_row<T, KW, TD>(x, dy, g, t, yy, xs * kConvStrip, c2, u, v, dwr, with_db, db);
+    if (++xs == nxs) {
+      xs = 0;
+      if (++yy == g.Hp) {
+        yy = 0;
+        t++;
+      }
     }
-    conv_strip<T, KW>(x, w, g, t, yy, x0, c2, flip != 0, acc);
-    const int64_t base = (((int64_t)t * g.Hp + yy) * g.Wp + x0) * g.C + 2 * c2;
+  }
+}
+
+#ifdef __CUDACC__
+// Writes the two strips acc (rows y0, y0 + 1 from column x0; channel pair c2), each element plus
+// add's (nullable; may equal y); rows and columns past the volume are not written.
+template <typename OutT>
+__device__ __forceinline__ void conv_store_strips(const float (&acc)[2][kConvStrip][2], const OutT* add,
+                                                  OutT* y, const ConvGeo& g, int t, int y0, int x0,
+                                                  int c2) {
+#pragma unroll
+  for (int r = 0; r < 2; r++) {
+    if (y0 + r >= g.Hp) break;
+    const int64_t base = (((int64_t)t * g.Hp + y0 + r) * g.Wp + x0) * g.C + 2 * c2;
 #pragma unroll
     for (int i = 0; i < kConvStrip; i++) {
       if (x0 + i >= g.Wp) break;
       const int64_t o = base + (int64_t)i * g.C;
-      float a = acc[i][0], b = acc[i][1];
+      float a = acc[r][i][0], b = acc[r][i][1];
       if (add) {
         float p, q;
         conv_load2(add + o, p, q);
@@ -216,10 +315,96 @@ __global__ void DSA3D_CONV_BOUNDS
   }
 }
 
+__device__ __forceinline__ void conv_acc_init(float (&acc)[2][kConvStrip][2], float b0, float b1) {
+#pragma unroll
+  for (int r = 0; r < 2; r++)
+#pragma unroll
+    for (int i = 0; i < kConvStrip; i++) {
+      acc[r][i][0] = b0;
+      acc[r][i][1] = b1;
+    }
+}
+
+// Y = conv(X) (+ bias) (+ add), the weights read from global memory (kernels of more than
+// kConvSwMaxTaps taps): one thread per (unit, channel pair), channel pairs fastest.  add
+// (nullable) is added element by element (the attention output of Eq. 1; may equal y).  OutT: the
+// output type (the input's, or fp32 for the offset network's first layer).
+template <typename T, int KW, typename OutT = T>
+__global__ void __launch_bounds__(kConvFwdThreads)
+    dsa3d_dwconv3d_kernel(const T* __restrict__ x, const float* __restrict__ w,
+                          const float* __restrict__ bias, const OutT* add, OutT* y,
+                          const ConvGeo g, const int flip) {
+  const int pairs = g.C / 2;
+  const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
+  const int nyp = (g.Hp + 1) / 2;  // row pairs
+  const int64_t items = (int64_t)g.F * nyp * nxs * pairs;
+  const int64_t K = (int64_t)g.kt * g.kh * KW;
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
+       it += (int64_t)gridDim.x * blockDim.x) {
+    const int c2 = (int)(it % pairs);
+    int t, y0, x0;
+    conv_unit(it / pairs, nxs, nyp, t, y0, x0);
+    float acc[2][kConvStrip][2];
+    conv_acc_init(acc, bias ? __ldg(bias + 2 * c2) : 0.f, bias ? __ldg(bias + 2 * c2 + 1) : 0.f);
+    conv_strip2<T, KW>(x, ConvWGlobal{w + 2 * c2 * K, K}, g, t, y0, x0, c2, flip != 0, acc);
+    conv_store_strips(acc, add, y, g, t, y0, x0, c2);
+  }
+}
+
+__device__ __forceinline__ void conv_cp_async4(float* dst, const float* src) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
+}
+
+// The same with the kernel staged in shared memory (at most kConvSwMaxTaps taps): a block owns
+// one group of kConvGroupPairs channel pairs (one per lane) and kConvSwUnits units of one slot
+// (conv_sw_unit), kConvSwUnits / kConvSwWarps per warp.  The group's weights are copied in once,
+// tap-major (conv_sw_index), before any unit runs; dynamic shared memory: conv_sw_bytes(kt kh
+// kw).  Blocks: group fastest, then slot.
+template <typename T, int KW, typename OutT = T>
+__global__ void __launch_bounds__(kConvSwWarps * 32)
+    dsa3d_dwconv3d_sw_kernel(const T* __restrict__ x, const float* __restrict__ w,
+                             const float* __restrict__ bias, const OutT* add, OutT* y,
+                             const ConvGeo g, const int flip) {
+  extern __shared__ __align__(16) float conv_sw[];
+  const int pairs = g.C / 2;
+  const unsigned groups = (unsigned)((pairs + kConvGroupPairs - 1) / kConvGroupPairs);
+  const int grp = (int)(blockIdx.x % groups);
+  const int64_t slot = blockIdx.x / groups;
+  const int K = g.kt * g.kh * KW;
+  const int c0 = 2 * kConvGroupPairs * grp;
+  const int nch = min(2 * kConvGroupPairs, g.C - c0);
+  const float* wg = w + (int64_t)c0 * K;  // the group's channels: nch x K contiguous floats
+  for (int cc = 0; cc < nch; cc++)
+    for (int k = threadIdx.x; k < K; k += blockDim.x)
+      conv_cp_async4(conv_sw + conv_sw_index(k, cc), wg + (int64_t)cc * K + k);
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c2 = kConvGroupPairs * grp + lane;
+  if (c2 >= pairs) return;
+  const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
+  const int nyp = (g.Hp + 1) / 2;
+  const int64_t units = (int64_t)g.F * nyp * nxs;
+  const int64_t slots = (units + kConvSwUnits - 1) / kConvSwUnits;
+  const ConvWShared ws{conv_sw + 2 * lane};
+  const float b0 = bias ? __ldg(bias + 2 * c2) : 0.f, b1 = bias ? __ldg(bias + 2 * c2 + 1) : 0.f;
+  for (int i = 0; i < kConvSwUnits / kConvSwWarps; i++) {
+    const int64_t unit = conv_sw_unit(slot, slots, warp, i);
+    if (unit >= units) break;  // later steps' units are larger still
+    int t, y0, x0;
+    conv_unit(unit, nxs, nyp, t, y0, x0);
+    float acc[2][kConvStrip][2];
+    conv_acc_init(acc, b0, b1);
+    conv_strip2<T, KW>(x, ws, g, t, y0, x0, c2, flip != 0, acc);
+    conv_store_strips(acc, add, y, g, t, y0, x0, c2);
+  }
+}
+
 // dW (and db): one thread per (channel pair, kernel row (u, v), range of strips); fp32 partial
 // sums reduced with atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).
 template <typename T, int KW, typename TD = T>
-__global__ void DSA3D_CONV_BOUNDS
+__global__ void __launch_bounds__(kConvDwThreads)
     dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const TD* __restrict__ dy, float* dweight,
                              float* dbias, const ConvGeo g, const int strips_per_item) {
   const int pairs = g.C / 2;
@@ -233,18 +418,13 @@ __global__ void DSA3D_CONV_BOUNDS
     const int c2 = (int)(it % pairs);
     const int r = (int)((it / pairs) % rows);
     const int64_t chunk = it / ((int64_t)pairs * rows);
-    const int u = r / g.kh, v = r % g.kh;
     float dwr[KW][2];
 #pragma unroll
     for (int j = 0; j < KW; j++) dwr[j][0] = dwr[j][1] = 0.f;
     float db[2] = {0.f, 0.f};
-    const int64_t s_end = (chunk + 1) * strips_per_item < strips ? (chunk + 1) * strips_per_item : strips;
-    for (int64_t s = chunk * strips_per_item; s < s_end; s++) {
-      const int x0 = (int)(s % nxs) * kConvStrip;
-      const int yy = (int)((s / nxs) % g.Hp);
-      const int t = (int)(s / ((int64_t)nxs * g.Hp));
-      dw_row<T, KW, TD>(x, dy, g, t, yy, x0, c2, u, v, dwr, r == 0 ? db : nullptr);
-    }
+    const int64_t s0 = chunk * strips_per_item;
+    dw_item<T, KW, TD>(x, dy, g, s0, s0 + strips_per_item < strips ? s0 + strips_per_item : strips, r,
+                       c2, dwr, r == 0, db);
     const int64_t K = (int64_t)rows * KW;
     float* d0 = dweight + (int64_t)(2 * c2) * K + (int64_t)r * KW;
 #pragma unroll

@@ -1,9 +1,13 @@
 // conv_host_harness.cu -- runs the depthwise-convolution kernels' per-thread routines
-// (conv_strip, dw_row from the library's dsa3d_conv.cuh) on the CPU, over every work item the
+// (conv_strip2, dw_item from the library's dsa3d_conv.cuh) on the CPU, over every work item the
 // GPU kernels would process, so that their indexing and arithmetic can be compared with the
 // oracle without a GPU.  Test infrastructure: built by tests/test_conv_host.py with nvcc as
 // host code; nothing here launches a kernel.
 #include <stdint.h>
+
+#include <algorithm>
+#include <cmath>
+#include <vector>
 
 #include "dsa3d_conv.cuh"
 #include "dsa3d_pointwise.cuh"
@@ -13,25 +17,70 @@ using namespace dsa3d;
 namespace {
 
 template <typename T, int KW>
+void store_strips(const float (&acc)[2][kConvStrip][2], const ConvGeo& g, int t, int y0, int x0, int c2,
+                  float* y) {
+  for (int r = 0; r < 2 && y0 + r < g.Hp; r++)
+    for (int i = 0; i < kConvStrip && x0 + i < g.Wp; i++) {
+      const int64_t o = (((int64_t)t * g.Hp + y0 + r) * g.Wp + x0 + i) * g.C + 2 * c2;
+      y[o] = acc[r][i][0];
+      y[o + 1] = acc[r][i][1];
+    }
+}
+
+void init_acc(float (&acc)[2][kConvStrip][2], const float* b, int c2) {
+  for (int r = 0; r < 2; r++)
+    for (int i = 0; i < kConvStrip; i++) {
+      acc[r][i][0] = b ? b[2 * c2] : 0.f;
+      acc[r][i][1] = b ? b[2 * c2 + 1] : 0.f;
+    }
+}
+
+// The forward as the library launches it: the staged kernel's blocks (channel group, run of
+// kConvSwUnits units), each staging its group's weights with conv_sw_index and its warps taking
+// the units in turn, when the kernel has at most kConvSwMaxTaps taps; else the global kernel's
+// items (unit, channel pair).
+template <typename T, int KW>
 void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, int flip, float* y) {
-  const int pairs = g.C / 2, nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
-  for (int t = 0; t < g.F; t++)
-    for (int yy = 0; yy < g.Hp; yy++)
-      for (int sx = 0; sx < nxs; sx++)
-        for (int c2 = 0; c2 < pairs; c2++) {
-          float acc[kConvStrip][2];
-          for (int i = 0; i < kConvStrip; i++) {
-            acc[i][0] = b ? b[2 * c2] : 0.f;
-            acc[i][1] = b ? b[2 * c2 + 1] : 0.f;
-          }
-          const int x0 = sx * kConvStrip;
-          conv_strip<T, KW>(x, w, g, t, yy, x0, c2, flip != 0, acc);
-          for (int i = 0; i < kConvStrip && x0 + i < g.Wp; i++) {
-            const int64_t o = (((int64_t)t * g.Hp + yy) * g.Wp + x0 + i) * g.C + 2 * c2;
-            y[o] = acc[i][0];
-            y[o + 1] = acc[i][1];
-          }
+  const int pairs = g.C / 2, nxs = (g.Wp + kConvStrip - 1) / kConvStrip, nyp = (g.Hp + 1) / 2;
+  const int64_t units = (int64_t)g.F * nyp * nxs;
+  const int K = g.kt * g.kh * KW;
+  float acc[2][kConvStrip][2];
+  int t, y0, x0;
+  if (K > kConvSwMaxTaps) {
+    for (int64_t it = 0; it < units * pairs; it++) {
+      const int c2 = (int)(it % pairs);
+      conv_unit(it / pairs, nxs, nyp, t, y0, x0);
+      init_acc(acc, b, c2);
+      conv_strip2<T, KW>(x, ConvWGlobal{w + 2 * c2 * (int64_t)K, K}, g, t, y0, x0, c2, flip != 0, acc);
+      store_strips<T, KW>(acc, g, t, y0, x0, c2, y);
+    }
+    return;
+  }
+  const int groups = (pairs + kConvGroupPairs - 1) / kConvGroupPairs;
+  const int64_t blocks = (units + kConvSwUnits - 1) / kConvSwUnits * groups;
+  std::vector<float> sw(conv_sw_bytes(K) / sizeof(float));
+  for (int64_t blk = 0; blk < blocks; blk++) {
+    const int grp = (int)(blk % groups);
+    const int64_t slot = blk / groups, slots = (units + kConvSwUnits - 1) / kConvSwUnits;
+    const int c0 = 2 * kConvGroupPairs * grp;
+    const int nch = std::min(2 * kConvGroupPairs, g.C - c0);
+    std::fill(sw.begin(), sw.end(), std::nanf(""));  // unstaged slots poison the result
+    for (int cc = 0; cc < nch; cc++)
+      for (int k = 0; k < K; k++) sw[conv_sw_index(k, cc)] = w[(int64_t)(c0 + cc) * K + k];
+    for (int warp = 0; warp < kConvSwWarps; warp++)
+      for (int lane = 0; lane < 32; lane++) {
+        const int c2 = kConvGroupPairs * grp + lane;
+        if (c2 >= pairs) continue;
+        for (int i = 0; i < kConvSwUnits / kConvSwWarps; i++) {
+          const int64_t unit = conv_sw_unit(slot, slots, warp, i);
+          if (unit >= units) break;
+          conv_unit(unit, nxs, nyp, t, y0, x0);
+          init_acc(acc, b, c2);
+          conv_strip2<T, KW>(x, ConvWShared{sw.data() + 2 * lane}, g, t, y0, x0, c2, flip != 0, acc);
+          store_strips<T, KW>(acc, g, t, y0, x0, c2, y);
         }
+      }
+  }
 }
 
 template <typename T, int KW, typename TD = T>
@@ -44,13 +93,9 @@ void dw_all(const T* x, const TD* dy, const ConvGeo& g, int strips_per_item, flo
       for (int c2 = 0; c2 < pairs; c2++) {
         float dwr[KW][2] = {};
         float dbl[2] = {0.f, 0.f};
-        const int64_t s_end = (chunk + 1) * strips_per_item < strips ? (chunk + 1) * strips_per_item : strips;
-        for (int64_t s = chunk * strips_per_item; s < s_end; s++) {
-          const int x0 = (int)(s % nxs) * kConvStrip;
-          const int yy = (int)((s / nxs) % g.Hp);
-          const int t = (int)(s / ((int64_t)nxs * g.Hp));
-          dw_row<T, KW, TD>(x, dy, g, t, yy, x0, c2, r / g.kh, r % g.kh, dwr, r == 0 ? dbl : nullptr);
-        }
+        const int64_t s0 = chunk * strips_per_item;
+        dw_item<T, KW, TD>(x, dy, g, s0, s0 + strips_per_item < strips ? s0 + strips_per_item : strips, r, c2,
+                           dwr, r == 0, dbl);
         for (int j = 0; j < KW; j++) {
           dw[(int64_t)(2 * c2) * K + (int64_t)r * KW + j] += dwr[j][0];
           dw[(int64_t)(2 * c2 + 1) * K + (int64_t)r * KW + j] += dwr[j][1];

@@ -1,9 +1,11 @@
-"""The depthwise-convolution kernels' per-thread routines (conv_strip, dw_row in
+"""The depthwise-convolution kernels' per-thread routines (conv_strip2, dw_row in
 csrc/dsa3d_conv.cuh) and the offset network's pointwise routine (pw_tile in
 csrc/dsa3d_pointwise.cuh), run on the CPU by a host harness over every work item the GPU kernels
-process, against the oracle's convolution (reading R9).  This checks their indexing, boundary
-handling, kernel flip and weight-gradient accumulation without a GPU; the GPU parity tests call
-the same code through the C ABI.
+process, against the oracle's convolution (reading R9).  The forward runs as the library launches
+it: the staged kernel's blocks (channel group, run of units, weights copied tap-major) or, past
+the staged tap limit, the global kernel's items.  This checks their indexing, boundary handling,
+kernel flip and weight-gradient accumulation without a GPU; the GPU parity tests call the same
+code through the C ABI.
 
 Tolerances: the routines accumulate in fp32 (the oracle in fp64): max-abs 1e-4 relative to the
 output scale for the forward and dX, 1e-4 relative for dW and db (sums over all tokens).
@@ -84,7 +86,12 @@ CASES = [((3, 5, 6), 4, (3, 3, 3)), ((2, 7, 19), 6, (3, 5, 9)), ((4, 3, 11), 2, 
          ((1, 4, 9), 8, (1, 3, 1)), ((5, 2, 17), 4, (5, 3, 7)), ((2, 3, 8), 2, (3, 3, 13))]
 
 
-@pytest.mark.parametrize("dims,C,window", CASES)
+# The forward's staged kernel: two runs of units and a last channel group of one pair (C = 66);
+# three groups, the last partial (C = 160); and 405 taps, past the staged limit (the global kernel).
+FWD_CASES = CASES + [((4, 7, 40), 66, (3, 5, 9)), ((3, 5, 6), 160, (3, 3, 3)), ((3, 5, 12), 4, (5, 9, 9))]
+
+
+@pytest.mark.parametrize("dims,C,window", FWD_CASES)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_forward_and_dx_match_oracle(harness, dims, C, window, dtype):
     g = torch.Generator().manual_seed(sum(dims) + C)

@@ -17,7 +17,10 @@ from tests.gpu_helpers import TOL, assert_close, f64
 pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gpu_lib", "oracle_lib")]
 
 CASES = [((3, 5, 6), 4, (3, 3, 3)), ((2, 7, 19), 6, (3, 5, 9)), ((4, 3, 11), 2, (1, 1, 15)),
-         ((1, 4, 9), 8, (1, 3, 1)), ((5, 2, 17), 4, (5, 3, 7)), ((4, 9, 16), 64, (3, 9, 9))]
+         ((1, 4, 9), 8, (1, 3, 1)), ((5, 2, 17), 4, (5, 3, 7)), ((4, 9, 16), 64, (3, 9, 9)),
+         # the forward's staged kernel over two runs of units with a last channel group of one pair,
+         # over three groups (the last partial), and a 405-tap kernel past its limit (global kernel)
+         ((4, 7, 40), 66, (3, 5, 9)), ((3, 5, 6), 160, (3, 3, 3)), ((3, 5, 12), 4, (5, 9, 9))]
 
 
 def _problem(dims, C, window, dtype, seed):
@@ -156,3 +159,45 @@ def test_layer_against_the_oracle_chain(dtype):
             oracle.dwconv3d_backward(x, w[0], dout.double().numpy().reshape(N, C), dims)[0])
     assert_close("dx", f64(grads["x"]), r_dx, 2 * TOL[dtype])
     assert_close("dq", f64(grads["q"]), r_dq, TOL[dtype])
+
+
+@pytest.mark.parametrize("name", ["720p-train-bf16", "1080p-long-bf16"])
+def test_full_size_sampled_channels(name):
+    """At a workload's full size, in the launch configuration bench.py times (C = heads x dh
+    channels, the window's kernel, y += conv(x) in place, then the backward): every output of
+    four channel pairs -- the first, the two on either side of the staged kernel's 64-channel
+    group boundary, and the last -- against the oracle run on those channels alone (depthwise: a
+    channel's outputs depend on that channel only).  bf16 outputs: |got - ref| <= 2^-8 |ref| +
+    1e-4 (half an ulp of the rounding, plus the fp32 sum); dweight, dbias: 1e-4 of the largest."""
+    from deformable_slide_attention_b200 import inputs
+    w = inputs.BY_NAME[name]
+    dev = torch.device("cuda", 0)
+    C, N, K = w.heads * w.dh, w.N, w.K
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    x, y, dy = (torch.empty((N, C), dtype=w.torch_dtype, device=dev) for _ in range(3))
+    for t in (x, y, dy):
+        inputs._fill_normal_chunked(t, gen)
+    weight = torch.empty((C, *w.window), dtype=torch.float32, device=dev)
+    weight.normal_(0.0, 1.0 / math.sqrt(K), generator=gen)
+    bias = torch.empty(C, dtype=torch.float32, device=dev).normal_(0.0, 1.0, generator=gen)
+    pairs = [0, 31, 32, C // 2 - 1]
+    add = {p: f64(y[:, 2 * p:2 * p + 2]) for p in pairs}
+    abi.dwconv3d(x, weight, bias, w.dims, add=y, out=y)
+    gx, gw, gb = abi.dwconv3d_backward(x, weight, dy, w.dims)
+    torch.cuda.synchronize()
+    try:
+        for p in pairs:
+            sl = slice(2 * p, 2 * p + 2)
+            xs, ws, bs = x[:, sl].cpu(), weight[sl].cpu(), bias[sl].cpu()
+            ref_y = oracle.dwconv3d(xs, ws, bs, w.dims) + add[p]
+            rx, rw, rb = oracle.dwconv3d_backward(xs, ws, f64(dy[:, sl]), w.dims)
+            for nm, got, ref in (("y", f64(y[:, sl]), ref_y), ("dx", f64(gx[:, sl]), rx)):
+                err = np.abs(got - ref) - 2.0 ** -8 * np.abs(ref)
+                assert err.max() <= 1e-4, (name, p, nm, float(err.max()))
+            for nm, got, ref in (("dweight", f64(gw[sl]), rw), ("dbias", f64(gb[sl]), rb)):
+                err = np.abs(got - ref).max()
+                assert err <= 1e-4 * max(1.0, np.abs(ref).max()), (name, p, nm, err)
+    finally:
+        del x, y, dy, gx, gw, gb
+        torch.cuda.empty_cache()
