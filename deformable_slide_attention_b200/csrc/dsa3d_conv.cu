@@ -119,22 +119,18 @@ dsa3d_status_t dwconv_launch(const ConvGeo& g, const void* x, const float* w, co
   }
 }
 
-// Strips per dW work item: about 8 items per resident thread (resident = the threads the GPU
+// dY frames per dW work item: about 8 items per resident thread (resident = the threads the GPU
 // holds at once), so that the items' last round leaves little of the GPU idle, each item long
 // enough that its final atomics are a small share of its work.
-int dw_strips_per_item(const ConvGeo& g, int64_t resident) {
-  const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
-  const int64_t lanes = (int64_t)(g.C / 2) * g.kt * g.kh;
-  const int64_t want_items = resident * 8;
-  int64_t chunks = want_items / (lanes > 0 ? lanes : 1);
-  if (chunks < 1) chunks = 1;
-  int64_t spi = (strips + chunks - 1) / chunks;
-  if (spi < 1) spi = 1;
-  if (spi > (1 << 20)) spi = 1 << 20;
-  return (int)spi;
+int dw_frames_per_item(const ConvGeo& g, int64_t resident) {
+  const int64_t per_run = dw_items(g, g.F);  // items when one run covers every frame
+  int64_t runs = resident * 8 / (per_run > 0 ? per_run : 1);
+  if (runs < 1) runs = 1;
+  if (runs > g.F) runs = g.F;
+  return (int)((g.F + runs - 1) / runs);
 }
 
-// dW and db: a grid of exactly the blocks the GPU holds at once, striding over the items.
+// dW and db: a grid of at most the blocks the GPU holds at once, striding over the items.
 template <typename T, int KW, typename TD = T>
 dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* dy, float* dw,
                                    float* db, cudaStream_t st) {
@@ -144,12 +140,11 @@ dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* 
     return DSA3D_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
   const int sms = std::max(device_info().sms, 1);
-  const int spi = dw_strips_per_item(g, (int64_t)sms * per_sm * kConvDwThreads);
-  const int64_t strips = g.N / g.Wp * ((g.Wp + kConvStrip - 1) / kConvStrip);
-  const int64_t items = (strips + spi - 1) / spi * g.kt * g.kh * (g.C / 2);
+  const int fpi = dw_frames_per_item(g, (int64_t)sms * per_sm * kConvDwThreads);
+  const int64_t items = dw_items(g, fpi);
   TimedLaunch tl(kKernDwconvDw, st);
   dsa3d_dwconv3d_dw_kernel<T, KW, TD><<<grid_for(items, kConvDwThreads, per_sm), kConvDwThreads, 0, st>>>(
-      static_cast<const T*>(x), static_cast<const TD*>(dy), dw, db, g, spi);
+      static_cast<const T*>(x), static_cast<const TD*>(dy), dw, db, g, fpi);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
 }

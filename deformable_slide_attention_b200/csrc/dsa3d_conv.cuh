@@ -15,24 +15,26 @@
 // coalesced 128- or 256-byte row segment) and, in the forward, two strips of kConvStrip outputs
 // along x in consecutive rows.  Per kernel plane u it loads each of the kh + 1 input rows'
 // kConvStrip + KW - 1 values once and each kernel row's KW weights once, and does
-// 2 kConvStrip KW FMAs per channel per kernel row from registers.
+// 2 kConvStrip KW FMAs per channel per kernel row from registers; in the forward the pair's two
+// channels share one packed fp32x2 FMA (conv_fma2).
 //
-// The per-thread arithmetic (conv_strip2, dw_row) is __host__ __device__ code so that a host
+// The per-thread arithmetic (conv_strip2, dw_walk) is __host__ __device__ code so that a host
 // harness can run exactly these routines on the CPU.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-// Threads per block of the two convolution kernels.  The forward/dX kernel holds two strips of
-// accumulators per thread (about 140 registers) and runs fastest in 128-thread blocks (at 1080p,
-// 68 x 120 x 256 tokens, 64 channels, 3 x 9 x 9: 326 ms at 128 threads, 412 ms at 256); the dW
-// kernel's per-thread work is lighter and 256 threads suit it (593 ms against 659 ms at 128).
+// Threads per block of the global-memory forward kernel and of the dW kernel (the staged forward
+// has its own, kConvSwWarps warps).  Both hold many accumulators per thread (about 165 and 235
+// registers): 128-thread blocks let the SM hold three and two of them.  At 1080p (256 x 68 x 120
+// tokens, 4096 channels, 3 x 9 x 9) the global-memory forward took 326 ms at 128 threads and 412
+// ms at 256.
 #ifndef DSA3D_CONV_FWD_THREADS
 #define DSA3D_CONV_FWD_THREADS 128
 #endif
 #ifndef DSA3D_CONV_DW_THREADS
-#define DSA3D_CONV_DW_THREADS 256
+#define DSA3D_CONV_DW_THREADS 128
 #endif
 
 namespace dsa3d {
@@ -88,6 +90,23 @@ __host__ __device__ __forceinline__ float conv_ldw(const float* p) {
   return *p;
 #endif
 }
+template <typename T>
+__host__ __device__ __forceinline__ float2 conv_load2v(const T* p) {
+  float2 v;
+  conv_load2(p, v.x, v.y);
+  return v;
+}
+
+// acc += w * x on both channels of a pair: on the GPU one fma.rn.f32x2 (one issue slot for the
+// two FMAs), each lane rounded as fmaf rounds it.
+__host__ __device__ __forceinline__ void conv_fma2(float2& acc, const float2 w, const float2 x) {
+#ifdef __CUDA_ARCH__
+  acc = __ffma2_rn(w, x, acc);
+#else
+  acc.x = fmaf(w.x, x.x, acc.x);
+  acc.y = fmaf(w.y, x.y, acc.y);
+#endif
+}
 
 // Where conv_strip2 reads the kernel: tap k (flattened (u, v, w)) of channel pair c2's two
 // channels.  ConvWGlobal reads W [C][kt][kh][kw] where it lies; its channels are K floats apart,
@@ -141,30 +160,29 @@ __host__ __device__ __forceinline__ int64_t conv_sw_unit(int64_t slot, int64_t s
 }
 
 // Convolution sums of channel pair c2 (channels 2 c2 and 2 c2 + 1) for the two output strips
-// (t, y0 + r, x0 + i), r < 2, i < kConvStrip, added into acc[r][i][0..1].  For kernel plane u the
-// input rows y0 - r_h .. y0 + 1 + r_h are loaded once each, and kernel row v's weights once for
-// both outputs: output row y0 takes input row y0 + v - r_h, output row y0 + 1 the next one, so
+// (t, y0 + r, x0 + i), r < 2, i < kConvStrip, added into acc[r][i] (.x: channel 2 c2, .y: 2 c2 +
+// 1).  For kernel plane u the input rows y0 - r_h .. y0 + 1 + r_h are loaded once each, and
+// kernel row v's weights once for both outputs: output row y0 takes input row y0 + v - r_h, output row y0 + 1 the next one, so
 // the row loaded for one v is carried to the next.  flip: use W[c][kt-1-u][kh-1-v][kw-1-w] (the
 // backward's dX).  An output row past the volume (y0 + 1 = Hp) is computed and not stored.  KW =
 // the kernel's width kw (a compile-time constant); wget: where the weights are read
 // (ConvWGlobal, ConvWShared).
 template <typename T, int KW>
 __host__ __device__ __forceinline__ void conv_load_row(const T* __restrict__ row, const ConvGeo& g, int x0,
-                                                       float (&a)[kConvStrip + KW - 1],
-                                                       float (&b)[kConvStrip + KW - 1]) {
+                                                       float2 (&a)[kConvStrip + KW - 1]) {
   const int rw = (KW - 1) / 2;
 #pragma unroll
   for (int j = 0; j < kConvStrip + KW - 1; j++) {
     const int xs = x0 - rw + j;
-    a[j] = b[j] = 0.f;
-    if (xs >= 0 && xs < g.Wp) conv_load2(row + (int64_t)xs * g.C, a[j], b[j]);
+    a[j] = make_float2(0.f, 0.f);
+    if (xs >= 0 && xs < g.Wp) a[j] = conv_load2v(row + (int64_t)xs * g.C);
   }
 }
 
 template <typename T, int KW, typename WGet>
 __host__ __device__ __forceinline__ void conv_strip2(const T* __restrict__ x, const WGet& wget,
                                                      const ConvGeo& g, int t, int y0, int x0, int c2,
-                                                     bool flip, float (&acc)[2][kConvStrip][2]) {
+                                                     bool flip, float2 (&acc)[2][kConvStrip]) {
   constexpr int NJ = kConvStrip + KW - 1;
   const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2;
   const int64_t rstride = (int64_t)g.Wp * g.C;  // one token row
@@ -172,119 +190,164 @@ __host__ __device__ __forceinline__ void conv_strip2(const T* __restrict__ x, co
     const int ts = t + u - rt;
     if (ts < 0 || ts >= g.F) continue;
     const T* plane = x + (int64_t)ts * g.Hp * rstride + 2 * c2;
-    // the row under output row y0 for kernel row v (pa, pb), and the one under y0 + 1 (ca, cb)
-    float pa[NJ], pb[NJ], ca[NJ], cb[NJ];
+    // the row under output row y0 for kernel row v (pr), and the one under y0 + 1 (cr)
+    float2 pr[NJ], cr[NJ];
     {
       const int ys = y0 - rh;
       if (ys >= 0 && ys < g.Hp) {
-        conv_load_row<T, KW>(plane + ys * rstride, g, x0, pa, pb);
+        conv_load_row<T, KW>(plane + ys * rstride, g, x0, pr);
       } else {
 #pragma unroll
-        for (int j = 0; j < NJ; j++) pa[j] = pb[j] = 0.f;
+        for (int j = 0; j < NJ; j++) pr[j] = make_float2(0.f, 0.f);
       }
     }
     for (int v = 0; v < g.kh; v++) {
       const int ys = y0 + 1 + v - rh;
       if (ys >= 0 && ys < g.Hp) {
-        conv_load_row<T, KW>(plane + ys * rstride, g, x0, ca, cb);
+        conv_load_row<T, KW>(plane + ys * rstride, g, x0, cr);
       } else {
 #pragma unroll
-        for (int j = 0; j < NJ; j++) ca[j] = cb[j] = 0.f;
+        for (int j = 0; j < NJ; j++) cr[j] = make_float2(0.f, 0.f);
       }
       // the kernel row's weights (flipped for the transposed convolution)
       const int64_t wrow = flip ? ((int64_t)(g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW
                                 : ((int64_t)u * g.kh + v) * KW;
-      float wa[KW], wb[KW];
+      float2 w[KW];
 #pragma unroll
-      for (int j = 0; j < KW; j++) {
-        const float2 p = wget(wrow + (flip ? KW - 1 - j : j));
-        wa[j] = p.x;
-        wb[j] = p.y;
-      }
+      for (int j = 0; j < KW; j++) w[j] = wget(wrow + (flip ? KW - 1 - j : j));
       // input column x0 - rw + j feeds output x0 + i through tap j - i
 #pragma unroll
       for (int j = 0; j < NJ; j++) {
 #pragma unroll
         for (int i = 0; i < kConvStrip; i++) {
           if (j - i >= 0 && j - i < KW) {
-            acc[0][i][0] = fmaf(wa[j - i], pa[j], acc[0][i][0]);
-            acc[0][i][1] = fmaf(wb[j - i], pb[j], acc[0][i][1]);
-            acc[1][i][0] = fmaf(wa[j - i], ca[j], acc[1][i][0]);
-            acc[1][i][1] = fmaf(wb[j - i], cb[j], acc[1][i][1]);
+            conv_fma2(acc[0][i], w[j - i], pr[j]);
+            conv_fma2(acc[1][i], w[j - i], cr[j]);
           }
         }
       }
 #pragma unroll
-      for (int j = 0; j < NJ; j++) {
-        pa[j] = ca[j];
-        pb[j] = cb[j];
-      }
+      for (int j = 0; j < NJ; j++) pr[j] = cr[j];
     }
   }
 }
 
-// The contribution of one output strip (t, y, x0 .. x0 + kConvStrip - 1) to the weight gradient
-// of kernel row (u, v) of channel pair c2: dwr[j][k] += sum_i dY[(t, y, x0 + i)][2 c2 + k] *
-// X[(t + u - r_t, y + v - r_h, x0 + i + j - r_w)][2 c2 + k]; and, if with_db, the bias
-// gradient db[k] += sum_i dY[...].  Outputs past the volume's last column are skipped.  TD: the
-// type of dY (the input's, or fp32 for the offset network's backward).
-template <typename T, int KW, typename TD = T>
-__host__ __device__ __forceinline__ void dw_row(const T* __restrict__ x, const TD* __restrict__ dy,
-                                                const ConvGeo& g, int t, int y, int x0, int c2, int u,
-                                                int v, float (&dwr)[KW][2], bool with_db,
-                                                float (&db)[2]) {
-  const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2, rw = (KW - 1) / 2;
-  float ga[kConvStrip], gb[kConvStrip];
-  const TD* dyrow = dy + ((int64_t)t * g.Hp + y) * g.Wp * g.C + 2 * c2;
+// dW and db.  A work item is channel pair c2, kernel plane u, kDwRows kernel rows v0 .. v0 +
+// kDwRows - 1 (those below kh), the strip column from x0 and a run of dY frames.  For each frame
+// it walks the input rows ys of frame t + u - r_t downward: input row ys meets dY row
+// ys - v + r_h for each kernel row v, so a step loads one input row (kConvStrip + KW - 1 values)
+// and one new dY strip (kConvStrip values), carries the other kDwRows - 1 dY strips (moved one
+// register slot per step), and does kDwRows kConvStrip KW FMAs per channel.
+constexpr int kDwRows = 3;
+
+// Work item `it` of the dW kernel: channel pairs fastest, then kernel-row groups, planes, strip
+// columns and runs of frames_per_item dY frames [t0, t1).
+__host__ __device__ __forceinline__ void dw_decode(int64_t it, const ConvGeo& g, int frames_per_item, int& c2,
+                                                   int& u, int& v0, int& x0, int& t0, int& t1) {
+  const int pairs = g.C / 2, groups = (g.kh + kDwRows - 1) / kDwRows;
+  const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
+  c2 = (int)(it % pairs);
+  int64_t r = it / pairs;
+  v0 = (int)(r % groups) * kDwRows;
+  r /= groups;
+  u = (int)(r % g.kt);
+  r /= g.kt;
+  x0 = (int)(r % nxs) * kConvStrip;
+  t0 = (int)(r / nxs) * frames_per_item;
+  t1 = t0 + frames_per_item < g.F ? t0 + frames_per_item : g.F;
+}
+
+__host__ __device__ __forceinline__ int64_t dw_items(const ConvGeo& g, int frames_per_item) {
+  const int groups = (g.kh + kDwRows - 1) / kDwRows;
+  const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
+  return (int64_t)(g.C / 2) * groups * g.kt * nxs * ((g.F + frames_per_item - 1) / frames_per_item);
+}
+
+// dY strip (row y of the frame at dplane, columns x0 .. x0 + kConvStrip - 1) of the pair as fp32;
+// zeros for a row outside the frame or columns past its last.
+template <typename TD>
+__host__ __device__ __forceinline__ void dw_load_dy(const TD* __restrict__ dplane, const ConvGeo& g, int y,
+                                                    int x0, float2 (&d)[kConvStrip]) {
+  const bool in = y >= 0 && y < g.Hp;
+  const TD* row = dplane + ((int64_t)y * g.Wp + x0) * g.C;
 #pragma unroll
   for (int i = 0; i < kConvStrip; i++) {
-    ga[i] = gb[i] = 0.f;
-    if (x0 + i < g.Wp) conv_load2(dyrow + (int64_t)(x0 + i) * g.C, ga[i], gb[i]);
-    if (with_db) {
-      db[0] += ga[i];
-      db[1] += gb[i];
-    }
+    d[i] = make_float2(0.f, 0.f);
+    if (in && x0 + i < g.Wp) d[i] = conv_load2v(row + (int64_t)i * g.C);
   }
-  const int ts = t + u - rt, ys = y + v - rh;
-  if (ts < 0 || ts >= g.F || ys < 0 || ys >= g.Hp) return;
-  const T* row = x + ((int64_t)ts * g.Hp + ys) * g.Wp * g.C + 2 * c2;
+}
+
+// Step ys of the walk: the carried dY strips move one slot down (slot i holds the dY row that
+// kernel row v0 + i meets, ys - v0 - i + r_h), slot 0 takes the new row ys - v0 + r_h, and the
+// input row ys is loaded and multiplied into every kernel row's sums.
+template <typename T, int KW, typename TD>
+__host__ __device__ __forceinline__ void dw_step(const T* __restrict__ xplane, const TD* __restrict__ dplane,
+                                                 const ConvGeo& g, int ys, int v0, int x0,
+                                                 float2 (&d)[kDwRows][kConvStrip],
+                                                 float2 (&dwr)[kDwRows][KW]) {
+  constexpr int NJ = kConvStrip + KW - 1;
+  const int rh = (g.kh - 1) / 2;
 #pragma unroll
-  for (int j = 0; j < kConvStrip + KW - 1; j++) {
-    const int xs = x0 - rw + j;
-    float a = 0.f, b = 0.f;
-    if (xs >= 0 && xs < g.Wp) conv_load2(row + (int64_t)xs * g.C, a, b);
+  for (int i = kDwRows - 1; i > 0; i--)
 #pragma unroll
-    for (int i = 0; i < kConvStrip; i++) {
-      if (j - i >= 0 && j - i < KW) {
-        dwr[j - i][0] = fmaf(ga[i], a, dwr[j - i][0]);
-        dwr[j - i][1] = fmaf(gb[i], b, dwr[j - i][1]);
+    for (int k = 0; k < kConvStrip; k++) d[i][k] = d[i - 1][k];
+  dw_load_dy<TD>(dplane, g, ys - v0 + rh, x0, d[0]);
+  float2 a[NJ];
+  conv_load_row<T, KW>(xplane + (int64_t)ys * g.Wp * g.C, g, x0, a);
+#pragma unroll
+  for (int i = 0; i < kDwRows; i++) {
+    if (v0 + i >= g.kh) break;
+    // input column x0 - r_w + j meets output x0 + k through tap j - k
+#pragma unroll
+    for (int j = 0; j < NJ; j++) {
+#pragma unroll
+      for (int k = 0; k < kConvStrip; k++) {
+        if (j - k >= 0 && j - k < KW) {  // scalar FMAs: the packed form took more registers here
+          dwr[i][j - k].x = fmaf(d[i][k].x, a[j].x, dwr[i][j - k].x);
+          dwr[i][j - k].y = fmaf(d[i][k].y, a[j].y, dwr[i][j - k].y);
+        }
       }
     }
   }
 }
 
-// One dW work item: kernel row r = u kh + v of channel pair c2 over strips [s0, s1) (strips
-// (t, y, x0) in token order, x0 fastest), added into dwr and, if with_db, db.  The strip
-// position advances by counters, with no division per strip.
+// One work item's sums: dwr[i][w] (.x, .y: channel 2 c2 + e, e = 0, 1) += sum over its frames t,
+// rows y and columns x0 + k of dY[(t, y, x0 + k)][2 c2 + e] * X[(t + u - r_t, y + v0 + i - r_h,
+// x0 + k + w - r_w)][2 c2 + e]; and, if with_db, db[e] += the sum of its dY strips over every row
+// of its frames.  Outputs past
+// the volume's last column are skipped; X and dY are zero outside the volume.  TD: the type of
+// dY (the input's, or fp32 for the offset network's backward).
 template <typename T, int KW, typename TD = T>
-__host__ __device__ __forceinline__ void dw_item(const T* __restrict__ x, const TD* __restrict__ dy,
-                                                 const ConvGeo& g, int64_t s0, int64_t s1, int r, int c2,
-                                                 float (&dwr)[KW][2], bool with_db, float (&db)[2]) {
-  if (s0 >= s1) return;
-  const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
-  const int u = r / g.kh, v = r % g.kh;
-  int xs = (int)(s0 % nxs);
-  const int64_t row = s0 / nxs;
-  int yy = (int)(row % g.Hp), t = (int)(row / g.Hp);
-  for (int64_t s = s0; s < s1; s++) {
-    dw_row<T, KW, TD>(x, dy, g, t, yy, xs * kConvStrip, c2, u, v, dwr, with_db, db);
-    if (++xs == nxs) {
-      xs = 0;
-      if (++yy == g.Hp) {
-        yy = 0;
-        t++;
+__host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const TD* __restrict__ dy,
+                                                 const ConvGeo& g, int c2, int u, int v0, int x0, int t0,
+                                                 int t1, float2 (&dwr)[kDwRows][KW], bool with_db,
+                                                 float (&db)[2]) {
+  const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2;
+  const int64_t fstride = (int64_t)g.Hp * g.Wp * g.C;  // one frame
+  for (int t = t0; t < t1; t++) {
+    const TD* dplane = dy + t * fstride + 2 * c2;
+    if (with_db) {
+      for (int y = 0; y < g.Hp; y++) {
+        float2 d[kConvStrip];
+        dw_load_dy<TD>(dplane, g, y, x0, d);
+#pragma unroll
+        for (int k = 0; k < kConvStrip; k++) {
+          db[0] += d[k].x;
+          db[1] += d[k].y;
+        }
       }
     }
+    const int ts = t + u - rt;
+    if (ts < 0 || ts >= g.F) continue;
+    const T* xplane = x + ts * fstride + 2 * c2;
+    // the input rows that meet some dY row through kernel rows v0 .. v0 + kDwRows - 1
+    const int ys0 = v0 - rh > 0 ? v0 - rh : 0;
+    const int ys1 = g.Hp - 1 + v0 + kDwRows - 1 - rh < g.Hp - 1 ? g.Hp - 1 + v0 + kDwRows - 1 - rh : g.Hp - 1;
+    // slot i - 1 holds, before the first step moves it to slot i, kernel row v0 + i's dY row
+    float2 d[kDwRows][kConvStrip];
+#pragma unroll
+    for (int i = 1; i < kDwRows; i++) dw_load_dy<TD>(dplane, g, ys0 - v0 - i + rh, x0, d[i - 1]);
+    for (int ys = ys0; ys <= ys1; ys++) dw_step<T, KW, TD>(xplane, dplane, g, ys, v0, x0, d, dwr);
   }
 }
 
@@ -292,7 +355,7 @@ __host__ __device__ __forceinline__ void dw_item(const T* __restrict__ x, const 
 // Writes the two strips acc (rows y0, y0 + 1 from column x0; channel pair c2), each element plus
 // add's (nullable; may equal y); rows and columns past the volume are not written.
 template <typename OutT>
-__device__ __forceinline__ void conv_store_strips(const float (&acc)[2][kConvStrip][2], const OutT* add,
+__device__ __forceinline__ void conv_store_strips(const float2 (&acc)[2][kConvStrip], const OutT* add,
                                                   OutT* y, const ConvGeo& g, int t, int y0, int x0,
                                                   int c2) {
 #pragma unroll
@@ -303,7 +366,7 @@ __device__ __forceinline__ void conv_store_strips(const float (&acc)[2][kConvStr
     for (int i = 0; i < kConvStrip; i++) {
       if (x0 + i >= g.Wp) break;
       const int64_t o = base + (int64_t)i * g.C;
-      float a = acc[r][i][0], b = acc[r][i][1];
+      float a = acc[r][i].x, b = acc[r][i].y;
       if (add) {
         float p, q;
         conv_load2(add + o, p, q);
@@ -315,14 +378,11 @@ __device__ __forceinline__ void conv_store_strips(const float (&acc)[2][kConvStr
   }
 }
 
-__device__ __forceinline__ void conv_acc_init(float (&acc)[2][kConvStrip][2], float b0, float b1) {
+__device__ __forceinline__ void conv_acc_init(float2 (&acc)[2][kConvStrip], float b0, float b1) {
 #pragma unroll
   for (int r = 0; r < 2; r++)
 #pragma unroll
-    for (int i = 0; i < kConvStrip; i++) {
-      acc[r][i][0] = b0;
-      acc[r][i][1] = b1;
-    }
+    for (int i = 0; i < kConvStrip; i++) acc[r][i] = make_float2(b0, b1);
 }
 
 // Y = conv(X) (+ bias) (+ add), the weights read from global memory (kernels of more than
@@ -344,7 +404,7 @@ __global__ void __launch_bounds__(kConvFwdThreads)
     const int c2 = (int)(it % pairs);
     int t, y0, x0;
     conv_unit(it / pairs, nxs, nyp, t, y0, x0);
-    float acc[2][kConvStrip][2];
+    float2 acc[2][kConvStrip];
     conv_acc_init(acc, bias ? __ldg(bias + 2 * c2) : 0.f, bias ? __ldg(bias + 2 * c2 + 1) : 0.f);
     conv_strip2<T, KW>(x, ConvWGlobal{w + 2 * c2 * K, K}, g, t, y0, x0, c2, flip != 0, acc);
     conv_store_strips(acc, add, y, g, t, y0, x0, c2);
@@ -394,45 +454,45 @@ __global__ void __launch_bounds__(kConvSwWarps * 32)
     if (unit >= units) break;  // later steps' units are larger still
     int t, y0, x0;
     conv_unit(unit, nxs, nyp, t, y0, x0);
-    float acc[2][kConvStrip][2];
+    float2 acc[2][kConvStrip];
     conv_acc_init(acc, b0, b1);
     conv_strip2<T, KW>(x, ws, g, t, y0, x0, c2, flip != 0, acc);
     conv_store_strips(acc, add, y, g, t, y0, x0, c2);
   }
 }
 
-// dW (and db): one thread per (channel pair, kernel row (u, v), range of strips); fp32 partial
-// sums reduced with atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).
+// dW (and db): one thread per work item (dw_decode, dw_walk); fp32 partial sums added with
+// atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).  The bias gradient is
+// summed by the items of plane 0 and the first kernel-row group.
 template <typename T, int KW, typename TD = T>
 __global__ void __launch_bounds__(kConvDwThreads)
     dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const TD* __restrict__ dy, float* dweight,
-                             float* dbias, const ConvGeo g, const int strips_per_item) {
-  const int pairs = g.C / 2;
-  const int rows = g.kt * g.kh;
-  const int nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
-  const int64_t strips = (int64_t)g.F * g.Hp * nxs;
-  const int64_t chunks = (strips + strips_per_item - 1) / strips_per_item;
-  const int64_t items = chunks * rows * pairs;
+                             float* dbias, const ConvGeo g, const int frames_per_item) {
+  const int64_t items = dw_items(g, frames_per_item);
+  const int64_t K = (int64_t)g.kt * g.kh * KW;
   for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
        it += (int64_t)gridDim.x * blockDim.x) {
-    const int c2 = (int)(it % pairs);
-    const int r = (int)((it / pairs) % rows);
-    const int64_t chunk = it / ((int64_t)pairs * rows);
-    float dwr[KW][2];
+    int c2, u, v0, x0, t0, t1;
+    dw_decode(it, g, frames_per_item, c2, u, v0, x0, t0, t1);
+    float2 dwr[kDwRows][KW];
 #pragma unroll
-    for (int j = 0; j < KW; j++) dwr[j][0] = dwr[j][1] = 0.f;
+    for (int i = 0; i < kDwRows; i++)
+#pragma unroll
+      for (int j = 0; j < KW; j++) dwr[i][j] = make_float2(0.f, 0.f);
     float db[2] = {0.f, 0.f};
-    const int64_t s0 = chunk * strips_per_item;
-    dw_item<T, KW, TD>(x, dy, g, s0, s0 + strips_per_item < strips ? s0 + strips_per_item : strips, r,
-                       c2, dwr, r == 0, db);
-    const int64_t K = (int64_t)rows * KW;
-    float* d0 = dweight + (int64_t)(2 * c2) * K + (int64_t)r * KW;
+    const bool with_db = u == 0 && v0 == 0;
+    dw_walk<T, KW, TD>(x, dy, g, c2, u, v0, x0, t0, t1, dwr, with_db, db);
 #pragma unroll
-    for (int j = 0; j < KW; j++) {
-      atomicAdd(d0 + j, dwr[j][0]);
-      atomicAdd(d0 + K + j, dwr[j][1]);
+    for (int i = 0; i < kDwRows; i++) {
+      if (v0 + i >= g.kh) break;
+      float* d0 = dweight + (int64_t)(2 * c2) * K + ((int64_t)u * g.kh + v0 + i) * KW;
+#pragma unroll
+      for (int j = 0; j < KW; j++) {
+        atomicAdd(d0 + j, dwr[i][j].x);
+        atomicAdd(d0 + K + j, dwr[i][j].y);
+      }
     }
-    if (r == 0) {
+    if (with_db) {
       atomicAdd(dbias + 2 * c2, db[0]);
       atomicAdd(dbias + 2 * c2 + 1, db[1]);
     }

@@ -1,5 +1,5 @@
 // conv_host_harness.cu -- runs the depthwise-convolution kernels' per-thread routines
-// (conv_strip2, dw_item from the library's dsa3d_conv.cuh) on the CPU, over every work item the
+// (conv_strip2, dw_walk from the library's dsa3d_conv.cuh) on the CPU, over every work item the
 // GPU kernels would process, so that their indexing and arithmetic can be compared with the
 // oracle without a GPU.  Test infrastructure: built by tests/test_conv_host.py with nvcc as
 // host code; nothing here launches a kernel.
@@ -17,22 +17,20 @@ using namespace dsa3d;
 namespace {
 
 template <typename T, int KW>
-void store_strips(const float (&acc)[2][kConvStrip][2], const ConvGeo& g, int t, int y0, int x0, int c2,
+void store_strips(const float2 (&acc)[2][kConvStrip], const ConvGeo& g, int t, int y0, int x0, int c2,
                   float* y) {
   for (int r = 0; r < 2 && y0 + r < g.Hp; r++)
     for (int i = 0; i < kConvStrip && x0 + i < g.Wp; i++) {
       const int64_t o = (((int64_t)t * g.Hp + y0 + r) * g.Wp + x0 + i) * g.C + 2 * c2;
-      y[o] = acc[r][i][0];
-      y[o + 1] = acc[r][i][1];
+      y[o] = acc[r][i].x;
+      y[o + 1] = acc[r][i].y;
     }
 }
 
-void init_acc(float (&acc)[2][kConvStrip][2], const float* b, int c2) {
+void init_acc(float2 (&acc)[2][kConvStrip], const float* b, int c2) {
   for (int r = 0; r < 2; r++)
-    for (int i = 0; i < kConvStrip; i++) {
-      acc[r][i][0] = b ? b[2 * c2] : 0.f;
-      acc[r][i][1] = b ? b[2 * c2 + 1] : 0.f;
-    }
+    for (int i = 0; i < kConvStrip; i++)
+      acc[r][i] = b ? make_float2(b[2 * c2], b[2 * c2 + 1]) : make_float2(0.f, 0.f);
 }
 
 // The forward as the library launches it: the staged kernel's blocks (channel group, run of
@@ -44,7 +42,7 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
   const int pairs = g.C / 2, nxs = (g.Wp + kConvStrip - 1) / kConvStrip, nyp = (g.Hp + 1) / 2;
   const int64_t units = (int64_t)g.F * nyp * nxs;
   const int K = g.kt * g.kh * KW;
-  float acc[2][kConvStrip][2];
+  float2 acc[2][kConvStrip];
   int t, y0, x0;
   if (K > kConvSwMaxTaps) {
     for (int64_t it = 0; it < units * pairs; it++) {
@@ -84,27 +82,26 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
 }
 
 template <typename T, int KW, typename TD = T>
-void dw_all(const T* x, const TD* dy, const ConvGeo& g, int strips_per_item, float* dw, float* db) {
-  const int pairs = g.C / 2, rows = g.kt * g.kh, nxs = (g.Wp + kConvStrip - 1) / kConvStrip;
-  const int64_t strips = (int64_t)g.F * g.Hp * nxs, K = (int64_t)rows * KW;
-  const int64_t chunks = (strips + strips_per_item - 1) / strips_per_item;
-  for (int64_t chunk = 0; chunk < chunks; chunk++)
-    for (int r = 0; r < rows; r++)
-      for (int c2 = 0; c2 < pairs; c2++) {
-        float dwr[KW][2] = {};
-        float dbl[2] = {0.f, 0.f};
-        const int64_t s0 = chunk * strips_per_item;
-        dw_item<T, KW, TD>(x, dy, g, s0, s0 + strips_per_item < strips ? s0 + strips_per_item : strips, r, c2,
-                           dwr, r == 0, dbl);
-        for (int j = 0; j < KW; j++) {
-          dw[(int64_t)(2 * c2) * K + (int64_t)r * KW + j] += dwr[j][0];
-          dw[(int64_t)(2 * c2 + 1) * K + (int64_t)r * KW + j] += dwr[j][1];
-        }
-        if (r == 0) {
-          db[2 * c2] += dbl[0];
-          db[2 * c2 + 1] += dbl[1];
-        }
+void dw_all(const T* x, const TD* dy, const ConvGeo& g, int frames_per_item, float* dw, float* db) {
+  const int64_t K = (int64_t)g.kt * g.kh * KW;
+  for (int64_t it = 0; it < dw_items(g, frames_per_item); it++) {
+    int c2, u, v0, x0, t0, t1;
+    dw_decode(it, g, frames_per_item, c2, u, v0, x0, t0, t1);
+    float2 dwr[kDwRows][KW] = {};
+    float dbl[2] = {0.f, 0.f};
+    const bool with_db = u == 0 && v0 == 0;
+    dw_walk<T, KW, TD>(x, dy, g, c2, u, v0, x0, t0, t1, dwr, with_db, dbl);
+    for (int i = 0; i < kDwRows && v0 + i < g.kh; i++)
+      for (int j = 0; j < KW; j++) {
+        const int64_t o = (int64_t)(2 * c2) * K + ((int64_t)u * g.kh + v0 + i) * KW + j;
+        dw[o] += dwr[i][j].x;
+        dw[o + K] += dwr[i][j].y;
       }
+    if (with_db) {
+      db[2 * c2] += dbl[0];
+      db[2 * c2 + 1] += dbl[1];
+    }
+  }
 }
 
 template <template <typename, int> class Fn, typename T, typename... A>
@@ -129,14 +126,14 @@ struct Fwd {
 };
 template <typename T, int KW>
 struct DwMixed {  // dY in fp32 (the offset network's backward)
-  static void run(const void* x, const void* dy, ConvGeo g, int spi, float* dw, float* db) {
-    dw_all<T, KW, float>(static_cast<const T*>(x), static_cast<const float*>(dy), g, spi, dw, db);
+  static void run(const void* x, const void* dy, ConvGeo g, int fpi, float* dw, float* db) {
+    dw_all<T, KW, float>(static_cast<const T*>(x), static_cast<const float*>(dy), g, fpi, dw, db);
   }
 };
 template <typename T, int KW>
 struct Dw {
-  static void run(const void* x, const void* dy, ConvGeo g, int spi, float* dw, float* db) {
-    dw_all<T, KW>(static_cast<const T*>(x), static_cast<const T*>(dy), g, spi, dw, db);
+  static void run(const void* x, const void* dy, ConvGeo g, int fpi, float* dw, float* db) {
+    dw_all<T, KW>(static_cast<const T*>(x), static_cast<const T*>(dy), g, fpi, dw, db);
   }
 };
 
@@ -162,20 +159,20 @@ int conv_host_forward(int io, const void* x, const float* w, const float* b, int
 
 // dw [C][kt][kh][kw], db [C]: fp32, accumulated into (zero them first).
 int conv_host_dw(int io, const void* x, const void* dy, int F, int Hp, int Wp, int C, int kt, int kh,
-                 int kw, int strips_per_item, float* dw, float* db) {
-  if (C % 2 || strips_per_item < 1) return -1;
+                 int kw, int frames_per_item, float* dw, float* db) {
+  if (C % 2 || frames_per_item < 1) return -1;
   const ConvGeo g = geo(F, Hp, Wp, C, kt, kh, kw);
-  return io ? by_kw<Dw, __nv_bfloat16>(kw, x, dy, g, strips_per_item, dw, db)
-            : by_kw<Dw, float>(kw, x, dy, g, strips_per_item, dw, db);
+  return io ? by_kw<Dw, __nv_bfloat16>(kw, x, dy, g, frames_per_item, dw, db)
+            : by_kw<Dw, float>(kw, x, dy, g, frames_per_item, dw, db);
 }
 
 // dW with x in the I/O type (io) and dY in fp32.
 int conv_host_dw_mixed(int io, const void* x, const float* dy, int F, int Hp, int Wp, int C, int kt,
-                       int kh, int kw, int strips_per_item, float* dw, float* db) {
-  if (C % 2 || strips_per_item < 1) return -1;
+                       int kh, int kw, int frames_per_item, float* dw, float* db) {
+  if (C % 2 || frames_per_item < 1) return -1;
   const ConvGeo g = geo(F, Hp, Wp, C, kt, kh, kw);
-  return io ? by_kw<DwMixed, __nv_bfloat16>(kw, x, (const void*)dy, g, strips_per_item, dw, db)
-            : by_kw<DwMixed, float>(kw, x, (const void*)dy, g, strips_per_item, dw, db);
+  return io ? by_kw<DwMixed, __nv_bfloat16>(kw, x, (const void*)dy, g, frames_per_item, dw, db)
+            : by_kw<DwMixed, float>(kw, x, (const void*)dy, g, frames_per_item, dw, db);
 }
 
 // The pointwise layer's backward over every work item of its two kernels: dz [N][C] written;

@@ -1,4 +1,4 @@
-"""The depthwise-convolution kernels' per-thread routines (conv_strip2, dw_row in
+"""The depthwise-convolution kernels' per-thread routines (conv_strip2, dw_walk in
 csrc/dsa3d_conv.cuh) and the offset network's pointwise routine (pw_tile in
 csrc/dsa3d_pointwise.cuh), run on the CPU by a host harness over every work item the GPU kernels
 process, against the oracle's convolution (reading R9).  The forward runs as the library launches
@@ -71,13 +71,13 @@ def host_forward(lib, x, w, b, dims, flip=False):
     return y
 
 
-def host_dw(lib, x, dy, dims, window, strips_per_item):
+def host_dw(lib, x, dy, dims, window, frames_per_item):
     io, xa = _io(x)
     _, da = _io(dy)
     C = x.shape[1]
     dw = np.zeros((C, *window), np.float32)
     db = np.zeros(C, np.float32)
-    rc = lib.conv_host_dw(io, _ptr(xa), _ptr(da), *dims, C, *window, strips_per_item, _ptr(dw), _ptr(db))
+    rc = lib.conv_host_dw(io, _ptr(xa), _ptr(da), *dims, C, *window, frames_per_item, _ptr(dw), _ptr(db))
     assert rc == 0
     return dw, db
 
@@ -89,6 +89,8 @@ CASES = [((3, 5, 6), 4, (3, 3, 3)), ((2, 7, 19), 6, (3, 5, 9)), ((4, 3, 11), 2, 
 # The forward's staged kernel: two runs of units and a last channel group of one pair (C = 66);
 # three groups, the last partial (C = 160); and 405 taps, past the staged limit (the global kernel).
 FWD_CASES = CASES + [((4, 7, 40), 66, (3, 5, 9)), ((3, 5, 6), 160, (3, 3, 3)), ((3, 5, 12), 4, (5, 9, 9))]
+# dW's kernel-row groups of three: kh = 7 (3 + 3 + 1) and kh = 9 as well
+DW_CASES = FWD_CASES + [((3, 4, 10), 4, (3, 7, 3))]
 
 
 @pytest.mark.parametrize("dims,C,window", FWD_CASES)
@@ -109,15 +111,15 @@ def test_forward_and_dx_match_oracle(harness, dims, C, window, dtype):
     assert np.abs(dx - ref_dx).max() <= 1e-4 * max(1.0, np.abs(ref_dx).max())
 
 
-@pytest.mark.parametrize("dims,C,window", CASES)
-@pytest.mark.parametrize("strips_per_item", [1, 3, 64])
-def test_weight_gradient_matches_oracle(harness, dims, C, window, strips_per_item):
+@pytest.mark.parametrize("dims,C,window", DW_CASES)
+@pytest.mark.parametrize("frames_per_item", [1, 2, 64])
+def test_weight_gradient_matches_oracle(harness, dims, C, window, frames_per_item):
     g = torch.Generator().manual_seed(7 + sum(window))
     N = math.prod(dims)
     x = torch.randn(N, C, generator=g).to(torch.bfloat16)
     dy = torch.randn(N, C, generator=g).to(torch.bfloat16)
     w = torch.randn(C, *window, generator=g)
-    dw, db = host_dw(harness, x, dy, dims, window, strips_per_item)
+    dw, db = host_dw(harness, x, dy, dims, window, frames_per_item)
     _, ref_dw, ref_db = oracle.dwconv3d_backward(x, w, dy.double().numpy(), dims)
     assert np.abs(dw - ref_dw).max() <= 1e-4 * max(1.0, np.abs(ref_dw).max())
     assert np.abs(db - ref_db).max() <= 1e-4 * max(1.0, np.abs(ref_db).max())
