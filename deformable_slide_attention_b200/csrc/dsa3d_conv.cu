@@ -134,16 +134,21 @@ int dw_frames_per_item(const ConvGeo& g, int64_t resident) {
 template <typename T, int KW, typename TD = T>
 dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* dy, float* dw,
                                    float* db, cudaStream_t st) {
+  // a staging ring per warp
+  const size_t smem = (size_t)(kConvDwThreads / 32) * DwRing<T, TD, KW>::warp_bytes();
+  if (cudaFuncSetAttribute(dsa3d_dwconv3d_dw_kernel<T, KW, TD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return DSA3D_ERR_CUDA;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dsa3d_dwconv3d_dw_kernel<T, KW, TD>,
-                                                    kConvDwThreads, 0) != cudaSuccess)
+                                                    kConvDwThreads, smem) != cudaSuccess)
     return DSA3D_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
   const int sms = std::max(device_info().sms, 1);
   const int fpi = dw_frames_per_item(g, (int64_t)sms * per_sm * kConvDwThreads);
   const int64_t items = dw_items(g, fpi);
   TimedLaunch tl(kKernDwconvDw, st);
-  dsa3d_dwconv3d_dw_kernel<T, KW, TD><<<grid_for(items, kConvDwThreads, per_sm), kConvDwThreads, 0, st>>>(
+  dsa3d_dwconv3d_dw_kernel<T, KW, TD><<<grid_for(items, kConvDwThreads, per_sm), kConvDwThreads, smem, st>>>(
       static_cast<const T*>(x), static_cast<const TD*>(dy), dw, db, g, fpi);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;

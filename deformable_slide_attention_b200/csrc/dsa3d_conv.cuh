@@ -277,23 +277,126 @@ __host__ __device__ __forceinline__ void dw_load_dy(const TD* __restrict__ dplan
   }
 }
 
-// Step ys of the walk: the carried dY strips move one slot down (slot i holds the dY row that
-// kernel row v0 + i meets, ys - v0 - i + r_h), slot 0 takes the new row ys - v0 + r_h, and the
-// input row ys is loaded and multiplied into every kernel row's sums.
+// The raw channel pair of T as the dW walk stages it (4 bytes for bf16, 8 for fp32), and its
+// fp32 values.
+template <typename T>
+struct ConvRaw;
+template <>
+struct ConvRaw<float> {
+  using type = float2;
+};
+template <>
+struct ConvRaw<__nv_bfloat16> {
+  using type = unsigned;
+};
+__host__ __device__ __forceinline__ float2 conv_unpack(float2 r) { return r; }
+__host__ __device__ __forceinline__ float2 conv_unpack(unsigned u) {
+  union {
+    unsigned i;
+    float f;
+  } lo, hi;
+  lo.i = u << 16;
+  hi.i = u & 0xffff0000u;
+  return make_float2(lo.f, hi.f);
+}
+
+// *dst = *src (a raw pair), or zeros when !ok.  On the GPU an asynchronous copy into shared
+// memory (cp.async; with !ok it copies no bytes, zero-fills, and src is only a valid address),
+// complete once dw_wait has covered its group.
+template <typename R>
+__host__ __device__ __forceinline__ void dw_copy(R* dst, const R* src, bool ok) {
+#ifdef __CUDA_ARCH__
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  const int n = ok ? (int)sizeof(R) : 0;
+  if constexpr (sizeof(R) == 8)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(d), "l"(src), "r"(n) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src), "r"(n) : "memory");
+#else
+  *dst = ok ? *src : R{};
+#endif
+}
+__host__ __device__ __forceinline__ void dw_commit() {
+#ifdef __CUDA_ARCH__
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+#endif
+}
+// Wait until at most N of this thread's committed copy groups are still in flight.
+template <int N>
+__host__ __device__ __forceinline__ void dw_wait() {
+#ifdef __CUDA_ARCH__
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+#endif
+}
+
+constexpr int kDwStages = 3;  // steps of the dW walk in its staging ring: fetched two steps ahead
+
+// One lane's staging ring of the dW walk: kDwStages steps of an input row (NJ raw pairs) and a
+// dY strip (kConvStrip raw pairs).  A warp's lanes are interleaved (entry e of a lane at
+// [e * 32]), so the warp's copies and reads of one entry are one contiguous row of shared memory,
+// and each lane reads back only what it copied itself.
+template <typename T, typename TD, int KW>
+struct DwRing {
+  static constexpr int NJ = kConvStrip + KW - 1;
+  using XR = typename ConvRaw<T>::type;
+  using DR = typename ConvRaw<TD>::type;
+  XR* x;  // the lane's entry (stage 0, column 0): [stage][NJ], stride 32
+  DR* d;  // the lane's entry (stage 0, strip output 0): [stage][kConvStrip], stride 32
+  __host__ __device__ static constexpr size_t x_bytes() { return (size_t)kDwStages * NJ * 32 * sizeof(XR); }
+  __host__ __device__ static constexpr size_t warp_bytes() { return x_bytes() + (size_t)kDwStages * kConvStrip * 32 * sizeof(DR); }
+  // the ring of lane `lane` in the warp's region at base (8-byte aligned)
+  __host__ __device__ static DwRing at(unsigned char* base, int lane) {
+    DwRing r;
+    r.x = reinterpret_cast<XR*>(base) + lane;
+    r.d = reinterpret_cast<DR*>(base + x_bytes()) + lane;
+    return r;
+  }
+};
+
+// Fetch step ys of the walk into ring stage st: input row ys (columns x0 - r_w .. x0 + kConvStrip
+// + r_w - 1) of the frame at xplane and dY row ys - v0 + r_h (columns x0 .. x0 + kConvStrip - 1)
+// of the frame at dplane; zeros outside the frames.
+template <typename T, typename TD, int KW>
+__host__ __device__ __forceinline__ void dw_fetch(const DwRing<T, TD, KW>& r, int st, const T* xplane,
+                                                  const TD* dplane, const ConvGeo& g, int ys, int v0, int x0) {
+  using R = DwRing<T, TD, KW>;
+  using XR = typename R::XR;
+  using DR = typename R::DR;
+  const int rw = (KW - 1) / 2, rh = (g.kh - 1) / 2;
+  const T* xrow = xplane + (int64_t)ys * g.Wp * g.C;
+#pragma unroll
+  for (int j = 0; j < R::NJ; j++) {
+    const int xs = x0 - rw + j;
+    const bool ok = xs >= 0 && xs < g.Wp;
+    dw_copy(r.x + (st * R::NJ + j) * 32, reinterpret_cast<const XR*>(ok ? xrow + (int64_t)xs * g.C : xplane), ok);
+  }
+  const int y = ys - v0 + rh;
+  const bool yin = y >= 0 && y < g.Hp;
+  const TD* drow = yin ? dplane + ((int64_t)y * g.Wp + x0) * g.C : dplane;
+#pragma unroll
+  for (int k = 0; k < kConvStrip; k++) {
+    const bool ok = yin && x0 + k < g.Wp;
+    dw_copy(r.d + (st * kConvStrip + k) * 32, reinterpret_cast<const DR*>(ok ? drow + (int64_t)k * g.C : dplane), ok);
+  }
+}
+
+// Step of the walk whose data sit in ring stage st: the carried dY strips move one slot down
+// (slot i holds the dY row that kernel row v0 + i meets, ys - v0 - i + r_h), slot 0 takes the new
+// row ys - v0 + r_h, and the input row ys is multiplied into every kernel row's sums.
 template <typename T, int KW, typename TD>
-__host__ __device__ __forceinline__ void dw_step(const T* __restrict__ xplane, const TD* __restrict__ dplane,
-                                                 const ConvGeo& g, int ys, int v0, int x0,
+__host__ __device__ __forceinline__ void dw_step(const DwRing<T, TD, KW>& r, int st, const ConvGeo& g, int v0,
                                                  float2 (&d)[kDwRows][kConvStrip],
                                                  float2 (&dwr)[kDwRows][KW]) {
   constexpr int NJ = kConvStrip + KW - 1;
-  const int rh = (g.kh - 1) / 2;
 #pragma unroll
   for (int i = kDwRows - 1; i > 0; i--)
 #pragma unroll
     for (int k = 0; k < kConvStrip; k++) d[i][k] = d[i - 1][k];
-  dw_load_dy<TD>(dplane, g, ys - v0 + rh, x0, d[0]);
+#pragma unroll
+  for (int k = 0; k < kConvStrip; k++) d[0][k] = conv_unpack(r.d[(st * kConvStrip + k) * 32]);
   float2 a[NJ];
-  conv_load_row<T, KW>(xplane + (int64_t)ys * g.Wp * g.C, g, x0, a);
+#pragma unroll
+  for (int j = 0; j < NJ; j++) a[j] = conv_unpack(r.x[(st * NJ + j) * 32]);
 #pragma unroll
   for (int i = 0; i < kDwRows; i++) {
     if (v0 + i >= g.kh) break;
@@ -314,19 +417,22 @@ __host__ __device__ __forceinline__ void dw_step(const T* __restrict__ xplane, c
 // One work item's sums: dwr[i][w] (.x, .y: channel 2 c2 + e, e = 0, 1) += sum over its frames t,
 // rows y and columns x0 + k of dY[(t, y, x0 + k)][2 c2 + e] * X[(t + u - r_t, y + v0 + i - r_h,
 // x0 + k + w - r_w)][2 c2 + e]; and, if with_db, db[e] += the sum of its dY strips over every row
-// of its frames.  Outputs past
-// the volume's last column are skipped; X and dY are zero outside the volume.  TD: the type of
-// dY (the input's, or fp32 for the offset network's backward).
+// of its frames.  Outputs past the volume's last column are skipped; X and dY are zero outside the
+// volume.  TD: the type of dY (the input's, or fp32 for the offset network's backward).  The
+// input rows and new dY strips go through the lane's ring, fetched kDwStages - 1 steps ahead.
 template <typename T, int KW, typename TD = T>
 __host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const TD* __restrict__ dy,
-                                                 const ConvGeo& g, int c2, int u, int v0, int x0, int t0,
-                                                 int t1, float2 (&dwr)[kDwRows][KW], bool with_db,
-                                                 float (&db)[2]) {
+                                                 const ConvGeo& g, const DwRing<T, TD, KW>& ring, int c2,
+                                                 int u, int v0, int x0, int t0, int t1,
+                                                 float2 (&dwr)[kDwRows][KW], bool with_db, float (&db)[2]) {
+  constexpr int D = kDwStages - 1;
   const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2;
   const int64_t fstride = (int64_t)g.Hp * g.Wp * g.C;  // one frame
+#pragma unroll 1
   for (int t = t0; t < t1; t++) {
     const TD* dplane = dy + t * fstride + 2 * c2;
     if (with_db) {
+#pragma unroll 1
       for (int y = 0; y < g.Hp; y++) {
         float2 d[kConvStrip];
         dw_load_dy<TD>(dplane, g, y, x0, d);
@@ -343,11 +449,24 @@ __host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const 
     // the input rows that meet some dY row through kernel rows v0 .. v0 + kDwRows - 1
     const int ys0 = v0 - rh > 0 ? v0 - rh : 0;
     const int ys1 = g.Hp - 1 + v0 + kDwRows - 1 - rh < g.Hp - 1 ? g.Hp - 1 + v0 + kDwRows - 1 - rh : g.Hp - 1;
+    const int n = ys1 - ys0 + 1;
     // slot i - 1 holds, before the first step moves it to slot i, kernel row v0 + i's dY row
     float2 d[kDwRows][kConvStrip];
 #pragma unroll
     for (int i = 1; i < kDwRows; i++) dw_load_dy<TD>(dplane, g, ys0 - v0 - i + rh, x0, d[i - 1]);
-    for (int ys = ys0; ys <= ys1; ys++) dw_step<T, KW, TD>(xplane, dplane, g, ys, v0, x0, d, dwr);
+    // copy group s carries step s (empty past the last step): D groups ahead of the step in use
+#pragma unroll
+    for (int s = 0; s < D; s++) {
+      if (s < n) dw_fetch(ring, s, xplane, dplane, g, ys0 + s, v0, x0);
+      dw_commit();
+    }
+#pragma unroll 1
+    for (int s = 0; s < n; s++) {
+      if (s + D < n) dw_fetch(ring, (s + D) % kDwStages, xplane, dplane, g, ys0 + s + D, v0, x0);
+      dw_commit();
+      dw_wait<D>();  // groups 0 .. s are complete
+      dw_step<T, KW, TD>(ring, s % kDwStages, g, v0, d, dwr);
+    }
   }
 }
 
@@ -463,11 +582,15 @@ __global__ void __launch_bounds__(kConvSwWarps * 32)
 
 // dW (and db): one thread per work item (dw_decode, dw_walk); fp32 partial sums added with
 // atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).  The bias gradient is
-// summed by the items of plane 0 and the first kernel-row group.
+// summed by the items of plane 0 and the first kernel-row group.  Dynamic shared memory: a
+// DwRing<T, TD, KW>::warp_bytes() region per warp.
 template <typename T, int KW, typename TD = T>
 __global__ void __launch_bounds__(kConvDwThreads)
     dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const TD* __restrict__ dy, float* dweight,
                              float* dbias, const ConvGeo g, const int frames_per_item) {
+  extern __shared__ __align__(16) unsigned char dw_rings[];  // a DwRing region per warp
+  using R = DwRing<T, TD, KW>;
+  const R ring = R::at(dw_rings + (threadIdx.x >> 5) * R::warp_bytes(), threadIdx.x & 31);
   const int64_t items = dw_items(g, frames_per_item);
   const int64_t K = (int64_t)g.kt * g.kh * KW;
   for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items;
@@ -481,7 +604,7 @@ __global__ void __launch_bounds__(kConvDwThreads)
       for (int j = 0; j < KW; j++) dwr[i][j] = make_float2(0.f, 0.f);
     float db[2] = {0.f, 0.f};
     const bool with_db = u == 0 && v0 == 0;
-    dw_walk<T, KW, TD>(x, dy, g, c2, u, v0, x0, t0, t1, dwr, with_db, db);
+    dw_walk<T, KW, TD>(x, dy, g, ring, c2, u, v0, x0, t0, t1, dwr, with_db, db);
 #pragma unroll
     for (int i = 0; i < kDwRows; i++) {
       if (v0 + i >= g.kh) break;
