@@ -159,6 +159,28 @@ __host__ __device__ __forceinline__ int64_t conv_sw_unit(int64_t slot, int64_t s
   return ((int64_t)i * slots + slot) * kConvSwWarps + warp;
 }
 
+// The raw channel pair of T as loaded (4 bytes for bf16, 8 for fp32), and its fp32 values.
+template <typename T>
+struct ConvRaw;
+template <>
+struct ConvRaw<float> {
+  using type = float2;
+};
+template <>
+struct ConvRaw<__nv_bfloat16> {
+  using type = unsigned;
+};
+__host__ __device__ __forceinline__ float2 conv_unpack(float2 r) { return r; }
+__host__ __device__ __forceinline__ float2 conv_unpack(unsigned u) {
+  union {
+    unsigned i;
+    float f;
+  } lo, hi;
+  lo.i = u << 16;
+  hi.i = u & 0xffff0000u;
+  return make_float2(lo.f, hi.f);
+}
+
 // Convolution sums of channel pair c2 (channels 2 c2 and 2 c2 + 1) for the two output strips
 // (t, y0 + r, x0 + i), r < 2, i < kConvStrip, added into acc[r][i] (.x: channel 2 c2, .y: 2 c2 +
 // 1).  For kernel plane u the input rows y0 - r_h .. y0 + 1 + r_h are loaded once each, and
@@ -179,50 +201,79 @@ __host__ __device__ __forceinline__ void conv_load_row(const T* __restrict__ row
   }
 }
 
+// The same row as raw pairs (zero past the volume's edges, and all zero when !in).
+template <typename T, int KW>
+__host__ __device__ __forceinline__ void conv_load_row_raw(const T* __restrict__ row, bool in, const ConvGeo& g,
+                                                           int x0, typename ConvRaw<T>::type (&r)[kConvStrip + KW - 1]) {
+  using R = typename ConvRaw<T>::type;
+  const int rw = (KW - 1) / 2;
+#pragma unroll
+  for (int j = 0; j < kConvStrip + KW - 1; j++) {
+    const int xs = x0 - rw + j;
+    r[j] = R{};
+    if (in && xs >= 0 && xs < g.Wp) {
+#ifdef __CUDA_ARCH__
+      r[j] = __ldg(reinterpret_cast<const R*>(row + (int64_t)xs * g.C));
+#else
+      r[j] = *reinterpret_cast<const R*>(row + (int64_t)xs * g.C);
+#endif
+    }
+  }
+}
+
 template <typename T, int KW, typename WGet>
 __host__ __device__ __forceinline__ void conv_strip2(const T* __restrict__ x, const WGet& wget,
                                                      const ConvGeo& g, int t, int y0, int x0, int c2,
                                                      bool flip, float2 (&acc)[2][kConvStrip]) {
   constexpr int NJ = kConvStrip + KW - 1;
+  using R = typename ConvRaw<T>::type;
   const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2;
   const int64_t rstride = (int64_t)g.Wp * g.C;  // one token row
+  // The input rows in order: plane u = 0 .. kt - 1, rows y0 - r_h + r, r = 0 .. kh; each row is
+  // loaded (raw) one row ahead of its use.  Row r = 0 of a plane is kernel row 0's input for
+  // output row y0; row r >= 1 is kernel row r - 1's input for output row y0 + 1 and kernel row r's
+  // for y0 (carried in pr).  Rows outside the volume are zeros (plane u outside it: all its rows).
+  const T* xc = x + 2 * c2;
+  auto row_at = [&](int u, int r, bool& in) {
+    const int ts = t + u - rt, ys = y0 - rh + r;
+    in = ts >= 0 && ts < g.F && ys >= 0 && ys < g.Hp;
+    return xc + ((int64_t)(in ? ts : 0) * g.Hp + (in ? ys : 0)) * rstride;
+  };
+  R nxt[NJ];
+  {
+    bool in;
+    const T* row = row_at(0, 0, in);
+    conv_load_row_raw<T, KW>(row, in, g, x0, nxt);
+  }
+  float2 pr[NJ];
   for (int u = 0; u < g.kt; u++) {
-    const int ts = t + u - rt;
-    if (ts < 0 || ts >= g.F) continue;
-    const T* plane = x + (int64_t)ts * g.Hp * rstride + 2 * c2;
-    // the row under output row y0 for kernel row v (pr), and the one under y0 + 1 (cr)
-    float2 pr[NJ], cr[NJ];
-    {
-      const int ys = y0 - rh;
-      if (ys >= 0 && ys < g.Hp) {
-        conv_load_row<T, KW>(plane + ys * rstride, g, x0, pr);
-      } else {
+    for (int r = 0; r <= g.kh; r++) {
+      float2 cr[NJ];
 #pragma unroll
-        for (int j = 0; j < NJ; j++) pr[j] = make_float2(0.f, 0.f);
+      for (int j = 0; j < NJ; j++) cr[j] = conv_unpack(nxt[j]);
+      // the next row: r + 1 of this plane, or row 0 of the next plane
+      if (r < g.kh || u + 1 < g.kt) {
+        bool in;
+        const T* row = r < g.kh ? row_at(u, r + 1, in) : row_at(u + 1, 0, in);
+        conv_load_row_raw<T, KW>(row, in, g, x0, nxt);
       }
-    }
-    for (int v = 0; v < g.kh; v++) {
-      const int ys = y0 + 1 + v - rh;
-      if (ys >= 0 && ys < g.Hp) {
-        conv_load_row<T, KW>(plane + ys * rstride, g, x0, cr);
-      } else {
+      if (r > 0) {
+        const int v = r - 1;
+        // the kernel row's weights (flipped for the transposed convolution)
+        const int64_t wrow = flip ? ((int64_t)(g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW
+                                  : ((int64_t)u * g.kh + v) * KW;
+        float2 w[KW];
 #pragma unroll
-        for (int j = 0; j < NJ; j++) cr[j] = make_float2(0.f, 0.f);
-      }
-      // the kernel row's weights (flipped for the transposed convolution)
-      const int64_t wrow = flip ? ((int64_t)(g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW
-                                : ((int64_t)u * g.kh + v) * KW;
-      float2 w[KW];
+        for (int j = 0; j < KW; j++) w[j] = wget(wrow + (flip ? KW - 1 - j : j));
+        // input column x0 - rw + j feeds output x0 + i through tap j - i
 #pragma unroll
-      for (int j = 0; j < KW; j++) w[j] = wget(wrow + (flip ? KW - 1 - j : j));
-      // input column x0 - rw + j feeds output x0 + i through tap j - i
+        for (int j = 0; j < NJ; j++) {
 #pragma unroll
-      for (int j = 0; j < NJ; j++) {
-#pragma unroll
-        for (int i = 0; i < kConvStrip; i++) {
-          if (j - i >= 0 && j - i < KW) {
-            conv_fma2(acc[0][i], w[j - i], pr[j]);
-            conv_fma2(acc[1][i], w[j - i], cr[j]);
+          for (int i = 0; i < kConvStrip; i++) {
+            if (j - i >= 0 && j - i < KW) {
+              conv_fma2(acc[0][i], w[j - i], pr[j]);
+              conv_fma2(acc[1][i], w[j - i], cr[j]);
+            }
           }
         }
       }
@@ -275,29 +326,6 @@ __host__ __device__ __forceinline__ void dw_load_dy(const TD* __restrict__ dplan
     d[i] = make_float2(0.f, 0.f);
     if (in && x0 + i < g.Wp) d[i] = conv_load2v(row + (int64_t)i * g.C);
   }
-}
-
-// The raw channel pair of T as the dW walk stages it (4 bytes for bf16, 8 for fp32), and its
-// fp32 values.
-template <typename T>
-struct ConvRaw;
-template <>
-struct ConvRaw<float> {
-  using type = float2;
-};
-template <>
-struct ConvRaw<__nv_bfloat16> {
-  using type = unsigned;
-};
-__host__ __device__ __forceinline__ float2 conv_unpack(float2 r) { return r; }
-__host__ __device__ __forceinline__ float2 conv_unpack(unsigned u) {
-  union {
-    unsigned i;
-    float f;
-  } lo, hi;
-  lo.i = u << 16;
-  hi.i = u & 0xffff0000u;
-  return make_float2(lo.f, hi.f);
 }
 
 // *dst = *src (a raw pair), or zeros when !ok.  On the GPU an asynchronous copy into shared
