@@ -131,27 +131,37 @@ int dw_frames_per_item(const ConvGeo& g, int64_t resident) {
 }
 
 // dW and db: a grid of at most the blocks the GPU holds at once, striding over the items.
-template <typename T, int KW, typename TD = T>
-dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* dy, float* dw,
-                                   float* db, cudaStream_t st) {
+template <typename T, int KW, typename TD, bool Coop>
+dsa3d_status_t dwconv_dw_launch_kernel(const ConvGeo& g, const void* x, const void* dy, float* dw,
+                                       float* db, cudaStream_t st) {
+  auto* kern = dsa3d_dwconv3d_dw_kernel<T, KW, TD, Coop>;
   // a staging ring per warp
   const size_t smem = (size_t)(kConvDwThreads / 32) * DwRing<T, TD, KW>::warp_bytes();
-  if (cudaFuncSetAttribute(dsa3d_dwconv3d_dw_kernel<T, KW, TD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return DSA3D_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dsa3d_dwconv3d_dw_kernel<T, KW, TD>,
-                                                    kConvDwThreads, smem) != cudaSuccess)
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kConvDwThreads, smem) != cudaSuccess)
     return DSA3D_ERR_CUDA;
   if (per_sm < 1) per_sm = 1;
   const int sms = std::max(device_info().sms, 1);
   const int fpi = dw_frames_per_item(g, (int64_t)sms * per_sm * kConvDwThreads);
   const int64_t items = dw_items(g, fpi);
   TimedLaunch tl(kKernDwconvDw, st);
-  dsa3d_dwconv3d_dw_kernel<T, KW, TD><<<grid_for(items, kConvDwThreads, per_sm), kConvDwThreads, smem, st>>>(
+  kern<<<grid_for(items, kConvDwThreads, per_sm), kConvDwThreads, smem, st>>>(
       static_cast<const T*>(x), static_cast<const TD*>(dy), dw, db, g, fpi);
   const bool launched = cudaGetLastError() == cudaSuccess;
   return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+}
+
+// The warp-cooperative copies when every warp is 32 aligned channel pairs of one work item: C a
+// multiple of 64 (the items run channel pairs fastest, and blocks and the grid stride are whole
+// warps).
+template <typename T, int KW, typename TD = T>
+dsa3d_status_t dwconv_dw_launch_kw(const ConvGeo& g, const void* x, const void* dy, float* dw,
+                                   float* db, cudaStream_t st) {
+  static_assert(kConvDwThreads % 32 == 0, "whole warps");
+  if (g.C % 64 == 0) return dwconv_dw_launch_kernel<T, KW, TD, true>(g, x, dy, dw, db, st);
+  return dwconv_dw_launch_kernel<T, KW, TD, false>(g, x, dy, dw, db, st);
 }
 
 template <typename T, typename TD = T>

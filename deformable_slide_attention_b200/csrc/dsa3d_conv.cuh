@@ -357,6 +357,24 @@ __host__ __device__ __forceinline__ void dw_wait() {
 #endif
 }
 
+// 16 bytes from src to dst, or zeros when !ok: on the GPU cp.async (through L2 only), otherwise
+// as dw_copy.
+__host__ __device__ __forceinline__ void dw_copy16(void* dst, const void* src, bool ok) {
+#ifdef __CUDA_ARCH__
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(ok ? 16 : 0) : "memory");
+#else
+  unsigned char* o = static_cast<unsigned char*>(dst);
+  const unsigned char* i = static_cast<const unsigned char*>(src);
+  for (int b = 0; b < 16; b++) o[b] = ok ? i[b] : 0;
+#endif
+}
+__host__ __device__ __forceinline__ void dw_syncwarp() {
+#ifdef __CUDA_ARCH__
+  __syncwarp();
+#endif
+}
+
 constexpr int kDwStages = 3;  // steps of the dW walk in its staging ring: fetched two steps ahead
 
 // One lane's staging ring of the dW walk: kDwStages steps of an input row (NJ raw pairs) and a
@@ -408,6 +426,50 @@ __host__ __device__ __forceinline__ void dw_fetch(const DwRing<T, TD, KW>& r, in
   }
 }
 
+// dw_fetch for the whole warp at once, when its 32 lanes are 32 consecutive channel pairs from a
+// multiple of 32 (C a multiple of 64) on the same work item: a token's 32 pairs are one
+// contiguous run of 128 (bf16) or 256 (fp32) bytes, copied as 16-byte chunks spread over the
+// lanes, each chunk into the 16 bytes of the ring entry that hold those pairs.  xplane and dplane
+// point at the lane's own pair; the chunks a lane copies belong to other lanes too, so the ring
+// is shared within the warp (dw_syncwarp around its use).  On the host one call copies every
+// chunk of the warp.
+template <typename T, typename TD, int KW>
+__host__ __device__ __forceinline__ void dw_fetch_warp(const DwRing<T, TD, KW>& r, int lane, int st,
+                                                       const T* xplane, const TD* dplane, const ConvGeo& g,
+                                                       int ys, int v0, int x0) {
+  using R = DwRing<T, TD, KW>;
+  using XR = typename R::XR;
+  using DR = typename R::DR;
+  constexpr int CX = 32 * (int)sizeof(XR) / 16, CD = 32 * (int)sizeof(DR) / 16;  // chunks per token
+  const int rw = (KW - 1) / 2, rh = (g.kh - 1) / 2;
+  const T* xw = xplane - 2 * lane;  // pair 0 of the warp
+  const TD* dw = dplane - 2 * lane;
+  unsigned char* rx = reinterpret_cast<unsigned char*>(r.x - lane);
+  unsigned char* rd = reinterpret_cast<unsigned char*>(r.d - lane);
+#ifdef __CUDA_ARCH__
+  const int m0 = lane, mstep = 32;
+#else
+  const int m0 = 0, mstep = 1;
+#endif
+  const T* xrow = xw + (int64_t)ys * g.Wp * g.C;
+  for (int m = m0; m < R::NJ * CX; m += mstep) {
+    const int j = m / CX, q = m - j * CX;
+    const int xs = x0 - rw + j;
+    const bool ok = xs >= 0 && xs < g.Wp;
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(ok ? xrow + (int64_t)xs * g.C : xw) + 16 * q;
+    dw_copy16(rx + ((size_t)(st * R::NJ + j) * 32) * sizeof(XR) + 16 * q, src, ok);
+  }
+  const int y = ys - v0 + rh;
+  const bool yin = y >= 0 && y < g.Hp;
+  const TD* drow = yin ? dw + ((int64_t)y * g.Wp + x0) * g.C : dw;
+  for (int m = m0; m < kConvStrip * CD; m += mstep) {
+    const int k = m / CD, q = m - k * CD;
+    const bool ok = yin && x0 + k < g.Wp;
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(ok ? drow + (int64_t)k * g.C : dw) + 16 * q;
+    dw_copy16(rd + ((size_t)(st * kConvStrip + k) * 32) * sizeof(DR) + 16 * q, src, ok);
+  }
+}
+
 // Step of the walk whose data sit in ring stage st: the carried dY strips move one slot down
 // (slot i holds the dY row that kernel row v0 + i meets, ys - v0 - i + r_h), slot 0 takes the new
 // row ys - v0 + r_h, and the input row ys is multiplied into every kernel row's sums.
@@ -448,7 +510,7 @@ __host__ __device__ __forceinline__ void dw_step(const DwRing<T, TD, KW>& r, int
 // of its frames.  Outputs past the volume's last column are skipped; X and dY are zero outside the
 // volume.  TD: the type of dY (the input's, or fp32 for the offset network's backward).  The
 // input rows and new dY strips go through the lane's ring, fetched kDwStages - 1 steps ahead.
-template <typename T, int KW, typename TD = T>
+template <typename T, int KW, typename TD = T, bool Coop = false>
 __host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const TD* __restrict__ dy,
                                                  const ConvGeo& g, const DwRing<T, TD, KW>& ring, int c2,
                                                  int u, int v0, int x0, int t0, int t1,
@@ -483,16 +545,25 @@ __host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const 
 #pragma unroll
     for (int i = 1; i < kDwRows; i++) dw_load_dy<TD>(dplane, g, ys0 - v0 - i + rh, x0, d[i - 1]);
     // copy group s carries step s (empty past the last step): D groups ahead of the step in use
+    auto fetch = [&](int st, int ys) {
+      if constexpr (Coop)
+        dw_fetch_warp(ring, c2 & 31, st, xplane, dplane, g, ys, v0, x0);
+      else
+        dw_fetch(ring, st, xplane, dplane, g, ys, v0, x0);
+    };
+    if (Coop) dw_syncwarp();  // the previous frame's last reads are done before the ring refills
 #pragma unroll
     for (int s = 0; s < D; s++) {
-      if (s < n) dw_fetch(ring, s, xplane, dplane, g, ys0 + s, v0, x0);
+      if (s < n) fetch(s, ys0 + s);
       dw_commit();
     }
 #pragma unroll 1
     for (int s = 0; s < n; s++) {
-      if (s + D < n) dw_fetch(ring, (s + D) % kDwStages, xplane, dplane, g, ys0 + s + D, v0, x0);
+      if (Coop) dw_syncwarp();  // every lane's reads of step s - 1's stage are done
+      if (s + D < n) fetch((s + D) % kDwStages, ys0 + s + D);
       dw_commit();
-      dw_wait<D>();  // groups 0 .. s are complete
+      dw_wait<D>();  // this lane's groups 0 .. s are complete
+      if (Coop) dw_syncwarp();  // and every lane's
       dw_step<T, KW, TD>(ring, s % kDwStages, g, v0, d, dwr);
     }
   }
@@ -611,9 +682,12 @@ __global__ void __launch_bounds__(kConvSwWarps * 32)
 // dW (and db): one thread per work item (dw_decode, dw_walk); fp32 partial sums added with
 // atomics into dweight [C][kt][kh][kw] and dbias [C] (both zeroed before).  The bias gradient is
 // summed by the items of plane 0 and the first kernel-row group.  Dynamic shared memory: a
-// DwRing<T, TD, KW>::warp_bytes() region per warp.
-template <typename T, int KW, typename TD = T>
-__global__ void __launch_bounds__(kConvDwThreads)
+// DwRing<T, TD, KW>::warp_bytes() region per warp.  Coop (C a multiple of 64, so that every warp
+// is 32 aligned pairs of one work item through the whole grid-stride loop): dw_fetch_warp, and a
+// register cap for three blocks per SM (168 registers, a 20-byte spill at bf16 and k_w = 9: 222
+// -> 183 ms per launch at 1080p); the per-lane copies spill over 100 bytes under that cap.
+template <typename T, int KW, typename TD = T, bool Coop = false>
+__global__ void __launch_bounds__(kConvDwThreads, Coop ? 3 : 1)
     dsa3d_dwconv3d_dw_kernel(const T* __restrict__ x, const TD* __restrict__ dy, float* dweight,
                              float* dbias, const ConvGeo g, const int frames_per_item) {
   extern __shared__ __align__(16) unsigned char dw_rings[];  // a DwRing region per warp
@@ -632,7 +706,7 @@ __global__ void __launch_bounds__(kConvDwThreads)
       for (int j = 0; j < KW; j++) dwr[i][j] = make_float2(0.f, 0.f);
     float db[2] = {0.f, 0.f};
     const bool with_db = u == 0 && v0 == 0;
-    dw_walk<T, KW, TD>(x, dy, g, ring, c2, u, v0, x0, t0, t1, dwr, with_db, db);
+    dw_walk<T, KW, TD, Coop>(x, dy, g, ring, c2, u, v0, x0, t0, t1, dwr, with_db, db);
 #pragma unroll
     for (int i = 0; i < kDwRows; i++) {
       if (v0 + i >= g.kh) break;

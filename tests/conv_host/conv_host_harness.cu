@@ -84,17 +84,23 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
 template <typename T, int KW, typename TD = T>
 void dw_all(const T* x, const TD* dy, const ConvGeo& g, int frames_per_item, float* dw, float* db) {
   const int64_t K = (int64_t)g.kt * g.kh * KW;
-  // one warp's staging region; the walk runs as lane 5 of it (the harness runs one lane at a time)
+  // one warp's staging region; each item runs as its pair's lane (c2 mod 32) of it, one lane at a
+  // time; with C a multiple of 64 the library's warp-cooperative copies (each call copies the
+  // whole warp's chunks here)
   using R = DwRing<T, TD, KW>;
   std::vector<double> region((R::warp_bytes() + sizeof(double) - 1) / sizeof(double));
-  const R ring = R::at(reinterpret_cast<unsigned char*>(region.data()), 5);
+  const bool coop = g.C % 64 == 0;
   for (int64_t it = 0; it < dw_items(g, frames_per_item); it++) {
     int c2, u, v0, x0, t0, t1;
     dw_decode(it, g, frames_per_item, c2, u, v0, x0, t0, t1);
     float2 dwr[kDwRows][KW] = {};
     float dbl[2] = {0.f, 0.f};
     const bool with_db = u == 0 && v0 == 0;
-    dw_walk<T, KW, TD>(x, dy, g, ring, c2, u, v0, x0, t0, t1, dwr, with_db, dbl);
+    const R ring = R::at(reinterpret_cast<unsigned char*>(region.data()), c2 & 31);
+    if (coop)
+      dw_walk<T, KW, TD, true>(x, dy, g, ring, c2, u, v0, x0, t0, t1, dwr, with_db, dbl);
+    else
+      dw_walk<T, KW, TD, false>(x, dy, g, ring, c2, u, v0, x0, t0, t1, dwr, with_db, dbl);
     for (int i = 0; i < kDwRows && v0 + i < g.kh; i++)
       for (int j = 0; j < KW; j++) {
         const int64_t o = (int64_t)(2 * c2) * K + ((int64_t)u * g.kh + v0 + i) * KW + j;
