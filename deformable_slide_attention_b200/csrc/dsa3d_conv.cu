@@ -72,8 +72,9 @@ dsa3d_status_t check_conv_shape(int F, int Hp, int Wp, int C, int kt, int kh, in
   return DSA3D_OK;
 }
 
-// The forward (and dX, flip = 1): the staged kernel when the kernel's taps fit in shared memory
-// and its grid in one dimension, else the global-memory one.
+// The forward (and dX, flip = 1): when the kernel's taps fit in shared memory and the grid in one
+// dimension, the strip-pair kernel for C a multiple of 32 and the staged kernel for the other
+// channel counts; else the global-memory one.
 template <typename T, int KW, typename OutT = T>
 dsa3d_status_t dwconv_launch_kw(const ConvGeo& g, const void* x, const float* w, const float* b,
                                 const void* add, void* y, int flip, cudaStream_t st) {
@@ -84,6 +85,20 @@ dsa3d_status_t dwconv_launch_kw(const ConvGeo& g, const void* x, const float* w,
   const T* xt = static_cast<const T*>(x);
   const OutT* at = static_cast<const OutT*>(add);
   OutT* yt = static_cast<OutT*>(y);
+  const int64_t sw2_units = (int64_t)g.F * ((g.Hp + 1) / 2) * ((g.Wp + 2 * kConvStrip - 1) / (2 * kConvStrip));
+  const int64_t sw2_grid = (sw2_units + kSw2Units - 1) / kSw2Units * (g.C / (2 * kSw2Pairs));
+  if (K <= kConvSwMaxTaps && g.C % (2 * kSw2Pairs) == 0 && sw2_grid <= INT_MAX) {
+    // strip pairs with a warp-shared row ring
+    const size_t smem = conv_sw2_weight_bytes(K) + kConvSwWarps * Sw2Ring<T, KW>::warp_bytes();
+    if (cudaFuncSetAttribute(dsa3d_dwconv3d_sw2_kernel<T, KW, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return DSA3D_ERR_CUDA;
+    TimedLaunch tl(kKernDwconvSw2, st);
+    dsa3d_dwconv3d_sw2_kernel<T, KW, OutT><<<(unsigned)sw2_grid, kConvSwWarps * 32, smem, st>>>(
+        xt, w, b, at, yt, g, flip);
+    const bool launched = cudaGetLastError() == cudaSuccess;
+    return (tl.finish() && launched) ? DSA3D_OK : DSA3D_ERR_CUDA;
+  }
   if (K <= kConvSwMaxTaps && sw_blocks <= INT_MAX) {
     // the staged kernel may take up to conv_sw_bytes(kConvSwMaxTaps) of dynamic shared memory
     if (cudaFuncSetAttribute(dsa3d_dwconv3d_sw_kernel<T, KW, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,

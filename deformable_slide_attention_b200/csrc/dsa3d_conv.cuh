@@ -134,12 +134,14 @@ __host__ __device__ __forceinline__ int conv_sw_index(int k, int cc) { return k 
 __host__ __device__ __forceinline__ size_t conv_sw_bytes(int K) {
   return (size_t)K * kConvGroupStride * sizeof(float);
 }
-struct ConvWShared {
-  const float* s;  // the staged group + 2 * lane (8-byte aligned: the stride is even)
+template <int Stride>
+struct ConvWSharedT {
+  const float* s;  // the staged group + 2 * (the lane's pair) (8-byte aligned: Stride is even)
   __host__ __device__ __forceinline__ float2 operator()(int64_t k) const {
-    return *reinterpret_cast<const float2*>(s + (int)k * kConvGroupStride);
+    return *reinterpret_cast<const float2*>(s + (int)k * Stride);
   }
 };
+using ConvWShared = ConvWSharedT<kConvGroupStride>;
 
 // Unit (t, y0, x0) of the forward's work: output rows y0, y0 + 1 from column x0, strips fastest,
 // then row pairs, then frames.
@@ -151,8 +153,8 @@ __host__ __device__ __forceinline__ void conv_unit(int64_t unit, int nxs, int ny
   t = (int)(r / nyp);
 }
 
-// The i-th unit (i < kConvSwUnits / kConvSwWarps) of warp `warp` in the staged kernel's block
-// slot `slot` of `slots` (= ceil(units / kConvSwUnits)).  The slots' units interleave: at step i
+// The i-th unit (i < units per block / kConvSwWarps) of warp `warp` in a staged kernel's block
+// slot `slot` of `slots` (= ceil(units / units per block)).  The slots' units interleave: at step i
 // the resident blocks, whose slots are consecutive, work on one run of consecutive units (the
 // rows they read stay in L2), and every unit below slots * kConvSwUnits is visited once.
 __host__ __device__ __forceinline__ int64_t conv_sw_unit(int64_t slot, int64_t slots, int warp, int i) {
@@ -569,6 +571,132 @@ __host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const 
   }
 }
 
+// ---- the forward on strip pairs, input rows through a warp-shared ring ----------------------
+// For C a multiple of 32: a block owns kSw2Pairs channel pairs and its warps take units of two
+// neighbouring strips (t, row pair y0, y0 + 1, columns xb .. xb + 2 kConvStrip - 1); lane 16 h +
+// p computes pair p of strip h.  The two strips' windows share one input row of NT tokens, which
+// the warp copies into a ring in shared memory with 16-byte cp.async chunks, kSw2Stages - 1 rows
+// ahead of its use.
+constexpr int kSw2Pairs = 16;
+constexpr int kSw2WStride = 2 * kSw2Pairs + 2;  // floats per staged tap row (2 of padding)
+constexpr int kSw2Units = 32;                   // units per block, kSw2Units / kConvSwWarps per warp
+constexpr int kSw2Stages = 3;
+
+template <typename T, int KW>
+struct Sw2Ring {
+  using R = typename ConvRaw<T>::type;
+  static constexpr int NT = 2 * kConvStrip + KW - 1;                 // tokens of a staged row
+  static constexpr int ROW = (NT + (NT + 7) / 8) * kSw2Pairs;        // R entries per staged row
+  // entry of token j, pair p: every 8 tokens shift by kSw2Pairs entries, so that the two strips'
+  // lanes (tokens j and j + 8) read different banks
+  __host__ __device__ static constexpr int at(int j, int p) { return (j + (j >> 3)) * kSw2Pairs + p; }
+  __host__ __device__ static constexpr size_t warp_bytes() { return (size_t)kSw2Stages * ROW * sizeof(R); }
+};
+
+// Unit `unit` of the strip-pair forward: frames, then row pairs, then strip pairs fastest.
+__host__ __device__ __forceinline__ void conv_unit2(int64_t unit, int nxp, int nyp, int& t, int& y0, int& xb) {
+  xb = (int)(unit % nxp) * 2 * kConvStrip;
+  const int64_t r = unit / nxp;
+  y0 = 2 * (int)(r % nyp);
+  t = (int)(r / nyp);
+}
+
+// Copy input row ys of frame ts (tokens xb - r_w .. xb - r_w + NT - 1 of the group's pairs; xg:
+// x at the group's first channel) into ring stage st, zeros outside the volume.  The warp's lanes
+// share the chunks; on the host one call copies them all.
+template <typename T, int KW>
+__host__ __device__ __forceinline__ void sw2_fetch(typename ConvRaw<T>::type* ring, int lane, int st,
+                                                   const T* xg, const ConvGeo& g, int ts, int ys, int xb) {
+  using S = Sw2Ring<T, KW>;
+  using R = typename S::R;
+  constexpr int CPT = kSw2Pairs * (int)sizeof(R) / 16;  // 16-byte chunks per token
+  const int rw = (KW - 1) / 2;
+  const bool rin = ts >= 0 && ts < g.F && ys >= 0 && ys < g.Hp;
+  const T* row = rin ? xg + ((int64_t)ts * g.Hp + ys) * g.Wp * g.C : xg;
+  R* dst = ring + st * S::ROW;
+#ifdef __CUDA_ARCH__
+  const int m0 = lane, mstep = 32;
+#else
+  const int m0 = 0, mstep = 1;
+  (void)lane;
+#endif
+  for (int m = m0; m < S::NT * CPT; m += mstep) {
+    const int j = m / CPT, q = m - j * CPT;
+    const int xs = xb - rw + j;
+    const bool ok = rin && xs >= 0 && xs < g.Wp;
+    const unsigned char* src = reinterpret_cast<const unsigned char*>(ok ? row + (int64_t)xs * g.C : xg) + 16 * q;
+    dw_copy16(reinterpret_cast<unsigned char*>(dst + S::at(j, 0)) + 16 * q, src, ok);
+  }
+}
+
+// conv_strip2 for lane 16 h + p of a strip-pair unit (strip x0 = xb + h kConvStrip, pair p of the
+// group), its input rows read from the warp's ring (ring: the warp's kSw2Stages rows).  The rows
+// run as one sequence over the kernel planes, as in conv_strip2.
+template <typename T, int KW, typename WGet>
+__host__ __device__ __forceinline__ void conv_strip2_ring(typename ConvRaw<T>::type* ring, int lane,
+                                                          const T* xg, const WGet& wget, const ConvGeo& g,
+                                                          int t, int y0, int xb, bool flip,
+                                                          float2 (&acc)[2][kConvStrip]) {
+  using S = Sw2Ring<T, KW>;
+  using R = typename S::R;
+  constexpr int NJ = kConvStrip + KW - 1;
+  constexpr int D = kSw2Stages - 1;
+  const int h = lane >> 4, p = lane & (kSw2Pairs - 1);
+  const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2;
+  const int rows = g.kh + 1, Q = g.kt * rows;
+  int fu = 0, fr = 0;  // plane and row of the next fetch
+  auto fetch_next = [&](int q) {
+    sw2_fetch<T, KW>(ring, lane, q % kSw2Stages, xg, g, t + fu - rt, y0 - rh + fr, xb);
+    if (++fr == rows) {
+      fr = 0;
+      fu++;
+    }
+  };
+  dw_syncwarp();  // the previous unit's last reads of the ring are done
+#pragma unroll
+  for (int q = 0; q < D; q++) {
+    if (q < Q) fetch_next(q);
+    dw_commit();
+  }
+  float2 pr[NJ];
+  int u = 0, r = 0;
+  for (int q = 0; q < Q; q++) {
+    dw_syncwarp();  // every lane's reads of row q - 1's stage are done
+    if (q + D < Q) fetch_next(q + D);
+    dw_commit();
+    dw_wait<D>();
+    dw_syncwarp();  // every lane's copies of row q have landed
+    const R* row = ring + (q % kSw2Stages) * S::ROW;
+    float2 cr[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; j++) cr[j] = conv_unpack(row[S::at(h * kConvStrip + j, p)]);
+    if (r > 0) {
+      const int v = r - 1;
+      const int64_t wrow = flip ? ((int64_t)(g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW
+                                : ((int64_t)u * g.kh + v) * KW;
+      float2 w[KW];
+#pragma unroll
+      for (int j = 0; j < KW; j++) w[j] = wget(wrow + (flip ? KW - 1 - j : j));
+#pragma unroll
+      for (int j = 0; j < NJ; j++) {
+#pragma unroll
+        for (int i = 0; i < kConvStrip; i++) {
+          if (j - i >= 0 && j - i < KW) {
+            conv_fma2(acc[0][i], w[j - i], pr[j]);
+            conv_fma2(acc[1][i], w[j - i], cr[j]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < NJ; j++) pr[j] = cr[j];
+    if (++r == rows) {
+      r = 0;
+      u++;
+    }
+  }
+}
+
 #ifdef __CUDACC__
 // Writes the two strips acc (rows y0, y0 + 1 from column x0; channel pair c2), each element plus
 // add's (nullable; may equal y); rows and columns past the volume are not written.
@@ -676,6 +804,62 @@ __global__ void __launch_bounds__(kConvSwWarps * 32)
     conv_acc_init(acc, b0, b1);
     conv_strip2<T, KW>(x, ws, g, t, y0, x0, c2, flip != 0, acc);
     conv_store_strips(acc, add, y, g, t, y0, x0, c2);
+  }
+}
+
+// Bytes of the strip-pair forward's staged weights (16-byte aligned; the warps' rings follow).
+__host__ __device__ __forceinline__ size_t conv_sw2_weight_bytes(int K) {
+  return ((size_t)K * kSw2WStride * sizeof(float) + 15) & ~size_t(15);
+}
+
+// The forward on strip pairs (C a multiple of 32, at most kConvSwMaxTaps taps): a block owns one
+// group of kSw2Pairs channel pairs and kSw2Units strip-pair units of one slot (conv_sw_unit over
+// the strip-pair units), which its warps take in turn.  The group's weights are copied in once,
+// tap-major with stride kSw2WStride; each warp then has kSw2Stages rows of ring.  Dynamic shared
+// memory: conv_sw2_weight_bytes(K) + kConvSwWarps Sw2Ring<T, KW>::warp_bytes().  Registers capped
+// for four blocks per SM up to k_w = 9 (126 at bf16 and k_w = 9, no spills: 180 -> 173 ms per
+// launch at 1080p) and three above (four would spill 40-340 bytes).
+template <typename T, int KW, typename OutT = T>
+__global__ void __launch_bounds__(kConvSwWarps * 32, KW <= 9 ? 4 : 3)
+    dsa3d_dwconv3d_sw2_kernel(const T* __restrict__ x, const float* __restrict__ w,
+                              const float* __restrict__ bias, const OutT* add, OutT* y,
+                              const ConvGeo g, const int flip) {
+  using S = Sw2Ring<T, KW>;
+  using R = typename S::R;
+  extern __shared__ __align__(16) unsigned char conv_sw2[];
+  float* ws_all = reinterpret_cast<float*>(conv_sw2);
+  const int K = g.kt * g.kh * KW;
+  const unsigned groups = (unsigned)(g.C / (2 * kSw2Pairs));
+  const int grp = (int)(blockIdx.x % groups);
+  const int64_t slot = blockIdx.x / groups;
+  const int c0 = 2 * kSw2Pairs * grp;
+  const float* wg = w + (int64_t)c0 * K;  // the group's 2 kSw2Pairs channels: contiguous floats
+  for (int cc = 0; cc < 2 * kSw2Pairs; cc++)
+    for (int k = threadIdx.x; k < K; k += blockDim.x)
+      conv_cp_async4(ws_all + k * kSw2WStride + cc, wg + (int64_t)cc * K + k);
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  R* ring = reinterpret_cast<R*>(conv_sw2 + conv_sw2_weight_bytes(K)) + (size_t)warp * kSw2Stages * S::ROW;
+  const int h = lane >> 4, p = lane & (kSw2Pairs - 1);
+  const int c2 = kSw2Pairs * grp + p;
+  const int nxp = (g.Wp + 2 * kConvStrip - 1) / (2 * kConvStrip);
+  const int nyp = (g.Hp + 1) / 2;
+  const int64_t units = (int64_t)g.F * nyp * nxp;
+  const int64_t slots = (units + kSw2Units - 1) / kSw2Units;
+  const ConvWSharedT<kSw2WStride> wsrc{ws_all + 2 * p};
+  const float b0 = bias ? __ldg(bias + 2 * c2) : 0.f, b1 = bias ? __ldg(bias + 2 * c2 + 1) : 0.f;
+  const T* xg = x + c0;
+  static_assert(kSw2Units % kConvSwWarps == 0, "whole steps of the warps");
+  for (int i = 0; i < kSw2Units / kConvSwWarps; i++) {
+    const int64_t unit = conv_sw_unit(slot, slots, warp, i);
+    if (unit >= units) break;  // warp-uniform; later steps' units are larger still
+    int t, y0, xb;
+    conv_unit2(unit, nxp, nyp, t, y0, xb);
+    float2 acc[2][kConvStrip];
+    conv_acc_init(acc, b0, b1);
+    conv_strip2_ring<T, KW>(ring, lane, xg, wsrc, g, t, y0, xb, flip != 0, acc);
+    conv_store_strips(acc, add, y, g, t, y0, xb + h * kConvStrip, c2);
   }
 }
 

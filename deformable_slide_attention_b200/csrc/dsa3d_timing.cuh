@@ -36,6 +36,7 @@ enum KernelId {
   kKernBwdKvTc,
   kKernBwdDqTc,
   kKernDwconvSw,
+  kKernDwconvSw2,
   kKernCount
 };
 inline const char* kernel_name(int id) {
@@ -47,7 +48,8 @@ inline const char* kernel_name(int id) {
       "dsa3d_fwd_taps_kernel", "dsa3d_bwd_taps_kernel", "dsa3d_dwconv3d_kernel",
       "dsa3d_dwconv3d_dw_kernel", "dsa3d_pointwise_offsets_kernel", "dsa3d_pointwise_dz_kernel",
       "dsa3d_pointwise_dw_kernel", "dsa3d_sort_order_kernels", "dsa3d_fwd_tc_kernel",
-      "dsa3d_bwd_kv_tc_kernel", "dsa3d_bwd_dq_tc_kernel", "dsa3d_dwconv3d_sw_kernel"};
+      "dsa3d_bwd_kv_tc_kernel", "dsa3d_bwd_dq_tc_kernel", "dsa3d_dwconv3d_sw_kernel",
+      "dsa3d_dwconv3d_sw2_kernel"};
   return names[id];
 }
 

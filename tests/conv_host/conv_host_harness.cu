@@ -33,10 +33,10 @@ void init_acc(float2 (&acc)[2][kConvStrip], const float* b, int c2) {
       acc[r][i] = b ? make_float2(b[2 * c2], b[2 * c2 + 1]) : make_float2(0.f, 0.f);
 }
 
-// The forward as the library launches it: the staged kernel's blocks (channel group, run of
-// kConvSwUnits units), each staging its group's weights with conv_sw_index and its warps taking
-// the units in turn, when the kernel has at most kConvSwMaxTaps taps; else the global kernel's
-// items (unit, channel pair).
+// The forward as the library launches it: with at most kConvSwMaxTaps taps, the strip-pair
+// kernel's blocks for C a multiple of 32 and the staged kernel's blocks otherwise (channel group,
+// slot of units; each stages its group's weights and its warps take the units in turn); else the
+// global kernel's items (unit, channel pair).
 template <typename T, int KW>
 void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, int flip, float* y) {
   const int pairs = g.C / 2, nxs = (g.Wp + kConvStrip - 1) / kConvStrip, nyp = (g.Hp + 1) / 2;
@@ -51,6 +51,41 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
       init_acc(acc, b, c2);
       conv_strip2<T, KW>(x, ConvWGlobal{w + 2 * c2 * (int64_t)K, K}, g, t, y0, x0, c2, flip != 0, acc);
       store_strips<T, KW>(acc, g, t, y0, x0, c2, y);
+    }
+    return;
+  }
+  if (g.C % (2 * kSw2Pairs) == 0) {
+    // the strip-pair kernel: each lane runs with its own copy of the warp's ring (the host fetch
+    // copies every chunk of a row, so a lane alone sees what the whole warp would)
+    using S = Sw2Ring<T, KW>;
+    const int nxp = (g.Wp + 2 * kConvStrip - 1) / (2 * kConvStrip);
+    const int64_t units2 = (int64_t)g.F * nyp * nxp;
+    const int64_t slots = (units2 + kSw2Units - 1) / kSw2Units;
+    const int groups2 = g.C / (2 * kSw2Pairs);
+    std::vector<float> ws((size_t)K * kSw2WStride);
+    std::vector<typename S::R> ring((size_t)kSw2Stages * S::ROW);
+    for (int64_t blk = 0; blk < slots * groups2; blk++) {
+      const int grp = (int)(blk % groups2);
+      const int64_t slot = blk / groups2;
+      const int c0 = 2 * kSw2Pairs * grp;
+      std::fill(ws.begin(), ws.end(), std::nanf(""));  // padding stays poisoned
+      for (int cc = 0; cc < 2 * kSw2Pairs; cc++)
+        for (int k = 0; k < K; k++) ws[(size_t)k * kSw2WStride + cc] = w[(int64_t)(c0 + cc) * K + k];
+      for (int warp = 0; warp < kConvSwWarps; warp++)
+        for (int lane = 0; lane < 32; lane++) {
+          const int h = lane >> 4, p = lane & (kSw2Pairs - 1);
+          const int c2 = kSw2Pairs * grp + p;
+          for (int i = 0; i < kSw2Units / kConvSwWarps; i++) {
+            const int64_t unit = conv_sw_unit(slot, slots, warp, i);
+            if (unit >= units2) break;
+            int xb;
+            conv_unit2(unit, nxp, nyp, t, y0, xb);
+            init_acc(acc, b, c2);
+            conv_strip2_ring<T, KW>(ring.data(), lane, x + c0, ConvWSharedT<kSw2WStride>{ws.data() + 2 * p}, g, t,
+                                    y0, xb, flip != 0, acc);
+            store_strips<T, KW>(acc, g, t, y0, xb + h * kConvStrip, c2, y);
+          }
+        }
     }
     return;
   }

@@ -87,8 +87,11 @@ CASES = [((3, 5, 6), 4, (3, 3, 3)), ((2, 7, 19), 6, (3, 5, 9)), ((4, 3, 11), 2, 
 
 
 # The forward's staged kernel: two runs of units and a last channel group of one pair (C = 66);
-# three groups, the last partial (C = 160); and 405 taps, past the staged limit (the global kernel).
-FWD_CASES = CASES + [((4, 7, 40), 66, (3, 5, 9)), ((3, 5, 6), 160, (3, 3, 3)), ((3, 5, 12), 4, (5, 9, 9))]
+# the strip-pair kernel over five groups (C = 160); and 405 taps, past the staged limit (the
+# global kernel).
+FWD_CASES = CASES + [((4, 7, 40), 66, (3, 5, 9)), ((3, 5, 6), 160, (3, 3, 3)), ((3, 5, 12), 4, (5, 9, 9)),
+                     # C a multiple of 32 (the strip-pair kernel): a ragged last strip pair, k_w = 15
+                     ((4, 9, 21), 64, (3, 9, 9)), ((2, 7, 40), 32, (1, 5, 15))]
 # dW's kernel-row groups of three: kh = 7 (3 + 3 + 1) and kh = 9 as well; C a multiple of 64 (the
 # warp-cooperative copies), with a ragged last strip
 DW_CASES = FWD_CASES + [((3, 4, 10), 4, (3, 7, 3)), ((3, 5, 12), 128, (3, 9, 9)), ((2, 4, 19), 64, (1, 3, 5))]

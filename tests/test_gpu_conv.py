@@ -19,8 +19,10 @@ pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("gpu_lib", "oracle_lib")]
 CASES = [((3, 5, 6), 4, (3, 3, 3)), ((2, 7, 19), 6, (3, 5, 9)), ((4, 3, 11), 2, (1, 1, 15)),
          ((1, 4, 9), 8, (1, 3, 1)), ((5, 2, 17), 4, (5, 3, 7)), ((4, 9, 16), 64, (3, 9, 9)),
          # the forward's staged kernel over two runs of units with a last channel group of one pair,
-         # over three groups (the last partial), and a 405-tap kernel past its limit (global kernel)
-         ((4, 7, 40), 66, (3, 5, 9)), ((3, 5, 6), 160, (3, 3, 3)), ((3, 5, 12), 4, (5, 9, 9))]
+         # the strip-pair kernel (C a multiple of 32) over five groups, with a ragged last strip pair
+         # and at k_w = 15, and a 405-tap kernel past the staged limit (global kernel)
+         ((4, 7, 40), 66, (3, 5, 9)), ((3, 5, 6), 160, (3, 3, 3)), ((4, 9, 21), 64, (3, 9, 9)),
+         ((2, 7, 40), 32, (1, 5, 15)), ((3, 5, 12), 4, (5, 9, 9))]
 
 
 def _problem(dims, C, window, dtype, seed):
