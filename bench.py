@@ -54,6 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--e2e-groups", type=int, default=0,
+                    help="head groups of the end-to-end leg (a divisor of the heads; 0: the default choice)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--part", choices=["attention", "dwconv"], default="attention",
@@ -669,10 +671,17 @@ def e2e_leg(args, w, host, abi, torch, dev, world, code):
     # the largest group that fits, with four groups or more where the heads allow it (the first
     # group's inputs and the last one's outputs are the pipeline's fill and drain)
     g = 1
-    for cand in list(range(H // 4, 0, -1)) + list(range(H // 2, H // 4, -1)):
-        if cand >= 1 and H % cand == 0 and 2 * slot_bytes(cand) + ws_bytes(cand) <= budget:
-            g = cand
-            break
+    if args.e2e_groups > 0:
+        if H % args.e2e_groups:
+            raise SystemExit(f"--e2e-groups {args.e2e_groups} does not divide the {H} heads")
+        g = H // args.e2e_groups
+        if 2 * slot_bytes(g) + ws_bytes(g) > budget:
+            raise SystemExit(f"--e2e-groups {args.e2e_groups}: the group's device buffers do not fit")
+    else:
+        for cand in list(range(H // 4, 0, -1)) + list(range(H // 2, H // 4, -1)):
+            if cand >= 1 and H % cand == 0 and 2 * slot_bytes(cand) + ws_bytes(cand) <= budget:
+                g = cand
+                break
     G = H // g
     slots = []
     for _ in range(2):
