@@ -85,7 +85,8 @@ dsa3d_status_t dwconv_launch_kw(const ConvGeo& g, const void* x, const float* w,
   const T* xt = static_cast<const T*>(x);
   const OutT* at = static_cast<const OutT*>(add);
   OutT* yt = static_cast<OutT*>(y);
-  const int64_t sw2_units = (int64_t)g.F * ((g.Hp + 1) / 2) * ((g.Wp + 2 * kConvStrip - 1) / (2 * kConvStrip));
+  const int64_t sw2_units =
+      (int64_t)g.F * ((g.Hp + kSw2Rows - 1) / kSw2Rows) * ((g.Wp + 2 * kConvStrip - 1) / (2 * kConvStrip));
   const int64_t sw2_grid = (sw2_units + kSw2Units - 1) / kSw2Units * (g.C / (2 * kSw2Pairs));
   if (K <= kConvSwMaxTaps && g.C % (2 * kSw2Pairs) == 0 && sw2_grid <= INT_MAX) {
     // strip pairs with a warp-shared row ring

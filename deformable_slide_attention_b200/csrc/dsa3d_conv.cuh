@@ -573,14 +573,15 @@ __host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const 
 
 // ---- the forward on strip pairs, input rows through a warp-shared ring ----------------------
 // For C a multiple of 32: a block owns kSw2Pairs channel pairs and its warps take units of two
-// neighbouring strips (t, row pair y0, y0 + 1, columns xb .. xb + 2 kConvStrip - 1); lane 16 h +
-// p computes pair p of strip h.  The two strips' windows share one input row of NT tokens, which
+// neighbouring strips on kSw2Rows rows (t, rows y0 .. y0 + kSw2Rows - 1, columns xb .. xb + 2
+// kConvStrip - 1); lane 16 h + p computes pair p of strip h.  The two strips' windows share one input row of NT tokens, which
 // the warp copies into a ring in shared memory with 16-byte cp.async chunks, kSw2Stages - 1 rows
 // ahead of its use.
 constexpr int kSw2Pairs = 16;
 constexpr int kSw2WStride = 2 * kSw2Pairs + 2;  // floats per staged tap row (2 of padding)
 constexpr int kSw2Units = 32;                   // units per block, kSw2Units / kConvSwWarps per warp
 constexpr int kSw2Stages = 3;
+constexpr int kSw2Rows = 4;                     // output rows per unit
 
 template <typename T, int KW>
 struct Sw2Ring {
@@ -593,12 +594,13 @@ struct Sw2Ring {
   __host__ __device__ static constexpr size_t warp_bytes() { return (size_t)kSw2Stages * ROW * sizeof(R); }
 };
 
-// Unit `unit` of the strip-pair forward: frames, then row pairs, then strip pairs fastest.
-__host__ __device__ __forceinline__ void conv_unit2(int64_t unit, int nxp, int nyp, int& t, int& y0, int& xb) {
+// Unit `unit` of the strip-pair forward: frames, then groups of kSw2Rows rows (nyr of them), then
+// strip pairs (nxp) fastest.
+__host__ __device__ __forceinline__ void conv_unit2(int64_t unit, int nxp, int nyr, int& t, int& y0, int& xb) {
   xb = (int)(unit % nxp) * 2 * kConvStrip;
   const int64_t r = unit / nxp;
-  y0 = 2 * (int)(r % nyp);
-  t = (int)(r / nyp);
+  y0 = kSw2Rows * (int)(r % nyr);
+  t = (int)(r / nyr);
 }
 
 // Copy input row ys of frame ts (tokens xb - r_w .. xb - r_w + NT - 1 of the group's pairs; xg:
@@ -629,21 +631,23 @@ __host__ __device__ __forceinline__ void sw2_fetch(typename ConvRaw<T>::type* ri
   }
 }
 
-// conv_strip2 for lane 16 h + p of a strip-pair unit (strip x0 = xb + h kConvStrip, pair p of the
-// group), its input rows read from the warp's ring (ring: the warp's kSw2Stages rows).  The rows
-// run as one sequence over the kernel planes, as in conv_strip2.
+// The convolution sums of lane 16 h + p of a strip-pair unit (strip x0 = xb + h kConvStrip, pair
+// p of the group) for output rows y0 + o, o < kSw2Rows, added into acc[o]; flip and wget as in
+// conv_strip2.  The input rows y0 - r_h + r, r < kh + kSw2Rows - 1, of each kernel plane run as one
+// sequence, read from the warp's ring (ring: the warp's kSw2Stages rows); input row r feeds output
+// row y0 + o through kernel row r - o, whose weights are read for it.
 template <typename T, int KW, typename WGet>
-__host__ __device__ __forceinline__ void conv_strip2_ring(typename ConvRaw<T>::type* ring, int lane,
+__host__ __device__ __forceinline__ void conv_strips_ring(typename ConvRaw<T>::type* ring, int lane,
                                                           const T* xg, const WGet& wget, const ConvGeo& g,
                                                           int t, int y0, int xb, bool flip,
-                                                          float2 (&acc)[2][kConvStrip]) {
+                                                          float2 (&acc)[kSw2Rows][kConvStrip]) {
   using S = Sw2Ring<T, KW>;
   using R = typename S::R;
   constexpr int NJ = kConvStrip + KW - 1;
   constexpr int D = kSw2Stages - 1;
   const int h = lane >> 4, p = lane & (kSw2Pairs - 1);
   const int rt = (g.kt - 1) / 2, rh = (g.kh - 1) / 2;
-  const int rows = g.kh + 1, Q = g.kt * rows;
+  const int rows = g.kh + kSw2Rows - 1, Q = g.kt * rows;
   int fu = 0, fr = 0;  // plane and row of the next fetch
   auto fetch_next = [&](int q) {
     sw2_fetch<T, KW>(ring, lane, q % kSw2Stages, xg, g, t + fu - rt, y0 - rh + fr, xb);
@@ -658,7 +662,6 @@ __host__ __device__ __forceinline__ void conv_strip2_ring(typename ConvRaw<T>::t
     if (q < Q) fetch_next(q);
     dw_commit();
   }
-  float2 pr[NJ];
   int u = 0, r = 0;
   for (int q = 0; q < Q; q++) {
     dw_syncwarp();  // every lane's reads of row q - 1's stage are done
@@ -670,26 +673,24 @@ __host__ __device__ __forceinline__ void conv_strip2_ring(typename ConvRaw<T>::t
     float2 cr[NJ];
 #pragma unroll
     for (int j = 0; j < NJ; j++) cr[j] = conv_unpack(row[S::at(h * kConvStrip + j, p)]);
-    if (r > 0) {
-      const int v = r - 1;
+#pragma unroll
+    for (int o = 0; o < kSw2Rows; o++) {
+      const int v = r - o;
+      if (v < 0 || v >= g.kh) continue;
       const int64_t wrow = flip ? ((int64_t)(g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW
                                 : ((int64_t)u * g.kh + v) * KW;
       float2 w[KW];
 #pragma unroll
       for (int j = 0; j < KW; j++) w[j] = wget(wrow + (flip ? KW - 1 - j : j));
+      // input column x0 - r_w + j feeds output x0 + i through tap j - i
 #pragma unroll
       for (int j = 0; j < NJ; j++) {
 #pragma unroll
         for (int i = 0; i < kConvStrip; i++) {
-          if (j - i >= 0 && j - i < KW) {
-            conv_fma2(acc[0][i], w[j - i], pr[j]);
-            conv_fma2(acc[1][i], w[j - i], cr[j]);
-          }
+          if (j - i >= 0 && j - i < KW) conv_fma2(acc[o][i], w[j - i], cr[j]);
         }
       }
     }
-#pragma unroll
-    for (int j = 0; j < NJ; j++) pr[j] = cr[j];
     if (++r == rows) {
       r = 0;
       u++;
@@ -700,12 +701,12 @@ __host__ __device__ __forceinline__ void conv_strip2_ring(typename ConvRaw<T>::t
 #ifdef __CUDACC__
 // Writes the two strips acc (rows y0, y0 + 1 from column x0; channel pair c2), each element plus
 // add's (nullable; may equal y); rows and columns past the volume are not written.
-template <typename OutT>
-__device__ __forceinline__ void conv_store_strips(const float2 (&acc)[2][kConvStrip], const OutT* add,
+template <typename OutT, int NR>
+__device__ __forceinline__ void conv_store_strips(const float2 (&acc)[NR][kConvStrip], const OutT* add,
                                                   OutT* y, const ConvGeo& g, int t, int y0, int x0,
                                                   int c2) {
 #pragma unroll
-  for (int r = 0; r < 2; r++) {
+  for (int r = 0; r < NR; r++) {
     if (y0 + r >= g.Hp) break;
     const int64_t base = (((int64_t)t * g.Hp + y0 + r) * g.Wp + x0) * g.C + 2 * c2;
 #pragma unroll
@@ -724,9 +725,10 @@ __device__ __forceinline__ void conv_store_strips(const float2 (&acc)[2][kConvSt
   }
 }
 
-__device__ __forceinline__ void conv_acc_init(float2 (&acc)[2][kConvStrip], float b0, float b1) {
+template <int NR>
+__device__ __forceinline__ void conv_acc_init(float2 (&acc)[NR][kConvStrip], float b0, float b1) {
 #pragma unroll
-  for (int r = 0; r < 2; r++)
+  for (int r = 0; r < NR; r++)
 #pragma unroll
     for (int i = 0; i < kConvStrip; i++) acc[r][i] = make_float2(b0, b1);
 }
@@ -813,12 +815,12 @@ __host__ __device__ __forceinline__ size_t conv_sw2_weight_bytes(int K) {
 }
 
 // The forward on strip pairs (C a multiple of 32, at most kConvSwMaxTaps taps): a block owns one
-// group of kSw2Pairs channel pairs and kSw2Units strip-pair units of one slot (conv_sw_unit over
-// the strip-pair units), which its warps take in turn.  The group's weights are copied in once,
+// group of kSw2Pairs channel pairs and kSw2Units strip-pair units (kSw2Rows rows each) of one slot
+// (conv_sw_unit over the strip-pair units), which its warps take in turn.  The group's weights are copied in once,
 // tap-major with stride kSw2WStride; each warp then has kSw2Stages rows of ring.  Dynamic shared
 // memory: conv_sw2_weight_bytes(K) + kConvSwWarps Sw2Ring<T, KW>::warp_bytes().  Registers capped
-// for four blocks per SM up to k_w = 9 (126 at bf16 and k_w = 9, no spills: 180 -> 173 ms per
-// launch at 1080p) and three above (four would spill 40-340 bytes).
+// for four blocks per SM up to k_w = 9 (126 at bf16 and k_w = 9, no spills; capped for three
+// blocks the kernel takes 150 ms per launch at 1080p instead of 139) and three above.
 template <typename T, int KW, typename OutT = T>
 __global__ void __launch_bounds__(kConvSwWarps * 32, KW <= 9 ? 4 : 3)
     dsa3d_dwconv3d_sw2_kernel(const T* __restrict__ x, const float* __restrict__ w,
@@ -844,8 +846,8 @@ __global__ void __launch_bounds__(kConvSwWarps * 32, KW <= 9 ? 4 : 3)
   const int h = lane >> 4, p = lane & (kSw2Pairs - 1);
   const int c2 = kSw2Pairs * grp + p;
   const int nxp = (g.Wp + 2 * kConvStrip - 1) / (2 * kConvStrip);
-  const int nyp = (g.Hp + 1) / 2;
-  const int64_t units = (int64_t)g.F * nyp * nxp;
+  const int nyr = (g.Hp + kSw2Rows - 1) / kSw2Rows;
+  const int64_t units = (int64_t)g.F * nyr * nxp;
   const int64_t slots = (units + kSw2Units - 1) / kSw2Units;
   const ConvWSharedT<kSw2WStride> wsrc{ws_all + 2 * p};
   const float b0 = bias ? __ldg(bias + 2 * c2) : 0.f, b1 = bias ? __ldg(bias + 2 * c2 + 1) : 0.f;
@@ -855,10 +857,10 @@ __global__ void __launch_bounds__(kConvSwWarps * 32, KW <= 9 ? 4 : 3)
     const int64_t unit = conv_sw_unit(slot, slots, warp, i);
     if (unit >= units) break;  // warp-uniform; later steps' units are larger still
     int t, y0, xb;
-    conv_unit2(unit, nxp, nyp, t, y0, xb);
-    float2 acc[2][kConvStrip];
+    conv_unit2(unit, nxp, nyr, t, y0, xb);
+    float2 acc[kSw2Rows][kConvStrip];
     conv_acc_init(acc, b0, b1);
-    conv_strip2_ring<T, KW>(ring, lane, xg, wsrc, g, t, y0, xb, flip != 0, acc);
+    conv_strips_ring<T, KW>(ring, lane, xg, wsrc, g, t, y0, xb, flip != 0, acc);
     conv_store_strips(acc, add, y, g, t, y0, xb + h * kConvStrip, c2);
   }
 }

@@ -16,10 +16,10 @@ using namespace dsa3d;
 
 namespace {
 
-template <typename T, int KW>
-void store_strips(const float2 (&acc)[2][kConvStrip], const ConvGeo& g, int t, int y0, int x0, int c2,
+template <typename T, int KW, int NR = 2>
+void store_strips(const float2 (&acc)[NR][kConvStrip], const ConvGeo& g, int t, int y0, int x0, int c2,
                   float* y) {
-  for (int r = 0; r < 2 && y0 + r < g.Hp; r++)
+  for (int r = 0; r < NR && y0 + r < g.Hp; r++)
     for (int i = 0; i < kConvStrip && x0 + i < g.Wp; i++) {
       const int64_t o = (((int64_t)t * g.Hp + y0 + r) * g.Wp + x0 + i) * g.C + 2 * c2;
       y[o] = acc[r][i].x;
@@ -27,8 +27,9 @@ void store_strips(const float2 (&acc)[2][kConvStrip], const ConvGeo& g, int t, i
     }
 }
 
-void init_acc(float2 (&acc)[2][kConvStrip], const float* b, int c2) {
-  for (int r = 0; r < 2; r++)
+template <int NR>
+void init_acc(float2 (&acc)[NR][kConvStrip], const float* b, int c2) {
+  for (int r = 0; r < NR; r++)
     for (int i = 0; i < kConvStrip; i++)
       acc[r][i] = b ? make_float2(b[2 * c2], b[2 * c2 + 1]) : make_float2(0.f, 0.f);
 }
@@ -59,7 +60,8 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
     // copies every chunk of a row, so a lane alone sees what the whole warp would)
     using S = Sw2Ring<T, KW>;
     const int nxp = (g.Wp + 2 * kConvStrip - 1) / (2 * kConvStrip);
-    const int64_t units2 = (int64_t)g.F * nyp * nxp;
+    const int nyr = (g.Hp + kSw2Rows - 1) / kSw2Rows;
+    const int64_t units2 = (int64_t)g.F * nyr * nxp;
     const int64_t slots = (units2 + kSw2Units - 1) / kSw2Units;
     const int groups2 = g.C / (2 * kSw2Pairs);
     std::vector<float> ws((size_t)K * kSw2WStride);
@@ -79,11 +81,12 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
             const int64_t unit = conv_sw_unit(slot, slots, warp, i);
             if (unit >= units2) break;
             int xb;
-            conv_unit2(unit, nxp, nyp, t, y0, xb);
-            init_acc(acc, b, c2);
-            conv_strip2_ring<T, KW>(ring.data(), lane, x + c0, ConvWSharedT<kSw2WStride>{ws.data() + 2 * p}, g, t,
-                                    y0, xb, flip != 0, acc);
-            store_strips<T, KW>(acc, g, t, y0, xb + h * kConvStrip, c2, y);
+            conv_unit2(unit, nxp, nyr, t, y0, xb);
+            float2 acc4[kSw2Rows][kConvStrip];
+            init_acc(acc4, b, c2);
+            conv_strips_ring<T, KW>(ring.data(), lane, x + c0, ConvWSharedT<kSw2WStride>{ws.data() + 2 * p}, g, t,
+                                    y0, xb, flip != 0, acc4);
+            store_strips<T, KW, kSw2Rows>(acc4, g, t, y0, xb + h * kConvStrip, c2, y);
           }
         }
     }
