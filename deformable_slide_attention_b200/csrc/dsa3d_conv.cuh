@@ -15,8 +15,8 @@
 // coalesced 128- or 256-byte row segment) and, in the forward, two strips of kConvStrip outputs
 // along x in consecutive rows.  Per kernel plane u it loads each of the kh + 1 input rows'
 // kConvStrip + KW - 1 values once and each kernel row's KW weights once, and does
-// 2 kConvStrip KW FMAs per channel per kernel row from registers; in the forward the pair's two
-// channels share one packed fp32x2 FMA (conv_fma2).
+// 2 kConvStrip KW FMAs per channel per kernel row from registers; the pair's two channels share
+// one packed fp32x2 FMA (conv_fma2).
 //
 // The per-thread arithmetic (conv_strip2, dw_walk) is __host__ __device__ code so that a host
 // harness can run exactly these routines on the CPU.
@@ -497,10 +497,7 @@ __host__ __device__ __forceinline__ void dw_step(const DwRing<T, TD, KW>& r, int
     for (int j = 0; j < NJ; j++) {
 #pragma unroll
       for (int k = 0; k < kConvStrip; k++) {
-        if (j - k >= 0 && j - k < KW) {  // scalar FMAs: the packed form took more registers here
-          dwr[i][j - k].x = fmaf(d[i][k].x, a[j].x, dwr[i][j - k].x);
-          dwr[i][j - k].y = fmaf(d[i][k].y, a[j].y, dwr[i][j - k].y);
-        }
+        if (j - k >= 0 && j - k < KW) conv_fma2(dwr[i][j - k], d[i][k], a[j]);
       }
     }
   }
