@@ -134,14 +134,12 @@ __host__ __device__ __forceinline__ int conv_sw_index(int k, int cc) { return k 
 __host__ __device__ __forceinline__ size_t conv_sw_bytes(int K) {
   return (size_t)K * kConvGroupStride * sizeof(float);
 }
-template <int Stride>
-struct ConvWSharedT {
-  const float* s;  // the staged group + 2 * (the lane's pair) (8-byte aligned: Stride is even)
+struct ConvWShared {
+  const float* s;  // the staged group + 2 * lane (8-byte aligned: the stride is even)
   __host__ __device__ __forceinline__ float2 operator()(int64_t k) const {
-    return *reinterpret_cast<const float2*>(s + (int)k * Stride);
+    return *reinterpret_cast<const float2*>(s + (int)k * kConvGroupStride);
   }
 };
-using ConvWShared = ConvWSharedT<kConvGroupStride>;
 
 // Unit (t, y0, x0) of the forward's work: output rows y0, y0 + 1 from column x0, strips fastest,
 // then row pairs, then frames.
@@ -629,14 +627,15 @@ __host__ __device__ __forceinline__ void sw2_fetch(typename ConvRaw<T>::type* ri
 }
 
 // The convolution sums of lane 16 h + p of a strip-pair unit (strip x0 = xb + h kConvStrip, pair
-// p of the group) for output rows y0 + o, o < kSw2Rows, added into acc[o]; flip and wget as in
-// conv_strip2.  The input rows y0 - r_h + r, r < kh + kSw2Rows - 1, of each kernel plane run as one
+// p of the group) for output rows y0 + o, o < kSw2Rows, added into acc[o]; Flip as in
+// conv_strip2, the weights read from the staged group at wsp (its tap rows kSw2WStride floats
+// apart, the lane's pair at 2 p).  The input rows y0 - r_h + r, r < kh + kSw2Rows - 1, of each kernel plane run as one
 // sequence, read from the warp's ring (ring: the warp's kSw2Stages rows); input row r feeds output
 // row y0 + o through kernel row r - o, whose weights are read for it.
-template <typename T, int KW, typename WGet>
+template <typename T, int KW, bool Flip>
 __host__ __device__ __forceinline__ void conv_strips_ring(typename ConvRaw<T>::type* ring, int lane,
-                                                          const T* xg, const WGet& wget, const ConvGeo& g,
-                                                          int t, int y0, int xb, bool flip,
+                                                          const T* xg, const float* wsp, const ConvGeo& g,
+                                                          int t, int y0, int xb,
                                                           float2 (&acc)[kSw2Rows][kConvStrip]) {
   using S = Sw2Ring<T, KW>;
   using R = typename S::R;
@@ -666,19 +665,24 @@ __host__ __device__ __forceinline__ void conv_strips_ring(typename ConvRaw<T>::t
     dw_commit();
     dw_wait<D>();
     dw_syncwarp();  // every lane's copies of row q have landed
-    const R* row = ring + (q % kSw2Stages) * S::ROW;
+    // the lane's tokens h kConvStrip + j: entry (h (kConvStrip + 1) + j + j / 8) kSw2Pairs + p
+    const R* row = ring + (q % kSw2Stages) * S::ROW + h * (kConvStrip + 1) * kSw2Pairs + p;
+    static_assert(kConvStrip == 8, "the ring's bank shift is per 8 tokens");
     float2 cr[NJ];
 #pragma unroll
-    for (int j = 0; j < NJ; j++) cr[j] = conv_unpack(row[S::at(h * kConvStrip + j, p)]);
+    for (int j = 0; j < NJ; j++) cr[j] = conv_unpack(row[(j + (j >> 3)) * kSw2Pairs]);
 #pragma unroll
     for (int o = 0; o < kSw2Rows; o++) {
       const int v = r - o;
       if (v < 0 || v >= g.kh) continue;
-      const int64_t wrow = flip ? ((int64_t)(g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW
-                                : ((int64_t)u * g.kh + v) * KW;
+      // kernel row (u, v)'s weights, tap j at wr[j kSw2WStride] (flipped for the transposed
+      // convolution: W[c][kt-1-u][kh-1-v][kw-1-j])
+      const int wrow = Flip ? ((g.kt - 1 - u) * g.kh + (g.kh - 1 - v)) * KW : (u * g.kh + v) * KW;
+      const float* wr = wsp + wrow * kSw2WStride;
       float2 w[KW];
 #pragma unroll
-      for (int j = 0; j < KW; j++) w[j] = wget(wrow + (flip ? KW - 1 - j : j));
+      for (int j = 0; j < KW; j++)
+        w[j] = *reinterpret_cast<const float2*>(wr + (Flip ? KW - 1 - j : j) * kSw2WStride);
       // input column x0 - r_w + j feeds output x0 + i through tap j - i
 #pragma unroll
       for (int j = 0; j < NJ; j++) {
@@ -846,7 +850,7 @@ __global__ void __launch_bounds__(kConvSwWarps * 32, KW <= 9 ? 4 : 3)
   const int nyr = (g.Hp + kSw2Rows - 1) / kSw2Rows;
   const int64_t units = (int64_t)g.F * nyr * nxp;
   const int64_t slots = (units + kSw2Units - 1) / kSw2Units;
-  const ConvWSharedT<kSw2WStride> wsrc{ws_all + 2 * p};
+  const float* wsp = ws_all + 2 * p;
   const float b0 = bias ? __ldg(bias + 2 * c2) : 0.f, b1 = bias ? __ldg(bias + 2 * c2 + 1) : 0.f;
   const T* xg = x + c0;
   static_assert(kSw2Units % kConvSwWarps == 0, "whole steps of the warps");
@@ -857,7 +861,10 @@ __global__ void __launch_bounds__(kConvSwWarps * 32, KW <= 9 ? 4 : 3)
     conv_unit2(unit, nxp, nyr, t, y0, xb);
     float2 acc[kSw2Rows][kConvStrip];
     conv_acc_init(acc, b0, b1);
-    conv_strips_ring<T, KW>(ring, lane, xg, wsrc, g, t, y0, xb, flip != 0, acc);
+    if (flip)
+      conv_strips_ring<T, KW, true>(ring, lane, xg, wsp, g, t, y0, xb, acc);
+    else
+      conv_strips_ring<T, KW, false>(ring, lane, xg, wsp, g, t, y0, xb, acc);
     conv_store_strips(acc, add, y, g, t, y0, xb + h * kConvStrip, c2);
   }
 }

@@ -84,8 +84,10 @@ void forward_all(const T* x, const float* w, const float* b, const ConvGeo& g, i
             conv_unit2(unit, nxp, nyr, t, y0, xb);
             float2 acc4[kSw2Rows][kConvStrip];
             init_acc(acc4, b, c2);
-            conv_strips_ring<T, KW>(ring.data(), lane, x + c0, ConvWSharedT<kSw2WStride>{ws.data() + 2 * p}, g, t,
-                                    y0, xb, flip != 0, acc4);
+            if (flip)
+              conv_strips_ring<T, KW, true>(ring.data(), lane, x + c0, ws.data() + 2 * p, g, t, y0, xb, acc4);
+            else
+              conv_strips_ring<T, KW, false>(ring.data(), lane, x + c0, ws.data() + 2 * p, g, t, y0, xb, acc4);
             store_strips<T, KW, kSw2Rows>(acc4, g, t, y0, xb + h * kConvStrip, c2, y);
           }
         }
