@@ -433,6 +433,37 @@ __host__ __device__ __forceinline__ void dw_fetch(const DwRing<T, TD, KW>& r, in
 // point at the lane's own pair; the chunks a lane copies belong to other lanes too, so the ring
 // is shared within the warp (dw_syncwarp around its use).  On the host one call copies every
 // chunk of the warp.
+// The 16-byte chunks of one staged run of `tokens` tokens (32 pairs of R each: CPT = 2 sizeof(R)
+// chunks per token) that lane `lane` copies: chunk m = lane + 32 i is token m / CPT, chunk m mod
+// CPT, so the lane's token advances by 32 / CPT per chunk and its offset in the token is fixed.
+// src0: pair 0 of token 0 of the run (tokens C elements apart), ok(j): token j inside the volume;
+// dst0: the run's ring entries (token j at dst0 + j 32 sizeof(R) bytes).
+template <typename R, int TOKENS, typename TS, typename OK>
+__host__ __device__ __forceinline__ void dw_copy_run(unsigned char* dst0, const TS* src0, const TS* fallback,
+                                                     int64_t C, int lane, OK ok) {
+  constexpr int CPT = 32 * (int)sizeof(R) / 16;
+  constexpr int TSTEP = 32 / CPT;  // tokens between a lane's chunks
+  const int j0 = lane / CPT, q = lane % CPT;
+  const unsigned char* src = reinterpret_cast<const unsigned char*>(src0 + j0 * C) + 16 * q;
+  unsigned char* dst = dst0 + (size_t)j0 * 32 * sizeof(R) + 16 * q;
+  const int64_t sstep = TSTEP * C * (int64_t)sizeof(TS);
+#pragma unroll
+  for (int i = 0; i < (TOKENS + TSTEP - 1) / TSTEP; i++) {
+    const int j = j0 + i * TSTEP;
+    if (j < TOKENS) {
+      const bool in = ok(j);
+      dw_copy16(dst + (size_t)i * TSTEP * 32 * sizeof(R), in ? src + i * sstep : reinterpret_cast<const unsigned char*>(fallback), in);
+    }
+  }
+}
+
+// dw_fetch for the whole warp at once, when its 32 lanes are 32 consecutive channel pairs from a
+// multiple of 32 (C a multiple of 64) on the same work item: a token's 32 pairs are one
+// contiguous run of 128 (bf16) or 256 (fp32) bytes, copied as 16-byte chunks spread over the
+// lanes (dw_copy_run), each chunk into the 16 bytes of the ring entry that hold those pairs.
+// xplane and dplane point at the lane's own pair; the chunks a lane copies belong to other lanes
+// too, so the ring is shared within the warp (dw_syncwarp around its use).  On the host one call
+// copies every lane's chunks.
 template <typename T, typename TD, int KW>
 __host__ __device__ __forceinline__ void dw_fetch_warp(const DwRing<T, TD, KW>& r, int lane, int st,
                                                        const T* xplane, const TD* dplane, const ConvGeo& g,
@@ -440,34 +471,27 @@ __host__ __device__ __forceinline__ void dw_fetch_warp(const DwRing<T, TD, KW>& 
   using R = DwRing<T, TD, KW>;
   using XR = typename R::XR;
   using DR = typename R::DR;
-  constexpr int CX = 32 * (int)sizeof(XR) / 16, CD = 32 * (int)sizeof(DR) / 16;  // chunks per token
   const int rw = (KW - 1) / 2, rh = (g.kh - 1) / 2;
   const T* xw = xplane - 2 * lane;  // pair 0 of the warp
   const TD* dw = dplane - 2 * lane;
-  unsigned char* rx = reinterpret_cast<unsigned char*>(r.x - lane);
-  unsigned char* rd = reinterpret_cast<unsigned char*>(r.d - lane);
-#ifdef __CUDA_ARCH__
-  const int m0 = lane, mstep = 32;
-#else
-  const int m0 = 0, mstep = 1;
-#endif
-  const T* xrow = xw + (int64_t)ys * g.Wp * g.C;
-  for (int m = m0; m < R::NJ * CX; m += mstep) {
-    const int j = m / CX, q = m - j * CX;
-    const int xs = x0 - rw + j;
-    const bool ok = xs >= 0 && xs < g.Wp;
-    const unsigned char* src = reinterpret_cast<const unsigned char*>(ok ? xrow + (int64_t)xs * g.C : xw) + 16 * q;
-    dw_copy16(rx + ((size_t)(st * R::NJ + j) * 32) * sizeof(XR) + 16 * q, src, ok);
-  }
+  unsigned char* rx = reinterpret_cast<unsigned char*>(r.x - lane) + (size_t)st * R::NJ * 32 * sizeof(XR);
+  unsigned char* rd = reinterpret_cast<unsigned char*>(r.d - lane) + (size_t)st * kConvStrip * 32 * sizeof(DR);
+  const int xs0 = x0 - rw;
+  const T* xsrc = xw + ((int64_t)ys * g.Wp + xs0) * g.C;  // token xs0 of row ys (not read unless inside)
   const int y = ys - v0 + rh;
   const bool yin = y >= 0 && y < g.Hp;
-  const TD* drow = yin ? dw + ((int64_t)y * g.Wp + x0) * g.C : dw;
-  for (int m = m0; m < kConvStrip * CD; m += mstep) {
-    const int k = m / CD, q = m - k * CD;
-    const bool ok = yin && x0 + k < g.Wp;
-    const unsigned char* src = reinterpret_cast<const unsigned char*>(ok ? drow + (int64_t)k * g.C : dw) + 16 * q;
-    dw_copy16(rd + ((size_t)(st * kConvStrip + k) * 32) * sizeof(DR) + 16 * q, src, ok);
+  const TD* dsrc = dw + ((int64_t)(yin ? y : 0) * g.Wp + x0) * g.C;
+  auto xok = [&](int j) { return xs0 + j >= 0 && xs0 + j < g.Wp; };
+  auto dok = [&](int k) { return yin && x0 + k < g.Wp; };
+#ifdef __CUDA_ARCH__
+  dw_copy_run<XR, R::NJ>(rx, xsrc, xw, g.C, lane, xok);
+  dw_copy_run<DR, kConvStrip>(rd, dsrc, dw, g.C, lane, dok);
+#else
+  for (int l = 0; l < 32; l++) {
+    dw_copy_run<XR, R::NJ>(rx, xsrc, xw, g.C, l, xok);
+    dw_copy_run<DR, kConvStrip>(rd, dsrc, dw, g.C, l, dok);
   }
+#endif
 }
 
 // Step of the walk whose data sit in ring stage st: the carried dY strips move one slot down
@@ -598,32 +622,47 @@ __host__ __device__ __forceinline__ void conv_unit2(int64_t unit, int nxp, int n
   t = (int)(r / nyr);
 }
 
-// Copy input row ys of frame ts (tokens xb - r_w .. xb - r_w + NT - 1 of the group's pairs; xg:
-// x at the group's first channel) into ring stage st, zeros outside the volume.  The warp's lanes
-// share the chunks; on the host one call copies them all.
 template <typename T, int KW>
-__host__ __device__ __forceinline__ void sw2_fetch(typename ConvRaw<T>::type* ring, int lane, int st,
-                                                   const T* xg, const ConvGeo& g, int ts, int ys, int xb) {
+__host__ __device__ __forceinline__ void sw2_fetch_lane(typename ConvRaw<T>::type* ring, int lane, int st,
+                                                        const T* xg, const ConvGeo& g, int ts, int ys, int xb) {
   using S = Sw2Ring<T, KW>;
   using R = typename S::R;
   constexpr int CPT = kSw2Pairs * (int)sizeof(R) / 16;  // 16-byte chunks per token
+  constexpr int TSTEP = 32 / CPT;                       // tokens between a lane's chunks
+  // the lane's first token j0 < TSTEP, so token j0 + i TSTEP's bank-shift group is (i TSTEP) / 8
+  static_assert(TSTEP % 8 == 0 || 8 % TSTEP == 0, "chunk steps aligned with the 8-token bank shift");
   const int rw = (KW - 1) / 2;
   const bool rin = ts >= 0 && ts < g.F && ys >= 0 && ys < g.Hp;
-  const T* row = rin ? xg + ((int64_t)ts * g.Hp + ys) * g.Wp * g.C : xg;
-  R* dst = ring + st * S::ROW;
+  const int xs0 = xb - rw;
+  const T* row = xg + (((int64_t)(rin ? ts : 0) * g.Hp + (rin ? ys : 0)) * g.Wp + xs0) * g.C;  // token xs0
+  const int j0 = lane / CPT, q = lane % CPT;
+  const unsigned char* src = reinterpret_cast<const unsigned char*>(row + (int64_t)j0 * g.C) + 16 * q;
+  unsigned char* dst = reinterpret_cast<unsigned char*>(ring + st * S::ROW + j0 * kSw2Pairs) + 16 * q;
+  const int64_t sstep = (int64_t)TSTEP * g.C * (int64_t)sizeof(T);
+#pragma unroll
+  for (int i = 0; i < (S::NT + TSTEP - 1) / TSTEP; i++) {
+    const int j = j0 + i * TSTEP;
+    if (j < S::NT) {
+      const bool ok = rin && xs0 + j >= 0 && xs0 + j < g.Wp;
+      const size_t doff = (size_t)(i * TSTEP + ((i * TSTEP) >> 3)) * kSw2Pairs * sizeof(R);  // S::at(j) - S::at(j0)
+      dw_copy16(dst + doff, ok ? src + i * sstep : reinterpret_cast<const unsigned char*>(xg), ok);
+    }
+  }
+}
+
+// Copy input row ys of frame ts (tokens xb - r_w .. xb - r_w + NT - 1 of the group's pairs; xg:
+// x at the group's first channel) into ring stage st, zeros outside the volume: chunk m = lane +
+// 32 i of the row's 16-byte chunks (token m / CPT, chunk m mod CPT) is lane `lane`'s.  On the
+// host one call copies every lane's chunks.
+template <typename T, int KW>
+__host__ __device__ __forceinline__ void sw2_fetch(typename ConvRaw<T>::type* ring, int lane, int st,
+                                                   const T* xg, const ConvGeo& g, int ts, int ys, int xb) {
 #ifdef __CUDA_ARCH__
-  const int m0 = lane, mstep = 32;
+  sw2_fetch_lane<T, KW>(ring, lane, st, xg, g, ts, ys, xb);
 #else
-  const int m0 = 0, mstep = 1;
+  for (int l = 0; l < 32; l++) sw2_fetch_lane<T, KW>(ring, l, st, xg, g, ts, ys, xb);
   (void)lane;
 #endif
-  for (int m = m0; m < S::NT * CPT; m += mstep) {
-    const int j = m / CPT, q = m - j * CPT;
-    const int xs = xb - rw + j;
-    const bool ok = rin && xs >= 0 && xs < g.Wp;
-    const unsigned char* src = reinterpret_cast<const unsigned char*>(ok ? row + (int64_t)xs * g.C : xg) + 16 * q;
-    dw_copy16(reinterpret_cast<unsigned char*>(dst + S::at(j, 0)) + 16 * q, src, ok);
-  }
 }
 
 // The convolution sums of lane 16 h + p of a strip-pair unit (strip x0 = xb + h kConvStrip, pair
