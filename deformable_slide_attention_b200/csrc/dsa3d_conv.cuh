@@ -9,17 +9,23 @@
 // with the kernel flipped on every axis; dW[c][u][v][w] = sum_p dY[p][c] X[p + tap offset][c].
 //
 // At the window's extent (3 x 9 x 9) the convolution does 2 C K flop per token for 4 C bytes of
-// bf16 traffic: about 120 flop per byte, so it is bound by the fp32 FMA pipes, not by HBM.  The
-// kernels block registers along x and y: a thread owns one channel pair (a 4-byte bf16x2 or
-// 8-byte float2 load, consecutive threads on consecutive pairs, so a warp's loads are one
-// coalesced 128- or 256-byte row segment) and, in the forward, two strips of kConvStrip outputs
-// along x in consecutive rows.  Per kernel plane u it loads each of the kh + 1 input rows'
-// kConvStrip + KW - 1 values once and each kernel row's KW weights once, and does
-// 2 kConvStrip KW FMAs per channel per kernel row from registers; the pair's two channels share
-// one packed fp32x2 FMA (conv_fma2).
+// bf16 traffic: about 120 flop per byte, so it is bound by the fp32 FMA pipes, not by HBM.  Every
+// kernel gives a thread one channel pair (consecutive lanes on consecutive pairs, so a warp's
+// loads of one token are one coalesced 128- or 256-byte run) and blocks registers along x (strips
+// of kConvStrip outputs) and y; the pair's two channels share one packed fp32x2 FMA (conv_fma2).
 //
-// The per-thread arithmetic (conv_strip2, dw_walk) is __host__ __device__ code so that a host
-// harness can run exactly these routines on the CPU.
+//   forward and dX, at most kConvSwMaxTaps taps:
+//     dsa3d_dwconv3d_sw2_kernel (C a multiple of 32): units of two neighbouring strips on
+//       kSw2Rows rows; the block's weights staged tap-major in shared memory, the input rows
+//       copied by the warp into a ring in shared memory (16-byte cp.async chunks, two rows ahead);
+//     dsa3d_dwconv3d_sw_kernel (other C): one strip on two rows per thread, the weights staged,
+//       the rows loaded one row ahead into registers;
+//   forward and dX, larger kernels: dsa3d_dwconv3d_kernel, the weights read from global memory;
+//   dW and db: dsa3d_dwconv3d_dw_kernel, a thread on three kernel rows of a plane walking a strip
+//     column down the input rows, the rows and dY strips through a per-warp cp.async ring.
+//
+// The per-thread arithmetic (conv_strip2, conv_strips_ring, dw_walk and their copy routines) is
+// __host__ __device__ code so that a host harness can run exactly these routines on the CPU.
 #pragma once
 
 #include <cuda_bf16.h>
