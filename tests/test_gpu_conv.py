@@ -203,3 +203,24 @@ def test_full_size_sampled_channels(name):
     finally:
         del x, y, dy, gx, gw, gb
         torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_forward_kernels_agree_bit_for_bit(dtype):
+    """The strip-pair kernel (C a multiple of 32) and the staged kernel (other channel counts) add
+    the same products in the same order (kernel planes, then kernel rows, then taps, each output's
+    sum starting from its bias), so a channel's outputs do not depend on which one ran: channels
+    0..63 of a 66-channel problem (staged kernel) equal the 64-channel problem made of them
+    (strip-pair kernel) exactly, for the forward with the add and for dX."""
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    dims, window = (4, 9, 21), (3, 9, 9)
+    x, w, b, add, dy = _problem(dims, 66, window, td, 66)
+    sub = lambda t: t[:, :64].contiguous()
+    y66 = abi.dwconv3d(x.cuda(), w.cuda(), b.cuda(), dims, add=add.cuda())
+    y64 = abi.dwconv3d(sub(x).cuda(), w[:64].contiguous().cuda(), b[:64].contiguous().cuda(), dims,
+                       add=sub(add).cuda())
+    gx66, _, _ = abi.dwconv3d_backward(x.cuda(), w.cuda(), dy.cuda(), dims)
+    gx64, _, _ = abi.dwconv3d_backward(sub(x).cuda(), w[:64].contiguous().cuda(), sub(dy).cuda(), dims)
+    torch.cuda.synchronize()
+    assert torch.equal(y66[:, :64], y64)
+    assert torch.equal(gx66[:, :64], gx64)
