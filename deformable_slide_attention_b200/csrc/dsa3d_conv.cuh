@@ -190,11 +190,11 @@ __host__ __device__ __forceinline__ float2 conv_unpack(unsigned u) {
 // Convolution sums of channel pair c2 (channels 2 c2 and 2 c2 + 1) for the two output strips
 // (t, y0 + r, x0 + i), r < 2, i < kConvStrip, added into acc[r][i] (.x: channel 2 c2, .y: 2 c2 +
 // 1).  For kernel plane u the input rows y0 - r_h .. y0 + 1 + r_h are loaded once each, and
-// kernel row v's weights once for both outputs: output row y0 takes input row y0 + v - r_h, output row y0 + 1 the next one, so
-// the row loaded for one v is carried to the next.  flip: use W[c][kt-1-u][kh-1-v][kw-1-w] (the
-// backward's dX).  An output row past the volume (y0 + 1 = Hp) is computed and not stored.  KW =
-// the kernel's width kw (a compile-time constant); wget: where the weights are read
-// (ConvWGlobal, ConvWShared).
+// kernel row v's weights once for both outputs: output row y0 takes input row y0 + v - r_h,
+// output row y0 + 1 the next one, so the row loaded for one v is carried to the next.  flip: use
+// W[c][kt-1-u][kh-1-v][kw-1-w] (the backward's dX).  An output row past the volume (y0 + 1 =
+// Hp) is computed and not stored.  KW = the kernel's width kw (a compile-time constant); wget:
+// where the weights are read (ConvWGlobal, ConvWShared).
 template <typename T, int KW>
 __host__ __device__ __forceinline__ void conv_load_row(const T* __restrict__ row, const ConvGeo& g, int x0,
                                                        float2 (&a)[kConvStrip + KW - 1]) {
@@ -210,7 +210,8 @@ __host__ __device__ __forceinline__ void conv_load_row(const T* __restrict__ row
 // The same row as raw pairs (zero past the volume's edges, and all zero when !in).
 template <typename T, int KW>
 __host__ __device__ __forceinline__ void conv_load_row_raw(const T* __restrict__ row, bool in, const ConvGeo& g,
-                                                           int x0, typename ConvRaw<T>::type (&r)[kConvStrip + KW - 1]) {
+                                                           int x0,
+                                                           typename ConvRaw<T>::type (&r)[kConvStrip + KW - 1]) {
   using R = typename ConvRaw<T>::type;
   const int rw = (KW - 1) / 2;
 #pragma unroll
@@ -395,7 +396,9 @@ struct DwRing {
   XR* x;  // the lane's entry (stage 0, column 0): [stage][NJ], stride 32
   DR* d;  // the lane's entry (stage 0, strip output 0): [stage][kConvStrip], stride 32
   __host__ __device__ static constexpr size_t x_bytes() { return (size_t)kDwStages * NJ * 32 * sizeof(XR); }
-  __host__ __device__ static constexpr size_t warp_bytes() { return x_bytes() + (size_t)kDwStages * kConvStrip * 32 * sizeof(DR); }
+  __host__ __device__ static constexpr size_t warp_bytes() {
+    return x_bytes() + (size_t)kDwStages * kConvStrip * 32 * sizeof(DR);
+  }
   // the ring of lane `lane` in the warp's region at base (8-byte aligned)
   __host__ __device__ static DwRing at(unsigned char* base, int lane) {
     DwRing r;
@@ -432,13 +435,6 @@ __host__ __device__ __forceinline__ void dw_fetch(const DwRing<T, TD, KW>& r, in
   }
 }
 
-// dw_fetch for the whole warp at once, when its 32 lanes are 32 consecutive channel pairs from a
-// multiple of 32 (C a multiple of 64) on the same work item: a token's 32 pairs are one
-// contiguous run of 128 (bf16) or 256 (fp32) bytes, copied as 16-byte chunks spread over the
-// lanes, each chunk into the 16 bytes of the ring entry that hold those pairs.  xplane and dplane
-// point at the lane's own pair; the chunks a lane copies belong to other lanes too, so the ring
-// is shared within the warp (dw_syncwarp around its use).  On the host one call copies every
-// chunk of the warp.
 // The 16-byte chunks of one staged run of `tokens` tokens (32 pairs of R each: CPT = 2 sizeof(R)
 // chunks per token) that lane `lane` copies: chunk m = lane + 32 i is token m / CPT, chunk m mod
 // CPT, so the lane's token advances by 32 / CPT per chunk and its offset in the token is fixed.
@@ -458,7 +454,8 @@ __host__ __device__ __forceinline__ void dw_copy_run(unsigned char* dst0, const 
     const int j = j0 + i * TSTEP;
     if (j < TOKENS) {
       const bool in = ok(j);
-      dw_copy16(dst + (size_t)i * TSTEP * 32 * sizeof(R), in ? src + i * sstep : reinterpret_cast<const unsigned char*>(fallback), in);
+      const unsigned char* from = in ? src + i * sstep : reinterpret_cast<const unsigned char*>(fallback);
+      dw_copy16(dst + (size_t)i * TSTEP * 32 * sizeof(R), from, in);
     }
   }
 }
@@ -599,9 +596,9 @@ __host__ __device__ __forceinline__ void dw_walk(const T* __restrict__ x, const 
 // ---- the forward on strip pairs, input rows through a warp-shared ring ----------------------
 // For C a multiple of 32: a block owns kSw2Pairs channel pairs and its warps take units of two
 // neighbouring strips on kSw2Rows rows (t, rows y0 .. y0 + kSw2Rows - 1, columns xb .. xb + 2
-// kConvStrip - 1); lane 16 h + p computes pair p of strip h.  The two strips' windows share one input row of NT tokens, which
-// the warp copies into a ring in shared memory with 16-byte cp.async chunks, kSw2Stages - 1 rows
-// ahead of its use.
+// kConvStrip - 1); lane 16 h + p computes pair p of strip h.  The two strips' windows share one
+// input row of NT tokens, which the warp copies into a ring in shared memory with 16-byte
+// cp.async chunks, kSw2Stages - 1 rows ahead of its use.
 constexpr int kSw2Pairs = 16;
 constexpr int kSw2WStride = 2 * kSw2Pairs + 2;  // floats per staged tap row (2 of padding)
 constexpr int kSw2Units = 32;                   // units per block, kSw2Units / kConvSwWarps per warp
@@ -674,9 +671,10 @@ __host__ __device__ __forceinline__ void sw2_fetch(typename ConvRaw<T>::type* ri
 // The convolution sums of lane 16 h + p of a strip-pair unit (strip x0 = xb + h kConvStrip, pair
 // p of the group) for output rows y0 + o, o < kSw2Rows, added into acc[o]; Flip as in
 // conv_strip2, the weights read from the staged group at wsp (its tap rows kSw2WStride floats
-// apart, the lane's pair at 2 p).  The input rows y0 - r_h + r, r < kh + kSw2Rows - 1, of each kernel plane run as one
-// sequence, read from the warp's ring (ring: the warp's kSw2Stages rows); input row r feeds output
-// row y0 + o through kernel row r - o, whose weights are read for it.
+// apart, the lane's pair at 2 p).  The input rows y0 - r_h + r, r < kh + kSw2Rows - 1, of each
+// kernel plane run as one sequence, read from the warp's ring (ring: the warp's kSw2Stages
+// rows); input row r feeds output row y0 + o through kernel row r - o, whose weights are read
+// for it.
 template <typename T, int KW, bool Flip>
 __host__ __device__ __forceinline__ void conv_strips_ring(typename ConvRaw<T>::type* ring, int lane,
                                                           const T* xg, const float* wsp, const ConvGeo& g,
