@@ -518,12 +518,12 @@ dsa3d_status_t bwd_mma_group(const Shape& s, const void* q, const void* k, const
   if (rc != DSA3D_OK) return rc;
   const int64_t rows = (int64_t)hg * sg.Et * sg.Ey;
   {
-    const int smem = 2 * bwdq_pair_floats() * (int)sizeof(float);  // two warp pairs per CTA
+    const int smem = bwdq_pair_floats() * (int)sizeof(float);  // one warp pair per CTA
     if (cudaFuncSetAttribute(dsa3d_bwd_q_kernel<DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return DSA3D_ERR_CUDA;
     TimedLaunch tl(kKernBwdQ, st);
-    dsa3d_bwd_q_kernel<DH><<<grid_for(rows, 2, 1 << 20), 128, smem, st>>>(
+    dsa3d_bwd_q_kernel<DH><<<grid_for(rows, 1, 1 << 20), 64, smem, st>>>(
         qb, kb, vb, ob, off, lse, doff, w.cnt, w.sorted_n, w.sorted_ex, gbox, bbox, dft, g, sg, bg,
         h0, hg);
     if (cudaGetLastError() != cudaSuccess || !tl.finish()) return DSA3D_ERR_CUDA;

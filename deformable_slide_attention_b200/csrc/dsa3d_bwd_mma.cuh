@@ -132,7 +132,7 @@ __host__ __device__ constexpr int bwdq_pair_floats() {
 }
 
 template <int DH>
-__global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
+__global__ void __launch_bounds__(64, DSA3D_BWDQ_MINB)
     dsa3d_bwd_q_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ dout,
                        const float* __restrict__ off, const float* __restrict__ lse,
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(128, DSA3D_BWDQ_MINB)
   const __nv_bfloat16* asrc = role ? dout : q;  // A operand rows of this warp
   int sidx = 0;                                  // box-row steps so far (ring slot = sidx % 3)
 
-  for (int64_t row = (int64_t)blockIdx.x * 2 + pair; row < rows; row += (int64_t)gridDim.x * 2) {
+  for (int64_t row = (int64_t)blockIdx.x + pair; row < rows; row += (int64_t)gridDim.x) {
     const int hh = (int)(row / ((int64_t)sg.Et * sg.Ey));
     const int rem = (int)(row - (int64_t)hh * sg.Et * sg.Ey);
     const int et = rem / sg.Ey, ey = rem % sg.Ey;

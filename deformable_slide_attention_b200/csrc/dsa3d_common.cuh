@@ -17,7 +17,7 @@
 #define DSA3D_MMA_MINB 3
 #endif
 #ifndef DSA3D_BWDQ_MINB
-#define DSA3D_BWDQ_MINB 3
+#define DSA3D_BWDQ_MINB 6  // the query side's CTAs are one warp pair (64 threads)
 #endif
 #ifndef DSA3D_DQ_MINB
 #define DSA3D_DQ_MINB 3
