@@ -84,3 +84,10 @@ def test_dwconv_part_units_and_default():
     C, K = 32 * 128, 243
     assert u["fwd_bytes"] == u["bwd_bytes"] == 3 * C * 2
     assert u["fwd_flop"] == 2 * C * K and u["bwd_flop"] == 4 * C * K
+
+
+def test_e2e_groups_option():
+    """--e2e-groups picks the end-to-end leg's head groups; 0 (the default) keeps bench.py's own
+    choice (the largest group with four groups or more that fits)."""
+    assert bench.parse_args([]).e2e_groups == 0
+    assert bench.parse_args(["--e2e-groups", "8"]).e2e_groups == 8
