@@ -196,3 +196,25 @@ def test_offset_network_backward_matches_oracle(harness, taps, tokens_per_item):
                             ("d pw_weight", dwp, ref[3]), ("d pw_bias", dbp, ref[4])):
         err = np.abs(got - want).max()
         assert err <= 1e-4 * max(1.0, np.abs(want).max()), (name, err)
+
+
+@pytest.mark.parametrize("frames_per_item", [1, 3])
+def test_weight_gradient_fp32_dy_cooperative(harness, frames_per_item):
+    """dW with x in bf16 and dY in fp32 (the offset network's backward) at C = 64, where the
+    library takes the warp-cooperative copies: a token's 32 fp32 pairs are 16 chunks, so a lane's
+    chunks are two tokens apart (eight for bf16)."""
+    dims, C, window = (3, 6, 19), 64, (3, 5, 7)
+    g = torch.Generator().manual_seed(19)
+    N = math.prod(dims)
+    x = torch.randn(N, C, generator=g).to(torch.bfloat16)
+    dy = torch.randn(N, C, generator=g)
+    w = torch.randn(C, *window, generator=g)
+    io, xa = _io(x)
+    dya = dy.contiguous().numpy()
+    dw = np.zeros((C, *window), np.float32)
+    db = np.zeros(C, np.float32)
+    assert harness.conv_host_dw_mixed(io, _ptr(xa), _ptr(dya), *dims, C, *window, frames_per_item,
+                                      _ptr(dw), _ptr(db)) == 0
+    _, ref_dw, ref_db = oracle.dwconv3d_backward(x, w, dy.double().numpy(), dims)
+    assert np.abs(dw - ref_dw).max() <= 1e-4 * max(1.0, np.abs(ref_dw).max())
+    assert np.abs(db - ref_db).max() <= 1e-4 * max(1.0, np.abs(ref_db).max())
